@@ -1,0 +1,358 @@
+#!/usr/bin/env python
+"""Benchmark of the JoLT KV-cache codec on one B200 (or N, one process per GPU).
+
+Workload: the Mistral-7B-shaped GQA cache (32 layers x 8 KV heads x 1024 tokens x 128
+features, bf16, K and V), compressed at 2x with 4 layer groups and separate K/V budgets by
+the randomized-SVD ("FlashJoLT") encoder, then decoded. One step = encode + decode + the
+relative Frobenius error of K and V (all rows of the hot path), on synthetic rank-structured
+data (the pages' real model caches are not available). Metric: KV tokens per second through
+encode + decode; a token is one position across all layers, K and V.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl jolt|reference]
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV tokens/s encode+decode (Mistral-7B-shape, 2x); rel. Frobenius error"
+UNIT = "tokens/s"
+SEED = 42
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["jolt", "reference"], default="jolt")
+    ap.add_argument("--ratio", type=float, default=2.0)
+    ap.add_argument("--encoder", choices=["sketch", "exact"], default="sketch")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-out", default=None, help="write the per-phase trace JSON here")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, sm_max_mhz=1965.0,
+                source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.idx)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if not self.proc:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(smax) if smax else None,
+                    reasons=sorted(reasons), samples=len(sm))
+
+
+# ------------------------------------------------------------------ oracle (CPU baseline and reference arm)
+def oracle_sample_tokens_per_s(cfg, ratio, encoder, budget_s=12.0, max_s=30.0):
+    """Oracle encode + decode of whole layers (K and V) of the workload until ~budget_s of CPU time;
+    returns (tokens/s scaled to the full cache, threads used, sample description)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+    import synth
+    from oracle import jolt as oj
+    n_lt_full = cfg.layers * (2 if cfg.has_v else 1)
+    budget_full = synth.kv.budget_bytes(cfg, ratio)
+    done, t_total, layers = 0, 0.0, []
+    l = 0
+    while (t_total < budget_s and l < cfg.layers) or done == 0:
+        K = synth.gen_layer_tensor(cfg, l, 0)[None]
+        V = synth.gen_layer_tensor(cfg, l, 1)[None] if cfg.has_v else None
+        kinds = 2 if cfg.has_v else 1
+        plan = oj.Plan(L=1, H=cfg.heads, T=cfg.tokens, D=cfg.head_dim, has_v=cfg.has_v,
+                       budget=budget_full * kinds // n_lt_full, num_groups=1, encoder=encoder,
+                       split_kv=cfg.split_kv, bits=tuple(cfg.bits))
+        t0 = time.perf_counter()
+        st, _ = oj.encode(plan, K, V, SEED)
+        oj.decode(st)
+        t_total += time.perf_counter() - t0
+        done += kinds
+        layers.append(l)
+        l += 1
+        if t_total > max_s:
+            break
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    full_time = t_total * n_lt_full / done
+    sample = (f"oracle encode+decode of layers {layers[0]}..{layers[-1]} (K and V, {done} of "
+              f"{n_lt_full} layer-tensors, each layer its own single-group plan at the same per-layer "
+              f"budget), {t_total:.1f} s, scaled to the full cache")
+    return cfg.tokens / full_time, threads, sample
+
+
+def run_reference(args):
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = synth.config(args.config)
+    times = []
+    threads = 1
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        tps, threads, sample = oracle_sample_tokens_per_s(cfg, args.ratio, args.encoder, budget_s=0.0, max_s=30.0)
+        if i >= args.warmup:
+            times.append(cfg.tokens / tps)
+    ms = 1e3 * sum(times) / len(times)
+    value = cfg.tokens / (ms / 1e3)
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": config_dict(cfg, args),
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+def config_dict(cfg, args):
+    return {"workload": f"{cfg.name} (Mistral-7B-v0.3 GQA KV shape), {args.ratio:g}x byte budget, "
+                        f"{cfg.groups} layer groups, separate K/V budgets, {args.encoder} token factor",
+            "layers": cfg.layers, "kv_heads": cfg.heads, "tokens": cfg.tokens, "head_dim": cfg.head_dim,
+            "kinds": "K+V" if cfg.has_v else "K", "ratio": args.ratio, "encoder": args.encoder,
+            "groups": cfg.groups, "seq_per_gpu": 1,
+            "l2": "inputs larger than L2 (K+V bf16 = 134 MB > 126 MB L2), no flush"}
+
+
+# ------------------------------------------------------------------ work models for the roofline
+def phase_models(cfg, plan_info, alloc, ratio, peaks):
+    """Algorithmic work of each traced phase per step (measurement section)."""
+    H, T, D, L = cfg.heads, cfg.tokens, cfg.head_dim, cfg.layers
+    n_lt = L * 2
+    N = H * T * D                      # entries per layer-tensor
+    l = plan_info["sketch_l"]
+    groups = alloc.shape[0]
+    ranks = []
+    for layer in range(L):
+        g = next(gi for gi in range(groups) if (gi * L) // groups <= layer < ((gi + 1) * L) // groups)
+        for k in (0, 1):
+            ranks.append(tuple(int(v) for v in alloc[g, k]))
+    stream_bytes = sum(2 * (T * rt + D * rd + H * rt * rd) + (H * T * (D * b // 8 + 2) if b else 0)
+                       for rt, rd, b in ranks)
+    clock = peaks["sm_max_mhz"] * 1e6
+    fp64_peak = 148 * 64 * 2 * clock / 1e12       # TFLOP/s, 64 FP64 FMA / clk / SM
+    fp32_peak = 148 * 128 * 2 * clock / 1e12      # TFLOP/s, 128 FP32 FMA / clk / SM
+    resid_flops = sum(2.0 * N * (D + rt) for rt, rd, b in ranks if b > 0)
+    dec_flops = sum(2.0 * N * (rt + (D if b else 0)) for rt, rd, b in ranks)
+    return {
+        "sketch_gemm": dict(bound="tensor", work=8.0 * T * H * D * l * n_lt / 1e12, unit="TFLOP/s",
+                            peak=peaks["bf16_tflops"], note="4 passes over X, 2 T HD l flops each"),
+        "feature_gram": dict(bound="tensor", work=2.0 * N * D * n_lt / 1e12, unit="TFLOP/s",
+                             peak=peaks["bf16_tflops"], note="C_D = sum_h X_h^T X_h"),
+        "residual": dict(bound="alu", work=resid_flops / 1e12, unit="TFLOP/s", peak=fp64_peak,
+                         note="float64 x Pi - u N per entry: 2 (D + r_t) flops; FP64 peak 148 SMs x 64 FMA x 2 x max clock"),
+        "decode": dict(bound="alu", work=dec_flops / 1e12, unit="TFLOP/s", peak=fp32_peak,
+                       note="float32 u M + y Pi^T per entry: 2 (r_t + D) flops; FP32 peak 148 x 128 FMA x 2 x max clock",
+                       hbm_bytes=2.0 * N * n_lt + stream_bytes),
+        "jacobi_feature": dict(bound="alu", work=None, unit="TFLOP/s", peak=fp32_peak, note="shared-memory Jacobi"),
+        "jacobi_sketch": dict(bound="alu", work=None, unit="TFLOP/s", peak=fp32_peak, note="shared-memory Jacobi"),
+    }, stream_bytes
+
+
+# ------------------------------------------------------------------ main (CUDA path)
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import synth
+    from tensor_decomposition_b200 import jolt as J
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    cfg = synth.config(args.config)
+    K, V = synth.gen_cache_torch(cfg, dev, seq=rank)       # weak scaling: one sequence per GPU
+    budget = synth.kv.budget_bytes(cfg, args.ratio)
+    c = J.jolt_config_default()
+    c.encoder = J.JOLT_ENC_SKETCH if args.encoder == "sketch" else J.JOLT_ENC_EXACT
+    c.split_kv_budget = int(cfg.split_kv)
+    plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, budget,
+                       cfg.groups, c)
+    info = J.jolt_plan_info(plan)
+    Ko, Vo = torch.empty_like(K), torch.empty_like(V)
+    errs = [None, None]
+
+    def step(Kin=K, Vin=V):
+        st = J.jolt_encode(plan, Kin, Vin, SEED)
+        J.jolt_decode(st, Ko, Vo)
+        errs[0] = J.jolt_rel_frob_error(Kin, Ko)
+        errs[1] = J.jolt_rel_frob_error(Vin, Vo)
+        return st
+
+    for _ in range(args.warmup):
+        st = step()
+    J.jolt_stream_status(st)
+    alloc = J.jolt_stream_info(st, cfg.groups)["alloc"]
+    del st
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- timed region: K steps, inputs resident in HBM
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    J.jolt_profile_enable(True)
+    barrier()
+    clocks.start()
+    l0 = J.jolt_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        st = step()
+    e1.record()
+    barrier()
+    clk = clocks.stop()
+    launches = J.jolt_launch_count() - l0
+    prof = J.jolt_profile_report()
+    J.jolt_profile_enable(False)
+    del st
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    value = cfg.tokens * args.steps * world / (ms_max / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    Kh = K.cpu().pin_memory()
+    Vh = V.cpu().pin_memory()
+    Kd, Vd = torch.empty_like(K), torch.empty_like(V)
+    for _ in range(2):
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        st = step(Kd, Vd)
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        st = step(Kd, Vd)          # ends with the device -> host read of the two errors
+    f1.record()
+    barrier()
+    del st
+    te = torch.tensor([f0.elapsed_time(f1)], device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = cfg.tokens * args.steps * world / (float(te.item()) / 1e3)
+
+    # ---- roofline of the dominant phase
+    peaks = measured_peaks()
+    models, stream_bytes = phase_models(cfg, info, alloc, args.ratio, peaks)
+    top = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
+    name, rec = top
+    per_launch_ms = rec["total_ms"] / max(1, rec["calls"])
+    m = models.get(name)
+    roof = None
+    if m and m["work"] is not None:
+        achieved = m["work"] / (per_launch_ms / 1e3)
+        roof = {"kernel": name, "bound": m["bound"], "achieved": achieved, "peak": m["peak"], "unit": m["unit"],
+                "frac": achieved / m["peak"], "traffic": None,
+                "peak_source": peaks["source"] if m["bound"] != "alu" else "derived: SM count x FMA/clk x max clock",
+                "ms_per_launch": per_launch_ms, "note": m["note"]}
+    phases = {k: round(v["total_ms"] / args.steps, 4) for k, v in prof.items()}
+
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "jolt",
+           "config": config_dict(cfg, args),
+           "rel_frob_error": {"K": errs[0], "V": errs[1]},
+           "compressed_bytes": stream_bytes, "budget_bytes": budget,
+           "alloc": alloc.tolist(),
+           "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(K.numel() * 2 + V.numel() * 2),
+                   "d2h_bytes_per_step": 16},
+           "gpu_launches": int(launches),
+           "phase_ms_per_step": phases,
+           "roofline": roof,
+           "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
+                      "samples": clk["samples"]}}
+    if args.profile_out and rank == 0:
+        json.dump(prof, open(args.profile_out, "w"), indent=1)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, threads, sample = oracle_sample_tokens_per_s(cfg, args.ratio, args.encoder)
+        out["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

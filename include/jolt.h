@@ -1,0 +1,207 @@
+/*
+ * jolt.h - C ABI of the JoLT KV-cache codec for NVIDIA B200 (sm_100a).
+ *
+ * The method is the one of "A JoLT for the KV Cache: Near-Lossless KV Cache Compression
+ * via Joint Tucker and JL-Residual Allocation for LLMs" (arXiv 2607.12550v2, Abstract):
+ * each layer's key (or value) cache X in R^{H x T x D} (heads x tokens x features) gets a
+ * partial Tucker decomposition over the token and feature axes only,
+ *     X[h] ~ U_T G[h] U_D^T,   U_T: T x r_t,  U_D: D x r_d,  G: H x r_t x r_d,
+ * the truncation residual is rotated by a seeded random orthogonal D x D matrix and
+ * quantised to b bits per entry with one fp16 scale per row, and a single Lagrangian dual
+ * picks (r_t, r_d, b) per layer group, separately for K and V, under one byte budget.
+ * The randomized-SVD token factor is the Abstract's "FlashJoLT" variant. Decode rebuilds
+ * G x2 U_T x3 U_D plus the inverse-rotated, dequantised residual.
+ *
+ * Conventions for every entry point:
+ *  - Tensors are row-major [layers][heads][tokens][head_dim] on the CUDA device that is
+ *    current when the call is made. Pointers marked "device" must be device pointers
+ *    (cudaMalloc / PyTorch CUDA storage), pointers marked "host" must be host memory.
+ *  - `cuda_stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Encode and decode enqueue work on it and return without waiting for the device.
+ *  - Every function returns a jolt_status. On failure, jolt_last_error() returns a
+ *    message for the calling thread. Nothing aborts the process.
+ *  - Errors found on the device (Jacobi not converged, non-finite input, spin timeout)
+ *    are recorded in a status word of the stream object; they surface at the next call
+ *    that synchronises (jolt_stream_status, jolt_stream_info, jolt_stream_to_host).
+ *  - The caller owns input and output tensors. The library owns plans and streams and
+ *    their device memory; release them with jolt_plan_destroy / jolt_stream_destroy.
+ *  - A plan holds one workspace: encodes that share a plan must be issued on one CUDA
+ *    stream (or otherwise serialised).
+ *
+ * This build supports head_dim == 128, batch of one sequence per stream, and token
+ * ranks r_t <= 112 (the sketch width r_t + oversample must stay <= 128).
+ */
+#ifndef JOLT_H
+#define JOLT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define JOLT_API __declspec(dllexport)
+#else
+#define JOLT_API __attribute__((visibility("default")))
+#endif
+
+typedef enum {
+  JOLT_OK = 0,
+  JOLT_ERR_INVALID_ARG = 1,       /* bad shape, pointer, size or option */
+  JOLT_ERR_BUDGET_INFEASIBLE = 2, /* the smallest allowed choices exceed the byte budget */
+  JOLT_ERR_OOM = 3,               /* device allocation failed */
+  JOLT_ERR_CUDA = 4,              /* a CUDA runtime call failed (message names it) */
+  JOLT_ERR_NOT_CONVERGED = 5,     /* an eigensolver hit its sweep limit (result still usable) */
+  JOLT_ERR_NONFINITE = 6,         /* NaN or Inf met in the input */
+  JOLT_ERR_TIMEOUT = 7,           /* a bounded device wait gave up */
+  JOLT_ERR_CORRUPT_STREAM = 8,    /* bad magic, version, size or CRC in a serialized stream */
+  JOLT_ERR_UNSUPPORTED = 9        /* valid request outside what this build implements */
+} jolt_status;
+
+typedef enum { JOLT_BF16 = 0, JOLT_F32 = 1 } jolt_dtype;
+
+typedef enum { JOLT_ENC_AUTO = 0, JOLT_ENC_EXACT = 1, JOLT_ENC_SKETCH = 2 } jolt_encoder;
+
+/* Shape of one sequence's cache. `dtype` is both the input and the decoded output type. */
+typedef struct {
+  int32_t layers, heads, tokens, head_dim;
+  int32_t has_v;      /* 0: keys only (V pointers are ignored), 1: keys and values */
+  jolt_dtype dtype;
+} jolt_shape;
+
+/* Codec options; jolt_config_default() fills the defaults shown. */
+typedef struct {
+  jolt_encoder encoder;      /* AUTO (default): exact if tokens <= 1024, else sketch */
+  int32_t oversample;        /* sketch oversampling p (16) */
+  int32_t power_iters;       /* sketch power iterations q (1) */
+  int32_t rank_step;         /* candidate ranks are multiples of this (16) */
+  int32_t rt_max;            /* cap on the token rank; 0 = 112 */
+  uint32_t bits_mask;        /* bit b set => residual bit-width b allowed (0x1FF = 0..8) */
+  int32_t split_kv_budget;   /* 0: one budget pool for K and V; 1: half the budget each */
+  int32_t max_jacobi_sweeps; /* eigensolver sweep limit (30) */
+} jolt_config;
+
+typedef struct jolt_plan_s* jolt_plan_t;
+typedef struct jolt_stream_s* jolt_stream_t;
+
+/* Parts of a stream, in the order they are laid out and counted. */
+enum { JOLT_PART_UT = 0, JOLT_PART_UD = 1, JOLT_PART_G = 2, JOLT_PART_SCALES = 3,
+       JOLT_PART_CODES = 4, JOLT_NUM_PARTS = 5 };
+
+/* Debug exports (parity tests): see jolt_export_debug. */
+enum { JOLT_DBG_PI = 0,        /* float32 [D][D] rotation Pi used by encode */
+       JOLT_DBG_UT_F32 = 1,    /* float32 [T][R] token factor before bf16 rounding, layer-tensor lt */
+       JOLT_DBG_UD_F32 = 2,    /* float32 [D][D] feature factor before bf16 rounding, lt */
+       JOLT_DBG_TABLE = 3,     /* float64 per-unit error table, unit = lt (group*2 + kind) */
+       JOLT_DBG_XX = 4,        /* float64 [2*L] squared Frobenius norm of every layer-tensor */
+       JOLT_DBG_LAMBDA = 5,    /* float64 [2] dual variable of each budget pool */
+       JOLT_DBG_OMEGA = 6 };   /* bf16 bits [HD][l] sketch matrix of layer-tensor lt */
+
+JOLT_API void jolt_config_default(jolt_config* cfg);
+
+/*
+ * jolt_plan - validate a shape and budget and reserve the encode workspace.
+ *
+ * byte_budget: bytes the whole stream may spend on stored factors, cores, packed codes and
+ *   scales (the "one byte budget" of the Abstract); the header and alignment padding are
+ *   not counted. A compression ratio N means byte_budget = bf16 bytes of the cache / N.
+ * num_groups: layers are split into contiguous groups, group g holding layers
+ *   [g*L/G, (g+1)*L/G); each group picks its own (r_t, r_d, b) for K and for V.
+ * cfg: NULL for defaults.
+ * Errors: INVALID_ARG (non-positive sizes, head_dim != 128, groups > layers, bad options),
+ *   BUDGET_INFEASIBLE (the cheapest allowed choice of every group exceeds the budget),
+ *   OOM, CUDA. On success *out owns device workspace until jolt_plan_destroy.
+ */
+JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, int32_t num_groups,
+                               const jolt_config* cfg, jolt_plan_t* out);
+
+/* Plan facts: largest token rank R, sketch width l (0 for exact), encoder used, workspace
+ * bytes. Any output pointer may be NULL. */
+JOLT_API jolt_status jolt_plan_info(jolt_plan_t plan, int32_t* rt_max, int32_t* sketch_l,
+                                    int32_t* encoder, uint64_t* workspace_bytes);
+
+/*
+ * jolt_encode - compress one sequence's cache (device K, and V when the shape has V).
+ *
+ * K, V: device tensors [L][H][T][D] of the plan's dtype. They are only read.
+ * seed: selects the rotation Pi (the Abstract's random orthogonal rotation) and the sketch
+ *   matrices; it is stored in the stream so decode can rebuild Pi.
+ * Phases, all on `cuda_stream`: factor analysis of every layer-tensor (Gram / sketch GEMMs,
+ *   Jacobi eigensolver, CholeskyQR, core projection, error table), the Lagrangian dual over
+ *   all groups, then residual coding. The host does not wait for the device.
+ * *out: a device-resident stream owned by the caller until jolt_stream_destroy.
+ */
+JOLT_API jolt_status jolt_encode(jolt_plan_t plan, const void* K, const void* V, uint64_t seed,
+                                 void* cuda_stream, jolt_stream_t* out);
+
+/*
+ * jolt_decode - rebuild the cache: X_hat[h] = U_T G[h] U_D^T + dequant(codes) Pi^T.
+ *
+ * K_out, V_out: device tensors [L][H][T][D] of the stream's dtype (bf16 output is rounded to
+ *   nearest even). V_out is ignored for a keys-only stream. Enqueued on `cuda_stream`.
+ */
+JOLT_API jolt_status jolt_decode(jolt_stream_t stream, void* K_out, void* V_out, void* cuda_stream);
+
+/*
+ * jolt_rel_frob_error - ||ref - approx||_F / ||ref||_F over n elements (the error measure the
+ *   Abstract reports), accumulated in float64. ref, approx: device arrays of `dtype`.
+ *   Synchronises `cuda_stream`; *out is host memory. Returns 0 when ||ref|| = 0.
+ */
+JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, uint64_t n,
+                                         jolt_dtype dtype, void* cuda_stream, double* out);
+
+/* Synchronise on the stream's CUDA stream and report device-side errors of its encode. */
+JOLT_API jolt_status jolt_stream_status(jolt_stream_t stream);
+
+/*
+ * jolt_stream_info - synchronise and report the allocation and the stored bytes.
+ * bytes_by_part: host [5] bytes of U_T, U_D, G, scales, codes over all layer-tensors (or NULL).
+ * alloc: host [num_groups][2][3] (r_t, r_d, b) per group and kind (or NULL).
+ * lambdas: host [2] dual variable of each pool (or NULL).
+ */
+JOLT_API jolt_status jolt_stream_info(jolt_stream_t stream, uint64_t* bytes_by_part,
+                                      int32_t* alloc, double* lambdas);
+
+/*
+ * jolt_stream_to_host - serialize: header (magic "JOLT", version 1, shape, seed, allocation
+ *   table), body (per layer-tensor lt = 2*layer + kind: U_T [T][r_t] bf16, U_D [D][r_d] bf16,
+ *   G [H][r_t][r_d] bf16, scales [H][T] fp16, codes [H][T][D*b/8] bytes with code i at bits
+ *   [i*b, i*b+b) LSB first; each part starts at a multiple of 256 bytes), then CRC-32.
+ * buf: host buffer of *len bytes, or NULL to query the size into *len.
+ */
+JOLT_API jolt_status jolt_stream_to_host(jolt_stream_t stream, void* buf, uint64_t* len);
+
+/* jolt_stream_from_host - parse a serialized stream (checks magic, version, sizes, CRC)
+ * into a new device stream; Pi is rebuilt from the stored seed on `cuda_stream`. */
+JOLT_API jolt_status jolt_stream_from_host(const void* buf, uint64_t len, void* cuda_stream,
+                                           jolt_stream_t* out);
+
+/* jolt_export_debug - copy an internal array (JOLT_DBG_*) of the last encode to host memory.
+ * lt selects the layer-tensor (or unit for JOLT_DBG_TABLE). buf NULL queries *len. Syncs. */
+JOLT_API jolt_status jolt_export_debug(jolt_stream_t stream, int32_t what, int32_t lt, void* buf,
+                                       uint64_t* len);
+
+/* Tracing. jolt_profile_enable(1) brackets every encode / decode / error phase with CUDA
+ * events recorded on the stream the phase runs on, and counts the kernel launches inside it.
+ * jolt_profile_report synchronises the device, writes a JSON object
+ * {"phase": {"calls": n, "launches": k, "total_ms": t}, ...} (NUL-terminated; buf NULL queries
+ * *len) and clears the records. jolt_launch_count returns the number of kernels this library
+ * has launched since it was loaded. */
+JOLT_API jolt_status jolt_profile_enable(int32_t on);
+JOLT_API jolt_status jolt_profile_report(char* buf, uint64_t* len);
+JOLT_API uint64_t jolt_launch_count(void);
+
+/* Release a stream. Its device memory is freed in order on the CUDA stream the stream was
+ * created on (encode or jolt_stream_from_host); synchronise any other CUDA stream that still
+ * reads it (e.g. a decode issued elsewhere) before destroying it. */
+JOLT_API void jolt_stream_destroy(jolt_stream_t stream);
+JOLT_API void jolt_plan_destroy(jolt_plan_t plan);
+
+/* Message of the last failed call on this thread ("" if none). */
+JOLT_API const char* jolt_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* JOLT_H */

@@ -1,0 +1,1056 @@
+// Host runtime of the JoLT codec behind the C ABI declared in include/jolt.h: plan
+// validation and workspace, encode / decode orchestration on one CUDA stream, stream
+// serialization with CRC-32, and error reporting.
+//
+// Method: "A JoLT for the KV Cache: Near-Lossless KV Cache Compression via Joint Tucker and
+// JL-Residual Allocation for LLMs" (arXiv 2607.12550v2, Abstract). Encode runs the three
+// stages of the Abstract in order: partial Tucker analysis of every layer-tensor (token and
+// feature factors, core at the largest ranks, truncation-energy table), the single
+// Lagrangian dual over all layer groups and both kinds, and the rotated low-bit residual.
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <type_traits>
+#include <string>
+#include <vector>
+
+#include "jolt_internal.h"
+
+using namespace jolt;
+
+namespace {
+
+thread_local std::string g_err;
+
+jolt_status fail(jolt_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+#define CK(call)                                                                          \
+  do {                                                                                    \
+    cudaError_t e_ = (call);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return fail(e_ == cudaErrorMemoryAllocation ? JOLT_ERR_OOM : JOLT_ERR_CUDA,        \
+                  "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__); \
+  } while (0)
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// kappa_D = E[max_{i<D} z_i^2], z ~ N(0, I_D) = int_0^inf 2y (1 - erf(y/sqrt 2)^D) dy, by
+// composite Simpson's rule on [0, 40] with step 1/1024; 1 - erf^D = -expm1(D log1p(-erfc)).
+double kappa_of(int D) {
+  const int n = 40 * 1024;
+  const double h = 40.0 / n;
+  auto f = [D](double y) {
+    const double e = std::erfc(y / std::sqrt(2.0));
+    return 2.0 * y * (-std::expm1((double)D * std::log1p(-e)));
+  };
+  double s = f(0.0) + f(40.0);
+  for (int i = 1; i < n; ++i) s += (i & 1 ? 4.0 : 2.0) * f(i * h);
+  return s * h / 3.0;
+}
+
+int64_t lt_bytes_h(int H, int T, int D, int rt, int rd, int b) {
+  const int64_t tucker = 2 * ((int64_t)T * rt + (int64_t)D * rd + (int64_t)H * rt * rd);
+  const int64_t resid = b > 0 ? (int64_t)H * T * (D * b / 8 + 2) : 0;
+  return tucker + resid;
+}
+
+int group_of_layer(int l, int L, int G) {
+  int g = 0;
+  while (g + 1 < G && ((int64_t)(g + 1) * L) / G <= l) ++g;
+  return g;
+}
+
+// CRC-32 (IEEE 802.3, reflected polynomial 0xEDB88320), table driven.
+uint32_t crc32_ieee(const uint8_t* p, size_t n, uint32_t crc = 0) {
+  static uint32_t table[256];
+  static bool init = false;
+  if (!init) {
+    for (uint32_t i = 0; i < 256; ++i) {
+      uint32_t c = i;
+      for (int k = 0; k < 8; ++k) c = (c & 1) ? 0xEDB88320u ^ (c >> 1) : c >> 1;
+      table[i] = c;
+    }
+    init = true;
+  }
+  crc = ~crc;
+  for (size_t i = 0; i < n; ++i) crc = table[(crc ^ p[i]) & 0xFFu] ^ (crc >> 8);
+  return ~crc;
+}
+
+template <typename T>
+T* carve(char*& cur, size_t count) {
+  cur = reinterpret_cast<char*>(align_up(reinterpret_cast<size_t>(cur), 256));
+  T* p = reinterpret_cast<T*>(cur);
+  cur += count * sizeof(T);
+  return p;
+}
+
+// ---------------------------------------------------------------- tracing
+// When enabled, each phase of encode / decode is bracketed by CUDA events recorded on the
+// stream it runs on, and the kernel launches inside it are counted.
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+  uint64_t launches;
+};
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+class Prof {
+ public:
+  Prof(const char* name, cudaStream_t s) : name_(name), s_(s) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    if (!g_prof_on) return;
+    a_ = take_event();
+    l0_ = g_launches.load();
+    cudaEventRecord(a_, s_);
+  }
+  ~Prof() {
+    if (!a_) return;
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    cudaEvent_t b = take_event();
+    cudaEventRecord(b, s_);
+    g_prof.push_back({name_, a_, b, g_launches.load() - l0_});
+  }
+
+ private:
+  const char* name_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr;
+  uint64_t l0_ = 0;
+};
+#define PROF_CAT2(a, b) a##b
+#define PROF_CAT(a, b) PROF_CAT2(a, b)
+#define PROF(name, s) Prof PROF_CAT(prof_, __LINE__)(name, s)
+
+}  // namespace
+
+namespace jolt {
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace jolt
+
+// ============================================================================ objects
+struct jolt_plan_s {
+  jolt_shape shape{};
+  jolt_config cfg{};
+  uint64_t budget = 0;
+  int G = 1, encoder = JOLT_ENC_SKETCH, R = 0, l = 0, step = 16, nbits = 0, ngrid = 1, n_lt = 0;
+  int bits[9] = {0};
+  double phi[9] = {0};
+  double kappa = 0;
+  int64_t pool_budget[2] = {0, 0};
+  std::vector<int32_t> lt_ids;   // buffer index i -> lt = 2*layer + kind (kind-major order)
+  int32_t* d_lt_ids = nullptr;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  // workspace views
+  double *xx = nullptr, *xx_part = nullptr;
+  float *CD = nullptr, *UD32 = nullptr, *UDf = nullptr, *lamD = nullptr;
+  __nv_bfloat16 *UDb = nullptr, *Om = nullptr, *UTb = nullptr;
+  float *Y = nullptr, *Y2 = nullptr, *Z = nullptr, *Z2 = nullptr, *Bm = nullptr, *BB = nullptr,
+        *Wv = nullptr, *lamB = nullptr, *UT32 = nullptr, *UTf = nullptr, *P = nullptr, *Gmax = nullptr,
+        *CT = nullptr, *VT = nullptr, *lamT = nullptr;
+  double *Wg = nullptr, *Rinv = nullptr, *E = nullptr, *unit_err = nullptr, *Nbuf = nullptr;
+  double* Gpi = nullptr;
+  float* Pi32 = nullptr;
+  __nv_bfloat16* Pib = nullptr;
+  bool pi_valid = false;
+  uint64_t pi_seed = 0;
+  jolt_stream_s* last = nullptr;
+  int device = 0;
+};
+
+struct jolt_stream_s {
+  int L = 0, H = 0, T = 0, D = 0, has_v = 0, G = 1, encoder = 0, step = 16, R = 0, split = 0;
+  jolt_dtype dtype = JOLT_BF16;
+  uint64_t seed = 0;
+  StreamMeta* d_meta = nullptr;
+  uint8_t* d_body = nullptr;
+  size_t body_cap = 0;
+  float* d_Pi = nullptr;
+  double* d_Gpi = nullptr;
+  int32_t* d_lt_ids = nullptr;
+  int n_lt = 0;
+  cudaStream_t cs = nullptr;
+  jolt_plan_s* plan = nullptr;
+};
+
+// ============================================================================ helpers
+namespace {
+
+Operand opnd(const void* p, ElemType t, Idx2 batch, Idx2 row, Idx2 k) {
+  Operand o;
+  o.p = p;
+  o.t = t;
+  o.batch = batch;
+  o.row = row;
+  o.k = k;
+  return o;
+}
+OutDesc outd(void* p, ElemType t, Idx2 batch, Idx2 m, Idx2 n) {
+  OutDesc o;
+  o.p = p;
+  o.t = t;
+  o.batch = batch;
+  o.m = m;
+  o.n = n;
+  return o;
+}
+Idx2 I1(int64_t s) {
+  Idx2 x;
+  x.s_in = s;
+  return x;
+}
+Idx2 I2(int32_t in, int64_t s_in, int64_t s_out) {
+  Idx2 x;
+  x.in = in;
+  x.s_in = s_in;
+  x.s_out = s_out;
+  return x;
+}
+
+// Shifted CholeskyQR3 of n_lt tall matrices Y (rows x l, row-major, batch stride rows*l):
+// pass 1 with shift s = 11 (rows l + l (l + 1)) 2^-53 ||Y||^2 (Fukaya, Kannan, Nakatsukasa,
+// Yamamoto & Yanagisawa 2020), passes 2 and 3 unshifted. Result in Qout; Y is clobbered.
+jolt_status cholqr3(jolt_plan_s* p, int rows, float* Yin, float* Qout, int32_t* status,
+                    cudaStream_t s) {
+  const int l = p->l, n = p->n_lt;
+  float* src = Yin;
+  float* dst = Qout;
+  for (int pass = 0; pass < 3; ++pass) {
+    // Wg = src^T src (l x l, float64)
+    CK(gemm_simt(n, l, l, rows, opnd(src, EL_F32, I1((int64_t)rows * l), I1(1), I1(l)),
+                 opnd(src, EL_F32, I1((int64_t)rows * l), I1(1), I1(l)),
+                 outd(p->Wg, EL_F64, I1((int64_t)l * l), I1(l), I1(1)), 1.0, 0.0, s));
+    const double shift =
+        pass == 0 ? 11.0 * ((double)rows * l + (double)l * (l + 1)) * std::ldexp(1.0, -53) * l : 0.0;
+    CK(chol_inv(n, l, p->Wg, (int64_t)l * l, p->Rinv, (int64_t)l * l, shift, status, s));
+    // dst = src * Rinv
+    CK(gemm_simt(n, rows, l, l, opnd(src, EL_F32, I1((int64_t)rows * l), I1(l), I1(1)),
+                 opnd(p->Rinv, EL_F64, I1((int64_t)l * l), I1(1), I1(l)),
+                 outd(dst, EL_F32, I1((int64_t)rows * l), I1(l), I1(1)), 1.0, 0.0, s));
+    std::swap(src, dst);
+  }
+  // after 3 passes the result sits in `src`
+  if (src != Qout)
+    CK(cudaMemcpyAsync(Qout, src, sizeof(float) * (size_t)n * rows * l, cudaMemcpyDeviceToDevice, s));
+  return JOLT_OK;
+}
+
+}  // namespace
+
+// ============================================================================ API
+extern "C" {
+
+JOLT_API void jolt_config_default(jolt_config* c) {
+  if (!c) return;
+  c->encoder = JOLT_ENC_AUTO;
+  c->oversample = 16;
+  c->power_iters = 1;
+  c->rank_step = 16;
+  c->rt_max = 0;
+  c->bits_mask = 0x1FFu;
+  c->split_kv_budget = 0;
+  c->max_jacobi_sweeps = 30;
+}
+
+JOLT_API const char* jolt_last_error(void) { return g_err.c_str(); }
+
+JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, int32_t num_groups,
+                               const jolt_config* cfg_in, jolt_plan_t* out) {
+  g_err.clear();
+  if (!shape || !out) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: null shape or out");
+  *out = nullptr;
+  jolt_config cfg;
+  jolt_config_default(&cfg);
+  if (cfg_in) cfg = *cfg_in;
+  const jolt_shape& sh = *shape;
+  if (sh.layers <= 0 || sh.heads <= 0 || sh.tokens <= 0 || sh.head_dim <= 0)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: non-positive dimension");
+  if (sh.head_dim != kD)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: head_dim %d unsupported (this build: 128)", sh.head_dim);
+  if (sh.layers > kMaxL) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: at most %d layers", kMaxL);
+  if (sh.dtype != JOLT_BF16 && sh.dtype != JOLT_F32) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: dtype");
+  if (num_groups <= 0 || num_groups > sh.layers || num_groups > kMaxGroups)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: num_groups must be in [1, min(layers, %d)]", kMaxGroups);
+  if (cfg.rank_step <= 0 || kD % cfg.rank_step != 0)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: rank_step must divide %d", kD);
+  if (cfg.oversample < 0 || cfg.power_iters < 0 || cfg.power_iters > 8 || cfg.max_jacobi_sweeps <= 0)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: bad sketch or solver option");
+  if ((cfg.bits_mask & 0x1FFu) == 0 || (cfg.bits_mask & ~0x1FFu))
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: bits_mask must select widths in 0..8");
+  if (cfg.rt_max < 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: rt_max < 0");
+  if (byte_budget == 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: zero byte budget");
+
+  jolt_plan_s* p = new (std::nothrow) jolt_plan_s();
+  if (!p) return fail(JOLT_ERR_OOM, "jolt_plan: host allocation");
+  p->shape = sh;
+  p->cfg = cfg;
+  p->budget = byte_budget;
+  p->G = num_groups;
+  p->step = cfg.rank_step;
+  const int L = sh.layers, H = sh.heads, T = sh.tokens, D = sh.head_dim;
+  const int kinds = sh.has_v ? 2 : 1;
+  p->n_lt = L * kinds;
+  for (int k = 0; k < kinds; ++k)
+    for (int l = 0; l < L; ++l) p->lt_ids.push_back(2 * l + k);
+  const int64_t per_lt = (int64_t)(byte_budget / (uint64_t)p->n_lt);
+  int cap = 112;
+  if (cfg.rt_max > 0) cap = std::min(cap, (int)cfg.rt_max);
+  int64_t R = std::min<int64_t>({(int64_t)T, (int64_t)H * D, per_lt / (2 * (int64_t)T), (int64_t)cap});
+  R -= R % p->step;
+  p->R = (int)std::max<int64_t>(0, R);
+  int enc = cfg.encoder;
+  if (enc == JOLT_ENC_AUTO) enc = T <= 1024 ? JOLT_ENC_EXACT : JOLT_ENC_SKETCH;
+  if (enc == JOLT_ENC_EXACT && T > kMaxN) {
+    delete p;
+    return fail(JOLT_ERR_UNSUPPORTED, "jolt_plan: exact token factor needs tokens <= %d in this build", kMaxN);
+  }
+  p->encoder = enc;
+  if (enc == JOLT_ENC_SKETCH) {
+    int l = (int)std::min<int64_t>({(int64_t)p->R + cfg.oversample, (int64_t)T, (int64_t)H * D});
+    if (l > kMaxN || (l & 1) || l < p->R || l <= 0) {
+      delete p;
+      return fail(JOLT_ERR_UNSUPPORTED, "jolt_plan: sketch width %d must be even, >= r_t max and <= %d", l, kMaxN);
+    }
+    p->l = l;
+  } else {
+    if (T & 1) {
+      delete p;
+      return fail(JOLT_ERR_UNSUPPORTED, "jolt_plan: exact path needs an even token count");
+    }
+  }
+  p->nbits = 0;
+  for (int b = 0; b <= 8; ++b)
+    if (cfg.bits_mask & (1u << b)) p->bits[p->nbits++] = b;
+  p->kappa = kappa_of(D);
+  for (int i = 0; i < p->nbits; ++i)
+    p->phi[i] = p->bits[i] == 0 ? 1.0 : p->kappa / (3.0 * std::pow(4.0, p->bits[i]));
+  p->ngrid = 1 + (p->R / p->step) * (D / p->step);
+  if (sh.has_v && cfg.split_kv_budget) {
+    p->pool_budget[0] = (int64_t)(byte_budget / 2);
+    p->pool_budget[1] = (int64_t)byte_budget - p->pool_budget[0];
+  } else {
+    p->pool_budget[0] = (int64_t)byte_budget;
+  }
+  // feasibility: the cheapest candidate of every unit must fit its pool
+  {
+    int64_t minb_lt = INT64_MAX;
+    for (int bi = 0; bi < p->nbits; ++bi) {
+      const int b = p->bits[bi];
+      minb_lt = std::min(minb_lt, lt_bytes_h(H, T, D, 0, 0, b));
+      if (p->R >= p->step) minb_lt = std::min(minb_lt, lt_bytes_h(H, T, D, p->step, p->step, b));
+    }
+    const int npools = (sh.has_v && cfg.split_kv_budget) ? 2 : 1;
+    const int64_t per_pool_lts = npools == 2 ? L : (int64_t)p->n_lt;
+    if (minb_lt * per_pool_lts > p->pool_budget[0]) {
+      delete p;
+      return fail(JOLT_ERR_BUDGET_INFEASIBLE, "jolt_plan: minimum %lld bytes exceed the budget",
+                  (long long)(minb_lt * per_pool_lts));
+    }
+  }
+  // workspace
+  const int64_t n = p->n_lt, HD = (int64_t)H * D, Rm = std::max(p->R, 1), l = std::max(p->l, 2);
+  auto layout = [&](char* base, bool assign) -> size_t {
+    char* cur = base;
+    auto take = [&](auto*& ptr, size_t count) {
+      using T_ = std::remove_reference_t<decltype(*ptr)>;
+      T_* v = carve<T_>(cur, count);
+      if (assign) ptr = v;
+    };
+    take(p->xx, n);
+    take(p->xx_part, n * 64);
+    take(p->CD, n * D * D);
+    take(p->UD32, n * D * D);
+    take(p->UDf, n * D * D);
+    take(p->lamD, n * D);
+    take(p->UDb, n * D * D);
+    take(p->UT32, n * T * Rm);
+    take(p->UTf, n * T * Rm);
+    take(p->UTb, n * T * Rm);
+    take(p->P, n * H * Rm * D);
+    take(p->Gmax, n * H * Rm * D);
+    take(p->E, 2 * (int64_t)L * p->ngrid);
+    take(p->unit_err, 2 * (int64_t)p->G * p->nbits * p->ngrid);
+    take(p->Nbuf, n * H * Rm * D);
+    take(p->Gpi, (int64_t)D * D);
+    take(p->Pi32, (int64_t)D * D);
+    take(p->Pib, (int64_t)D * D);
+    if (p->encoder == JOLT_ENC_SKETCH) {
+      take(p->Om, n * HD * l);
+      take(p->Y, n * T * l);
+      take(p->Y2, n * T * l);
+      take(p->Z, n * HD * l);
+      take(p->Z2, n * HD * l);
+      take(p->Wg, n * l * l);
+      take(p->Rinv, n * l * l);
+      take(p->Bm, n * l * HD);
+      take(p->BB, n * l * l);
+      take(p->Wv, n * l * l);
+      take(p->lamB, n * l);
+    } else {
+      take(p->CT, n * T * T);
+      take(p->VT, n * T * T);
+      take(p->lamT, n * T);
+    }
+    return (size_t)(cur - base) + 256;
+  };
+  p->ws_bytes = layout(nullptr, false);
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e == cudaSuccess) e = cudaMalloc(&p->ws, p->ws_bytes);
+  if (e == cudaSuccess) e = cudaMalloc(&p->d_lt_ids, sizeof(int32_t) * p->lt_ids.size());
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->d_lt_ids, p->lt_ids.data(), sizeof(int32_t) * p->lt_ids.size(), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    jolt_status st = fail(e == cudaErrorMemoryAllocation ? JOLT_ERR_OOM : JOLT_ERR_CUDA,
+                          "jolt_plan: workspace of %zu bytes: %s", p->ws_bytes, cudaGetErrorString(e));
+    if (p->ws) cudaFree(p->ws);
+    if (p->d_lt_ids) cudaFree(p->d_lt_ids);
+    delete p;
+    return st;
+  }
+  layout(reinterpret_cast<char*>(align_up(reinterpret_cast<size_t>(p->ws), 256)), true);
+  *out = p;
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_plan_info(jolt_plan_t p, int32_t* rt_max, int32_t* sketch_l, int32_t* encoder,
+                                    uint64_t* workspace_bytes) {
+  if (!p) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan_info: null plan");
+  if (rt_max) *rt_max = p->R;
+  if (sketch_l) *sketch_l = p->encoder == JOLT_ENC_SKETCH ? p->l : 0;
+  if (encoder) *encoder = p->encoder;
+  if (workspace_bytes) *workspace_bytes = p->ws_bytes;
+  return JOLT_OK;
+}
+
+static jolt_status make_stream(jolt_plan_s* p, uint64_t seed, cudaStream_t cs, jolt_stream_s** out) {
+  jolt_stream_s* st = new (std::nothrow) jolt_stream_s();
+  if (!st) return fail(JOLT_ERR_OOM, "stream: host allocation");
+  const jolt_shape& sh = p->shape;
+  st->L = sh.layers; st->H = sh.heads; st->T = sh.tokens; st->D = sh.head_dim;
+  st->has_v = sh.has_v ? 1 : 0; st->G = p->G; st->encoder = p->encoder; st->step = p->step;
+  st->R = p->R; st->split = (sh.has_v && p->cfg.split_kv_budget) ? 1 : 0; st->dtype = sh.dtype;
+  st->seed = seed; st->cs = cs; st->plan = p; st->n_lt = p->n_lt;
+  st->body_cap = align_up((size_t)p->budget + (size_t)JOLT_NUM_PARTS * kAlign * p->n_lt + kAlign, kAlign);
+  cudaError_t e = cudaMallocAsync(&st->d_body, st->body_cap, cs);
+  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_meta, sizeof(StreamMeta), cs);
+  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_Pi, sizeof(float) * kD * kD, cs);
+  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_lt_ids, sizeof(int32_t) * p->n_lt, cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->d_meta, 0, sizeof(StreamMeta), cs);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(st->d_lt_ids, p->d_lt_ids, sizeof(int32_t) * p->n_lt, cudaMemcpyDeviceToDevice, cs);
+  if (e != cudaSuccess) {
+    jolt_stream_destroy(st);
+    return fail(e == cudaErrorMemoryAllocation ? JOLT_ERR_OOM : JOLT_ERR_CUDA, "stream allocation: %s",
+                cudaGetErrorString(e));
+  }
+  *out = st;
+  return JOLT_OK;
+}
+
+static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], uint64_t seed, cudaStream_t s) {
+  const jolt_shape& sh = p->shape;
+  const int L = sh.layers, H = sh.heads, T = sh.tokens, D = sh.head_dim, R = p->R;
+  const int kinds = sh.has_v ? 2 : 1;
+  const int n = p->n_lt;
+  const int64_t HD = (int64_t)H * D, HTD = (int64_t)H * T * D;
+  const ElemType xt = sh.dtype == JOLT_BF16 ? EL_BF16 : EL_F32;
+  int32_t* status = &st->d_meta->status;
+  {
+    PROF("check_norms", s);
+    for (int k = 0; k < kinds; ++k) {
+      CK(check_finite(L * HTD, X[k], xt, status, s));
+      CK(sumsq_batched(L, HTD, X[k], xt, HTD, p->xx + (int64_t)k * L, p->xx_part + (int64_t)k * L * 64, s));
+    }
+  }
+  {
+    PROF("feature_gram", s);
+    // C_D = sum over rows r = (h, t) of X[r, :]^T X[r, :]
+    for (int k = 0; k < kinds; ++k)
+      CK(gemm_simt(L, D, D, H * T, opnd(X[k], xt, I1(HTD), I1(1), I1(D)), opnd(X[k], xt, I1(HTD), I1(1), I1(D)),
+                   outd(p->CD + (int64_t)k * L * D * D, EL_F32, I1((int64_t)D * D), I1(D), I1(1)), 1.0, 0.0, s));
+  }
+  {
+    PROF("jacobi_feature", s);
+    CK(jacobi_eig(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, p->cfg.max_jacobi_sweeps,
+                  status, s));
+  }
+  {
+    PROF("sign_round", s);
+    CK(sign_fix(n, D, D, p->UD32, D, (int64_t)D * D, nullptr, 0, 0, 0, s));
+    CK(round_bf16((int64_t)n * D * D, p->UD32, p->UDb, p->UDf, s));
+  }
+  if (R > 0) {
+    if (p->encoder == JOLT_ENC_SKETCH) {
+      const int l = p->l;
+      {
+        PROF("sketch_omega", s);
+        std::vector<int32_t> ids = p->lt_ids;
+        CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, s));
+      }
+      jolt_status r;
+      {
+        PROF("sketch_gemm", s);
+        // Y0 = A Omega, A[t, h*D + d] = X[h][t][d]
+        for (int k = 0; k < kinds; ++k)
+          CK(gemm_simt(L, T, l, (int)HD, opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
+                       opnd(p->Om + (int64_t)k * L * HD * l, EL_BF16, I1(HD * l), I1(1), I1(l)),
+                       outd(p->Y + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(l), I1(1)), 1.0, 0.0, s));
+      }
+      {
+        PROF("cholqr", s);
+        r = cholqr3(p, T, p->Y, p->Y2, status, s);
+        if (r != JOLT_OK) return r;
+      }
+      for (int it = 0; it < p->cfg.power_iters; ++it) {
+        {
+          PROF("sketch_gemm", s);
+          // Z = A^T Q  (HD x l)
+          for (int k = 0; k < kinds; ++k)
+            CK(gemm_simt(L, (int)HD, l, T, opnd(X[k], xt, I1(HTD), I2(D, 1, (int64_t)T * D), I1(D)),
+                         opnd(p->Y2 + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(1), I1(l)),
+                         outd(p->Z + (int64_t)k * L * HD * l, EL_F32, I1(HD * l), I1(l), I1(1)), 1.0, 0.0, s));
+        }
+        {
+          PROF("cholqr", s);
+          r = cholqr3(p, (int)HD, p->Z, p->Z2, status, s);
+          if (r != JOLT_OK) return r;
+        }
+        {
+          PROF("sketch_gemm", s);
+          // Y = A Q'
+          for (int k = 0; k < kinds; ++k)
+            CK(gemm_simt(L, T, l, (int)HD, opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
+                         opnd(p->Z2 + (int64_t)k * L * HD * l, EL_F32, I1(HD * l), I1(1), I1(l)),
+                         outd(p->Y + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(l), I1(1)), 1.0, 0.0, s));
+        }
+        {
+          PROF("cholqr", s);
+          r = cholqr3(p, T, p->Y, p->Y2, status, s);
+          if (r != JOLT_OK) return r;
+        }
+      }
+      {
+        PROF("sketch_gemm", s);
+        // B = Q^T A (l x HD)
+        for (int k = 0; k < kinds; ++k)
+          CK(gemm_simt(L, l, (int)HD, T, opnd(p->Y2 + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(1), I1(l)),
+                       opnd(X[k], xt, I1(HTD), I2(D, 1, (int64_t)T * D), I1(D)),
+                       outd(p->Bm + (int64_t)k * L * l * HD, EL_F32, I1(l * HD), I1(HD), I1(1)), 1.0, 0.0, s));
+      }
+      {
+        PROF("small_gemm", s);
+        // B B^T
+        CK(gemm_simt(n, l, l, (int)HD, opnd(p->Bm, EL_F32, I1(l * HD), I1(HD), I1(1)),
+                     opnd(p->Bm, EL_F32, I1(l * HD), I1(HD), I1(1)),
+                     outd(p->BB, EL_F32, I1((int64_t)l * l), I1(l), I1(1)), 1.0, 0.0, s));
+      }
+      {
+        PROF("jacobi_sketch", s);
+        CK(jacobi_eig(n, l, p->BB, (int64_t)l * l, p->Wv, (int64_t)l * l, p->lamB, l, p->cfg.max_jacobi_sweeps,
+                      status, s));
+      }
+      {
+        PROF("small_gemm", s);
+        // U_T = Q W[:, :R]
+        CK(gemm_simt(n, T, R, l, opnd(p->Y2, EL_F32, I1((int64_t)T * l), I1(l), I1(1)),
+                     opnd(p->Wv, EL_F32, I1((int64_t)l * l), I1(1), I1(l)),
+                     outd(p->UT32, EL_F32, I1((int64_t)T * R), I1(R), I1(1)), 1.0, 0.0, s));
+      }
+      {
+        PROF("sign_round", s);
+        CK(sign_fix(n, T, R, p->UT32, R, (int64_t)T * R, p->Wv, l, l, (int64_t)l * l, s));
+        CK(round_bf16((int64_t)n * T * R, p->UT32, p->UTb, p->UTf, s));
+      }
+      {
+        PROF("core", s);
+        // core: P[h] = W_R^T B_h (R x D); G_max[h] = P[h] U_D(rounded) below
+        CK(gemm_simt(n * H, R, D, l, opnd(p->Wv, EL_F32, I2(H, 0, (int64_t)l * l), I1(1), I1(l)),
+                     opnd(p->Bm, EL_F32, I2(H, D, l * HD), I1(1), I1(HD)),
+                     outd(p->P, EL_F32, I1((int64_t)R * D), I1(D), I1(1)), 1.0, 0.0, s));
+      }
+    } else {
+      {
+        PROF("token_gram", s);
+        // exact: C_T = A A^T (T x T), all eigenvectors, keep the leading R
+        for (int k = 0; k < kinds; ++k)
+          CK(gemm_simt(L, T, T, (int)HD, opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
+                       opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
+                       outd(p->CT + (int64_t)k * L * T * T, EL_F32, I1((int64_t)T * T), I1(T), I1(1)), 1.0, 0.0, s));
+      }
+      {
+        PROF("jacobi_token", s);
+        CK(jacobi_eig(n, T, p->CT, (int64_t)T * T, p->VT, (int64_t)T * T, p->lamT, T, p->cfg.max_jacobi_sweeps,
+                      status, s));
+      }
+      {
+        PROF("sign_round", s);
+        CK(cudaMemcpy2DAsync(p->UT32, sizeof(float) * R, p->VT, sizeof(float) * T, sizeof(float) * R,
+                             (size_t)n * T, cudaMemcpyDeviceToDevice, s));
+        CK(sign_fix(n, T, R, p->UT32, R, (int64_t)T * R, nullptr, 0, 0, 0, s));
+        CK(round_bf16((int64_t)n * T * R, p->UT32, p->UTb, p->UTf, s));
+      }
+      {
+        PROF("core", s);
+        // P[h] = U_T(rounded)^T X_h  (R x D)
+        for (int k = 0; k < kinds; ++k)
+          CK(gemm_simt(L * H, R, D, T, opnd(p->UTf + (int64_t)k * L * T * R, EL_F32, I2(H, 0, (int64_t)T * R), I1(1), I1(R)),
+                       opnd(X[k], xt, I1((int64_t)T * D), I1(1), I1(D)),
+                       outd(p->P + (int64_t)k * L * H * R * D, EL_F32, I1((int64_t)R * D), I1(D), I1(1)), 1.0, 0.0, s));
+      }
+    }
+    {
+      PROF("core", s);
+      CK(gemm_simt(n * H, R, D, D, opnd(p->P, EL_F32, I1((int64_t)R * D), I1(D), I1(1)),
+                   opnd(p->UDf, EL_F32, I2(H, 0, (int64_t)D * D), I1(1), I1(D)),
+                   outd(p->Gmax, EL_F32, I1((int64_t)R * D), I1(D), I1(1)), 1.0, 0.0, s));
+    }
+  }
+  {
+    PROF("energy_table", s);
+    TableArgs ta;
+    ta.n_lt = n; ta.H = H; ta.R = R; ta.D = D; ta.step = p->step; ta.lt_ids = p->d_lt_ids;
+    ta.Gmax = p->Gmax; ta.xx = p->xx; ta.E = p->E; ta.ngrid = p->ngrid;
+    CK(energy_table(ta, s));
+  }
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, uint64_t seed, void* cuda_stream,
+                                 jolt_stream_t* out) {
+  g_err.clear();
+  if (!p || !K || !out) return fail(JOLT_ERR_INVALID_ARG, "jolt_encode: null plan, K or out");
+  if (p->shape.has_v && !V) return fail(JOLT_ERR_INVALID_ARG, "jolt_encode: the plan has V but V is null");
+  *out = nullptr;
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  CK(cudaSetDevice(p->device));
+  jolt_stream_s* st = nullptr;
+  jolt_status r = make_stream(p, seed, s, &st);
+  if (r != JOLT_OK) return r;
+  const jolt_shape& sh = p->shape;
+  const int D = sh.head_dim;
+  auto bail = [&](jolt_status x) { jolt_stream_destroy(st); return x; };
+  // rotation Pi for this seed (cached in the plan), copied into the stream for decode
+  if (!(p->pi_valid && p->pi_seed == seed)) {
+    PROF("rotation", s);
+    cudaError_t e = gauss_f64(seed, 1, (int64_t)D * D, p->Gpi, s);
+    if (e == cudaSuccess) e = haar_from_gauss(p->Gpi, D, p->Pi32, p->Pib, s);
+    if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "rotation: %s", cudaGetErrorString(e)));
+    p->pi_valid = true;
+    p->pi_seed = seed;
+  }
+  cudaError_t e = cudaMemcpyAsync(st->d_Pi, p->Pi32, sizeof(float) * D * D, cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "copy Pi: %s", cudaGetErrorString(e)));
+  const void* X[2] = {K, V};
+  r = analyse(p, st, X, seed, s);
+  if (r != JOLT_OK) return bail(r);
+  DualArgs da;
+  da.L = sh.layers; da.H = sh.heads; da.T = sh.tokens; da.D = D; da.G = p->G; da.has_v = sh.has_v ? 1 : 0;
+  da.step = p->step; da.R = p->R; da.split = st->split; da.nbits = p->nbits;
+  for (int i = 0; i < 9; ++i) { da.bits[i] = p->bits[i]; da.phi[i] = p->phi[i]; }
+  da.budget_pool[0] = p->pool_budget[0]; da.budget_pool[1] = p->pool_budget[1];
+  da.ngrid = p->ngrid; da.E = p->E; da.unit_err = p->unit_err; da.meta = st->d_meta;
+  {
+    PROF("dual", s);
+    e = dual_allocate(da, s);
+  }
+  if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "dual: %s", cudaGetErrorString(e)));
+  PackArgs pa;
+  pa.n_lt = p->n_lt; pa.H = sh.heads; pa.T = sh.tokens; pa.D = D; pa.R = std::max(p->R, 1);
+  pa.lt_ids = p->d_lt_ids; pa.UT = p->UTb; pa.UD = p->UDb; pa.Gmax = p->Gmax; pa.meta = st->d_meta;
+  pa.body = st->d_body;
+  {
+    PROF("pack", s);
+    e = pack_factors(pa, s);
+  }
+  if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "pack: %s", cudaGetErrorString(e)));
+  ResidualArgs ra;
+  ra.n_lt = p->n_lt; ra.H = sh.heads; ra.T = sh.tokens; ra.D = D; ra.lt_ids = p->d_lt_ids;
+  ra.X[0] = K; ra.X[1] = V; ra.xt = sh.dtype == JOLT_BF16 ? EL_BF16 : EL_F32; ra.Pi = st->d_Pi;
+  ra.meta = st->d_meta; ra.body = st->d_body;
+  {
+    PROF("residual", s);
+    e = residual_encode(ra, p->Nbuf, std::max(p->R, 1), s);
+  }
+  if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "residual: %s", cudaGetErrorString(e)));
+  p->last = st;
+  *out = st;
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_decode(jolt_stream_t st, void* K_out, void* V_out, void* cuda_stream) {
+  g_err.clear();
+  if (!st || !K_out) return fail(JOLT_ERR_INVALID_ARG, "jolt_decode: null stream or K_out");
+  if (st->has_v && !V_out) return fail(JOLT_ERR_INVALID_ARG, "jolt_decode: stream has V but V_out is null");
+  DecodeArgs a;
+  a.n_lt = st->n_lt; a.H = st->H; a.T = st->T; a.D = st->D; a.lt_ids = st->d_lt_ids;
+  a.out[0] = K_out; a.out[1] = V_out; a.ot = st->dtype == JOLT_BF16 ? EL_BF16 : EL_F32;
+  a.Pi = st->d_Pi; a.meta = st->d_meta; a.body = st->d_body;
+  PROF("decode", (cudaStream_t)cuda_stream);
+  CK(decode(a, (cudaStream_t)cuda_stream));
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, uint64_t n, jolt_dtype dtype,
+                                         void* cuda_stream, double* out) {
+  g_err.clear();
+  if (!ref || !approx || !out) return fail(JOLT_ERR_INVALID_ARG, "jolt_rel_frob_error: null pointer");
+  if (dtype != JOLT_BF16 && dtype != JOLT_F32) return fail(JOLT_ERR_INVALID_ARG, "jolt_rel_frob_error: dtype");
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  const int nb = relfrob_blocks(n);
+  Prof prof_rf("rel_frob", s);
+  double* scratch = nullptr;
+  CK(cudaMallocAsync(&scratch, sizeof(double) * (2 * (size_t)nb + 2), s));
+  cudaError_t e = relfrob_partial(ref, approx, n, dtype == JOLT_BF16 ? EL_BF16 : EL_F32, scratch + 2, nb, scratch, s);
+  double h[2] = {0.0, 0.0};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h, scratch, sizeof(h), cudaMemcpyDeviceToHost, s);
+  cudaError_t e2 = cudaFreeAsync(scratch, s);
+  if (e == cudaSuccess) e = e2;
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_rel_frob_error: %s", cudaGetErrorString(e));
+  *out = h[1] > 0.0 ? std::sqrt(h[0]) / std::sqrt(h[1]) : 0.0;
+  return JOLT_OK;
+}
+
+static jolt_status read_meta(jolt_stream_s* st, StreamMeta* m) {
+  CK(cudaStreamSynchronize(st->cs));
+  CK(cudaMemcpy(m, st->d_meta, sizeof(StreamMeta), cudaMemcpyDeviceToHost));
+  return JOLT_OK;
+}
+
+static jolt_status status_of(int32_t bits) {
+  if (bits & ST_NONFINITE) return fail(JOLT_ERR_NONFINITE, "non-finite value in the input");
+  if (bits & ST_INFEASIBLE) return fail(JOLT_ERR_BUDGET_INFEASIBLE, "budget infeasible");
+  if (bits & ST_TIMEOUT) return fail(JOLT_ERR_TIMEOUT, "a bounded device wait gave up");
+  if (bits & ST_NOT_CONVERGED) return fail(JOLT_ERR_NOT_CONVERGED, "an eigensolver or Cholesky step hit its limit");
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_stream_status(jolt_stream_t st) {
+  g_err.clear();
+  if (!st) return fail(JOLT_ERR_INVALID_ARG, "jolt_stream_status: null stream");
+  StreamMeta m;
+  jolt_status r = read_meta(st, &m);
+  if (r != JOLT_OK) return r;
+  return status_of(m.status);
+}
+
+JOLT_API jolt_status jolt_stream_info(jolt_stream_t st, uint64_t* bytes_by_part, int32_t* alloc, double* lambdas) {
+  g_err.clear();
+  if (!st) return fail(JOLT_ERR_INVALID_ARG, "jolt_stream_info: null stream");
+  StreamMeta m;
+  jolt_status r = read_meta(st, &m);
+  if (r != JOLT_OK) return r;
+  if (bytes_by_part)
+    for (int i = 0; i < JOLT_NUM_PARTS; ++i) bytes_by_part[i] = (uint64_t)m.bytes_by_part[i];
+  if (alloc)
+    for (int g = 0; g < st->G; ++g)
+      for (int k = 0; k < 2; ++k)
+        for (int j = 0; j < 3; ++j) alloc[(g * 2 + k) * 3 + j] = m.alloc[g][k][j];
+  if (lambdas) { lambdas[0] = m.lambda[0]; lambdas[1] = m.lambda[1]; }
+  return status_of(m.status);
+}
+
+// ---------------------------------------------------------------- serialization
+static size_t header_bytes(int G) { return align_up(64 + 24 * (size_t)G, 16); }
+
+static void put32(std::vector<uint8_t>& b, size_t off, uint32_t v) { memcpy(&b[off], &v, 4); }
+static void put64(std::vector<uint8_t>& b, size_t off, uint64_t v) { memcpy(&b[off], &v, 8); }
+
+JOLT_API jolt_status jolt_stream_to_host(jolt_stream_t st, void* buf, uint64_t* len) {
+  g_err.clear();
+  if (!st || !len) return fail(JOLT_ERR_INVALID_ARG, "jolt_stream_to_host: null stream or len");
+  StreamMeta m;
+  jolt_status r = read_meta(st, &m);
+  if (r != JOLT_OK) return r;
+  if (m.status & (ST_NONFINITE | ST_INFEASIBLE)) return status_of(m.status);
+  const size_t hb = header_bytes(st->G);
+  const size_t total = hb + (size_t)m.body_bytes + 4;
+  if (!buf) { *len = total; return JOLT_OK; }
+  if (*len < total) return fail(JOLT_ERR_INVALID_ARG, "jolt_stream_to_host: buffer of %llu < %zu bytes",
+                                (unsigned long long)*len, total);
+  std::vector<uint8_t> head(hb, 0);
+  memcpy(&head[0], "JOLT", 4);
+  put32(head, 4, 1);
+  put32(head, 8, (uint32_t)hb);
+  const uint32_t flags = (uint32_t)st->has_v | ((st->dtype == JOLT_F32 ? 1u : 0u) << 1) |
+                         ((uint32_t)st->split << 2) | ((uint32_t)st->encoder << 8);
+  put32(head, 12, flags);
+  const int32_t ints[8] = {st->L, st->H, st->T, st->D, st->G, st->step, st->R, 0};
+  memcpy(&head[16], ints, sizeof(ints));
+  put64(head, 48, st->seed);
+  put64(head, 56, (uint64_t)m.body_bytes);
+  for (int g = 0; g < st->G; ++g)
+    for (int k = 0; k < 2; ++k) {
+      int32_t a3[3] = {0, 0, 0};
+      if (k == 0 || st->has_v)
+        for (int j = 0; j < 3; ++j) a3[j] = m.alloc[g][k][j];
+      memcpy(&head[64 + 24 * g + 12 * k], a3, 12);
+    }
+  uint8_t* o = reinterpret_cast<uint8_t*>(buf);
+  memcpy(o, head.data(), hb);
+  CK(cudaMemcpy(o + hb, st->d_body, (size_t)m.body_bytes, cudaMemcpyDeviceToHost));
+  // padding between parts is not guaranteed zero on the device: clear it on the host
+  {
+    size_t cur = 0;
+    for (int l = 0; l < st->L; ++l)
+      for (int k = 0; k < (st->has_v ? 2 : 1); ++k) {
+        const int lt = 2 * l + k;
+        const int rt = m.lt_rank[lt][0], rd = m.lt_rank[lt][1], b = m.lt_rank[lt][2];
+        const size_t sz[5] = {(size_t)st->T * rt * 2, (size_t)st->D * rd * 2, (size_t)st->H * rt * rd * 2,
+                              b > 0 ? (size_t)st->H * st->T * 2 : 0,
+                              b > 0 ? (size_t)st->H * st->T * (st->D * b / 8) : 0};
+        for (int pp = 0; pp < 5; ++pp) {
+          const size_t off = (size_t)m.off[lt][pp];
+          if (off > cur) memset(o + hb + cur, 0, off - cur);
+          cur = off + sz[pp];
+        }
+      }
+  }
+  const uint32_t crc = crc32_ieee(o, hb + (size_t)m.body_bytes);
+  memcpy(o + hb + (size_t)m.body_bytes, &crc, 4);
+  *len = total;
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_stream_from_host(const void* buf, uint64_t len, void* cuda_stream, jolt_stream_t* out) {
+  g_err.clear();
+  if (!buf || !out) return fail(JOLT_ERR_INVALID_ARG, "jolt_stream_from_host: null pointer");
+  *out = nullptr;
+  const uint8_t* b = reinterpret_cast<const uint8_t*>(buf);
+  if (len < 68 || memcmp(b, "JOLT", 4) != 0) return fail(JOLT_ERR_CORRUPT_STREAM, "bad magic or short buffer");
+  uint32_t ver, hb, flags;
+  memcpy(&ver, b + 4, 4);
+  memcpy(&hb, b + 8, 4);
+  memcpy(&flags, b + 12, 4);
+  if (ver != 1) return fail(JOLT_ERR_CORRUPT_STREAM, "unsupported version %u", ver);
+  int32_t ints[8];
+  memcpy(ints, b + 16, sizeof(ints));
+  uint64_t seed, body;
+  memcpy(&seed, b + 48, 8);
+  memcpy(&body, b + 56, 8);
+  const int L = ints[0], H = ints[1], T = ints[2], D = ints[3], G = ints[4];
+  if (L <= 0 || L > kMaxL || H <= 0 || T <= 0 || D != kD || G <= 0 || G > L || G > kMaxGroups)
+    return fail(JOLT_ERR_CORRUPT_STREAM, "header shape out of range");
+  if (hb != header_bytes(G) || len != (uint64_t)hb + body + 4) return fail(JOLT_ERR_CORRUPT_STREAM, "size mismatch");
+  uint32_t crc;
+  memcpy(&crc, b + hb + body, 4);
+  if (crc != crc32_ieee(b, hb + body)) return fail(JOLT_ERR_CORRUPT_STREAM, "CRC mismatch");
+  const int has_v = flags & 1;
+  StreamMeta m;
+  memset(&m, 0, sizeof(m));
+  for (int g = 0; g < G; ++g)
+    for (int k = 0; k < 2; ++k) memcpy(m.alloc[g][k], b + 64 + 24 * g + 12 * k, 12);
+  int64_t cur = 0;
+  for (int l = 0; l < L; ++l) {
+    const int g = group_of_layer(l, L, G);
+    for (int k = 0; k < (has_v ? 2 : 1); ++k) {
+      const int lt = 2 * l + k;
+      const int rt = m.alloc[g][k][0], rd = m.alloc[g][k][1], bb = m.alloc[g][k][2];
+      if (rt < 0 || rt > kMaxN || rd < 0 || rd > D || bb < 0 || bb > 8 || (rt == 0) != (rd == 0))
+        return fail(JOLT_ERR_CORRUPT_STREAM, "allocation table out of range");
+      m.lt_rank[lt][0] = rt; m.lt_rank[lt][1] = rd; m.lt_rank[lt][2] = bb;
+      const int64_t sz[5] = {(int64_t)T * rt * 2, (int64_t)D * rd * 2, (int64_t)H * rt * rd * 2,
+                             bb > 0 ? (int64_t)H * T * 2 : 0, bb > 0 ? (int64_t)H * T * (D * bb / 8) : 0};
+      for (int pp = 0; pp < 5; ++pp) {
+        const int64_t off = (cur + kAlign - 1) / kAlign * kAlign;
+        m.off[lt][pp] = off;
+        cur = off + sz[pp];
+        m.bytes_by_part[pp] += sz[pp];
+      }
+    }
+  }
+  if ((uint64_t)cur != body) return fail(JOLT_ERR_CORRUPT_STREAM, "body size does not match the allocation table");
+  m.body_bytes = cur;
+  m.num_lt = L * (has_v ? 2 : 1);
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  jolt_stream_s* st = new (std::nothrow) jolt_stream_s();
+  if (!st) return fail(JOLT_ERR_OOM, "host allocation");
+  st->L = L; st->H = H; st->T = T; st->D = D; st->has_v = has_v; st->G = G;
+  st->encoder = (flags >> 8) & 0xFF; st->step = ints[5]; st->R = ints[6]; st->split = (flags >> 2) & 1;
+  st->dtype = (flags & 2) ? JOLT_F32 : JOLT_BF16; st->seed = seed; st->cs = s; st->n_lt = m.num_lt;
+  st->body_cap = std::max<size_t>((size_t)body, 256);
+  std::vector<int32_t> ids;
+  for (int k = 0; k < (has_v ? 2 : 1); ++k)
+    for (int l = 0; l < L; ++l) ids.push_back(2 * l + k);
+  cudaError_t e = cudaMallocAsync(&st->d_body, st->body_cap, s);
+  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_meta, sizeof(StreamMeta), s);
+  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_Pi, sizeof(float) * D * D, s);
+  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_Gpi, sizeof(double) * D * D, s);
+  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_lt_ids, sizeof(int32_t) * ids.size(), s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->d_body, b + hb, (size_t)body, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->d_meta, &m, sizeof(m), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(st->d_lt_ids, ids.data(), sizeof(int32_t) * ids.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = gauss_f64(seed, 1, (int64_t)D * D, st->d_Gpi, s);
+  if (e == cudaSuccess) e = haar_from_gauss(st->d_Gpi, D, st->d_Pi, nullptr, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);   // host buffers above are stack / vector
+  if (e != cudaSuccess) {
+    jolt_stream_destroy(st);
+    return fail(JOLT_ERR_CUDA, "jolt_stream_from_host: %s", cudaGetErrorString(e));
+  }
+  *out = st;
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_export_debug(jolt_stream_t st, int32_t what, int32_t lt, void* buf, uint64_t* len) {
+  g_err.clear();
+  if (!st || !len) return fail(JOLT_ERR_INVALID_ARG, "jolt_export_debug: null stream or len");
+  CK(cudaStreamSynchronize(st->cs));
+  jolt_plan_s* p = st->plan;
+  const void* src = nullptr;
+  size_t n = 0;
+  bool host_src = false;
+  StreamMeta m;
+  std::vector<double> tmp;
+  auto index_of = [&](int lt_) -> int {
+    if (!p) return -1;
+    for (size_t i = 0; i < p->lt_ids.size(); ++i)
+      if (p->lt_ids[i] == lt_) return (int)i;
+    return -1;
+  };
+  if (what == JOLT_DBG_PI) {
+    src = st->d_Pi;
+    n = sizeof(float) * st->D * st->D;
+  } else if (what == JOLT_DBG_LAMBDA) {
+    CK(cudaMemcpy(&m, st->d_meta, sizeof(m), cudaMemcpyDeviceToHost));
+    tmp.assign(m.lambda, m.lambda + 2);
+    src = tmp.data();
+    n = sizeof(double) * 2;
+    host_src = true;
+  } else {
+    if (!p || p->last != st) return fail(JOLT_ERR_INVALID_ARG, "jolt_export_debug: plan no longer holds this stream's encode");
+    const int i = index_of(lt);
+    switch (what) {
+      case JOLT_DBG_UT_F32:
+        if (i < 0) return fail(JOLT_ERR_INVALID_ARG, "bad lt");
+        src = p->UT32 + (int64_t)i * st->T * p->R;
+        n = sizeof(float) * st->T * p->R;
+        break;
+      case JOLT_DBG_UD_F32:
+        if (i < 0) return fail(JOLT_ERR_INVALID_ARG, "bad lt");
+        src = p->UD32 + (int64_t)i * st->D * st->D;
+        n = sizeof(float) * st->D * st->D;
+        break;
+      case JOLT_DBG_TABLE:
+        if (lt < 0 || lt >= 2 * st->G) return fail(JOLT_ERR_INVALID_ARG, "bad unit");
+        src = p->unit_err + (int64_t)lt * p->nbits * p->ngrid;
+        n = sizeof(double) * p->nbits * p->ngrid;
+        break;
+      case JOLT_DBG_XX:
+        tmp.assign(2 * (size_t)st->L, 0.0);
+        for (size_t j = 0; j < p->lt_ids.size(); ++j)
+          CK(cudaMemcpy(&tmp[p->lt_ids[j]], p->xx + j, sizeof(double), cudaMemcpyDeviceToHost));
+        src = tmp.data();
+        n = sizeof(double) * tmp.size();
+        host_src = true;
+        break;
+      case JOLT_DBG_OMEGA:
+        if (i < 0 || p->encoder != JOLT_ENC_SKETCH) return fail(JOLT_ERR_INVALID_ARG, "no sketch for this lt");
+        src = p->Om + (int64_t)i * st->H * st->D * p->l;
+        n = sizeof(__nv_bfloat16) * st->H * st->D * p->l;
+        break;
+      default:
+        return fail(JOLT_ERR_INVALID_ARG, "jolt_export_debug: unknown item %d", what);
+    }
+  }
+  if (!buf) { *len = n; return JOLT_OK; }
+  if (*len < n) return fail(JOLT_ERR_INVALID_ARG, "jolt_export_debug: buffer too small");
+  if (host_src) memcpy(buf, src, n);
+  else CK(cudaMemcpy(buf, src, n, cudaMemcpyDeviceToHost));
+  *len = n;
+  return JOLT_OK;
+}
+
+JOLT_API uint64_t jolt_launch_count(void) { return g_launches.load(); }
+
+JOLT_API jolt_status jolt_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = on != 0;
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_profile_report(char* buf, uint64_t* len) {
+  g_err.clear();
+  if (!len) return fail(JOLT_ERR_INVALID_ARG, "jolt_profile_report: null len");
+  CK(cudaDeviceSynchronize());
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  struct Agg { std::string name; uint64_t calls = 0, launches = 0; double ms = 0.0; };
+  std::vector<Agg> agg;
+  for (const ProfRec& r : g_prof) {
+    float ms = 0.0f;
+    cudaEventElapsedTime(&ms, r.a, r.b);
+    size_t i = 0;
+    while (i < agg.size() && agg[i].name != r.name) ++i;
+    if (i == agg.size()) { agg.push_back(Agg()); agg.back().name = r.name; }
+    agg[i].calls += 1;
+    agg[i].launches += r.launches;
+    agg[i].ms += ms;
+  }
+  std::string out = "{";
+  for (size_t i = 0; i < agg.size(); ++i) {
+    char tmp[256];
+    snprintf(tmp, sizeof(tmp), "%s\"%s\": {\"calls\": %llu, \"launches\": %llu, \"total_ms\": %.6f}",
+             i ? ", " : "", agg[i].name.c_str(), (unsigned long long)agg[i].calls,
+             (unsigned long long)agg[i].launches, agg[i].ms);
+    out += tmp;
+  }
+  out += "}";
+  if (!buf) { *len = out.size() + 1; return JOLT_OK; }
+  if (*len < out.size() + 1) return fail(JOLT_ERR_INVALID_ARG, "jolt_profile_report: buffer too small");
+  memcpy(buf, out.c_str(), out.size() + 1);
+  *len = out.size() + 1;
+  for (const ProfRec& r : g_prof) { g_pool.push_back(r.a); g_pool.push_back(r.b); }
+  g_prof.clear();
+  return JOLT_OK;
+}
+
+JOLT_API void jolt_stream_destroy(jolt_stream_t st) {
+  if (!st) return;
+  if (st->plan && st->plan->last == st) st->plan->last = nullptr;
+  // stream-ordered release after the work already enqueued on the encode stream
+  if (st->d_body) cudaFreeAsync(st->d_body, st->cs);
+  if (st->d_meta) cudaFreeAsync(st->d_meta, st->cs);
+  if (st->d_Pi) cudaFreeAsync(st->d_Pi, st->cs);
+  if (st->d_Gpi) cudaFreeAsync(st->d_Gpi, st->cs);
+  if (st->d_lt_ids) cudaFreeAsync(st->d_lt_ids, st->cs);
+  delete st;
+}
+
+JOLT_API void jolt_plan_destroy(jolt_plan_t p) {
+  if (!p) return;
+  cudaDeviceSynchronize();
+  if (p->ws) cudaFree(p->ws);
+  if (p->d_lt_ids) cudaFree(p->d_lt_ids);
+  delete p;
+}
+
+}  // extern "C"

@@ -1,0 +1,155 @@
+// Internal declarations shared by the host runtime (jolt_api.cpp) and the kernel files.
+// Nothing here is part of the public C ABI (include/jolt.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/jolt.h"
+
+namespace jolt {
+
+constexpr int kD = 128;            // head_dim supported by this build
+constexpr int kMaxL = 128;         // layers per stream
+constexpr int kMaxLT = 2 * kMaxL;  // layer-tensors per stream
+constexpr int kMaxGroups = 64;
+constexpr int kMaxN = 128;         // largest in-shared-memory eigenproblem / sketch width
+constexpr int kAlign = 256;        // byte alignment of every stream part
+
+// Device status word bits (OR-ed by kernels, read by the host after a sync).
+enum : int32_t { ST_NOT_CONVERGED = 1, ST_NONFINITE = 2, ST_INFEASIBLE = 4, ST_TIMEOUT = 8 };
+
+// Per-stream metadata written on the device by the allocator and read by the
+// residual-coding and decode kernels, so no host round trip sits inside encode.
+struct StreamMeta {
+  int32_t status;
+  int32_t num_lt;
+  int64_t body_bytes;
+  double lambda[2];
+  int32_t alloc[kMaxGroups][2][3];      // (r_t, r_d, b) per group and kind
+  int32_t lt_rank[kMaxLT][3];           // (r_t, r_d, b) per layer-tensor
+  int64_t off[kMaxLT][JOLT_NUM_PARTS];  // byte offset of each part in the body
+  int64_t bytes_by_part[JOLT_NUM_PARTS];
+};
+
+// Counts kernel launches made by this library (read through jolt_launch_count).
+void note_launch();
+
+// ------------------------------------------------------------------ generic SIMT GEMM
+// Index map with an optional second level: i -> (i / in) * s_out + (i % in) * s_in when
+// in > 0, else i * s_in. It expresses the token unfolding X_(2)[t, h*D + d] = X[h][t][d]
+// without copying X.
+struct Idx2 {
+  int64_t s_in = 0, s_out = 0;
+  int32_t in = 0;
+};
+enum ElemType : int32_t { EL_BF16 = 0, EL_F32 = 1, EL_F64 = 2 };
+struct Operand {
+  const void* p = nullptr;
+  ElemType t = EL_F32;
+  Idx2 batch, row, k;  // row = m for the A operand, n for the B operand
+};
+struct OutDesc {
+  void* p = nullptr;
+  ElemType t = EL_F32;  // EL_F32 or EL_F64
+  Idx2 batch, m, n;
+};
+// C[b](m, n) = alpha * sum_k A[b](m, k) * B[b](n, k) + beta * C[b](m, n), fp64 accumulation.
+cudaError_t gemm_simt(int batch, int M, int N, int K, const Operand& A, const Operand& B,
+                      const OutDesc& C, double alpha, double beta, cudaStream_t s);
+
+// ------------------------------------------------------------------ kernels (launchers)
+// Counter-based normals (SplitMix64 + Box-Muller), see rotation.cu.
+cudaError_t gauss_f64(uint64_t seed, uint64_t stream_id, int64_t n, double* out, cudaStream_t s);
+// Sketch matrices Omega_lt = bf16(N(0,1)) of shape [HD][l], lt in [0, n_lt) uses stream 2 + lt_id[lt].
+cudaError_t sketch_omega(uint64_t seed, const int32_t* lt_ids_host, int n_lt, int64_t HD, int l,
+                         __nv_bfloat16* out, cudaStream_t s);
+// Haar rotation from a D x D float64 Gaussian (Householder QR, signs of diag(R) moved into Q).
+cudaError_t haar_from_gauss(const double* G, int D, float* Pi_f32, __nv_bfloat16* Pi_bf16,
+                            cudaStream_t s);
+// Batched two-sided cyclic Jacobi, n even, n <= 128; V columns = eigenvectors, eigenvalues
+// descending. Sets ST_NOT_CONVERGED in *status when max_sweeps is reached.
+cudaError_t jacobi_eig(int batch, int n, const float* A, int64_t sA, float* V, int64_t sV,
+                       float* lam, int64_t sL, int max_sweeps, int32_t* status, cudaStream_t s);
+// Shifted-CholeskyQR helper: Rinv = inverse of chol(W + shift * trace(W)/n * I), W n x n.
+cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv, int64_t sR,
+                     double shift, int32_t* status, cudaStream_t s);
+// Column sign rule: largest |entry| of each column positive (lowest index on ties).
+// Signs are computed on U (rows x cols, row stride ldu) and applied to U and to the
+// optional companion W (w_rows x cols, row stride ldw).
+cudaError_t sign_fix(int batch, int rows, int cols, float* U, int64_t ldu, int64_t sU, float* W,
+                     int w_rows, int64_t ldw, int64_t sW, cudaStream_t s);
+// Round float -> bf16 (RNE) into two copies: bf16 and float-of-bf16.
+cudaError_t round_bf16(int64_t n, const float* in, __nv_bfloat16* out_b, float* out_f, cudaStream_t s);
+// Squared Frobenius norm (float64, fixed reduction order) of each of `batch` arrays of n elements.
+// `scratch` holds batch * 64 doubles.
+cudaError_t sumsq_batched(int batch, int64_t n, const void* x, ElemType t, int64_t stride,
+                          double* out, double* scratch, cudaStream_t s);
+// Sum of squared differences and squared reference (float64), deterministic.
+cudaError_t relfrob_partial(const void* ref, const void* approx, uint64_t n, ElemType t,
+                            double* partials, int nblocks, double* out2, cudaStream_t s);
+int relfrob_blocks(uint64_t n);
+
+struct TableArgs {
+  int n_lt, H, R, D, step;
+  const int32_t* lt_ids;  // device [n_lt]: row of E written for buffer index i
+  const float* Gmax;   // [n_lt][H][R][D]
+  const double* xx;    // [n_lt]
+  double* E;           // [2L][ngrid], row lt = 2*layer + kind
+  int ngrid;           // 1 + (R/step)*(D/step)
+};
+cudaError_t energy_table(const TableArgs& a, cudaStream_t s);
+
+struct DualArgs {
+  int L, H, T, D, G, has_v, step, R, split;
+  int nbits;
+  int32_t bits[9];
+  double phi[9];
+  int64_t budget_pool[2];
+  int ngrid;
+  const double* E;    // [2L][ngrid] (lt = 2*layer + kind)
+  double* unit_err;   // [G*2][nbits*ngrid] debug copy of the tables
+  StreamMeta* meta;
+};
+cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s);
+
+struct PackArgs {
+  int n_lt, H, T, D, R;
+  const int32_t* lt_ids;     // device [n_lt] -> lt index (2*layer + kind)
+  const __nv_bfloat16* UT;   // [n_lt][T][R]
+  const __nv_bfloat16* UD;   // [n_lt][D][D]
+  const float* Gmax;         // [n_lt][H][R][D]
+  const StreamMeta* meta;
+  uint8_t* body;
+};
+cudaError_t pack_factors(const PackArgs& a, cudaStream_t s);
+
+struct ResidualArgs {
+  int n_lt, H, T, D;
+  const int32_t* lt_ids;     // device [n_lt]
+  const void* X[2];          // K, V base pointers [L][H][T][D]
+  ElemType xt;
+  const float* Pi;           // [D][D] float32
+  const StreamMeta* meta;
+  uint8_t* body;
+};
+// Nbuf: float64 scratch [n_lt][H][R][D] for N_h = (G_h U_D^T) Pi.
+cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStream_t s);
+
+struct DecodeArgs {
+  int n_lt, H, T, D;
+  const int32_t* lt_ids;     // device [n_lt]
+  void* out[2];              // K_out, V_out
+  ElemType ot;
+  const float* Pi;           // [D][D] float32
+  const StreamMeta* meta;
+  const uint8_t* body;
+};
+cudaError_t decode(const DecodeArgs& a, cudaStream_t s);
+
+// Check for NaN/Inf in an input tensor (sets ST_NONFINITE).
+cudaError_t check_finite(int64_t n, const void* x, ElemType t, int32_t* status, cudaStream_t s);
+
+}  // namespace jolt

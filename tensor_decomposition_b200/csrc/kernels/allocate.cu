@@ -1,0 +1,291 @@
+// Error table, Lagrangian dual allocator and factor packing of the JoLT codec.
+//
+// "A JoLT for the KV Cache" (arXiv 2607.12550v2, Abstract): "A single Lagrangian dual
+// allocates the Tucker ranks and the residual bit-widths together, per layer group and
+// separately for keys and values, under one byte budget." The pages give no formula, so:
+//  * candidate (r_t, r_d) are (0, 0) and every multiple of the rank step up to (R, D);
+//  * table entry E(r_t, r_d) = max(0, ||X||^2 - sum_{h, i < r_t, j < r_d} G_max[h, i, j]^2),
+//    the exact truncation energy of orthonormal nested factors, summed over a group's layers;
+//  * err(r_t, r_d, b) = E * phi(b), phi(0) = 1, phi(b) = kappa_D / (3 * 4^b) (uniform
+//    quantisation error over a cell of the whitened residual, kappa_D = E[max_i z_i^2]);
+//  * bytes = layers * (2 (T r_t + D r_d + H r_t r_d) + [b > 0] H T (D b / 8 + 2));
+//  * per budget pool, lambda is bisected geometrically on [1e-30, 1e30] * (energy / budget)
+//    until hi / lo <= 1 + 1e-15; each unit takes argmin err + lambda * bytes with ties broken
+//    by fewer bytes, then smaller (b, r_t, r_d); the feasible choice at `hi` is kept.
+// The arithmetic uses explicit round-to-nearest double operations (no fused multiply-add),
+// so the same table gives the same allocation as a plain float64 restatement.
+#include "../jolt_internal.h"
+
+namespace jolt {
+namespace {
+
+// One CTA per layer-tensor; thread (I, J) sums the squared core over block rows
+// [I*step, (I+1)*step) and columns [J*step, (J+1)*step) in a fixed order.
+__global__ void k_energy_table(int H, int R, int D, int step, const float* Gmax, const double* xx,
+                               double* E, int ngrid, const int32_t* lt_ids) {
+  extern __shared__ double sb[];  // [R/step][D/step] block sums, then prefix sums
+  const int lt = blockIdx.x;
+  const int nI = R / step, nJ = D / step;
+  const float* g = Gmax + (int64_t)lt * H * R * D;
+  for (int blk = threadIdx.x; blk < nI * nJ; blk += blockDim.x) {
+    const int I = blk / nJ, J = blk % nJ;
+    double acc = 0.0;
+    for (int h = 0; h < H; ++h)
+      for (int i = I * step; i < (I + 1) * step; ++i)
+        for (int j = J * step; j < (J + 1) * step; ++j) {
+          const double v = (double)g[((int64_t)h * R + i) * D + j];
+          acc += v * v;
+        }
+    sb[blk] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const double x2 = xx[lt];
+    double* e = E + (int64_t)lt_ids[lt] * ngrid;
+    e[0] = x2;
+    // prefix over J within each row block, then over I
+    for (int I = 0; I < nI; ++I)
+      for (int J = 1; J < nJ; ++J) sb[I * nJ + J] += sb[I * nJ + J - 1];
+    for (int I = 1; I < nI; ++I)
+      for (int J = 0; J < nJ; ++J) sb[I * nJ + J] += sb[(I - 1) * nJ + J];
+    for (int I = 0; I < nI; ++I)
+      for (int J = 0; J < nJ; ++J) {
+        const double r = x2 - sb[I * nJ + J];
+        e[1 + I * nJ + J] = r > 0.0 ? r : 0.0;
+      }
+  }
+}
+
+struct Cand {
+  double cost;
+  int64_t bytes;
+  int b, rt, rd, idx;
+};
+
+__device__ __forceinline__ bool less_key(const Cand& a, const Cand& b) {
+  if (a.cost != b.cost) return a.cost < b.cost;
+  if (a.bytes != b.bytes) return a.bytes < b.bytes;
+  if (a.b != b.b) return a.b < b.b;
+  if (a.rt != b.rt) return a.rt < b.rt;
+  return a.rd < b.rd;
+}
+
+__device__ __forceinline__ int64_t lt_bytes(int H, int T, int D, int rt, int rd, int b) {
+  const int64_t tucker = 2 * ((int64_t)T * rt + (int64_t)D * rd + (int64_t)H * rt * rd);
+  const int64_t resid = b > 0 ? (int64_t)H * T * (D * b / 8 + 2) : 0;
+  return tucker + resid;
+}
+
+__device__ __forceinline__ void grid_rank(int gi, int step, int D, int& rt, int& rd) {
+  if (gi == 0) { rt = 0; rd = 0; return; }
+  const int nJ = D / step;
+  rt = ((gi - 1) / nJ + 1) * step;
+  rd = ((gi - 1) % nJ + 1) * step;
+}
+
+constexpr int kMaxUnits = 2 * kMaxGroups;
+
+// Single CTA of 1024 threads: warp w evaluates units w, w + 32, ...
+__global__ void __launch_bounds__(1024) k_dual(DualArgs a) {
+  __shared__ int nlay[kMaxGroups];
+  __shared__ int choice[kMaxUnits];
+  __shared__ int64_t cbytes[kMaxUnits];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nu = a.G * 2;
+  const int ncand = a.nbits * a.ngrid;
+  StreamMeta* meta = a.meta;
+  for (int g = tid; g < a.G; g += blockDim.x)
+    nlay[g] = (int)(((int64_t)(g + 1) * a.L) / a.G - ((int64_t)g * a.L) / a.G);
+  // Unit tables: E summed over the group's layers in increasing layer order, times phi(b).
+  for (int e = tid; e < nu * a.ngrid; e += blockDim.x) {
+    const int u = e / a.ngrid, gi = e % a.ngrid;
+    const int g = u / 2, k = u % 2;
+    if (k == 1 && !a.has_v) continue;
+    const int l0 = (int)(((int64_t)g * a.L) / a.G), l1 = (int)(((int64_t)(g + 1) * a.L) / a.G);
+    double s = 0.0;
+    for (int l = l0; l < l1; ++l) s = __dadd_rn(s, a.E[(int64_t)(2 * l + k) * a.ngrid + gi]);
+    for (int bi = 0; bi < a.nbits; ++bi)
+      a.unit_err[(int64_t)u * ncand + bi * a.ngrid + gi] = __dmul_rn(s, a.phi[bi]);
+  }
+  __syncthreads();
+  const int npools = (a.has_v && a.split) ? 2 : 1;
+  for (int pool = 0; pool < npools; ++pool) {
+    const int64_t budget = a.budget_pool[pool];
+    // unit u belongs to this pool?
+    auto in_pool = [&](int u) -> bool {
+      const int k = u % 2;
+      if (k == 1 && !a.has_v) return false;
+      if (npools == 1) return true;
+      return k == pool;
+    };
+    // choose(lam) for every unit of the pool; writes choice[] and cbytes[]
+    auto choose_all = [&](double lam, bool min_bytes_only) {
+      for (int u = warp; u < nu; u += (int)(blockDim.x >> 5)) {
+        if (!in_pool(u)) continue;
+        const int g = u / 2;
+        Cand best;
+        best.cost = 0.0;
+        best.idx = -1;
+        for (int c = lane; c < ncand; c += 32) {
+          const int bi = c / a.ngrid, gi = c % a.ngrid;
+          Cand x;
+          grid_rank(gi, a.step, a.D, x.rt, x.rd);
+          x.b = a.bits[bi];
+          x.bytes = (int64_t)nlay[g] * lt_bytes(a.H, a.T, a.D, x.rt, x.rd, x.b);
+          x.cost = min_bytes_only ? 0.0
+                                  : __dadd_rn(a.unit_err[(int64_t)u * ncand + c],
+                                              __dmul_rn(lam, (double)x.bytes));
+          x.idx = c;
+          if (best.idx < 0 || less_key(x, best)) best = x;
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          Cand y;
+          y.cost = __shfl_down_sync(0xffffffffu, best.cost, o);
+          y.bytes = __shfl_down_sync(0xffffffffu, best.bytes, o);
+          y.b = __shfl_down_sync(0xffffffffu, best.b, o);
+          y.rt = __shfl_down_sync(0xffffffffu, best.rt, o);
+          y.rd = __shfl_down_sync(0xffffffffu, best.rd, o);
+          y.idx = __shfl_down_sync(0xffffffffu, best.idx, o);
+          if (y.idx >= 0 && (best.idx < 0 || less_key(y, best))) best = y;
+        }
+        if (lane == 0) {
+          choice[u] = best.idx;
+          cbytes[u] = best.bytes;
+        }
+      }
+      __syncthreads();
+      int64_t tb = 0;
+      for (int u = 0; u < nu; ++u)
+        if (in_pool(u)) tb += cbytes[u];
+      __syncthreads();
+      return tb;
+    };
+    const int64_t minb = choose_all(0.0, true);
+    double lam = 0.0;
+    if (minb > budget) {
+      if (tid == 0) atomicOr(&meta->status, ST_INFEASIBLE);
+    } else {
+      int64_t tb = choose_all(0.0, false);
+      if (tb > budget) {
+        // sum of the pool's unit energies E(0, 0), each summed over its layers in order
+        double esum = 0.0;
+        for (int u = 0; u < nu; ++u) {
+          if (!in_pool(u)) continue;
+          const int g = u / 2, k = u % 2;
+          const int l0 = (int)(((int64_t)g * a.L) / a.G), l1 = (int)(((int64_t)(g + 1) * a.L) / a.G);
+          double s = 0.0;
+          for (int l = l0; l < l1; ++l) s = __dadd_rn(s, a.E[(int64_t)(2 * l + k) * a.ngrid]);
+          esum = __dadd_rn(esum, s);
+        }
+        const double scale = __ddiv_rn(esum, (double)budget);
+        double lo = __dmul_rn(1e-30, scale), hi = __dmul_rn(1e30, scale);
+        for (int it = 0; it < 200; ++it) {
+          if (!(__ddiv_rn(hi, lo) > 1.0 + 1e-15)) break;
+          const double mid = __dsqrt_rn(__dmul_rn(lo, hi));
+          const int64_t t = choose_all(mid, false);
+          if (t <= budget) hi = mid;
+          else lo = mid;
+        }
+        lam = hi;
+        choose_all(hi, false);
+      }
+    }
+    if (tid == 0) {
+      meta->lambda[pool] = lam;
+      for (int u = 0; u < nu; ++u) {
+        if (!in_pool(u)) continue;
+        const int c = choice[u];
+        const int bi = c / a.ngrid, gi = c % a.ngrid;
+        int rt, rd;
+        grid_rank(gi, a.step, a.D, rt, rd);
+        meta->alloc[u / 2][u % 2][0] = rt;
+        meta->alloc[u / 2][u % 2][1] = rd;
+        meta->alloc[u / 2][u % 2][2] = a.bits[bi];
+      }
+    }
+    __syncthreads();
+  }
+  // Layout of the body: lt-major, parts U_T, U_D, G, scales, codes, each 256-aligned.
+  if (tid == 0) {
+    int64_t cur = 0;
+    int64_t bp[JOLT_NUM_PARTS] = {0, 0, 0, 0, 0};
+    for (int l = 0; l < a.L; ++l) {
+      int g = 0;
+      while (g + 1 < a.G && ((int64_t)(g + 1) * a.L) / a.G <= l) ++g;
+      for (int k = 0; k < (a.has_v ? 2 : 1); ++k) {
+        const int lt = 2 * l + k;
+        const int rt = meta->alloc[g][k][0], rd = meta->alloc[g][k][1], b = meta->alloc[g][k][2];
+        meta->lt_rank[lt][0] = rt;
+        meta->lt_rank[lt][1] = rd;
+        meta->lt_rank[lt][2] = b;
+        const int64_t sz[JOLT_NUM_PARTS] = {
+            (int64_t)a.T * rt * 2, (int64_t)a.D * rd * 2, (int64_t)a.H * rt * rd * 2,
+            b > 0 ? (int64_t)a.H * a.T * 2 : 0, b > 0 ? (int64_t)a.H * a.T * (a.D * b / 8) : 0};
+        for (int p = 0; p < JOLT_NUM_PARTS; ++p) {
+          const int64_t off = (cur + kAlign - 1) / kAlign * kAlign;
+          meta->off[lt][p] = off;
+          cur = off + sz[p];
+          bp[p] += sz[p];
+        }
+      }
+    }
+    meta->body_bytes = cur;
+    for (int p = 0; p < JOLT_NUM_PARTS; ++p) meta->bytes_by_part[p] = bp[p];
+  }
+}
+
+// Copy the chosen leading blocks of the factors and the bf16-rounded core into the body.
+__global__ void k_pack_factors(PackArgs a) {
+  const int i = blockIdx.y;            // index into lt_ids
+  const int lt = a.lt_ids[i];
+  const StreamMeta* m = a.meta;
+  const int rt = m->lt_rank[lt][0], rd = m->lt_rank[lt][1];
+  __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UT]);
+  __nv_bfloat16* ud = reinterpret_cast<__nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UD]);
+  __nv_bfloat16* gg = reinterpret_cast<__nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_G]);
+  const __nv_bfloat16* UT = a.UT + (int64_t)i * a.T * a.R;
+  const __nv_bfloat16* UD = a.UD + (int64_t)i * a.D * a.D;
+  const float* Gm = a.Gmax + (int64_t)i * a.H * a.R * a.D;
+  const int64_t n_ut = (int64_t)a.T * rt, n_ud = (int64_t)a.D * rd, n_g = (int64_t)a.H * rt * rd;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n_ut + n_ud + n_g; e += stride) {
+    if (e < n_ut) {
+      const int64_t t = e / rt, c = e % rt;
+      ut[e] = UT[t * a.R + c];
+    } else if (e < n_ut + n_ud) {
+      const int64_t f = e - n_ut;
+      const int64_t d = f / rd, c = f % rd;
+      ud[f] = UD[d * a.D + c];
+    } else {
+      const int64_t f = e - n_ut - n_ud;
+      const int64_t h = f / ((int64_t)rt * rd), r = f % ((int64_t)rt * rd);
+      const int64_t ii = r / rd, j = r % rd;
+      gg[f] = __float2bfloat16_rn(Gm[(h * a.R + ii) * a.D + j]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t energy_table(const TableArgs& a, cudaStream_t s) {
+  const size_t smem = (size_t)(a.R / a.step) * (a.D / a.step) * sizeof(double) + sizeof(double);
+  k_energy_table<<<a.n_lt, 128, smem, s>>>(a.H, a.R, a.D, a.step, a.Gmax, a.xx, a.E, a.ngrid,
+                                           a.lt_ids);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s) {
+  if (a.G > kMaxGroups || a.L > kMaxL) return cudaErrorInvalidValue;
+  k_dual<<<1, 1024, 0, s>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t pack_factors(const PackArgs& a, cudaStream_t s) {
+  k_pack_factors<<<dim3(64, a.n_lt), 256, 0, s>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace jolt

@@ -1,0 +1,220 @@
+// Small helper kernels: storage rounding, float64 norms (the relative Frobenius error the
+// JoLT abstract reports, arXiv 2607.12550v2), the factor column sign rule and the
+// non-finite input check. Reductions use a fixed grid and a fixed tree so results are
+// bit-reproducible from run to run.
+#include "../jolt_internal.h"
+
+namespace jolt {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ double ld_as_double(const T* p, int64_t i);
+template <>
+__device__ __forceinline__ double ld_as_double<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
+  return (double)__bfloat162float(p[i]);
+}
+template <>
+__device__ __forceinline__ double ld_as_double<float>(const float* p, int64_t i) {
+  return (double)p[i];
+}
+
+__device__ __forceinline__ double block_sum(double v, double* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  double t = 0.0;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+  __syncthreads();
+  return t;
+}
+
+__global__ void k_round_bf16(int64_t n, const float* in, __nv_bfloat16* ob, float* of) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(in[i]);
+    if (ob) ob[i] = b;
+    if (of) of[i] = __bfloat162float(b);
+  }
+}
+
+constexpr int kSumBlocks = 64;
+
+template <typename T>
+__global__ void k_sumsq_part(int64_t n, const T* x, int64_t stride, double* part) {
+  __shared__ double red[32];
+  const T* p = x + (int64_t)blockIdx.y * stride;
+  double acc = 0.0;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const double v = ld_as_double(p, i);
+    acc += v * v;
+  }
+  const double t = block_sum(acc, red);
+  if (threadIdx.x == 0) part[blockIdx.y * gridDim.x + blockIdx.x] = t;
+}
+
+__global__ void k_sum_rows(int rows, int cols, const double* part, double* out) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  double t = 0.0;
+  for (int c = 0; c < cols; ++c) t += part[(int64_t)r * cols + c];
+  out[r] = t;
+}
+
+template <typename T>
+__global__ void k_relfrob_part(uint64_t n, const T* a, const T* b, double* part) {
+  __shared__ double red[32];
+  double sd = 0.0, sr = 0.0;
+  for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n;
+       i += (uint64_t)gridDim.x * blockDim.x) {
+    const double x = ld_as_double(a, (int64_t)i), y = ld_as_double(b, (int64_t)i);
+    sd += (x - y) * (x - y);
+    sr += x * x;
+  }
+  const double td = block_sum(sd, red);
+  const double tr = block_sum(sr, red);
+  if (threadIdx.x == 0) {
+    part[2 * blockIdx.x] = td;
+    part[2 * blockIdx.x + 1] = tr;
+  }
+}
+
+__global__ void k_relfrob_final(int nb, const double* part, double* out2) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    double d = 0.0, r = 0.0;
+    for (int i = 0; i < nb; ++i) {
+      d += part[2 * i];
+      r += part[2 * i + 1];
+    }
+    out2[0] = d;
+    out2[1] = r;
+  }
+}
+
+// Sign rule per column: the entry of largest magnitude (first on ties) becomes positive.
+// Block = 32 columns x 8 row lanes; the same block then flips U's and W's columns.
+__global__ void k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU, float* W,
+                           int w_rows, int64_t ldw, int64_t sW) {
+  __shared__ float bv[8][32];
+  __shared__ int bi[8][32];
+  __shared__ float sgn[32];
+  const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + cx;
+  float* u = U + (int64_t)blockIdx.y * sU;
+  float best = -1.0f;
+  int bidx = 0x7fffffff;
+  if (c < cols) {
+    for (int r = ry; r < rows; r += 8) {
+      const float a = fabsf(u[(int64_t)r * ldu + c]);
+      if (a > best) { best = a; bidx = r; }   // rows visited in increasing order: first wins ties
+    }
+  }
+  bv[ry][cx] = best;
+  bi[ry][cx] = bidx;
+  __syncthreads();
+  if (ry == 0) {
+    for (int k = 1; k < 8; ++k) {
+      const float v = bv[k][cx];
+      const int i = bi[k][cx];
+      if (v > best || (v == best && i < bidx)) { best = v; bidx = i; }
+    }
+    float sg = 1.0f;
+    if (c < cols && bidx < rows && u[(int64_t)bidx * ldu + c] < 0.0f) sg = -1.0f;
+    sgn[cx] = sg;
+  }
+  __syncthreads();
+  if (c >= cols) return;
+  const float sg = sgn[cx];
+  if (sg > 0.0f) return;
+  for (int r = ry; r < rows; r += 8) u[(int64_t)r * ldu + c] = -u[(int64_t)r * ldu + c];
+  if (W) {
+    float* w = W + (int64_t)blockIdx.y * sW;
+    for (int r = ry; r < w_rows; r += 8) w[(int64_t)r * ldw + c] = -w[(int64_t)r * ldw + c];
+  }
+}
+
+__global__ void k_check_finite_bf16(int64_t n, const __nv_bfloat16* x, int32_t* status) {
+  bool bad = false;
+  const uint16_t* u = reinterpret_cast<const uint16_t*>(x);
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    bad |= ((u[i] & 0x7F80u) == 0x7F80u);
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, ST_NONFINITE);
+}
+
+__global__ void k_check_finite_f32(int64_t n, const float* x, int32_t* status) {
+  bool bad = false;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    bad |= !isfinite(x[i]);
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, ST_NONFINITE);
+}
+
+}  // namespace
+
+cudaError_t round_bf16(int64_t n, const float* in, __nv_bfloat16* ob, float* of, cudaStream_t s) {
+  int b = (int)((n + 255) / 256);
+  if (b > 1184) b = 1184;
+  if (b < 1) b = 1;
+  k_round_bf16<<<b, 256, 0, s>>>(n, in, ob, of);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t sumsq_batched(int batch, int64_t n, const void* x, ElemType t, int64_t stride,
+                          double* out, double* part, cudaStream_t s) {
+  dim3 g(kSumBlocks, batch);
+  if (t == EL_BF16)
+    k_sumsq_part<__nv_bfloat16><<<g, 256, 0, s>>>(n, (const __nv_bfloat16*)x, stride, part);
+  else
+    k_sumsq_part<float><<<g, 256, 0, s>>>(n, (const float*)x, stride, part);
+  note_launch();
+  k_sum_rows<<<(batch + 127) / 128, 128, 0, s>>>(batch, kSumBlocks, part, out);
+  note_launch();
+  return cudaGetLastError();
+}
+
+int relfrob_blocks(uint64_t n) {
+  uint64_t b = (n + 1023) / 1024;
+  if (b > 592) b = 592;
+  if (b < 1) b = 1;
+  return (int)b;
+}
+
+cudaError_t relfrob_partial(const void* ref, const void* approx, uint64_t n, ElemType t,
+                            double* partials, int nblocks, double* out2, cudaStream_t s) {
+  if (t == EL_BF16)
+    k_relfrob_part<__nv_bfloat16><<<nblocks, 256, 0, s>>>(n, (const __nv_bfloat16*)ref,
+                                                          (const __nv_bfloat16*)approx, partials);
+  else
+    k_relfrob_part<float><<<nblocks, 256, 0, s>>>(n, (const float*)ref, (const float*)approx,
+                                                  partials);
+  note_launch();
+  k_relfrob_final<<<1, 32, 0, s>>>(nblocks, partials, out2);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t sign_fix(int batch, int rows, int cols, float* U, int64_t ldu, int64_t sU, float* W,
+                     int w_rows, int64_t ldw, int64_t sW, cudaStream_t s) {
+  dim3 g((cols + 31) / 32, batch);
+  k_sign_fix<<<g, 256, 0, s>>>(rows, cols, U, ldu, sU, W, w_rows, ldw, sW);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t check_finite(int64_t n, const void* x, ElemType t, int32_t* status, cudaStream_t s) {
+  int b = (int)((n + 255) / 256);
+  if (b > 2368) b = 2368;
+  if (b < 1) b = 1;
+  if (t == EL_BF16)
+    k_check_finite_bf16<<<b, 256, 0, s>>>(n, (const __nv_bfloat16*)x, status);
+  else
+    k_check_finite_f32<<<b, 256, 0, s>>>(n, (const float*)x, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace jolt

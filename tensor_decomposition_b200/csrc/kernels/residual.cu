@@ -1,0 +1,212 @@
+// Fused residual coding of the JoLT codec: reconstruct, subtract, rotate, row absmax,
+// b-bit quantisation and bit packing, in one pass over X.
+//
+// "A JoLT for the KV Cache" (arXiv 2607.12550v2, Abstract) restores the energy the
+// truncation discards "with a rotated low-bit residual: a random orthogonal rotation
+// followed by low-bit quantization". For a row x = X[h, t, :] (D features), with the stored
+// (bf16) factors and core, the rotated residual is
+//     y = (x - u_t G_h U_D^T) Pi = x Pi - u_t N_h,   N_h = (G_h U_D^T) Pi   (r_t x D),
+// u_t = U_T[t, :r_t]. Quantiser (a reading; the pages fix none): s = fp16(max_i |y_i|)
+// (round to nearest even, saturating at 65504), c_i = clamp(floor(y_i 2^(b-1) / s + 2^(b-1)),
+// 0, 2^b - 1), codes packed LSB first, code i at bits [i b, i b + b) of the row.
+//
+// Arithmetic is float64 end to end (the inputs are bf16 / fp32 values, so products are
+// exact), which keeps every code equal to the one a float64 restatement computes from the
+// same stored factors, except for values within ~1e-13 s of a cell boundary.
+#include "../jolt_internal.h"
+
+namespace jolt {
+namespace {
+
+constexpr int kRowsPerWarp = 4;
+constexpr int kWarps = 8;
+constexpr int kChunk = 256;          // tokens per CTA
+
+__device__ __forceinline__ const void* x_row_ptr(const ResidualArgs& a, int lt, int h, int t) {
+  const int layer = lt >> 1, kind = lt & 1;
+  const int64_t off = (((int64_t)layer * a.H + h) * a.T + t) * a.D;
+  return a.xt == EL_BF16
+             ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.X[kind]) + off)
+             : (const void*)(reinterpret_cast<const float*>(a.X[kind]) + off);
+}
+
+// N_h = (G_h U_D^T) Pi in float64 for one (layer-tensor, head); 16 rows of M at a time.
+__global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf, int R) {
+  extern __shared__ unsigned char smraw[];
+  const int h = blockIdx.x, i = blockIdx.y;
+  const int lt = a.lt_ids[i];
+  const StreamMeta* m = a.meta;
+  const int rt = m->lt_rank[lt][0], rd = m->lt_rank[lt][1], b = m->lt_rank[lt][2];
+  if (b == 0 || rt == 0) return;
+  const int D = a.D;
+  float* Pi_s = reinterpret_cast<float*>(smraw);                       // D x D
+  float* G_s = Pi_s + D * D;                                           // rt x rd
+  float* UDt = G_s + kMaxN * kMaxN;                                    // rd x D (transposed)
+  double* M_s = reinterpret_cast<double*>(UDt + kMaxN * kMaxN);        // 16 x D
+  const __nv_bfloat16* G = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_G]) +
+                           (int64_t)h * rt * rd;
+  const __nv_bfloat16* UD = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UD]);
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) Pi_s[e] = a.Pi[e];
+  for (int e = threadIdx.x; e < rt * rd; e += blockDim.x) G_s[e] = __bfloat162float(G[e]);
+  for (int e = threadIdx.x; e < D * rd; e += blockDim.x) {
+    const int d = e / rd, j = e % rd;
+    UDt[j * D + d] = __bfloat162float(UD[e]);
+  }
+  __syncthreads();
+  double* N = Nbuf + (((int64_t)i * a.H + h) * R) * D;
+  for (int k0 = 0; k0 < rt; k0 += 16) {
+    for (int e = threadIdx.x; e < 16 * D; e += blockDim.x) {
+      const int kk = e / D, d = e % D;
+      double acc = 0.0;
+      if (k0 + kk < rt)
+        for (int j = 0; j < rd; ++j) acc = fma((double)G_s[(k0 + kk) * rd + j], (double)UDt[j * D + d], acc);
+      M_s[kk * D + d] = acc;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < 16 * D; e += blockDim.x) {
+      const int kk = e / D, j = e % D;
+      if (k0 + kk >= rt) continue;
+      double acc = 0.0;
+      for (int ii = 0; ii < D; ++ii) acc = fma(M_s[kk * D + ii], (double)Pi_s[ii * D + j], acc);
+      N[(int64_t)(k0 + kk) * D + j] = acc;
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* Nbuf, int R) {
+  extern __shared__ unsigned char smraw[];
+  const int chunk = blockIdx.x, h = blockIdx.y, i = blockIdx.z;
+  const int lt = a.lt_ids[i];
+  const StreamMeta* m = a.meta;
+  const int rt = m->lt_rank[lt][0], b = m->lt_rank[lt][2];
+  if (b == 0) return;
+  const int D = a.D;   // 128
+  double* N_s = reinterpret_cast<double*>(smraw);                      // rt x D
+  float* Pi_s = reinterpret_cast<float*>(N_s + (int64_t)rt * D);       // D x D
+  float* stage = Pi_s + D * D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* xs = stage + warp * (kRowsPerWarp * (2 * kMaxN));             // [4][128] x, then [4][128] u
+  float* us = xs + kRowsPerWarp * kMaxN;
+  unsigned char* cs = reinterpret_cast<unsigned char*>(stage + kWarps * kRowsPerWarp * 2 * kMaxN) +
+                      warp * kRowsPerWarp * kMaxN;
+  const double* Ng = Nbuf + (((int64_t)i * a.H + h) * R) * D;
+  for (int e = threadIdx.x; e < rt * D; e += blockDim.x) N_s[e] = Ng[e];
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) Pi_s[e] = a.Pi[e];
+  __syncthreads();
+  const __nv_bfloat16* UT = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UT]);
+  __half* scales = reinterpret_cast<__half*>(a.body + m->off[lt][JOLT_PART_SCALES]);
+  unsigned char* codes = a.body + m->off[lt][JOLT_PART_CODES];
+  const int rowbytes = D * b / 8;
+  const double half = (double)(1 << (b - 1));
+  const int cmax = (1 << b) - 1;
+  const int t_begin = chunk * kChunk;
+  const int t_end = min(a.T, t_begin + kChunk);
+  for (int t0 = t_begin + warp * kRowsPerWarp; t0 < t_end; t0 += kWarps * kRowsPerWarp) {
+    // stage x rows and u rows
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+      const int t = t0 + r;
+      for (int q = 0; q < 4; ++q) {
+        const int d = lane + 32 * q;
+        float xv = 0.0f, uv = 0.0f;
+        if (t < t_end) {
+          const void* xp = x_row_ptr(a, lt, h, t);
+          xv = a.xt == EL_BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xp)[d])
+                               : reinterpret_cast<const float*>(xp)[d];
+          if (d < rt) uv = __bfloat162float(UT[(int64_t)t * rt + d]);
+        }
+        xs[r * kMaxN + d] = xv;
+        us[r * kMaxN + d] = uv;
+      }
+    }
+    __syncwarp();
+    double acc[kRowsPerWarp][4];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[r][q] = 0.0;
+    for (int ii = 0; ii < D; ++ii) {
+      double p[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) p[q] = (double)Pi_s[ii * D + lane + 32 * q];
+#pragma unroll
+      for (int r = 0; r < kRowsPerWarp; ++r) {
+        const double xv = (double)xs[r * kMaxN + ii];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[r][q] = fma(xv, p[q], acc[r][q]);
+      }
+    }
+    for (int k = 0; k < rt; ++k) {
+      double nv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) nv[q] = N_s[k * D + lane + 32 * q];
+#pragma unroll
+      for (int r = 0; r < kRowsPerWarp; ++r) {
+        const double uv = -(double)us[r * kMaxN + k];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[r][q] = fma(uv, nv[q], acc[r][q]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+      const int t = t0 + r;
+      double mx = 0.0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mx = fmax(mx, fabs(acc[r][q]));
+      for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const __half sh = mx >= 65504.0 ? __float2half_rn(65504.0f) : __double2half(mx);
+      const double sd = (double)__half2float(sh);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        int c = 0;
+        if (sd > 0.0) {
+          const double u = __dadd_rn(__ddiv_rn(acc[r][q] * half, sd), half);
+          const double f = floor(u);
+          c = f < 0.0 ? 0 : (f > (double)cmax ? cmax : (int)f);
+        }
+        cs[r * kMaxN + lane + 32 * q] = (unsigned char)c;
+      }
+      __syncwarp();
+      if (t < t_end) {
+        const int64_t row = (int64_t)h * a.T + t;
+        for (int k = lane; k < rowbytes; k += 32) {
+          unsigned int byte = 0;
+#pragma unroll
+          for (int bit = 0; bit < 8; ++bit) {
+            const int pos = 8 * k + bit;
+            byte |= ((unsigned int)(cs[r * kMaxN + pos / b] >> (pos % b)) & 1u) << bit;
+          }
+          codes[row * rowbytes + k] = (unsigned char)byte;
+        }
+        if (lane == 0) scales[row] = sh;
+      }
+      __syncwarp();
+    }
+  }
+}
+
+}  // namespace
+
+static size_t residual_prep_smem() {
+  return ((size_t)kD * kD + 2 * (size_t)kMaxN * kMaxN) * sizeof(float) + 16 * (size_t)kD * sizeof(double);
+}
+
+cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStream_t s) {
+  if (a.D != kD) return cudaErrorInvalidValue;
+  const size_t sp = residual_prep_smem();
+  cudaError_t e = cudaFuncSetAttribute(k_resid_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp);
+  if (e != cudaSuccess) return e;
+  k_resid_prep<<<dim3(a.H, a.n_lt), 256, sp, s>>>(a, Nbuf, R);
+  note_launch();
+  const size_t sm = (size_t)R * kD * sizeof(double) + (size_t)kD * kD * sizeof(float) +
+                    (size_t)kWarps * kRowsPerWarp * 2 * kMaxN * sizeof(float) +
+                    (size_t)kWarps * kRowsPerWarp * kMaxN;
+  e = cudaFuncSetAttribute(k_residual, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const dim3 g((a.T + kChunk - 1) / kChunk, a.H, a.n_lt);
+  k_residual<<<g, kWarps * 32, sm, s>>>(a, Nbuf, R);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace jolt

@@ -1,0 +1,120 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI, then
+compare with the CPU oracle on the same seeded inputs."""
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+from oracle import jolt as oj
+from oracle import numerics as onum
+from oracle import stream as ostream
+
+ANGLE_TOL = 1e-3           # rad, leading subspace of the exact HOSVD factors
+GAP_REL = 1e-3             # eigengap (relative to the top eigenvalue) that makes a column "leading"
+REL_ERR_TOL = 0.01         # GPU relative Frobenius error within 1% (relative) of the oracle's
+BOUNDARY_BAND = 1e-6       # codes may differ only within this distance (units of the row scale)
+
+
+def to_torch(a: np.ndarray, dtype: str):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    t = t.to(torch.bfloat16) if dtype == "bf16" else t
+    return t.cuda()
+
+
+def decode_tol(ref: np.ndarray, out_f32: bool) -> np.ndarray:
+    """max(1e-3, one output ulp at the oracle's value): bf16 output rounding alone reaches
+    half an ulp, which exceeds 1e-3 once |x| >= 0.5."""
+    if out_f32:
+        return np.full(ref.shape, 1e-3)
+    a = np.abs(ref)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    ulp = np.ldexp(1.0, (e - 7).astype(np.int64))
+    return np.maximum(1e-3, ulp)
+
+
+def oracle_plan(cfg, budget, encoder, groups=None, split=None, bits=None, **kw):
+    return oj.Plan(L=cfg.layers, H=cfg.heads, T=cfg.tokens, D=cfg.head_dim, has_v=cfg.has_v,
+                   budget=budget, num_groups=groups or cfg.groups, encoder=encoder,
+                   split_kv=cfg.split_kv if split is None else split,
+                   bits=tuple(bits or cfg.bits), out_f32=(cfg.dtype == "f32"), **kw)
+
+
+def gpu_encode(cfg, K, V, budget, encoder, seed=42, groups=None, split=None, bits=None):
+    """Encode on the GPU through the C ABI. Returns (plan, stream, K_dev, V_dev)."""
+    from tensor_decomposition_b200 import jolt as J
+    c = J.jolt_config_default()
+    c.encoder = J.JOLT_ENC_EXACT if encoder == "exact" else J.JOLT_ENC_SKETCH
+    c.split_kv_budget = int(cfg.split_kv if split is None else split)
+    mask = 0
+    for b in (bits or cfg.bits):
+        mask |= 1 << b
+    c.bits_mask = mask
+    dt = J.JOLT_BF16 if cfg.dtype == "bf16" else J.JOLT_F32
+    plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, dt, budget,
+                       groups or cfg.groups, c)
+    Kd = to_torch(K, cfg.dtype)
+    Vd = to_torch(V, cfg.dtype) if cfg.has_v else None
+    st = J.jolt_encode(plan, Kd, Vd, seed)
+    J.jolt_stream_status(st)
+    return plan, st, Kd, Vd
+
+
+def gpu_decode(cfg, st, Kd, Vd):
+    import torch
+    from tensor_decomposition_b200 import jolt as J
+    Ko = torch.empty_like(Kd)
+    Vo = torch.empty_like(Vd) if Vd is not None else None
+    J.jolt_decode(st, Ko, Vo)
+    torch.cuda.synchronize()
+    return Ko, Vo
+
+
+def host(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def leading_count(w, kmax):
+    """Number of leading eigenvectors whose next relative eigengap is at least GAP_REL."""
+    w = np.asarray(w, dtype=np.float64)
+    k = 0
+    for i in range(min(kmax, len(w) - 1)):
+        if (w[i] - w[i + 1]) / w[0] < GAP_REL:
+            break
+        k = i + 1
+    return k
+
+
+def codes_parity(ost, Xs: dict, Pi_gpu: np.ndarray):
+    """Re-code the GPU's stored factors with the oracle; return (mismatches outside the band,
+    mismatches inside it, scale mismatches, compared codes)."""
+    out_band = in_band = scale_bad = total = 0
+    for lt, c in ost.lts.items():
+        if c.b == 0:
+            continue
+        X = Xs[lt]
+        Y = oj.residual_rotated(X, c.U_T, c.G, c.U_D, Pi_gpu)
+        s, codes, dist = oj.quantize_rows(Y, c.b)
+        same_scale = s == c.scales
+        scale_bad += int((~same_scale).sum())
+        diff = (codes != c.codes) & same_scale[..., None]
+        out_band += int((diff & (dist > BOUNDARY_BAND)).sum())
+        in_band += int((diff & (dist <= BOUNDARY_BAND)).sum())
+        total += codes.size
+    return out_band, in_band, scale_bad, total
+
+
+def oracle_lt_reconstruction(plan, X, seed, lt, rt, rd, b, Pi=None):
+    """Oracle float64 reconstruction of one layer-tensor at forced (r_t, r_d, b), with the
+    oracle's own factors (spec mode) and the same sketch stream as layer-tensor `lt`."""
+    a = oj.analyse_layer_tensor(plan, X, seed, lt, spec=True)
+    if Pi is None:
+        Pi = onum.haar_rotation(seed, plan.D)
+    U_T, U_D = a["U_T"][:, :rt], a["U_D"][:, :rd]
+    G = onum.round_bf16(a["Gmax"][:, :rt, :rd])
+    rec = oj.tucker_part(U_T, G, U_D, plan.H, plan.T, plan.D)
+    if b > 0:
+        Y = oj.residual_rotated(X, U_T, G, U_D, Pi)
+        s, c, _ = oj.quantize_rows(Y, b)
+        rec = rec + np.einsum("hte,de->htd", oj.dequantize_rows(s, c, b), Pi)
+    return oj.round_output(rec, plan.out_f32), a

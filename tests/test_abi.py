@@ -1,0 +1,101 @@
+"""C-ABI library checks that need no GPU: it builds, loads, exports every declared symbol,
+and rejects bad requests before touching the device."""
+import ctypes
+import os
+import re
+import struct
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def jolt():
+    from tensor_decomposition_b200 import build as b
+    b.build()
+    from tensor_decomposition_b200 import jolt as j
+    return j
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "jolt.h")).read()
+    return re.findall(r"JOLT_API\s+[\w\s\*]+?\b(jolt_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_symbols())
+    for n in ("jolt_plan", "jolt_encode", "jolt_decode", "jolt_rel_frob_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(jolt):
+    lib = ctypes.CDLL(jolt.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(declared_symbols()) == set(jolt.EXPORTED)
+
+
+def test_config_defaults(jolt):
+    c = jolt.jolt_config_default()
+    assert (c.encoder, c.oversample, c.power_iters, c.rank_step, c.rt_max, c.bits_mask,
+            c.split_kv_budget, c.max_jacobi_sweeps) == (0, 16, 1, 16, 0, 0x1FF, 0, 30)
+
+
+@pytest.mark.parametrize("args", [
+    dict(layers=0, heads=8, tokens=64, head_dim=128),
+    dict(layers=2, heads=8, tokens=64, head_dim=64),
+    dict(layers=2, heads=8, tokens=64, head_dim=128, groups=3),
+    dict(layers=200, heads=8, tokens=64, head_dim=128),
+])
+def test_plan_rejects_bad_shapes(jolt, args):
+    groups = args.pop("groups", 1)
+    with pytest.raises(jolt.JoltError) as e:
+        jolt.jolt_plan(args["layers"], args["heads"], args["tokens"], args["head_dim"], True,
+                       jolt.JOLT_BF16, 10 ** 6, groups)
+    assert e.value.status == 1
+
+
+def test_plan_rejects_infeasible_budget(jolt):
+    c = jolt.jolt_config_default()
+    c.bits_mask = 0b11110            # b in 1..4 only: the residual alone needs H T (D/8 + 2) bytes
+    with pytest.raises(jolt.JoltError) as e:
+        jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 1000, 1, c)
+    assert e.value.status == 2
+
+
+def test_plan_rejects_bad_options(jolt):
+    c = jolt.jolt_config_default()
+    c.bits_mask = 0
+    with pytest.raises(jolt.JoltError):
+        jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 10 ** 6, 1, c)
+    c = jolt.jolt_config_default()
+    c.rank_step = 48
+    with pytest.raises(jolt.JoltError):
+        jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 10 ** 6, 1, c)
+
+
+def test_stream_from_host_rejects_corrupt_buffers(jolt):
+    with pytest.raises(jolt.JoltError) as e:
+        jolt.jolt_stream_from_host(b"NOPE" + bytes(100), cuda_stream=0)
+    assert e.value.status == 8
+    # well-formed header, wrong CRC
+    import zlib
+    hb = 64 + 24
+    hb = (hb + 15) // 16 * 16
+    head = bytearray(hb)
+    struct.pack_into("<4sIII", head, 0, b"JOLT", 1, hb, 0)
+    struct.pack_into("<8i", head, 16, 1, 8, 64, 128, 1, 16, 0, 0)
+    struct.pack_into("<QQ", head, 48, 42, 0)
+    data = bytes(head)
+    good = data + struct.pack("<I", zlib.crc32(data))
+    bad = data + struct.pack("<I", zlib.crc32(data) ^ 1)
+    with pytest.raises(jolt.JoltError) as e:
+        jolt.jolt_stream_from_host(bad, cuda_stream=0)
+    assert e.value.status == 8
+    # version mismatch
+    v2 = bytearray(good)
+    struct.pack_into("<I", v2, 4, 2)
+    with pytest.raises(jolt.JoltError) as e:
+        jolt.jolt_stream_from_host(bytes(v2), cuda_stream=0)
+    assert e.value.status == 8
