@@ -196,6 +196,8 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks):
     clock = peaks["sm_max_mhz"] * 1e6
     fp64_peak = 148 * 64 * 2 * clock / 1e12       # TFLOP/s, 64 FP64 FMA / clk / SM
     fp32_peak = 148 * 128 * 2 * clock / 1e12      # TFLOP/s, 128 FP32 FMA / clk / SM
+    passes = getattr(phase_models, "cholqr_passes", (3, 3, 3))
+    cholqr_flops = n_lt * 4.0 * l * l * (passes[0] * T + passes[1] * H * D + passes[2] * T)
     resid_flops = sum(2.0 * N * (D + rt) for rt, rd, b in ranks if b > 0)
     dec_flops = sum(2.0 * N * (rt + (D if b else 0)) for rt, rd, b in ranks)
     return {
@@ -208,8 +210,12 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks):
         "decode": dict(bound="alu", work=dec_flops / 1e12, unit="TFLOP/s", peak=fp32_peak,
                        note="float32 u M + y Pi^T per entry: 2 (r_t + D) flops; FP32 peak 148 x 128 FMA x 2 x max clock",
                        hbm_bytes=2.0 * N * n_lt + stream_bytes),
-        "jacobi_feature": dict(bound="alu", work=None, unit="TFLOP/s", peak=fp32_peak, note="shared-memory Jacobi"),
-        "jacobi_sketch": dict(bound="alu", work=None, unit="TFLOP/s", peak=fp32_peak, note="shared-memory Jacobi"),
+        "jacobi_feature": dict(bound="alu", work=9.0 * D ** 3 * n_lt / 1e12, unit="TFLOP/s", peak=fp32_peak,
+                               note="symmetric eigenproblem with vectors, 9 n^3 flops (Golub & Van Loan count), n = D"),
+        "jacobi_sketch": dict(bound="alu", work=9.0 * l ** 3 * n_lt / 1e12, unit="TFLOP/s", peak=fp32_peak,
+                              note="symmetric eigenproblem with vectors, 9 n^3 flops, n = l"),
+        "cholqr": dict(bound="tensor", work=cholqr_flops / 1e12, unit="TFLOP/s", peak=peaks["bf16_tflops"] * 0.5,
+                       note="per pass 4 rows l^2 flops (Gram + triangular update) on float32 data: tf32 peak = bf16 x 1/2"),
     }, stream_bytes
 
 
