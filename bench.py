@@ -196,8 +196,8 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks):
     clock = peaks["sm_max_mhz"] * 1e6
     fp64_peak = 148 * 64 * 2 * clock / 1e12       # TFLOP/s, 64 FP64 FMA / clk / SM
     fp32_peak = 148 * 128 * 2 * clock / 1e12      # TFLOP/s, 128 FP32 FMA / clk / SM
-    passes = getattr(phase_models, "cholqr_passes", (3, 3, 3))
-    cholqr_flops = n_lt * 4.0 * l * l * (passes[0] * T + passes[1] * H * D + passes[2] * T)
+    # CholeskyQR passes: 1 for Omega's and the transposed sketch's bases, 2 for the final one
+    cholqr_flops = n_lt * 4.0 * l * l * (1 * T + 1 * H * D + 2 * T)
     resid_flops = sum(2.0 * N * (D + rt) for rt, rd, b in ranks if b > 0)
     dec_flops = sum(2.0 * N * (rt + (D if b else 0)) for rt, rd, b in ranks)
     return {

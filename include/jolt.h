@@ -192,6 +192,14 @@ JOLT_API jolt_status jolt_profile_enable(int32_t on);
 JOLT_API jolt_status jolt_profile_report(char* buf, uint64_t* len);
 JOLT_API uint64_t jolt_launch_count(void);
 
+/* jolt_selftest_gemm_bf16 - C = A B^T on the tensor cores (tcgen05.mma with TMA tile loads),
+ * the building block of the factor analysis, exposed so its numerics can be tested alone.
+ * A: device bf16 [M][K], B: device bf16 [N][K] (row-major, K contiguous, K a multiple of 8),
+ * C: device float32 [M][N]. Products are exact, sums are float32. Synchronises `cuda_stream`;
+ * returns JOLT_ERR_TIMEOUT if a bounded wait inside the kernel gave up. */
+JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const void* B,
+                                             float* C, void* cuda_stream);
+
 /* Release a stream. Its device memory is freed in order on the CUDA stream the stream was
  * created on (encode or jolt_stream_from_host); synchronise any other CUDA stream that still
  * reads it (e.g. a decode issued elsewhere) before destroying it. */

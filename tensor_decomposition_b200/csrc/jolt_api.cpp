@@ -20,6 +20,7 @@
 #include <vector>
 
 #include "jolt_internal.h"
+#include "kernels/gemm_tc.h"
 
 using namespace jolt;
 
@@ -178,6 +179,12 @@ struct jolt_plan_s {
         *Wv = nullptr, *lamB = nullptr, *UT32 = nullptr, *UTf = nullptr, *P = nullptr, *Gmax = nullptr,
         *CT = nullptr, *VT = nullptr, *lamT = nullptr;
   double *Wg = nullptr, *Rinv = nullptr, *E = nullptr, *unit_err = nullptr, *Nbuf = nullptr;
+  float* Qfinal = nullptr;   // final sketch basis (one of Y / Y2)
+  bool q_t = false;          // Qfinal stored as Q^T [l][T] (tensor-core path) instead of Q [T][l]
+  bool use_tc = false;       // bf16 inputs with T % 8 == 0: contractions over X on tcgen05
+  __nv_bfloat16* XT = nullptr;       // [n][H][D][T]
+  float* Cpart = nullptr;            // [n][H][D][D] per-head Gram partials
+  __nv_bfloat16* QTp[3] = {nullptr, nullptr, nullptr};   // bf16 parts of a float32 basis
   double* Gpi = nullptr;
   float* Pi32 = nullptr;
   __nv_bfloat16* Pib = nullptr;
@@ -236,32 +243,79 @@ Idx2 I2(int32_t in, int64_t s_in, int64_t s_out) {
   return x;
 }
 
-// Shifted CholeskyQR3 of n_lt tall matrices Y (rows x l, row-major, batch stride rows*l):
+// Shifted CholeskyQR of n_lt tall matrices Y (rows x l, row-major, batch stride rows*l):
 // pass 1 with shift s = 11 (rows l + l (l + 1)) 2^-53 ||Y||^2 (Fukaya, Kannan, Nakatsukasa,
-// Yamamoto & Yanagisawa 2020), passes 2 and 3 unshifted. Result in Qout; Y is clobbered.
-jolt_status cholqr3(jolt_plan_s* p, int rows, float* Yin, float* Qout, int32_t* status,
-                    cudaStream_t s) {
+// Yamamoto & Yanagisawa 2020), later passes unshifted. Intermediate bases of the power
+// iteration only need their column space, so they take one pass; the final basis takes two.
+// The passes ping-pong between bufA (holding Y) and bufB; the result pointer is returned.
+float* cholqr(jolt_plan_s* p, int rows, float* bufA, float* bufB, int passes, int32_t* status,
+              cudaStream_t s, jolt_status* st) {
   const int l = p->l, n = p->n_lt;
-  float* src = Yin;
-  float* dst = Qout;
-  for (int pass = 0; pass < 3; ++pass) {
+  float* src = bufA;
+  float* dst = bufB;
+  *st = JOLT_OK;
+  auto ck = [&](cudaError_t e) {
+    if (e != cudaSuccess && *st == JOLT_OK) *st = fail(JOLT_ERR_CUDA, "cholqr: %s", cudaGetErrorString(e));
+  };
+  for (int pass = 0; pass < passes; ++pass) {
     // Wg = src^T src (l x l, float64)
-    CK(gemm_simt(n, l, l, rows, opnd(src, EL_F32, I1((int64_t)rows * l), I1(1), I1(l)),
+    ck(gemm_simt(n, l, l, rows, opnd(src, EL_F32, I1((int64_t)rows * l), I1(1), I1(l)),
                  opnd(src, EL_F32, I1((int64_t)rows * l), I1(1), I1(l)),
                  outd(p->Wg, EL_F64, I1((int64_t)l * l), I1(l), I1(1)), 1.0, 0.0, s));
     const double shift =
         pass == 0 ? 11.0 * ((double)rows * l + (double)l * (l + 1)) * std::ldexp(1.0, -53) * l : 0.0;
-    CK(chol_inv(n, l, p->Wg, (int64_t)l * l, p->Rinv, (int64_t)l * l, shift, status, s));
+    ck(chol_inv(n, l, p->Wg, (int64_t)l * l, p->Rinv, (int64_t)l * l, shift, status, s));
     // dst = src * Rinv
-    CK(gemm_simt(n, rows, l, l, opnd(src, EL_F32, I1((int64_t)rows * l), I1(l), I1(1)),
+    ck(gemm_simt(n, rows, l, l, opnd(src, EL_F32, I1((int64_t)rows * l), I1(l), I1(1)),
                  opnd(p->Rinv, EL_F64, I1((int64_t)l * l), I1(1), I1(l)),
                  outd(dst, EL_F32, I1((int64_t)rows * l), I1(l), I1(1)), 1.0, 0.0, s));
     std::swap(src, dst);
   }
-  // after 3 passes the result sits in `src`
-  if (src != Qout)
-    CK(cudaMemcpyAsync(Qout, src, sizeof(float) * (size_t)n * rows * l, cudaMemcpyDeviceToDevice, s));
-  return JOLT_OK;
+  return src;
+}
+
+// Tensor maps of the operand views (see kernels/gemm_tc.h).
+bool map_x(CUtensorMap* m, const void* X, int L, int H, int T, int D) {
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)T, (uint64_t)H, (uint64_t)L};
+  const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)T * D * 2, (uint64_t)H * T * D * 2};
+  return tc_map_bf16(m, X, 4, dims, str);
+}
+bool map_xt(CUtensorMap* m, const void* XT, int n, int H, int T, int D) {
+  const uint64_t dims[4] = {(uint64_t)T, (uint64_t)D, (uint64_t)H, (uint64_t)n};
+  const uint64_t str[3] = {(uint64_t)T * 2, (uint64_t)D * T * 2, (uint64_t)H * D * T * 2};
+  return tc_map_bf16(m, XT, 4, dims, str);
+}
+bool map_rows(CUtensorMap* m, const void* P, int64_t K, int64_t rows, int64_t batch) {
+  const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)batch};
+  const uint64_t str[2] = {(uint64_t)K * 2, (uint64_t)(rows * K * 2)};
+  return tc_map_bf16(m, P, 3, dims, str);
+}
+
+// CholeskyQR on the transposed layout: Y^T [n][l][rows] -> Q^T (same layout), passes as above.
+float* cholqr_t(jolt_plan_s* p, int rows, float* bufA, float* bufB, int passes, int32_t* status, cudaStream_t s,
+                jolt_status* st) {
+  const int l = p->l, n = p->n_lt;
+  float* src = bufA;
+  float* dst = bufB;
+  *st = JOLT_OK;
+  auto ck = [&](cudaError_t e) {
+    if (e != cudaSuccess && *st == JOLT_OK) *st = fail(JOLT_ERR_CUDA, "cholqr: %s", cudaGetErrorString(e));
+  };
+  for (int pass = 0; pass < passes; ++pass) {
+    // W[i][j] = sum_t Y^T[i][t] Y^T[j][t]
+    ck(gemm_simt(n, l, l, rows, opnd(src, EL_F32, I1((int64_t)rows * l), I1(rows), I1(1)),
+                 opnd(src, EL_F32, I1((int64_t)rows * l), I1(rows), I1(1)),
+                 outd(p->Wg, EL_F64, I1((int64_t)l * l), I1(l), I1(1)), 1.0, 0.0, s));
+    const double shift =
+        pass == 0 ? 11.0 * ((double)rows * l + (double)l * (l + 1)) * std::ldexp(1.0, -53) * l : 0.0;
+    ck(chol_inv(n, l, p->Wg, (int64_t)l * l, p->Rinv, (int64_t)l * l, shift, status, s));
+    // Q^T[j][t] = sum_i Rinv[i][j] Y^T[i][t]
+    ck(gemm_simt(n, l, rows, l, opnd(p->Rinv, EL_F64, I1((int64_t)l * l), I1(1), I1(l)),
+                 opnd(src, EL_F32, I1((int64_t)rows * l), I1(1), I1(rows)),
+                 outd(dst, EL_F32, I1((int64_t)rows * l), I1(rows), I1(1)), 1.0, 0.0, s));
+    std::swap(src, dst);
+  }
+  return src;
 }
 
 }  // namespace
@@ -376,6 +430,8 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
                   (long long)(minb_lt * per_pool_lts));
     }
   }
+  // tensor-core path: bf16 inputs whose token stride is a multiple of 16 bytes (TMA rule)
+  p->use_tc = sh.dtype == JOLT_BF16 && (T % 8) == 0;
   // workspace
   const int64_t n = p->n_lt, HD = (int64_t)H * D, Rm = std::max(p->R, 1), l = std::max(p->l, 2);
   auto layout = [&](char* base, bool assign) -> size_t {
@@ -403,6 +459,12 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     take(p->Gpi, (int64_t)D * D);
     take(p->Pi32, (int64_t)D * D);
     take(p->Pib, (int64_t)D * D);
+    if (p->use_tc) {
+      take(p->XT, n * HD * T);
+      take(p->Cpart, n * H * D * D);
+      if (p->encoder == JOLT_ENC_SKETCH)
+        for (int i = 0; i < 3; ++i) take(p->QTp[i], n * l * std::max<int64_t>(T, HD));
+    }
     if (p->encoder == JOLT_ENC_SKETCH) {
       take(p->Om, n * HD * l);
       take(p->Y, n * T * l);
@@ -491,7 +553,30 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       CK(sumsq_batched(L, HTD, X[k], xt, HTD, p->xx + (int64_t)k * L, p->xx_part + (int64_t)k * L * 64, s));
     }
   }
-  {
+  CUtensorMap mx[2], mxt;
+  if (p->use_tc) {
+    {
+      PROF("transpose", s);
+      for (int k = 0; k < kinds; ++k)
+        CK(transpose_x((const __nv_bfloat16*)X[k], p->XT, L, H, T, D, k * L, s));
+    }
+    for (int k = 0; k < kinds; ++k)
+      if (!map_x(&mx[k], X[k], L, H, T, D)) return fail(JOLT_ERR_CUDA, "tensor map of X rejected");
+    if (!map_xt(&mxt, p->XT, n, H, T, D)) return fail(JOLT_ERR_CUDA, "tensor map of X^T rejected");
+    PROF("feature_gram", s);
+    // per-head partials C_D[lt][h] = X_h^T X_h on the tensor cores, then a float64 sum over heads
+    TcGemmParams g;
+    g.amap[0] = mxt;
+    g.bmap[0] = mxt;
+    g.av.mode = g.bv.mode = VIEW_XT_PERHEAD;
+    g.av.H = g.bv.H = H;
+    g.av.D = g.bv.D = D;
+    g.M = D; g.N = D; g.KB = (T + 63) / 64;
+    g.C = p->Cpart; g.c_sm = D; g.c_sn = 1; g.c_sb = (int64_t)D * D;
+    g.status = status;
+    CK(gemm_tc(n * H, g, s));
+    CK(sum_heads(n, H, (int64_t)D * D, p->Cpart, p->CD, nullptr, s));
+  } else {
     PROF("feature_gram", s);
     // C_D = sum over rows r = (h, t) of X[r, :]^T X[r, :]
     for (int k = 0; k < kinds; ++k)
@@ -509,14 +594,113 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
     CK(round_bf16((int64_t)n * D * D, p->UD32, p->UDb, p->UDf, s));
   }
   if (R > 0) {
-    if (p->encoder == JOLT_ENC_SKETCH) {
+    if (p->encoder == JOLT_ENC_SKETCH && p->use_tc) {
       const int l = p->l;
+      p->q_t = true;
       {
         PROF("sketch_omega", s);
         std::vector<int32_t> ids = p->lt_ids;
-        CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, s));
+        CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, true, s));   // Omega^T [l][HD]
       }
-      jolt_status r;
+      jolt_status r = JOLT_OK;
+      auto tc_params = [&]() {
+        TcGemmParams g;
+        g.status = status;
+        return g;
+      };
+      // Y^T = (A Omega)^T or (A Q')^T: rows t, K = (h, d); transposed store into [l][T]
+      auto y_pass = [&](const __nv_bfloat16* const* bparts, int nparts, float* Yout) -> jolt_status {
+        for (int k = 0; k < kinds; ++k) {
+          TcGemmParams g = tc_params();
+          g.amap[0] = mx[k];
+          g.av.mode = VIEW_X_TOKENROWS;
+          g.av.D = D;
+          for (int i = 0; i < nparts; ++i)
+            if (!map_rows(&g.bmap[i], bparts[i] + (int64_t)k * L * l * HD, HD, l, L))
+              return fail(JOLT_ERR_CUDA, "tensor map rejected");
+          g.na = 1; g.nb = nparts;
+          g.M = T; g.N = l; g.KB = (int)(HD / 64);
+          g.C = Yout + (int64_t)k * L * l * T; g.c_sm = 1; g.c_sn = T; g.c_sb = (int64_t)l * T;
+          CK(gemm_tc(L, g, s));
+        }
+        return JOLT_OK;
+      };
+      {
+        PROF("sketch_gemm", s);
+        const __nv_bfloat16* om[1] = {p->Om};
+        r = y_pass(om, 1, p->Y);
+        if (r != JOLT_OK) return r;
+      }
+      const int q = p->cfg.power_iters;
+      float* Q;
+      {
+        PROF("cholqr", s);
+        Q = cholqr_t(p, T, p->Y, p->Y2, q > 0 ? 1 : 2, status, s, &r);
+        if (r != JOLT_OK) return r;
+      }
+      for (int it = 0; it < q; ++it) {
+        {
+          PROF("sketch_gemm", s);
+          CK(split_bf16((int64_t)n * l * T, Q, p->QTp[0], p->QTp[1], nullptr, s));
+          // Z^T = (A^T Q)^T: rows (h, d), K = t; transposed store into [l][HD]
+          TcGemmParams g = tc_params();
+          g.amap[0] = mxt;
+          g.av.mode = VIEW_XT_FEATROWS;
+          g.av.D = D;
+          for (int i = 0; i < 2; ++i)
+            if (!map_rows(&g.bmap[i], p->QTp[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+          g.na = 1; g.nb = 2;
+          g.M = (int)HD; g.N = l; g.KB = (T + 63) / 64;
+          g.C = p->Z; g.c_sm = 1; g.c_sn = HD; g.c_sb = (int64_t)l * HD;
+          CK(gemm_tc(n, g, s));
+        }
+        float* Qz;
+        {
+          PROF("cholqr", s);
+          Qz = cholqr_t(p, (int)HD, p->Z, p->Z2, 1, status, s, &r);
+          if (r != JOLT_OK) return r;
+        }
+        float* Ydst = (Q == p->Y) ? p->Y2 : p->Y;
+        float* Yalt = (Q == p->Y) ? p->Y : p->Y2;
+        {
+          PROF("sketch_gemm", s);
+          CK(split_bf16((int64_t)n * l * HD, Qz, p->QTp[0], p->QTp[1], nullptr, s));
+          const __nv_bfloat16* qp[2] = {p->QTp[0], p->QTp[1]};
+          r = y_pass(qp, 2, Ydst);
+          if (r != JOLT_OK) return r;
+        }
+        {
+          PROF("cholqr", s);
+          Q = cholqr_t(p, T, Ydst, Yalt, it + 1 == q ? 2 : 1, status, s, &r);
+          if (r != JOLT_OK) return r;
+        }
+      }
+      {
+        PROF("sketch_gemm", s);
+        // B = Q^T A (l x HD): rows j, K = t; Q^T in three bf16 parts for float32 accuracy
+        CK(split_bf16((int64_t)n * l * T, Q, p->QTp[0], p->QTp[1], p->QTp[2], s));
+        TcGemmParams g = tc_params();
+        for (int i = 0; i < 3; ++i)
+          if (!map_rows(&g.amap[i], p->QTp[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+        g.bmap[0] = mxt;
+        g.bv.mode = VIEW_XT_FEATROWS;
+        g.bv.D = D;
+        g.na = 3; g.nb = 1;
+        g.M = l; g.N = (int)HD; g.KB = (T + 63) / 64;
+        g.C = p->Bm; g.c_sm = HD; g.c_sn = 1; g.c_sb = (int64_t)l * HD;
+        CK(gemm_tc(n, g, s));
+      }
+      p->Qfinal = Q;
+    }
+    if (p->encoder == JOLT_ENC_SKETCH && !p->use_tc) {
+      const int l = p->l;
+      p->q_t = false;
+      {
+        PROF("sketch_omega", s);
+        std::vector<int32_t> ids = p->lt_ids;
+        CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, false, s));
+      }
+      jolt_status r = JOLT_OK;
       {
         PROF("sketch_gemm", s);
         // Y0 = A Omega, A[t, h*D + d] = X[h][t][d]
@@ -525,36 +709,41 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
                        opnd(p->Om + (int64_t)k * L * HD * l, EL_BF16, I1(HD * l), I1(1), I1(l)),
                        outd(p->Y + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(l), I1(1)), 1.0, 0.0, s));
       }
+      const int q = p->cfg.power_iters;
+      float* Q;
       {
         PROF("cholqr", s);
-        r = cholqr3(p, T, p->Y, p->Y2, status, s);
+        Q = cholqr(p, T, p->Y, p->Y2, q > 0 ? 1 : 2, status, s, &r);
         if (r != JOLT_OK) return r;
       }
-      for (int it = 0; it < p->cfg.power_iters; ++it) {
+      for (int it = 0; it < q; ++it) {
         {
           PROF("sketch_gemm", s);
           // Z = A^T Q  (HD x l)
           for (int k = 0; k < kinds; ++k)
             CK(gemm_simt(L, (int)HD, l, T, opnd(X[k], xt, I1(HTD), I2(D, 1, (int64_t)T * D), I1(D)),
-                         opnd(p->Y2 + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(1), I1(l)),
+                         opnd(Q + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(1), I1(l)),
                          outd(p->Z + (int64_t)k * L * HD * l, EL_F32, I1(HD * l), I1(l), I1(1)), 1.0, 0.0, s));
         }
+        float* Qz;
         {
           PROF("cholqr", s);
-          r = cholqr3(p, (int)HD, p->Z, p->Z2, status, s);
+          Qz = cholqr(p, (int)HD, p->Z, p->Z2, 1, status, s, &r);
           if (r != JOLT_OK) return r;
         }
+        float* Ydst = (Q == p->Y) ? p->Y2 : p->Y;
+        float* Yalt = (Q == p->Y) ? p->Y : p->Y2;
         {
           PROF("sketch_gemm", s);
           // Y = A Q'
           for (int k = 0; k < kinds; ++k)
             CK(gemm_simt(L, T, l, (int)HD, opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
-                         opnd(p->Z2 + (int64_t)k * L * HD * l, EL_F32, I1(HD * l), I1(1), I1(l)),
-                         outd(p->Y + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(l), I1(1)), 1.0, 0.0, s));
+                         opnd(Qz + (int64_t)k * L * HD * l, EL_F32, I1(HD * l), I1(1), I1(l)),
+                         outd(Ydst + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(l), I1(1)), 1.0, 0.0, s));
         }
         {
           PROF("cholqr", s);
-          r = cholqr3(p, T, p->Y, p->Y2, status, s);
+          Q = cholqr(p, T, Ydst, Yalt, it + 1 == q ? 2 : 1, status, s, &r);
           if (r != JOLT_OK) return r;
         }
       }
@@ -562,10 +751,14 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         PROF("sketch_gemm", s);
         // B = Q^T A (l x HD)
         for (int k = 0; k < kinds; ++k)
-          CK(gemm_simt(L, l, (int)HD, T, opnd(p->Y2 + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(1), I1(l)),
+          CK(gemm_simt(L, l, (int)HD, T, opnd(Q + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(1), I1(l)),
                        opnd(X[k], xt, I1(HTD), I2(D, 1, (int64_t)T * D), I1(D)),
                        outd(p->Bm + (int64_t)k * L * l * HD, EL_F32, I1(l * HD), I1(HD), I1(1)), 1.0, 0.0, s));
       }
+      p->Qfinal = Q;
+    }
+    if (p->encoder == JOLT_ENC_SKETCH) {
+      const int l = p->l;
       {
         PROF("small_gemm", s);
         // B B^T
@@ -581,7 +774,8 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       {
         PROF("small_gemm", s);
         // U_T = Q W[:, :R]
-        CK(gemm_simt(n, T, R, l, opnd(p->Y2, EL_F32, I1((int64_t)T * l), I1(l), I1(1)),
+        CK(gemm_simt(n, T, R, l, opnd(p->Qfinal, EL_F32, I1((int64_t)T * l), p->q_t ? I1(1) : I1(l),
+                                      p->q_t ? I1(T) : I1(1)),
                      opnd(p->Wv, EL_F32, I1((int64_t)l * l), I1(1), I1(l)),
                      outd(p->UT32, EL_F32, I1((int64_t)T * R), I1(R), I1(1)), 1.0, 0.0, s));
       }
@@ -973,11 +1167,20 @@ JOLT_API jolt_status jolt_export_debug(jolt_stream_t st, int32_t what, int32_t l
         n = sizeof(double) * tmp.size();
         host_src = true;
         break;
-      case JOLT_DBG_OMEGA:
+      case JOLT_DBG_OMEGA: {
         if (i < 0 || p->encoder != JOLT_ENC_SKETCH) return fail(JOLT_ERR_INVALID_ARG, "no sketch for this lt");
-        src = p->Om + (int64_t)i * st->H * st->D * p->l;
-        n = sizeof(__nv_bfloat16) * st->H * st->D * p->l;
+        const int64_t HD = (int64_t)st->H * st->D, l = p->l;
+        n = sizeof(__nv_bfloat16) * HD * l;
+        std::vector<uint16_t> raw((size_t)(HD * l));
+        CK(cudaMemcpy(raw.data(), p->Om + (int64_t)i * HD * l, n, cudaMemcpyDeviceToHost));
+        tmp.assign((n + 7) / 8, 0.0);
+        uint16_t* o = reinterpret_cast<uint16_t*>(tmp.data());
+        for (int64_t r = 0; r < HD; ++r)          // always exported as [HD][l]
+          for (int64_t c = 0; c < l; ++c) o[r * l + c] = p->use_tc ? raw[(size_t)(c * HD + r)] : raw[(size_t)(r * l + c)];
+        src = tmp.data();
+        host_src = true;
         break;
+      }
       default:
         return fail(JOLT_ERR_INVALID_ARG, "jolt_export_debug: unknown item %d", what);
     }
@@ -988,6 +1191,33 @@ JOLT_API jolt_status jolt_export_debug(jolt_stream_t st, int32_t what, int32_t l
   else CK(cudaMemcpy(buf, src, n, cudaMemcpyDeviceToHost));
   *len = n;
   return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const void* B,
+                                             float* C, void* cuda_stream) {
+  g_err.clear();
+  if (M <= 0 || N <= 0 || K <= 0 || (K % 8) || !A || !B || !C)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_selftest_gemm_bf16: bad sizes or pointers");
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  TcGemmParams p;
+  const uint64_t adims[3] = {(uint64_t)K, (uint64_t)M, 1}, astr[2] = {(uint64_t)K * 2, (uint64_t)K * M * 2};
+  const uint64_t bdims[3] = {(uint64_t)K, (uint64_t)N, 1}, bstr[2] = {(uint64_t)K * 2, (uint64_t)K * N * 2};
+  if (!tc_map_bf16(&p.amap[0], A, 3, adims, astr) || !tc_map_bf16(&p.bmap[0], B, 3, bdims, bstr))
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_selftest_gemm_bf16: tensor map rejected");
+  p.na = p.nb = 1;
+  p.M = M; p.N = N; p.KB = (K + 63) / 64;
+  p.C = C; p.c_sm = N; p.c_sn = 1; p.c_sb = (int64_t)M * N;
+  int32_t* st = nullptr;
+  CK(cudaMallocAsync(&st, sizeof(int32_t), s));
+  CK(cudaMemsetAsync(st, 0, sizeof(int32_t), s));
+  p.status = st;
+  cudaError_t e = gemm_tc(1, p, s);
+  int32_t h = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h, st, sizeof(h), cudaMemcpyDeviceToHost, s);
+  cudaFreeAsync(st, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_selftest_gemm_bf16: %s", cudaGetErrorString(e));
+  return status_of(h);
 }
 
 JOLT_API uint64_t jolt_launch_count(void) { return g_launches.load(); }

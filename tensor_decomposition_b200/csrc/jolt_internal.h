@@ -64,8 +64,9 @@ cudaError_t gemm_simt(int batch, int M, int N, int K, const Operand& A, const Op
 // Counter-based normals (SplitMix64 + Box-Muller), see rotation.cu.
 cudaError_t gauss_f64(uint64_t seed, uint64_t stream_id, int64_t n, double* out, cudaStream_t s);
 // Sketch matrices Omega_lt = bf16(N(0,1)) of shape [HD][l], lt in [0, n_lt) uses stream 2 + lt_id[lt].
+// transposed = true stores element (i, j) at [j][i] (layout [l][HD]).
 cudaError_t sketch_omega(uint64_t seed, const int32_t* lt_ids_host, int n_lt, int64_t HD, int l,
-                         __nv_bfloat16* out, cudaStream_t s);
+                         __nv_bfloat16* out, bool transposed, cudaStream_t s);
 // Haar rotation from a D x D float64 Gaussian (Householder QR, signs of diag(R) moved into Q).
 cudaError_t haar_from_gauss(const double* G, int D, float* Pi_f32, __nv_bfloat16* Pi_bf16,
                             cudaStream_t s);
@@ -148,6 +149,13 @@ struct DecodeArgs {
   const uint8_t* body;
 };
 cudaError_t decode(const DecodeArgs& a, cudaStream_t s);
+
+// Layout helpers of the tensor-core path (layout.cu).
+cudaError_t transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int L, int H, int T, int D, int lt_base,
+                        cudaStream_t s);
+cudaError_t split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2,
+                       cudaStream_t s);
+cudaError_t sum_heads(int n, int H, int64_t per, const float* part, float* out32, double* out64, cudaStream_t s);
 
 // Check for NaN/Inf in an input tensor (sets ST_NONFINITE).
 cudaError_t check_finite(int64_t n, const void* x, ElemType t, int32_t* status, cudaStream_t s);

@@ -85,17 +85,31 @@ __device__ __forceinline__ void grid_rank(int gi, int step, int D, int& rt, int&
 
 constexpr int kMaxUnits = 2 * kMaxGroups;
 
-// Single CTA of 1024 threads: warp w evaluates units w, w + 32, ...
+// Single CTA of 1024 threads: warp w evaluates units w, w + 32, ... The candidates' bytes per
+// layer and, when they fit, the pool's error tables are staged in shared memory.
+constexpr size_t kDualSmem = 160 * 1024;
+
 __global__ void __launch_bounds__(1024) k_dual(DualArgs a) {
+  extern __shared__ unsigned char dsm[];
   __shared__ int nlay[kMaxGroups];
   __shared__ int choice[kMaxUnits];
   __shared__ int64_t cbytes[kMaxUnits];
+  __shared__ Cand wbest[32];
+  __shared__ int wunit[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nu = a.G * 2;
   const int ncand = a.nbits * a.ngrid;
   StreamMeta* meta = a.meta;
+  int64_t* cand_bytes = reinterpret_cast<int64_t*>(dsm);           // per layer, [ncand]
+  double* err_s = reinterpret_cast<double*>(cand_bytes + ncand);    // [units of pool][ncand]
+  const size_t err_cap = (kDualSmem - (size_t)ncand * 8) / 8;
   for (int g = tid; g < a.G; g += blockDim.x)
     nlay[g] = (int)(((int64_t)(g + 1) * a.L) / a.G - ((int64_t)g * a.L) / a.G);
+  for (int c = tid; c < ncand; c += blockDim.x) {
+    int rt, rd;
+    grid_rank(c % a.ngrid, a.step, a.D, rt, rd);
+    cand_bytes[c] = lt_bytes(a.H, a.T, a.D, rt, rd, a.bits[c / a.ngrid]);
+  }
   // Unit tables: E summed over the group's layers in increasing layer order, times phi(b).
   for (int e = tid; e < nu * a.ngrid; e += blockDim.x) {
     const int u = e / a.ngrid, gi = e % a.ngrid;
@@ -107,36 +121,58 @@ __global__ void __launch_bounds__(1024) k_dual(DualArgs a) {
     for (int bi = 0; bi < a.nbits; ++bi)
       a.unit_err[(int64_t)u * ncand + bi * a.ngrid + gi] = __dmul_rn(s, a.phi[bi]);
   }
+  __threadfence_block();
   __syncthreads();
   const int npools = (a.has_v && a.split) ? 2 : 1;
   for (int pool = 0; pool < npools; ++pool) {
     const int64_t budget = a.budget_pool[pool];
-    // unit u belongs to this pool?
     auto in_pool = [&](int u) -> bool {
       const int k = u % 2;
       if (k == 1 && !a.has_v) return false;
       if (npools == 1) return true;
       return k == pool;
     };
-    // choose(lam) for every unit of the pool; writes choice[] and cbytes[]
+    // stage this pool's tables (slot = rank of u among the pool's units)
+    int nslot = 0;
+    for (int u = 0; u < nu; ++u) nslot += in_pool(u);
+    const bool cached = (size_t)nslot * ncand <= err_cap;
+    if (cached) {
+      for (int e = tid; e < nslot * ncand; e += blockDim.x) {
+        const int slot = e / ncand, c = e % ncand;
+        int u = -1;
+        for (int v = 0, seen = 0; v < nu; ++v)
+          if (in_pool(v)) { if (seen == slot) { u = v; break; } ++seen; }
+        err_s[e] = a.unit_err[(int64_t)u * ncand + c];
+      }
+    }
+    __syncthreads();
+    // choose(lam) for every unit of the pool; writes choice[] and cbytes[], returns total bytes.
+    // Units get 32 / nslot warps each (at least one); each warp scans a strided share of the
+    // candidates, then one thread per unit merges its warps' bests in warp order.
+    const int nwarps = (int)(blockDim.x >> 5);
+    const int wpu = nslot >= nwarps ? 1 : nwarps / nslot;
     auto choose_all = [&](double lam, bool min_bytes_only) {
-      for (int u = warp; u < nu; u += (int)(blockDim.x >> 5)) {
-        if (!in_pool(u)) continue;
-        const int g = u / 2;
+      for (int base = 0; base < nslot; base += nwarps / wpu) {
+        const int us = base + warp % (nwarps / wpu);          // unit slot of this warp
+        const int part = warp / (nwarps / wpu);
         Cand best;
         best.cost = 0.0;
         best.idx = -1;
-        for (int c = lane; c < ncand; c += 32) {
-          const int bi = c / a.ngrid, gi = c % a.ngrid;
-          Cand x;
-          grid_rank(gi, a.step, a.D, x.rt, x.rd);
-          x.b = a.bits[bi];
-          x.bytes = (int64_t)nlay[g] * lt_bytes(a.H, a.T, a.D, x.rt, x.rd, x.b);
-          x.cost = min_bytes_only ? 0.0
-                                  : __dadd_rn(a.unit_err[(int64_t)u * ncand + c],
-                                              __dmul_rn(lam, (double)x.bytes));
-          x.idx = c;
-          if (best.idx < 0 || less_key(x, best)) best = x;
+        int u = -1;
+        if (us < nslot && part < wpu) {
+          for (int v = 0, seen = 0; v < nu; ++v)
+            if (in_pool(v)) { if (seen == us) { u = v; break; } ++seen; }
+          const int g = u / 2;
+          const double* errp = cached ? err_s + (size_t)us * ncand : a.unit_err + (int64_t)u * ncand;
+          for (int c = part * 32 + lane; c < ncand; c += 32 * wpu) {
+            Cand x;
+            grid_rank(c % a.ngrid, a.step, a.D, x.rt, x.rd);
+            x.b = a.bits[c / a.ngrid];
+            x.bytes = (int64_t)nlay[g] * cand_bytes[c];
+            x.cost = min_bytes_only ? 0.0 : __dadd_rn(errp[c], __dmul_rn(lam, (double)x.bytes));
+            x.idx = c;
+            if (best.idx < 0 || less_key(x, best)) best = x;
+          }
         }
         for (int o = 16; o > 0; o >>= 1) {
           Cand y;
@@ -149,11 +185,27 @@ __global__ void __launch_bounds__(1024) k_dual(DualArgs a) {
           if (y.idx >= 0 && (best.idx < 0 || less_key(y, best))) best = y;
         }
         if (lane == 0) {
-          choice[u] = best.idx;
-          cbytes[u] = best.bytes;
+          wbest[warp] = best;
+          wunit[warp] = u;
         }
+        __syncthreads();
+        if (tid < nwarps / wpu && base + tid < nslot) {
+          Cand m;
+          m.idx = -1;
+          int uu = -1;
+          for (int pp = 0; pp < wpu; ++pp) {
+            const int w = pp * (nwarps / wpu) + tid;
+            const Cand y = wbest[w];
+            if (wunit[w] >= 0) uu = wunit[w];
+            if (y.idx >= 0 && (m.idx < 0 || less_key(y, m))) m = y;
+          }
+          if (uu >= 0) {
+            choice[uu] = m.idx;
+            cbytes[uu] = m.bytes;
+          }
+        }
+        __syncthreads();
       }
-      __syncthreads();
       int64_t tb = 0;
       for (int u = 0; u < nu; ++u)
         if (in_pool(u)) tb += cbytes[u];
@@ -277,7 +329,9 @@ cudaError_t energy_table(const TableArgs& a, cudaStream_t s) {
 
 cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s) {
   if (a.G > kMaxGroups || a.L > kMaxL) return cudaErrorInvalidValue;
-  k_dual<<<1, 1024, 0, s>>>(a);
+  cudaError_t e = cudaFuncSetAttribute(k_dual, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
+  if (e != cudaSuccess) return e;
+  k_dual<<<1, 1024, kDualSmem, s>>>(a);
   note_launch();
   return cudaGetLastError();
 }

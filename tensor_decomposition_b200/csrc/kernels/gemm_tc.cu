@@ -1,0 +1,224 @@
+// Batched bf16 GEMM on the 5th-generation tensor cores: C[b] = sum_p A_p[b] B_p[b]^T.
+//
+// It carries the dense contractions of the JoLT factor analysis ("A JoLT for the KV Cache",
+// arXiv 2607.12550v2, Abstract: the partial Tucker factors of the token and feature axes and
+// the randomized-SVD "FlashJoLT" sketch): the feature Gram C_D = sum_h X_h^T X_h and the
+// four sketch passes A Omega, A^T Q, A Q', Q^T A over the token unfolding A = X_(2).
+// float32 operands enter as a sum of up to three bf16 parts (hi + lo + lo2), each part one
+// more pass of the tensor core over the same accumulator.
+//
+// Structure: one CTA per 128 x 128 output tile. Warp 0 issues TMA tile loads (128 rows x 64
+// bf16, 128-byte swizzle, no multicast) into a ring of stages; warp 1 owns the Tensor Memory
+// accumulator and issues tcgen05.mma (M = 128, N = 128, K = 16) from one thread; warps 4-7
+// read the accumulator back with tcgen05.ld and store float32. Every wait is bounded and
+// reports ST_TIMEOUT instead of hanging.
+#include "../jolt_internal.h"
+#include "sm100.cuh"
+#include "gemm_tc.h"
+
+namespace jolt {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTile = 128;
+constexpr int kBK = 64;
+constexpr int kTileBytes = kTile * kBK * 2;   // 16 KB per operand part and stage
+constexpr uint32_t kMaxPoll = 1u << 22;
+
+__device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, int b, int& c0, int& c1, int& c2,
+                                            int& c3) {
+  switch (v.mode) {
+    case VIEW_X_TOKENROWS: {           // map (D, T, H, L): rows t, K = (h, d)
+      const int kpd = v.D / kBK;
+      c0 = (kb % kpd) * kBK; c1 = row0; c2 = kb / kpd; c3 = b;
+      break;
+    }
+    case VIEW_XT_FEATROWS:             // map (T, D, H, n): rows (h, d), K = t
+      c0 = kb * kBK; c1 = row0 % v.D; c2 = row0 / v.D; c3 = b;
+      break;
+    case VIEW_XT_PERHEAD:              // same map, batch b = i * H + h: rows d, K = t
+      c0 = kb * kBK; c1 = row0; c2 = b % v.H; c3 = b / v.H;
+      break;
+    default:                           // VIEW_ROWS_K: map (K, rows, batch)
+      c0 = kb * kBK; c1 = row0; c2 = b; c3 = 0;
+      break;
+  }
+}
+
+__device__ __forceinline__ void view_load(const TcView& v, const CUtensorMap* map, void* dst, uint64_t* bar,
+                                          int row0, int kb, int b) {
+  int c0, c1, c2, c3;
+  view_coords(v, row0, kb, b, c0, c1, c2, c3);
+  if (v.mode == VIEW_ROWS_K) tma_load_3d(dst, map, bar, c0, c1, c2);
+  else tma_load_4d(dst, map, bar, c0, c1, c2, c3);
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGemmParams p) {
+  extern __shared__ uint8_t smraw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ uint32_t tmem_base;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile, b = blockIdx.z;
+  const int parts = p.na > p.nb ? p.na : p.nb;
+  const int stage_bytes = (p.na + p.nb) * kTileBytes;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&accum_bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < p.na; ++i) prefetch_tensormap(&p.amap[i]);
+    for (int i = 0; i < p.nb; ++i) prefetch_tensormap(&p.bmap[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base, kTile);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      for (int kb = 0; kb < p.KB; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t parity = ((kb / STAGES) & 1) ^ 1;
+        if (!mbar_wait(&empty_bar[s], parity, kMaxPoll)) {
+          atomicOr(p.status, ST_TIMEOUT);
+          break;
+        }
+        uint8_t* st = smem + s * stage_bytes;
+        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)stage_bytes);
+        for (int i = 0; i < p.na; ++i) view_load(p.av, &p.amap[i], st + i * kTileBytes, &full_bar[s], m0, kb, b);
+        for (int i = 0; i < p.nb; ++i)
+          view_load(p.bv, &p.bmap[i], st + (p.na + i) * kTileBytes, &full_bar[s], n0, kb, b);
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      const uint32_t idesc = idesc_bf16_f32(kTile, kTile);
+      bool ok = true;
+      for (int kb = 0; kb < p.KB && ok; ++kb) {
+        const int s = kb % STAGES;
+        if (!mbar_wait(&full_bar[s], (kb / STAGES) & 1, kMaxPoll)) {
+          atomicOr(p.status, ST_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * stage_bytes);
+        for (int t = 0; t < parts; ++t) {
+          const int ia = t < p.na ? t : p.na - 1, ib = t < p.nb ? t : p.nb - 1;
+          const uint32_t abase = st + ia * kTileBytes, bbase = st + (p.na + ib) * kTileBytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = desc_kmajor_sw128(abase + k * 32);
+            const uint64_t bd = desc_kmajor_sw128(bbase + k * 32);
+            umma_bf16(tmem, ad, bd, idesc, (kb | t | k) != 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty_bar[s]);   // frees the stage once these MMAs have read it
+      }
+      umma_commit(&accum_bar);
+    }
+  } else if (warp >= 4) {
+    const int e = warp - 4;                      // TMEM lanes 32e .. 32e + 31
+    const bool ok = mbar_wait(&accum_bar, 0, kMaxPoll);
+    if (!ok && lane == 0) atomicOr(p.status, ST_TIMEOUT);
+    tc_fence_after();
+    const int m = m0 + 32 * e + lane;
+    int64_t boff;
+    if (p.c_batch_in > 0) boff = (int64_t)(b / p.c_batch_in) * p.c_sb_out + (int64_t)(b % p.c_batch_in) * p.c_sb;
+    else boff = (int64_t)b * p.c_sb;
+    float* C = p.C + boff;
+#pragma unroll 1
+    for (int c = 0; c < kTile / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * e) << 16) + (uint32_t)(c * 32), r);
+      tmem_ld_wait();
+      if (ok && m < p.M) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int n = n0 + c * 32 + j;
+          if (n < p.N) C[(int64_t)m * p.c_sm + (int64_t)n * p.c_sn] = __uint_as_float(r[j]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, kTile);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rank < 2 || rank > 5) return false;
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t box[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    estr[i] = 1;
+    box[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) {
+    gstr[i] = strides[i];
+    if (strides[i] % 16) return false;
+  }
+  if (reinterpret_cast<uintptr_t>(base) % 16) return false;
+  box[0] = kBK;     // 64 bf16 = 128 bytes, the swizzle span
+  box[1] = kTile;   // 128 rows
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gdim, gstr,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
+  if (batch <= 0 || p.M <= 0 || p.N <= 0) return cudaSuccess;
+  if (p.na < 1 || p.na > 3 || p.nb < 1 || p.nb > 3 || batch > 65535) return cudaErrorInvalidValue;
+  const int stage_bytes = (p.na + p.nb) * kTileBytes;
+  const dim3 g((p.N + kTile - 1) / kTile, (p.M + kTile - 1) / kTile, batch);
+  if (stage_bytes * 4 + 1024 <= 200 * 1024) {
+    const int smem = stage_bytes * 4 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_gemm_tc<4><<<g, 256, smem, s>>>(p);
+  } else {
+    const int smem = stage_bytes * 2 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_gemm_tc<2><<<g, 256, smem, s>>>(p);
+  }
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace jolt

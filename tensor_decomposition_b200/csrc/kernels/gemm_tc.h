@@ -1,0 +1,44 @@
+// Host-visible description of the tensor-core GEMM (gemm_tc.cu). Separate from
+// jolt_internal.h because it needs the driver API's CUtensorMap type.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace jolt {
+
+// How an operand's 128-row x 64-column tiles are addressed in its tensor map.
+enum TcViewMode : int32_t {
+  VIEW_ROWS_K = 0,        // 3-D map (K, rows, batch)
+  VIEW_X_TOKENROWS = 1,   // 4-D map of X [L][H][T][D] as (D, T, H, L): rows = tokens, K = (head, feature)
+  VIEW_XT_FEATROWS = 2,   // 4-D map of X^T [n][H][D][T] as (T, D, H, n): rows = (head, feature), K = tokens
+  VIEW_XT_PERHEAD = 3     // same map, batch index = layer-tensor * H + head: rows = features, K = tokens
+};
+
+struct TcView {
+  int32_t mode = VIEW_ROWS_K;
+  int32_t D = 128;
+  int32_t H = 1;
+};
+
+struct TcGemmParams {
+  CUtensorMap amap[3];
+  CUtensorMap bmap[3];
+  TcView av, bv;
+  int32_t na = 1, nb = 1;   // bf16 parts of A and B; products pair part t of each (clamped)
+  int32_t M = 0, N = 0, KB = 0;
+  float* C = nullptr;       // C[b] + m * c_sm + n * c_sn
+  int64_t c_sm = 0, c_sn = 0, c_sb = 0, c_sb_out = 0;
+  int32_t c_batch_in = 0;   // > 0: batch offset = (b / c_batch_in) * c_sb_out + (b % c_batch_in) * c_sb
+  int32_t* status = nullptr;
+};
+
+// 2-D..5-D bf16 tensor map with a 64 x 128 box and 128-byte swizzle. dims[0] is the
+// contiguous dimension; strides[i] is the byte stride of dims[i + 1]. False if the driver
+// entry point is missing or an alignment rule fails.
+bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides);
+
+cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s);
+
+}  // namespace jolt

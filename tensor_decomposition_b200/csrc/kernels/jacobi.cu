@@ -6,7 +6,7 @@
 // C_D = sum_h X_h^T X_h (D x D), and, for the randomized-SVD ("FlashJoLT") token factor,
 // the Rayleigh-Ritz rotation W from B B^T (l x l) and the orthonormalisation of sketches.
 //
-// Jacobi: n even, n <= 128. Each sweep runs n - 1 rounds of the circle-method tournament,
+// Jacobi: n <= 128, padded to 128. Each sweep runs 127 rounds of the circle-method tournament,
 // so a round rotates n/2 disjoint (p, q) pairs at once. The rotation is the symmetric Schur
 // 2x2 step (Golub & Van Loan, Matrix Computations, sec. 8.5): tau = (a_qq - a_pp) / (2 a_pq),
 // t = sign(tau) / (|tau| + sqrt(1 + tau^2)), c = 1 / sqrt(1 + t^2), s = t c, and
@@ -23,28 +23,40 @@ namespace {
 
 constexpr int kLd = kMaxN + 1;   // padded row stride of the shared matrices
 
-__device__ __forceinline__ int tour_player(int pos, int r, int n) {
-  return pos == 0 ? 0 : ((pos - 1 + r) % (n - 1)) + 1;
+__device__ __forceinline__ int tour_player(int pos, int r) {
+  return pos == 0 ? 0 : ((pos - 1 + r) % (kMaxN - 1)) + 1;
 }
 
+// Every problem is embedded in a 128 x 128 one (indices >= n get the diagonal value
+// -(1 + trace), zero coupling, so they never rotate against the real block and sort last);
+// the fixed size turns all index arithmetic into shifts and masks.
 __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t sA, float* Vout,
                                                 int64_t sV, float* lam, int64_t sL, int max_sweeps,
                                                 int32_t* status) {
+  constexpr int NP = kMaxN, HP = kMaxN / 2;
   extern __shared__ double smd[];
-  double* V = smd;                      // n x kLd, float64: stays orthogonal over many rounds
-  double* csd = V + kMaxN * kLd;        // c[64], s[64] in float64
-  float* A = reinterpret_cast<float*>(csd + kMaxN);   // n x kLd
-  float* cs = A + kMaxN * kLd;          // c[64], s[64] in float32 for the A update
-  int* pq = reinterpret_cast<int*>(cs + kMaxN);  // p[64], q[64]
-  int* rank = pq + kMaxN;               // n
+  double* V = smd;                      // NP x kLd, float64: stays orthogonal over many rounds
+  double* csd = V + NP * kLd;           // c[64], s[64] in float64
+  float* A = reinterpret_cast<float*>(csd + NP);   // NP x kLd
+  float* cs = A + NP * kLd;             // c[64], s[64] in float32 for the A update
+  int* pq = reinterpret_cast<int*>(cs + NP);       // p[64], q[64]
+  int* rank = pq + NP;                  // NP
   __shared__ int rotated;
-  __shared__ float dmax_s;
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int h = n / 2;
+  __shared__ float dmax_s, pad_s;
+  const int tid = threadIdx.x;
   const float* a_in = Ain + (int64_t)blockIdx.x * sA;
-  for (int i = tid; i < n * n; i += nt) {
-    const int r = i / n, c = i % n;
-    A[r * kLd + c] = a_in[i];
+  if (tid == 0) {
+    float tr = 0.0f;
+    for (int i = 0; i < n; ++i) tr += fabsf(a_in[(int64_t)i * n + i]);
+    pad_s = -(1.0f + tr);
+  }
+  __syncthreads();
+  for (int e = tid; e < NP * NP; e += 512) {
+    const int r = e >> 7, c = e & (NP - 1);
+    float v = 0.0f;
+    if (r < n && c < n) v = a_in[(int64_t)r * n + c];
+    else if (r == c) v = pad_s;
+    A[r * kLd + c] = v;
     V[r * kLd + c] = (r == c) ? 1.0 : 0.0;
   }
   __syncthreads();
@@ -59,9 +71,9 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
   for (; sweep < max_sweeps; ++sweep) {
     if (tid == 0) rotated = 0;
     __syncthreads();
-    for (int r = 0; r < n - 1; ++r) {
-      if (tid < h) {
-        int p = tour_player(tid, r, n), q = tour_player(n - 1 - tid, r, n);
+    for (int r = 0; r < NP - 1; ++r) {
+      if (tid < HP) {
+        int p = tour_player(tid, r), q = tour_player(NP - 1 - tid, r);
         if (p > q) { const int t = p; p = q; q = t; }
         const float app = A[p * kLd + p], aqq = A[q * kLd + q], apq = A[p * kLd + q];
         double c = 1.0, s = 0.0;
@@ -74,18 +86,22 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
           rotated = 1;
         }
         csd[tid] = c;
-        csd[kMaxN / 2 + tid] = s;
+        csd[HP + tid] = s;
         cs[tid] = (float)c;
-        cs[kMaxN / 2 + tid] = (float)s;
+        cs[HP + tid] = (float)s;
         pq[tid] = p;
-        pq[kMaxN / 2 + tid] = q;
+        pq[HP + tid] = q;
       }
       __syncthreads();
-      // A <- J^T A J over all 2x2 blocks of pairs (disjoint, so in place).
-      for (int blk = tid; blk < h * h; blk += nt) {
-        const int a = blk / h, b = blk % h;
-        const int pa = pq[a], qa = pq[kMaxN / 2 + a], pb = pq[b], qb = pq[kMaxN / 2 + b];
-        const float ca = cs[a], sa = cs[kMaxN / 2 + a], cb = cs[b], sb = cs[kMaxN / 2 + b];
+      // A <- J^T A J over the 2x2 blocks (a, b), a <= b, of pairs (disjoint, so in place);
+      // block (b, a) is the transpose and is written by the same thread.
+#pragma unroll 2
+      for (int j = 0; j < HP * HP / 512; ++j) {
+        const int blk = tid + 512 * j;
+        const int a = blk >> 6, b = blk & (HP - 1);
+        if (a > b) continue;
+        const int pa = pq[a], qa = pq[HP + a], pb = pq[b], qb = pq[HP + b];
+        const float ca = cs[a], sa = cs[HP + a], cb = cs[b], sb = cs[HP + b];
         const float a00 = A[pa * kLd + pb], a01 = A[pa * kLd + qb];
         const float a10 = A[qa * kLd + pb], a11 = A[qa * kLd + qb];
         const float t00 = cb * a00 - sb * a01, t01 = sb * a00 + cb * a01;
@@ -97,12 +113,20 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
         A[pa * kLd + qb] = n01;
         A[qa * kLd + pb] = n10;
         A[qa * kLd + qb] = n11;
+        if (a != b) {
+          A[pb * kLd + pa] = n00;
+          A[qb * kLd + pa] = n01;
+          A[pb * kLd + qa] = n10;
+          A[qb * kLd + qa] = n11;
+        }
       }
-      // V <- V J
-      for (int idx = tid; idx < n * h; idx += nt) {
-        const int i = idx / h, k = idx % h;
-        const int p = pq[k], q = pq[kMaxN / 2 + k];
-        const double c = csd[k], s = csd[kMaxN / 2 + k];
+      // V <- V J; a warp walks one column pair down 32 consecutive rows
+#pragma unroll 4
+      for (int j = 0; j < NP * HP / 512; ++j) {
+        const int idx = tid + 512 * j;
+        const int k = idx >> 7, i = idx & (NP - 1);
+        const int p = pq[k], q = pq[HP + k];
+        const double c = csd[k], s = csd[HP + k];
         const double vp = V[i * kLd + p], vq = V[i * kLd + q];
         V[i * kLd + p] = c * vp - s * vq;
         V[i * kLd + q] = s * vp + c * vq;
@@ -113,11 +137,11 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
     __syncthreads();
   }
   if (sweep == max_sweeps && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
-  // Descending order; equal eigenvalues keep index order.
-  for (int i = tid; i < n; i += nt) {
+  // Descending order; equal eigenvalues keep index order (padding sorts last).
+  for (int i = tid; i < NP; i += 512) {
     const float li = A[i * kLd + i];
     int rk = 0;
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < NP; ++j) {
       const float lj = A[j * kLd + j];
       rk += (lj > li) || (lj == li && j < i);
     }
@@ -125,76 +149,82 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
   }
   __syncthreads();
   float* vo = Vout + (int64_t)blockIdx.x * sV;
-  for (int e = tid; e < n * n; e += nt) {
+  for (int e = tid; e < n * n; e += 512) {
     const int r = e / n, c = e % n;     // eigenvector c, component r
     vo[r * n + rank[c]] = (float)V[r * kLd + c];
   }
   if (lam)
-    for (int i = tid; i < n; i += nt) lam[(int64_t)blockIdx.x * sL + rank[i]] = A[i * kLd + i];
+    for (int i = tid; i < n; i += 512) lam[(int64_t)blockIdx.x * sL + rank[i]] = A[i * kLd + i];
 }
 
-// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (upper triangular R), float64 in
-// shared memory (one n x (n+1) array, the inverse overwrites the factor in place). A
-// non-positive pivot is raised to a tiny floor and flags ST_NOT_CONVERGED.
-__global__ void __launch_bounds__(256) k_chol_inv(int n, const double* W, int64_t sW, double* Rinv,
+// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
+// R and its inverse are kept as packed upper triangles in shared memory (n (n + 1) / 2 each).
+// Cholesky: right-looking, 3 barriers per pivot. Inverse: thread c back-substitutes column c
+// (R x = e_c), reading its own earlier entries of X. A non-positive pivot is raised to a tiny
+// floor and flags ST_NOT_CONVERGED.
+__device__ __forceinline__ int pk(int i, int k, int n) { return i * n - (i * (i - 1)) / 2 + (k - i); }
+
+__global__ void __launch_bounds__(512) k_chol_inv(int n, const double* W, int64_t sW, double* Rinv,
                                                   int64_t sR, double shift, int32_t* status) {
   extern __shared__ double dm[];
-  const int ld = n + 1;
-  double* R = dm;              // n x ld
-  double* x = R + n * ld;      // n
+  const int np = n * (n + 1) / 2;
+  double* R = dm;              // packed upper triangle of the factor
+  double* X = R + np;          // packed upper triangle of the inverse
   __shared__ double tr_s;
   const int tid = threadIdx.x, nt = blockDim.x;
   const double* w = W + (int64_t)blockIdx.x * sW;
-  for (int i = tid; i < n * n; i += nt) R[(i / n) * ld + (i % n)] = w[i];
+  for (int e = tid; e < n * n; e += nt) {
+    const int i = e / n, k = e % n;
+    if (k >= i) R[pk(i, k, n)] = w[e];
+  }
   __syncthreads();
   if (tid == 0) {
     double t = 0.0;
-    for (int i = 0; i < n; ++i) t += R[i * ld + i];
+    for (int i = 0; i < n; ++i) t += R[pk(i, i, n)];
     tr_s = t;
   }
   __syncthreads();
   const double add = shift * tr_s / n;
-  for (int i = tid; i < n; i += nt) R[i * ld + i] += add;
+  for (int i = tid; i < n; i += nt) R[pk(i, i, n)] += add;
   __syncthreads();
-  // Right-looking Cholesky, W = R^T R, R upper triangular (kept in the upper triangle).
   for (int k = 0; k < n; ++k) {
     if (tid == 0) {
-      double d = R[k * ld + k];
+      double d = R[pk(k, k, n)];
       const double floor_v = 1e-30 + 1e-14 * (tr_s > 0 ? tr_s / n : 1.0);
       if (!(d > floor_v)) {
         d = floor_v;
         if (status) atomicOr(status, ST_NOT_CONVERGED);
       }
-      R[k * ld + k] = sqrt(d);
+      R[pk(k, k, n)] = sqrt(d);
     }
     __syncthreads();
-    const double rkk = R[k * ld + k];
-    for (int j = k + 1 + tid; j < n; j += nt) R[k * ld + j] /= rkk;
+    const double rkk = R[pk(k, k, n)];
+    for (int j = k + 1 + tid; j < n; j += nt) R[pk(k, j, n)] /= rkk;
     __syncthreads();
-    for (int idx = tid; idx < (n - k - 1) * (n - k - 1); idx += nt) {
-      const int i = k + 1 + idx / (n - k - 1), j = k + 1 + idx % (n - k - 1);
-      if (j >= i) R[i * ld + j] -= R[k * ld + i] * R[k * ld + j];
+    const int m = n - k - 1;
+    for (int e = tid; e < m * m; e += nt) {
+      const int i = k + 1 + e / m, j = k + 1 + e % m;
+      if (j >= i) R[pk(i, j, n)] -= R[pk(k, i, n)] * R[pk(k, j, n)];
     }
     __syncthreads();
   }
-  // In-place inverse of the upper triangle, column by column: with the leading j x j block
-  // already inverted, column j above the diagonal is -R^{-1}_jj * (R^{-1}_{0:j,0:j} R_{0:j,j}).
-  for (int j = 0; j < n; ++j) {
-    const double inv_jj = 1.0 / R[j * ld + j];
-    for (int i = tid; i < j; i += nt) {
-      double v = 0.0;
-      for (int k = i; k < j; ++k) v += R[i * ld + k] * R[k * ld + j];
-      x[i] = v;
+  for (int c = tid; c < n; c += nt) {
+    for (int i = c; i >= 0; --i) {
+      double v0 = (i == c) ? 1.0 : 0.0, v1 = 0.0;
+      int k = i + 1;
+      for (; k + 1 <= c; k += 2) {
+        v0 -= R[pk(i, k, n)] * X[pk(k, c, n)];
+        v1 -= R[pk(i, k + 1, n)] * X[pk(k + 1, c, n)];
+      }
+      if (k <= c) v0 -= R[pk(i, k, n)] * X[pk(k, c, n)];
+      X[pk(i, c, n)] = (v0 + v1) / R[pk(i, i, n)];
     }
-    __syncthreads();
-    for (int i = tid; i < j; i += nt) R[i * ld + j] = -inv_jj * x[i];
-    if (tid == 0) R[j * ld + j] = inv_jj;
-    __syncthreads();
   }
+  __syncthreads();
   double* o = Rinv + (int64_t)blockIdx.x * sR;
-  for (int i = tid; i < n * n; i += nt) {
-    const int r = i / n, c = i % n;
-    o[i] = (c >= r) ? R[r * ld + c] : 0.0;
+  for (int e = tid; e < n * n; e += nt) {
+    const int r = e / n, c = e % n;
+    o[e] = (c >= r) ? X[pk(r, c, n)] : 0.0;
   }
 }
 
@@ -202,7 +232,7 @@ __global__ void __launch_bounds__(256) k_chol_inv(int n, const double* W, int64_
 
 cudaError_t jacobi_eig(int batch, int n, const float* A, int64_t sA, float* V, int64_t sV,
                        float* lam, int64_t sL, int max_sweeps, int32_t* status, cudaStream_t s) {
-  if (n <= 0 || n > kMaxN || (n & 1)) return cudaErrorInvalidValue;
+  if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
   if (batch <= 0) return cudaSuccess;
   const size_t smem = ((size_t)kMaxN * kLd + kMaxN) * sizeof(double) +
                       ((size_t)kMaxN * kLd + kMaxN) * sizeof(float) + 2 * kMaxN * sizeof(int);
@@ -218,11 +248,11 @@ cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv
                      double shift, int32_t* status, cudaStream_t s) {
   if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
   if (batch <= 0) return cudaSuccess;
-  const size_t smem = ((size_t)n * (n + 1) + n) * sizeof(double);
+  const size_t smem = (size_t)n * (n + 1) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_chol_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  k_chol_inv<<<batch, 256, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
+  k_chol_inv<<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
   note_launch();
   return cudaGetLastError();
 }

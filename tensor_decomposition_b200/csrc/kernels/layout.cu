@@ -1,0 +1,87 @@
+// Layout helpers for the tensor-core path of the factor analysis:
+//  * the token-contiguous copy X^T[lt][h][d][t] of every layer-tensor, so that contractions
+//    over tokens read K-major tiles (the JoLT token unfolding, "A JoLT for the KV Cache",
+//    arXiv 2607.12550v2, Abstract, is contracted over tokens for the sketch passes A^T Q and
+//    Q^T A and for the feature Gram);
+//  * splitting a float32 array into up to three bf16 parts (x = p0 + p1 + p2 to ~2^-24);
+//  * summing per-head float32 Gram partials in float64.
+#include "../jolt_internal.h"
+
+namespace jolt {
+namespace {
+
+// One 32 x 32 tile of X[l][h] (T x D) -> X^T[base + l][h] (D x T).
+__global__ void k_transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int H, int T, int D, int lt_base) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int lh = blockIdx.z;                   // l * H + h within this kind
+  const int t0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
+  const __nv_bfloat16* src = X + (int64_t)lh * T * D;
+  const int l = lh / H, h = lh % H;
+  __nv_bfloat16* dst = XT + ((int64_t)(lt_base + l) * H + h) * D * T;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+  for (int r = ty; r < 32; r += 8) {
+    const int t = t0 + r, d = d0 + tx;
+    if (t < T && d < D) tile[r][tx] = src[(int64_t)t * D + d];
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int d = d0 + r, t = t0 + tx;
+    if (t < T && d < D) dst[(int64_t)d * T + t] = tile[tx][r];
+  }
+}
+
+__global__ void k_split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1,
+                             __nv_bfloat16* p2) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = x[i];
+    const __nv_bfloat16 a = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(a);
+    const __nv_bfloat16 b = __float2bfloat16_rn(r1);
+    p0[i] = a;
+    if (p1) p1[i] = b;
+    if (p2) p2[i] = __float2bfloat16_rn(r1 - __bfloat162float(b));
+  }
+}
+
+// out[i][e] = sum_h part[i][h][e] in float64 (fixed order), stored as float32 and float64.
+__global__ void k_sum_heads(int n, int H, int64_t per, const float* part, float* out32, double* out64) {
+  const int64_t total = (int64_t)n * per;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / per, r = e % per;
+    double s = 0.0;
+    for (int h = 0; h < H; ++h) s += (double)part[(i * H + h) * per + r];
+    if (out32) out32[e] = (float)s;
+    if (out64) out64[e] = s;
+  }
+}
+
+int grid_for(int64_t n) {
+  int64_t b = (n + 255) / 256;
+  if (b > 4096) b = 4096;
+  return (int)(b < 1 ? 1 : b);
+}
+
+}  // namespace
+
+cudaError_t transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int L, int H, int T, int D, int lt_base,
+                        cudaStream_t s) {
+  const dim3 g((T + 31) / 32, (D + 31) / 32, L * H);
+  k_transpose_x<<<g, 256, 0, s>>>(X, XT, H, T, D, lt_base);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2,
+                       cudaStream_t s) {
+  k_split_bf16<<<grid_for(n), 256, 0, s>>>(n, x, p0, p1, p2);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t sum_heads(int n, int H, int64_t per, const float* part, float* out32, double* out64, cudaStream_t s) {
+  k_sum_heads<<<grid_for((int64_t)n * per), 256, 0, s>>>(n, H, per, part, out32, out64);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace jolt

@@ -49,13 +49,18 @@ struct OmegaKeys {
   uint64_t key[kMaxLT];
 };
 
-__global__ void k_sketch_omega(OmegaKeys keys, int64_t per, __nv_bfloat16* out) {
+// Omega element (i, j) is normal number i * l + j of the layer-tensor's stream.
+__global__ void k_sketch_omega(OmegaKeys keys, int64_t HD, int l, int transposed, __nv_bfloat16* out) {
   const int lt = blockIdx.y;
   const uint64_t key = keys.key[lt];
+  const int64_t per = HD * l;
   __nv_bfloat16* o = out + (int64_t)lt * per;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < per;
-       i += (int64_t)gridDim.x * blockDim.x)
-    o[i] = __double2bfloat16(normal_at(key, (uint64_t)i));
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < per;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    // transposed: output index e = j * HD + i holds element (i, j); writes stay contiguous
+    const uint64_t n = transposed ? (uint64_t)((e % HD) * l + e / HD) : (uint64_t)e;
+    o[e] = __double2bfloat16(normal_at(key, n));
+  }
 }
 
 // One CTA: Householder QR of G (D x D, float64, in shared memory), Q formed in place by
@@ -165,7 +170,7 @@ cudaError_t gauss_f64(uint64_t seed, uint64_t stream_id, int64_t n, double* out,
 }
 
 cudaError_t sketch_omega(uint64_t seed, const int32_t* lt_ids, int n_lt, int64_t HD, int l,
-                         __nv_bfloat16* out, cudaStream_t s) {
+                         __nv_bfloat16* out, bool transposed, cudaStream_t s) {
   if (n_lt > kMaxLT) return cudaErrorInvalidValue;
   OmegaKeys keys;
   for (int i = 0; i < n_lt; ++i)
@@ -173,7 +178,7 @@ cudaError_t sketch_omega(uint64_t seed, const int32_t* lt_ids, int n_lt, int64_t
   const int64_t per = HD * l;
   int bx = (int)((per + 255) / 256);
   if (bx > 64) bx = 64;
-  k_sketch_omega<<<dim3(bx, n_lt), 256, 0, s>>>(keys, per, out);
+  k_sketch_omega<<<dim3(bx, n_lt), 256, 0, s>>>(keys, HD, l, transposed ? 1 : 0, out);
   note_launch();
   return cudaGetLastError();
 }

@@ -29,7 +29,7 @@ EXPORTED = ["jolt_config_default", "jolt_plan", "jolt_plan_info", "jolt_encode",
             "jolt_rel_frob_error", "jolt_stream_status", "jolt_stream_info", "jolt_stream_to_host",
             "jolt_stream_from_host", "jolt_export_debug", "jolt_stream_destroy",
             "jolt_plan_destroy", "jolt_last_error", "jolt_profile_enable", "jolt_profile_report",
-            "jolt_launch_count"]
+            "jolt_launch_count", "jolt_selftest_gemm_bf16"]
 
 
 class JoltError(RuntimeError):
@@ -74,6 +74,7 @@ def _load():
         "jolt_profile_enable": (st, [i32]),
         "jolt_profile_report": (st, [ctypes.c_char_p, ctypes.POINTER(u64)]),
         "jolt_launch_count": (u64, []),
+        "jolt_selftest_gemm_bf16": (st, [i32, i32, i32, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -233,3 +234,10 @@ def jolt_profile_report() -> dict:
 
 def jolt_launch_count() -> int:
     return int(_lib.jolt_launch_count())
+
+
+def jolt_selftest_gemm_bf16(A, B, C, cuda_stream=None):
+    """C = A B^T on the tensor cores; A [M][K], B [N][K] bf16, C [M][N] float32 (CUDA tensors)."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check(_lib.jolt_selftest_gemm_bf16(M, N, K, _dptr(A), _dptr(B), _dptr(C), _stream_ptr(cuda_stream)))

@@ -236,3 +236,19 @@ def test_corrupt_stream_rejected(J):
     with pytest.raises(J.JoltError) as e:
         J.jolt_stream_from_host(bytes(buf))
     assert e.value.status == 8
+
+
+# ------------------------------------------------------------------ tensor-core GEMM building block
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (200, 136, 200), (256, 128, 1024), (384, 256, 72)])
+def test_tcgen05_gemm_matches_float64(J, M, N, K):
+    import torch
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K)
+    A = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    B = torch.randn((N, K), generator=g, device="cuda").to(torch.bfloat16)
+    C = torch.full((M, N), float("nan"), device="cuda", dtype=torch.float32)
+    J.jolt_selftest_gemm_bf16(A, B, C)
+    ref = (A.double() @ B.double().T)
+    err = (C.double() - ref).abs().max().item()
+    scale = (A.double().abs() @ B.double().abs().T).max().item()
+    assert torch.isfinite(C).all()
+    assert err <= 1e-5 * scale, (err, scale)
