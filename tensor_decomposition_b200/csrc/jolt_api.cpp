@@ -173,11 +173,13 @@ struct jolt_plan_s {
   size_t ws_bytes = 0;
   // workspace views
   double *xx = nullptr, *xx_part = nullptr;
-  float *CD = nullptr, *UD32 = nullptr, *UDf = nullptr, *lamD = nullptr;
+  double* CD = nullptr;      // feature Grams, float64
+  float *UD32 = nullptr, *UDf = nullptr, *lamD = nullptr;
   __nv_bfloat16 *UDb = nullptr, *Om = nullptr, *UTb = nullptr;
-  float *Y = nullptr, *Y2 = nullptr, *Z = nullptr, *Z2 = nullptr, *Bm = nullptr, *BB = nullptr,
+  float *Y = nullptr, *Y2 = nullptr, *Z = nullptr, *Z2 = nullptr, *Bm = nullptr,
         *Wv = nullptr, *lamB = nullptr, *UT32 = nullptr, *UTf = nullptr, *P = nullptr, *Gmax = nullptr,
-        *CT = nullptr, *VT = nullptr, *lamT = nullptr;
+        *VT = nullptr, *lamT = nullptr;
+  double *BB = nullptr, *CT = nullptr;   // sketch and token Grams, float64
   double *Wg = nullptr, *Rinv = nullptr, *E = nullptr, *unit_err = nullptr, *Nbuf = nullptr;
   float* Qfinal = nullptr;   // final sketch basis (one of Y / Y2)
   bool q_t = false;          // Qfinal stored as Q^T [l][T] (tensor-core path) instead of Q [T][l]
@@ -575,18 +577,18 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
     g.C = p->Cpart; g.c_sm = D; g.c_sn = 1; g.c_sb = (int64_t)D * D;
     g.status = status;
     CK(gemm_tc(n * H, g, s));
-    CK(sum_heads(n, H, (int64_t)D * D, p->Cpart, p->CD, nullptr, s));
+    CK(sum_heads(n, H, (int64_t)D * D, p->Cpart, nullptr, p->CD, s));
   } else {
     PROF("feature_gram", s);
     // C_D = sum over rows r = (h, t) of X[r, :]^T X[r, :]
     for (int k = 0; k < kinds; ++k)
       CK(gemm_simt(L, D, D, H * T, opnd(X[k], xt, I1(HTD), I1(1), I1(D)), opnd(X[k], xt, I1(HTD), I1(1), I1(D)),
-                   outd(p->CD + (int64_t)k * L * D * D, EL_F32, I1((int64_t)D * D), I1(D), I1(1)), 1.0, 0.0, s));
+                   outd(p->CD + (int64_t)k * L * D * D, EL_F64, I1((int64_t)D * D), I1(D), I1(1)), 1.0, 0.0, s));
   }
   {
     PROF("jacobi_feature", s);
-    CK(jacobi_eig(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, p->cfg.max_jacobi_sweeps,
-                  status, s));
+    CK(eig_psd(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, p->cfg.max_jacobi_sweeps,
+               status, s));
   }
   {
     PROF("sign_round", s);
@@ -764,12 +766,12 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         // B B^T
         CK(gemm_simt(n, l, l, (int)HD, opnd(p->Bm, EL_F32, I1(l * HD), I1(HD), I1(1)),
                      opnd(p->Bm, EL_F32, I1(l * HD), I1(HD), I1(1)),
-                     outd(p->BB, EL_F32, I1((int64_t)l * l), I1(l), I1(1)), 1.0, 0.0, s));
+                     outd(p->BB, EL_F64, I1((int64_t)l * l), I1(l), I1(1)), 1.0, 0.0, s));
       }
       {
         PROF("jacobi_sketch", s);
-        CK(jacobi_eig(n, l, p->BB, (int64_t)l * l, p->Wv, (int64_t)l * l, p->lamB, l, p->cfg.max_jacobi_sweeps,
-                      status, s));
+        CK(eig_psd(n, l, p->BB, (int64_t)l * l, p->Wv, (int64_t)l * l, p->lamB, l, p->cfg.max_jacobi_sweeps,
+                   status, s));
       }
       {
         PROF("small_gemm", s);
@@ -798,12 +800,12 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         for (int k = 0; k < kinds; ++k)
           CK(gemm_simt(L, T, T, (int)HD, opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
                        opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
-                       outd(p->CT + (int64_t)k * L * T * T, EL_F32, I1((int64_t)T * T), I1(T), I1(1)), 1.0, 0.0, s));
+                       outd(p->CT + (int64_t)k * L * T * T, EL_F64, I1((int64_t)T * T), I1(T), I1(1)), 1.0, 0.0, s));
       }
       {
         PROF("jacobi_token", s);
-        CK(jacobi_eig(n, T, p->CT, (int64_t)T * T, p->VT, (int64_t)T * T, p->lamT, T, p->cfg.max_jacobi_sweeps,
-                      status, s));
+        CK(eig_psd(n, T, p->CT, (int64_t)T * T, p->VT, (int64_t)T * T, p->lamT, T, p->cfg.max_jacobi_sweeps,
+                   status, s));
       }
       {
         PROF("sign_round", s);

@@ -74,6 +74,10 @@ cudaError_t haar_from_gauss(const double* G, int D, float* Pi_f32, __nv_bfloat16
 // descending. Sets ST_NOT_CONVERGED in *status when max_sweeps is reached.
 cudaError_t jacobi_eig(int batch, int n, const float* A, int64_t sA, float* V, int64_t sV,
                        float* lam, int64_t sL, int max_sweeps, int32_t* status, cudaStream_t s);
+// Eigenpairs of PSD matrices (n <= 128, float64 input) by one-sided Jacobi on a Cholesky
+// factor; same output convention as jacobi_eig.
+cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int64_t sV, float* lam, int64_t sL,
+                    int max_sweeps, int32_t* status, cudaStream_t s);
 // Shifted-CholeskyQR helper: Rinv = inverse of chol(W + shift * trace(W)/n * I), W n x n.
 cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv, int64_t sR,
                      double shift, int32_t* status, cudaStream_t s);

@@ -85,33 +85,11 @@ __device__ __forceinline__ void grid_rank(int gi, int step, int D, int& rt, int&
 
 constexpr int kMaxUnits = 2 * kMaxGroups;
 
-// Single CTA of 1024 threads: warp w evaluates units w, w + 32, ... The candidates' bytes per
-// layer and, when they fit, the pool's error tables are staged in shared memory.
-constexpr size_t kDualSmem = 160 * 1024;
-
-__global__ void __launch_bounds__(1024) k_dual(DualArgs a) {
-  extern __shared__ unsigned char dsm[];
-  __shared__ int nlay[kMaxGroups];
-  __shared__ int choice[kMaxUnits];
-  __shared__ int64_t cbytes[kMaxUnits];
-  __shared__ Cand wbest[32];
-  __shared__ int wunit[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nu = a.G * 2;
+// Unit tables: err[u][b][grid] = (sum over the group's layers, in increasing layer order, of
+// E_lt[grid]) * phi(b), for u = 2 g + kind.
+__global__ void k_unit_tables(DualArgs a) {
   const int ncand = a.nbits * a.ngrid;
-  StreamMeta* meta = a.meta;
-  int64_t* cand_bytes = reinterpret_cast<int64_t*>(dsm);           // per layer, [ncand]
-  double* err_s = reinterpret_cast<double*>(cand_bytes + ncand);    // [units of pool][ncand]
-  const size_t err_cap = (kDualSmem - (size_t)ncand * 8) / 8;
-  for (int g = tid; g < a.G; g += blockDim.x)
-    nlay[g] = (int)(((int64_t)(g + 1) * a.L) / a.G - ((int64_t)g * a.L) / a.G);
-  for (int c = tid; c < ncand; c += blockDim.x) {
-    int rt, rd;
-    grid_rank(c % a.ngrid, a.step, a.D, rt, rd);
-    cand_bytes[c] = lt_bytes(a.H, a.T, a.D, rt, rd, a.bits[c / a.ngrid]);
-  }
-  // Unit tables: E summed over the group's layers in increasing layer order, times phi(b).
-  for (int e = tid; e < nu * a.ngrid; e += blockDim.x) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < a.G * 2 * a.ngrid; e += gridDim.x * blockDim.x) {
     const int u = e / a.ngrid, gi = e % a.ngrid;
     const int g = u / 2, k = u % 2;
     if (k == 1 && !a.has_v) continue;
@@ -121,169 +99,178 @@ __global__ void __launch_bounds__(1024) k_dual(DualArgs a) {
     for (int bi = 0; bi < a.nbits; ++bi)
       a.unit_err[(int64_t)u * ncand + bi * a.ngrid + gi] = __dmul_rn(s, a.phi[bi]);
   }
-  __threadfence_block();
-  __syncthreads();
+}
+
+constexpr size_t kDualSmem = 160 * 1024;
+
+// One CTA per budget pool, one warp per unit of the pool (units beyond the warp count are
+// taken in turn). A bisection step costs one barrier: every warp writes its unit's choice into
+// one of two alternating buffers, then all threads sum the bytes and move lo / hi identically.
+__global__ void __launch_bounds__(1024) k_dual_pool(DualArgs a) {
+  extern __shared__ unsigned char dsm[];
+  __shared__ int slot_unit[kMaxUnits];
+  __shared__ int slot_nlay[kMaxUnits];
+  __shared__ int64_t sbytes[2][kMaxUnits];
+  __shared__ int schoice[2][kMaxUnits];
+  __shared__ int nslot_s;
+  __shared__ double esum_s;
+  const int pool = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = (int)(blockDim.x >> 5);
+  const int nu = a.G * 2;
+  const int ncand = a.nbits * a.ngrid;
   const int npools = (a.has_v && a.split) ? 2 : 1;
-  for (int pool = 0; pool < npools; ++pool) {
-    const int64_t budget = a.budget_pool[pool];
-    auto in_pool = [&](int u) -> bool {
-      const int k = u % 2;
-      if (k == 1 && !a.has_v) return false;
-      if (npools == 1) return true;
-      return k == pool;
-    };
-    // stage this pool's tables (slot = rank of u among the pool's units)
-    int nslot = 0;
-    for (int u = 0; u < nu; ++u) nslot += in_pool(u);
-    const bool cached = (size_t)nslot * ncand <= err_cap;
-    if (cached) {
-      for (int e = tid; e < nslot * ncand; e += blockDim.x) {
-        const int slot = e / ncand, c = e % ncand;
-        int u = -1;
-        for (int v = 0, seen = 0; v < nu; ++v)
-          if (in_pool(v)) { if (seen == slot) { u = v; break; } ++seen; }
-        err_s[e] = a.unit_err[(int64_t)u * ncand + c];
-      }
-    }
-    __syncthreads();
-    // choose(lam) for every unit of the pool; writes choice[] and cbytes[], returns total bytes.
-    // Units get 32 / nslot warps each (at least one); each warp scans a strided share of the
-    // candidates, then one thread per unit merges its warps' bests in warp order.
-    const int nwarps = (int)(blockDim.x >> 5);
-    const int wpu = nslot >= nwarps ? 1 : nwarps / nslot;
-    auto choose_all = [&](double lam, bool min_bytes_only) {
-      for (int base = 0; base < nslot; base += nwarps / wpu) {
-        const int us = base + warp % (nwarps / wpu);          // unit slot of this warp
-        const int part = warp / (nwarps / wpu);
-        Cand best;
-        best.cost = 0.0;
-        best.idx = -1;
-        int u = -1;
-        if (us < nslot && part < wpu) {
-          for (int v = 0, seen = 0; v < nu; ++v)
-            if (in_pool(v)) { if (seen == us) { u = v; break; } ++seen; }
-          const int g = u / 2;
-          const double* errp = cached ? err_s + (size_t)us * ncand : a.unit_err + (int64_t)u * ncand;
-          for (int c = part * 32 + lane; c < ncand; c += 32 * wpu) {
-            Cand x;
-            grid_rank(c % a.ngrid, a.step, a.D, x.rt, x.rd);
-            x.b = a.bits[c / a.ngrid];
-            x.bytes = (int64_t)nlay[g] * cand_bytes[c];
-            x.cost = min_bytes_only ? 0.0 : __dadd_rn(errp[c], __dmul_rn(lam, (double)x.bytes));
-            x.idx = c;
-            if (best.idx < 0 || less_key(x, best)) best = x;
-          }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          Cand y;
-          y.cost = __shfl_down_sync(0xffffffffu, best.cost, o);
-          y.bytes = __shfl_down_sync(0xffffffffu, best.bytes, o);
-          y.b = __shfl_down_sync(0xffffffffu, best.b, o);
-          y.rt = __shfl_down_sync(0xffffffffu, best.rt, o);
-          y.rd = __shfl_down_sync(0xffffffffu, best.rd, o);
-          y.idx = __shfl_down_sync(0xffffffffu, best.idx, o);
-          if (y.idx >= 0 && (best.idx < 0 || less_key(y, best))) best = y;
-        }
-        if (lane == 0) {
-          wbest[warp] = best;
-          wunit[warp] = u;
-        }
-        __syncthreads();
-        if (tid < nwarps / wpu && base + tid < nslot) {
-          Cand m;
-          m.idx = -1;
-          int uu = -1;
-          for (int pp = 0; pp < wpu; ++pp) {
-            const int w = pp * (nwarps / wpu) + tid;
-            const Cand y = wbest[w];
-            if (wunit[w] >= 0) uu = wunit[w];
-            if (y.idx >= 0 && (m.idx < 0 || less_key(y, m))) m = y;
-          }
-          if (uu >= 0) {
-            choice[uu] = m.idx;
-            cbytes[uu] = m.bytes;
-          }
-        }
-        __syncthreads();
-      }
-      int64_t tb = 0;
-      for (int u = 0; u < nu; ++u)
-        if (in_pool(u)) tb += cbytes[u];
-      __syncthreads();
-      return tb;
-    };
-    const int64_t minb = choose_all(0.0, true);
-    double lam = 0.0;
-    if (minb > budget) {
-      if (tid == 0) atomicOr(&meta->status, ST_INFEASIBLE);
-    } else {
-      int64_t tb = choose_all(0.0, false);
-      if (tb > budget) {
-        // sum of the pool's unit energies E(0, 0), each summed over its layers in order
-        double esum = 0.0;
-        for (int u = 0; u < nu; ++u) {
-          if (!in_pool(u)) continue;
-          const int g = u / 2, k = u % 2;
-          const int l0 = (int)(((int64_t)g * a.L) / a.G), l1 = (int)(((int64_t)(g + 1) * a.L) / a.G);
-          double s = 0.0;
-          for (int l = l0; l < l1; ++l) s = __dadd_rn(s, a.E[(int64_t)(2 * l + k) * a.ngrid]);
-          esum = __dadd_rn(esum, s);
-        }
-        const double scale = __ddiv_rn(esum, (double)budget);
-        double lo = __dmul_rn(1e-30, scale), hi = __dmul_rn(1e30, scale);
-        for (int it = 0; it < 200; ++it) {
-          if (!(__ddiv_rn(hi, lo) > 1.0 + 1e-15)) break;
-          const double mid = __dsqrt_rn(__dmul_rn(lo, hi));
-          const int64_t t = choose_all(mid, false);
-          if (t <= budget) hi = mid;
-          else lo = mid;
-        }
-        lam = hi;
-        choose_all(hi, false);
-      }
-    }
-    if (tid == 0) {
-      meta->lambda[pool] = lam;
-      for (int u = 0; u < nu; ++u) {
-        if (!in_pool(u)) continue;
-        const int c = choice[u];
-        const int bi = c / a.ngrid, gi = c % a.ngrid;
-        int rt, rd;
-        grid_rank(gi, a.step, a.D, rt, rd);
-        meta->alloc[u / 2][u % 2][0] = rt;
-        meta->alloc[u / 2][u % 2][1] = rd;
-        meta->alloc[u / 2][u % 2][2] = a.bits[bi];
-      }
-    }
-    __syncthreads();
-  }
-  // Layout of the body: lt-major, parts U_T, U_D, G, scales, codes, each 256-aligned.
+  StreamMeta* meta = a.meta;
+  int64_t* cbytes = reinterpret_cast<int64_t*>(dsm);                 // bytes per layer [ncand]
+  int* cattr = reinterpret_cast<int*>(cbytes + ncand);               // b | rt << 8 | rd << 20
+  double* err_s = reinterpret_cast<double*>(cattr + ((ncand + 1) & ~1));
   if (tid == 0) {
-    int64_t cur = 0;
-    int64_t bp[JOLT_NUM_PARTS] = {0, 0, 0, 0, 0};
-    for (int l = 0; l < a.L; ++l) {
-      int g = 0;
-      while (g + 1 < a.G && ((int64_t)(g + 1) * a.L) / a.G <= l) ++g;
-      for (int k = 0; k < (a.has_v ? 2 : 1); ++k) {
-        const int lt = 2 * l + k;
-        const int rt = meta->alloc[g][k][0], rd = meta->alloc[g][k][1], b = meta->alloc[g][k][2];
-        meta->lt_rank[lt][0] = rt;
-        meta->lt_rank[lt][1] = rd;
-        meta->lt_rank[lt][2] = b;
-        const int64_t sz[JOLT_NUM_PARTS] = {
-            (int64_t)a.T * rt * 2, (int64_t)a.D * rd * 2, (int64_t)a.H * rt * rd * 2,
-            b > 0 ? (int64_t)a.H * a.T * 2 : 0, b > 0 ? (int64_t)a.H * a.T * (a.D * b / 8) : 0};
-        for (int p = 0; p < JOLT_NUM_PARTS; ++p) {
-          const int64_t off = (cur + kAlign - 1) / kAlign * kAlign;
-          meta->off[lt][p] = off;
-          cur = off + sz[p];
-          bp[p] += sz[p];
-        }
+    int ns = 0;
+    for (int u = 0; u < nu; ++u) {
+      const int k = u % 2;
+      if (k == 1 && !a.has_v) continue;
+      if (npools == 2 && k != pool) continue;
+      slot_unit[ns] = u;
+      const int g = u / 2;
+      slot_nlay[ns] = (int)(((int64_t)(g + 1) * a.L) / a.G - ((int64_t)g * a.L) / a.G);
+      ++ns;
+    }
+    nslot_s = ns;
+    // sum of the pool's unit energies E(0, 0), each summed over its layers in order
+    double esum = 0.0;
+    for (int i = 0; i < ns; ++i) {
+      const int u = slot_unit[i], g = u / 2, k = u % 2;
+      const int l0 = (int)(((int64_t)g * a.L) / a.G), l1 = (int)(((int64_t)(g + 1) * a.L) / a.G);
+      double s = 0.0;
+      for (int l = l0; l < l1; ++l) s = __dadd_rn(s, a.E[(int64_t)(2 * l + k) * a.ngrid]);
+      esum = __dadd_rn(esum, s);
+    }
+    esum_s = esum;
+  }
+  for (int c = tid; c < ncand; c += blockDim.x) {
+    int rt, rd;
+    grid_rank(c % a.ngrid, a.step, a.D, rt, rd);
+    const int b = a.bits[c / a.ngrid];
+    cbytes[c] = lt_bytes(a.H, a.T, a.D, rt, rd, b);
+    cattr[c] = b | (rt << 8) | (rd << 20);
+  }
+  __syncthreads();
+  const int nslot = nslot_s;
+  const size_t err_cap = (kDualSmem - (size_t)ncand * 12 - 16) / 8;
+  const bool cached = (size_t)nslot * ncand <= err_cap;
+  if (cached)
+    for (int e = tid; e < nslot * ncand; e += blockDim.x)
+      err_s[e] = a.unit_err[(int64_t)slot_unit[e / ncand] * ncand + e % ncand];
+  __syncthreads();
+  const int64_t budget = a.budget_pool[pool];
+  // choices of every slot at lam into buffer `buf`; the caller synchronises
+  auto choose = [&](double lam, bool min_bytes_only, int buf) {
+    for (int us = warp; us < nslot; us += nwarps) {
+      const double* errp = cached ? err_s + (size_t)us * ncand : a.unit_err + (int64_t)slot_unit[us] * ncand;
+      const int64_t nl = slot_nlay[us];
+      Cand best;
+      best.cost = 0.0;
+      best.idx = -1;
+      for (int c = lane; c < ncand; c += 32) {
+        Cand x;
+        const int at = cattr[c];
+        x.b = at & 0xFF;
+        x.rt = (at >> 8) & 0xFFF;
+        x.rd = at >> 20;
+        x.bytes = nl * cbytes[c];
+        x.cost = min_bytes_only ? 0.0 : __dadd_rn(errp[c], __dmul_rn(lam, (double)x.bytes));
+        x.idx = c;
+        if (best.idx < 0 || less_key(x, best)) best = x;
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        Cand y;
+        y.cost = __shfl_down_sync(0xffffffffu, best.cost, o);
+        y.bytes = __shfl_down_sync(0xffffffffu, best.bytes, o);
+        y.b = __shfl_down_sync(0xffffffffu, best.b, o);
+        y.rt = __shfl_down_sync(0xffffffffu, best.rt, o);
+        y.rd = __shfl_down_sync(0xffffffffu, best.rd, o);
+        y.idx = __shfl_down_sync(0xffffffffu, best.idx, o);
+        if (y.idx >= 0 && (best.idx < 0 || less_key(y, best))) best = y;
+      }
+      if (lane == 0) {
+        sbytes[buf][us] = best.bytes;
+        schoice[buf][us] = best.idx;
       }
     }
-    meta->body_bytes = cur;
-    for (int p = 0; p < JOLT_NUM_PARTS; ++p) meta->bytes_by_part[p] = bp[p];
+  };
+  auto total = [&](int buf) {
+    int64_t tb = 0;
+    for (int us = 0; us < nslot; ++us) tb += sbytes[buf][us];
+    return tb;
+  };
+  int buf = 0;
+  choose(0.0, true, buf);
+  __syncthreads();
+  const int64_t minb = total(buf);
+  double lam = 0.0;
+  buf ^= 1;
+  if (minb > budget) {
+    if (tid == 0) atomicOr(&meta->status, ST_INFEASIBLE);
+    buf ^= 1;   // keep the minimum-bytes choice
+  } else {
+    choose(0.0, false, buf);
+    __syncthreads();
+    if (total(buf) > budget) {
+      const double scale = __ddiv_rn(esum_s, (double)budget);
+      double lo = __dmul_rn(1e-30, scale), hi = __dmul_rn(1e30, scale);
+      for (int it = 0; it < 200; ++it) {
+        if (!(__ddiv_rn(hi, lo) > 1.0 + 1e-15)) break;
+        const double mid = __dsqrt_rn(__dmul_rn(lo, hi));
+        buf ^= 1;
+        choose(mid, false, buf);
+        __syncthreads();
+        if (total(buf) <= budget) hi = mid;
+        else lo = mid;
+      }
+      lam = hi;
+      buf ^= 1;
+      choose(hi, false, buf);
+      __syncthreads();
+    }
   }
+  if (tid == 0) {
+    meta->lambda[pool] = lam;
+    for (int us = 0; us < nslot; ++us) {
+      const int u = slot_unit[us];
+      const int at = cattr[schoice[buf][us]];
+      meta->alloc[u / 2][u % 2][0] = (at >> 8) & 0xFFF;
+      meta->alloc[u / 2][u % 2][1] = at >> 20;
+      meta->alloc[u / 2][u % 2][2] = at & 0xFF;
+    }
+  }
+}
+
+// Layout of the body: lt-major, parts U_T, U_D, G, scales, codes, each 256-aligned.
+__global__ void k_layout(DualArgs a) {
+  StreamMeta* meta = a.meta;
+  int64_t cur = 0;
+  int64_t bp[JOLT_NUM_PARTS] = {0, 0, 0, 0, 0};
+  for (int l = 0; l < a.L; ++l) {
+    int g = 0;
+    while (g + 1 < a.G && ((int64_t)(g + 1) * a.L) / a.G <= l) ++g;
+    for (int k = 0; k < (a.has_v ? 2 : 1); ++k) {
+      const int lt = 2 * l + k;
+      const int rt = meta->alloc[g][k][0], rd = meta->alloc[g][k][1], b = meta->alloc[g][k][2];
+      meta->lt_rank[lt][0] = rt;
+      meta->lt_rank[lt][1] = rd;
+      meta->lt_rank[lt][2] = b;
+      const int64_t sz[JOLT_NUM_PARTS] = {
+          (int64_t)a.T * rt * 2, (int64_t)a.D * rd * 2, (int64_t)a.H * rt * rd * 2,
+          b > 0 ? (int64_t)a.H * a.T * 2 : 0, b > 0 ? (int64_t)a.H * a.T * (a.D * b / 8) : 0};
+      for (int p = 0; p < JOLT_NUM_PARTS; ++p) {
+        const int64_t off = (cur + kAlign - 1) / kAlign * kAlign;
+        meta->off[lt][p] = off;
+        cur = off + sz[p];
+        bp[p] += sz[p];
+      }
+    }
+  }
+  meta->body_bytes = cur;
+  for (int p = 0; p < JOLT_NUM_PARTS; ++p) meta->bytes_by_part[p] = bp[p];
 }
 
 // Copy the chosen leading blocks of the factors and the bf16-rounded core into the body.
@@ -329,9 +316,17 @@ cudaError_t energy_table(const TableArgs& a, cudaStream_t s) {
 
 cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s) {
   if (a.G > kMaxGroups || a.L > kMaxL) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_dual, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
+  const int units = a.G * 2 * a.ngrid;
+  k_unit_tables<<<(units + 255) / 256, 256, 0, s>>>(a);
+  note_launch();
+  cudaError_t e = cudaFuncSetAttribute(k_dual_pool, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
   if (e != cudaSuccess) return e;
-  k_dual<<<1, 1024, kDualSmem, s>>>(a);
+  const int npools = (a.has_v && a.split) ? 2 : 1;
+  int slots = a.has_v && !a.split ? 2 * a.G : a.G;
+  int threads = 32 * (slots < 32 ? slots : 32);
+  k_dual_pool<<<npools, threads, kDualSmem, s>>>(a);
+  note_launch();
+  k_layout<<<1, 1, 0, s>>>(a);
   note_launch();
   return cudaGetLastError();
 }

@@ -157,6 +157,173 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
     for (int i = tid; i < n; i += 512) lam[(int64_t)blockIdx.x * sL + rank[i]] = A[i * kLd + i];
 }
 
+// Eigenpairs of a batch of symmetric positive semi-definite n x n matrices C (n <= 128),
+// float64 input, by one-sided (Hestenes) Jacobi on a Cholesky factor:
+//   C + sigma I = M M^T (M = R^T, R the upper Cholesky factor, sigma = 1e-13 trace / n keeps
+//   the factorisation defined; it shifts every eigenvalue by sigma and leaves the vectors);
+//   column pairs (p, q) of M are rotated, M <- M J, until all columns are mutually orthogonal;
+//   then M = U Sigma, so the normalised columns are the eigenvectors of C and the squared
+//   column norms (minus sigma) its eigenvalues. No eigenvector matrix is accumulated.
+// M lives in shared memory in float64, column-major, padded with zero rows/columns to 128.
+// Each round of the circle-method tournament rotates 64 disjoint pairs:
+// the three dot products are warp-shuffle reductions; the rotation (Golub & Van Loan sec.
+// 8.6, one-sided Jacobi) uses zeta = (beta - alpha) / (2 gamma), t = sign(zeta) /
+// (|zeta| + sqrt(1 + zeta^2)), c = 1 / sqrt(1 + t^2), s = t c, computed in float32 and
+// renormalised in float64 by one Newton step so that c^2 + s^2 = 1 to ~1e-15. A pair rotates
+// when gamma^2 > 1e-14 alpha beta; a sweep with no rotation ends the solve. Each warp works on
+// four pairs of a round at once, eight lanes per pair (16 rows each), so the dot products need
+// only three shuffle steps.
+__global__ void __launch_bounds__(512) k_eig_psd(int n, const double* Cin, int64_t sC, float* Vout, int64_t sV,
+                                                 float* lam, int64_t sL, int max_sweeps, int32_t* status) {
+  constexpr int NP = kMaxN, HP = kMaxN / 2;
+  extern __shared__ double ms[];
+  double* M = ms;                 // column-major: column j at M + j * NP (during Cholesky: row-major R)
+  double* nrm = M + NP * NP;      // NP squared column norms
+  int* rank = reinterpret_cast<int*>(nrm + NP);
+  __shared__ int rotated;
+  __shared__ double sigma_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const double* c_in = Cin + (int64_t)blockIdx.x * sC;
+  // load C (upper triangle used), zero padding
+  for (int e = tid; e < NP * NP; e += 512) {
+    const int r = e >> 7, c = e & (NP - 1);
+    M[e] = (r < n && c < n) ? c_in[(int64_t)r * n + c] : 0.0;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double tr = 0.0;
+    for (int i = 0; i < n; ++i) tr += fabs(M[i * NP + i]);
+    sigma_s = 1e-13 * (tr > 0.0 ? tr / n : 1.0);
+  }
+  __syncthreads();
+  const double sigma = sigma_s;
+  for (int i = tid; i < n; i += 512) M[i * NP + i] += sigma;
+  __syncthreads();
+  // right-looking Cholesky, upper factor R in the upper triangle (row-major)
+  for (int k = 0; k < n; ++k) {
+    if (tid == 0) {
+      const double d = M[k * NP + k];
+      M[k * NP + k] = d > sigma * 1e-3 ? sqrt(d) : sqrt(sigma * 1e-3);
+    }
+    __syncthreads();
+    const double rkk = M[k * NP + k];
+    for (int j = k + 1 + tid; j < n; j += 512) M[k * NP + j] /= rkk;
+    __syncthreads();
+    const int m = n - k - 1;
+    for (int e = tid; e < m * NP; e += 512) {
+      const int i = k + 1 + (e >> 7), j = e & (NP - 1);
+      if (j >= i && j < n) M[i * NP + j] -= M[k * NP + i] * M[k * NP + j];
+    }
+    __syncthreads();
+  }
+  // M = R^T column-major == R row-major with the strict lower part cleared
+  for (int e = tid; e < NP * NP; e += 512) {
+    const int r = e >> 7, c = e & (NP - 1);
+    if (c < r) M[e] = 0.0;
+  }
+  __syncthreads();
+  int sweep = 0;
+  for (; sweep < max_sweeps; ++sweep) {
+    if (tid == 0) rotated = 0;
+    __syncthreads();
+    int any = 0;
+    // lane = 8 grp + sub: the warp rotates four pairs at once, one per 8-lane group; sub-lane
+    // `sub` owns rows 16 sub .. 16 sub + 15 of both columns and visits its eight 16-byte chunks
+    // in an order rotated by `sub`, so the four groups' loads spread over all banks.
+    const int grp = lane >> 3, sub = lane & 7;
+    for (int r = 0; r < NP - 1; ++r) {
+      const int k = warp + 16 * grp;
+      const int p = tour_player(k, r), q = tour_player(NP - 1 - k, r);
+      double* mp = M + p * NP + 16 * sub;
+      double* mq = M + q * NP + 16 * sub;
+      double pv[16], qv[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int ch = (i + sub) & 7;
+        const double2 a2 = *reinterpret_cast<const double2*>(mp + 2 * ch);
+        const double2 b2 = *reinterpret_cast<const double2*>(mq + 2 * ch);
+        pv[2 * i] = a2.x; pv[2 * i + 1] = a2.y;
+        qv[2 * i] = b2.x; qv[2 * i + 1] = b2.y;
+      }
+      double a = 0.0, b = 0.0, g = 0.0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        a = fma(pv[i], pv[i], a);
+        b = fma(qv[i], qv[i], b);
+        g = fma(pv[i], qv[i], g);
+      }
+      // reduce to the group's first lane, then broadcast: bit-identical sums in the group
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) {
+        a += __shfl_down_sync(0xffffffffu, a, o, 8);
+        b += __shfl_down_sync(0xffffffffu, b, o, 8);
+        g += __shfl_down_sync(0xffffffffu, g, o, 8);
+      }
+      a = __shfl_sync(0xffffffffu, a, 0, 8);
+      b = __shfl_sync(0xffffffffu, b, 0, 8);
+      g = __shfl_sync(0xffffffffu, g, 0, 8);
+      const float gf = (float)g;
+      if (g * g > 1e-14 * (a * b) && gf != 0.0f) {
+        const float zeta = __fdividef((float)(b - a), 2.0f * gf);
+        const float az = fabsf(zeta);
+        const float t = az > 1e18f ? __fdividef(0.5f, zeta)
+                                   : copysignf(__fdividef(1.0f, az + sqrtf(1.0f + zeta * zeta)), zeta);
+        const float cf = rsqrtf(1.0f + t * t);
+        double c = (double)cf, sn = (double)(t * cf);
+        const double fix = 1.5 - 0.5 * (c * c + sn * sn);   // one Newton step: c^2 + s^2 = 1
+        c *= fix;
+        sn *= fix;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int ch = (i + sub) & 7;
+          double2 u, v;
+          u.x = c * pv[2 * i] - sn * qv[2 * i];
+          u.y = c * pv[2 * i + 1] - sn * qv[2 * i + 1];
+          v.x = sn * pv[2 * i] + c * qv[2 * i];
+          v.y = sn * pv[2 * i + 1] + c * qv[2 * i + 1];
+          *reinterpret_cast<double2*>(mp + 2 * ch) = u;
+          *reinterpret_cast<double2*>(mq + 2 * ch) = v;
+        }
+        any = 1;
+      }
+      __syncthreads();
+    }
+    if (any && lane == 0) rotated = 1;
+    __syncthreads();
+    if (!rotated) break;
+  }
+  if (sweep == max_sweeps && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
+  // column norms, descending order (zero padding sorts last)
+  for (int j = warp; j < NP; j += 16) {
+    const double* mj = M + j * NP + 4 * lane;
+    double a = mj[0] * mj[0] + mj[1] * mj[1] + mj[2] * mj[2] + mj[3] * mj[3];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) nrm[j] = a;
+  }
+  __syncthreads();
+  for (int i = tid; i < NP; i += 512) {
+    const double li = nrm[i];
+    int rk = 0;
+    for (int j = 0; j < NP; ++j) {
+      const double lj = nrm[j];
+      rk += (lj > li) || (lj == li && j < i);
+    }
+    rank[i] = rk;
+  }
+  __syncthreads();
+  float* vo = Vout + (int64_t)blockIdx.x * sV;
+  for (int e = tid; e < n * NP; e += 512) {
+    const int c = e >> 7, r = e & (NP - 1);   // column c of M, row r
+    if (r >= n || rank[c] >= n) continue;
+    const double inv = nrm[c] > 0.0 ? 1.0 / sqrt(nrm[c]) : 0.0;
+    vo[(int64_t)r * n + rank[c]] = (float)(M[c * NP + r] * inv);
+  }
+  if (lam)
+    for (int c = tid; c < NP; c += 512)
+      if (rank[c] < n) lam[(int64_t)blockIdx.x * sL + rank[c]] = (float)(nrm[c] - sigma);
+}
+
 // Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
 // R and its inverse are kept as packed upper triangles in shared memory (n (n + 1) / 2 each).
 // Cholesky: right-looking, 3 barriers per pivot. Inverse: thread c back-substitutes column c
@@ -240,6 +407,18 @@ cudaError_t jacobi_eig(int batch, int n, const float* A, int64_t sA, float* V, i
                                        (int)smem);
   if (e != cudaSuccess) return e;
   k_jacobi<<<batch, 512, smem, s>>>(n, A, sA, V, sV, lam, sL, max_sweeps, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int64_t sV, float* lam, int64_t sL,
+                    int max_sweeps, int32_t* status, cudaStream_t s) {
+  if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
+  if (batch <= 0) return cudaSuccess;
+  const size_t smem = ((size_t)kMaxN * kMaxN + kMaxN) * sizeof(double) + kMaxN * sizeof(int);
+  cudaError_t e = cudaFuncSetAttribute(k_eig_psd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_eig_psd<<<batch, 512, smem, s>>>(n, C, sC, V, sV, lam, sL, max_sweeps, status);
   note_launch();
   return cudaGetLastError();
 }
