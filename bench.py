@@ -210,10 +210,9 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks):
         "decode": dict(bound="alu", work=dec_flops / 1e12, unit="TFLOP/s", peak=fp32_peak,
                        note="float32 u M + y Pi^T per entry: 2 (r_t + D) flops; FP32 peak 148 x 128 FMA x 2 x max clock",
                        hbm_bytes=2.0 * N * n_lt + stream_bytes),
-        "jacobi_feature": dict(bound="alu", work=9.0 * D ** 3 * n_lt / 1e12, unit="TFLOP/s", peak=fp32_peak,
-                               note="symmetric eigenproblem with vectors, 9 n^3 flops (Golub & Van Loan count), n = D"),
-        "jacobi_sketch": dict(bound="alu", work=9.0 * l ** 3 * n_lt / 1e12, unit="TFLOP/s", peak=fp32_peak,
-                              note="symmetric eigenproblem with vectors, 9 n^3 flops, n = l"),
+        "jacobi": dict(bound="alu", work=9.0 * (D ** 3 + l ** 3) * n_lt / 1e12, unit="TFLOP/s", peak=fp64_peak,
+                       note="feature (n = D) and sketch (n = l) symmetric eigenproblems with vectors, 9 n^3 flops "
+                            "each (Golub & Van Loan count), float64 one-sided Jacobi: FP64 peak"),
         "cholqr": dict(bound="tensor", work=cholqr_flops / 1e12, unit="TFLOP/s", peak=peaks["bf16_tflops"] * 0.5,
                        note="per pass 4 rows l^2 flops (Gram + triangular update) on float32 data: tf32 peak = bf16 x 1/2"),
     }, stream_bytes

@@ -187,6 +187,9 @@ struct jolt_plan_s {
   __nv_bfloat16* XT = nullptr;       // [n][H][D][T]
   float* Cpart = nullptr;            // [n][H][D][D] per-head Gram partials
   __nv_bfloat16* QTp[3] = {nullptr, nullptr, nullptr};   // bf16 parts of a float32 basis
+  __nv_bfloat16* QNp[3] = {nullptr, nullptr, nullptr};   // the same parts, transposed layout
+  __nv_bfloat16* RTp[3] = {nullptr, nullptr, nullptr};   // parts of R^{-T} (CholeskyQR)
+  float* Wf = nullptr;                                   // float32 CholeskyQR Grams
   double* Gpi = nullptr;
   float* Pi32 = nullptr;
   __nv_bfloat16* Pib = nullptr;
@@ -291,6 +294,55 @@ bool map_rows(CUtensorMap* m, const void* P, int64_t K, int64_t rows, int64_t ba
   const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)batch};
   const uint64_t str[2] = {(uint64_t)K * 2, (uint64_t)(rows * K * 2)};
   return tc_map_bf16(m, P, 3, dims, str);
+}
+
+// CholeskyQR on the tensor cores, transposed layout Y^T [n][l][rows] -> Q^T. Each pass splits
+// Y into three bf16 parts (both layouts), forms the Gram W = Y^T Y from the six part products
+// of order <= 2 (float32 accumulation), inverts its Cholesky factor in float64, and forms
+// Q^T = R^{-T} Y^T from the six part products of R^{-T} and Y. Pass 1 adds 1e-6 trace(W) to
+// the diagonal (a shifted CholeskyQR step; the accumulation error of the Gram is ~1e-6), so the
+// factorisation exists for any sketch; the column space is unchanged by the shift.
+float* cholqr_tc(jolt_plan_s* p, int rows, float* bufA, float* bufB, int passes, int32_t* status, cudaStream_t s,
+                 jolt_status* st) {
+  const int l = p->l, n = p->n_lt;
+  float* src = bufA;
+  float* dst = bufB;
+  *st = JOLT_OK;
+  auto ck = [&](cudaError_t e) {
+    if (e != cudaSuccess && *st == JOLT_OK) *st = fail(JOLT_ERR_CUDA, "cholqr: %s", cudaGetErrorString(e));
+  };
+  static const int8_t pa[6] = {0, 0, 1, 1, 0, 2}, pb[6] = {0, 1, 0, 1, 2, 0};
+  for (int pass = 0; pass < passes && *st == JOLT_OK; ++pass) {
+    ck(split_dual(n, l, rows, src, false, p->QTp, p->QNp, s));
+    TcGemmParams g;
+    g.status = status;
+    for (int i = 0; i < 3; ++i)
+      if (!map_rows(&g.amap[i], p->QTp[i], rows, l, n)) { *st = fail(JOLT_ERR_CUDA, "tensor map rejected"); return src; }
+    g.na = g.nb = 3;
+    g.b_same = 1;
+    g.npairs = 6;
+    for (int i = 0; i < 6; ++i) { g.pair_a[i] = pa[i]; g.pair_b[i] = pb[i]; }
+    g.M = l; g.N = l; g.KB = (rows + 63) / 64;
+    g.C = p->Wf; g.c_sm = l; g.c_sn = 1; g.c_sb = (int64_t)l * l;
+    ck(gemm_tc(n, g, s));
+    ck(chol_inv_f32(n, l, p->Wf, (int64_t)l * l, p->Rinv, (int64_t)l * l, pass == 0 ? 1e-6 * l : 0.0, status, s));
+    ck(split_dual(n, l, l, p->Rinv, true, nullptr, p->RTp, s));
+    TcGemmParams m;
+    m.status = status;
+    for (int i = 0; i < 3; ++i)
+      if (!map_rows(&m.amap[i], p->RTp[i], l, l, n) || !map_rows(&m.bmap[i], p->QNp[i], l, rows, n)) {
+        *st = fail(JOLT_ERR_CUDA, "tensor map rejected");
+        return src;
+      }
+    m.na = m.nb = 3;
+    m.npairs = 6;
+    for (int i = 0; i < 6; ++i) { m.pair_a[i] = pa[i]; m.pair_b[i] = pb[i]; }
+    m.M = l; m.N = rows; m.KB = (l + 63) / 64;
+    m.C = dst; m.c_sm = rows; m.c_sn = 1; m.c_sb = (int64_t)l * rows;
+    ck(gemm_tc(n, m, s));
+    std::swap(src, dst);
+  }
+  return src;
 }
 
 // CholeskyQR on the transposed layout: Y^T [n][l][rows] -> Q^T (same layout), passes as above.
@@ -464,8 +516,12 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     if (p->use_tc) {
       take(p->XT, n * HD * T);
       take(p->Cpart, n * H * D * D);
-      if (p->encoder == JOLT_ENC_SKETCH)
+      if (p->encoder == JOLT_ENC_SKETCH) {
         for (int i = 0; i < 3; ++i) take(p->QTp[i], n * l * std::max<int64_t>(T, HD));
+        for (int i = 0; i < 3; ++i) take(p->QNp[i], n * l * std::max<int64_t>(T, HD));
+        for (int i = 0; i < 3; ++i) take(p->RTp[i], n * l * l);
+        take(p->Wf, n * l * l);
+      }
     }
     if (p->encoder == JOLT_ENC_SKETCH) {
       take(p->Om, n * HD * l);
@@ -551,8 +607,8 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
   {
     PROF("check_norms", s);
     for (int k = 0; k < kinds; ++k) {
-      CK(check_finite(L * HTD, X[k], xt, status, s));
-      CK(sumsq_batched(L, HTD, X[k], xt, HTD, p->xx + (int64_t)k * L, p->xx_part + (int64_t)k * L * 64, s));
+      CK(sumsq_batched(L, HTD, X[k], xt, HTD, p->xx + (int64_t)k * L, p->xx_part + (int64_t)k * L * 64,
+                       status, s));
     }
   }
   CUtensorMap mx[2], mxt;
@@ -585,15 +641,25 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       CK(gemm_simt(L, D, D, H * T, opnd(X[k], xt, I1(HTD), I1(1), I1(D)), opnd(X[k], xt, I1(HTD), I1(1), I1(D)),
                    outd(p->CD + (int64_t)k * L * D * D, EL_F64, I1((int64_t)D * D), I1(D), I1(1)), 1.0, 0.0, s));
   }
-  {
-    PROF("jacobi_feature", s);
-    CK(eig_psd(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, p->cfg.max_jacobi_sweeps,
-               status, s));
-  }
-  {
+  // The feature eigenproblems are solved together with the token ones (one launch, both batches
+  // side by side on the SMs); U_D is first needed by the core projection.
+  auto feature_sign_round = [&]() -> jolt_status {
     PROF("sign_round", s);
     CK(sign_fix(n, D, D, p->UD32, D, (int64_t)D * D, nullptr, 0, 0, 0, s));
     CK(round_bf16((int64_t)n * D * D, p->UD32, p->UDb, p->UDf, s));
+    return JOLT_OK;
+  };
+  auto eig_feature_and = [&](int n1, const double* C1, float* V1, float* lam1) -> jolt_status {
+    PROF("jacobi", s);
+    CK(eig_psd2(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, n1 > 0 ? n : 0, n1, C1,
+                (int64_t)n1 * n1, V1, (int64_t)n1 * n1, lam1, n1, p->cfg.max_jacobi_sweeps, status, s));
+    return JOLT_OK;
+  };
+  if (R == 0) {
+    jolt_status r = eig_feature_and(0, nullptr, nullptr, nullptr);
+    if (r != JOLT_OK) return r;
+    r = feature_sign_round();
+    if (r != JOLT_OK) return r;
   }
   if (R > 0) {
     if (p->encoder == JOLT_ENC_SKETCH && p->use_tc) {
@@ -637,7 +703,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       float* Q;
       {
         PROF("cholqr", s);
-        Q = cholqr_t(p, T, p->Y, p->Y2, q > 0 ? 1 : 2, status, s, &r);
+        Q = cholqr_tc(p, T, p->Y, p->Y2, q > 0 ? 1 : 3, status, s, &r);
         if (r != JOLT_OK) return r;
       }
       for (int it = 0; it < q; ++it) {
@@ -659,7 +725,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         float* Qz;
         {
           PROF("cholqr", s);
-          Qz = cholqr_t(p, (int)HD, p->Z, p->Z2, 1, status, s, &r);
+          Qz = cholqr_tc(p, (int)HD, p->Z, p->Z2, 1, status, s, &r);
           if (r != JOLT_OK) return r;
         }
         float* Ydst = (Q == p->Y) ? p->Y2 : p->Y;
@@ -673,7 +739,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         }
         {
           PROF("cholqr", s);
-          Q = cholqr_t(p, T, Ydst, Yalt, it + 1 == q ? 2 : 1, status, s, &r);
+          Q = cholqr_tc(p, T, Ydst, Yalt, it + 1 == q ? 3 : 1, status, s, &r);
           if (r != JOLT_OK) return r;
         }
       }
@@ -769,9 +835,10 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
                      outd(p->BB, EL_F64, I1((int64_t)l * l), I1(l), I1(1)), 1.0, 0.0, s));
       }
       {
-        PROF("jacobi_sketch", s);
-        CK(eig_psd(n, l, p->BB, (int64_t)l * l, p->Wv, (int64_t)l * l, p->lamB, l, p->cfg.max_jacobi_sweeps,
-                   status, s));
+        jolt_status r = eig_feature_and(l, p->BB, p->Wv, p->lamB);
+        if (r != JOLT_OK) return r;
+        r = feature_sign_round();
+        if (r != JOLT_OK) return r;
       }
       {
         PROF("small_gemm", s);
@@ -803,9 +870,10 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
                        outd(p->CT + (int64_t)k * L * T * T, EL_F64, I1((int64_t)T * T), I1(T), I1(1)), 1.0, 0.0, s));
       }
       {
-        PROF("jacobi_token", s);
-        CK(eig_psd(n, T, p->CT, (int64_t)T * T, p->VT, (int64_t)T * T, p->lamT, T, p->cfg.max_jacobi_sweeps,
-                   status, s));
+        jolt_status r = eig_feature_and(T, p->CT, p->VT, p->lamT);
+        if (r != JOLT_OK) return r;
+        r = feature_sign_round();
+        if (r != JOLT_OK) return r;
       }
       {
         PROF("sign_round", s);

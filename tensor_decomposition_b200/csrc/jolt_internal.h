@@ -78,9 +78,15 @@ cudaError_t jacobi_eig(int batch, int n, const float* A, int64_t sA, float* V, i
 // factor; same output convention as jacobi_eig.
 cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int64_t sV, float* lam, int64_t sL,
                     int max_sweeps, int32_t* status, cudaStream_t s);
+// Two independent batches in one launch (e.g. the feature and the token eigenproblems).
+cudaError_t eig_psd2(int batch0, int n0, const double* C0, int64_t sC0, float* V0, int64_t sV0, float* lam0,
+                     int64_t sL0, int batch1, int n1, const double* C1, int64_t sC1, float* V1, int64_t sV1,
+                     float* lam1, int64_t sL1, int max_sweeps, int32_t* status, cudaStream_t s);
 // Shifted-CholeskyQR helper: Rinv = inverse of chol(W + shift * trace(W)/n * I), W n x n.
 cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv, int64_t sR,
                      double shift, int32_t* status, cudaStream_t s);
+cudaError_t chol_inv_f32(int batch, int n, const float* W, int64_t sW, double* Rinv, int64_t sR,
+                         double shift, int32_t* status, cudaStream_t s);
 // Column sign rule: largest |entry| of each column positive (lowest index on ties).
 // Signs are computed on U (rows x cols, row stride ldu) and applied to U and to the
 // optional companion W (w_rows x cols, row stride ldw).
@@ -90,8 +96,9 @@ cudaError_t sign_fix(int batch, int rows, int cols, float* U, int64_t ldu, int64
 cudaError_t round_bf16(int64_t n, const float* in, __nv_bfloat16* out_b, float* out_f, cudaStream_t s);
 // Squared Frobenius norm (float64, fixed reduction order) of each of `batch` arrays of n elements.
 // `scratch` holds batch * 64 doubles.
+// A non-finite norm sets ST_NONFINITE in *status (when status is not null).
 cudaError_t sumsq_batched(int batch, int64_t n, const void* x, ElemType t, int64_t stride,
-                          double* out, double* scratch, cudaStream_t s);
+                          double* out, double* scratch, int32_t* status, cudaStream_t s);
 // Sum of squared differences and squared reference (float64), deterministic.
 cudaError_t relfrob_partial(const void* ref, const void* approx, uint64_t n, ElemType t,
                             double* partials, int nblocks, double* out2, cudaStream_t s);
@@ -160,6 +167,9 @@ cudaError_t transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int L, int H,
 cudaError_t split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2,
                        cudaStream_t s);
 cudaError_t sum_heads(int n, int H, int64_t per, const float* part, float* out32, double* out64, cudaStream_t s);
+// bf16 parts (3) of batch R x C float32 / float64 matrices, in the same and/or transposed layout.
+cudaError_t split_dual(int batch, int R, int C, const void* in, bool in_f64, __nv_bfloat16* const* same,
+                       __nv_bfloat16* const* tr, cudaStream_t s);
 
 // Check for NaN/Inf in an input tensor (sets ST_NONFINITE).
 cudaError_t check_finite(int64_t n, const void* x, ElemType t, int32_t* status, cudaStream_t s);

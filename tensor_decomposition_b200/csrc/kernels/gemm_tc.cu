@@ -64,8 +64,22 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile, b = blockIdx.z;
-  const int parts = p.na > p.nb ? p.na : p.nb;
-  const int stage_bytes = (p.na + p.nb) * kTileBytes;
+  const int nbl = p.b_same ? 0 : p.nb;   // B parts loaded per stage
+  const int stage_bytes = (p.na + nbl) * kTileBytes;
+  int npairs = p.npairs;
+  int8_t pa[9], pb[9];
+  if (npairs == 0) {
+    npairs = p.na > p.nb ? p.na : p.nb;
+    for (int t = 0; t < npairs; ++t) {
+      pa[t] = (int8_t)(t < p.na ? t : p.na - 1);
+      pb[t] = (int8_t)(t < p.nb ? t : p.nb - 1);
+    }
+  } else {
+    for (int t = 0; t < npairs; ++t) {
+      pa[t] = p.pair_a[t];
+      pb[t] = p.pair_b[t];
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -100,7 +114,7 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
         uint8_t* st = smem + s * stage_bytes;
         mbar_arrive_expect_tx(&full_bar[s], (uint32_t)stage_bytes);
         for (int i = 0; i < p.na; ++i) view_load(p.av, &p.amap[i], st + i * kTileBytes, &full_bar[s], m0, kb, b);
-        for (int i = 0; i < p.nb; ++i)
+        for (int i = 0; i < nbl; ++i)
           view_load(p.bv, &p.bmap[i], st + (p.na + i) * kTileBytes, &full_bar[s], n0, kb, b);
       }
     }
@@ -117,9 +131,10 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
         }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * stage_bytes);
-        for (int t = 0; t < parts; ++t) {
-          const int ia = t < p.na ? t : p.na - 1, ib = t < p.nb ? t : p.nb - 1;
-          const uint32_t abase = st + ia * kTileBytes, bbase = st + (p.na + ib) * kTileBytes;
+        for (int t = 0; t < npairs; ++t) {
+          const int ia = pa[t], ib = pb[t];
+          const uint32_t abase = st + ia * kTileBytes;
+          const uint32_t bbase = p.b_same ? st + ib * kTileBytes : st + (p.na + ib) * kTileBytes;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t ad = desc_kmajor_sw128(abase + k * 32);
@@ -203,8 +218,12 @@ bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
 
 cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
   if (batch <= 0 || p.M <= 0 || p.N <= 0) return cudaSuccess;
-  if (p.na < 1 || p.na > 3 || p.nb < 1 || p.nb > 3 || batch > 65535) return cudaErrorInvalidValue;
-  const int stage_bytes = (p.na + p.nb) * kTileBytes;
+  if (p.na < 1 || p.na > 3 || p.nb < 1 || p.nb > 3 || batch > 65535 || p.npairs < 0 || p.npairs > 9)
+    return cudaErrorInvalidValue;
+  for (int t = 0; t < p.npairs; ++t)
+    if (p.pair_a[t] < 0 || p.pair_a[t] >= p.na || p.pair_b[t] < 0 || p.pair_b[t] >= p.nb) return cudaErrorInvalidValue;
+  if (p.b_same && (p.M > kTile || p.N > kTile || p.nb > p.na)) return cudaErrorInvalidValue;
+  const int stage_bytes = (p.na + (p.b_same ? 0 : p.nb)) * kTileBytes;
   const dim3 g((p.N + kTile - 1) / kTile, (p.M + kTile - 1) / kTile, batch);
   if (stage_bytes * 4 + 1024 <= 200 * 1024) {
     const int smem = stage_bytes * 4 + 1024;

@@ -26,7 +26,13 @@ struct TcGemmParams {
   CUtensorMap amap[3];
   CUtensorMap bmap[3];
   TcView av, bv;
-  int32_t na = 1, nb = 1;   // bf16 parts of A and B; products pair part t of each (clamped)
+  int32_t na = 1, nb = 1;   // bf16 parts of A and B
+  // Products summed into the accumulator: A part pair_a[i] times B part pair_b[i]. With
+  // npairs = 0 the products are (t, t) for t < max(na, nb), each index clamped to its count.
+  int32_t npairs = 0;
+  int8_t pair_a[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  int8_t pair_b[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  int32_t b_same = 0;       // 1: B is A (same maps, same tile: M = N <= 128); B tiles are not loaded
   int32_t M = 0, N = 0, KB = 0;
   float* C = nullptr;       // C[b] + m * c_sm + n * c_sn
   int64_t c_sm = 0, c_sn = 0, c_sb = 0, c_sb_out = 0;

@@ -173,9 +173,27 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
 // when gamma^2 > 1e-14 alpha beta; a sweep with no rotation ends the solve. Each warp works on
 // four pairs of a round at once, eight lanes per pair (16 rows each), so the dot products need
 // only three shuffle steps.
-__global__ void __launch_bounds__(512) k_eig_psd(int n, const double* Cin, int64_t sC, float* Vout, int64_t sV,
-                                                 float* lam, int64_t sL, int max_sweeps, int32_t* status) {
+struct EigBatch {
+  const double* C;
+  int64_t sC;
+  float* V;
+  int64_t sV;
+  float* lam;
+  int64_t sL;
+  int n, count;
+};
+
+// Two independent batches share one launch (blocks [0, b0.count) take the first).
+__global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int max_sweeps, int32_t* status) {
   constexpr int NP = kMaxN, HP = kMaxN / 2;
+  const bool first = (int)blockIdx.x < b0.count;
+  const EigBatch& eb = first ? b0 : b1;
+  const int bi = first ? (int)blockIdx.x : (int)blockIdx.x - b0.count;
+  const int n = eb.n;
+  const double* Cin = eb.C;
+  const int64_t sC = eb.sC, sV = eb.sV, sL = eb.sL;
+  float* Vout = eb.V;
+  float* lam = eb.lam;
   extern __shared__ double ms[];
   double* M = ms;                 // column-major: column j at M + j * NP (during Cholesky: row-major R)
   double* nrm = M + NP * NP;      // NP squared column norms
@@ -183,7 +201,7 @@ __global__ void __launch_bounds__(512) k_eig_psd(int n, const double* Cin, int64
   __shared__ int rotated;
   __shared__ double sigma_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const double* c_in = Cin + (int64_t)blockIdx.x * sC;
+  const double* c_in = Cin + (int64_t)bi * sC;
   // load C (upper triangle used), zero padding
   for (int e = tid; e < NP * NP; e += 512) {
     const int r = e >> 7, c = e & (NP - 1);
@@ -312,7 +330,7 @@ __global__ void __launch_bounds__(512) k_eig_psd(int n, const double* Cin, int64
     rank[i] = rk;
   }
   __syncthreads();
-  float* vo = Vout + (int64_t)blockIdx.x * sV;
+  float* vo = Vout + (int64_t)bi * sV;
   for (int e = tid; e < n * NP; e += 512) {
     const int c = e >> 7, r = e & (NP - 1);   // column c of M, row r
     if (r >= n || rank[c] >= n) continue;
@@ -321,7 +339,7 @@ __global__ void __launch_bounds__(512) k_eig_psd(int n, const double* Cin, int64
   }
   if (lam)
     for (int c = tid; c < NP; c += 512)
-      if (rank[c] < n) lam[(int64_t)blockIdx.x * sL + rank[c]] = (float)(nrm[c] - sigma);
+      if (rank[c] < n) lam[(int64_t)bi * sL + rank[c]] = (float)(nrm[c] - sigma);
 }
 
 // Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
@@ -331,7 +349,8 @@ __global__ void __launch_bounds__(512) k_eig_psd(int n, const double* Cin, int64
 // floor and flags ST_NOT_CONVERGED.
 __device__ __forceinline__ int pk(int i, int k, int n) { return i * n - (i * (i - 1)) / 2 + (k - i); }
 
-__global__ void __launch_bounds__(512) k_chol_inv(int n, const double* W, int64_t sW, double* Rinv,
+template <typename TW>
+__global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
                                                   int64_t sR, double shift, int32_t* status) {
   extern __shared__ double dm[];
   const int np = n * (n + 1) / 2;
@@ -339,10 +358,10 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const double* W, int64_
   double* X = R + np;          // packed upper triangle of the inverse
   __shared__ double tr_s;
   const int tid = threadIdx.x, nt = blockDim.x;
-  const double* w = W + (int64_t)blockIdx.x * sW;
+  const TW* w = W + (int64_t)blockIdx.x * sW;
   for (int e = tid; e < n * n; e += nt) {
     const int i = e / n, k = e % n;
-    if (k >= i) R[pk(i, k, n)] = w[e];
+    if (k >= i) R[pk(i, k, n)] = (double)w[e];
   }
   __syncthreads();
   if (tid == 0) {
@@ -411,29 +430,47 @@ cudaError_t jacobi_eig(int batch, int n, const float* A, int64_t sA, float* V, i
   return cudaGetLastError();
 }
 
-cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int64_t sV, float* lam, int64_t sL,
-                    int max_sweeps, int32_t* status, cudaStream_t s) {
-  if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
-  if (batch <= 0) return cudaSuccess;
+cudaError_t eig_psd2(int batch0, int n0, const double* C0, int64_t sC0, float* V0, int64_t sV0, float* lam0,
+                     int64_t sL0, int batch1, int n1, const double* C1, int64_t sC1, float* V1, int64_t sV1,
+                     float* lam1, int64_t sL1, int max_sweeps, int32_t* status, cudaStream_t s) {
+  if (n0 <= 0 || n0 > kMaxN || (batch1 > 0 && (n1 <= 0 || n1 > kMaxN))) return cudaErrorInvalidValue;
+  if (batch0 + batch1 <= 0) return cudaSuccess;
   const size_t smem = ((size_t)kMaxN * kMaxN + kMaxN) * sizeof(double) + kMaxN * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(k_eig_psd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_eig_psd<<<batch, 512, smem, s>>>(n, C, sC, V, sV, lam, sL, max_sweeps, status);
+  EigBatch b0{C0, sC0, V0, sV0, lam0, sL0, n0, batch0};
+  EigBatch b1{C1, sC1, V1, sV1, lam1, sL1, batch1 > 0 ? n1 : n0, batch1 > 0 ? batch1 : 0};
+  k_eig_psd<<<batch0 + b1.count, 512, smem, s>>>(b0, b1, max_sweeps, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int64_t sV, float* lam, int64_t sL,
+                    int max_sweeps, int32_t* status, cudaStream_t s) {
+  return eig_psd2(batch, n, C, sC, V, sV, lam, sL, 0, 0, nullptr, 0, nullptr, 0, nullptr, 0, max_sweeps, status, s);
+}
+
+template <typename TW>
+static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, double* Rinv, int64_t sR, double shift,
+                              int32_t* status, cudaStream_t s) {
+  if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
+  if (batch <= 0) return cudaSuccess;
+  const size_t smem = (size_t)n * (n + 1) * sizeof(double);
+  cudaError_t e = cudaFuncSetAttribute(k_chol_inv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv, int64_t sR,
                      double shift, int32_t* status, cudaStream_t s) {
-  if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
-  if (batch <= 0) return cudaSuccess;
-  const size_t smem = (size_t)n * (n + 1) * sizeof(double);
-  cudaError_t e = cudaFuncSetAttribute(k_chol_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  k_chol_inv<<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
-  note_launch();
-  return cudaGetLastError();
+  return chol_inv_t<double>(batch, n, W, sW, Rinv, sR, shift, status, s);
+}
+
+cudaError_t chol_inv_f32(int batch, int n, const float* W, int64_t sW, double* Rinv, int64_t sR,
+                         double shift, int32_t* status, cudaStream_t s) {
+  return chol_inv_t<float>(batch, n, W, sW, Rinv, sR, shift, status, s);
 }
 
 }  // namespace jolt

@@ -41,37 +41,89 @@ __global__ void k_round_bf16(int64_t n, const float* in, __nv_bfloat16* ob, floa
 
 constexpr int kSumBlocks = 64;
 
+// 16-byte vector of 8 bf16 or 4 float values, widened to double.
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, int64_t i, double* out) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      out[2 * k] = (double)__uint_as_float(w[k] << 16);
+      out[2 * k + 1] = (double)__uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, int64_t i, double* out) {
+    const float4 f = *reinterpret_cast<const float4*>(p + i);
+    out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
+  }
+};
+
+// Squared norms, vectorised when the array and its length allow 16-byte loads.
 template <typename T>
 __global__ void k_sumsq_part(int64_t n, const T* x, int64_t stride, double* part) {
   __shared__ double red[32];
   const T* p = x + (int64_t)blockIdx.y * stride;
+  constexpr int V = Vec16<T>::N;
   double acc = 0.0;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+  const bool vec = (reinterpret_cast<uintptr_t>(p) % 16 == 0);
+  const int64_t nv = vec ? n / V : 0;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nv; i += (int64_t)gridDim.x * blockDim.x) {
+    double v[V];
+    Vec16<T>::load(p, i * V, v);
+#pragma unroll
+    for (int k = 0; k < V; ++k) acc = fma(v[k], v[k], acc);
+  }
+  for (int64_t i = nv * V + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     const double v = ld_as_double(p, i);
-    acc += v * v;
+    acc = fma(v, v, acc);
   }
   const double t = block_sum(acc, red);
   if (threadIdx.x == 0) part[blockIdx.y * gridDim.x + blockIdx.x] = t;
 }
 
-__global__ void k_sum_rows(int rows, int cols, const double* part, double* out) {
+// A non-finite input makes its squared norm non-finite (bf16 / float32 squares cannot
+// overflow float64), so the norm pass doubles as the NaN / Inf check.
+__global__ void k_sum_rows(int rows, int cols, const double* part, double* out, int32_t* status) {
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= rows) return;
   double t = 0.0;
   for (int c = 0; c < cols; ++c) t += part[(int64_t)r * cols + c];
   out[r] = t;
+  if (status && !isfinite(t)) atomicOr(status, ST_NONFINITE);
 }
 
 template <typename T>
 __global__ void k_relfrob_part(uint64_t n, const T* a, const T* b, double* part) {
   __shared__ double red[32];
+  constexpr int V = Vec16<T>::N;
   double sd = 0.0, sr = 0.0;
-  for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n;
-       i += (uint64_t)gridDim.x * blockDim.x) {
-    const double x = ld_as_double(a, (int64_t)i), y = ld_as_double(b, (int64_t)i);
-    sd += (x - y) * (x - y);
-    sr += x * x;
+  const bool vec = (reinterpret_cast<uintptr_t>(a) % 16 == 0) && (reinterpret_cast<uintptr_t>(b) % 16 == 0);
+  const int64_t nv = vec ? (int64_t)(n / V) : 0;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nv; i += (int64_t)gridDim.x * blockDim.x) {
+    double x[V], y[V];
+    Vec16<T>::load(a, i * V, x);
+    Vec16<T>::load(b, i * V, y);
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+      const double d = x[k] - y[k];
+      sd = fma(d, d, sd);
+      sr = fma(x[k], x[k], sr);
+    }
+  }
+  for (int64_t i = nv * V + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < (int64_t)n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const double x = ld_as_double(a, i), y = ld_as_double(b, i);
+    sd = fma(x - y, x - y, sd);
+    sr = fma(x, x, sr);
   }
   const double td = block_sum(sd, red);
   const double tr = block_sum(sr, red);
@@ -164,21 +216,21 @@ cudaError_t round_bf16(int64_t n, const float* in, __nv_bfloat16* ob, float* of,
 }
 
 cudaError_t sumsq_batched(int batch, int64_t n, const void* x, ElemType t, int64_t stride,
-                          double* out, double* part, cudaStream_t s) {
+                          double* out, double* part, int32_t* status, cudaStream_t s) {
   dim3 g(kSumBlocks, batch);
   if (t == EL_BF16)
     k_sumsq_part<__nv_bfloat16><<<g, 256, 0, s>>>(n, (const __nv_bfloat16*)x, stride, part);
   else
     k_sumsq_part<float><<<g, 256, 0, s>>>(n, (const float*)x, stride, part);
   note_launch();
-  k_sum_rows<<<(batch + 127) / 128, 128, 0, s>>>(batch, kSumBlocks, part, out);
+  k_sum_rows<<<(batch + 127) / 128, 128, 0, s>>>(batch, kSumBlocks, part, out, status);
   note_launch();
   return cudaGetLastError();
 }
 
 int relfrob_blocks(uint64_t n) {
-  uint64_t b = (n + 1023) / 1024;
-  if (b > 592) b = 592;
+  uint64_t b = (n + 2047) / 2048;
+  if (b > 1184) b = 1184;
   if (b < 1) b = 1;
   return (int)b;
 }
