@@ -342,75 +342,79 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
       if (rank[c] < n) lam[(int64_t)bi * sL + rank[c]] = (float)(nrm[c] - sigma);
 }
 
-// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
-// R and its inverse are kept as packed upper triangles in shared memory (n (n + 1) / 2 each).
-// Cholesky: right-looking, 3 barriers per pivot. Inverse: thread c back-substitutes column c
-// (R x = e_c), reading its own earlier entries of X. A non-positive pivot is raised to a tiny
-// floor and flags ST_NOT_CONVERGED.
-__device__ __forceinline__ int pk(int i, int k, int n) { return i * n - (i * (i - 1)) / 2 + (k - i); }
-
+// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64 in
+// shared memory. The n x n problem is embedded in a 128 x 128 one (identity on the padding),
+// so all indexing is shifts and masks.
+//  * Cholesky, right-looking: at pivot k every thread takes sqrt(a_kk) itself, scales its share
+//    of row k, and after one barrier updates its share of the trailing block (2 barriers / pivot).
+//    A pivot below a tiny floor is raised to it and flags ST_NOT_CONVERGED.
+//  * Inverse by back substitution over rows, in place: row i of X = R^{-1} is
+//    (e_i - sum_{k > i} R[i][k] X[k][:]) / R[i][i]; four threads share each column's sum.
 template <typename TW>
 __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
                                                   int64_t sR, double shift, int32_t* status) {
+  constexpr int NP = kMaxN, LD = kMaxN + 1;
   extern __shared__ double dm[];
-  const int np = n * (n + 1) / 2;
-  double* R = dm;              // packed upper triangle of the factor
-  double* X = R + np;          // packed upper triangle of the inverse
+  double* A = dm;                 // NP x LD
+  double* rowi = A + NP * LD;     // NP: row i of R during the inversion
   __shared__ double tr_s;
-  const int tid = threadIdx.x, nt = blockDim.x;
+  __shared__ int floored;
+  const int tid = threadIdx.x;
   const TW* w = W + (int64_t)blockIdx.x * sW;
-  for (int e = tid; e < n * n; e += nt) {
-    const int i = e / n, k = e % n;
-    if (k >= i) R[pk(i, k, n)] = (double)w[e];
+  for (int e = tid; e < NP * NP; e += 512) {
+    const int i = e >> 7, k = e & (NP - 1);
+    A[i * LD + k] = (i < n && k < n) ? (double)w[(int64_t)i * n + k] : (i == k ? 1.0 : 0.0);
   }
+  if (tid == 0) floored = 0;
   __syncthreads();
-  if (tid == 0) {
+  if (tid < 32) {
     double t = 0.0;
-    for (int i = 0; i < n; ++i) t += R[pk(i, i, n)];
-    tr_s = t;
+    for (int i = tid; i < n; i += 32) t += A[i * LD + i];
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_down_sync(0xffffffffu, t, o);
+    if (tid == 0) tr_s = t;
   }
   __syncthreads();
-  const double add = shift * tr_s / n;
-  for (int i = tid; i < n; i += nt) R[pk(i, i, n)] += add;
+  const double tr = tr_s;
+  const double add = shift * tr / n;
+  const double floor_v = 1e-30 + 1e-14 * (tr > 0 ? tr / n : 1.0);
+  for (int i = tid; i < n; i += 512) A[i * LD + i] += add;
   __syncthreads();
-  for (int k = 0; k < n; ++k) {
-    if (tid == 0) {
-      double d = R[pk(k, k, n)];
-      const double floor_v = 1e-30 + 1e-14 * (tr_s > 0 ? tr_s / n : 1.0);
-      if (!(d > floor_v)) {
-        d = floor_v;
-        if (status) atomicOr(status, ST_NOT_CONVERGED);
-      }
-      R[pk(k, k, n)] = sqrt(d);
+  for (int k = 0; k < NP; ++k) {
+    double d = A[k * LD + k];
+    if (!(d > floor_v)) {
+      d = floor_v;
+      if (tid == 0 && k < n) floored = 1;
     }
+    const double rkk = sqrt(d);
+    const double inv = 1.0 / rkk;
+    __syncthreads();                               // everyone has read a_kk
+    if (tid == 0) A[k * LD + k] = rkk;
+    for (int j = k + 1 + tid; j < NP; j += 512) A[k * LD + j] *= inv;
     __syncthreads();
-    const double rkk = R[pk(k, k, n)];
-    for (int j = k + 1 + tid; j < n; j += nt) R[pk(k, j, n)] /= rkk;
-    __syncthreads();
-    const int m = n - k - 1;
-    for (int e = tid; e < m * m; e += nt) {
-      const int i = k + 1 + e / m, j = k + 1 + e % m;
-      if (j >= i) R[pk(i, j, n)] -= R[pk(k, i, n)] * R[pk(k, j, n)];
+    const int m = NP - k - 1;
+    for (int e = tid; e < m * NP; e += 512) {      // rows k+1 .. NP-1, all columns, j >= i kept
+      const int i = k + 1 + (e >> 7), j = e & (NP - 1);
+      if (j >= i) A[i * LD + j] -= A[k * LD + i] * A[k * LD + j];
     }
     __syncthreads();
   }
-  for (int c = tid; c < n; c += nt) {
-    for (int i = c; i >= 0; --i) {
-      double v0 = (i == c) ? 1.0 : 0.0, v1 = 0.0;
-      int k = i + 1;
-      for (; k + 1 <= c; k += 2) {
-        v0 -= R[pk(i, k, n)] * X[pk(k, c, n)];
-        v1 -= R[pk(i, k + 1, n)] * X[pk(k + 1, c, n)];
-      }
-      if (k <= c) v0 -= R[pk(i, k, n)] * X[pk(k, c, n)];
-      X[pk(i, c, n)] = (v0 + v1) / R[pk(i, i, n)];
-    }
+  if (floored && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
+  // back substitution, in place: after step i, row i of A holds row i of X
+  const int col = tid >> 2, part = tid & 3;       // 128 columns x 4 partial sums
+  for (int i = NP - 1; i >= 0; --i) {
+    if (tid < NP) rowi[tid] = tid > i ? A[i * LD + tid] : (tid == i ? A[i * LD + i] : 0.0);
+    __syncthreads();
+    double acc = 0.0;
+    for (int k = i + 1 + part; k < NP; k += 4) acc = fma(rowi[k], A[k * LD + col], acc);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (part == 0) A[i * LD + col] = col < i ? 0.0 : ((col == i ? 1.0 : 0.0) - acc) / rowi[i];
+    __syncthreads();
   }
-  __syncthreads();
   double* o = Rinv + (int64_t)blockIdx.x * sR;
-  for (int e = tid; e < n * n; e += nt) {
+  for (int e = tid; e < n * n; e += 512) {
     const int r = e / n, c = e % n;
-    o[e] = (c >= r) ? X[pk(r, c, n)] : 0.0;
+    o[e] = A[r * LD + c];
   }
 }
 
@@ -455,7 +459,7 @@ static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, double*
                               int32_t* status, cudaStream_t s) {
   if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
   if (batch <= 0) return cudaSuccess;
-  const size_t smem = (size_t)n * (n + 1) * sizeof(double);
+  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + kMaxN) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_chol_inv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);

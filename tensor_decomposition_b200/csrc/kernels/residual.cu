@@ -10,16 +10,15 @@
 // (round to nearest even, saturating at 65504), c_i = clamp(floor(y_i 2^(b-1) / s + 2^(b-1)),
 // 0, 2^b - 1), codes packed LSB first, code i at bits [i b, i b + b) of the row.
 //
-// Arithmetic is float64 end to end (the inputs are bf16 / fp32 values, so products are
-// exact), which keeps every code equal to the one a float64 restatement computes from the
-// same stored factors, except for values within ~1e-13 s of a cell boundary.
+// Arithmetic is float64 end to end (IEEE float64 products and sums on the FP64 tensor-core
+// MMA; the inputs are bf16 / fp32 values), which keeps every code equal to the one a float64
+// restatement computes from the same stored factors, except for values within ~1e-13 s of a
+// cell boundary.
 #include "../jolt_internal.h"
 
 namespace jolt {
 namespace {
 
-constexpr int kRowsPerWarp = 4;
-constexpr int kWarps = 8;
 constexpr int kChunk = 256;          // tokens per CTA
 
 __device__ __forceinline__ const void* x_row_ptr(const ResidualArgs& a, int lt, int h, int t) {
@@ -74,85 +73,113 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf
   }
 }
 
+// y = [x | u] [Pi ; -N]: one float64 GEMM with K = D + r_t on the FP64 tensor-core MMA
+// (m8n8k4: a warp multiplies an 8 x 4 by a 4 x 8 block; fragments per the PTX ISA). A CTA
+// works on 256 tokens of one (layer-tensor, head) in tiles of 16 rows; warp w computes rows
+// 8 (w / 4) .. +7 and columns 32 (w % 4) .. +31 of the tile.
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
+constexpr int kRows = 16;          // rows per tile
+constexpr int kPS = 132;           // row stride (floats) of Pi^T: conflict-free fragment loads
+
 __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* Nbuf, int R) {
-  extern __shared__ unsigned char smraw[];
+  extern __shared__ __align__(16) unsigned char smraw[];
   const int chunk = blockIdx.x, h = blockIdx.y, i = blockIdx.z;
   const int lt = a.lt_ids[i];
   const StreamMeta* m = a.meta;
   const int rt = m->lt_rank[lt][0], b = m->lt_rank[lt][2];
   if (b == 0) return;
-  const int D = a.D;   // 128
-  double* N_s = reinterpret_cast<double*>(smraw);                      // rt x D
-  float* Pi_s = reinterpret_cast<float*>(N_s + (int64_t)rt * D);       // D x D
-  float* stage = Pi_s + D * D;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* xs = stage + warp * (kRowsPerWarp * (2 * kMaxN));             // [4][128] x, then [4][128] u
-  float* us = xs + kRowsPerWarp * kMaxN;
-  unsigned char* cs = reinterpret_cast<unsigned char*>(stage + kWarps * kRowsPerWarp * 2 * kMaxN) +
-                      warp * kRowsPerWarp * kMaxN;
+  const int D = a.D;                       // 128
+  const int K = D + rt;                    // GEMM depth
+  const int SN = rt + 4;                   // row stride (doubles) of N^T
+  const int SA = K + 4;                    // row stride (doubles) of the A / y tile
+  float* PT = reinterpret_cast<float*>(smraw);                                   // [D][kPS]
+  double* NT = reinterpret_cast<double*>(PT + D * kPS);                          // [D][SN] = -N^T
+  double* At = NT + (size_t)D * SN;                                              // [kRows][SA]
+  unsigned char* cs = reinterpret_cast<unsigned char*>(At + (size_t)kRows * SA); // [kRows][D]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < D * D; e += 256) {
+    const int k = e / D, n = e % D;
+    PT[n * kPS + k] = a.Pi[e];
+  }
   const double* Ng = Nbuf + (((int64_t)i * a.H + h) * R) * D;
-  for (int e = threadIdx.x; e < rt * D; e += blockDim.x) N_s[e] = Ng[e];
-  for (int e = threadIdx.x; e < D * D; e += blockDim.x) Pi_s[e] = a.Pi[e];
-  __syncthreads();
+  for (int e = tid; e < rt * D; e += 256) {
+    const int kk = e / D, n = e % D;
+    NT[n * SN + kk] = -Ng[e];
+  }
   const __nv_bfloat16* UT = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UT]);
   __half* scales = reinterpret_cast<__half*>(a.body + m->off[lt][JOLT_PART_SCALES]);
   unsigned char* codes = a.body + m->off[lt][JOLT_PART_CODES];
   const int rowbytes = D * b / 8;
   const double half = (double)(1 << (b - 1));
   const int cmax = (1 << b) - 1;
-  const int t_begin = chunk * kChunk;
-  const int t_end = min(a.T, t_begin + kChunk);
-  for (int t0 = t_begin + warp * kRowsPerWarp; t0 < t_end; t0 += kWarps * kRowsPerWarp) {
-    // stage x rows and u rows
-    for (int r = 0; r < kRowsPerWarp; ++r) {
+  const int t_begin = chunk * kChunk, t_end = min(a.T, t_begin + kChunk);
+  const int rg = warp >> 2, cg = warp & 3;
+  const int ar = 8 * rg + (lane >> 2), ak = lane & 3;
+  __syncthreads();
+  for (int t0 = t_begin; t0 < t_end; t0 += kRows) {
+    // A tile: x rows (float64 of bf16 / float32) followed by u rows
+    for (int e = tid; e < kRows * K; e += 256) {
+      const int r = e / K, c = e % K;
       const int t = t0 + r;
-      for (int q = 0; q < 4; ++q) {
-        const int d = lane + 32 * q;
-        float xv = 0.0f, uv = 0.0f;
-        if (t < t_end) {
+      double v = 0.0;
+      if (t < t_end) {
+        if (c < D) {
           const void* xp = x_row_ptr(a, lt, h, t);
-          xv = a.xt == EL_BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xp)[d])
-                               : reinterpret_cast<const float*>(xp)[d];
-          if (d < rt) uv = __bfloat162float(UT[(int64_t)t * rt + d]);
+          v = a.xt == EL_BF16 ? (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xp)[c])
+                              : (double)reinterpret_cast<const float*>(xp)[c];
+        } else {
+          v = (double)__bfloat162float(UT[(int64_t)t * rt + (c - D)]);
         }
-        xs[r * kMaxN + d] = xv;
-        us[r * kMaxN + d] = uv;
+      }
+      At[r * SA + c] = v;
+    }
+    __syncthreads();
+    double acc[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = 0.0;
+    const double* arow = At + ar * SA + ak;
+#pragma unroll 4
+    for (int k0 = 0; k0 < D; k0 += 4) {
+      const double av = arow[k0];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = 32 * cg + 8 * j + (lane >> 2);
+        dmma_8x8x4(acc[j][0], acc[j][1], av, (double)PT[n * kPS + k0 + ak]);
       }
     }
-    __syncwarp();
-    double acc[kRowsPerWarp][4];
+    for (int k0 = 0; k0 < rt; k0 += 4) {
+      const double av = arow[D + k0];
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[r][q] = 0.0;
-    for (int ii = 0; ii < D; ++ii) {
-      double p[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) p[q] = (double)Pi_s[ii * D + lane + 32 * q];
-#pragma unroll
-      for (int r = 0; r < kRowsPerWarp; ++r) {
-        const double xv = (double)xs[r * kMaxN + ii];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[r][q] = fma(xv, p[q], acc[r][q]);
+      for (int j = 0; j < 4; ++j) {
+        const int n = 32 * cg + 8 * j + (lane >> 2);
+        dmma_8x8x4(acc[j][0], acc[j][1], av, NT[n * SN + k0 + ak]);
       }
     }
-    for (int k = 0; k < rt; ++k) {
-      double nv[4];
+    __syncthreads();                                   // A no longer read: reuse it for y
 #pragma unroll
-      for (int q = 0; q < 4; ++q) nv[q] = N_s[k * D + lane + 32 * q];
-#pragma unroll
-      for (int r = 0; r < kRowsPerWarp; ++r) {
-        const double uv = -(double)us[r * kMaxN + k];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[r][q] = fma(uv, nv[q], acc[r][q]);
-      }
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * cg + 8 * j + 2 * (lane & 3);
+      At[ar * SA + c] = acc[j][0];
+      At[ar * SA + c + 1] = acc[j][1];
     }
+    __syncthreads();
+    // quantise: warp w handles rows 2 w and 2 w + 1; lane owns features lane + 32 q
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
+    for (int rr = 0; rr < 2; ++rr) {
+      const int r = 2 * warp + rr;
       const int t = t0 + r;
+      double y[4];
       double mx = 0.0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) mx = fmax(mx, fabs(acc[r][q]));
+      for (int q = 0; q < 4; ++q) {
+        y[q] = At[r * SA + lane + 32 * q];
+        mx = fmax(mx, fabs(y[q]));
+      }
       for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const __half sh = mx >= 65504.0 ? __float2half_rn(65504.0f) : __double2half(mx);
       const double sd = (double)__half2float(sh);
@@ -160,11 +187,11 @@ __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* 
       for (int q = 0; q < 4; ++q) {
         int c = 0;
         if (sd > 0.0) {
-          const double u = __dadd_rn(__ddiv_rn(acc[r][q] * half, sd), half);
+          const double u = __dadd_rn(__ddiv_rn(y[q] * half, sd), half);
           const double f = floor(u);
           c = f < 0.0 ? 0 : (f > (double)cmax ? cmax : (int)f);
         }
-        cs[r * kMaxN + lane + 32 * q] = (unsigned char)c;
+        cs[r * D + lane + 32 * q] = (unsigned char)c;
       }
       __syncwarp();
       if (t < t_end) {
@@ -174,14 +201,14 @@ __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* 
 #pragma unroll
           for (int bit = 0; bit < 8; ++bit) {
             const int pos = 8 * k + bit;
-            byte |= ((unsigned int)(cs[r * kMaxN + pos / b] >> (pos % b)) & 1u) << bit;
+            byte |= ((unsigned int)(cs[r * D + pos / b] >> (pos % b)) & 1u) << bit;
           }
           codes[row * rowbytes + k] = (unsigned char)byte;
         }
         if (lane == 0) scales[row] = sh;
       }
-      __syncwarp();
     }
+    __syncthreads();
   }
 }
 
@@ -198,13 +225,12 @@ cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStre
   if (e != cudaSuccess) return e;
   k_resid_prep<<<dim3(a.H, a.n_lt), 256, sp, s>>>(a, Nbuf, R);
   note_launch();
-  const size_t sm = (size_t)R * kD * sizeof(double) + (size_t)kD * kD * sizeof(float) +
-                    (size_t)kWarps * kRowsPerWarp * 2 * kMaxN * sizeof(float) +
-                    (size_t)kWarps * kRowsPerWarp * kMaxN;
+  const size_t sm = (size_t)kD * kPS * sizeof(float) + (size_t)kD * (R + 4) * sizeof(double) +
+                    (size_t)kRows * (kD + R + 4) * sizeof(double) + (size_t)kRows * kD;
   e = cudaFuncSetAttribute(k_residual, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const dim3 g((a.T + kChunk - 1) / kChunk, a.H, a.n_lt);
-  k_residual<<<g, kWarps * 32, sm, s>>>(a, Nbuf, R);
+  k_residual<<<g, 256, sm, s>>>(a, Nbuf, R);
   note_launch();
   return cudaGetLastError();
 }
