@@ -342,34 +342,54 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
       if (rank[c] < n) lam[(int64_t)bi * sL + rank[c]] = (float)(nrm[c] - sigma);
 }
 
-// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64 in
-// shared memory. The n x n problem is embedded in a 128 x 128 one (identity on the padding),
-// so all indexing is shifts and masks.
-//  * Cholesky, right-looking: at pivot k every thread takes sqrt(a_kk) itself, scales its share
-//    of row k, and after one barrier updates its share of the trailing block (2 barriers / pivot).
-//    A pivot below a tiny floor is raised to it and flags ST_NOT_CONVERGED.
-//  * Inverse by back substitution over rows, in place: row i of X = R^{-1} is
-//    (e_i - sum_{k > i} R[i][k] X[k][:]) / R[i][i]; four threads share each column's sum.
+// 1 / sqrt(d) to float64 accuracy: float32 seed and two Newton steps.
+__device__ __forceinline__ double rsqrt_f64(double d) {
+  if (d < 1e-30 || d > 1e30) return 1.0 / sqrt(d);
+  double r = (double)rsqrtf((float)d);
+  r = r * (1.5 - 0.5 * d * r * r);
+  r = r * (1.5 - 0.5 * d * r * r);
+  return r;
+}
+
+// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
+// The n x n problem is embedded in a 128 x 128 one (identity on the padding). Thread t keeps
+// the 4 x 8 block rows 4 (t / 16) .., columns 8 (t % 16) .. in registers; the 16 threads of a
+// row block are one half-warp.
+//  * Cholesky, right-looking, one barrier per pivot: in step k every thread applies the rank-1
+//    update with the published row k; the half-warp owning row k + 1 then takes its pivot
+//    (shuffle broadcast, reciprocal square root by a float32 seed and two Newton steps),
+//    scales the row and publishes it in the other buffer. A pivot below a tiny floor is
+//    raised to it and flags ST_NOT_CONVERGED.
+//  * Inverse: R X = I from the last row up, also one barrier per step: X[k][:] = B[k][:] /
+//    R[k][k] is published, then B[i][:] -= R[i][k] X[k][:] for i < k (B = I initially).
 template <typename TW>
 __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
                                                   int64_t sR, double shift, int32_t* status) {
   constexpr int NP = kMaxN, LD = kMaxN + 1;
   extern __shared__ double dm[];
-  double* A = dm;                 // NP x LD
-  double* rowi = A + NP * LD;     // NP: row i of R during the inversion
+  double* Rs = dm;                     // NP x LD: the factor R (rows as published)
+  double* rowb = Rs + NP * LD;         // 2 x NP published rows
+  double* invd = rowb + 2 * NP;        // NP: 1 / R[k][k]
   __shared__ double tr_s;
   __shared__ int floored;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int rb = tid >> 4, cb = tid & 15;
+  const int r0 = 4 * rb, c0 = 8 * cb;
+  const unsigned hmask = 0xFFFFu << (16 * (rb & 1));
+  const int hbase = 16 * (rb & 1);
   const TW* w = W + (int64_t)blockIdx.x * sW;
-  for (int e = tid; e < NP * NP; e += 512) {
-    const int i = e >> 7, k = e & (NP - 1);
-    A[i * LD + k] = (i < n && k < n) ? (double)w[(int64_t)i * n + k] : (i == k ? 1.0 : 0.0);
-  }
+  double a[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = r0 + i, c = c0 + j;
+      a[i][j] = (r < n && c < n) ? (double)w[(int64_t)r * n + c] : (r == c ? 1.0 : 0.0);
+    }
   if (tid == 0) floored = 0;
-  __syncthreads();
   if (tid < 32) {
     double t = 0.0;
-    for (int i = tid; i < n; i += 32) t += A[i * LD + i];
+    for (int i = tid; i < n; i += 32) t += (double)w[(int64_t)i * n + i];
     for (int o = 16; o > 0; o >>= 1) t += __shfl_down_sync(0xffffffffu, t, o);
     if (tid == 0) tr_s = t;
   }
@@ -377,45 +397,105 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   const double tr = tr_s;
   const double add = shift * tr / n;
   const double floor_v = 1e-30 + 1e-14 * (tr > 0 ? tr / n : 1.0);
-  for (int i = tid; i < n; i += 512) A[i * LD + i] += add;
-  __syncthreads();
-  for (int k = 0; k < NP; ++k) {
-    double d = A[k * LD + k];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (r0 + i == c0 + j && r0 + i < n) a[i][j] += add;
+  // scale and publish row `k` (called by the half-warp owning it)
+  auto publish_row = [&](int k, double* buf) {
+    const int i = k & 3;
+    double mine = 0.0;
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (ii == i && c0 + j == k) mine = a[ii][j];
+    double d = __shfl_sync(hmask, mine, hbase + (k >> 3));
     if (!(d > floor_v)) {
       d = floor_v;
-      if (tid == 0 && k < n) floored = 1;
+      if (cb == 0 && k < n) floored = 1;
     }
-    const double rkk = sqrt(d);
-    const double inv = 1.0 / rkk;
-    __syncthreads();                               // everyone has read a_kk
-    if (tid == 0) A[k * LD + k] = rkk;
-    for (int j = k + 1 + tid; j < NP; j += 512) A[k * LD + j] *= inv;
-    __syncthreads();
-    const int m = NP - k - 1;
-    for (int e = tid; e < m * NP; e += 512) {      // rows k+1 .. NP-1, all columns, j >= i kept
-      const int i = k + 1 + (e >> 7), j = e & (NP - 1);
-      if (j >= i) A[i * LD + j] -= A[k * LD + i] * A[k * LD + j];
+    const double inv = rsqrt_f64(d);
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+      if (ii == i) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = c0 + j;
+          double v = a[ii][j];
+          if (c == k) v = d * inv;
+          else if (c > k) v *= inv;
+          else v = 0.0;
+          a[ii][j] = v;
+          buf[c] = v;
+          Rs[k * LD + c] = v;
+        }
+      }
+    if (cb == 0) invd[k] = 1.0 / (d * inv);
+  };
+  if (rb == 0) publish_row(0, rowb);
+  __syncthreads();
+  for (int k = 0; k < NP; ++k) {
+    const double* rk = rowb + (k & 1) * NP;
+    if (r0 + 3 > k) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = r0 + i;
+        if (r <= k) continue;
+        const double u = rk[r];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (c0 + j > k) a[i][j] -= u * rk[c0 + j];
+      }
     }
+    if (k + 1 < NP && rb == ((k + 1) >> 2)) publish_row(k + 1, rowb + ((k + 1) & 1) * NP);
     __syncthreads();
   }
   if (floored && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
-  // back substitution, in place: after step i, row i of A holds row i of X
-  const int col = tid >> 2, part = tid & 3;       // 128 columns x 4 partial sums
-  for (int i = NP - 1; i >= 0; --i) {
-    if (tid < NP) rowi[tid] = tid > i ? A[i * LD + tid] : (tid == i ? A[i * LD + i] : 0.0);
-    __syncthreads();
-    double acc = 0.0;
-    for (int k = i + 1 + part; k < NP; k += 4) acc = fma(rowi[k], A[k * LD + col], acc);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (part == 0) A[i * LD + col] = col < i ? 0.0 : ((col == i ? 1.0 : 0.0) - acc) / rowi[i];
+  // B = I in the registers; X rows published from the last one up
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[i][j] = (r0 + i == c0 + j) ? 1.0 : 0.0;
+  auto publish_x = [&](int k, double* buf) {
+    const double iv = invd[k];
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+      if (r0 + ii == k) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          a[ii][j] *= iv;
+          buf[c0 + j] = a[ii][j];
+        }
+      }
+  };
+  if (rb == ((NP - 1) >> 2)) publish_x(NP - 1, rowb + ((NP - 1) & 1) * NP);
+  __syncthreads();
+  for (int k = NP - 1; k >= 0; --k) {
+    const double* xk = rowb + (k & 1) * NP;
+    if (r0 < k) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = r0 + i;
+        if (r >= k) continue;
+        const double u = Rs[r * LD + k];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[i][j] -= u * xk[c0 + j];
+      }
+    }
+    if (k > 0 && rb == ((k - 1) >> 2)) publish_x(k - 1, rowb + ((k - 1) & 1) * NP);
     __syncthreads();
   }
   double* o = Rinv + (int64_t)blockIdx.x * sR;
-  for (int e = tid; e < n * n; e += 512) {
-    const int r = e / n, c = e % n;
-    o[e] = A[r * LD + c];
-  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = r0 + i, c = c0 + j;
+      if (r < n && c < n) o[(int64_t)r * n + c] = a[i][j];
+    }
+  (void)lane;
 }
 
 }  // namespace
@@ -459,7 +539,7 @@ static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, double*
                               int32_t* status, cudaStream_t s) {
   if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
   if (batch <= 0) return cudaSuccess;
-  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + kMaxN) * sizeof(double);
+  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 3 * kMaxN) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_chol_inv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);

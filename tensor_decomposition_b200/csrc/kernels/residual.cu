@@ -8,7 +8,8 @@
 //     y = (x - u_t G_h U_D^T) Pi = x Pi - u_t N_h,   N_h = (G_h U_D^T) Pi   (r_t x D),
 // u_t = U_T[t, :r_t]. Quantiser (a reading; the pages fix none): s = fp16(max_i |y_i|)
 // (round to nearest even, saturating at 65504), c_i = clamp(floor(y_i 2^(b-1) / s + 2^(b-1)),
-// 0, 2^b - 1), codes packed LSB first, code i at bits [i b, i b + b) of the row.
+// 0, 2^b - 1), codes packed LSB first, code i at bits [i b, i b + b) of the row, written as
+// whole 32-bit words.
 //
 // Arithmetic is float64 end to end (IEEE float64 products and sums on the FP64 tensor-core
 // MMA; the inputs are bf16 / fp32 values), which keeps every code equal to the one a float64
@@ -120,23 +121,46 @@ __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* 
   const int t_begin = chunk * kChunk, t_end = min(a.T, t_begin + kChunk);
   const int rg = warp >> 2, cg = warp & 3;
   const int ar = 8 * rg + (lane >> 2), ak = lane & 3;
+  const int wpr = rowbytes / 4;                         // 32-bit words per packed row (4 b)
+  const int c_first = (32 * lane) / b;                  // codes overlapping word `lane`
+  const int c_last = min(D - 1, (32 * lane + 31) / b);
   __syncthreads();
   for (int t0 = t_begin; t0 < t_end; t0 += kRows) {
-    // A tile: x rows (float64 of bf16 / float32) followed by u rows
-    for (int e = tid; e < kRows * K; e += 256) {
-      const int r = e / K, c = e % K;
+    // A tile: x rows (float64 of bf16 / float32) followed by u rows, 16-byte vector loads:
+    // thread (r = tid / 16, j = tid % 16) takes chunk j of row r (x) and chunk j of u (if any).
+    {
+      const int r = tid >> 4, j = tid & 15;
       const int t = t0 + r;
-      double v = 0.0;
-      if (t < t_end) {
-        if (c < D) {
-          const void* xp = x_row_ptr(a, lt, h, t);
-          v = a.xt == EL_BF16 ? (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xp)[c])
-                              : (double)reinterpret_cast<const float*>(xp)[c];
-        } else {
-          v = (double)__bfloat162float(UT[(int64_t)t * rt + (c - D)]);
+      double* dst = At + r * SA;
+      const bool live = t < t_end;
+      if (a.xt == EL_BF16) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (live) v = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[j];
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          dst[8 * j + 2 * q] = (double)__uint_as_float(wv[q] << 16);
+          dst[8 * j + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (live) f = reinterpret_cast<const float4*>(x_row_ptr(a, lt, h, t))[2 * j + q];
+          dst[8 * j + 4 * q] = f.x; dst[8 * j + 4 * q + 1] = f.y;
+          dst[8 * j + 4 * q + 2] = f.z; dst[8 * j + 4 * q + 3] = f.w;
         }
       }
-      At[r * SA + c] = v;
+      if (8 * j < rt) {                            // rt is a multiple of 16
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (live) v = *reinterpret_cast<const uint4*>(UT + (int64_t)t * rt + 8 * j);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          dst[D + 8 * j + 2 * q] = (double)__uint_as_float(wv[q] << 16);
+          dst[D + 8 * j + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
+        }
+      }
     }
     __syncthreads();
     double acc[4][2];
@@ -168,7 +192,9 @@ __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* 
       At[ar * SA + c + 1] = acc[j][1];
     }
     __syncthreads();
-    // quantise: warp w handles rows 2 w and 2 w + 1; lane owns features lane + 32 q
+    // quantise: warp w handles rows 2 w and 2 w + 1; lane owns features lane + 32 q. The
+    // code is floor(y * (2^(b-1) / s) + 2^(b-1)) with one reciprocal per row (it can differ
+    // from a divide-per-entry only for values within ~1e-16 s of a cell boundary).
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int r = 2 * warp + rr;
@@ -183,12 +209,12 @@ __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* 
       for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const __half sh = mx >= 65504.0 ? __float2half_rn(65504.0f) : __double2half(mx);
       const double sd = (double)__half2float(sh);
+      const double inv = sd > 0.0 ? half / sd : 0.0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         int c = 0;
         if (sd > 0.0) {
-          const double u = __dadd_rn(__ddiv_rn(y[q] * half, sd), half);
-          const double f = floor(u);
+          const double f = floor(fma(y[q], inv, half));
           c = f < 0.0 ? 0 : (f > (double)cmax ? cmax : (int)f);
         }
         cs[r * D + lane + 32 * q] = (unsigned char)c;
@@ -196,14 +222,14 @@ __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* 
       __syncwarp();
       if (t < t_end) {
         const int64_t row = (int64_t)h * a.T + t;
-        for (int k = lane; k < rowbytes; k += 32) {
-          unsigned int byte = 0;
-#pragma unroll
-          for (int bit = 0; bit < 8; ++bit) {
-            const int pos = 8 * k + bit;
-            byte |= ((unsigned int)(cs[r * D + pos / b] >> (pos % b)) & 1u) << bit;
+        if (lane < wpr) {                         // 32-bit word `lane` of the row's bit stream
+          uint32_t word = 0;
+          for (int i = c_first; i <= c_last; ++i) {
+            const int sh2 = i * b - 32 * lane;
+            const uint32_t cv = cs[r * D + i];
+            word |= sh2 >= 0 ? (cv << sh2) : (cv >> (-sh2));
           }
-          codes[row * rowbytes + k] = (unsigned char)byte;
+          reinterpret_cast<uint32_t*>(codes + row * rowbytes)[lane] = word;
         }
         if (lane == 0) scales[row] = sh;
       }
