@@ -151,6 +151,26 @@ JOLT_API jolt_status jolt_decode(jolt_stream_t stream, void* K_out, void* V_out,
 JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, uint64_t n,
                                          jolt_dtype dtype, void* cuda_stream, double* out);
 
+/*
+ * jolt_rel_frob_error_noalloc - the value jolt_rel_frob_error returns, computed with the same
+ *   kernels, grid and reduction order, but without allocating anything: the per-block partial
+ *   sums and the two totals live in one fixed device array inside the library, of
+ *   2 * 1184 + 2 float64 (18,960 bytes) per device. The method has no counterpart of this
+ *   entry point (the paper only defines the error measure); it exists for callers that must
+ *   not allocate device memory.
+ *
+ *   Arguments, layout and the result are those of jolt_rel_frob_error; ref and approx must be
+ *   on the current device. n above JOLT_REL_FROB_NOALLOC_MAX_N returns JOLT_ERR_INVALID_ARG
+ *   (any smaller n fits the fixed scratch: the grid is capped at 1184 blocks).
+ *   Set-up: the first call on each device looks up the array's device address (with that
+ *   device current) and keeps it; make that first call before any stream capture. The call
+ *   synchronises `cuda_stream`. The array is shared by every caller on a device: overlapping
+ *   calls (other threads, or other streams) race on it and may return wrong values.
+ */
+#define JOLT_REL_FROB_NOALLOC_MAX_N (1ULL << 62)
+JOLT_API jolt_status jolt_rel_frob_error_noalloc(const void* ref, const void* approx, uint64_t n,
+                                                 jolt_dtype dtype, void* cuda_stream, double* out);
+
 /* Synchronise on the stream's CUDA stream and report device-side errors of its encode. */
 JOLT_API jolt_status jolt_stream_status(jolt_stream_t stream);
 

@@ -1004,6 +1004,58 @@ JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, ui
   return JOLT_OK;
 }
 
+// Device address of the fixed scratch of jolt_rel_frob_error_noalloc, looked up once per
+// device (with that device current) on the first call made on it.
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_rf_mu;
+double* g_rf_scratch[kMaxDevices] = {};
+}  // namespace
+
+JOLT_API jolt_status jolt_rel_frob_error_noalloc(const void* ref, const void* approx, uint64_t n,
+                                                 jolt_dtype dtype, void* cuda_stream, double* out) {
+  g_err.clear();
+  if (!ref || !approx || !out) return fail(JOLT_ERR_INVALID_ARG, "jolt_rel_frob_error_noalloc: null pointer");
+  if (dtype != JOLT_BF16 && dtype != JOLT_F32)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_rel_frob_error_noalloc: dtype");
+  if (n > JOLT_REL_FROB_NOALLOC_MAX_N)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_rel_frob_error_noalloc: n = %llu exceeds the limit %llu",
+                (unsigned long long)n, (unsigned long long)JOLT_REL_FROB_NOALLOC_MAX_N);
+  const int nb = relfrob_blocks(n);
+  if (nb > kRelfrobStaticBlocks)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_rel_frob_error_noalloc: %d partial sums exceed the fixed scratch of %d",
+                nb, kRelfrobStaticBlocks);
+  int dev = -1;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(JOLT_ERR_UNSUPPORTED, "jolt_rel_frob_error_noalloc: device ordinal %d", dev);
+  double* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_rf_mu);
+    if (!g_rf_scratch[dev]) {
+      double* p = nullptr;
+      const cudaError_t e = relfrob_static_scratch(&p);
+      if (e != cudaSuccess || !p)
+        return fail(JOLT_ERR_CUDA, "jolt_rel_frob_error_noalloc: scratch set-up on device %d: %s", dev,
+                    cudaGetErrorString(e));
+      g_rf_scratch[dev] = p;
+    }
+    scratch = g_rf_scratch[dev];
+  }
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  Prof prof_rf("rel_frob", s);
+  // The two totals are cleared before the kernels run (every partial slot is written).
+  cudaError_t e = cudaMemsetAsync(scratch, 0, 2 * sizeof(double), s);
+  if (e == cudaSuccess)
+    e = relfrob_partial(ref, approx, n, dtype == JOLT_BF16 ? EL_BF16 : EL_F32, scratch + 2, nb, scratch, s);
+  double h[2] = {0.0, 0.0};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h, scratch, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_rel_frob_error_noalloc: %s", cudaGetErrorString(e));
+  *out = h[1] > 0.0 ? std::sqrt(h[0]) / std::sqrt(h[1]) : 0.0;
+  return JOLT_OK;
+}
+
 static jolt_status read_meta(jolt_stream_s* st, StreamMeta* m) {
   CK(cudaStreamSynchronize(st->cs));
   CK(cudaMemcpy(m, st->d_meta, sizeof(StreamMeta), cudaMemcpyDeviceToHost));

@@ -103,6 +103,11 @@ cudaError_t sumsq_batched(int batch, int64_t n, const void* x, ElemType t, int64
 cudaError_t relfrob_partial(const void* ref, const void* approx, uint64_t n, ElemType t,
                             double* partials, int nblocks, double* out2, cudaStream_t s);
 int relfrob_blocks(uint64_t n);
+// Block cap of relfrob_blocks and capacity of the fixed scratch of the allocation-free
+// variant; relfrob_static_scratch returns that scratch's device address for the current device
+// (2 * kRelfrobStaticBlocks partial sums, then the two totals).
+constexpr int kRelfrobStaticBlocks = 1184;
+cudaError_t relfrob_static_scratch(double** p);
 
 struct TableArgs {
   int n_lt, H, R, D, step;

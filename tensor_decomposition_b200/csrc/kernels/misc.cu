@@ -228,6 +228,15 @@ cudaError_t sumsq_batched(int batch, int64_t n, const void* x, ElemType t, int64
   return cudaGetLastError();
 }
 
+// Fixed device scratch of the allocation-free relative-error entry point: the per-block
+// partial sums (2 per block, up to kRelfrobStaticBlocks blocks) followed by the two totals.
+// One array per device, shared by every caller of that entry point: concurrent calls race.
+static __device__ __align__(256) double g_relfrob_scratch[2 * kRelfrobStaticBlocks + 2];
+
+cudaError_t relfrob_static_scratch(double** p) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(p), g_relfrob_scratch);
+}
+
 int relfrob_blocks(uint64_t n) {
   uint64_t b = (n + 2047) / 2048;
   if (b > 1184) b = 1184;

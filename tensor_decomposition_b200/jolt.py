@@ -26,8 +26,8 @@ JOLT_DBG_PI, JOLT_DBG_UT_F32, JOLT_DBG_UD_F32, JOLT_DBG_TABLE, JOLT_DBG_XX, JOLT
 PART_NAMES = ("U_T", "U_D", "G", "scales", "codes")
 
 EXPORTED = ["jolt_config_default", "jolt_plan", "jolt_plan_info", "jolt_encode", "jolt_decode",
-            "jolt_rel_frob_error", "jolt_stream_status", "jolt_stream_info", "jolt_stream_to_host",
-            "jolt_stream_from_host", "jolt_export_debug", "jolt_stream_destroy",
+            "jolt_rel_frob_error", "jolt_rel_frob_error_noalloc", "jolt_stream_status",
+            "jolt_stream_info", "jolt_stream_to_host", "jolt_stream_from_host", "jolt_export_debug", "jolt_stream_destroy",
             "jolt_plan_destroy", "jolt_last_error", "jolt_profile_enable", "jolt_profile_report",
             "jolt_launch_count", "jolt_selftest_gemm_bf16"]
 
@@ -63,6 +63,7 @@ def _load():
         "jolt_encode": (st, [vp, vp, vp, u64, vp, ctypes.POINTER(vp)]),
         "jolt_decode": (st, [vp, vp, vp, vp]),
         "jolt_rel_frob_error": (st, [vp, vp, u64, i32, vp, ctypes.POINTER(ctypes.c_double)]),
+        "jolt_rel_frob_error_noalloc": (st, [vp, vp, u64, i32, vp, ctypes.POINTER(ctypes.c_double)]),
         "jolt_stream_status": (st, [vp]),
         "jolt_stream_info": (st, [vp, ctypes.POINTER(u64), ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double)]),
         "jolt_stream_to_host": (st, [vp, vp, ctypes.POINTER(u64)]),
@@ -175,6 +176,15 @@ def jolt_rel_frob_error(ref, approx, cuda_stream=None) -> float:
     out = ctypes.c_double()
     _check(_lib.jolt_rel_frob_error(_dptr(ref), _dptr(approx), ref.numel(), _dtype_code(ref),
                                     _stream_ptr(cuda_stream), ctypes.byref(out)))
+    return out.value
+
+
+def jolt_rel_frob_error_noalloc(ref, approx, cuda_stream=None) -> float:
+    if ref.shape != approx.shape or ref.dtype != approx.dtype:
+        raise ValueError("ref and approx must share shape and dtype")
+    out = ctypes.c_double()
+    _check(_lib.jolt_rel_frob_error_noalloc(_dptr(ref), _dptr(approx), ref.numel(), _dtype_code(ref),
+                                            _stream_ptr(cuda_stream), ctypes.byref(out)))
     return out.value
 
 
