@@ -352,40 +352,31 @@ __device__ __forceinline__ double rsqrt_f64(double d) {
 }
 
 // Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
-// The n x n problem is embedded in a 128 x 128 one (identity on the padding). Thread t keeps
-// the 4 x 8 block rows 4 (t / 16) .., columns 8 (t % 16) .. in registers; the 16 threads of a
-// row block are one half-warp.
-//  * Cholesky, right-looking, one barrier per pivot: in step k every thread applies the rank-1
-//    update with the published row k; the half-warp owning row k + 1 then takes its pivot
-//    (shuffle broadcast, reciprocal square root by a float32 seed and two Newton steps),
-//    scales the row and publishes it in the other buffer. A pivot below a tiny floor is
+// The n x n problem is embedded in a 128 x 128 one (identity on the padding) and blocked by 16.
+// With L = R^T (W = L L^T) and X = L^{-1}, R^{-1} = X^T. One shared 128 x 129 array holds L
+// in its lower triangle and T = X^T in its upper triangle; the diagonal blocks of L are not
+// needed once their inverses are formed, so T takes over their upper half.
+//  * Cholesky, right-looking by 16-column blocks: warp 0 factors the diagonal block in
+//    registers (shuffle broadcasts, reciprocal square root by a float32 seed and two Newton
+//    steps) and inverts it; the panel below is L21 = A21 L11^{-T}; the trailing lower
+//    triangle takes the rank-16 update in 4 x 4 register tiles. A pivot below a tiny floor is
 //    raised to it and flags ST_NOT_CONVERGED.
-//  * Inverse: R X = I from the last row up, also one barrier per step: X[k][:] = B[k][:] /
-//    R[k][k] is published, then B[i][:] -= R[i][k] X[k][:] for i < k (B = I initially).
+//  * Inverse, right-looking block forward substitution of L X = I: X_k = L_kk^{-1} B_k, then
+//    B_i -= L_ik X_k for the block rows below (B = I initially, kept transposed in T).
 template <typename TW>
 __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
                                                   int64_t sR, double shift, int32_t* status) {
-  constexpr int NP = kMaxN, LD = kMaxN + 1;
+  constexpr int NP = kMaxN, LD = kMaxN + 1, BS = 16, NBLK = NP / BS;
   extern __shared__ double dm[];
-  double* Rs = dm;                     // NP x LD: the factor R (rows as published)
-  double* rowb = Rs + NP * LD;         // 2 x NP published rows
-  double* invd = rowb + 2 * NP;        // NP: 1 / R[k][k]
+  double* A = dm;                          // NP x LD
+  double* Dv = A + NP * LD;                // NBLK x BS x BS: L_kk^{-1} (lower, zero above)
+  double* Pt = Dv + NBLK * BS * BS;        // BS x NP: the current panel, transposed
+  double* Ls = Pt + BS * NP;               // BS x (BS + 1): the current diagonal factor
+  double* Is = Ls + BS * (BS + 1);         // BS: 1 / L_kk diagonal
   __shared__ double tr_s;
   __shared__ int floored;
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int rb = tid >> 4, cb = tid & 15;
-  const int r0 = 4 * rb, c0 = 8 * cb;
-  const unsigned hmask = 0xFFFFu << (16 * (rb & 1));
-  const int hbase = 16 * (rb & 1);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const TW* w = W + (int64_t)blockIdx.x * sW;
-  double a[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int r = r0 + i, c = c0 + j;
-      a[i][j] = (r < n && c < n) ? (double)w[(int64_t)r * n + c] : (r == c ? 1.0 : 0.0);
-    }
   if (tid == 0) floored = 0;
   if (tid < 32) {
     double t = 0.0;
@@ -397,104 +388,182 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   const double tr = tr_s;
   const double add = shift * tr / n;
   const double floor_v = 1e-30 + 1e-14 * (tr > 0 ? tr / n : 1.0);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (r0 + i == c0 + j && r0 + i < n) a[i][j] += add;
-  // scale and publish row `k` (called by the half-warp owning it)
-  auto publish_row = [&](int k, double* buf) {
-    const int i = k & 3;
-    double mine = 0.0;
-#pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (ii == i && c0 + j == k) mine = a[ii][j];
-    double d = __shfl_sync(hmask, mine, hbase + (k >> 3));
-    if (!(d > floor_v)) {
-      d = floor_v;
-      if (cb == 0 && k < n) floored = 1;
+  // lower triangle from W plus the shift, identity on the padding; upper triangle zero
+  for (int e = tid; e < NP * NP; e += 512) {
+    const int r = e >> 7, c = e & (NP - 1);
+    double v = 0.0;
+    if (c <= r) {
+      if (r < n) v = (double)w[(int64_t)r * n + c] + (r == c ? add : 0.0);
+      else v = (r == c) ? 1.0 : 0.0;
     }
-    const double inv = rsqrt_f64(d);
+    A[r * LD + c] = v;
+  }
+  __syncthreads();
+  for (int kb = 0; kb < NBLK; ++kb) {
+    const int k0 = kb * BS;
+    double* D = Dv + kb * BS * BS;
+    if (warp == 0) {
+      // lane i (and its mirror i + 16) holds row i of the diagonal block
+      const int i = lane & (BS - 1);
+      double a[BS];
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
-      if (ii == i) {
+      for (int j = 0; j < BS; ++j) a[j] = A[(k0 + i) * LD + k0 + j];
+      bool fl = false;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int c = c0 + j;
-          double v = a[ii][j];
-          if (c == k) v = d * inv;
-          else if (c > k) v *= inv;
-          else v = 0.0;
-          a[ii][j] = v;
-          buf[c] = v;
-          Rs[k * LD + c] = v;
+      for (int k = 0; k < BS; ++k) {
+        double d = __shfl_sync(0xffffffffu, a[k], k);
+        if (!(d > floor_v)) {
+          d = floor_v;
+          fl = fl || (k0 + k < n);
+        }
+        const double inv = rsqrt_f64(d);
+        const double lk = (i == k) ? d * inv : (i > k ? a[k] * inv : 0.0);
+        a[k] = lk;
+        if (i == k && lane < BS) Is[k] = inv;
+#pragma unroll
+        for (int j = 1; j < BS; ++j) {
+          if (j <= k) continue;
+          const double ljk = __shfl_sync(0xffffffffu, lk, j);
+          if (i >= j) a[j] = fma(-lk, ljk, a[j]);
         }
       }
-    if (cb == 0) invd[k] = 1.0 / (d * inv);
-  };
-  if (rb == 0) publish_row(0, rowb);
-  __syncthreads();
-  for (int k = 0; k < NP; ++k) {
-    const double* rk = rowb + (k & 1) * NP;
-    if (r0 + 3 > k) {
+      if (lane < BS) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = r0 + i;
-        if (r <= k) continue;
-        const double u = rk[r];
+        for (int j = 0; j < BS; ++j) Ls[i * (BS + 1) + j] = a[j];
+      }
+      __syncwarp();
+      // column i of L_kk^{-1}, right-looking substitution (entries above the diagonal stay 0)
+      double acc[BS], x[BS];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (c0 + j > k) a[i][j] -= u * rk[c0 + j];
+      for (int r = 0; r < BS; ++r) acc[r] = (r == i) ? 1.0 : 0.0;
+#pragma unroll
+      for (int m = 0; m < BS; ++m) {
+        x[m] = acc[m] * Is[m];
+#pragma unroll
+        for (int r = 1; r < BS; ++r)
+          if (r > m) acc[r] = fma(-Ls[r * (BS + 1) + m], x[m], acc[r]);
+      }
+      if (lane < BS) {
+#pragma unroll
+        for (int r = 0; r < BS; ++r) {
+          D[r * BS + i] = x[r];
+          if (r >= i) A[(k0 + i) * LD + k0 + r] = x[r];   // T = X^T, upper half of the block
+        }
+        if (fl && lane == 0) floored = 1;
       }
     }
-    if (k + 1 < NP && rb == ((k + 1) >> 2)) publish_row(k + 1, rowb + ((k + 1) & 1) * NP);
+    __syncthreads();
+    const int rows = NP - k0 - BS;
+    // panel L21 = A21 L11^{-T}: one thread per row, in place and into Pt
+    if (tid < rows) {
+      const int i = k0 + BS + tid;
+      double v[BS];
+#pragma unroll
+      for (int m = 0; m < BS; ++m) v[m] = A[i * LD + k0 + m];
+#pragma unroll
+      for (int j = 0; j < BS; ++j) {
+        double o = 0.0;
+#pragma unroll
+        for (int m = 0; m <= j; ++m) o = fma(v[m], D[j * BS + m], o);
+        A[i * LD + k0 + j] = o;
+        Pt[j * NP + i] = o;
+      }
+    }
+    __syncthreads();
+    // trailing update of the lower triangle, 4 x 4 tiles (ti >= tj)
+    const int t4 = rows / 4;
+    const int cnt = t4 * (t4 + 1) / 2;
+    for (int p = tid; p < cnt; p += 512) {
+      int ti = (int)((sqrtf(8.0f * (float)p + 1.0f) - 1.0f) * 0.5f);
+      while ((ti + 1) * (ti + 2) / 2 <= p) ++ti;
+      while (ti * (ti + 1) / 2 > p) --ti;
+      const int tj = p - ti * (ti + 1) / 2;
+      const int i0 = k0 + BS + 4 * ti, j0 = k0 + BS + 4 * tj;
+      double c[4][4];
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) c[ii][jj] = A[(i0 + ii) * LD + j0 + jj];
+#pragma unroll
+      for (int m = 0; m < BS; ++m) {
+        const double2 a01 = *reinterpret_cast<const double2*>(Pt + m * NP + i0);
+        const double2 a23 = *reinterpret_cast<const double2*>(Pt + m * NP + i0 + 2);
+        const double2 b01 = *reinterpret_cast<const double2*>(Pt + m * NP + j0);
+        const double2 b23 = *reinterpret_cast<const double2*>(Pt + m * NP + j0 + 2);
+        const double av[4] = {a01.x, a01.y, a23.x, a23.y};
+        const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) c[ii][jj] = fma(-av[ii], bv[jj], c[ii][jj]);
+      }
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) A[(i0 + ii) * LD + j0 + jj] = c[ii][jj];
+    }
     __syncthreads();
   }
   if (floored && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
-  // B = I in the registers; X rows published from the last one up
+  // Inverse. B (transposed in the upper triangle, zero off the diagonal blocks) -> X^T.
+  for (int kb = 0; kb < NBLK; ++kb) {
+    const int k0 = kb * BS;
+    const double* D = Dv + kb * BS * BS;
+    // X_k[:, c] = L_kk^{-1} B_k[:, c] for the columns c < k0 (the diagonal block is already T)
+    if (tid < k0) {
+      const int c = tid;
+      double b[BS];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+      for (int r = 0; r < BS; ++r) b[r] = A[c * LD + k0 + r];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a[i][j] = (r0 + i == c0 + j) ? 1.0 : 0.0;
-  auto publish_x = [&](int k, double* buf) {
-    const double iv = invd[k];
+      for (int r = 0; r < BS; ++r) {
+        double o = 0.0;
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
-      if (r0 + ii == k) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          a[ii][j] *= iv;
-          buf[c0 + j] = a[ii][j];
-        }
-      }
-  };
-  if (rb == ((NP - 1) >> 2)) publish_x(NP - 1, rowb + ((NP - 1) & 1) * NP);
-  __syncthreads();
-  for (int k = NP - 1; k >= 0; --k) {
-    const double* xk = rowb + (k & 1) * NP;
-    if (r0 < k) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = r0 + i;
-        if (r >= k) continue;
-        const double u = Rs[r * LD + k];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) a[i][j] -= u * xk[c0 + j];
+        for (int m = 0; m <= r; ++m) o = fma(D[r * BS + m], b[m], o);
+        A[c * LD + k0 + r] = o;
       }
     }
-    if (k > 0 && rb == ((k - 1) >> 2)) publish_x(k - 1, rowb + ((k - 1) & 1) * NP);
+    __syncthreads();
+    if (kb == NBLK - 1) break;
+    // B_i[:, c] -= L_ik X_k[:, c] for rows i below the block and columns c < k0 + BS; a thread
+    // takes rows q, q + rows/4, ... (consecutive lanes on consecutive rows) and 4 columns
+    const int rows = NP - k0 - BS, q4 = rows / 4, tc = (k0 + BS) / 4;
+    for (int p = tid; p < q4 * tc; p += 512) {
+      const int q = p % q4, c0 = 4 * (p / q4);
+      int ri[4];
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) ri[ii] = k0 + BS + q + ii * q4;
+      double acc[4][4];
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = A[(c0 + cc) * LD + ri[ii]];
+      const bool diag = c0 >= k0;
+#pragma unroll
+      for (int m = 0; m < BS; ++m) {
+        double xv[4], lv[4];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          xv[cc] = diag ? D[m * BS + (c0 - k0) + cc] : A[(c0 + cc) * LD + k0 + m];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) lv[ii] = A[ri[ii] * LD + k0 + m];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = fma(-lv[ii], xv[cc], acc[ii][cc]);
+      }
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) A[(c0 + cc) * LD + ri[ii]] = acc[ii][cc];
+    }
     __syncthreads();
   }
   double* o = Rinv + (int64_t)blockIdx.x * sR;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int r = r0 + i, c = c0 + j;
-      if (r < n && c < n) o[(int64_t)r * n + c] = a[i][j];
-    }
+  for (int e = tid; e < n * n; e += 512) {
+    const int r = e / n, c = e - r * n;
+    o[e] = (c >= r) ? A[r * LD + c] : 0.0;
+  }
   (void)lane;
 }
 
@@ -539,7 +608,9 @@ static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, double*
                               int32_t* status, cudaStream_t s) {
   if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
   if (batch <= 0) return cudaSuccess;
-  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 3 * kMaxN) * sizeof(double);
+  // A (128 x 129), diagonal-block inverses (8 x 16 x 16), panel (16 x 128), diagonal factor
+  // (16 x 17) and its reciprocal diagonal (16), float64
+  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 8 * 256 + 16 * kMaxN + 16 * 17 + 16) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_chol_inv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
