@@ -1,136 +1,323 @@
-// Fused decode of the JoLT codec: unpack, dequantise, inverse-rotate, add the Tucker part
-// and store, one pass per row.
+// Fused decode of the JoLT codec on the 5th-generation tensor cores: unpack, dequantise,
+// inverse-rotate, add the Tucker part and store.
 //
 // "A JoLT for the KV Cache" (arXiv 2607.12550v2, Abstract) reconstructs the cache from the
-// partial Tucker factors plus the rotated low-bit residual. For row t of head h:
-//     x_hat = u_t M_h + y_hat Pi^T,   M_h = G_h U_D^T (r_t x D),
-//     y_hat_i = s (2 c_i + 1 - 2^b) / 2^b      (mid-rise cell centres),
-// with u_t = U_T[t, :r_t] and the row's fp16 scale s and b-bit codes c. Arithmetic is
-// float32 (the stored parts are bf16 / fp16 / small integers, so every product is exact);
-// the output is rounded to nearest even into bf16, or stored as float32.
+// partial Tucker factors plus the rotated low-bit residual. For the rows t of head h:
+//     X_hat = U_T M_h + diag(s) Y_hat Pi^T,   M_h = G_h U_D^T (r_t x D),
+//     Y_hat[t][i] = (2 c + 1 - 2^b) / 2^b     (mid-rise cell centres at unit scale),
+// with U_T[:, :r_t], the row's fp16 scale s and b-bit codes c.
+//
+// One CTA per (layer-tensor, head) walks the T rows in tiles of 128:
+//  * prologue: M_h^T = U_D G_h^T on the tensor core (both operands are the stored bf16
+//    factors, so the products are exact and only the float32 sum rounds); M_h^T and Pi
+//    (float32) are kept in shared memory as two bf16 parts each (hi + lo, ~2^-17 relative);
+//  * producers (warps 4-7) copy the tile's U_T rows and unpack its codes into bf16 cell
+//    centres (exact: odd integers below 2^8 over 2^b), both in the 128-byte-swizzled K-major
+//    layout; the codes arrive by one bulk copy per tile;
+//  * warp 8 issues tcgen05.mma: acc1 = U_T (M_h^T)_p^T and acc2 = Y_hat Pi_p^T over the
+//    parts p, double-buffered in Tensor Memory (4 x 128 columns);
+//  * the epilogue (warps 0-3, one row per thread) forms acc1 + s acc2 and stores bf16
+//    (round to nearest even) or float32.
+// Every wait is bounded: a timeout sets ST_TIMEOUT in the stream status and the CTA runs on
+// to its end without hanging.
 #include "../jolt_internal.h"
+#include "sm100.cuh"
 
 namespace jolt {
 namespace {
 
-constexpr int kRowsPerWarp = 4;
-constexpr int kWarps = 8;
-constexpr int kChunk = 1024;   // tokens per CTA (M_h is built once per CTA)
+using namespace sm100;
 
-__global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
-  extern __shared__ unsigned char smraw[];
-  const int chunk = blockIdx.x, h = blockIdx.y, i = blockIdx.z;
-  const int lt = a.lt_ids[i];
+constexpr int kTileRows = 128;
+constexpr int kThreads = 288;                 // 9 warps
+constexpr int kOpBytes = 128 * 128 * 2;       // one 128 x 128 bf16 operand (two swizzle atoms)
+constexpr int kCodesBytes = 128 * 128;        // codes of one tile, b <= 8
+constexpr uint32_t kMaxPoll = 1u << 22;
+// dynamic shared memory: B1 parts, B2 parts, A1, A2, codes
+constexpr int kOffB1 = 0;
+constexpr int kOffB2 = 2 * kOpBytes;
+constexpr int kOffA1 = 4 * kOpBytes;
+constexpr int kOffA2 = 5 * kOpBytes;
+constexpr int kOffCodes = 6 * kOpBytes;
+constexpr int kSmemBytes = kOffCodes + kCodesBytes + 1024;
+
+// Byte offset of the 16-byte chunk `c16` (8 bf16, k = 8 c16 ..) of row `row` in a K-major
+// 128-row operand with 128-byte swizzling: 64-element atoms of 16 KB, rows of 128 bytes, the
+// chunk index XOR-ed with the row's position in its 8-row group.
+__device__ __forceinline__ uint32_t sw128(int row, int c16) {
+  return (uint32_t)((c16 >> 3) * 16384 + row * 128 + (((c16 & 7) ^ (row & 7)) << 4));
+}
+
+// Descriptor of the 16-wide K slice `kk` of a 128-row operand at shared address `base`.
+__device__ __forceinline__ uint64_t slice_desc(uint32_t base, int kk) {
+  return desc_kmajor_sw128(base + (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32));
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Split 8 floats into bf16 hi and lo parts (16 bytes each).
+__device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo) {
+  float h[8], l[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+    l[i] = v[i] - h[i];
+  }
+  hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+  lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
+}
+
+__device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int32_t* status) {
+  if (mbar_wait(bar, parity, kMaxPoll)) return true;
+  atomicOr(status, ST_TIMEOUT);
+  return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
+  extern __shared__ uint8_t smraw[];
+  __shared__ __align__(8) uint64_t bar_pro, bar_afull, bar_aempty, bar_codes;
+  __shared__ __align__(8) uint64_t bar_accfull[2], bar_accempty[2];
+  __shared__ uint32_t tmem_base;
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x, li = blockIdx.y;
+  const int lt = a.lt_ids[li];
   const StreamMeta* m = a.meta;
+  int32_t* status = const_cast<int32_t*>(&m->status);
   const int rt = m->lt_rank[lt][0], rd = m->lt_rank[lt][1], b = m->lt_rank[lt][2];
-  const int D = a.D;
-  float* M_s = reinterpret_cast<float*>(smraw);        // rt x D
-  float* PT = M_s + kMaxN * D;                          // PT[i][d] = Pi[d][i]
-  float* work = PT + D * D;                             // G_h (rt x rd) + U_D^T (rd x D), later row staging
-  __nv_bfloat16* G_s = reinterpret_cast<__nv_bfloat16*>(work);
-  __nv_bfloat16* UDt = G_s + kMaxN * kMaxN;
+  const bool tucker = rt > 0 && rd > 0, resid = b > 0;
+  const int T = a.T, H = a.H;
   const __nv_bfloat16* UT = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UT]);
   const __nv_bfloat16* UD = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UD]);
   const __nv_bfloat16* G = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_G]) +
                            (int64_t)h * rt * rd;
   const __half* scales = reinterpret_cast<const __half*>(a.body + m->off[lt][JOLT_PART_SCALES]);
-  const unsigned char* codes = a.body + m->off[lt][JOLT_PART_CODES];
-  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
-    const int r = e / D, c = e % D;
-    PT[c * D + r] = a.Pi[e];
+  const uint8_t* codes = a.body + m->off[lt][JOLT_PART_CODES];
+  const int rowbytes = 16 * b;             // D * b / 8 bytes per row, D = 128
+  const int ntiles = (T + kTileRows - 1) / kTileRows;
+  const uint32_t sB1 = smem_u32(sm + kOffB1), sB2 = smem_u32(sm + kOffB2);
+  const uint32_t sA1 = smem_u32(sm + kOffA1), sA2 = smem_u32(sm + kOffA2);
+
+  if (tid == 0) {
+    mbar_init(&bar_pro, 1);
+    mbar_init(&bar_afull, 128);
+    mbar_init(&bar_aempty, 1);
+    mbar_init(&bar_codes, 1);
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&bar_accfull[j], 1);
+      mbar_init(&bar_accempty[j], 128);
+    }
+    fence_barrier_init();
   }
-  for (int e = threadIdx.x; e < rt * rd; e += blockDim.x) G_s[e] = G[e];
-  for (int e = threadIdx.x; e < D * rd; e += blockDim.x) {
-    const int d = e / rd, j = e % rd;
-    UDt[j * D + d] = UD[e];
+  if (warp == 8) {
+    tmem_alloc(&tmem_base, 512);
+    tmem_relinquish();
   }
+  tc_fence_before();
   __syncthreads();
-  for (int e = threadIdx.x; e < rt * D; e += blockDim.x) {
-    const int k = e / D, d = e % D;
-    float acc = 0.0f;
-    for (int j = 0; j < rd; ++j)
-      acc = fmaf(__bfloat162float(G_s[k * rd + j]), __bfloat162float(UDt[j * D + d]), acc);
-    M_s[e] = acc;
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  // ---------------------------------------------------------------- prologue
+  // Pi (float32, row n = output feature, k = rotated coordinate) -> two bf16 parts (B2)
+  for (int u = tid; u < 128 * 16; u += kThreads) {
+    const int n = u >> 4, c = u & 15;
+    const float4 p0 = *reinterpret_cast<const float4*>(a.Pi + n * 128 + 8 * c);
+    const float4 p1 = *reinterpret_cast<const float4*>(a.Pi + n * 128 + 8 * c + 4);
+    const float v[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint4 hi, lo;
+    split8(v, hi, lo);
+    *reinterpret_cast<uint4*>(sm + kOffB2 + sw128(n, c)) = hi;
+    *reinterpret_cast<uint4*>(sm + kOffB2 + kOpBytes + sw128(n, c)) = lo;
   }
+  // U_D (rows n, K = r_d) into A1 and G_h (rows k, K = r_d) into A2 for M_h^T = U_D G_h^T
+  if (tucker) {
+    const int cpr = rd / 8;
+    for (int u = tid; u < 128 * cpr; u += kThreads) {
+      const int n = u / cpr, c = u - n * cpr;
+      *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(n, c)) =
+          *reinterpret_cast<const uint4*>(UD + (int64_t)n * rd + 8 * c);
+    }
+    for (int u = tid; u < rt * cpr; u += kThreads) {
+      const int k = u / cpr, c = u - k * cpr;
+      *reinterpret_cast<uint4*>(sm + kOffA2 + sw128(k, c)) =
+          *reinterpret_cast<const uint4*>(G + (int64_t)k * rd + 8 * c);
+    }
+  }
+  fence_async_shared();
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* us = work + warp * kRowsPerWarp * 2 * kMaxN;   // [4][128] u rows, then [4][128] y_hat rows
-  float* ys = us + kRowsPerWarp * kMaxN;
-  const int rowbytes = D * b / 8;
-  const float inv2b = 1.0f / (float)(1 << b);
-  const float off2b = 1.0f - (float)(1 << b);
-  const int t_begin = chunk * kChunk, t_end = min(a.T, t_begin + kChunk);
-  const int layer = lt >> 1, kind = lt & 1;
-  const int64_t obase = (((int64_t)layer * a.H + h) * a.T) * D;
-  for (int t0 = t_begin + warp * kRowsPerWarp; t0 < t_end; t0 += kWarps * kRowsPerWarp) {
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-      const int t = t0 + r;
-      const int64_t row = (int64_t)h * a.T + t;
-      float sc = 0.0f;
-      if (b > 0 && t < t_end) sc = __half2float(scales[row]);
-      for (int q = 0; q < 4; ++q) {
-        const int d = lane + 32 * q;
-        float uv = 0.0f, yv = 0.0f;
-        if (t < t_end) {
-          if (d < rt) uv = __bfloat162float(UT[(int64_t)t * rt + d]);
-          if (b > 0) {
-            const int bitpos = d * b;
-            const unsigned char* rp = codes + row * rowbytes;
-            unsigned int w = rp[bitpos >> 3];
-            if ((bitpos >> 3) + 1 < rowbytes) w |= (unsigned int)rp[(bitpos >> 3) + 1] << 8;
-            const int c = (int)((w >> (bitpos & 7)) & ((1u << b) - 1u));
-            yv = sc * (((float)(2 * c) + off2b) * inv2b);
+  if (tucker) {
+    if (warp == 8) {
+      if (elect_one()) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16_f32(128, rt);
+        for (int kk = 0; kk < rd / 16; ++kk)
+          umma_bf16(tmem, slice_desc(sA1, kk), slice_desc(sA2, kk), id, kk > 0 ? 1u : 0u);
+        umma_commit(&bar_pro);
+      }
+      __syncwarp();
+    } else if (warp < 4) {
+      wait_or_flag(&bar_pro, 0, status);
+      tc_fence_after();
+      const int n = 32 * warp + lane;   // feature row of M_h^T
+      for (int c = 0; c < (rt + 31) / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * c), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c16 = 4 * c + q;
+          if (8 * c16 < rt) {
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[8 * q + j]);
+            uint4 hi, lo;
+            split8(v, hi, lo);
+            *reinterpret_cast<uint4*>(sm + kOffB1 + sw128(n, c16)) = hi;
+            *reinterpret_cast<uint4*>(sm + kOffB1 + kOpBytes + sw128(n, c16)) = lo;
           }
         }
-        us[r * kMaxN + d] = uv;
-        ys[r * kMaxN + d] = yv;
       }
+      fence_async_shared();
     }
-    __syncwarp();
-    float acc[kRowsPerWarp][4];
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[r][q] = 0.0f;
-    for (int k = 0; k < rt; ++k) {
-      float mv[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) mv[q] = M_s[k * D + lane + 32 * q];
-#pragma unroll
-      for (int r = 0; r < kRowsPerWarp; ++r) {
-        const float uv = us[r * kMaxN + k];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[r][q] = fmaf(uv, mv[q], acc[r][q]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- tiles of 128 rows
+  if (warp >= 4 && warp < 8) {
+    // producers: U_T rows -> A1, unpacked cell centres -> A2
+    const int pt = tid - 128;
+    const float inv2b = resid ? 1.0f / (float)(1 << b) : 0.0f;
+    const float off2b = resid ? 1.0f - (float)(1 << b) : 0.0f;
+    const uint32_t mask = resid ? (1u << b) - 1u : 0u;
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(sm + kOffCodes);
+    for (int it = 0; it < ntiles; ++it) {
+      const int t0 = it * kTileRows, rows = min(kTileRows, T - t0);
+      if (resid && pt == 0) {
+        const uint32_t bytes = (uint32_t)(rows * rowbytes);
+        mbar_arrive_expect_tx(&bar_codes, bytes);
+        bulk_load(sm + kOffCodes, codes + ((int64_t)h * T + t0) * rowbytes, bytes, &bar_codes);
       }
-    }
-    if (b > 0) {
-      for (int ii = 0; ii < D; ++ii) {
-        float pv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) pv[q] = PT[ii * D + lane + 32 * q];
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) {
-          const float yv = ys[r * kMaxN + ii];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[r][q] = fmaf(yv, pv[q], acc[r][q]);
+      wait_or_flag(&bar_aempty, (uint32_t)((it & 1) ^ 1), status);
+      if (tucker) {
+        const int cpr = rt / 8;
+        const __nv_bfloat16* src = UT + (int64_t)t0 * rt;
+        for (int u = pt; u < rows * cpr; u += 128) {
+          const int r = u / cpr, c = u - r * cpr;
+          *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(r, c)) =
+              *reinterpret_cast<const uint4*>(src + (int64_t)r * rt + 8 * c);
         }
       }
+      if (resid) {
+        wait_or_flag(&bar_codes, (uint32_t)(it & 1), status);
+        for (int u = pt; u < rows * 16; u += 128) {
+          const int r = u >> 4, c = u & 15;
+          const int byte0 = r * rowbytes + c * b;   // eight codes = b bytes
+          const int w0 = byte0 >> 2, sh = (byte0 & 3) * 8;
+          uint64_t v = ((uint64_t)cw[w0] | ((uint64_t)cw[w0 + 1] << 32)) >> sh;
+          if (sh) v |= (uint64_t)cw[w0 + 2] << (64 - sh);
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t q = (uint32_t)(v >> (e * b)) & mask;
+            y[e] = ((float)(2 * q) + off2b) * inv2b;
+          }
+          *reinterpret_cast<uint4*>(sm + kOffA2 + sw128(r, c)) =
+              make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                         pack_bf16x2(y[6], y[7]));
+        }
+      }
+      fence_async_shared();
+      mbar_arrive(&bar_afull);
+      // every producer is done with the codes buffer before the next tile's copy lands in it
+      asm volatile("bar.sync 1, 128;" ::: "memory");
     }
+  } else if (warp == 8) {
+    if (elect_one()) {
+      const uint32_t id = idesc_bf16_f32(128, 128);
+      for (int it = 0; it < ntiles; ++it) {
+        const int buf = it & 1, use = it >> 1;
+        wait_or_flag(&bar_afull, (uint32_t)(it & 1), status);
+        wait_or_flag(&bar_accempty[buf], (uint32_t)((use & 1) ^ 1), status);
+        tc_fence_after();
+        const uint32_t d1 = tmem + (uint32_t)(buf * 256), d2 = d1 + 128;
+        if (tucker)
+          for (int kk = 0; kk < rt / 16; ++kk)
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-      const int t = t0 + r;
-      if (t >= t_end) continue;
-      const int64_t o = obase + (int64_t)t * D;
+            for (int p = 0; p < 2; ++p)
+              umma_bf16(d1, slice_desc(sA1, kk), slice_desc(sB1 + p * kOpBytes, kk), id, (kk | p) ? 1u : 0u);
+        if (resid)
+          for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int d = lane + 32 * q;
-        if (a.ot == EL_BF16)
-          reinterpret_cast<__nv_bfloat16*>(a.out[kind])[o + d] = __float2bfloat16_rn(acc[r][q]);
-        else
-          reinterpret_cast<float*>(a.out[kind])[o + d] = acc[r][q];
+            for (int p = 0; p < 2; ++p)
+              umma_bf16(d2, slice_desc(sA2, kk), slice_desc(sB2 + p * kOpBytes, kk), id, (kk | p) ? 1u : 0u);
+        umma_commit(&bar_aempty);
+        umma_commit(&bar_accfull[buf]);
       }
     }
     __syncwarp();
+  } else if (warp < 4) {
+    // epilogue: TMEM lanes 32 warp .. 32 warp + 31 = rows of the tile
+    const int layer = lt >> 1, kind = lt & 1;
+    const int64_t obase = ((int64_t)layer * H + h) * T * 128;
+    for (int it = 0; it < ntiles; ++it) {
+      const int buf = it & 1, use = it >> 1;
+      wait_or_flag(&bar_accfull[buf], (uint32_t)(use & 1), status);
+      tc_fence_after();
+      const int t = it * kTileRows + 32 * warp + lane;
+      const bool valid = t < T;
+      const float s = (resid && valid) ? __half2float(scales[(int64_t)h * T + t]) : 0.0f;
+      const uint32_t tb = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(buf * 256);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r1[32], r2[32];
+        if (tucker) tmem_ld32(tb + (uint32_t)(32 * c), r1);
+        if (resid) tmem_ld32(tb + 128u + (uint32_t)(32 * c), r2);
+        tmem_ld_wait();
+        float o[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float v = tucker ? __uint_as_float(r1[j]) : 0.0f;
+          if (resid) v = fmaf(s, __uint_as_float(r2[j]), v);
+          o[j] = v;
+        }
+        if (valid) {
+          if (a.ot == EL_BF16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out[kind]) + obase +
+                                                  (int64_t)t * 128 + 32 * c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                                  pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out[kind]) + obase +
+                                                    (int64_t)t * 128 + 32 * c);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_accempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -138,12 +325,11 @@ __global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
 
 cudaError_t decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.D != kD) return cudaErrorInvalidValue;
-  const size_t sm = ((size_t)kMaxN * kD + (size_t)kD * kD) * sizeof(float) +
-                    2 * (size_t)kMaxN * kMaxN * sizeof(__nv_bfloat16);
-  cudaError_t e = cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (a.n_lt <= 0 || a.T <= 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k_decode_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  const dim3 g((a.T + kChunk - 1) / kChunk, a.H, a.n_lt);
-  k_decode<<<g, kWarps * 32, sm, s>>>(a);
+  const dim3 g(a.H, a.n_lt);
+  k_decode_tc<<<g, kThreads, kSmemBytes, s>>>(a);
   note_launch();
   return cudaGetLastError();
 }
