@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
     }
   } else if (warp >= 4) {
     const int e = warp - 4;                      // TMEM lanes 32e .. 32e + 31
-    const bool ok = mbar_wait(&accum_bar, 0, kMaxPoll);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&accum_bar, 0, kMaxPoll));   // warp-uniform
     if (!ok && lane == 0) atomicOr(p.status, ST_TIMEOUT);
     tc_fence_after();
     const int m = m0 + 32 * e + lane;
@@ -156,12 +156,29 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
     if (p.c_batch_in > 0) boff = (int64_t)(b / p.c_batch_in) * p.c_sb_out + (int64_t)(b % p.c_batch_in) * p.c_sb;
     else boff = (int64_t)b * p.c_sb;
     float* C = p.C + boff;
+    // Row-major C (c_sn = 1): each 32 x 32 chunk goes through shared memory (the pipeline
+    // stages are free once the accumulator is complete) so that a store instruction writes
+    // 32 consecutive floats of one row instead of one float of 32 rows.
+    float* stg = reinterpret_cast<float*>(smem) + e * (32 * 33);
+    const bool rowmajor = p.c_sn == 1;
 #pragma unroll 1
     for (int c = 0; c < kTile / 32; ++c) {
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(32 * e) << 16) + (uint32_t)(c * 32), r);
       tmem_ld_wait();
-      if (ok && m < p.M) {
+      if (!ok) continue;
+      if (rowmajor) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
+        __syncwarp();
+        const int n = n0 + c * 32 + lane;
+#pragma unroll 4
+        for (int rr = 0; rr < 32; ++rr) {
+          const int mm = m0 + 32 * e + rr;
+          if (mm < p.M && n < p.N) C[(int64_t)mm * p.c_sm + n] = stg[rr * 33 + lane];
+        }
+        __syncwarp();
+      } else if (m < p.M) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int n = n0 + c * 32 + j;

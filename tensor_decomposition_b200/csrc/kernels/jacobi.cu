@@ -342,25 +342,16 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
       if (rank[c] < n) lam[(int64_t)bi * sL + rank[c]] = (float)(nrm[c] - sigma);
 }
 
-// 1 / sqrt(d) to float64 accuracy: float32 seed and two Newton steps.
-__device__ __forceinline__ double rsqrt_f64(double d) {
-  if (d < 1e-30 || d > 1e30) return 1.0 / sqrt(d);
-  double r = (double)rsqrtf((float)d);
-  r = r * (1.5 - 0.5 * d * r * r);
-  r = r * (1.5 - 0.5 * d * r * r);
-  return r;
-}
-
 // Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
 // The n x n problem is embedded in a 128 x 128 one (identity on the padding) and blocked by 16.
 // With L = R^T (W = L L^T) and X = L^{-1}, R^{-1} = X^T. One shared 128 x 129 array holds L
 // in its lower triangle and T = X^T in its upper triangle; the diagonal blocks of L are not
 // needed once their inverses are formed, so T takes over their upper half.
 //  * Cholesky, right-looking by 16-column blocks: warp 0 factors the diagonal block in
-//    registers (shuffle broadcasts, reciprocal square root by a float32 seed and two Newton
-//    steps) and inverts it; the panel below is L21 = A21 L11^{-T}; the trailing lower
-//    triangle takes the rank-16 update in 4 x 4 register tiles. A pivot below a tiny floor is
-//    raised to it and flags ST_NOT_CONVERGED.
+//    registers (shuffle broadcasts, CUDA's float64 reciprocal square root) and inverts it;
+//    the panel below is L21 = A21 L11^{-T} (1 x 4 strips per thread); the trailing lower
+//    triangle takes the rank-16 update in 4 x 4 register tiles. A pivot below a tiny floor
+//    is raised to it and flags ST_NOT_CONVERGED.
 //  * Inverse, right-looking block forward substitution of L X = I: X_k = L_kk^{-1} B_k, then
 //    B_i -= L_ik X_k for the block rows below (B = I initially, kept transposed in T).
 template <typename TW>
@@ -378,6 +369,13 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const TW* w = W + (int64_t)blockIdx.x * sW;
   if (tid == 0) floored = 0;
+  // every load of W in flight before the first barrier (32 elements per thread)
+  TW wv[NP * NP / 512];
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+    wv[q] = (c <= r && r < n) ? w[(int64_t)r * n + c] : (TW)0;
+  }
   if (tid < 32) {
     double t = 0.0;
     for (int i = tid; i < n; i += 32) t += (double)w[(int64_t)i * n + i];
@@ -389,13 +387,11 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   const double add = shift * tr / n;
   const double floor_v = 1e-30 + 1e-14 * (tr > 0 ? tr / n : 1.0);
   // lower triangle from W plus the shift, identity on the padding; upper triangle zero
-  for (int e = tid; e < NP * NP; e += 512) {
-    const int r = e >> 7, c = e & (NP - 1);
-    double v = 0.0;
-    if (c <= r) {
-      if (r < n) v = (double)w[(int64_t)r * n + c] + (r == c ? add : 0.0);
-      else v = (r == c) ? 1.0 : 0.0;
-    }
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+    double v = (c <= r && r < n) ? (double)wv[q] + (r == c ? add : 0.0) : 0.0;
+    if (r >= n && r == c) v = 1.0;
     A[r * LD + c] = v;
   }
   __syncthreads();
@@ -409,23 +405,29 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
 #pragma unroll
       for (int j = 0; j < BS; ++j) a[j] = A[(k0 + i) * LD + k0 + j];
       bool fl = false;
+      // next pivot: lane k + 1 forms its updated diagonal from its own l_{k+1,k}, so the
+      // broadcast of the pivot does not wait for the column shuffles of step k
+      double dn = a[0];
 #pragma unroll
       for (int k = 0; k < BS; ++k) {
-        double d = __shfl_sync(0xffffffffu, a[k], k);
+        double d = __shfl_sync(0xffffffffu, dn, k);
         if (!(d > floor_v)) {
           d = floor_v;
           fl = fl || (k0 + k < n);
         }
-        const double inv = rsqrt_f64(d);
+        const double inv = rsqrt(d);
         const double lk = (i == k) ? d * inv : (i > k ? a[k] * inv : 0.0);
         a[k] = lk;
+        if (k + 1 < BS) dn = fma(-lk, lk, a[k + 1]);
         if (i == k && lane < BS) Is[k] = inv;
+        // all broadcasts of column k first, then the updates: the shuffles overlap
+        double lj[BS];
 #pragma unroll
-        for (int j = 1; j < BS; ++j) {
-          if (j <= k) continue;
-          const double ljk = __shfl_sync(0xffffffffu, lk, j);
-          if (i >= j) a[j] = fma(-lk, ljk, a[j]);
-        }
+        for (int j = 1; j < BS; ++j)
+          if (j > k) lj[j] = __shfl_sync(0xffffffffu, lk, j);
+#pragma unroll
+        for (int j = 1; j < BS; ++j)
+          if (j > k && i >= j) a[j] = fma(-lk, lj[j], a[j]);
       }
       if (lane < BS) {
 #pragma unroll
@@ -454,22 +456,29 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
     }
     __syncthreads();
     const int rows = NP - k0 - BS;
-    // panel L21 = A21 L11^{-T}: one thread per row, in place and into Pt
-    if (tid < rows) {
-      const int i = k0 + BS + tid;
+    // panel L21 = A21 L11^{-T} into Pt only; thread = (group g of 4 columns, row), consecutive
+    // lanes on consecutive rows. L11^{-1} is stored with zeros above its diagonal, so every
+    // output is a full 16-term sum. A keeps A21 until the trailing phase copies L21 back.
+    for (int u = tid; u < 4 * rows; u += 512) {
+      const int g = u / rows, i = k0 + BS + (u - g * rows);
       double v[BS];
 #pragma unroll
       for (int m = 0; m < BS; ++m) v[m] = A[i * LD + k0 + m];
 #pragma unroll
-      for (int j = 0; j < BS; ++j) {
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = 4 * g + jj;
         double o = 0.0;
 #pragma unroll
-        for (int m = 0; m <= j; ++m) o = fma(v[m], D[j * BS + m], o);
-        A[i * LD + k0 + j] = o;
+        for (int m = 0; m < BS; ++m) o = fma(v[m], D[j * BS + m], o);
         Pt[j * NP + i] = o;
       }
     }
     __syncthreads();
+    // L21 back into A (the trailing tiles below read Pt and write only columns >= k0 + BS)
+    for (int u = tid; u < BS * rows; u += 512) {
+      const int j = u / rows, i = k0 + BS + (u - j * rows);
+      A[i * LD + k0 + j] = Pt[j * NP + i];
+    }
     // trailing update of the lower triangle, 4 x 4 tiles (ti >= tj)
     const int t4 = rows / 4;
     const int cnt = t4 * (t4 + 1) / 2;
@@ -509,18 +518,25 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   for (int kb = 0; kb < NBLK; ++kb) {
     const int k0 = kb * BS;
     const double* D = Dv + kb * BS * BS;
-    // X_k[:, c] = L_kk^{-1} B_k[:, c] for the columns c < k0 (the diagonal block is already T)
-    if (tid < k0) {
-      const int c = tid;
-      double b[BS];
+    // X_k[:, c] = L_kk^{-1} B_k[:, c] for the columns c < k0 (the diagonal block is already T);
+    // thread = (group g of 4 rows, column c): all reads, a barrier, then the in-place writes
+    {
+      const bool act = tid < 4 * k0;
+      const int g = act ? tid / k0 : 0, c = act ? tid - g * k0 : 0;
+      double o[4] = {0.0, 0.0, 0.0, 0.0};
+      if (act) {
+        double bv[BS];
 #pragma unroll
-      for (int r = 0; r < BS; ++r) b[r] = A[c * LD + k0 + r];
+        for (int m = 0; m < BS; ++m) bv[m] = A[c * LD + k0 + m];
 #pragma unroll
-      for (int r = 0; r < BS; ++r) {
-        double o = 0.0;
+        for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
-        for (int m = 0; m <= r; ++m) o = fma(D[r * BS + m], b[m], o);
-        A[c * LD + k0 + r] = o;
+          for (int m = 0; m < BS; ++m) o[rr] = fma(D[(4 * g + rr) * BS + m], bv[m], o[rr]);
+      }
+      __syncthreads();
+      if (act) {
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) A[c * LD + k0 + 4 * g + rr] = o[rr];
       }
     }
     __syncthreads();
