@@ -190,6 +190,8 @@ struct jolt_plan_s {
   __nv_bfloat16* QNp[3] = {nullptr, nullptr, nullptr};   // the same parts, transposed layout
   __nv_bfloat16* RTp[3] = {nullptr, nullptr, nullptr};   // parts of R^{-T} (CholeskyQR)
   float* Wf = nullptr;                                   // float32 CholeskyQR Grams
+  __nv_bfloat16* UDt = nullptr;                          // U_D^T (rounded factor, exact in bf16)
+  __nv_bfloat16* Pp[3] = {nullptr, nullptr, nullptr};    // bf16 parts of the core intermediate P
   double* Gpi = nullptr;
   float* Pi32 = nullptr;
   __nv_bfloat16* Pib = nullptr;
@@ -294,6 +296,26 @@ bool map_rows(CUtensorMap* m, const void* P, int64_t K, int64_t rows, int64_t ba
   const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)batch};
   const uint64_t str[2] = {(uint64_t)K * 2, (uint64_t)(rows * K * 2)};
   return tc_map_bf16(m, P, 3, dims, str);
+}
+
+// [n][rows][chunks * 128] bf16 seen as (128, rows, chunks, n): one batch per (i, chunk), the
+// tile box spanning 64 entries of a chunk and 128 rows.
+bool map_kchunk(CUtensorMap* m, const void* P, int64_t rows, int64_t K, int64_t batch) {
+  const uint64_t dims[4] = {128, (uint64_t)rows, (uint64_t)(K / 128), (uint64_t)batch};
+  const uint64_t str[3] = {(uint64_t)K * 2, 256, (uint64_t)(rows * K * 2)};
+  return tc_map_bf16(m, P, 4, dims, str);
+}
+// [n][H][D][K] bf16 seen as (K, D, H, n): per-head row blocks.
+bool map_perhead(CUtensorMap* m, const void* P, int64_t K, int64_t D, int64_t H, int64_t batch) {
+  const uint64_t dims[4] = {(uint64_t)K, (uint64_t)D, (uint64_t)H, (uint64_t)batch};
+  const uint64_t str[3] = {(uint64_t)K * 2, (uint64_t)(D * K * 2), (uint64_t)(H * D * K * 2)};
+  return tc_map_bf16(m, P, 4, dims, str);
+}
+// Products of two three-part operands kept for float32 accuracy: (0,0) (0,1) (1,0) (1,1) (0,2) (2,0).
+void six_products(TcGemmParams& g) {
+  static const int8_t pa[6] = {0, 0, 1, 1, 0, 2}, pb[6] = {0, 1, 0, 1, 2, 0};
+  g.npairs = 6;
+  for (int i = 0; i < 6; ++i) { g.pair_a[i] = pa[i]; g.pair_b[i] = pb[i]; }
 }
 
 // CholeskyQR on the tensor cores, transposed layout Y^T [n][l][rows] -> Q^T. Each pass splits
@@ -522,6 +544,8 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
         for (int i = 0; i < 3; ++i) take(p->RTp[i], n * l * l);
         take(p->Wf, n * l * l);
       }
+      take(p->UDt, n * D * D);
+      for (int i = 0; i < 3; ++i) take(p->Pp[i], n * H * Rm * D);
     }
     if (p->encoder == JOLT_ENC_SKETCH) {
       take(p->Om, n * HD * l);
@@ -825,7 +849,76 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       }
       p->Qfinal = Q;
     }
-    if (p->encoder == JOLT_ENC_SKETCH) {
+    if (p->encoder == JOLT_ENC_SKETCH && p->use_tc) {
+      const int l = p->l;
+      const int nch = (int)(HD / 128);
+      {
+        PROF("small_gemm", s);
+        // B B^T: float32 partial Grams over 128-wide chunks of the (head, feature) axis on the
+        // tensor cores (B in three bf16 parts), summed over the chunks in float64
+        CK(split_bf16((int64_t)n * l * HD, p->Bm, p->QTp[0], p->QTp[1], p->QTp[2], s));
+        TcGemmParams g;
+        g.status = status;
+        for (int i = 0; i < 3; ++i)
+          if (!map_kchunk(&g.amap[i], p->QTp[i], l, HD, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+        g.av.mode = VIEW_XT_PERHEAD;      // (K, rows, chunk, i)
+        g.av.H = nch;
+        g.na = g.nb = 3;
+        g.b_same = 1;
+        six_products(g);
+        g.M = l; g.N = l; g.KB = 2;
+        g.C = p->Cpart; g.c_sm = l; g.c_sn = 1; g.c_sb = (int64_t)l * l;
+        CK(gemm_tc(n * nch, g, s));
+        CK(sum_heads(n, nch, (int64_t)l * l, p->Cpart, nullptr, p->BB, s));
+      }
+      {
+        jolt_status r = eig_feature_and(l, p->BB, p->Wv, p->lamB);
+        if (r != JOLT_OK) return r;
+        r = feature_sign_round();
+        if (r != JOLT_OK) return r;
+      }
+      {
+        PROF("small_gemm", s);
+        // U_T = Q W[:, :R]: rows t, K = the sketch index; Q^T -> Q parts, W -> W^T parts
+        CK(split_dual(n, l, T, p->Qfinal, false, nullptr, p->QNp, s));
+        CK(split_dual(n, l, l, p->Wv, false, nullptr, p->RTp, s));
+        TcGemmParams g;
+        g.status = status;
+        for (int i = 0; i < 3; ++i)
+          if (!map_rows(&g.amap[i], p->QNp[i], l, T, n) || !map_rows(&g.bmap[i], p->RTp[i], l, l, n))
+            return fail(JOLT_ERR_CUDA, "tensor map rejected");
+        g.na = g.nb = 3;
+        six_products(g);
+        g.M = T; g.N = R; g.KB = (l + 63) / 64;
+        g.C = p->UT32; g.c_sm = R; g.c_sn = 1; g.c_sb = (int64_t)T * R;
+        CK(gemm_tc(n, g, s));
+      }
+      {
+        PROF("sign_round", s);
+        CK(sign_fix(n, T, R, p->UT32, R, (int64_t)T * R, p->Wv, l, l, (int64_t)l * l, s));
+        CK(round_bf16((int64_t)n * T * R, p->UT32, p->UTb, p->UTf, s));
+      }
+      {
+        PROF("core", s);
+        // P[h] = W_R^T B_h (R x D): W^T parts (signs fixed), B^T parts per head
+        CK(split_dual(n, l, l, p->Wv, false, nullptr, p->RTp, s));
+        CK(split_dual(n, l, (int)HD, p->Bm, false, nullptr, p->QNp, s));
+        TcGemmParams g;
+        g.status = status;
+        for (int i = 0; i < 3; ++i)
+          if (!map_rows(&g.amap[i], p->RTp[i], l, l, n) || !map_perhead(&g.bmap[i], p->QNp[i], l, D, H, n))
+            return fail(JOLT_ERR_CUDA, "tensor map rejected");
+        g.av.H = H;                       // W^T shared by the heads of a layer-tensor
+        g.bv.mode = VIEW_XT_PERHEAD;
+        g.bv.H = H;
+        g.bv.D = D;
+        g.na = g.nb = 3;
+        six_products(g);
+        g.M = R; g.N = D; g.KB = (l + 63) / 64;
+        g.C = p->P; g.c_sm = D; g.c_sn = 1; g.c_sb = (int64_t)R * D;
+        CK(gemm_tc(n * H, g, s));
+      }
+    } else if (p->encoder == JOLT_ENC_SKETCH) {
       const int l = p->l;
       {
         PROF("small_gemm", s);
@@ -891,7 +984,24 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
                        outd(p->P + (int64_t)k * L * H * R * D, EL_F32, I1((int64_t)R * D), I1(D), I1(1)), 1.0, 0.0, s));
       }
     }
-    {
+    if (p->use_tc) {
+      PROF("core", s);
+      // G_max[h] = P[h] U_D: P in three bf16 parts, U_D (rounded, exact in bf16) transposed
+      __nv_bfloat16* udt[3] = {p->UDt, nullptr, nullptr};
+      __nv_bfloat16* const* pp = p->Pp;
+      CK(split_dual(n, D, D, p->UDf, false, nullptr, udt, s));
+      CK(split_bf16((int64_t)n * H * R * D, p->P, pp[0], pp[1], pp[2], s));
+      TcGemmParams g;
+      g.status = status;
+      for (int i = 0; i < 3; ++i)
+        if (!map_rows(&g.amap[i], pp[i], D, R, (int64_t)n * H)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+      if (!map_rows(&g.bmap[0], p->UDt, D, D, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+      g.bv.H = H;                         // U_D shared by the heads of a layer-tensor
+      g.na = 3; g.nb = 1;
+      g.M = R; g.N = D; g.KB = (D + 63) / 64;
+      g.C = p->Gmax; g.c_sm = D; g.c_sn = 1; g.c_sb = (int64_t)R * D;
+      CK(gemm_tc(n * H, g, s));
+    } else {
       PROF("core", s);
       CK(gemm_simt(n * H, R, D, D, opnd(p->P, EL_F32, I1((int64_t)R * D), I1(D), I1(1)),
                    opnd(p->UDf, EL_F32, I2(H, 0, (int64_t)D * D), I1(1), I1(D)),

@@ -40,8 +40,8 @@ __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, i
     case VIEW_XT_PERHEAD:              // same map, batch b = i * H + h: rows d, K = t
       c0 = kb * kBK; c1 = row0; c2 = b % v.H; c3 = b / v.H;
       break;
-    default:                           // VIEW_ROWS_K: map (K, rows, batch)
-      c0 = kb * kBK; c1 = row0; c2 = b; c3 = 0;
+    default:                           // VIEW_ROWS_K: map (K, rows, batch), batch index b / H
+      c0 = kb * kBK; c1 = row0; c2 = b / v.H; c3 = 0;
       break;
   }
 }

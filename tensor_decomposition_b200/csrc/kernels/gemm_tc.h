@@ -13,13 +13,14 @@ enum TcViewMode : int32_t {
   VIEW_ROWS_K = 0,        // 3-D map (K, rows, batch)
   VIEW_X_TOKENROWS = 1,   // 4-D map of X [L][H][T][D] as (D, T, H, L): rows = tokens, K = (head, feature)
   VIEW_XT_FEATROWS = 2,   // 4-D map of X^T [n][H][D][T] as (T, D, H, n): rows = (head, feature), K = tokens
-  VIEW_XT_PERHEAD = 3     // same map, batch index = layer-tensor * H + head: rows = features, K = tokens
+  VIEW_XT_PERHEAD = 3     // same map, batch index = layer-tensor * H + head: rows = features, K = tokens;
+                          // any 4-D map (K, rows, H, n) is addressed this way
 };
 
 struct TcView {
   int32_t mode = VIEW_ROWS_K;
   int32_t D = 128;
-  int32_t H = 1;
+  int32_t H = 1;   // VIEW_ROWS_K: batch index divisor (operands shared by H consecutive batches)
 };
 
 struct TcGemmParams {
