@@ -59,54 +59,104 @@ def measured_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled during the timed region.
+
+    In-process NVML queries every 100 ms from a background thread (a separate nvidia-smi
+    process polling the driver perturbed the timed kernels); nvidia-smi is the fallback when
+    the NVML binding is missing. Reads only, no GPU setting is changed."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, cuda_device: int = 0):
         self.idx = gpu_index
+        self.cuda_device = cuda_device
+        self.samples = []          # (sm_mhz, sm_max_mhz, reasons)
+        self.stop_ev = threading.Event()
+        self.t = None
         self.proc = None
-        self.lines = []
+        self.nvml = None
+        self.handle = None
+
+    def _open_nvml(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        h = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.cuda_device).uuid)
+            h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            h = None
+        if h is None:
+            h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+        self.nvml, self.handle = nv, h
 
     def start(self):
+        try:
+            self._open_nvml()
+            self.t = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-lms", "200", "-i", str(self.idx)], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t = threading.Thread(target=self._read_smi, daemon=True)
             self.t.start()
         except OSError:
             self.proc = None
 
-    def _read(self):
-        for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+    def _poll_nvml(self):
+        nv, h = self.nvml, self.handle
+        while True:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                reasons = {n for n, attr in self.REASONS if bits & getattr(nv, attr)}
+                self.samples.append((float(sm), float(smax), reasons))
+            except Exception:
+                pass
+            if self.stop_ev.wait(0.1):
+                break
 
-    def stop(self):
-        if not self.proc:
-            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.t.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
+        for ln in self.proc.stdout:
+            parts = [x.strip() for x in ln.strip().split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
+                sm, smax = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+            self.samples.append((sm, smax, {n for n, v in zip(names, parts[5:9]) if v.lower() == "active"}))
+
+    def stop(self):
+        if self.nvml is None and not self.proc:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["clock sampling unavailable"], samples=0)
+        self.stop_ev.set()
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm = [x[0] for x in self.samples]
+        smax = [x[1] for x in self.samples]
+        reasons = set().union(*[x[2] for x in self.samples]) if self.samples else set()
         return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(smax) if smax else None,
-                    reasons=sorted(reasons), samples=len(sm))
+                    reasons=sorted(reasons), samples=len(sm),
+                    source="nvml" if self.nvml is not None else "nvidia-smi")
 
 
 # ------------------------------------------------------------------ oracle (CPU baseline and reference arm)
@@ -271,7 +321,7 @@ def main():
 
     # ---- timed region: K steps, inputs resident in HBM
     clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local])
-                          if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+                          if os.environ.get("CUDA_VISIBLE_DEVICES") else local, local)
     J.jolt_profile_enable(True)
     barrier()
     clocks.start()

@@ -157,6 +157,49 @@ namespace jolt {
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 }  // namespace jolt
 
+namespace {
+// Stream-ordered allocations (stream bodies, small scratch) come from one memory pool per
+// device owned by the library. Its release threshold is unbounded, so memory freed with
+// cudaFreeAsync stays mapped for the next encode instead of being returned to the driver at
+// every synchronisation (the default pool's behaviour, which re-maps tens of MB per call).
+constexpr int kPoolDevices = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pools[kPoolDevices] = {};
+
+cudaError_t pool_malloc(void** ptr, size_t bytes, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kPoolDevices) return cudaMallocAsync(ptr, bytes, s);
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> g(g_pool_mu);
+    if (!g_pools[dev]) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaMemPool_t np;
+      e = cudaMemPoolCreate(&np, &props);
+      if (e != cudaSuccess) return e;
+      uint64_t keep = UINT64_MAX;
+      e = cudaMemPoolSetAttribute(np, cudaMemPoolAttrReleaseThreshold, &keep);
+      if (e != cudaSuccess) {
+        cudaMemPoolDestroy(np);
+        return e;
+      }
+      g_pools[dev] = np;
+    }
+    pool = g_pools[dev];
+  }
+  return cudaMallocFromPoolAsync(ptr, bytes, pool, s);
+}
+template <typename T>
+cudaError_t pool_malloc(T** ptr, size_t bytes, cudaStream_t s) {
+  return pool_malloc(reinterpret_cast<void**>(ptr), bytes, s);
+}
+}  // namespace
+
 // ============================================================================ objects
 struct jolt_plan_s {
   jolt_shape shape{};
@@ -604,10 +647,10 @@ static jolt_status make_stream(jolt_plan_s* p, uint64_t seed, cudaStream_t cs, j
   st->R = p->R; st->split = (sh.has_v && p->cfg.split_kv_budget) ? 1 : 0; st->dtype = sh.dtype;
   st->seed = seed; st->cs = cs; st->plan = p; st->n_lt = p->n_lt;
   st->body_cap = align_up((size_t)p->budget + (size_t)JOLT_NUM_PARTS * kAlign * p->n_lt + kAlign, kAlign);
-  cudaError_t e = cudaMallocAsync(&st->d_body, st->body_cap, cs);
-  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_meta, sizeof(StreamMeta), cs);
-  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_Pi, sizeof(float) * kD * kD, cs);
-  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_lt_ids, sizeof(int32_t) * p->n_lt, cs);
+  cudaError_t e = pool_malloc(&st->d_body, st->body_cap, cs);
+  if (e == cudaSuccess) e = pool_malloc(&st->d_meta, sizeof(StreamMeta), cs);
+  if (e == cudaSuccess) e = pool_malloc(&st->d_Pi, sizeof(float) * kD * kD, cs);
+  if (e == cudaSuccess) e = pool_malloc(&st->d_lt_ids, sizeof(int32_t) * p->n_lt, cs);
   if (e == cudaSuccess) e = cudaMemsetAsync(st->d_meta, 0, sizeof(StreamMeta), cs);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(st->d_lt_ids, p->d_lt_ids, sizeof(int32_t) * p->n_lt, cudaMemcpyDeviceToDevice, cs);
@@ -1102,7 +1145,7 @@ JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, ui
   const int nb = relfrob_blocks(n);
   Prof prof_rf("rel_frob", s);
   double* scratch = nullptr;
-  CK(cudaMallocAsync(&scratch, sizeof(double) * (2 * (size_t)nb + 2), s));
+  CK(pool_malloc(&scratch, sizeof(double) * (2 * (size_t)nb + 2), s));
   cudaError_t e = relfrob_partial(ref, approx, n, dtype == JOLT_BF16 ? EL_BF16 : EL_F32, scratch + 2, nb, scratch, s);
   double h[2] = {0.0, 0.0};
   if (e == cudaSuccess) e = cudaMemcpyAsync(h, scratch, sizeof(h), cudaMemcpyDeviceToHost, s);
@@ -1327,11 +1370,11 @@ JOLT_API jolt_status jolt_stream_from_host(const void* buf, uint64_t len, void* 
   std::vector<int32_t> ids;
   for (int k = 0; k < (has_v ? 2 : 1); ++k)
     for (int l = 0; l < L; ++l) ids.push_back(2 * l + k);
-  cudaError_t e = cudaMallocAsync(&st->d_body, st->body_cap, s);
-  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_meta, sizeof(StreamMeta), s);
-  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_Pi, sizeof(float) * D * D, s);
-  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_Gpi, sizeof(double) * D * D, s);
-  if (e == cudaSuccess) e = cudaMallocAsync(&st->d_lt_ids, sizeof(int32_t) * ids.size(), s);
+  cudaError_t e = pool_malloc(&st->d_body, st->body_cap, s);
+  if (e == cudaSuccess) e = pool_malloc(&st->d_meta, sizeof(StreamMeta), s);
+  if (e == cudaSuccess) e = pool_malloc(&st->d_Pi, sizeof(float) * D * D, s);
+  if (e == cudaSuccess) e = pool_malloc(&st->d_Gpi, sizeof(double) * D * D, s);
+  if (e == cudaSuccess) e = pool_malloc(&st->d_lt_ids, sizeof(int32_t) * ids.size(), s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->d_body, b + hb, (size_t)body, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->d_meta, &m, sizeof(m), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
@@ -1440,7 +1483,7 @@ JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, co
   p.M = M; p.N = N; p.KB = (K + 63) / 64;
   p.C = C; p.c_sm = N; p.c_sn = 1; p.c_sb = (int64_t)M * N;
   int32_t* st = nullptr;
-  CK(cudaMallocAsync(&st, sizeof(int32_t), s));
+  CK(pool_malloc(&st, sizeof(int32_t), s));
   CK(cudaMemsetAsync(st, 0, sizeof(int32_t), s));
   p.status = st;
   cudaError_t e = gemm_tc(1, p, s);
