@@ -157,244 +157,22 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
     for (int i = tid; i < n; i += 512) lam[(int64_t)blockIdx.x * sL + rank[i]] = A[i * kLd + i];
 }
 
-// Eigenpairs of a batch of symmetric positive semi-definite n x n matrices C (n <= 128),
-// float64 input, by one-sided (Hestenes) Jacobi on a Cholesky factor:
-//   C + sigma I = M M^T (M = R^T, R the upper Cholesky factor, sigma = 1e-13 trace / n keeps
-//   the factorisation defined; it shifts every eigenvalue by sigma and leaves the vectors);
-//   column pairs (p, q) of M are rotated, M <- M J, until all columns are mutually orthogonal;
-//   then M = U Sigma, so the normalised columns are the eigenvectors of C and the squared
-//   column norms (minus sigma) its eigenvalues. No eigenvector matrix is accumulated.
-// M lives in shared memory in float64, column-major, padded with zero rows/columns to 128.
-// Each round of the circle-method tournament rotates 64 disjoint pairs:
-// the three dot products are warp-shuffle reductions; the rotation (Golub & Van Loan sec.
-// 8.6, one-sided Jacobi) uses zeta = (beta - alpha) / (2 gamma), t = sign(zeta) /
-// (|zeta| + sqrt(1 + zeta^2)), c = 1 / sqrt(1 + t^2), s = t c, computed in float32 and
-// renormalised in float64 by one Newton step so that c^2 + s^2 = 1 to ~1e-15. A pair rotates
-// when gamma^2 > 1e-14 alpha beta; a sweep with no rotation ends the solve. Each warp works on
-// four pairs of a round at once, eight lanes per pair (16 rows each), so the dot products need
-// only three shuffle steps.
-struct EigBatch {
-  const double* C;
-  int64_t sC;
-  float* V;
-  int64_t sV;
-  float* lam;
-  int64_t sL;
-  int n, count;
-};
-
-// Two independent batches share one launch (blocks [0, b0.count) take the first).
-__global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int max_sweeps, int32_t* status) {
-  constexpr int NP = kMaxN, HP = kMaxN / 2;
-  const bool first = (int)blockIdx.x < b0.count;
-  const EigBatch& eb = first ? b0 : b1;
-  const int bi = first ? (int)blockIdx.x : (int)blockIdx.x - b0.count;
-  const int n = eb.n;
-  const double* Cin = eb.C;
-  const int64_t sC = eb.sC, sV = eb.sV, sL = eb.sL;
-  float* Vout = eb.V;
-  float* lam = eb.lam;
-  extern __shared__ double ms[];
-  double* M = ms;                 // column-major: column j at M + j * NP (during Cholesky: row-major R)
-  double* nrm = M + NP * NP;      // NP squared column norms
-  int* rank = reinterpret_cast<int*>(nrm + NP);
-  __shared__ int rotated;
-  __shared__ double sigma_s;
+// Right-looking Cholesky by 16-column blocks of the 128 x 128 array A (row stride LD): on
+// entry the lower triangle holds the matrix (identity on the padding, upper triangle zero),
+// on exit the blocks below the diagonal hold L (A = L L^T) and Dv the inverses of the
+// diagonal blocks of L (zero above their diagonal). The diagonal blocks then hold
+// T = L_kk^{-T} in their upper half (kKeepL = false) or L_kk in their lower half
+// (kKeepL = true). Warp 0 factors each diagonal block in registers (shuffle broadcasts,
+// CUDA's float64 reciprocal square root) and inverts it; the panel below is L21 = A21 L11^{-T}
+// (1 x 4 strips per thread); the trailing lower triangle takes the rank-16 update in 4 x 4
+// register tiles. A pivot not above floor_v is raised to it and sets *floored (pivots of
+// the n x n problem only). Called by all 512 threads of the block.
+constexpr int kCholLD = kMaxN + 1;
+template <bool kKeepL>
+__device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, double* Ls, double* Is, int n,
+                                            double floor_v, int* floored) {
+  constexpr int NP = kMaxN, LD = kCholLD, BS = 16, NBLK = NP / BS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const double* c_in = Cin + (int64_t)bi * sC;
-  // load C (upper triangle used), zero padding
-  for (int e = tid; e < NP * NP; e += 512) {
-    const int r = e >> 7, c = e & (NP - 1);
-    M[e] = (r < n && c < n) ? c_in[(int64_t)r * n + c] : 0.0;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    double tr = 0.0;
-    for (int i = 0; i < n; ++i) tr += fabs(M[i * NP + i]);
-    sigma_s = 1e-13 * (tr > 0.0 ? tr / n : 1.0);
-  }
-  __syncthreads();
-  const double sigma = sigma_s;
-  for (int i = tid; i < n; i += 512) M[i * NP + i] += sigma;
-  __syncthreads();
-  // right-looking Cholesky, upper factor R in the upper triangle (row-major)
-  for (int k = 0; k < n; ++k) {
-    if (tid == 0) {
-      const double d = M[k * NP + k];
-      M[k * NP + k] = d > sigma * 1e-3 ? sqrt(d) : sqrt(sigma * 1e-3);
-    }
-    __syncthreads();
-    const double rkk = M[k * NP + k];
-    for (int j = k + 1 + tid; j < n; j += 512) M[k * NP + j] /= rkk;
-    __syncthreads();
-    const int m = n - k - 1;
-    for (int e = tid; e < m * NP; e += 512) {
-      const int i = k + 1 + (e >> 7), j = e & (NP - 1);
-      if (j >= i && j < n) M[i * NP + j] -= M[k * NP + i] * M[k * NP + j];
-    }
-    __syncthreads();
-  }
-  // M = R^T column-major == R row-major with the strict lower part cleared
-  for (int e = tid; e < NP * NP; e += 512) {
-    const int r = e >> 7, c = e & (NP - 1);
-    if (c < r) M[e] = 0.0;
-  }
-  __syncthreads();
-  int sweep = 0;
-  for (; sweep < max_sweeps; ++sweep) {
-    if (tid == 0) rotated = 0;
-    __syncthreads();
-    int any = 0;
-    // lane = 8 grp + sub: the warp rotates four pairs at once, one per 8-lane group; sub-lane
-    // `sub` owns rows 16 sub .. 16 sub + 15 of both columns and visits its eight 16-byte chunks
-    // in an order rotated by `sub`, so the four groups' loads spread over all banks.
-    const int grp = lane >> 3, sub = lane & 7;
-    for (int r = 0; r < NP - 1; ++r) {
-      const int k = warp + 16 * grp;
-      const int p = tour_player(k, r), q = tour_player(NP - 1 - k, r);
-      double* mp = M + p * NP + 16 * sub;
-      double* mq = M + q * NP + 16 * sub;
-      double pv[16], qv[16];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int ch = (i + sub) & 7;
-        const double2 a2 = *reinterpret_cast<const double2*>(mp + 2 * ch);
-        const double2 b2 = *reinterpret_cast<const double2*>(mq + 2 * ch);
-        pv[2 * i] = a2.x; pv[2 * i + 1] = a2.y;
-        qv[2 * i] = b2.x; qv[2 * i + 1] = b2.y;
-      }
-      double a = 0.0, b = 0.0, g = 0.0;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        a = fma(pv[i], pv[i], a);
-        b = fma(qv[i], qv[i], b);
-        g = fma(pv[i], qv[i], g);
-      }
-      // reduce to the group's first lane, then broadcast: bit-identical sums in the group
-#pragma unroll
-      for (int o = 4; o > 0; o >>= 1) {
-        a += __shfl_down_sync(0xffffffffu, a, o, 8);
-        b += __shfl_down_sync(0xffffffffu, b, o, 8);
-        g += __shfl_down_sync(0xffffffffu, g, o, 8);
-      }
-      a = __shfl_sync(0xffffffffu, a, 0, 8);
-      b = __shfl_sync(0xffffffffu, b, 0, 8);
-      g = __shfl_sync(0xffffffffu, g, 0, 8);
-      const float gf = (float)g;
-      if (g * g > 1e-14 * (a * b) && gf != 0.0f) {
-        const float zeta = __fdividef((float)(b - a), 2.0f * gf);
-        const float az = fabsf(zeta);
-        const float t = az > 1e18f ? __fdividef(0.5f, zeta)
-                                   : copysignf(__fdividef(1.0f, az + sqrtf(1.0f + zeta * zeta)), zeta);
-        const float cf = rsqrtf(1.0f + t * t);
-        double c = (double)cf, sn = (double)(t * cf);
-        const double fix = 1.5 - 0.5 * (c * c + sn * sn);   // one Newton step: c^2 + s^2 = 1
-        c *= fix;
-        sn *= fix;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int ch = (i + sub) & 7;
-          double2 u, v;
-          u.x = c * pv[2 * i] - sn * qv[2 * i];
-          u.y = c * pv[2 * i + 1] - sn * qv[2 * i + 1];
-          v.x = sn * pv[2 * i] + c * qv[2 * i];
-          v.y = sn * pv[2 * i + 1] + c * qv[2 * i + 1];
-          *reinterpret_cast<double2*>(mp + 2 * ch) = u;
-          *reinterpret_cast<double2*>(mq + 2 * ch) = v;
-        }
-        any = 1;
-      }
-      __syncthreads();
-    }
-    if (any && lane == 0) rotated = 1;
-    __syncthreads();
-    if (!rotated) break;
-  }
-  if (sweep == max_sweeps && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
-  // column norms, descending order (zero padding sorts last)
-  for (int j = warp; j < NP; j += 16) {
-    const double* mj = M + j * NP + 4 * lane;
-    double a = mj[0] * mj[0] + mj[1] * mj[1] + mj[2] * mj[2] + mj[3] * mj[3];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (lane == 0) nrm[j] = a;
-  }
-  __syncthreads();
-  for (int i = tid; i < NP; i += 512) {
-    const double li = nrm[i];
-    int rk = 0;
-    for (int j = 0; j < NP; ++j) {
-      const double lj = nrm[j];
-      rk += (lj > li) || (lj == li && j < i);
-    }
-    rank[i] = rk;
-  }
-  __syncthreads();
-  float* vo = Vout + (int64_t)bi * sV;
-  for (int e = tid; e < n * NP; e += 512) {
-    const int c = e >> 7, r = e & (NP - 1);   // column c of M, row r
-    if (r >= n || rank[c] >= n) continue;
-    const double inv = nrm[c] > 0.0 ? 1.0 / sqrt(nrm[c]) : 0.0;
-    vo[(int64_t)r * n + rank[c]] = (float)(M[c * NP + r] * inv);
-  }
-  if (lam)
-    for (int c = tid; c < NP; c += 512)
-      if (rank[c] < n) lam[(int64_t)bi * sL + rank[c]] = (float)(nrm[c] - sigma);
-}
-
-// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
-// The n x n problem is embedded in a 128 x 128 one (identity on the padding) and blocked by 16.
-// With L = R^T (W = L L^T) and X = L^{-1}, R^{-1} = X^T. One shared 128 x 129 array holds L
-// in its lower triangle and T = X^T in its upper triangle; the diagonal blocks of L are not
-// needed once their inverses are formed, so T takes over their upper half.
-//  * Cholesky, right-looking by 16-column blocks: warp 0 factors the diagonal block in
-//    registers (shuffle broadcasts, CUDA's float64 reciprocal square root) and inverts it;
-//    the panel below is L21 = A21 L11^{-T} (1 x 4 strips per thread); the trailing lower
-//    triangle takes the rank-16 update in 4 x 4 register tiles. A pivot below a tiny floor
-//    is raised to it and flags ST_NOT_CONVERGED.
-//  * Inverse, right-looking block forward substitution of L X = I: X_k = L_kk^{-1} B_k, then
-//    B_i -= L_ik X_k for the block rows below (B = I initially, kept transposed in T).
-template <typename TW>
-__global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
-                                                  int64_t sR, double shift, int32_t* status) {
-  constexpr int NP = kMaxN, LD = kMaxN + 1, BS = 16, NBLK = NP / BS;
-  extern __shared__ double dm[];
-  double* A = dm;                          // NP x LD
-  double* Dv = A + NP * LD;                // NBLK x BS x BS: L_kk^{-1} (lower, zero above)
-  double* Pt = Dv + NBLK * BS * BS;        // BS x NP: the current panel, transposed
-  double* Ls = Pt + BS * NP;               // BS x (BS + 1): the current diagonal factor
-  double* Is = Ls + BS * (BS + 1);         // BS: 1 / L_kk diagonal
-  __shared__ double tr_s;
-  __shared__ int floored;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const TW* w = W + (int64_t)blockIdx.x * sW;
-  if (tid == 0) floored = 0;
-  // every load of W in flight before the first barrier (32 elements per thread)
-  TW wv[NP * NP / 512];
-#pragma unroll
-  for (int q = 0; q < NP * NP / 512; ++q) {
-    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
-    wv[q] = (c <= r && r < n) ? w[(int64_t)r * n + c] : (TW)0;
-  }
-  if (tid < 32) {
-    double t = 0.0;
-    for (int i = tid; i < n; i += 32) t += (double)w[(int64_t)i * n + i];
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_down_sync(0xffffffffu, t, o);
-    if (tid == 0) tr_s = t;
-  }
-  __syncthreads();
-  const double tr = tr_s;
-  const double add = shift * tr / n;
-  const double floor_v = 1e-30 + 1e-14 * (tr > 0 ? tr / n : 1.0);
-  // lower triangle from W plus the shift, identity on the padding; upper triangle zero
-#pragma unroll
-  for (int q = 0; q < NP * NP / 512; ++q) {
-    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
-    double v = (c <= r && r < n) ? (double)wv[q] + (r == c ? add : 0.0) : 0.0;
-    if (r >= n && r == c) v = 1.0;
-    A[r * LD + c] = v;
-  }
-  __syncthreads();
   for (int kb = 0; kb < NBLK; ++kb) {
     const int k0 = kb * BS;
     double* D = Dv + kb * BS * BS;
@@ -449,9 +227,10 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
 #pragma unroll
         for (int r = 0; r < BS; ++r) {
           D[r * BS + i] = x[r];
-          if (r >= i) A[(k0 + i) * LD + k0 + r] = x[r];   // T = X^T, upper half of the block
+          if (!kKeepL && r >= i) A[(k0 + i) * LD + k0 + r] = x[r];   // T = X^T, upper half of the block
+          if (kKeepL && r <= i) A[(k0 + i) * LD + k0 + r] = a[r];    // L_kk, lower half of the block
         }
-        if (fl && lane == 0) floored = 1;
+        if (fl && lane == 0) *floored = 1;
       }
     }
     __syncthreads();
@@ -513,6 +292,321 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
     }
     __syncthreads();
   }
+}
+
+// Eigenpairs of a batch of symmetric positive semi-definite n x n matrices C (n <= 128),
+// float64 input, by one-sided (Hestenes) Jacobi on a Cholesky factor:
+//   C + sigma I = M M^T (M = R^T, R the upper Cholesky factor, sigma = 1e-13 trace / n keeps
+//   the factorisation defined; it shifts every eigenvalue by sigma and leaves the vectors);
+//   column pairs (p, q) of M are rotated, M <- M J, until all columns are mutually orthogonal;
+//   then M = U Sigma, so the normalised columns are the eigenvectors of C and the squared
+//   column norms (minus sigma) its eigenvalues. No eigenvector matrix is accumulated.
+// M lives in shared memory in float64, column-major, padded with zero rows/columns to 128.
+// Each round of the circle-method tournament rotates 64 disjoint pairs:
+// the three dot products are warp-shuffle reductions; the rotation (Golub & Van Loan sec.
+// 8.6, one-sided Jacobi) uses zeta = (beta - alpha) / (2 gamma), t = sign(zeta) /
+// (|zeta| + sqrt(1 + zeta^2)), c = 1 / sqrt(1 + t^2), s = t c, computed in float32 and
+// renormalised in float64 by one Newton step so that c^2 + s^2 = 1 to ~1e-15. A pair rotates
+// when gamma^2 > 1e-14 alpha beta; a sweep with no rotation ends the solve. Each warp works on
+// four pairs of a round at once, eight lanes per pair (16 rows each), so the dot products need
+// only three shuffle steps.
+struct EigBatch {
+  const double* C;
+  int64_t sC;
+  float* V;
+  int64_t sV;
+  float* lam;
+  int64_t sL;
+  int n, count;
+};
+
+// Two independent batches share one launch (blocks [0, b0.count) take the first).
+__global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int max_sweeps, int32_t* status) {
+  constexpr int NP = kMaxN;
+  const bool first = (int)blockIdx.x < b0.count;
+  const EigBatch& eb = first ? b0 : b1;
+  const int bi = first ? (int)blockIdx.x : (int)blockIdx.x - b0.count;
+  const int n = eb.n;
+  const double* Cin = eb.C;
+  const int64_t sC = eb.sC, sV = eb.sV, sL = eb.sL;
+  float* Vout = eb.V;
+  float* lam = eb.lam;
+  extern __shared__ double ms[];
+  double* M = ms;                 // column-major: column j at M + j * NP (during Cholesky: row-major R)
+  double* nrm = M + NP * NP;      // NP squared column norms
+  int* rank = reinterpret_cast<int*>(nrm + NP);
+  __shared__ int rotated[2];
+  __shared__ double sigma_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const double* c_in = Cin + (int64_t)bi * sC;
+  // C + sigma I = L L^T by the blocked Cholesky (sigma = 1e-13 trace / n; pivots floored at
+  // 1e-3 sigma), in the padded row-major array A that overlays M
+  double* A = ms;                                  // NP x kCholLD
+  double* Dv = A + NP * kCholLD;
+  double* Pt = Dv + NP * 16;
+  double* Ls = Pt + 16 * NP;
+  double* Is = Ls + 16 * 17;
+  __shared__ int floored;
+  double cv[NP * NP / 512];
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+    cv[q] = (c <= r && r < n) ? c_in[(int64_t)r * n + c] : 0.0;
+  }
+  if (tid < 32) {
+    double t = 0.0;
+    for (int i = tid; i < n; i += 32) t += fabs(c_in[(int64_t)i * n + i]);
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_down_sync(0xffffffffu, t, o);
+    if (tid == 0) {
+      sigma_s = 1e-13 * (t > 0.0 ? t / n : 1.0);
+      floored = 0;
+    }
+  }
+  __syncthreads();
+  const double sigma = sigma_s;
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+    double v = (c <= r && r < n) ? cv[q] + (r == c ? sigma : 0.0) : 0.0;
+    if (r >= n && r == c) v = 1.0;
+    A[r * kCholLD + c] = v;
+  }
+  __syncthreads();
+  chol_blocks<true>(A, Dv, Pt, Ls, Is, n, sigma * 1e-3, &floored);
+  // M = L column-major (column j of M is column j of L), padding columns zero
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, c = e >> 7, r = e & (NP - 1);
+    cv[q] = (r >= c && r < n && c < n) ? A[r * kCholLD + c] : 0.0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) M[tid + 512 * q] = cv[q];
+  __syncthreads();
+  // ---- sweeps with the columns in registers. Warp w holds the tournament slots 4w .. 4w + 3;
+  // slot k pairs position k (top) with position 127 - k (bottom), and position j starts with
+  // column j. Lane l holds rows l, l + 32, l + 64, l + 96 of its 8 columns.
+  constexpr int RPL = NP / 32;
+  double top[4][RPL], bot[4][RPL];
+#pragma unroll
+  for (int s = 0; s < 4; ++s)
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+      top[s][i] = M[(4 * warp + s) * NP + lane + 32 * i];
+      bot[s][i] = M[(NP - 1 - 4 * warp - s) * NP + lane + 32 * i];
+    }
+  __syncthreads();
+  // column exchange at the warp boundaries, double-buffered by round parity (reuses M)
+  double* XT = M;                    // [2][16][NP]: top of slot 4w + 3 handed to warp w + 1
+  double* XB = M + 2 * 16 * NP;      // [2][16][NP]: bottom of slot 4w handed to warp w - 1
+  const int gbase = lane & ~7;
+  const int l4 = (lane >> 4) & 1, l3 = (lane >> 3) & 1, l2 = (lane >> 2) & 1, l1 = (lane >> 1) & 1;
+  // rotated[sweep & 1] collects this sweep's flag; the other entry is reset for the next
+  // sweep while nobody reads it
+  if (tid == 0) rotated[0] = rotated[1] = 0;
+  __syncthreads();
+  int sweep = 0;
+  for (; sweep < max_sweeps; ++sweep) {
+    int any = 0;
+    for (int r = 0; r < NP - 1; ++r) {
+      // partial (alpha, beta, gamma) of the four slots over this lane's rows: v[4 s + q]
+      double v[16];
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        double a = 0.0, b = 0.0, g = 0.0;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+          a = fma(top[s][i], top[s][i], a);
+          b = fma(bot[s][i], bot[s][i], b);
+          g = fma(top[s][i], bot[s][i], g);
+        }
+        v[4 * s] = a;
+        v[4 * s + 1] = b;
+        v[4 * s + 2] = g;
+        v[4 * s + 3] = 0.0;
+      }
+      // transposed butterfly: each step halves the values a lane keeps; afterwards lanes
+      // 2m, 2m + 1 hold the full sum of value 8 l4 + 4 l3 + 2 l2 + l1 (identical in both)
+      double w8[8], w4[4], w2[2];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const double keep = l4 ? v[i + 8] : v[i], send = l4 ? v[i] : v[i + 8];
+        w8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const double keep = l3 ? w8[i + 4] : w8[i], send = l3 ? w8[i] : w8[i + 4];
+        w4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const double keep = l2 ? w4[i + 2] : w4[i], send = l2 ? w4[i] : w4[i + 2];
+        w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+      double w1;
+      {
+        const double keep = l1 ? w2[1] : w2[0], send = l1 ? w2[0] : w2[1];
+        w1 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+      const double tot = w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
+      // the 8 lanes of group `grp` hold slot grp: alpha at +0, beta at +2, gamma at +4
+      const double a = __shfl_sync(0xffffffffu, tot, gbase);
+      const double b = __shfl_sync(0xffffffffu, tot, gbase + 2);
+      const double g = __shfl_sync(0xffffffffu, tot, gbase + 4);
+      double c = 1.0, sn = 0.0;
+      const float gf = (float)g;
+      if (g * g > 1e-14 * (a * b) && gf != 0.0f) {
+        const float zeta = __fdividef((float)(b - a), 2.0f * gf);
+        const float az = fabsf(zeta);
+        const float t = az > 1e18f ? __fdividef(0.5f, zeta)
+                                   : copysignf(__fdividef(1.0f, az + sqrtf(1.0f + zeta * zeta)), zeta);
+        const float cf = rsqrtf(1.0f + t * t);
+        c = (double)cf;
+        sn = (double)(t * cf);
+        const double fix = 1.5 - 0.5 * (c * c + sn * sn);   // one Newton step: c^2 + s^2 = 1
+        c *= fix;
+        sn *= fix;
+        any = 1;
+      }
+      // rotate every slot with its group's (c, s); (1, 0) leaves a pair unchanged exactly
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const double cs = __shfl_sync(0xffffffffu, c, 8 * s);
+        const double ss = __shfl_sync(0xffffffffu, sn, 8 * s);
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+          const double p = top[s][i], q = bot[s][i];
+          top[s][i] = cs * p - ss * q;
+          bot[s][i] = ss * p + cs * q;
+        }
+      }
+      // next round of the circle tournament: position 0 stays, positions 1 .. 127 advance by
+      // one. Tops move to the next slot, bottoms to the previous; slot 0's bottom becomes
+      // slot 1's top and slot 63's top becomes its own bottom.
+      const int par = r & 1;
+      double* xt = XT + (par * 16 + warp) * NP;
+      double* xb = XB + (par * 16 + warp) * NP;
+#pragma unroll
+      for (int i = 0; i < RPL; ++i) {
+        if (warp < 15) xt[lane + 32 * i] = top[3][i];
+        if (warp > 0) xb[lane + 32 * i] = bot[0][i];
+      }
+      __syncthreads();
+      const double* xin_t = XT + (par * 16 + (warp > 0 ? warp - 1 : 0)) * NP;
+      const double* xin_b = XB + (par * 16 + (warp < 15 ? warp + 1 : 15)) * NP;
+#pragma unroll
+      for (int i = 0; i < RPL; ++i) {
+        const double t3 = top[3][i], b0 = bot[0][i];
+        top[3][i] = top[2][i];
+        top[2][i] = top[1][i];
+        top[1][i] = warp == 0 ? b0 : top[0][i];
+        if (warp > 0) top[0][i] = xin_t[lane + 32 * i];
+        bot[0][i] = bot[1][i];
+        bot[1][i] = bot[2][i];
+        bot[2][i] = bot[3][i];
+        bot[3][i] = warp < 15 ? xin_b[lane + 32 * i] : t3;
+      }
+    }
+    if (any) rotated[sweep & 1] = 1;
+    if (tid == 0) rotated[(sweep + 1) & 1] = 0;
+    __syncthreads();
+    if (!rotated[sweep & 1]) break;
+  }
+  if (sweep == max_sweeps && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
+  // after whole sweeps every column is back at its starting position
+#pragma unroll
+  for (int s = 0; s < 4; ++s)
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+      M[(4 * warp + s) * NP + lane + 32 * i] = top[s][i];
+      M[(NP - 1 - 4 * warp - s) * NP + lane + 32 * i] = bot[s][i];
+    }
+  __syncthreads();
+  // column norms, descending order (zero padding sorts last)
+  for (int j = warp; j < NP; j += 16) {
+    const double* mj = M + j * NP + 4 * lane;
+    double a = mj[0] * mj[0] + mj[1] * mj[1] + mj[2] * mj[2] + mj[3] * mj[3];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) nrm[j] = a;
+  }
+  __syncthreads();
+  for (int i = tid; i < NP; i += 512) {
+    const double li = nrm[i];
+    int rk = 0;
+    for (int j = 0; j < NP; ++j) {
+      const double lj = nrm[j];
+      rk += (lj > li) || (lj == li && j < i);
+    }
+    rank[i] = rk;
+  }
+  __syncthreads();
+  float* vo = Vout + (int64_t)bi * sV;
+  for (int e = tid; e < n * NP; e += 512) {
+    const int c = e >> 7, r = e & (NP - 1);   // column c of M, row r
+    if (r >= n || rank[c] >= n) continue;
+    const double inv = nrm[c] > 0.0 ? 1.0 / sqrt(nrm[c]) : 0.0;
+    vo[(int64_t)r * n + rank[c]] = (float)(M[c * NP + r] * inv);
+  }
+  if (lam)
+    for (int c = tid; c < NP; c += 512)
+      if (rank[c] < n) lam[(int64_t)bi * sL + rank[c]] = (float)(nrm[c] - sigma);
+}
+
+// Rinv = R^{-1} with R^T R = W + shift * (trace(W) / n) I (R upper triangular), float64.
+// The n x n problem is embedded in a 128 x 128 one (identity on the padding) and blocked by 16.
+// With L = R^T (W = L L^T) and X = L^{-1}, R^{-1} = X^T. One shared 128 x 129 array holds L
+// in its lower triangle and T = X^T in its upper triangle; the diagonal blocks of L are not
+// needed once their inverses are formed, so T takes over their upper half.
+//  * Cholesky, right-looking by 16-column blocks: warp 0 factors the diagonal block in
+//    registers (shuffle broadcasts, CUDA's float64 reciprocal square root) and inverts it;
+//    the panel below is L21 = A21 L11^{-T} (1 x 4 strips per thread); the trailing lower
+//    triangle takes the rank-16 update in 4 x 4 register tiles. A pivot below a tiny floor
+//    is raised to it and flags ST_NOT_CONVERGED.
+//  * Inverse, right-looking block forward substitution of L X = I: X_k = L_kk^{-1} B_k, then
+//    B_i -= L_ik X_k for the block rows below (B = I initially, kept transposed in T).
+template <typename TW>
+__global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
+                                                  int64_t sR, double shift, int32_t* status) {
+  constexpr int NP = kMaxN, LD = kMaxN + 1, BS = 16, NBLK = NP / BS;
+  extern __shared__ double dm[];
+  double* A = dm;                          // NP x LD
+  double* Dv = A + NP * LD;                // NBLK x BS x BS: L_kk^{-1} (lower, zero above)
+  double* Pt = Dv + NBLK * BS * BS;        // BS x NP: the current panel, transposed
+  double* Ls = Pt + BS * NP;               // BS x (BS + 1): the current diagonal factor
+  double* Is = Ls + BS * (BS + 1);         // BS: 1 / L_kk diagonal
+  __shared__ double tr_s;
+  __shared__ int floored;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const TW* w = W + (int64_t)blockIdx.x * sW;
+  if (tid == 0) floored = 0;
+  // every load of W in flight before the first barrier (32 elements per thread)
+  TW wv[NP * NP / 512];
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+    wv[q] = (c <= r && r < n) ? w[(int64_t)r * n + c] : (TW)0;
+  }
+  if (tid < 32) {
+    double t = 0.0;
+    for (int i = tid; i < n; i += 32) t += (double)w[(int64_t)i * n + i];
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_down_sync(0xffffffffu, t, o);
+    if (tid == 0) tr_s = t;
+  }
+  __syncthreads();
+  const double tr = tr_s;
+  const double add = shift * tr / n;
+  const double floor_v = 1e-30 + 1e-14 * (tr > 0 ? tr / n : 1.0);
+  // lower triangle from W plus the shift, identity on the padding; upper triangle zero
+#pragma unroll
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+    double v = (c <= r && r < n) ? (double)wv[q] + (r == c ? add : 0.0) : 0.0;
+    if (r >= n && r == c) v = 1.0;
+    A[r * LD + c] = v;
+  }
+  __syncthreads();
+  chol_blocks<false>(A, Dv, Pt, Ls, Is, n, floor_v, &floored);
   if (floored && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
   // Inverse. B (transposed in the upper triangle, zero off the diagonal blocks) -> X^T.
   for (int kb = 0; kb < NBLK; ++kb) {
@@ -604,7 +698,9 @@ cudaError_t eig_psd2(int batch0, int n0, const double* C0, int64_t sC0, float* V
                      float* lam1, int64_t sL1, int max_sweeps, int32_t* status, cudaStream_t s) {
   if (n0 <= 0 || n0 > kMaxN || (batch1 > 0 && (n1 <= 0 || n1 > kMaxN))) return cudaErrorInvalidValue;
   if (batch0 + batch1 <= 0) return cudaSuccess;
-  const size_t smem = ((size_t)kMaxN * kMaxN + kMaxN) * sizeof(double) + kMaxN * sizeof(int);
+  // the blocked Cholesky's arrays (A, diagonal inverses, panel, diagonal factor) overlay M,
+  // the column norms and the ranks
+  const size_t smem = ((size_t)kMaxN * kCholLD + 8 * 256 + 16 * kMaxN + 16 * 17 + 16) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_eig_psd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   EigBatch b0{C0, sC0, V0, sV0, lam0, sL0, n0, batch0};

@@ -133,15 +133,20 @@ __global__ void k_relfrob_part(uint64_t n, const T* a, const T* b, double* part)
   }
 }
 
+// Sum of the per-block partials: one block, each thread a fixed strided subset, then the
+// fixed block tree (deterministic).
 __global__ void k_relfrob_final(int nb, const double* part, double* out2) {
-  if (threadIdx.x == 0 && blockIdx.x == 0) {
-    double d = 0.0, r = 0.0;
-    for (int i = 0; i < nb; ++i) {
-      d += part[2 * i];
-      r += part[2 * i + 1];
-    }
-    out2[0] = d;
-    out2[1] = r;
+  __shared__ double red[32];
+  double d = 0.0, r = 0.0;
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    d += part[2 * i];
+    r += part[2 * i + 1];
+  }
+  const double td = block_sum(d, red);
+  const double tr = block_sum(r, red);
+  if (threadIdx.x == 0) {
+    out2[0] = td;
+    out2[1] = tr;
   }
 }
 
@@ -253,7 +258,7 @@ cudaError_t relfrob_partial(const void* ref, const void* approx, uint64_t n, Ele
     k_relfrob_part<float><<<nblocks, 256, 0, s>>>(n, (const float*)ref, (const float*)approx,
                                                   partials);
   note_launch();
-  k_relfrob_final<<<1, 32, 0, s>>>(nblocks, partials, out2);
+  k_relfrob_final<<<1, 256, 0, s>>>(nblocks, partials, out2);
   note_launch();
   return cudaGetLastError();
 }
