@@ -229,6 +229,30 @@ def config_dict(cfg, args):
 
 
 # ------------------------------------------------------------------ work models for the roofline
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, median of five launches)
+# of the kernel behind a phase, from the ncu launch list of this workload, with the first 16
+# hex digits of the sha256 of the kernel's source file when it was captured: reported only
+# while that file is unchanged (profiles/launch_list_c1_mistral7b_2x_sketch.md).
+NCU_TRAFFIC = {
+    "jacobi": ("tensor_decomposition_b200/csrc/kernels/jacobi.cu", "56af0dedd9b44373", 9_530_880),
+    "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "1be23e64cb8a6340", 178_881_280),
+    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "74e9f46a9cfaa1d6", 146_885_120),
+}
+
+
+def ncu_traffic(phase):
+    import hashlib
+    rec = NCU_TRAFFIC.get(phase)
+    if rec is None:
+        return None
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), rec[0])
+    try:
+        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return rec[2] if sha == rec[1] else None
+
+
 def phase_models(cfg, plan_info, alloc, ratio, peaks):
     """Algorithmic work of each traced phase per step (measurement section)."""
     H, T, D, L = cfg.heads, cfg.tokens, cfg.head_dim, cfg.layers
@@ -245,9 +269,8 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks):
                        for rt, rd, b in ranks)
     clock = peaks["sm_max_mhz"] * 1e6
     fp64_peak = 148 * 64 * 2 * clock / 1e12       # TFLOP/s, 64 FP64 FMA / clk / SM
-    fp32_peak = 148 * 128 * 2 * clock / 1e12      # TFLOP/s, 128 FP32 FMA / clk / SM
-    # CholeskyQR passes: 1 for Omega's and the transposed sketch's bases, 2 for the final one
-    cholqr_flops = n_lt * 4.0 * l * l * (1 * T + 1 * H * D + 2 * T)
+    # CholeskyQR passes: 1 for Omega's and the transposed sketch's bases, 3 for the final one
+    cholqr_flops = n_lt * 4.0 * l * l * (1 * T + 1 * H * D + 3 * T)
     resid_flops = sum(2.0 * N * (D + rt) for rt, rd, b in ranks if b > 0)
     dec_flops = sum(2.0 * N * (rt + (D if b else 0)) for rt, rd, b in ranks)
     return {
@@ -256,10 +279,10 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks):
         "feature_gram": dict(bound="tensor", work=2.0 * N * D * n_lt / 1e12, unit="TFLOP/s",
                              peak=peaks["bf16_tflops"], note="C_D = sum_h X_h^T X_h"),
         "residual": dict(bound="alu", work=resid_flops / 1e12, unit="TFLOP/s", peak=fp64_peak,
-                         note="float64 x Pi - u N per entry: 2 (D + r_t) flops; FP64 peak 148 SMs x 64 FMA x 2 x max clock"),
-        "decode": dict(bound="alu", work=dec_flops / 1e12, unit="TFLOP/s", peak=fp32_peak,
-                       note="float32 u M + y Pi^T per entry: 2 (r_t + D) flops; FP32 peak 148 x 128 FMA x 2 x max clock",
-                       hbm_bytes=2.0 * N * n_lt + stream_bytes),
+                         note="float64 x Pi - u N per entry: 2 (D + r_t) flops on the FP64 tensor-core MMA; "
+                              "FP64 peak 148 SMs x 64 FMA x 2 x max clock (the DMMA pipe reaches the same rate)"),
+        "decode": dict(bound="hbm", work=(2.0 * N * n_lt + stream_bytes) / 1e9, unit="GB/s", peak=peaks["hbm_gbs"],
+                       note="reads the stream, writes the bf16 cache: 2 N bytes per layer-tensor + stream bytes"),
         "jacobi": dict(bound="alu", work=9.0 * (D ** 3 + l ** 3) * n_lt / 1e12, unit="TFLOP/s", peak=fp64_peak,
                        note="feature (n = D) and sketch (n = l) symmetric eigenproblems with vectors, 9 n^3 flops "
                             "each (Golub & Van Loan count), float64 one-sided Jacobi: FP64 peak"),
@@ -379,7 +402,7 @@ def main():
     if m and m["work"] is not None:
         achieved = m["work"] / (per_launch_ms / 1e3)
         roof = {"kernel": name, "bound": m["bound"], "achieved": achieved, "peak": m["peak"], "unit": m["unit"],
-                "frac": achieved / m["peak"], "traffic": None,
+                "frac": achieved / m["peak"], "traffic": ncu_traffic(name),
                 "peak_source": peaks["source"] if m["bound"] != "alu" else "derived: SM count x FMA/clk x max clock",
                 "ms_per_launch": per_launch_ms, "note": m["note"]}
     phases = {k: round(v["total_ms"] / args.steps, 4) for k, v in prof.items()}
