@@ -8,6 +8,7 @@
 // feature factors, core at the largest ranks, truncation-energy table), the single
 // Lagrangian dual over all layer groups and both kinds, and the rotated low-bit residual.
 #include <algorithm>
+#include <array>
 #include <atomic>
 #include <mutex>
 #include <cmath>
@@ -212,6 +213,8 @@ struct jolt_plan_s {
   int64_t pool_budget[2] = {0, 0};
   std::vector<int32_t> lt_ids;   // buffer index i -> lt = 2*layer + kind (kind-major order)
   int32_t* d_lt_ids = nullptr;
+  int32_t* d_cand_order = nullptr;   // dual candidates in tie-break order (bytes, b, r_t, r_d)
+  std::vector<int32_t> cand_order;
   char* ws = nullptr;
   size_t ws_bytes = 0;
   // workspace views
@@ -527,6 +530,19 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   for (int i = 0; i < p->nbits; ++i)
     p->phi[i] = p->bits[i] == 0 ? 1.0 : p->kappa / (3.0 * std::pow(4.0, p->bits[i]));
   p->ngrid = 1 + (p->R / p->step) * (D / p->step);
+  {
+    // dual candidates c = bit index * ngrid + grid index, ordered by the tie-break key
+    const int ncand = p->nbits * p->ngrid, nJ = D / p->step;
+    std::vector<std::array<int64_t, 4>> key(ncand);
+    for (int c = 0; c < ncand; ++c) {
+      const int gi = c % p->ngrid, b = p->bits[c / p->ngrid];
+      const int rt = gi == 0 ? 0 : ((gi - 1) / nJ + 1) * p->step, rd = gi == 0 ? 0 : ((gi - 1) % nJ + 1) * p->step;
+      key[c] = {lt_bytes_h(H, T, D, rt, rd, b), b, rt, rd};
+    }
+    p->cand_order.resize(ncand);
+    for (int c = 0; c < ncand; ++c) p->cand_order[c] = c;
+    std::sort(p->cand_order.begin(), p->cand_order.end(), [&](int x, int y) { return key[x] < key[y]; });
+  }
   if (sh.has_v && cfg.split_kv_budget) {
     p->pool_budget[0] = (int64_t)(byte_budget / 2);
     p->pool_budget[1] = (int64_t)byte_budget - p->pool_budget[0];
@@ -613,6 +629,10 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess) e = cudaMalloc(&p->ws, p->ws_bytes);
   if (e == cudaSuccess) e = cudaMalloc(&p->d_lt_ids, sizeof(int32_t) * p->lt_ids.size());
+  if (e == cudaSuccess) e = cudaMalloc(&p->d_cand_order, sizeof(int32_t) * p->cand_order.size());
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->d_cand_order, p->cand_order.data(), sizeof(int32_t) * p->cand_order.size(),
+                   cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(p->d_lt_ids, p->lt_ids.data(), sizeof(int32_t) * p->lt_ids.size(), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
@@ -620,6 +640,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
                           "jolt_plan: workspace of %zu bytes: %s", p->ws_bytes, cudaGetErrorString(e));
     if (p->ws) cudaFree(p->ws);
     if (p->d_lt_ids) cudaFree(p->d_lt_ids);
+    if (p->d_cand_order) cudaFree(p->d_cand_order);
     delete p;
     return st;
   }
@@ -1095,6 +1116,7 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, ui
   for (int i = 0; i < 9; ++i) { da.bits[i] = p->bits[i]; da.phi[i] = p->phi[i]; }
   da.budget_pool[0] = p->pool_budget[0]; da.budget_pool[1] = p->pool_budget[1];
   da.ngrid = p->ngrid; da.E = p->E; da.unit_err = p->unit_err; da.meta = st->d_meta;
+  da.cand_order = p->d_cand_order;
   {
     PROF("dual", s);
     e = dual_allocate(da, s);
@@ -1555,6 +1577,7 @@ JOLT_API void jolt_plan_destroy(jolt_plan_t p) {
   cudaDeviceSynchronize();
   if (p->ws) cudaFree(p->ws);
   if (p->d_lt_ids) cudaFree(p->d_lt_ids);
+  if (p->d_cand_order) cudaFree(p->d_cand_order);
   delete p;
 }
 

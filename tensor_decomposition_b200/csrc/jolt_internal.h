@@ -128,6 +128,7 @@ struct DualArgs {
   int ngrid;
   const double* E;    // [2L][ngrid] (lt = 2*layer + kind)
   double* unit_err;   // [G*2][nbits*ngrid] debug copy of the tables
+  const int32_t* cand_order;   // [nbits*ngrid] candidates (bi * ngrid + grid) by (bytes, b, r_t, r_d)
   StreamMeta* meta;
 };
 cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s);

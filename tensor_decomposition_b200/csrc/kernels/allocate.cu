@@ -56,20 +56,6 @@ __global__ void k_energy_table(int H, int R, int D, int step, const float* Gmax,
   }
 }
 
-struct Cand {
-  double cost;
-  int64_t bytes;
-  int b, rt, rd, idx;
-};
-
-__device__ __forceinline__ bool less_key(const Cand& a, const Cand& b) {
-  if (a.cost != b.cost) return a.cost < b.cost;
-  if (a.bytes != b.bytes) return a.bytes < b.bytes;
-  if (a.b != b.b) return a.b < b.b;
-  if (a.rt != b.rt) return a.rt < b.rt;
-  return a.rd < b.rd;
-}
-
 __device__ __forceinline__ int64_t lt_bytes(int H, int T, int D, int rt, int rd, int b) {
   const int64_t tucker = 2 * ((int64_t)T * rt + (int64_t)D * rd + (int64_t)H * rt * rd);
   const int64_t resid = b > 0 ? (int64_t)H * T * (D * b / 8 + 2) : 0;
@@ -103,15 +89,20 @@ __global__ void k_unit_tables(DualArgs a) {
 
 constexpr size_t kDualSmem = 160 * 1024;
 
-// One CTA per budget pool, one warp per unit of the pool (units beyond the warp count are
-// taken in turn). A bisection step costs one barrier: every warp writes its unit's choice into
-// one of two alternating buffers, then all threads sum the bytes and move lo / hi identically.
+// One CTA per budget pool. The candidates come ranked by the tie-break key (bytes, b, r_t,
+// r_d), so a unit's choice at lambda is the smallest (cost, rank): each warp scans one unit's
+// candidates. The geometric bisection of lambda is evaluated three steps at a time: the seven
+// midpoints the next three steps can visit (a binary tree of intervals) are computed exactly as
+// the sequential search computes them and evaluated in parallel, then every thread walks the
+// tree with the sequential rule (termination test and step cap included). The result is
+// bit-identical to one bisection step per barrier, with a third of the barriers.
+constexpr int kTreeNodes = 7;      // three bisection levels
+
 __global__ void __launch_bounds__(1024) k_dual_pool(DualArgs a) {
   extern __shared__ unsigned char dsm[];
   __shared__ int slot_unit[kMaxUnits];
   __shared__ int slot_nlay[kMaxUnits];
-  __shared__ int64_t sbytes[2][kMaxUnits];
-  __shared__ int schoice[2][kMaxUnits];
+  __shared__ int schoice[2][kTreeNodes][kMaxUnits];
   __shared__ int nslot_s;
   __shared__ double esum_s;
   const int pool = blockIdx.x;
@@ -120,9 +111,13 @@ __global__ void __launch_bounds__(1024) k_dual_pool(DualArgs a) {
   const int ncand = a.nbits * a.ngrid;
   const int npools = (a.has_v && a.split) ? 2 : 1;
   StreamMeta* meta = a.meta;
-  int64_t* cbytes = reinterpret_cast<int64_t*>(dsm);                 // bytes per layer [ncand]
-  int* cattr = reinterpret_cast<int*>(cbytes + ncand);               // b | rt << 8 | rd << 20
-  double* err_s = reinterpret_cast<double*>(cattr + ((ncand + 1) & ~1));
+  // shared: rank -> bytes per layer (int64 and float64) and attributes, then the cached errors
+  int64_t* cb = reinterpret_cast<int64_t*>(dsm);                     // [ncand] by rank
+  double* cbd = reinterpret_cast<double*>(cb + ncand);               // [ncand] by rank
+  int* cattr = reinterpret_cast<int*>(cbd + ncand);                  // [ncand] b | rt << 8 | rd << 20
+  int* rank_of = cattr + ncand;                                      // [ncand] candidate -> rank
+  int* cand_of = rank_of + ncand;                                    // [ncand] rank -> candidate
+  double* err_s = reinterpret_cast<double*>(cand_of + ncand + (ncand & 1));   // [nslot][ncand] by rank
   if (tid == 0) {
     int ns = 0;
     for (int u = 0; u < nu; ++u) {
@@ -146,89 +141,121 @@ __global__ void __launch_bounds__(1024) k_dual_pool(DualArgs a) {
     }
     esum_s = esum;
   }
-  for (int c = tid; c < ncand; c += blockDim.x) {
+  // candidates in tie-break order (ranked on the host when the plan was made)
+  for (int r = tid; r < ncand; r += blockDim.x) {
+    const int c = a.cand_order[r];
     int rt, rd;
     grid_rank(c % a.ngrid, a.step, a.D, rt, rd);
     const int b = a.bits[c / a.ngrid];
-    cbytes[c] = lt_bytes(a.H, a.T, a.D, rt, rd, b);
-    cattr[c] = b | (rt << 8) | (rd << 20);
+    const int64_t by = lt_bytes(a.H, a.T, a.D, rt, rd, b);
+    rank_of[c] = r;
+    cand_of[r] = c;
+    cb[r] = by;
+    cbd[r] = (double)by;
+    cattr[r] = b | (rt << 8) | (rd << 20);
   }
   __syncthreads();
   const int nslot = nslot_s;
-  const size_t err_cap = (kDualSmem - (size_t)ncand * 12 - 16) / 8;
+  const size_t err_cap = (kDualSmem - (size_t)ncand * 32 - 16) / 8;
   const bool cached = (size_t)nslot * ncand <= err_cap;
   if (cached)
-    for (int e = tid; e < nslot * ncand; e += blockDim.x)
-      err_s[e] = a.unit_err[(int64_t)slot_unit[e / ncand] * ncand + e % ncand];
+    for (int e = tid; e < nslot * ncand; e += blockDim.x) {
+      const int us = e / ncand, c = e % ncand;
+      err_s[(size_t)us * ncand + rank_of[c]] = a.unit_err[(int64_t)slot_unit[us] * ncand + c];
+    }
   __syncthreads();
   const int64_t budget = a.budget_pool[pool];
-  // choices of every slot at lam into buffer `buf`; the caller synchronises
-  auto choose = [&](double lam, bool min_bytes_only, int buf) {
-    for (int us = warp; us < nslot; us += nwarps) {
-      const double* errp = cached ? err_s + (size_t)us * ncand : a.unit_err + (int64_t)slot_unit[us] * ncand;
-      const int64_t nl = slot_nlay[us];
-      Cand best;
-      best.cost = 0.0;
-      best.idx = -1;
-      for (int c = lane; c < ncand; c += 32) {
-        Cand x;
-        const int at = cattr[c];
-        x.b = at & 0xFF;
-        x.rt = (at >> 8) & 0xFFF;
-        x.rd = at >> 20;
-        x.bytes = nl * cbytes[c];
-        x.cost = min_bytes_only ? 0.0 : __dadd_rn(errp[c], __dmul_rn(lam, (double)x.bytes));
-        x.idx = c;
-        if (best.idx < 0 || less_key(x, best)) best = x;
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        Cand y;
-        y.cost = __shfl_down_sync(0xffffffffu, best.cost, o);
-        y.bytes = __shfl_down_sync(0xffffffffu, best.bytes, o);
-        y.b = __shfl_down_sync(0xffffffffu, best.b, o);
-        y.rt = __shfl_down_sync(0xffffffffu, best.rt, o);
-        y.rd = __shfl_down_sync(0xffffffffu, best.rd, o);
-        y.idx = __shfl_down_sync(0xffffffffu, best.idx, o);
-        if (y.idx >= 0 && (best.idx < 0 || less_key(y, best))) best = y;
-      }
-      if (lane == 0) {
-        sbytes[buf][us] = best.bytes;
-        schoice[buf][us] = best.idx;
+  // rank of the smallest (cost, rank) of slot us at lam; warp-collective, every lane returns it
+  auto choose_rank = [&](double lam, int us) -> int {
+    const double nl = (double)slot_nlay[us];
+    const double* ep = err_s + (size_t)us * ncand;
+    const double* eg = a.unit_err + (int64_t)slot_unit[us] * ncand;
+    double best = 0.0;
+    int bi = -1;
+    for (int r = lane; r < ncand; r += 32) {
+      const double e = cached ? ep[r] : eg[cand_of[r]];
+      const double cost = __dadd_rn(e, __dmul_rn(lam, __dmul_rn(nl, cbd[r])));
+      if (bi < 0 || cost < best) {
+        best = cost;
+        bi = r;
       }
     }
+    for (int o = 16; o > 0; o >>= 1) {
+      const double oc = __shfl_xor_sync(0xffffffffu, best, o);
+      const int ob = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob >= 0 && (bi < 0 || oc < best || (oc == best && ob < bi))) {
+        best = oc;
+        bi = ob;
+      }
+    }
+    return bi;
   };
-  auto total = [&](int buf) {
+  // choices of every slot at lams[0 .. nn) into buffer buf; the caller synchronises
+  auto evaluate = [&](const double* lams, int nn, int buf) {
+    for (int item = warp; item < nn * nslot; item += nwarps) {
+      const int node = item / nslot, us = item - node * nslot;
+      const int r = choose_rank(lams[node], us);
+      if (lane == 0) schoice[buf][node][us] = r;
+    }
+  };
+  auto total = [&](int buf, int node) {
     int64_t tb = 0;
-    for (int us = 0; us < nslot; ++us) tb += sbytes[buf][us];
+    for (int us = 0; us < nslot; ++us) tb += (int64_t)slot_nlay[us] * cb[schoice[buf][node][us]];
     return tb;
   };
   int buf = 0;
-  choose(0.0, true, buf);
-  __syncthreads();
-  const int64_t minb = total(buf);
   double lam = 0.0;
-  buf ^= 1;
+  bool use_min = false;
+  int64_t minb = 0;
+  for (int us = 0; us < nslot; ++us) minb += (int64_t)slot_nlay[us] * cb[0];
   if (minb > budget) {
     if (tid == 0) atomicOr(&meta->status, ST_INFEASIBLE);
-    buf ^= 1;   // keep the minimum-bytes choice
+    use_min = true;                       // keep the minimum-bytes choice
   } else {
-    choose(0.0, false, buf);
+    const double zero[1] = {0.0};
+    evaluate(zero, 1, buf);
     __syncthreads();
-    if (total(buf) > budget) {
+    if (total(buf, 0) > budget) {
       const double scale = __ddiv_rn(esum_s, (double)budget);
       double lo = __dmul_rn(1e-30, scale), hi = __dmul_rn(1e30, scale);
-      for (int it = 0; it < 200; ++it) {
-        if (!(__ddiv_rn(hi, lo) > 1.0 + 1e-15)) break;
-        const double mid = __dsqrt_rn(__dmul_rn(lo, hi));
+      int it = 0;
+      bool done = false;
+      while (!done) {
+        // the midpoints of the next three steps: node i has interval [nlo, nhi]; its left
+        // child follows a feasible midpoint ([nlo, mid]), its right child an infeasible one
+        double nlo[kTreeNodes], nhi[kTreeNodes], mid[kTreeNodes];
+        nlo[0] = lo;
+        nhi[0] = hi;
+#pragma unroll
+        for (int i = 0; i < kTreeNodes; ++i) {
+          mid[i] = __dsqrt_rn(__dmul_rn(nlo[i], nhi[i]));
+          if (2 * i + 2 < kTreeNodes) {
+            nlo[2 * i + 1] = nlo[i];
+            nhi[2 * i + 1] = mid[i];
+            nlo[2 * i + 2] = mid[i];
+            nhi[2 * i + 2] = nhi[i];
+          }
+        }
         buf ^= 1;
-        choose(mid, false, buf);
+        evaluate(mid, kTreeNodes, buf);
         __syncthreads();
-        if (total(buf) <= budget) hi = mid;
-        else lo = mid;
+        int node = 0;
+        for (int lvl = 0; lvl < 3; ++lvl) {
+          if (it >= 200 || !(__ddiv_rn(hi, lo) > 1.0 + 1e-15)) {
+            done = true;
+            break;
+          }
+          const bool feas = total(buf, node) <= budget;
+          if (feas) hi = mid[node];
+          else lo = mid[node];
+          ++it;
+          node = feas ? 2 * node + 1 : 2 * node + 2;
+        }
       }
       lam = hi;
       buf ^= 1;
-      choose(hi, false, buf);
+      const double at_hi[1] = {hi};
+      evaluate(at_hi, 1, buf);
       __syncthreads();
     }
   }
@@ -236,7 +263,7 @@ __global__ void __launch_bounds__(1024) k_dual_pool(DualArgs a) {
     meta->lambda[pool] = lam;
     for (int us = 0; us < nslot; ++us) {
       const int u = slot_unit[us];
-      const int at = cattr[schoice[buf][us]];
+      const int at = cattr[use_min ? 0 : schoice[buf][0][us]];
       meta->alloc[u / 2][u % 2][0] = (at >> 8) & 0xFFF;
       meta->alloc[u / 2][u % 2][1] = at >> 20;
       meta->alloc[u / 2][u % 2][2] = at & 0xFF;
@@ -322,8 +349,9 @@ cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k_dual_pool, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
   if (e != cudaSuccess) return e;
   const int npools = (a.has_v && a.split) ? 2 : 1;
-  int slots = a.has_v && !a.split ? 2 * a.G : a.G;
-  int threads = 32 * (slots < 32 ? slots : 32);
+  const int slots = a.has_v && !a.split ? 2 * a.G : a.G;
+  const int items = slots * kTreeNodes;
+  const int threads = 32 * (items < 32 ? items : 32);
   k_dual_pool<<<npools, threads, kDualSmem, s>>>(a);
   note_launch();
   k_layout<<<1, 1, 0, s>>>(a);

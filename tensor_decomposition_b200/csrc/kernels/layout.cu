@@ -10,23 +10,35 @@
 namespace jolt {
 namespace {
 
-// One 32 x 32 tile of X[l][h] (T x D) -> X^T[base + l][h] (D x T).
-__global__ void k_transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int H, int T, int D, int lt_base) {
-  __shared__ __nv_bfloat16 tile[32][33];
+// One 64 x 64 tile of X[l][h] (T x D) -> X^T[base + l][h] (D x T): 16-byte loads of 8
+// features, a shared tile, 16-byte stores of 8 tokens. T and D are multiples of 8.
+constexpr int kTT = 64, kTS = kTT + 8;   // tile edge, shared row stride (bf16)
+__global__ void __launch_bounds__(256) k_transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int H, int T, int D,
+                                                     int lt_base) {
+  __shared__ __align__(16) __nv_bfloat16 tile[kTT * kTS];
   const int lh = blockIdx.z;                   // l * H + h within this kind
-  const int t0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
+  const int t0 = blockIdx.x * kTT, d0 = blockIdx.y * kTT;
   const __nv_bfloat16* src = X + (int64_t)lh * T * D;
   const int l = lh / H, h = lh % H;
   __nv_bfloat16* dst = XT + ((int64_t)(lt_base + l) * H + h) * D * T;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-  for (int r = ty; r < 32; r += 8) {
-    const int t = t0 + r, d = d0 + tx;
-    if (t < T && d < D) tile[r][tx] = src[(int64_t)t * D + d];
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    const int q = threadIdx.x + 256 * v, r = q >> 3, c = q & 7;   // token row r, 8-feature chunk c
+    const int t = t0 + r, d = d0 + 8 * c;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (t < T && d < D) w = *reinterpret_cast<const uint4*>(src + (int64_t)t * D + d);
+    *reinterpret_cast<uint4*>(tile + r * kTS + 8 * c) = w;
   }
   __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int d = d0 + r, t = t0 + tx;
-    if (t < T && d < D) dst[(int64_t)d * T + t] = tile[tx][r];
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    const int q = threadIdx.x + 256 * v, r = q >> 3, c = q & 7;   // feature row r, 8-token chunk c
+    const int d = d0 + r, t = t0 + 8 * c;
+    if (d >= D || t >= T) continue;
+    __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = tile[(8 * c + j) * kTS + r];
+    *reinterpret_cast<uint4*>(dst + (int64_t)d * T + t) = *reinterpret_cast<const uint4*>(o);
   }
 }
 
@@ -106,7 +118,8 @@ int grid_for(int64_t n) {
 
 cudaError_t transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int L, int H, int T, int D, int lt_base,
                         cudaStream_t s) {
-  const dim3 g((T + 31) / 32, (D + 31) / 32, L * H);
+  if (T % 8 || D % 8) return cudaErrorInvalidValue;
+  const dim3 g((T + kTT - 1) / kTT, (D + kTT - 1) / kTT, L * H);
   k_transpose_x<<<g, 256, 0, s>>>(X, XT, H, T, D, lt_base);
   note_launch();
   return cudaGetLastError();
