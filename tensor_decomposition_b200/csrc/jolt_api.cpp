@@ -234,7 +234,11 @@ struct jolt_plan_s {
   float* Cpart = nullptr;            // [n][H][D][D] per-head Gram partials
   __nv_bfloat16* QTp[3] = {nullptr, nullptr, nullptr};   // bf16 parts of a float32 basis
   __nv_bfloat16* QNp[3] = {nullptr, nullptr, nullptr};   // the same parts, transposed layout
+  __nv_bfloat16* QTp2[3] = {nullptr, nullptr, nullptr};  // second part set (CholeskyQR ping-pong)
+  __nv_bfloat16* QNp2[3] = {nullptr, nullptr, nullptr};
   __nv_bfloat16* RTp[3] = {nullptr, nullptr, nullptr};   // parts of R^{-T} (CholeskyQR)
+  float* Wpart = nullptr;                                // K-chunk partial Grams (CholeskyQR)
+  int qset = 0;                                          // part set holding the final sketch basis
   float* Wf = nullptr;                                   // float32 CholeskyQR Grams
   __nv_bfloat16* UDt = nullptr;                          // U_D^T (rounded factor, exact in bf16)
   __nv_bfloat16* Pp[3] = {nullptr, nullptr, nullptr};    // bf16 parts of the core intermediate P
@@ -344,11 +348,11 @@ bool map_rows(CUtensorMap* m, const void* P, int64_t K, int64_t rows, int64_t ba
   return tc_map_bf16(m, P, 3, dims, str);
 }
 
-// [n][rows][chunks * 128] bf16 seen as (128, rows, chunks, n): one batch per (i, chunk), the
-// tile box spanning 64 entries of a chunk and 128 rows.
-bool map_kchunk(CUtensorMap* m, const void* P, int64_t rows, int64_t K, int64_t batch) {
-  const uint64_t dims[4] = {128, (uint64_t)rows, (uint64_t)(K / 128), (uint64_t)batch};
-  const uint64_t str[3] = {(uint64_t)K * 2, 256, (uint64_t)(rows * K * 2)};
+// [n][rows][K] bf16 with K = chunks * chunk, seen as (chunk, rows, chunks, n): one batch per
+// (i, chunk), the tile box spanning 64 entries of a chunk and 128 rows.
+bool map_kchunk(CUtensorMap* m, const void* P, int64_t rows, int64_t K, int64_t chunk, int64_t batch) {
+  const uint64_t dims[4] = {(uint64_t)chunk, (uint64_t)rows, (uint64_t)(K / chunk), (uint64_t)batch};
+  const uint64_t str[3] = {(uint64_t)K * 2, (uint64_t)chunk * 2, (uint64_t)(rows * K * 2)};
   return tc_map_bf16(m, P, 4, dims, str);
 }
 // [n][H][D][K] bf16 seen as (K, D, H, n): per-head row blocks.
@@ -357,6 +361,12 @@ bool map_perhead(CUtensorMap* m, const void* P, int64_t K, int64_t D, int64_t H,
   const uint64_t str[3] = {(uint64_t)K * 2, (uint64_t)(D * K * 2), (uint64_t)(H * D * K * 2)};
   return tc_map_bf16(m, P, 4, dims, str);
 }
+// Three bf16 parts of a float32 basis [n][l][rows]: in that layout (s) and transposed (t).
+struct PartSet {
+  __nv_bfloat16* s[3];
+  __nv_bfloat16* t[3];
+};
+
 // Products of two three-part operands kept for float32 accuracy: (0,0) (0,1) (1,0) (1,1) (0,2) (2,0).
 void six_products(TcGemmParams& g) {
   static const int8_t pa[6] = {0, 0, 1, 1, 0, 2}, pb[6] = {0, 1, 0, 1, 2, 0};
@@ -364,53 +374,74 @@ void six_products(TcGemmParams& g) {
   for (int i = 0; i < 6; ++i) { g.pair_a[i] = pa[i]; g.pair_b[i] = pb[i]; }
 }
 
-// CholeskyQR on the tensor cores, transposed layout Y^T [n][l][rows] -> Q^T. Each pass splits
-// Y into three bf16 parts (both layouts), forms the Gram W = Y^T Y from the six part products
-// of order <= 2 (float32 accumulation), inverts its Cholesky factor in float64, and forms
-// Q^T = R^{-T} Y^T from the six part products of R^{-T} and Y. Pass 1 adds 1e-6 trace(W) to
-// the diagonal (a shifted CholeskyQR step; the accumulation error of the Gram is ~1e-6), so the
-// factorisation exists for any sketch; the column space is unchanged by the shift.
-float* cholqr_tc(jolt_plan_s* p, int rows, float* bufA, float* bufB, int passes, int32_t* status, cudaStream_t s,
-                 jolt_status* st) {
+// Number of K chunks of a K-split Gram over `rows` entries: up to 16, each a whole number of
+// 8-element groups (TMA row-stride rule) and at least 256 long (a chunk's float32 partial Gram
+// should not outweigh the operand tiles it reads); 1 when rows does not split.
+int gram_chunks(int rows) {
+  for (int c = 16; c > 1; c /= 2)
+    if (rows % c == 0 && (rows / c) % 8 == 0 && rows / c >= 256) return c;
+  return 1;
+}
+
+// CholeskyQR on the tensor cores over bf16 parts. A basis Y^T [n][l][rows] is held as three
+// bf16 parts in its own layout (set.s) and transposed, [n][rows][l] (set.t). Each pass forms
+// the Gram W = Y^T Y from the six part products of order <= 2 as float32 partial sums over up to
+// 16 chunks of the rows (one CTA each), sums the chunks in float64, inverts its Cholesky
+// factor in float64, and forms Q^T = R^{-T} Y^T from the six part products of R^{-T} and Y,
+// whose epilogue writes Q's parts (both layouts) into the other set. Pass 1 adds 1e-6 trace(W)
+// to the diagonal (a shifted CholeskyQR step; the accumulation error of the Gram is ~1e-7), so
+// the factorisation exists for any sketch; the column space is unchanged by the shift.
+// Returns the index of the set that holds the result.
+int cholqr_tc(jolt_plan_s* p, int rows, PartSet* sets, int cur, int passes, int32_t* status, cudaStream_t s,
+              jolt_status* st) {
   const int l = p->l, n = p->n_lt;
-  float* src = bufA;
-  float* dst = bufB;
   *st = JOLT_OK;
   auto ck = [&](cudaError_t e) {
     if (e != cudaSuccess && *st == JOLT_OK) *st = fail(JOLT_ERR_CUDA, "cholqr: %s", cudaGetErrorString(e));
   };
-  static const int8_t pa[6] = {0, 0, 1, 1, 0, 2}, pb[6] = {0, 1, 0, 1, 2, 0};
+  const int nch = gram_chunks(rows);
   for (int pass = 0; pass < passes && *st == JOLT_OK; ++pass) {
-    ck(split_dual(n, l, rows, src, false, p->QTp, p->QNp, s));
+    const PartSet& in = sets[cur];
+    const PartSet& out = sets[cur ^ 1];
     TcGemmParams g;
     g.status = status;
     for (int i = 0; i < 3; ++i)
-      if (!map_rows(&g.amap[i], p->QTp[i], rows, l, n)) { *st = fail(JOLT_ERR_CUDA, "tensor map rejected"); return src; }
+      if (!map_kchunk(&g.amap[i], in.s[i], l, rows, rows / nch, n)) {
+        *st = fail(JOLT_ERR_CUDA, "tensor map rejected");
+        return cur;
+      }
+    g.av.mode = VIEW_XT_PERHEAD;      // (K chunk, rows, chunk, i)
+    g.av.H = nch;
     g.na = g.nb = 3;
     g.b_same = 1;
-    g.npairs = 6;
-    for (int i = 0; i < 6; ++i) { g.pair_a[i] = pa[i]; g.pair_b[i] = pb[i]; }
-    g.M = l; g.N = l; g.KB = (rows + 63) / 64;
-    g.C = p->Wf; g.c_sm = l; g.c_sn = 1; g.c_sb = (int64_t)l * l;
-    ck(gemm_tc(n, g, s));
-    ck(chol_inv_f32(n, l, p->Wf, (int64_t)l * l, p->Rinv, (int64_t)l * l, pass == 0 ? 1e-6 * l : 0.0, status, s));
+    six_products(g);
+    g.M = l; g.N = l; g.KB = (rows / nch + 63) / 64;
+    g.C = p->Wpart; g.c_sm = l; g.c_sn = 1; g.c_sb = (int64_t)l * l;
+    ck(gemm_tc(n * nch, g, s));
+    ck(sum_heads(n, nch, (int64_t)l * l, p->Wpart, nullptr, p->Wg, s));
+    ck(chol_inv(n, l, p->Wg, (int64_t)l * l, p->Rinv, (int64_t)l * l, pass == 0 ? 1e-6 * l : 0.0, status, s));
     ck(split_dual(n, l, l, p->Rinv, true, nullptr, p->RTp, s));
     TcGemmParams m;
     m.status = status;
     for (int i = 0; i < 3; ++i)
-      if (!map_rows(&m.amap[i], p->RTp[i], l, l, n) || !map_rows(&m.bmap[i], p->QNp[i], l, rows, n)) {
+      if (!map_rows(&m.amap[i], p->RTp[i], l, l, n) || !map_rows(&m.bmap[i], in.t[i], l, rows, n)) {
         *st = fail(JOLT_ERR_CUDA, "tensor map rejected");
-        return src;
+        return cur;
       }
     m.na = m.nb = 3;
-    m.npairs = 6;
-    for (int i = 0; i < 6; ++i) { m.pair_a[i] = pa[i]; m.pair_b[i] = pb[i]; }
+    six_products(m);
     m.M = l; m.N = rows; m.KB = (l + 63) / 64;
-    m.C = dst; m.c_sm = rows; m.c_sn = 1; m.c_sb = (int64_t)l * rows;
+    m.C = nullptr;
+    m.c_sm = rows; m.c_sn = 1; m.c_sb = (int64_t)l * rows;       // Q^T parts [l][rows]
+    m.t_sm = 1; m.t_sn = l; m.t_sb = (int64_t)rows * l;          // Q parts [rows][l]
+    for (int i = 0; i < 3; ++i) {
+      m.ps[i] = out.s[i];
+      m.pt[i] = out.t[i];
+    }
     ck(gemm_tc(n, m, s));
-    std::swap(src, dst);
+    cur ^= 1;
   }
-  return src;
+  return cur;
 }
 
 // CholeskyQR on the transposed layout: Y^T [n][l][rows] -> Q^T (same layout), passes as above.
@@ -600,8 +631,11 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
       if (p->encoder == JOLT_ENC_SKETCH) {
         for (int i = 0; i < 3; ++i) take(p->QTp[i], n * l * std::max<int64_t>(T, HD));
         for (int i = 0; i < 3; ++i) take(p->QNp[i], n * l * std::max<int64_t>(T, HD));
+        for (int i = 0; i < 3; ++i) take(p->QTp2[i], n * l * std::max<int64_t>(T, HD));
+        for (int i = 0; i < 3; ++i) take(p->QNp2[i], n * l * std::max<int64_t>(T, HD));
         for (int i = 0; i < 3; ++i) take(p->RTp[i], n * l * l);
         take(p->Wf, n * l * l);
+        take(p->Wpart, n * 16 * l * l);
       }
       take(p->UDt, n * D * D);
       for (int i = 0; i < 3; ++i) take(p->Pp[i], n * H * Rm * D);
@@ -759,13 +793,19 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, true, s));   // Omega^T [l][HD]
       }
       jolt_status r = JOLT_OK;
+      // two part sets: every basis lives as bf16 parts, written by the epilogue that makes it
+      PartSet sets[2];
+      for (int i = 0; i < 3; ++i) {
+        sets[0].s[i] = p->QTp[i]; sets[0].t[i] = p->QNp[i];
+        sets[1].s[i] = p->QTp2[i]; sets[1].t[i] = p->QNp2[i];
+      }
       auto tc_params = [&]() {
         TcGemmParams g;
         g.status = status;
         return g;
       };
-      // Y^T = (A Omega)^T or (A Q')^T: rows t, K = (h, d); transposed store into [l][T]
-      auto y_pass = [&](const __nv_bfloat16* const* bparts, int nparts, float* Yout) -> jolt_status {
+      // Y^T = (A Omega)^T or (A Q')^T: rows t, K = (h, d); parts of Y^T [l][T] and Y [T][l]
+      auto y_pass = [&](const __nv_bfloat16* const* bparts, int nparts, const PartSet& out) -> jolt_status {
         for (int k = 0; k < kinds; ++k) {
           TcGemmParams g = tc_params();
           g.amap[0] = mx[k];
@@ -776,68 +816,76 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
               return fail(JOLT_ERR_CUDA, "tensor map rejected");
           g.na = 1; g.nb = nparts;
           g.M = T; g.N = l; g.KB = (int)(HD / 64);
-          g.C = Yout + (int64_t)k * L * l * T; g.c_sm = 1; g.c_sn = T; g.c_sb = (int64_t)l * T;
+          g.C = nullptr;
+          g.c_sm = 1; g.c_sn = T; g.c_sb = (int64_t)l * T;
+          g.t_sm = l; g.t_sn = 1; g.t_sb = (int64_t)T * l;
+          for (int i = 0; i < 3; ++i) {
+            g.ps[i] = out.s[i] + (int64_t)k * L * l * T;
+            g.pt[i] = out.t[i] + (int64_t)k * L * l * T;
+          }
           CK(gemm_tc(L, g, s));
         }
         return JOLT_OK;
       };
+      int cur = 0;
       {
         PROF("sketch_gemm", s);
         const __nv_bfloat16* om[1] = {p->Om};
-        r = y_pass(om, 1, p->Y);
+        r = y_pass(om, 1, sets[cur]);
         if (r != JOLT_OK) return r;
       }
       const int q = p->cfg.power_iters;
-      float* Q;
       {
         PROF("cholqr", s);
-        Q = cholqr_tc(p, T, p->Y, p->Y2, q > 0 ? 1 : 3, status, s, &r);
+        cur = cholqr_tc(p, T, sets, cur, q > 0 ? 1 : 3, status, s, &r);
         if (r != JOLT_OK) return r;
       }
       for (int it = 0; it < q; ++it) {
         {
           PROF("sketch_gemm", s);
-          CK(split_bf16((int64_t)n * l * T, Q, p->QTp[0], p->QTp[1], nullptr, s));
-          // Z^T = (A^T Q)^T: rows (h, d), K = t; transposed store into [l][HD]
+          // Z^T = (A^T Q)^T: rows (h, d), K = t; parts of Z^T [l][HD] and Z [HD][l]
           TcGemmParams g = tc_params();
           g.amap[0] = mxt;
           g.av.mode = VIEW_XT_FEATROWS;
           g.av.D = D;
           for (int i = 0; i < 2; ++i)
-            if (!map_rows(&g.bmap[i], p->QTp[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+            if (!map_rows(&g.bmap[i], sets[cur].s[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
           g.na = 1; g.nb = 2;
           g.M = (int)HD; g.N = l; g.KB = (T + 63) / 64;
-          g.C = p->Z; g.c_sm = 1; g.c_sn = HD; g.c_sb = (int64_t)l * HD;
+          g.C = nullptr;
+          g.c_sm = 1; g.c_sn = HD; g.c_sb = (int64_t)l * HD;
+          g.t_sm = l; g.t_sn = 1; g.t_sb = (int64_t)HD * l;
+          for (int i = 0; i < 3; ++i) {
+            g.ps[i] = sets[cur ^ 1].s[i];
+            g.pt[i] = sets[cur ^ 1].t[i];
+          }
           CK(gemm_tc(n, g, s));
+          cur ^= 1;
         }
-        float* Qz;
         {
           PROF("cholqr", s);
-          Qz = cholqr_tc(p, (int)HD, p->Z, p->Z2, 1, status, s, &r);
+          cur = cholqr_tc(p, (int)HD, sets, cur, 1, status, s, &r);
           if (r != JOLT_OK) return r;
         }
-        float* Ydst = (Q == p->Y) ? p->Y2 : p->Y;
-        float* Yalt = (Q == p->Y) ? p->Y : p->Y2;
         {
           PROF("sketch_gemm", s);
-          CK(split_bf16((int64_t)n * l * HD, Qz, p->QTp[0], p->QTp[1], nullptr, s));
-          const __nv_bfloat16* qp[2] = {p->QTp[0], p->QTp[1]};
-          r = y_pass(qp, 2, Ydst);
+          const __nv_bfloat16* qp[2] = {sets[cur].s[0], sets[cur].s[1]};
+          r = y_pass(qp, 2, sets[cur ^ 1]);
           if (r != JOLT_OK) return r;
+          cur ^= 1;
         }
         {
           PROF("cholqr", s);
-          Q = cholqr_tc(p, T, Ydst, Yalt, it + 1 == q ? 3 : 1, status, s, &r);
+          cur = cholqr_tc(p, T, sets, cur, it + 1 == q ? 3 : 1, status, s, &r);
           if (r != JOLT_OK) return r;
         }
       }
       {
         PROF("sketch_gemm", s);
         // B = Q^T A (l x HD): rows j, K = t; Q^T in three bf16 parts for float32 accuracy
-        CK(split_bf16((int64_t)n * l * T, Q, p->QTp[0], p->QTp[1], p->QTp[2], s));
         TcGemmParams g = tc_params();
         for (int i = 0; i < 3; ++i)
-          if (!map_rows(&g.amap[i], p->QTp[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+          if (!map_rows(&g.amap[i], sets[cur].s[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
         g.bmap[0] = mxt;
         g.bv.mode = VIEW_XT_FEATROWS;
         g.bv.D = D;
@@ -846,7 +894,8 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         g.C = p->Bm; g.c_sm = HD; g.c_sn = 1; g.c_sb = (int64_t)l * HD;
         CK(gemm_tc(n, g, s));
       }
-      p->Qfinal = Q;
+      p->Qfinal = nullptr;
+      p->qset = cur;
     }
     if (p->encoder == JOLT_ENC_SKETCH && !p->use_tc) {
       const int l = p->l;
@@ -924,7 +973,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         TcGemmParams g;
         g.status = status;
         for (int i = 0; i < 3; ++i)
-          if (!map_kchunk(&g.amap[i], p->QTp[i], l, HD, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+          if (!map_kchunk(&g.amap[i], p->QTp[i], l, HD, 128, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
         g.av.mode = VIEW_XT_PERHEAD;      // (K, rows, chunk, i)
         g.av.H = nch;
         g.na = g.nb = 3;
@@ -943,13 +992,13 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       }
       {
         PROF("small_gemm", s);
-        // U_T = Q W[:, :R]: rows t, K = the sketch index; Q^T -> Q parts, W -> W^T parts
-        CK(split_dual(n, l, T, p->Qfinal, false, nullptr, p->QNp, s));
+        // U_T = Q W[:, :R]: rows t, K = the sketch index; Q parts [T][l] from CholeskyQR, W^T parts
         CK(split_dual(n, l, l, p->Wv, false, nullptr, p->RTp, s));
+        __nv_bfloat16* const* qn = p->qset ? p->QNp2 : p->QNp;
         TcGemmParams g;
         g.status = status;
         for (int i = 0; i < 3; ++i)
-          if (!map_rows(&g.amap[i], p->QNp[i], l, T, n) || !map_rows(&g.bmap[i], p->RTp[i], l, l, n))
+          if (!map_rows(&g.amap[i], qn[i], l, T, n) || !map_rows(&g.bmap[i], p->RTp[i], l, l, n))
             return fail(JOLT_ERR_CUDA, "tensor map rejected");
         g.na = g.nb = 3;
         six_products(g);

@@ -54,6 +54,81 @@ __device__ __forceinline__ void view_load(const TcView& v, const CUtensorMap* ma
   else tma_load_4d(dst, map, bar, c0, c1, c2, c3);
 }
 
+// bf16 parts of v at offset off: v = p0 + p1 + p2 (each remainder is exact in float32).
+__device__ __forceinline__ void put_parts(__nv_bfloat16* const (&P)[3], int64_t off, float v) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h0);
+  const __nv_bfloat16 h1 = __float2bfloat16_rn(r1);
+  P[0][off] = h0;
+  if (P[1]) P[1][off] = h1;
+  if (P[2]) P[2][off] = __float2bfloat16_rn(r1 - __bfloat162float(h1));
+}
+
+// Three bf16 parts of 8 floats (16 bytes per part).
+__device__ __forceinline__ void parts8(const float (&v)[8], uint4& h0, uint4& h1, uint4& h2) {
+  uint32_t w0[4], w1[4], w2[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float a[2], b[2], c[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float x = v[2 * i + k];
+      a[k] = __bfloat162float(__float2bfloat16_rn(x));
+      const float r1 = x - a[k];
+      b[k] = __bfloat162float(__float2bfloat16_rn(r1));
+      c[k] = r1 - b[k];
+    }
+    const __nv_bfloat162 pa = __floats2bfloat162_rn(a[0], a[1]), pb = __floats2bfloat162_rn(b[0], b[1]),
+                         pc = __floats2bfloat162_rn(c[0], c[1]);
+    w0[i] = *reinterpret_cast<const uint32_t*>(&pa);
+    w1[i] = *reinterpret_cast<const uint32_t*>(&pb);
+    w2[i] = *reinterpret_cast<const uint32_t*>(&pc);
+  }
+  h0 = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+  h1 = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  h2 = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+}
+
+// Parts of one warp's 32 x 32 chunk (staged as stg[m][n], row stride 33) into a layout with
+// unit stride along m (sm == 1) or along n (sn == 1): each lane stores 8 consecutive values
+// per part as one 16-byte vector (4 vectors per lane); other cases and ragged edges store
+// element by element.
+__device__ __forceinline__ void store_parts_chunk(__nv_bfloat16* const (&P)[3], int64_t off, int64_t sm, int64_t sn,
+                                                  const float* stg, int lane, int mrow0, int ncol0, int M, int N) {
+  const bool mcont = sm == 1, ncont = sn == 1 && !mcont;
+  const int64_t other = mcont ? sn : sm;
+  bool vec = (mcont || ncont) && (off % 8 == 0) && (other % 8 == 0);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) vec = vec && (!P[i] || (reinterpret_cast<uintptr_t>(P[i]) & 15) == 0);
+  const int q = lane & 3;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    // m-contiguous: column j = 8 pass + lane / 4, rows 8 q .. 8 q + 7
+    // n-contiguous: row r = 8 pass + lane / 4, columns 8 q .. 8 q + 7
+    const int a = 8 * pass + (lane >> 2);
+    const int mm0 = mcont ? mrow0 + 8 * q : mrow0 + a;
+    const int nn0 = mcont ? ncol0 + a : ncol0 + 8 * q;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = mcont ? stg[(8 * q + i) * 33 + a] : stg[a * 33 + 8 * q + i];
+    const bool full = mcont ? (nn0 < N && mm0 + 7 < M) : (mm0 < M && nn0 + 7 < N);
+    if (vec && full) {
+      uint4 h0, h1, h2;
+      parts8(v, h0, h1, h2);
+      const int64_t o = off + (int64_t)mm0 * sm + (int64_t)nn0 * sn;
+      *reinterpret_cast<uint4*>(P[0] + o) = h0;
+      if (P[1]) *reinterpret_cast<uint4*>(P[1] + o) = h1;
+      if (P[2]) *reinterpret_cast<uint4*>(P[2] + o) = h2;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int mm = mcont ? mm0 + i : mm0, nn = mcont ? nn0 : nn0 + i;
+        if (mm < M && nn < N) put_parts(P, off + (int64_t)mm * sm + (int64_t)nn * sn, v[i]);
+      }
+    }
+  }
+}
+
 template <int STAGES>
 __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGemmParams p) {
   extern __shared__ uint8_t smraw[];
@@ -155,30 +230,40 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
     int64_t boff;
     if (p.c_batch_in > 0) boff = (int64_t)(b / p.c_batch_in) * p.c_sb_out + (int64_t)(b % p.c_batch_in) * p.c_sb;
     else boff = (int64_t)b * p.c_sb;
-    float* C = p.C + boff;
-    // Row-major C (c_sn = 1): each 32 x 32 chunk goes through shared memory (the pipeline
-    // stages are free once the accumulator is complete) so that a store instruction writes
-    // 32 consecutive floats of one row instead of one float of 32 rows.
+    float* C = p.C ? p.C + boff : nullptr;
+    const int64_t poff = (int64_t)b * p.c_sb, toff = (int64_t)b * p.t_sb;
+    // Outputs contiguous along n (row-major C: c_sn = 1, or a part layout with unit n stride)
+    // go through shared memory in 32 x 32 chunks (the pipeline stages are free once the
+    // accumulator is complete), so that a store instruction covers consecutive n of one row;
+    // outputs contiguous along m are stored from the registers (consecutive lanes, consecutive m).
     float* stg = reinterpret_cast<float*>(smem) + e * (32 * 33);
-    const bool rowmajor = p.c_sn == 1;
+    const bool c_n = C && p.c_sn == 1, c_m = C && p.c_sn != 1;
+    const bool parts = p.ps[0] || p.pt[0];
 #pragma unroll 1
     for (int c = 0; c < kTile / 32; ++c) {
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(32 * e) << 16) + (uint32_t)(c * 32), r);
       tmem_ld_wait();
       if (!ok) continue;
-      if (rowmajor) {
+      if (c_n || parts) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
         __syncwarp();
-        const int n = n0 + c * 32 + lane;
+        if (c_n) {
+          const int n = n0 + c * 32 + lane;
 #pragma unroll 4
-        for (int rr = 0; rr < 32; ++rr) {
-          const int mm = m0 + 32 * e + rr;
-          if (mm < p.M && n < p.N) C[(int64_t)mm * p.c_sm + n] = stg[rr * 33 + lane];
+          for (int rr = 0; rr < 32; ++rr) {
+            const int mm = m0 + 32 * e + rr;
+            if (mm < p.M && n < p.N) C[(int64_t)mm * p.c_sm + n] = stg[rr * 33 + lane];
+          }
         }
+        if (p.ps[0])
+          store_parts_chunk(p.ps, poff, p.c_sm, p.c_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
+        if (p.pt[0])
+          store_parts_chunk(p.pt, toff, p.t_sm, p.t_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
         __syncwarp();
-      } else if (m < p.M) {
+      }
+      if (c_m && m < p.M) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int n = n0 + c * 32 + j;
@@ -240,6 +325,7 @@ cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
   for (int t = 0; t < p.npairs; ++t)
     if (p.pair_a[t] < 0 || p.pair_a[t] >= p.na || p.pair_b[t] < 0 || p.pair_b[t] >= p.nb) return cudaErrorInvalidValue;
   if (p.b_same && (p.M > kTile || p.N > kTile || p.nb > p.na)) return cudaErrorInvalidValue;
+  if ((p.ps[0] || p.pt[0]) && p.c_batch_in > 0) return cudaErrorInvalidValue;
   const int stage_bytes = (p.na + (p.b_same ? 0 : p.nb)) * kTileBytes;
   const dim3 g((p.N + kTile - 1) / kTile, (p.M + kTile - 1) / kTile, batch);
   if (stage_bytes * 4 + 1024 <= 200 * 1024) {

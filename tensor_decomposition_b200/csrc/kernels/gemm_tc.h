@@ -38,6 +38,12 @@ struct TcGemmParams {
   float* C = nullptr;       // C[b] + m * c_sm + n * c_sn
   int64_t c_sm = 0, c_sn = 0, c_sb = 0, c_sb_out = 0;
   int32_t c_batch_in = 0;   // > 0: batch offset = (b / c_batch_in) * c_sb_out + (b % c_batch_in) * c_sb
+  // Optional bf16 parts of the float32 result (v = p0 + p1 + p2, ~2^-24 relative), written in
+  // C's layout (ps[i] + b * c_sb + m * c_sm + n * c_sn) and/or a second layout (pt[i] + b * t_sb
+  // + m * t_sm + n * t_sn); null parts are skipped, C may be null. Not with c_batch_in.
+  __nv_bfloat16* ps[3] = {nullptr, nullptr, nullptr};
+  __nv_bfloat16* pt[3] = {nullptr, nullptr, nullptr};
+  int64_t t_sm = 0, t_sn = 0, t_sb = 0;
   int32_t* status = nullptr;
 };
 
