@@ -219,6 +219,19 @@ def run_reference(args):
     print(json.dumps(out))
 
 
+def job_throughput(local_ms, tokens, steps, world, device):
+    """Whole-job throughput of a weak-scaling run. Every rank processed `tokens` tokens per step
+    for `steps` steps; the job takes as long as its slowest rank (a MAX all-reduce over the
+    process group when world > 1). Returns (job milliseconds, tokens per second)."""
+    import torch
+    t = torch.tensor([float(local_ms)], device=device, dtype=torch.float64)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    return ms_max, tokens * steps * world / (ms_max / 1e3)
+
+
 def config_dict(cfg, args):
     return {"workload": f"{cfg.name} (Mistral-7B-v0.3 GQA KV shape), {args.ratio:g}x byte budget, "
                         f"{cfg.groups} layer groups, separate K/V budgets, {args.encoder} token factor",
@@ -360,13 +373,8 @@ def main():
     prof = J.jolt_profile_report()
     J.jolt_profile_enable(False)
     del st
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max, value = job_throughput(e0.elapsed_time(e1), cfg.tokens, args.steps, world, dev)
     ms_step = ms_max / args.steps
-    value = cfg.tokens * args.steps * world / (ms_max / 1e3)
 
     # ---- end to end through the public API with host buffers
     Kh = K.cpu().pin_memory()
@@ -386,10 +394,7 @@ def main():
     f1.record()
     barrier()
     del st
-    te = torch.tensor([f0.elapsed_time(f1)], device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = cfg.tokens * args.steps * world / (float(te.item()) / 1e3)
+    _, e2e_value = job_throughput(f0.elapsed_time(f1), cfg.tokens, args.steps, world, dev)
 
     # ---- roofline of the dominant phase
     peaks = measured_peaks()
