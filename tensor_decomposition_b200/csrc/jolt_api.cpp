@@ -27,6 +27,12 @@ using namespace jolt;
 
 namespace {
 
+// Power iterations that realise the exact token factor for T > 128 (subspace iteration on the
+// token Gram with a subspace of R + 16 columns). The slowest asserted eigenvectors sit at the
+// top of the noise bulk, where lambda_{l+1} / lambda_j ~ 0.57 per step: 16 steps left 5e-4 rad
+// against a dense eigensolver at T = 1024, 24 steps take it below 1e-5 rad.
+constexpr int kExactPowerIters = 24;
+
 thread_local std::string g_err;
 
 jolt_status fail(jolt_status st, const char* fmt, ...) {
@@ -239,6 +245,8 @@ struct jolt_plan_s {
   __nv_bfloat16* RTp[3] = {nullptr, nullptr, nullptr};   // parts of R^{-T} (CholeskyQR)
   float* Wpart = nullptr;                                // K-chunk partial Grams (CholeskyQR)
   int qset = 0;                                          // part set holding the final sketch basis
+  int q_iters = 1;                                       // power iterations of the subspace iteration
+  bool exact_by_iteration = false;                       // exact encoder realised by converged iteration
   float* Wf = nullptr;                                   // float32 CholeskyQR Grams
   __nv_bfloat16* UDt = nullptr;                          // U_D^T (rounded factor, exact in bf16)
   __nv_bfloat16* Pp[3] = {nullptr, nullptr, nullptr};    // bf16 parts of the core intermediate P
@@ -536,9 +544,14 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   p->R = (int)std::max<int64_t>(0, R);
   int enc = cfg.encoder;
   if (enc == JOLT_ENC_AUTO) enc = T <= 1024 ? JOLT_ENC_EXACT : JOLT_ENC_SKETCH;
+  p->q_iters = cfg.power_iters;
   if (enc == JOLT_ENC_EXACT && T > kMaxN) {
-    delete p;
-    return fail(JOLT_ERR_UNSUPPORTED, "jolt_plan: exact token factor needs tokens <= %d in this build", kMaxN);
+    // The token Gram is too large for one CTA's eigensolver: its leading eigenvectors come from
+    // block subspace iteration on C_T = A A^T, orthonormalised at every step, followed by the
+    // Rayleigh-Ritz step of the sketch path, run long enough to converge (kExactPowerIters).
+    p->exact_by_iteration = true;
+    p->q_iters = kExactPowerIters;
+    enc = JOLT_ENC_SKETCH;
   }
   p->encoder = enc;
   if (enc == JOLT_ENC_SKETCH) {
@@ -688,7 +701,7 @@ JOLT_API jolt_status jolt_plan_info(jolt_plan_t p, int32_t* rt_max, int32_t* ske
   if (!p) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan_info: null plan");
   if (rt_max) *rt_max = p->R;
   if (sketch_l) *sketch_l = p->encoder == JOLT_ENC_SKETCH ? p->l : 0;
-  if (encoder) *encoder = p->encoder;
+  if (encoder) *encoder = p->exact_by_iteration ? JOLT_ENC_EXACT : p->encoder;
   if (workspace_bytes) *workspace_bytes = p->ws_bytes;
   return JOLT_OK;
 }
@@ -698,7 +711,7 @@ static jolt_status make_stream(jolt_plan_s* p, uint64_t seed, cudaStream_t cs, j
   if (!st) return fail(JOLT_ERR_OOM, "stream: host allocation");
   const jolt_shape& sh = p->shape;
   st->L = sh.layers; st->H = sh.heads; st->T = sh.tokens; st->D = sh.head_dim;
-  st->has_v = sh.has_v ? 1 : 0; st->G = p->G; st->encoder = p->encoder; st->step = p->step;
+  st->has_v = sh.has_v ? 1 : 0; st->G = p->G; st->encoder = p->exact_by_iteration ? JOLT_ENC_EXACT : p->encoder; st->step = p->step;
   st->R = p->R; st->split = (sh.has_v && p->cfg.split_kv_budget) ? 1 : 0; st->dtype = sh.dtype;
   st->seed = seed; st->cs = cs; st->plan = p; st->n_lt = p->n_lt;
   st->body_cap = align_up((size_t)p->budget + (size_t)JOLT_NUM_PARTS * kAlign * p->n_lt + kAlign, kAlign);
@@ -834,7 +847,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         r = y_pass(om, 1, sets[cur]);
         if (r != JOLT_OK) return r;
       }
-      const int q = p->cfg.power_iters;
+      const int q = p->q_iters;
       {
         PROF("cholqr", s);
         cur = cholqr_tc(p, T, sets, cur, q > 0 ? 1 : 3, status, s, &r);
@@ -914,7 +927,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
                        opnd(p->Om + (int64_t)k * L * HD * l, EL_BF16, I1(HD * l), I1(1), I1(l)),
                        outd(p->Y + (int64_t)k * L * T * l, EL_F32, I1((int64_t)T * l), I1(l), I1(1)), 1.0, 0.0, s));
       }
-      const int q = p->cfg.power_iters;
+      const int q = p->q_iters;
       float* Q;
       {
         PROF("cholqr", s);

@@ -211,6 +211,18 @@ def test_exact_encode_parity_single_layer(J):
     print(r)
 
 
+def test_exact_encode_parity_config0_full(J):
+    cfg = synth.config(0)                          # 1 x 8 x 256 x 128, float32: token Gram 256 x 256
+    r = _parity(J, cfg, "exact", synth.bf16_bytes(cfg) // 2)
+    print(r)
+
+
+def test_exact_encode_parity_t1024(J):
+    cfg = synth.config(1, layers=2, seed=1404, groups=2)   # Mistral shape at T = 1024, exact token factor
+    r = _parity(J, cfg, "exact", synth.bf16_bytes(cfg) // 2)
+    print(r)
+
+
 def test_restricted_bits_and_joint_pool(J):
     cfg = synth.config(1, layers=3, tokens=136, seed=1303, groups=3, split_kv=False, bits=(1, 2, 3, 4))
     r = _parity(J, cfg, "sketch", synth.bf16_bytes(cfg) // 3)
