@@ -103,8 +103,9 @@ def serialize(st: OracleStream) -> bytes:
     return data + struct.pack("<I", zlib.crc32(data) & 0xFFFFFFFF)
 
 
-def parse(buf: bytes) -> OracleStream:
-    """Inverse of `serialize`; raises CorruptStream on a bad magic, version, size or CRC."""
+def parse(buf: bytes, lts=None) -> OracleStream:
+    """Inverse of `serialize`; raises CorruptStream on a bad magic, version, size or CRC.
+    `lts`: unpack only these layer-tensors (all when None); the whole buffer is still checked."""
     if len(buf) < 68 or buf[:4] != MAGIC:
         raise CorruptStream("bad magic or short buffer")
     _, ver, hb, flags = struct.unpack_from("<4sIII", buf, 0)
@@ -131,6 +132,8 @@ def parse(buf: bytes) -> OracleStream:
     body = memoryview(buf)[hb:hb + body_n]
     group_of = {l: g for g, lay in enumerate(group_ranges(L, G)) for l in lay}
     for lt, parts in layout.items():
+        if lts is not None and lt not in lts:
+            continue
         rt, rd, b = (int(v) for v in alloc[group_of[lt // KINDS]][lt % KINDS])
         raw = [np.frombuffer(body[o:o + s], dtype=np.uint8) for o, s in parts]
         U_T = bf16_from_bits(raw[0].view(np.uint16)).reshape(T, rt)

@@ -382,6 +382,18 @@ void six_products(TcGemmParams& g) {
   for (int i = 0; i < 6; ++i) { g.pair_a[i] = pa[i]; g.pair_b[i] = pb[i]; }
 }
 
+// K chunks of a long contraction over K entries: the fewest chunks of at most 2048 entries that
+// split K into whole 64-entry blocks; the tensor cores accumulate along one chunk in float32 and
+// the chunks are summed in float64 (a float32 accumulator chained over tens of thousands of
+// entries lost ~1e-3 rad of the leading token factors at T = 32768). 1 when K <= 2048 or when K
+// does not split that way.
+int k_chunks(int64_t K) {
+  if (K <= 2048) return 1;
+  for (int c = 2; c <= 64; ++c)
+    if (K % c == 0 && (K / c) % 64 == 0 && K / c <= 2048) return c;
+  return 1;
+}
+
 // Number of K chunks of a K-split Gram over `rows` entries: up to 16, each a whole number of
 // 8-element groups (TMA row-stride rule) and at least 256 long (a chunk's float32 partial Gram
 // should not outweigh the operand tiles it reads); 1 when rows does not split.
@@ -640,7 +652,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     take(p->Pib, (int64_t)D * D);
     if (p->use_tc) {
       take(p->XT, n * HD * T);
-      take(p->Cpart, n * H * D * D);
+      take(p->Cpart, n * H * D * D * k_chunks(T));   // per-head (and per K chunk) partials
       if (p->encoder == JOLT_ENC_SKETCH) {
         for (int i = 0; i < 3; ++i) take(p->QTp[i], n * l * std::max<int64_t>(T, HD));
         for (int i = 0; i < 3; ++i) take(p->QNp[i], n * l * std::max<int64_t>(T, HD));
@@ -764,11 +776,14 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
     g.av.mode = g.bv.mode = VIEW_XT_PERHEAD;
     g.av.H = g.bv.H = H;
     g.av.D = g.bv.D = D;
-    g.M = D; g.N = D; g.KB = (T + 63) / 64;
+    const int kc = k_chunks(T);
+    g.av.nch = g.bv.nch = kc;
+    g.av.ckb = g.bv.ckb = T / kc / 64;
+    g.M = D; g.N = D; g.KB = kc > 1 ? T / kc / 64 : (T + 63) / 64;
     g.C = p->Cpart; g.c_sm = D; g.c_sn = 1; g.c_sb = (int64_t)D * D;
     g.status = status;
-    CK(gemm_tc(n * H, g, s));
-    CK(sum_heads(n, H, (int64_t)D * D, p->Cpart, nullptr, p->CD, s));
+    CK(gemm_tc(n * H * kc, g, s));
+    CK(sum_heads(n, H * kc, (int64_t)D * D, p->Cpart, nullptr, p->CD, s));
   } else {
     PROF("feature_gram", s);
     // C_D = sum over rows r = (h, t) of X[r, :]^T X[r, :]
@@ -865,14 +880,26 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
             if (!map_rows(&g.bmap[i], sets[cur].s[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
           g.na = 1; g.nb = 2;
           g.M = (int)HD; g.N = l; g.KB = (T + 63) / 64;
-          g.C = nullptr;
           g.c_sm = 1; g.c_sn = HD; g.c_sb = (int64_t)l * HD;
-          g.t_sm = l; g.t_sn = 1; g.t_sb = (int64_t)HD * l;
-          for (int i = 0; i < 3; ++i) {
-            g.ps[i] = sets[cur ^ 1].s[i];
-            g.pt[i] = sets[cur ^ 1].t[i];
+          const int kc = k_chunks(T);
+          if (kc == 1) {
+            g.C = nullptr;
+            g.t_sm = l; g.t_sn = 1; g.t_sb = (int64_t)HD * l;
+            for (int i = 0; i < 3; ++i) {
+              g.ps[i] = sets[cur ^ 1].s[i];
+              g.pt[i] = sets[cur ^ 1].t[i];
+            }
+            CK(gemm_tc(n, g, s));
+          } else {
+            // long K: float32 partials per chunk of tokens, float64 sum, then the parts
+            g.av.nch = g.bv.nch = kc;
+            g.av.ckb = g.bv.ckb = T / kc / 64;
+            g.KB = T / kc / 64;
+            g.C = p->Cpart;
+            CK(gemm_tc(n * kc, g, s));
+            CK(sum_heads(n, kc, (int64_t)l * HD, p->Cpart, p->Z, nullptr, s));
+            CK(split_dual(n, l, (int)HD, p->Z, false, sets[cur ^ 1].s, sets[cur ^ 1].t, s));
           }
-          CK(gemm_tc(n, g, s));
           cur ^= 1;
         }
         {
@@ -904,8 +931,20 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         g.bv.D = D;
         g.na = 3; g.nb = 1;
         g.M = l; g.N = (int)HD; g.KB = (T + 63) / 64;
-        g.C = p->Bm; g.c_sm = HD; g.c_sn = 1; g.c_sb = (int64_t)l * HD;
-        CK(gemm_tc(n, g, s));
+        g.c_sm = HD; g.c_sn = 1; g.c_sb = (int64_t)l * HD;
+        const int kc = k_chunks(T);
+        if (kc == 1) {
+          g.C = p->Bm;
+          CK(gemm_tc(n, g, s));
+        } else {
+          // long K: float32 partials per chunk of tokens, summed in float64
+          g.av.nch = g.bv.nch = kc;
+          g.av.ckb = g.bv.ckb = T / kc / 64;
+          g.KB = T / kc / 64;
+          g.C = p->Cpart;
+          CK(gemm_tc(n * kc, g, s));
+          CK(sum_heads(n, kc, (int64_t)l * HD, p->Cpart, p->Bm, nullptr, s));
+        }
       }
       p->Qfinal = nullptr;
       p->qset = cur;

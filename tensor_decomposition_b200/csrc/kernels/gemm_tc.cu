@@ -28,6 +28,10 @@ constexpr uint32_t kMaxPoll = 1u << 22;
 
 __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, int b, int& c0, int& c1, int& c2,
                                             int& c3) {
+  if (v.nch > 1) {
+    kb += (b % v.nch) * v.ckb;
+    b /= v.nch;
+  }
   switch (v.mode) {
     case VIEW_X_TOKENROWS: {           // map (D, T, H, L): rows t, K = (h, d)
       const int kpd = v.D / kBK;

@@ -21,6 +21,10 @@ struct TcView {
   int32_t mode = VIEW_ROWS_K;
   int32_t D = 128;
   int32_t H = 1;   // VIEW_ROWS_K: batch index divisor (operands shared by H consecutive batches)
+  // K split: with nch > 1 the batch index is (b / nch, chunk = b % nch) and chunk covers the
+  // 64-entry K blocks [chunk * ckb, chunk * ckb + ckb) of the view
+  int32_t nch = 1;
+  int32_t ckb = 0;
 };
 
 struct TcGemmParams {

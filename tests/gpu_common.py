@@ -118,3 +118,44 @@ def oracle_lt_reconstruction(plan, X, seed, lt, rt, rd, b, Pi=None):
         s, c, _ = oj.quantize_rows(Y, b)
         rec = rec + np.einsum("hte,de->htd", oj.dequantize_rows(s, c, b), Pi)
     return oj.round_output(rec, plan.out_f32), a
+
+
+def check_allocation(J, st, ost, op, cfg):
+    """Budget and allocation checks that need only the GPU's exported tables: every pool within
+    its budget, the accounting formula equal to the stored array sizes, and the oracle's dual fed
+    the GPU's tables (and squared norms) reproducing the GPU's allocation exactly. Returns the
+    oracle units (one per group and kind)."""
+    kinds = (0, 1) if cfg.has_v else (0,)
+    info = J.jolt_stream_info(st, op.num_groups)
+    assert np.array_equal(info["alloc"], ost.alloc)
+    ranges = oj.group_ranges(cfg.layers, op.num_groups)
+    for kinds_p, bud in op.pools():
+        used = sum(oj.layer_bytes(cfg.heads, cfg.tokens, 128, *ost.alloc[g, k]) * len(lay)
+                   for g, lay in enumerate(ranges) for k in kinds_p)
+        assert used <= bud
+    total = 0
+    for g, lay in enumerate(ranges):
+        for k in kinds:
+            total += len(lay) * oj.layer_bytes(cfg.heads, cfg.tokens, 128, *(int(v) for v in ost.alloc[g, k]))
+    assert sum(info["bytes_by_part"].values()) == total
+    units = []
+    grid = op.grid()
+    for g, lay in enumerate(ranges):
+        for k in kinds:
+            tab = J.jolt_export_debug(st, J.JOLT_DBG_TABLE, 2 * g + k)
+            bb, rts, rds, nb = [], [], [], []
+            for b in op.bits:
+                for rt, rd in grid:
+                    bb.append(b), rts.append(rt), rds.append(rd)
+                    nb.append(len(lay) * oj.layer_bytes(cfg.heads, cfg.tokens, 128, rt, rd, b))
+            units.append(oj.Unit(g, k, tab, np.array(nb, dtype=np.int64), np.array(bb), np.array(rts),
+                                 np.array(rds), 0.0))
+    xx = J.jolt_export_debug(st, J.JOLT_DBG_XX)
+    for u in units:
+        e = 0.0
+        for l in ranges[u.group]:
+            e = e + xx[2 * l + u.kind]
+        u.energy = e
+    alloc_o, _ = oj.allocate(op, units)
+    assert np.array_equal(alloc_o, ost.alloc)
+    return units
