@@ -399,8 +399,9 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
   // column exchange at the warp boundaries, double-buffered by round parity (reuses M)
   double* XT = M;                    // [2][16][NP]: top of slot 4w + 3 handed to warp w + 1
   double* XB = M + 2 * 16 * NP;      // [2][16][NP]: bottom of slot 4w handed to warp w - 1
-  const int gbase = lane & ~7;
-  const int l4 = (lane >> 4) & 1, l3 = (lane >> 3) & 1, l2 = (lane >> 2) & 1, l1 = (lane >> 1) & 1;
+  double* XN = M + 4 * 16 * NP;      // [2][16][2]: the squared norms of those two columns
+  const int grp = lane >> 3;
+  const int l4 = (lane >> 4) & 1, l3 = (lane >> 3) & 1;
   // rotated[sweep & 1] collects this sweep's flag; the other entry is reset for the next
   // sweep while nobody reads it
   if (tid == 0) rotated[0] = rotated[1] = 0;
@@ -408,51 +409,61 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
   int sweep = 0;
   for (; sweep < max_sweeps; ++sweep) {
     int any = 0;
-    for (int r = 0; r < NP - 1; ++r) {
-      // partial (alpha, beta, gamma) of the four slots over this lane's rows: v[4 s + q]
-      double v[16];
+    // squared column norms of slot `grp` (top: na, bottom: nb), exact at the start of the
+    // sweep: per-lane partial sums, then butterflies over the 32 lanes
+    double na, nb;
+    {
+      double v[8];
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        double a = 0.0, b = 0.0, g = 0.0;
+        double a = 0.0, b = 0.0;
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
           a = fma(top[s][i], top[s][i], a);
           b = fma(bot[s][i], bot[s][i], b);
-          g = fma(top[s][i], bot[s][i], g);
         }
-        v[4 * s] = a;
-        v[4 * s + 1] = b;
-        v[4 * s + 2] = g;
-        v[4 * s + 3] = 0.0;
-      }
-      // transposed butterfly: each step halves the values a lane keeps; afterwards lanes
-      // 2m, 2m + 1 hold the full sum of value 8 l4 + 4 l3 + 2 l2 + l1 (identical in both)
-      double w8[8], w4[4], w2[2];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const double keep = l4 ? v[i + 8] : v[i], send = l4 ? v[i] : v[i + 8];
-        w8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        v[2 * s] = a;
+        v[2 * s + 1] = b;
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const double keep = l3 ? w8[i + 4] : w8[i], send = l3 ? w8[i] : w8[i + 4];
-        w4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v[j] += __shfl_xor_sync(0xffffffffu, v[j], o);
+      na = v[0];
+      nb = v[1];
+#pragma unroll
+      for (int s = 1; s < 4; ++s)
+        if (grp == s) {
+          na = v[2 * s];
+          nb = v[2 * s + 1];
+        }
+    }
+    for (int r = 0; r < NP - 1; ++r) {
+      // gamma of the four slots: per-lane partial sums, then a transposed butterfly that leaves
+      // slot grp's sum in the 8 lanes of group grp (identical in all of them)
+      double v[4];
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        double g = 0.0;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) g = fma(top[s][i], bot[s][i], g);
+        v[s] = g;
       }
+      double w2[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const double keep = l2 ? w4[i + 2] : w4[i], send = l2 ? w4[i] : w4[i + 2];
-        w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        const double keep = l4 ? v[i + 2] : v[i], send = l4 ? v[i] : v[i + 2];
+        w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
       }
-      double w1;
+      double g;
       {
-        const double keep = l1 ? w2[1] : w2[0], send = l1 ? w2[0] : w2[1];
-        w1 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        const double keep = l3 ? w2[1] : w2[0], send = l3 ? w2[0] : w2[1];
+        g = keep + __shfl_xor_sync(0xffffffffu, send, 8);
       }
-      const double tot = w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
-      // the 8 lanes of group `grp` hold slot grp: alpha at +0, beta at +2, gamma at +4
-      const double a = __shfl_sync(0xffffffffu, tot, gbase);
-      const double b = __shfl_sync(0xffffffffu, tot, gbase + 2);
-      const double g = __shfl_sync(0xffffffffu, tot, gbase + 4);
+      g += __shfl_xor_sync(0xffffffffu, g, 4);
+      g += __shfl_xor_sync(0xffffffffu, g, 2);
+      g += __shfl_xor_sync(0xffffffffu, g, 1);
+      const double a = na, b = nb;
       double c = 1.0, sn = 0.0;
       const float gf = (float)g;
       if (g * g > 1e-14 * (a * b) && gf != 0.0f) {
@@ -467,6 +478,10 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
         c *= fix;
         sn *= fix;
         any = 1;
+        // squared norms after p' = c p - s q, q' = s p + c q
+        const double cc = c * c, ss = sn * sn, cs2 = 2.0 * c * sn * g;
+        na = fma(cc, a, fma(ss, b, -cs2));
+        nb = fma(ss, a, fma(cc, b, cs2));
       }
       // rotate every slot with its group's (c, s); (1, 0) leaves a pair unchanged exactly
 #pragma unroll
@@ -482,7 +497,8 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
       }
       // next round of the circle tournament: position 0 stays, positions 1 .. 127 advance by
       // one. Tops move to the next slot, bottoms to the previous; slot 0's bottom becomes
-      // slot 1's top and slot 63's top becomes its own bottom.
+      // slot 1's top and slot 63's top becomes its own bottom. The squared norms move with
+      // their columns.
       const int par = r & 1;
       double* xt = XT + (par * 16 + warp) * NP;
       double* xb = XB + (par * 16 + warp) * NP;
@@ -491,6 +507,10 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
         if (warp < 15) xt[lane + 32 * i] = top[3][i];
         if (warp > 0) xb[lane + 32 * i] = bot[0][i];
       }
+      if (warp < 15 && lane == 24) XN[(par * 16 + warp) * 2] = na;        // top of slot 4w + 3
+      if (warp > 0 && lane == 0) XN[(par * 16 + warp) * 2 + 1] = nb;      // bottom of slot 4w
+      const double up_a = __shfl_up_sync(0xffffffffu, (warp == 0 && grp == 0) ? nb : na, 8);
+      const double dn_b = __shfl_down_sync(0xffffffffu, nb, 8);
       __syncthreads();
       const double* xin_t = XT + (par * 16 + (warp > 0 ? warp - 1 : 0)) * NP;
       const double* xin_b = XB + (par * 16 + (warp < 15 ? warp + 1 : 15)) * NP;
@@ -506,6 +526,10 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
         bot[2][i] = bot[3][i];
         bot[3][i] = warp < 15 ? xin_b[lane + 32 * i] : t3;
       }
+      const double na_new = grp >= 1 ? up_a : (warp == 0 ? na : XN[(par * 16 + warp - 1) * 2]);
+      const double nb_new = grp <= 2 ? dn_b : (warp < 15 ? XN[(par * 16 + warp + 1) * 2 + 1] : na);
+      na = na_new;
+      nb = nb_new;
     }
     if (any) rotated[sweep & 1] = 1;
     if (tid == 0) rotated[(sweep + 1) & 1] = 0;

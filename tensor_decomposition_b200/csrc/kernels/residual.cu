@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf
 // works on 256 tokens of one (layer-tensor, head) in tiles of 16 rows; warp w computes rows
 // 8 (w / 4) .. +7 and columns 32 (w % 4) .. +31 of the tile.
 __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
                : "+d"(d0), "+d"(d1)
                : "d"(a), "d"(b));
 }
@@ -87,7 +87,7 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
 constexpr int kRows = 16;          // rows per tile
 constexpr int kPS = 132;           // row stride (floats) of Pi^T: conflict-free fragment loads
 
-__global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* Nbuf, int R) {
+__global__ void __launch_bounds__(256, 1) k_residual(ResidualArgs a, const double* Nbuf, int R) {
   extern __shared__ __align__(16) unsigned char smraw[];
   const int chunk = blockIdx.x, h = blockIdx.y, i = blockIdx.z;
   const int lt = a.lt_ids[i];
@@ -125,63 +125,76 @@ __global__ void __launch_bounds__(256) k_residual(ResidualArgs a, const double* 
   const int c_first = (32 * lane) / b;                  // codes overlapping word `lane`
   const int c_last = min(D - 1, (32 * lane + 31) / b);
   __syncthreads();
-  for (int t0 = t_begin; t0 < t_end; t0 += kRows) {
-    // A tile: x rows (float64 of bf16 / float32) followed by u rows, 16-byte vector loads:
-    // thread (r = tid / 16, j = tid % 16) takes chunk j of row r (x) and chunk j of u (if any).
-    {
-      const int r = tid >> 4, j = tid & 15;
-      const int t = t0 + r;
-      double* dst = At + r * SA;
-      const bool live = t < t_end;
+  // A tile: x rows (float64 of bf16 / float32) followed by u rows from 16-byte vector loads;
+  // thread (r = tid / 16, j = tid % 16) takes chunk j of row r (x) and chunk j of u (if any).
+  // The next tile's loads are issued before the current tile's GEMM and land in registers.
+  const int fr = tid >> 4, fj = tid & 15;
+  uint4 px[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)}, pu = make_uint4(0, 0, 0, 0);
+  auto fetch = [&](int t0) {
+    const int t = t0 + fr;
+    const bool live = t < t_end;
+    px[0] = px[1] = pu = make_uint4(0, 0, 0, 0);
+    if (live) {
       if (a.xt == EL_BF16) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (live) v = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[j];
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          dst[8 * j + 2 * q] = (double)__uint_as_float(wv[q] << 16);
-          dst[8 * j + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
-        }
+        px[0] = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[fj];
       } else {
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (live) f = reinterpret_cast<const float4*>(x_row_ptr(a, lt, h, t))[2 * j + q];
-          dst[8 * j + 4 * q] = f.x; dst[8 * j + 4 * q + 1] = f.y;
-          dst[8 * j + 4 * q + 2] = f.z; dst[8 * j + 4 * q + 3] = f.w;
-        }
+        px[0] = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[2 * fj];
+        px[1] = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[2 * fj + 1];
       }
-      if (8 * j < rt) {                            // rt is a multiple of 16
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (live) v = *reinterpret_cast<const uint4*>(UT + (int64_t)t * rt + 8 * j);
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      if (8 * fj < rt) pu = *reinterpret_cast<const uint4*>(UT + (int64_t)t * rt + 8 * fj);   // rt: multiple of 16
+    }
+  };
+  auto stage = [&]() {
+    double* dst = At + fr * SA;
+    if (a.xt == EL_BF16) {
+      const uint32_t wv[4] = {px[0].x, px[0].y, px[0].z, px[0].w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          dst[D + 8 * j + 2 * q] = (double)__uint_as_float(wv[q] << 16);
-          dst[D + 8 * j + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
-        }
+      for (int q = 0; q < 4; ++q) {
+        dst[8 * fj + 2 * q] = (double)__uint_as_float(wv[q] << 16);
+        dst[8 * fj + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t wv[4] = {px[q].x, px[q].y, px[q].z, px[q].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[8 * fj + 4 * q + e] = (double)__uint_as_float(wv[e]);
       }
     }
+    if (8 * fj < rt) {
+      const uint32_t wv[4] = {pu.x, pu.y, pu.z, pu.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        dst[D + 8 * fj + 2 * q] = (double)__uint_as_float(wv[q] << 16);
+        dst[D + 8 * fj + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
+      }
+    }
+  };
+  fetch(t_begin);
+  for (int t0 = t_begin; t0 < t_end; t0 += kRows) {
+    stage();
     __syncthreads();
+    if (t0 + kRows < t_end) fetch(t0 + kRows);
     double acc[4][2];
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = 0.0;
     const double* arow = At + ar * SA + ak;
-#pragma unroll 4
-    for (int k0 = 0; k0 < D; k0 += 4) {
+    const float* pb = PT + (32 * cg + (lane >> 2)) * kPS + ak;    // fragment j at + 8 j kPS
+    const double* qb = NT + (32 * cg + (lane >> 2)) * SN + ak;
+    // K = D part (x Pi), fully unrolled so the fragment loads of later steps can be issued early
+#pragma unroll
+    for (int k0 = 0; k0 < kD; k0 += 4) {
       const double av = arow[k0];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = 32 * cg + 8 * j + (lane >> 2);
-        dmma_8x8x4(acc[j][0], acc[j][1], av, (double)PT[n * kPS + k0 + ak]);
-      }
+      for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[j][0], acc[j][1], av, (double)pb[8 * j * kPS + k0]);
     }
-    for (int k0 = 0; k0 < rt; k0 += 4) {
-      const double av = arow[D + k0];
+    // K = r_t part (-u N), four steps per unrolled block (r_t is a multiple of 16)
+    for (int k0 = 0; k0 < rt; k0 += 16) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = 32 * cg + 8 * j + (lane >> 2);
-        dmma_8x8x4(acc[j][0], acc[j][1], av, NT[n * SN + k0 + ak]);
+      for (int kk = 0; kk < 16; kk += 4) {
+        const double av = arow[kD + k0 + kk];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[j][0], acc[j][1], av, qb[8 * j * SN + k0 + kk]);
       }
     }
     __syncthreads();                                   // A no longer read: reuse it for y
