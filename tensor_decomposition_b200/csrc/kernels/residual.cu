@@ -30,47 +30,48 @@ __device__ __forceinline__ const void* x_row_ptr(const ResidualArgs& a, int lt, 
              : (const void*)(reinterpret_cast<const float*>(a.X[kind]) + off);
 }
 
-// N_h = (G_h U_D^T) Pi in float64 for one (layer-tensor, head); 16 rows of M at a time.
+// N_h = G_h (U_D^T Pi) in float64 for one (layer-tensor, head): P = U_D[:, :r_d]^T Pi (r_d x D)
+// in shared memory, then N_h = G_h P. Every product of stored values (bf16 x fp32) is exact in
+// float64; only the sums round.
 __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf, int R) {
-  extern __shared__ unsigned char smraw[];
+  extern __shared__ double P_s[];                 // [r_d][D]
   const int h = blockIdx.x, i = blockIdx.y;
   const int lt = a.lt_ids[i];
   const StreamMeta* m = a.meta;
   const int rt = m->lt_rank[lt][0], rd = m->lt_rank[lt][1], b = m->lt_rank[lt][2];
   if (b == 0 || rt == 0) return;
-  const int D = a.D;
-  float* Pi_s = reinterpret_cast<float*>(smraw);                       // D x D
-  float* G_s = Pi_s + D * D;                                           // rt x rd
-  float* UDt = G_s + kMaxN * kMaxN;                                    // rd x D (transposed)
-  double* M_s = reinterpret_cast<double*>(UDt + kMaxN * kMaxN);        // 16 x D
+  constexpr int D = kD, Q = kD / 4;
   const __nv_bfloat16* G = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_G]) +
                            (int64_t)h * rt * rd;
   const __nv_bfloat16* UD = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UD]);
-  for (int e = threadIdx.x; e < D * D; e += blockDim.x) Pi_s[e] = a.Pi[e];
-  for (int e = threadIdx.x; e < rt * rd; e += blockDim.x) G_s[e] = __bfloat162float(G[e]);
-  for (int e = threadIdx.x; e < D * rd; e += blockDim.x) {
-    const int d = e / rd, j = e % rd;
-    UDt[j * D + d] = __bfloat162float(UD[e]);
+  // P[j][e0 .. e0 + 3] = sum_d U_D[d][j] Pi[d][e0 ..]
+  for (int task = threadIdx.x; task < rd * Q; task += blockDim.x) {
+    const int j = task / Q, e0 = 4 * (task - j * Q);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int d = 0; d < D; ++d) {
+      const double u = (double)__bfloat162float(UD[d * rd + j]);
+      const float4 pv = *reinterpret_cast<const float4*>(a.Pi + d * D + e0);
+      acc[0] = fma(u, (double)pv.x, acc[0]);
+      acc[1] = fma(u, (double)pv.y, acc[1]);
+      acc[2] = fma(u, (double)pv.z, acc[2]);
+      acc[3] = fma(u, (double)pv.w, acc[3]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) P_s[j * D + e0 + q] = acc[q];
   }
   __syncthreads();
+  // N_h[k][e0 ..] = sum_j G_h[k][j] P[j][e0 ..]
   double* N = Nbuf + (((int64_t)i * a.H + h) * R) * D;
-  for (int k0 = 0; k0 < rt; k0 += 16) {
-    for (int e = threadIdx.x; e < 16 * D; e += blockDim.x) {
-      const int kk = e / D, d = e % D;
-      double acc = 0.0;
-      if (k0 + kk < rt)
-        for (int j = 0; j < rd; ++j) acc = fma((double)G_s[(k0 + kk) * rd + j], (double)UDt[j * D + d], acc);
-      M_s[kk * D + d] = acc;
+  for (int task = threadIdx.x; task < rt * Q; task += blockDim.x) {
+    const int k = task / Q, e0 = 4 * (task - k * Q);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int j = 0; j < rd; ++j) {
+      const double g = (double)__bfloat162float(G[k * rd + j]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = fma(g, P_s[j * D + e0 + q], acc[q]);
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < 16 * D; e += blockDim.x) {
-      const int kk = e / D, j = e % D;
-      if (k0 + kk >= rt) continue;
-      double acc = 0.0;
-      for (int ii = 0; ii < D; ++ii) acc = fma(M_s[kk * D + ii], (double)Pi_s[ii * D + j], acc);
-      N[(int64_t)(k0 + kk) * D + j] = acc;
-    }
-    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) N[(int64_t)k * D + e0 + q] = acc[q];
   }
 }
 
@@ -253,9 +254,7 @@ __global__ void __launch_bounds__(256, 1) k_residual(ResidualArgs a, const doubl
 
 }  // namespace
 
-static size_t residual_prep_smem() {
-  return ((size_t)kD * kD + 2 * (size_t)kMaxN * kMaxN) * sizeof(float) + 16 * (size_t)kD * sizeof(double);
-}
+static size_t residual_prep_smem() { return (size_t)kD * kD * sizeof(double); }
 
 cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStream_t s) {
   if (a.D != kD) return cudaErrorInvalidValue;
