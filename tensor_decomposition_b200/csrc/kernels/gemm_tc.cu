@@ -134,7 +134,7 @@ __device__ __forceinline__ void store_parts_chunk(__nv_bfloat16* const (&P)[3], 
 }
 
 template <int STAGES>
-__global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGemmParams p) {
+__global__ void __launch_bounds__(256, 2) k_gemm_tc(const __grid_constant__ TcGemmParams p) {
   extern __shared__ uint8_t smraw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
@@ -332,17 +332,28 @@ cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
   if ((p.ps[0] || p.pt[0]) && p.c_batch_in > 0) return cudaErrorInvalidValue;
   const int stage_bytes = (p.na + (p.b_same ? 0 : p.nb)) * kTileBytes;
   const dim3 g((p.N + kTile - 1) / kTile, (p.M + kTile - 1) / kTile, batch);
-  if (stage_bytes * 4 + 1024 <= 200 * 1024) {
-    const int smem = stage_bytes * 4 + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    k_gemm_tc<4><<<g, 256, smem, s>>>(p);
+  // Two CTAs per SM (one's epilogue overlapping the other's loads and MMAs, twice the tiles
+  // per wave) when a ring of 3, else 2, stages fits in half the shared memory; otherwise one
+  // CTA with the deepest ring that fits.
+  constexpr int kHalf = 110 * 1024, kFull = 200 * 1024;
+  int stages;
+  if (3 * stage_bytes + 1024 <= kHalf) stages = 3;
+  else if (2 * stage_bytes + 1024 <= kHalf) stages = 2;
+  else if (4 * stage_bytes + 1024 <= kFull) stages = 4;
+  else stages = 2;
+  const int smem = stages * stage_bytes + 1024;
+  cudaError_t e;
+  if (stages == 3) {
+    e = cudaFuncSetAttribute(k_gemm_tc<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) k_gemm_tc<3><<<g, 256, smem, s>>>(p);
+  } else if (stages == 4) {
+    e = cudaFuncSetAttribute(k_gemm_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) k_gemm_tc<4><<<g, 256, smem, s>>>(p);
   } else {
-    const int smem = stage_bytes * 2 + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    k_gemm_tc<2><<<g, 256, smem, s>>>(p);
+    e = cudaFuncSetAttribute(k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) k_gemm_tc<2><<<g, 256, smem, s>>>(p);
   }
+  if (e != cudaSuccess) return e;
   note_launch();
   return cudaGetLastError();
 }
