@@ -238,7 +238,8 @@ def config_dict(cfg, args):
             "layers": cfg.layers, "kv_heads": cfg.heads, "tokens": cfg.tokens, "head_dim": cfg.head_dim,
             "kinds": "K+V" if cfg.has_v else "K", "ratio": args.ratio, "encoder": args.encoder,
             "groups": cfg.groups, "seq_per_gpu": 1,
-            "l2": "inputs larger than L2 (K+V bf16 = 134 MB > 126 MB L2), no flush"}
+            "l2": "inputs larger than L2 (K+V bf16 = 134 MB > 126 MB L2), no flush",
+            "codec_seed": "fixed across steps: the seed-derived rotation and sketch matrices are built once per plan"}
 
 
 # ------------------------------------------------------------------ work models for the roofline

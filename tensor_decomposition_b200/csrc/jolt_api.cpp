@@ -255,6 +255,8 @@ struct jolt_plan_s {
   __nv_bfloat16* Pib = nullptr;
   bool pi_valid = false;
   uint64_t pi_seed = 0;
+  bool om_valid = false;     // the sketch matrices in Om belong to om_seed (a function of the seed only)
+  uint64_t om_seed = 0;
   jolt_stream_s* last = nullptr;
   int device = 0;
 };
@@ -817,8 +819,12 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       p->q_t = true;
       {
         PROF("sketch_omega", s);
-        std::vector<int32_t> ids = p->lt_ids;
-        CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, true, s));   // Omega^T [l][HD]
+        if (!(p->om_valid && p->om_seed == seed)) {
+          std::vector<int32_t> ids = p->lt_ids;
+          CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, true, s));   // Omega^T [l][HD]
+          p->om_valid = true;
+          p->om_seed = seed;
+        }
       }
       jolt_status r = JOLT_OK;
       // two part sets: every basis lives as bf16 parts, written by the epilogue that makes it
@@ -954,8 +960,12 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       p->q_t = false;
       {
         PROF("sketch_omega", s);
-        std::vector<int32_t> ids = p->lt_ids;
-        CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, false, s));
+        if (!(p->om_valid && p->om_seed == seed)) {
+          std::vector<int32_t> ids = p->lt_ids;
+          CK(sketch_omega(seed, ids.data(), n, HD, l, p->Om, false, s));
+          p->om_valid = true;
+          p->om_seed = seed;
+        }
       }
       jolt_status r = JOLT_OK;
       {

@@ -271,33 +271,55 @@ __global__ void __launch_bounds__(1024) k_dual_pool(DualArgs a) {
   }
 }
 
-// Layout of the body: lt-major, parts U_T, U_D, G, scales, codes, each 256-aligned.
-__global__ void k_layout(DualArgs a) {
+// Layout of the body: lt-major (layer, then kind), parts U_T, U_D, G, scales, codes, each
+// starting at a 256-byte boundary. A layer-tensor's parts occupy the sum of their sizes rounded
+// up to 256 bytes, so the offsets follow from one exclusive prefix sum over the layer-tensors
+// (one thread per layer-tensor, launched with kMaxLT threads).
+__global__ void __launch_bounds__(kMaxLT) k_layout(DualArgs a) {
+  __shared__ int64_t foot[kMaxLT];
+  __shared__ unsigned long long bp[JOLT_NUM_PARTS];
   StreamMeta* meta = a.meta;
-  int64_t cur = 0;
-  int64_t bp[JOLT_NUM_PARTS] = {0, 0, 0, 0, 0};
-  for (int l = 0; l < a.L; ++l) {
+  const int kinds = a.has_v ? 2 : 1, nlt = a.L * kinds, t = threadIdx.x;
+  if (t < JOLT_NUM_PARTS) bp[t] = 0;
+  int64_t sz[JOLT_NUM_PARTS] = {0, 0, 0, 0, 0};
+  int64_t f = 0;
+  int lt = 0;
+  if (t < nlt) {
+    const int l = t / kinds, k = t % kinds;
+    lt = 2 * l + k;
     int g = 0;
     while (g + 1 < a.G && ((int64_t)(g + 1) * a.L) / a.G <= l) ++g;
-    for (int k = 0; k < (a.has_v ? 2 : 1); ++k) {
-      const int lt = 2 * l + k;
-      const int rt = meta->alloc[g][k][0], rd = meta->alloc[g][k][1], b = meta->alloc[g][k][2];
-      meta->lt_rank[lt][0] = rt;
-      meta->lt_rank[lt][1] = rd;
-      meta->lt_rank[lt][2] = b;
-      const int64_t sz[JOLT_NUM_PARTS] = {
-          (int64_t)a.T * rt * 2, (int64_t)a.D * rd * 2, (int64_t)a.H * rt * rd * 2,
-          b > 0 ? (int64_t)a.H * a.T * 2 : 0, b > 0 ? (int64_t)a.H * a.T * (a.D * b / 8) : 0};
-      for (int p = 0; p < JOLT_NUM_PARTS; ++p) {
-        const int64_t off = (cur + kAlign - 1) / kAlign * kAlign;
-        meta->off[lt][p] = off;
-        cur = off + sz[p];
-        bp[p] += sz[p];
-      }
-    }
+    const int rt = meta->alloc[g][k][0], rd = meta->alloc[g][k][1], b = meta->alloc[g][k][2];
+    meta->lt_rank[lt][0] = rt;
+    meta->lt_rank[lt][1] = rd;
+    meta->lt_rank[lt][2] = b;
+    sz[0] = (int64_t)a.T * rt * 2;
+    sz[1] = (int64_t)a.D * rd * 2;
+    sz[2] = (int64_t)a.H * rt * rd * 2;
+    sz[3] = b > 0 ? (int64_t)a.H * a.T * 2 : 0;
+    sz[4] = b > 0 ? (int64_t)a.H * a.T * (a.D * b / 8) : 0;
+    for (int p = 0; p < JOLT_NUM_PARTS; ++p) f += (sz[p] + kAlign - 1) / kAlign * kAlign;
   }
-  meta->body_bytes = cur;
-  for (int p = 0; p < JOLT_NUM_PARTS; ++p) meta->bytes_by_part[p] = bp[p];
+  foot[t] = f;
+  __syncthreads();
+  // inclusive scan of the footprints (Hillis-Steele, fixed order of additions)
+  for (int o = 1; o < kMaxLT; o <<= 1) {
+    const int64_t v = t >= o ? foot[t - o] : 0;
+    __syncthreads();
+    foot[t] += v;
+    __syncthreads();
+  }
+  if (t < nlt) {
+    int64_t cur = t > 0 ? foot[t - 1] : 0;          // 256-aligned start of this layer-tensor
+    for (int p = 0; p < JOLT_NUM_PARTS; ++p) {
+      meta->off[lt][p] = cur;
+      atomicAdd(&bp[p], (unsigned long long)sz[p]);
+      cur += (sz[p] + kAlign - 1) / kAlign * kAlign;
+    }
+    if (t == nlt - 1) meta->body_bytes = cur - (sz[4] + kAlign - 1) / kAlign * kAlign + sz[4];
+  }
+  __syncthreads();
+  if (t < JOLT_NUM_PARTS) meta->bytes_by_part[t] = (int64_t)bp[t];
 }
 
 // Copy the chosen leading blocks of the factors and the bf16-rounded core into the body.
@@ -354,7 +376,7 @@ cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s) {
   const int threads = 32 * (items < 32 ? items : 32);
   k_dual_pool<<<npools, threads, kDualSmem, s>>>(a);
   note_launch();
-  k_layout<<<1, 1, 0, s>>>(a);
+  k_layout<<<1, kMaxLT, 0, s>>>(a);
   note_launch();
   return cudaGetLastError();
 }
