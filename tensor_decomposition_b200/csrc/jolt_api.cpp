@@ -938,18 +938,27 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         g.na = 3; g.nb = 1;
         g.M = l; g.N = (int)HD; g.KB = (T + 63) / 64;
         g.c_sm = HD; g.c_sn = 1; g.c_sb = (int64_t)l * HD;
+        // B's bf16 parts, [l][HD] for B B^T and [HD][l] for the per-head core, go to the part
+        // set that does not hold Q
+        const PartSet& bs = sets[cur ^ 1];
         const int kc = k_chunks(T);
         if (kc == 1) {
           g.C = p->Bm;
+          g.t_sm = 1; g.t_sn = l; g.t_sb = (int64_t)HD * l;
+          for (int i = 0; i < 3; ++i) {
+            g.ps[i] = bs.s[i];
+            g.pt[i] = bs.t[i];
+          }
           CK(gemm_tc(n, g, s));
         } else {
-          // long K: float32 partials per chunk of tokens, summed in float64
+          // long K: float32 partials per chunk of tokens, summed in float64, then the parts
           g.av.nch = g.bv.nch = kc;
           g.av.ckb = g.bv.ckb = T / kc / 64;
           g.KB = T / kc / 64;
           g.C = p->Cpart;
           CK(gemm_tc(n * kc, g, s));
           CK(sum_heads(n, kc, (int64_t)l * HD, p->Cpart, p->Bm, nullptr, s));
+          CK(split_dual(n, l, (int)HD, p->Bm, false, bs.s, bs.t, s));
         }
       }
       p->Qfinal = nullptr;
@@ -1031,11 +1040,11 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         PROF("small_gemm", s);
         // B B^T: float32 partial Grams over 128-wide chunks of the (head, feature) axis on the
         // tensor cores (B in three bf16 parts), summed over the chunks in float64
-        CK(split_bf16((int64_t)n * l * HD, p->Bm, p->QTp[0], p->QTp[1], p->QTp[2], s));
+        __nv_bfloat16* const* bsame = p->qset ? p->QTp : p->QTp2;     // B parts [l][HD] (set qset ^ 1)
         TcGemmParams g;
         g.status = status;
         for (int i = 0; i < 3; ++i)
-          if (!map_kchunk(&g.amap[i], p->QTp[i], l, HD, 128, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
+          if (!map_kchunk(&g.amap[i], bsame[i], l, HD, 128, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
         g.av.mode = VIEW_XT_PERHEAD;      // (K, rows, chunk, i)
         g.av.H = nch;
         g.na = g.nb = 3;
@@ -1077,11 +1086,11 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         PROF("core", s);
         // P[h] = W_R^T B_h (R x D): W^T parts (signs fixed), B^T parts per head
         CK(split_dual(n, l, l, p->Wv, false, nullptr, p->RTp, s));
-        CK(split_dual(n, l, (int)HD, p->Bm, false, nullptr, p->QNp, s));
+        __nv_bfloat16* const* btr = p->qset ? p->QNp : p->QNp2;       // B parts [HD][l] (set qset ^ 1)
         TcGemmParams g;
         g.status = status;
         for (int i = 0; i < 3; ++i)
-          if (!map_rows(&g.amap[i], p->RTp[i], l, l, n) || !map_perhead(&g.bmap[i], p->QNp[i], l, D, H, n))
+          if (!map_rows(&g.amap[i], p->RTp[i], l, l, n) || !map_perhead(&g.bmap[i], btr[i], l, D, H, n))
             return fail(JOLT_ERR_CUDA, "tensor map rejected");
         g.av.H = H;                       // W^T shared by the heads of a layer-tensor
         g.bv.mode = VIEW_XT_PERHEAD;

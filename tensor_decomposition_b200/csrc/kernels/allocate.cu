@@ -56,6 +56,47 @@ __global__ void k_energy_table(int H, int R, int D, int step, const float* Gmax,
   }
 }
 
+// The same table for the default grid (step 16, D = 128): warp w sums row block I = w, w + 8,
+// .. over every head and its 16 rows with coalesced float4 loads (lane l holds columns
+// 4l .. 4l + 3, so the 4 lanes 4J .. 4J + 3 cover column block J), in float64 and a fixed order.
+__global__ void __launch_bounds__(256) k_energy_table16(int H, int R, const float* Gmax, const double* xx,
+                                                        double* E, int ngrid, const int32_t* lt_ids) {
+  constexpr int D = kD, step = 16, nJ = D / step;
+  __shared__ double sb[(kMaxN / step) * nJ];
+  const int lt = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nI = R / step;
+  const float* g = Gmax + (int64_t)lt * H * R * D;
+  for (int I = warp; I < nI; I += 8) {
+    double acc = 0.0;
+    for (int h = 0; h < H; ++h) {
+      const float4* row = reinterpret_cast<const float4*>(g + ((int64_t)h * R + I * step) * D) + lane;
+#pragma unroll 4
+      for (int i = 0; i < step; ++i) {
+        const float4 v = row[i * (D / 4)];
+        acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+      }
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if ((lane & 3) == 0) sb[I * nJ + (lane >> 2)] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const double x2 = xx[lt];
+    double* e = E + (int64_t)lt_ids[lt] * ngrid;
+    e[0] = x2;
+    for (int I = 0; I < nI; ++I)
+      for (int J = 1; J < nJ; ++J) sb[I * nJ + J] += sb[I * nJ + J - 1];
+    for (int I = 1; I < nI; ++I)
+      for (int J = 0; J < nJ; ++J) sb[I * nJ + J] += sb[(I - 1) * nJ + J];
+    for (int I = 0; I < nI; ++I)
+      for (int J = 0; J < nJ; ++J) {
+        const double r = x2 - sb[I * nJ + J];
+        e[1 + I * nJ + J] = r > 0.0 ? r : 0.0;
+      }
+  }
+}
+
 __device__ __forceinline__ int64_t lt_bytes(int H, int T, int D, int rt, int rd, int b) {
   const int64_t tucker = 2 * ((int64_t)T * rt + (int64_t)D * rd + (int64_t)H * rt * rd);
   const int64_t resid = b > 0 ? (int64_t)H * T * (D * b / 8 + 2) : 0;
@@ -356,6 +397,11 @@ __global__ void k_pack_factors(PackArgs a) {
 }  // namespace
 
 cudaError_t energy_table(const TableArgs& a, cudaStream_t s) {
+  if (a.step == 16 && a.D == kD && a.R <= kMaxN) {
+    k_energy_table16<<<a.n_lt, 256, 0, s>>>(a.H, a.R, a.Gmax, a.xx, a.E, a.ngrid, a.lt_ids);
+    note_launch();
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)(a.R / a.step) * (a.D / a.step) * sizeof(double) + sizeof(double);
   k_energy_table<<<a.n_lt, 128, smem, s>>>(a.H, a.R, a.D, a.step, a.Gmax, a.xx, a.E, a.ngrid,
                                            a.lt_ids);
