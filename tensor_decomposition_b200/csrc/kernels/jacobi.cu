@@ -17,6 +17,7 @@
 // rotation ends the solve. Eigenvalues are returned in descending order with their
 // eigenvector columns (no sign normalisation here).
 #include "../jolt_internal.h"
+#include <type_traits>
 
 namespace jolt {
 namespace {
@@ -438,15 +439,40 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
           nb = v[2 * s + 1];
         }
     }
-    for (int r = 0; r < NP - 1; ++r) {
-      // gamma of the four slots: per-lane partial sums, then a transposed butterfly that leaves
-      // slot grp's sum in the 8 lanes of group grp (identical in all of them)
-      double v[4];
+    // One round at tournament phase K (rounds done in this sweep, mod 4). The slots' columns
+    // are not moved between registers from round to round: logical top slot s lives in
+    // top[(s - K) & 3] and logical bottom slot s in bot[(s + K) & 3], so the column leaving a
+    // warp and the one arriving share a register and nothing else is copied.
+    // partial sums (this lane's rows) of gamma for slots 1 and 2 at phase K
+    double vpre[2];
+    auto partials12 = [&](auto kc) {
+      constexpr int K = decltype(kc)::value;
 #pragma unroll
-      for (int s = 0; s < 4; ++s) {
+      for (int s = 1; s <= 2; ++s) {
         double g = 0.0;
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) g = fma(top[s][i], bot[s][i], g);
+        for (int i = 0; i < RPL; ++i) g = fma(top[(s - K) & 3][i], bot[(s + K) & 3][i], g);
+        vpre[s - 1] = g;
+      }
+    };
+    partials12(std::integral_constant<int, 0>{});
+    auto round = [&](auto kc) {
+      constexpr int K = decltype(kc)::value;
+      // a power of two within a factor 2 of 1 / (a + b) for this group's pair
+      const int ex = (__double2hiint(na + nb) >> 20) & 0x7ff;
+      const double sc2 = __hiloint2double((2046 - ex) << 20, 0);
+      // gamma of the four slots: per-lane partial sums, then a transposed butterfly that leaves
+      // slot grp's sum in the 8 lanes of group grp (identical in all of them)
+      // (slots 1 and 2 never wait for another warp: their partial sums were formed before the
+      // previous round's barrier)
+      double v[4];
+      v[1] = vpre[0];
+      v[2] = vpre[1];
+#pragma unroll
+      for (int s = 0; s < 4; s += 3) {
+        double g = 0.0;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) g = fma(top[(s - K) & 3][i], bot[(s + K) & 3][i], g);
         v[s] = g;
       }
       double w2[2];
@@ -464,72 +490,102 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
       g += __shfl_xor_sync(0xffffffffu, g, 2);
       g += __shfl_xor_sync(0xffffffffu, g, 1);
       const double a = na, b = nb;
-      double c = 1.0, sn = 0.0;
-      const float gf = (float)g;
-      if (g * g > 1e-14 * (a * b) && gf != 0.0f) {
-        const float zeta = __fdividef((float)(b - a), 2.0f * gf);
-        const float az = fabsf(zeta);
-        const float t = az > 1e18f ? __fdividef(0.5f, zeta)
-                                   : copysignf(__fdividef(1.0f, az + sqrtf(1.0f + zeta * zeta)), zeta);
-        const float cf = rsqrtf(1.0f + t * t);
-        c = (double)cf;
-        sn = (double)(t * cf);
-        const double fix = 1.5 - 0.5 * (c * c + sn * sn);   // one Newton step: c^2 + s^2 = 1
-        c *= fix;
-        sn *= fix;
-        any = 1;
+      // rotation angle in float on (b - a, 2 gamma) scaled by the power of two of a + b (both
+      // are at most a + b, so the squares below stay in range): with d = b - a,
+      // r = sqrt(d^2 + 4 gamma^2) and w = |d| + r, the rotation that zeroes gamma is
+      // c = w / sqrt(w^2 + 4 gamma^2), s = sign(d) 2 gamma / sqrt(w^2 + 4 gamma^2), i.e.
+      // t = s / c = sign(zeta) / (|zeta| + sqrt(1 + zeta^2)) with zeta = d / (2 gamma)
+      // (Golub & Van Loan sec. 8.5.2) using two reciprocal square roots and no division
+      const float df = (float)((b - a) * sc2), gf = (float)(g * (2.0 * sc2));
+      const bool rot = g * g > 1e-14 * (a * b) && gf != 0.0f;
+      // the angle is computed whether or not the pair rotates (no divergent branch); a pair that
+      // does not rotate takes (c, s) = (1, 0) and keeps its norms
+      double c, sn;
+      {
+        const float q = fmaf(df, df, gf * gf);
+        const float w = fabsf(df) + q * rsqrtf(q);
+        const float z = rsqrtf(fmaf(w, w, gf * gf));
+        const double c0 = (double)(w * z), s0 = (double)((df < 0.0f ? -gf : gf) * z);
+        const double fix = 1.5 - 0.5 * (c0 * c0 + s0 * s0);   // one Newton step: c^2 + s^2 = 1
+        c = rot ? c0 * fix : 1.0;
+        sn = rot ? s0 * fix : 0.0;
         // squared norms after p' = c p - s q, q' = s p + c q
         const double cc = c * c, ss = sn * sn, cs2 = 2.0 * c * sn * g;
-        na = fma(cc, a, fma(ss, b, -cs2));
-        nb = fma(ss, a, fma(cc, b, cs2));
+        const double na_r = fma(cc, a, fma(ss, b, -cs2)), nb_r = fma(ss, a, fma(cc, b, cs2));
+        na = rot ? na_r : a;
+        nb = rot ? nb_r : b;
       }
-      // rotate every slot with its group's (c, s); (1, 0) leaves a pair unchanged exactly
+      any |= (int)rot;
+      // rotate every slot with its group's (c, s); (1, 0) leaves a pair unchanged exactly, so a
+      // warp none of whose pairs rotates skips the arithmetic
+      if (__any_sync(0xffffffffu, rot)) {
 #pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const double cs = __shfl_sync(0xffffffffu, c, 8 * s);
-        const double ss = __shfl_sync(0xffffffffu, sn, 8 * s);
+        for (int s = 0; s < 4; ++s) {
+          const double cs = __shfl_sync(0xffffffffu, c, 8 * s);
+          const double ss = __shfl_sync(0xffffffffu, sn, 8 * s);
+          double* tp = top[(s - K) & 3];
+          double* bp = bot[(s + K) & 3];
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-          const double p = top[s][i], q = bot[s][i];
-          top[s][i] = cs * p - ss * q;
-          bot[s][i] = ss * p + cs * q;
+          for (int i = 0; i < RPL; ++i) {
+            // both s products first, so that each result overwrites its own input
+            const double sq = ss * bp[i], sp = ss * tp[i];
+            tp[i] = fma(cs, tp[i], -sq);
+            bp[i] = fma(cs, bp[i], sp);
+          }
         }
       }
       // next round of the circle tournament: position 0 stays, positions 1 .. 127 advance by
       // one. Tops move to the next slot, bottoms to the previous; slot 0's bottom becomes
       // slot 1's top and slot 63's top becomes its own bottom. The squared norms move with
-      // their columns.
-      const int par = r & 1;
+      // their columns. Leaving: top slot 3 (to warp + 1) and bottom slot 0 (to warp - 1).
+      constexpr int kOutT = (3 - K) & 3, kOutB = K & 3, kFixed = (0 - K) & 3;
+      constexpr int par = K & 1;
       double* xt = XT + (par * 16 + warp) * NP;
       double* xb = XB + (par * 16 + warp) * NP;
 #pragma unroll
       for (int i = 0; i < RPL; ++i) {
-        if (warp < 15) xt[lane + 32 * i] = top[3][i];
-        if (warp > 0) xb[lane + 32 * i] = bot[0][i];
+        if (warp < 15) xt[lane + 32 * i] = top[kOutT][i];
+        if (warp > 0) xb[lane + 32 * i] = bot[kOutB][i];
       }
       if (warp < 15 && lane == 24) XN[(par * 16 + warp) * 2] = na;        // top of slot 4w + 3
       if (warp > 0 && lane == 0) XN[(par * 16 + warp) * 2 + 1] = nb;      // bottom of slot 4w
       const double up_a = __shfl_up_sync(0xffffffffu, (warp == 0 && grp == 0) ? nb : na, 8);
       const double dn_b = __shfl_down_sync(0xffffffffu, nb, 8);
+      // moves that stay inside the edge warps, then the next round's partial sums of slots 1 and
+      // 2 (their columns are all here), then the barrier and the two arriving columns
+      if (warp == 0) {
+        // position 0 stays in slot 0's top; the leaving bottom becomes slot 1's top
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+          top[kOutT][i] = top[kFixed][i];
+          top[kFixed][i] = bot[kOutB][i];
+        }
+      } else if (warp == 15) {
+        // slot 63's top turns into its own bottom
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) bot[kOutB][i] = top[kOutT][i];
+      }
+      partials12(std::integral_constant<int, (K + 1) & 3>{});
       __syncthreads();
       const double* xin_t = XT + (par * 16 + (warp > 0 ? warp - 1 : 0)) * NP;
       const double* xin_b = XB + (par * 16 + (warp < 15 ? warp + 1 : 15)) * NP;
 #pragma unroll
       for (int i = 0; i < RPL; ++i) {
-        const double t3 = top[3][i], b0 = bot[0][i];
-        top[3][i] = top[2][i];
-        top[2][i] = top[1][i];
-        top[1][i] = warp == 0 ? b0 : top[0][i];
-        if (warp > 0) top[0][i] = xin_t[lane + 32 * i];
-        bot[0][i] = bot[1][i];
-        bot[1][i] = bot[2][i];
-        bot[2][i] = bot[3][i];
-        bot[3][i] = warp < 15 ? xin_b[lane + 32 * i] : t3;
+        if (warp > 0) top[kOutT][i] = xin_t[lane + 32 * i];
+        if (warp < 15) bot[kOutB][i] = xin_b[lane + 32 * i];
       }
       const double na_new = grp >= 1 ? up_a : (warp == 0 ? na : XN[(par * 16 + warp - 1) * 2]);
       const double nb_new = grp <= 2 ? dn_b : (warp < 15 ? XN[(par * 16 + warp + 1) * 2 + 1] : na);
       na = na_new;
       nb = nb_new;
+    };
+    // 128 rounds: the 127 of the tournament and the first one again, so that every sweep starts
+    // at phase 0 (the columns end one position further on per sweep; only their set matters)
+    for (int r = 0; r < NP; r += 4) {
+      round(std::integral_constant<int, 0>{});
+      round(std::integral_constant<int, 1>{});
+      round(std::integral_constant<int, 2>{});
+      round(std::integral_constant<int, 3>{});
     }
     if (any) rotated[sweep & 1] = 1;
     if (tid == 0) rotated[(sweep + 1) & 1] = 0;
@@ -537,7 +593,8 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
     if (!rotated[sweep & 1]) break;
   }
   if (sweep == max_sweeps && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
-  // after whole sweeps every column is back at its starting position
+  // the columns, in the positions the last sweep left them in (their order does not matter:
+  // they are ranked by norm below)
 #pragma unroll
   for (int s = 0; s < 4; ++s)
 #pragma unroll

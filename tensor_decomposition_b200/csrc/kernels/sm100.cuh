@@ -33,9 +33,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Wait for the phase with the given parity; gives up after `max_iter` polls and returns false.
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Longest time one bounded wait may take. try_wait may suspend the thread for a system-defined
+// interval on each poll, so a poll count alone bounds no time; the clock does.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// Wait for the phase with the given parity; gives up after `max_iter` polls or kWaitLimitNs,
+// whichever comes first, and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter) {
   const uint32_t a = smem_u32(bar);
+  uint64_t t0 = 0;
   for (uint32_t it = 0; it < max_iter; ++it) {
     uint32_t done;
     asm volatile(
@@ -46,6 +58,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
         : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
+    if ((it & 31) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (it == 0) t0 = now;
+      else if (now - t0 > kWaitLimitNs) return false;
+    }
   }
   return false;
 }
