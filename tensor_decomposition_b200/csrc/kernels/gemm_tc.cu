@@ -7,10 +7,12 @@
 // float32 operands enter as a sum of up to three bf16 parts (hi + lo + lo2), each part one
 // more pass of the tensor core over the same accumulator.
 //
-// Structure: one CTA per 128 x 128 output tile. Warp 0 issues TMA tile loads (128 rows x 64
-// bf16, 128-byte swizzle, no multicast) into a ring of stages; warp 1 owns the Tensor Memory
-// accumulator and issues tcgen05.mma (M = 128, N = 128, K = 16) from one thread; warps 4-7
-// read the accumulator back with tcgen05.ld and store float32. Every wait is bounded and
+// Structure: persistent, one CTA per SM looping over 128 x 128 output tiles. Warp 0 issues
+// TMA tile loads (128 rows x 64 bf16, 128-byte swizzle, no multicast) into a ring of stages
+// that runs on across tiles; warp 1 owns two Tensor Memory accumulators and issues
+// tcgen05.mma (M = 128, N = 128, K = 16) from one thread, alternating between them tile by
+// tile; warps 4-7 read a finished accumulator back with tcgen05.ld and store float32 (and/or
+// bf16 parts) while the next tile is being loaded and multiplied. Every wait is bounded and
 // reports ST_TIMEOUT instead of hanging.
 #include "../jolt_internal.h"
 #include "sm100.cuh"
@@ -133,16 +135,35 @@ __device__ __forceinline__ void store_parts_chunk(__nv_bfloat16* const (&P)[3], 
   }
 }
 
+constexpr int kStgBytes = 4 * 32 * 33 * 4;   // epilogue staging: one 32 x 33 float chunk per warp
+
+// Tile t of the launch: n tiles fastest (consecutive tiles of a CTA share A rows through L2),
+// then m tiles, then the batch.
+__device__ __forceinline__ void tile_coords(int t, int ntn, int ntm, int& n0, int& m0, int& b) {
+  const int per_b = ntn * ntm;
+  b = t / per_b;
+  const int r = t - b * per_b;
+  m0 = (r / ntn) * kTile;
+  n0 = (r % ntn) * kTile;
+}
+
+// Persistent: CTA c takes the tiles c, c + gridDim.x, ... Warp 0 streams the operand tiles of
+// all of them through the stage ring; warp 1 accumulates tile i in TMEM buffer i & 1 (two
+// 128-column buffers), so that warps 4-7 read tile i back and store it while tile i + 1 is
+// loaded and multiplied. Barriers: full / empty per stage (TMA bytes / MMA completion),
+// acc_full per buffer (MMA completion), acc_empty per buffer (the four epilogue warps).
 template <int STAGES>
-__global__ void __launch_bounds__(256, 2) k_gemm_tc(const __grid_constant__ TcGemmParams p) {
+__global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGemmParams p, int ntiles, int ntn,
+                                                     int ntm) {
   extern __shared__ uint8_t smraw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ __align__(8) uint64_t acc_full[2];
+  __shared__ __align__(8) uint64_t acc_empty[2];
   __shared__ uint32_t tmem_base;
+  __shared__ int abort_s;   // a wait ran out: every role stops at its next tile or k-block
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile, b = blockIdx.z;
   const int nbl = p.b_same ? 0 : p.nb;   // B parts loaded per stage
   const int stage_bytes = (p.na + nbl) * kTileBytes;
   int npairs = p.npairs;
@@ -159,13 +180,22 @@ __global__ void __launch_bounds__(256, 2) k_gemm_tc(const __grid_constant__ TcGe
       pb[t] = p.pair_b[t];
     }
   }
+  volatile int* abort_v = &abort_s;
+  auto fail = [&]() {
+    *abort_v = 1;
+    atomicOr(p.status, ST_TIMEOUT);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(&accum_bar, 1);
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&acc_full[j], 1);
+      mbar_init(&acc_empty[j], 4);
+    }
+    abort_s = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -173,7 +203,7 @@ __global__ void __launch_bounds__(256, 2) k_gemm_tc(const __grid_constant__ TcGe
     for (int i = 0; i < p.nb; ++i) prefetch_tensormap(&p.bmap[i]);
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base, kTile);
+    tmem_alloc(&tmem_base, 2 * kTile);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -183,102 +213,135 @@ __global__ void __launch_bounds__(256, 2) k_gemm_tc(const __grid_constant__ TcGe
 
   if (warp == 0) {
     if (elect_one()) {
-      for (int kb = 0; kb < p.KB; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t parity = ((kb / STAGES) & 1) ^ 1;
-        if (!mbar_wait(&empty_bar[s], parity, kMaxPoll)) {
-          atomicOr(p.status, ST_TIMEOUT);
-          break;
+      uint32_t g = 0;   // k-blocks issued by this CTA (stage ring position)
+      for (int t = blockIdx.x; t < ntiles && !*abort_v; t += gridDim.x) {
+        int n0, m0, b;
+        tile_coords(t, ntn, ntm, n0, m0, b);
+        for (int kb = 0; kb < p.KB; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          if (!mbar_wait(&empty_bar[s], ((g / STAGES) & 1) ^ 1, kMaxPoll) || *abort_v) {
+            fail();
+            break;
+          }
+          uint8_t* st = smem + s * stage_bytes;
+          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)stage_bytes);
+          for (int i = 0; i < p.na; ++i) view_load(p.av, &p.amap[i], st + i * kTileBytes, &full_bar[s], m0, kb, b);
+          for (int i = 0; i < nbl; ++i)
+            view_load(p.bv, &p.bmap[i], st + (p.na + i) * kTileBytes, &full_bar[s], n0, kb, b);
         }
-        uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)stage_bytes);
-        for (int i = 0; i < p.na; ++i) view_load(p.av, &p.amap[i], st + i * kTileBytes, &full_bar[s], m0, kb, b);
-        for (int i = 0; i < nbl; ++i)
-          view_load(p.bv, &p.bmap[i], st + (p.na + i) * kTileBytes, &full_bar[s], n0, kb, b);
       }
     }
   } else if (warp == 1) {
     if (elect_one()) {
       const uint32_t idesc = idesc_bf16_f32(kTile, kTile);
-      bool ok = true;
-      for (int kb = 0; kb < p.KB && ok; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(&full_bar[s], (kb / STAGES) & 1, kMaxPoll)) {
-          atomicOr(p.status, ST_TIMEOUT);
-          ok = false;
+      uint32_t g = 0;
+      int i = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort_v; t += gridDim.x, ++i) {
+        const int ab = i & 1;
+        const uint32_t use = (uint32_t)(i >> 1);
+        if (!mbar_wait(&acc_empty[ab], (use & 1) ^ 1, kMaxPoll)) {
+          fail();
           break;
         }
         tc_fence_after();
-        const uint32_t st = smem_u32(smem + s * stage_bytes);
-        for (int t = 0; t < npairs; ++t) {
-          const int ia = pa[t], ib = pb[t];
-          const uint32_t abase = st + ia * kTileBytes;
-          const uint32_t bbase = p.b_same ? st + ib * kTileBytes : st + (p.na + ib) * kTileBytes;
-#pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t ad = desc_kmajor_sw128(abase + k * 32);
-            const uint64_t bd = desc_kmajor_sw128(bbase + k * 32);
-            umma_bf16(tmem, ad, bd, idesc, (kb | t | k) != 0 ? 1u : 0u);
+        const uint32_t d = tmem + (uint32_t)(ab * kTile);
+        bool ok = true;
+        for (int kb = 0; kb < p.KB; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          if (!mbar_wait(&full_bar[s], (g / STAGES) & 1, kMaxPoll) || *abort_v) {
+            fail();
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * stage_bytes);
+          for (int q = 0; q < npairs; ++q) {
+            const int ia = pa[q], ib = pb[q];
+            const uint32_t abase = st + ia * kTileBytes;
+            const uint32_t bbase = p.b_same ? st + ib * kTileBytes : st + (p.na + ib) * kTileBytes;
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t ad = desc_kmajor_sw128(abase + k * 32);
+              const uint64_t bd = desc_kmajor_sw128(bbase + k * 32);
+              umma_bf16(d, ad, bd, idesc, (kb | q | k) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty_bar[s]);   // frees the stage once these MMAs have read it
         }
-        umma_commit(&empty_bar[s]);   // frees the stage once these MMAs have read it
+        if (!ok) break;
+        umma_commit(&acc_full[ab]);
       }
-      umma_commit(&accum_bar);
     }
   } else if (warp >= 4) {
     const int e = warp - 4;                      // TMEM lanes 32e .. 32e + 31
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&accum_bar, 0, kMaxPoll));   // warp-uniform
-    if (!ok && lane == 0) atomicOr(p.status, ST_TIMEOUT);
-    tc_fence_after();
-    const int m = m0 + 32 * e + lane;
-    int64_t boff;
-    if (p.c_batch_in > 0) boff = (int64_t)(b / p.c_batch_in) * p.c_sb_out + (int64_t)(b % p.c_batch_in) * p.c_sb;
-    else boff = (int64_t)b * p.c_sb;
-    float* C = p.C ? p.C + boff : nullptr;
-    const int64_t poff = (int64_t)b * p.c_sb, toff = (int64_t)b * p.t_sb;
     // Outputs contiguous along n (row-major C: c_sn = 1, or a part layout with unit n stride)
-    // go through shared memory in 32 x 32 chunks (the pipeline stages are free once the
-    // accumulator is complete), so that a store instruction covers consecutive n of one row;
-    // outputs contiguous along m are stored from the registers (consecutive lanes, consecutive m).
-    float* stg = reinterpret_cast<float*>(smem) + e * (32 * 33);
-    const bool c_n = C && p.c_sn == 1, c_m = C && p.c_sn != 1;
+    // go through shared memory in 32 x 32 chunks, so that a store instruction covers
+    // consecutive n of one row; outputs contiguous along m are stored from the registers
+    // (consecutive lanes, consecutive m).
+    float* stg = reinterpret_cast<float*>(smem + STAGES * stage_bytes) + e * (32 * 33);
+    const bool c_n = p.C && p.c_sn == 1, c_m = p.C && p.c_sn != 1;
     const bool parts = p.ps[0] || p.pt[0];
-#pragma unroll 1
-    for (int c = 0; c < kTile / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(32 * e) << 16) + (uint32_t)(c * 32), r);
-      tmem_ld_wait();
-      if (!ok) continue;
-      if (c_n || parts) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
-        __syncwarp();
-        if (c_n) {
-          const int n = n0 + c * 32 + lane;
-#pragma unroll 4
-          for (int rr = 0; rr < 32; ++rr) {
-            const int mm = m0 + 32 * e + rr;
-            if (mm < p.M && n < p.N) C[(int64_t)mm * p.c_sm + n] = stg[rr * 33 + lane];
-          }
-        }
-        if (p.ps[0])
-          store_parts_chunk(p.ps, poff, p.c_sm, p.c_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
-        if (p.pt[0])
-          store_parts_chunk(p.pt, toff, p.t_sm, p.t_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
-        __syncwarp();
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+      const int ab = i & 1;
+      const uint32_t use = (uint32_t)(i >> 1);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], use & 1, kMaxPoll));   // warp-uniform
+      if (!ok || *abort_v) {
+        if (lane == 0 && !ok) fail();
+        break;
       }
-      if (c_m && m < p.M) {
+      tc_fence_after();
+      int n0, m0, b;
+      tile_coords(t, ntn, ntm, n0, m0, b);
+      const int m = m0 + 32 * e + lane;
+      int64_t boff;
+      if (p.c_batch_in > 0) boff = (int64_t)(b / p.c_batch_in) * p.c_sb_out + (int64_t)(b % p.c_batch_in) * p.c_sb;
+      else boff = (int64_t)b * p.c_sb;
+      float* C = p.C ? p.C + boff : nullptr;
+      const int64_t poff = (int64_t)b * p.c_sb, toff = (int64_t)b * p.t_sb;
+      const uint32_t tbase = tmem + (uint32_t)(ab * kTile) + ((uint32_t)(32 * e) << 16);
+#pragma unroll 1
+      for (int c = 0; c < kTile / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + (uint32_t)(c * 32), r);
+        tmem_ld_wait();
+        if (c == kTile / 32 - 1) {
+          // the whole accumulator is in registers or staged: hand the buffer back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+        if (c_n || parts) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int n = n0 + c * 32 + j;
-          if (n < p.N) C[(int64_t)m * p.c_sm + (int64_t)n * p.c_sn] = __uint_as_float(r[j]);
+          for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
+          __syncwarp();
+          if (c_n) {
+            const int n = n0 + c * 32 + lane;
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr) {
+              const int mm = m0 + 32 * e + rr;
+              if (mm < p.M && n < p.N) C[(int64_t)mm * p.c_sm + n] = stg[rr * 33 + lane];
+            }
+          }
+          if (p.ps[0])
+            store_parts_chunk(p.ps, poff, p.c_sm, p.c_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
+          if (p.pt[0])
+            store_parts_chunk(p.pt, toff, p.t_sm, p.t_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
+          __syncwarp();
+        }
+        if (c_m && m < p.M) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = n0 + c * 32 + j;
+            if (n < p.N) C[(int64_t)m * p.c_sm + (int64_t)n * p.c_sn] = __uint_as_float(r[j]);
+          }
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, kTile);
+  if (warp == 1) tmem_dealloc(tmem, 2 * kTile);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -331,27 +394,45 @@ cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
   if (p.b_same && (p.M > kTile || p.N > kTile || p.nb > p.na)) return cudaErrorInvalidValue;
   if ((p.ps[0] || p.pt[0]) && p.c_batch_in > 0) return cudaErrorInvalidValue;
   const int stage_bytes = (p.na + (p.b_same ? 0 : p.nb)) * kTileBytes;
-  const dim3 g((p.N + kTile - 1) / kTile, (p.M + kTile - 1) / kTile, batch);
-  // Two CTAs per SM (one's epilogue overlapping the other's loads and MMAs, twice the tiles
-  // per wave) when a ring of 3, else 2, stages fits in half the shared memory; otherwise one
-  // CTA with the deepest ring that fits.
-  constexpr int kHalf = 110 * 1024, kFull = 200 * 1024;
-  int stages;
-  if (3 * stage_bytes + 1024 <= kHalf) stages = 3;
-  else if (2 * stage_bytes + 1024 <= kHalf) stages = 2;
-  else if (4 * stage_bytes + 1024 <= kFull) stages = 4;
-  else stages = 2;
-  const int smem = stages * stage_bytes + 1024;
-  cudaError_t e;
-  if (stages == 3) {
-    e = cudaFuncSetAttribute(k_gemm_tc<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) k_gemm_tc<3><<<g, 256, smem, s>>>(p);
-  } else if (stages == 4) {
-    e = cudaFuncSetAttribute(k_gemm_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) k_gemm_tc<4><<<g, 256, smem, s>>>(p);
-  } else {
-    e = cudaFuncSetAttribute(k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) k_gemm_tc<2><<<g, 256, smem, s>>>(p);
+  const int ntn = (p.N + kTile - 1) / kTile, ntm = (p.M + kTile - 1) / kTile;
+  const int64_t nt64 = (int64_t)ntn * ntm * batch;
+  if (nt64 > INT32_MAX) return cudaErrorInvalidValue;
+  const int ntiles = (int)nt64;
+  static int nsm[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (nsm[dev] == 0) {
+    e = cudaDeviceGetAttribute(&nsm[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  const int grid = ntiles < nsm[dev] ? ntiles : nsm[dev];
+  // One persistent CTA per SM with the deepest ring (at most 6 stages) that fits next to the
+  // epilogue staging buffer.
+  constexpr int kAvail = 226 * 1024 - kStgBytes - 1024;
+  int stages = kAvail / stage_bytes;
+  if (stages > 6) stages = 6;
+  if (stages == 5) stages = 4;
+  if (stages < 2) return cudaErrorInvalidValue;
+  const int smem = stages * stage_bytes + kStgBytes + 1024;
+  switch (stages) {
+    case 2:
+      e = cudaFuncSetAttribute(k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_gemm_tc<2><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      break;
+    case 3:
+      e = cudaFuncSetAttribute(k_gemm_tc<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_gemm_tc<3><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      break;
+    case 4:
+      e = cudaFuncSetAttribute(k_gemm_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_gemm_tc<4><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      break;
+    default:
+      e = cudaFuncSetAttribute(k_gemm_tc<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess) k_gemm_tc<6><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      break;
   }
   if (e != cudaSuccess) return e;
   note_launch();

@@ -163,9 +163,19 @@ __global__ void k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU
   float best = -1.0f;
   int bidx = 0x7fffffff;
   if (c < cols) {
-    for (int r = ry; r < rows; r += 8) {
+    // rows visited in increasing order (first wins ties), eight loads in flight per thread
+    int r = ry;
+    for (; r + 56 < rows; r += 64) {
+      float a[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) a[k] = fabsf(u[(int64_t)(r + 8 * k) * ldu + c]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (a[k] > best) { best = a[k]; bidx = r + 8 * k; }
+    }
+    for (; r < rows; r += 8) {
       const float a = fabsf(u[(int64_t)r * ldu + c]);
-      if (a > best) { best = a; bidx = r; }   // rows visited in increasing order: first wins ties
+      if (a > best) { best = a; bidx = r; }
     }
   }
   bv[ry][cx] = best;
@@ -185,9 +195,11 @@ __global__ void k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU
   if (c >= cols) return;
   const float sg = sgn[cx];
   if (sg > 0.0f) return;
+#pragma unroll 8
   for (int r = ry; r < rows; r += 8) u[(int64_t)r * ldu + c] = -u[(int64_t)r * ldu + c];
   if (W) {
     float* w = W + (int64_t)blockIdx.y * sW;
+#pragma unroll 8
     for (int r = ry; r < w_rows; r += 8) w[(int64_t)r * ldw + c] = -w[(int64_t)r * ldw + c];
   }
 }
