@@ -279,8 +279,15 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
     // consecutive n of one row; outputs contiguous along m are stored from the registers
     // (consecutive lanes, consecutive m).
     float* stg = reinterpret_cast<float*>(smem + STAGES * stage_bytes) + e * (32 * 33);
-    const bool c_n = p.C && p.c_sn == 1, c_m = p.C && p.c_sn != 1;
+    const bool has_c = p.C != nullptr;
+    const bool c_n = has_c && p.c_sn == 1;
     const bool parts = p.ps[0] || p.pt[0];
+    // float32 C goes out as 16-byte vectors, 8 lanes on 32 consecutive entries of one row (n
+    // contiguous) or of one column (m contiguous), when the strides and the base allow it
+    const int64_t c_other = c_n ? p.c_sm : p.c_sn;
+    const bool c_vec = has_c && (p.c_sn == 1 || p.c_sm == 1) && (c_other % 4 == 0) && (p.c_sb % 4 == 0) &&
+                       (p.c_batch_in <= 0 || p.c_sb_out % 4 == 0) && (reinterpret_cast<uintptr_t>(p.C) & 15) == 0;
+    const int q8 = lane & 7, r4 = lane >> 3;
     int i = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
       const int ab = i & 1;
@@ -293,13 +300,13 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
       tc_fence_after();
       int n0, m0, b;
       tile_coords(t, ntn, ntm, n0, m0, b);
-      const int m = m0 + 32 * e + lane;
       int64_t boff;
       if (p.c_batch_in > 0) boff = (int64_t)(b / p.c_batch_in) * p.c_sb_out + (int64_t)(b % p.c_batch_in) * p.c_sb;
       else boff = (int64_t)b * p.c_sb;
-      float* C = p.C ? p.C + boff : nullptr;
+      float* C = has_c ? p.C + boff : nullptr;
       const int64_t poff = (int64_t)b * p.c_sb, toff = (int64_t)b * p.t_sb;
       const uint32_t tbase = tmem + (uint32_t)(ab * kTile) + ((uint32_t)(32 * e) << 16);
+      const int mr0 = m0 + 32 * e;   // first row of this warp's chunks
 #pragma unroll 1
       for (int c = 0; c < kTile / 32; ++c) {
         uint32_t r[32];
@@ -311,31 +318,53 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
-        if (c_n || parts) {
+        // staged as stg[m][n] (row stride 33: conflict-free by rows and by columns)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
-          __syncwarp();
-          if (c_n) {
-            const int n = n0 + c * 32 + lane;
-#pragma unroll 4
-            for (int rr = 0; rr < 32; ++rr) {
-              const int mm = m0 + 32 * e + rr;
-              if (mm < p.M && n < p.N) C[(int64_t)mm * p.c_sm + n] = stg[rr * 33 + lane];
+        for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
+        __syncwarp();
+        const int nc0 = n0 + c * 32;
+        if (has_c) {
+          if (c_vec) {
+            // lane = (vector q8 of 4 entries, line r4 + 4 k): n-contiguous lines are rows,
+            // m-contiguous lines are columns
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int ln = r4 + 4 * k;
+              const int mm = c_n ? mr0 + ln : mr0 + 4 * q8, nn = c_n ? nc0 + 4 * q8 : nc0 + ln;
+              float4 v4;
+              if (c_n) v4 = make_float4(stg[ln * 33 + 4 * q8], stg[ln * 33 + 4 * q8 + 1], stg[ln * 33 + 4 * q8 + 2],
+                                        stg[ln * 33 + 4 * q8 + 3]);
+              else v4 = make_float4(stg[(4 * q8) * 33 + ln], stg[(4 * q8 + 1) * 33 + ln], stg[(4 * q8 + 2) * 33 + ln],
+                                    stg[(4 * q8 + 3) * 33 + ln]);
+              float* dst = C + (int64_t)mm * p.c_sm + (int64_t)nn * p.c_sn;
+              const bool full = c_n ? (mm < p.M && nn + 3 < p.N) : (nn < p.N && mm + 3 < p.M);
+              if (full) {
+                *reinterpret_cast<float4*>(dst) = v4;
+              } else {
+                const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const int m2 = c_n ? mm : mm + u, n2 = c_n ? nn + u : nn;
+                  if (m2 < p.M && n2 < p.N) C[(int64_t)m2 * p.c_sm + (int64_t)n2 * p.c_sn] = vv[u];
+                }
+              }
+            }
+          } else {
+            const int m = mr0 + lane;
+            if (m < p.M) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int n = nc0 + j;
+                if (n < p.N) C[(int64_t)m * p.c_sm + (int64_t)n * p.c_sn] = stg[lane * 33 + j];
+              }
             }
           }
-          if (p.ps[0])
-            store_parts_chunk(p.ps, poff, p.c_sm, p.c_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
-          if (p.pt[0])
-            store_parts_chunk(p.pt, toff, p.t_sm, p.t_sn, stg, lane, m0 + 32 * e, n0 + 32 * c, p.M, p.N);
-          __syncwarp();
         }
-        if (c_m && m < p.M) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int n = n0 + c * 32 + j;
-            if (n < p.N) C[(int64_t)m * p.c_sm + (int64_t)n * p.c_sn] = __uint_as_float(r[j]);
-          }
+        if (parts) {
+          if (p.ps[0]) store_parts_chunk(p.ps, poff, p.c_sm, p.c_sn, stg, lane, mr0, nc0, p.M, p.N);
+          if (p.pt[0]) store_parts_chunk(p.pt, toff, p.t_sm, p.t_sn, stg, lane, mr0, nc0, p.M, p.N);
         }
+        __syncwarp();
       }
     }
   }
