@@ -77,18 +77,26 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf
 
 // y = [x | u] [Pi ; -N]: one float64 GEMM with K = D + r_t on the FP64 tensor-core MMA
 // (m8n8k4: a warp multiplies an 8 x 4 by a 4 x 8 block; fragments per the PTX ISA). A CTA
-// works on 256 tokens of one (layer-tensor, head) in tiles of 16 rows; warp w computes rows
-// 8 (w / 4) .. +7 and columns 32 (w % 4) .. +31 of the tile.
+// works on 256 tokens of one (layer-tensor, head) in tiles of 16 rows, with two groups of
+// eight warps taking alternate tiles: while one group multiplies, the other quantises and
+// packs, so the MMA pipe does not wait for the row-wise steps. Within a group, warp w computes
+// rows 8 (w / 4) .. +7 and columns 32 (w % 4) .. +31 of its tile; y stays in the
+// accumulators (the row absmax is combined through a 16 x 4 table in shared memory).
 __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
   asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
                : "+d"(d0), "+d"(d1)
                : "d"(a), "d"(b));
 }
 
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, 256;" ::"r"(1 + g) : "memory");
+}
+
 constexpr int kRows = 16;          // rows per tile
 constexpr int kPS = 132;           // row stride (floats) of Pi^T: conflict-free fragment loads
+constexpr int kGroups = 2;
 
-__global__ void __launch_bounds__(256, 1) k_residual(ResidualArgs a, const double* Nbuf, int R) {
+__global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const double* Nbuf, int R) {
   extern __shared__ __align__(16) unsigned char smraw[];
   const int chunk = blockIdx.x, h = blockIdx.y, i = blockIdx.z;
   const int lt = a.lt_ids[i];
@@ -98,18 +106,19 @@ __global__ void __launch_bounds__(256, 1) k_residual(ResidualArgs a, const doubl
   const int D = a.D;                       // 128
   const int K = D + rt;                    // GEMM depth
   const int SN = rt + 4;                   // row stride (doubles) of N^T
-  const int SA = K + 4;                    // row stride (doubles) of the A / y tile
-  float* PT = reinterpret_cast<float*>(smraw);                                   // [D][kPS]
-  double* NT = reinterpret_cast<double*>(PT + D * kPS);                          // [D][SN] = -N^T
-  double* At = NT + (size_t)D * SN;                                              // [kRows][SA]
-  unsigned char* cs = reinterpret_cast<unsigned char*>(At + (size_t)kRows * SA); // [kRows][D]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < D * D; e += 256) {
+  const int SA = K + 4;                    // row stride (floats) of an A tile
+  float* PT = reinterpret_cast<float*>(smraw);                                    // [D][kPS]
+  double* NT = reinterpret_cast<double*>(PT + D * kPS);                           // [D][SN] = -N^T
+  double* PM = NT + (size_t)D * SN;                                               // [2][kRows][4] row maxima
+  float* AT = reinterpret_cast<float*>(PM + kGroups * kRows * 4);                 // [2][kRows][SA]
+  unsigned char* CS = reinterpret_cast<unsigned char*>(AT + (size_t)kGroups * kRows * SA);   // [2][kRows][D]
+  const int tid = threadIdx.x;
+  for (int e = tid; e < D * D; e += 512) {
     const int k = e / D, n = e % D;
     PT[n * kPS + k] = a.Pi[e];
   }
   const double* Ng = Nbuf + (((int64_t)i * a.H + h) * R) * D;
-  for (int e = tid; e < rt * D; e += 256) {
+  for (int e = tid; e < rt * D; e += 512) {
     const int kk = e / D, n = e % D;
     NT[n * SN + kk] = -Ng[e];
   }
@@ -120,72 +129,81 @@ __global__ void __launch_bounds__(256, 1) k_residual(ResidualArgs a, const doubl
   const double half = (double)(1 << (b - 1));
   const int cmax = (1 << b) - 1;
   const int t_begin = chunk * kChunk, t_end = min(a.T, t_begin + kChunk);
+  // group g takes the tiles t_begin + (2 k + g) kRows
+  const int g = tid >> 8, gt = tid & 255, warp = gt >> 5, lane = tid & 31;
+  float* At = AT + (size_t)g * kRows * SA;
+  double* pm = PM + g * kRows * 4;
+  unsigned char* cs = CS + g * kRows * D;
   const int rg = warp >> 2, cg = warp & 3;
   const int ar = 8 * rg + (lane >> 2), ak = lane & 3;
   const int wpr = rowbytes / 4;                         // 32-bit words per packed row (4 b)
   const int c_first = (32 * lane) / b;                  // codes overlapping word `lane`
   const int c_last = min(D - 1, (32 * lane + 31) / b);
   __syncthreads();
-  // A tile: x rows (float64 of bf16 / float32) followed by u rows from 16-byte vector loads;
-  // thread (r = tid / 16, j = tid % 16) takes chunk j of row r (x) and chunk j of u (if any).
-  // The next tile's loads are issued before the current tile's GEMM and land in registers.
-  const int fr = tid >> 4, fj = tid & 15;
-  uint4 px[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)}, pu = make_uint4(0, 0, 0, 0);
+  // A tile: x rows followed by u rows, as float (bf16 and float32 inputs are exact), from
+  // 16-byte vector loads; thread (r = gt / 16, j = gt % 16) takes chunk j of row r (x) and
+  // chunk j of u (if any). The group's next tile is loaded into registers during the MMAs.
+  const int fr = gt >> 4, fj = gt & 15;
+  uint4 px0 = make_uint4(0, 0, 0, 0), px1 = make_uint4(0, 0, 0, 0), pu = make_uint4(0, 0, 0, 0);
   auto fetch = [&](int t0) {
     const int t = t0 + fr;
     const bool live = t < t_end;
-    px[0] = px[1] = pu = make_uint4(0, 0, 0, 0);
+    px0 = px1 = pu = make_uint4(0, 0, 0, 0);
     if (live) {
+      const uint4* xr = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t));
       if (a.xt == EL_BF16) {
-        px[0] = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[fj];
+        px0 = xr[fj];
       } else {
-        px[0] = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[2 * fj];
-        px[1] = reinterpret_cast<const uint4*>(x_row_ptr(a, lt, h, t))[2 * fj + 1];
+        px0 = xr[2 * fj];
+        px1 = xr[2 * fj + 1];
       }
       if (8 * fj < rt) pu = *reinterpret_cast<const uint4*>(UT + (int64_t)t * rt + 8 * fj);   // rt: multiple of 16
     }
   };
   auto stage = [&]() {
-    double* dst = At + fr * SA;
+    float* dst = At + fr * SA;
     if (a.xt == EL_BF16) {
-      const uint32_t wv[4] = {px[0].x, px[0].y, px[0].z, px[0].w};
+      const uint32_t wv[4] = {px0.x, px0.y, px0.z, px0.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        dst[8 * fj + 2 * q] = (double)__uint_as_float(wv[q] << 16);
-        dst[8 * fj + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
+        dst[8 * fj + 2 * q] = __uint_as_float(wv[q] << 16);
+        dst[8 * fj + 2 * q + 1] = __uint_as_float(wv[q] & 0xFFFF0000u);
       }
     } else {
+      const uint32_t wv[8] = {px0.x, px0.y, px0.z, px0.w, px1.x, px1.y, px1.z, px1.w};
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const uint32_t wv[4] = {px[q].x, px[q].y, px[q].z, px[q].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[8 * fj + 4 * q + e] = (double)__uint_as_float(wv[e]);
-      }
+      for (int e = 0; e < 8; ++e) dst[8 * fj + e] = __uint_as_float(wv[e]);
     }
     if (8 * fj < rt) {
       const uint32_t wv[4] = {pu.x, pu.y, pu.z, pu.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        dst[D + 8 * fj + 2 * q] = (double)__uint_as_float(wv[q] << 16);
-        dst[D + 8 * fj + 2 * q + 1] = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
+        dst[D + 8 * fj + 2 * q] = __uint_as_float(wv[q] << 16);
+        dst[D + 8 * fj + 2 * q + 1] = __uint_as_float(wv[q] & 0xFFFF0000u);
       }
     }
   };
-  fetch(t_begin);
-  for (int t0 = t_begin; t0 < t_end; t0 += kRows) {
+  // fp16 scale of a row from its absmax (round to nearest even, saturating at 65504)
+  auto row_scale = [&](int r) -> __half {
+    const double mx = fmax(fmax(pm[r * 4], pm[r * 4 + 1]), fmax(pm[r * 4 + 2], pm[r * 4 + 3]));
+    return mx >= 65504.0 ? __float2half_rn(65504.0f) : __double2half(mx);
+  };
+  const int t_first = t_begin + g * kRows;
+  if (t_first < t_end) fetch(t_first);
+  for (int t0 = t_first; t0 < t_end; t0 += kGroups * kRows) {
     stage();
-    __syncthreads();
-    if (t0 + kRows < t_end) fetch(t0 + kRows);
+    group_sync(g);
+    if (t0 + kGroups * kRows < t_end) fetch(t0 + kGroups * kRows);
     double acc[4][2];
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = 0.0;
-    const double* arow = At + ar * SA + ak;
+    const float* arow = At + ar * SA + ak;
     const float* pb = PT + (32 * cg + (lane >> 2)) * kPS + ak;    // fragment j at + 8 j kPS
     const double* qb = NT + (32 * cg + (lane >> 2)) * SN + ak;
     // K = D part (x Pi), fully unrolled so the fragment loads of later steps can be issued early
 #pragma unroll
     for (int k0 = 0; k0 < kD; k0 += 4) {
-      const double av = arow[k0];
+      const double av = (double)arow[k0];
 #pragma unroll
       for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[j][0], acc[j][1], av, (double)pb[8 * j * kPS + k0]);
     }
@@ -193,62 +211,61 @@ __global__ void __launch_bounds__(256, 1) k_residual(ResidualArgs a, const doubl
     for (int k0 = 0; k0 < rt; k0 += 16) {
 #pragma unroll
       for (int kk = 0; kk < 16; kk += 4) {
-        const double av = arow[kD + k0 + kk];
+        const double av = (double)arow[kD + k0 + kk];
 #pragma unroll
         for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[j][0], acc[j][1], av, qb[8 * j * SN + k0 + kk]);
       }
     }
-    __syncthreads();                                   // A no longer read: reuse it for y
+    // row absmax: this thread's 8 entries of row ar, the 4 lanes of the row, then the 4 warps
+    // of the row (columns 32 cg .. +31) through the table
+    double mx = 0.0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * cg + 8 * j + 2 * (lane & 3);
-      At[ar * SA + c] = acc[j][0];
-      At[ar * SA + c + 1] = acc[j][1];
+    for (int j = 0; j < 4; ++j) mx = fmax(mx, fmax(fabs(acc[j][0]), fabs(acc[j][1])));
+    mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if ((lane & 3) == 0) pm[ar * 4 + cg] = mx;
+    group_sync(g);
+    // codes: c = floor(y * (2^(b-1) / s) + 2^(b-1)), clamped, with one reciprocal per row
+    // (it can differ from a divide-per-entry only for values within ~1e-16 s of a cell boundary)
+    {
+      const double sd = (double)__half2float(row_scale(ar));
+      const double inv = sd > 0.0 ? half / sd : 0.0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int cc[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          int c = 0;
+          if (sd > 0.0) {
+            const double f = floor(fma(acc[j][e], inv, half));
+            c = f < 0.0 ? 0 : (f > (double)cmax ? cmax : (int)f);
+          }
+          cc[e] = c;
+        }
+        const int col = 32 * cg + 8 * j + 2 * (lane & 3);
+        *reinterpret_cast<uint16_t*>(cs + ar * D + col) = (uint16_t)(cc[0] | (cc[1] << 8));
+      }
     }
-    __syncthreads();
-    // quantise: warp w handles rows 2 w and 2 w + 1; lane owns features lane + 32 q. The
-    // code is floor(y * (2^(b-1) / s) + 2^(b-1)) with one reciprocal per row (it can differ
-    // from a divide-per-entry only for values within ~1e-16 s of a cell boundary).
+    group_sync(g);
+    // pack: warp w of the group handles rows 2 w and 2 w + 1; lane owns 32-bit word `lane`
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int r = 2 * warp + rr;
       const int t = t0 + r;
-      double y[4];
-      double mx = 0.0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        y[q] = At[r * SA + lane + 32 * q];
-        mx = fmax(mx, fabs(y[q]));
-      }
-      for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const __half sh = mx >= 65504.0 ? __float2half_rn(65504.0f) : __double2half(mx);
-      const double sd = (double)__half2float(sh);
-      const double inv = sd > 0.0 ? half / sd : 0.0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        int c = 0;
-        if (sd > 0.0) {
-          const double f = floor(fma(y[q], inv, half));
-          c = f < 0.0 ? 0 : (f > (double)cmax ? cmax : (int)f);
-        }
-        cs[r * D + lane + 32 * q] = (unsigned char)c;
-      }
-      __syncwarp();
       if (t < t_end) {
         const int64_t row = (int64_t)h * a.T + t;
-        if (lane < wpr) {                         // 32-bit word `lane` of the row's bit stream
+        if (lane < wpr) {
           uint32_t word = 0;
-          for (int i = c_first; i <= c_last; ++i) {
-            const int sh2 = i * b - 32 * lane;
-            const uint32_t cv = cs[r * D + i];
+          for (int q = c_first; q <= c_last; ++q) {
+            const int sh2 = q * b - 32 * lane;
+            const uint32_t cv = cs[r * D + q];
             word |= sh2 >= 0 ? (cv << sh2) : (cv >> (-sh2));
           }
           reinterpret_cast<uint32_t*>(codes + row * rowbytes)[lane] = word;
         }
-        if (lane == 0) scales[row] = sh;
+        if (lane == 0) scales[row] = row_scale(r);
       }
     }
-    __syncthreads();
   }
 }
 
@@ -263,12 +280,14 @@ cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStre
   if (e != cudaSuccess) return e;
   k_resid_prep<<<dim3(a.H, a.n_lt), 256, sp, s>>>(a, Nbuf, R);
   note_launch();
+  // Pi^T (float), -N^T (float64), the row-max tables, the two groups' A tiles (float) and codes
   const size_t sm = (size_t)kD * kPS * sizeof(float) + (size_t)kD * (R + 4) * sizeof(double) +
-                    (size_t)kRows * (kD + R + 4) * sizeof(double) + (size_t)kRows * kD;
+                    (size_t)kGroups * kRows * 4 * sizeof(double) +
+                    (size_t)kGroups * kRows * (kD + R + 4) * sizeof(float) + (size_t)kGroups * kRows * kD;
   e = cudaFuncSetAttribute(k_residual, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const dim3 g((a.T + kChunk - 1) / kChunk, a.H, a.n_lt);
-  k_residual<<<g, 256, sm, s>>>(a, Nbuf, R);
+  k_residual<<<g, 512, sm, s>>>(a, Nbuf, R);
   note_launch();
   return cudaGetLastError();
 }
