@@ -440,8 +440,9 @@ int cholqr_tc(jolt_plan_s* p, int rows, PartSet* sets, int cur, int passes, int3
     g.M = l; g.N = l; g.KB = (rows / nch + 63) / 64;
     g.C = p->Wpart; g.c_sm = l; g.c_sn = 1; g.c_sb = (int64_t)l * l;
     ck(gemm_tc(n * nch, g, s));
-    // chunk sums (float64, in order), Cholesky, inverse and the bf16 parts of R^{-T} in one launch
-    ck(chol_inv_parts(n, l, p->Wpart, nch, p->RTp, pass == 0 ? 1e-6 * l : 0.0, status, s));
+    ck(sum_heads(n, nch, (int64_t)l * l, p->Wpart, nullptr, p->Wg, s));
+    ck(chol_inv(n, l, p->Wg, (int64_t)l * l, p->Rinv, (int64_t)l * l, pass == 0 ? 1e-6 * l : 0.0, status, s));
+    ck(split_dual(n, l, l, p->Rinv, true, nullptr, p->RTp, s));
     TcGemmParams m;
     m.status = status;
     for (int i = 0; i < 3; ++i)

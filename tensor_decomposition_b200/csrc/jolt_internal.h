@@ -87,11 +87,6 @@ cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv
                      double shift, int32_t* status, cudaStream_t s);
 cudaError_t chol_inv_f32(int batch, int n, const float* W, int64_t sW, double* Rinv, int64_t sR,
                          double shift, int32_t* status, cudaStream_t s);
-// Same factorisation with W the float64 sum (in order) of `nparts` float32 partial matrices
-// [batch][nparts][n][n]; writes the three bf16 parts of R^{-T} ([batch][n][n], RT[1] and RT[2]
-// may be null) instead of a float64 R^{-1}.
-cudaError_t chol_inv_parts(int batch, int n, const float* Wparts, int nparts, __nv_bfloat16* const* RT,
-                           double shift, int32_t* status, cudaStream_t s);
 // Column sign rule: largest |entry| of each column positive (lowest index on ties).
 // Signs are computed on U (rows x cols, row stride ldu) and applied to U and to the
 // optional companion W (w_rows x cols, row stride ldw).

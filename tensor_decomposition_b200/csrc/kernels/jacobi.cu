@@ -647,9 +647,8 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
 //  * Inverse, right-looking block forward substitution of L X = I: X_k = L_kk^{-1} B_k, then
 //    B_i -= L_ik X_k for the block rows below (B = I initially, kept transposed in T).
 template <typename TW>
-__global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, int nparts, double* Rinv,
-                                                  int64_t sR, __nv_bfloat16* rt0, __nv_bfloat16* rt1,
-                                                  __nv_bfloat16* rt2, double shift, int32_t* status) {
+__global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
+                                                  int64_t sR, double shift, int32_t* status) {
   constexpr int NP = kMaxN, LD = kMaxN + 1, BS = 16, NBLK = NP / BS;
   extern __shared__ double dm[];
   double* A = dm;                          // NP x LD
@@ -660,30 +659,18 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   __shared__ double tr_s;
   __shared__ int floored;
   const int tid = threadIdx.x, lane = tid & 31;
-  // W of this problem is the float64 sum, in order, of its nparts partial matrices
-  const TW* w = W + (int64_t)blockIdx.x * nparts * sW;
+  const TW* w = W + (int64_t)blockIdx.x * sW;
   if (tid == 0) floored = 0;
-  // all 32 loads of a part in flight at once (32 elements per thread), parts added in order
-  double wv[NP * NP / 512];
+  // every load of W in flight before the first barrier (32 elements per thread)
+  TW wv[NP * NP / 512];
 #pragma unroll
-  for (int q = 0; q < NP * NP / 512; ++q) wv[q] = 0.0;
-  for (int pp = 0; pp < nparts; ++pp) {
-    TW tv[NP * NP / 512];
-#pragma unroll
-    for (int q = 0; q < NP * NP / 512; ++q) {
-      const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
-      tv[q] = (c <= r && r < n) ? w[(int64_t)pp * sW + (int64_t)r * n + c] : (TW)0;
-    }
-#pragma unroll
-    for (int q = 0; q < NP * NP / 512; ++q) wv[q] += (double)tv[q];
+  for (int q = 0; q < NP * NP / 512; ++q) {
+    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+    wv[q] = (c <= r && r < n) ? w[(int64_t)r * n + c] : (TW)0;
   }
   if (tid < 32) {
     double t = 0.0;
-    for (int i = tid; i < n; i += 32) {
-      double v = 0.0;
-      for (int pp = 0; pp < nparts; ++pp) v += (double)w[(int64_t)pp * sW + (int64_t)i * n + i];
-      t += v;
-    }
+    for (int i = tid; i < n; i += 32) t += (double)w[(int64_t)i * n + i];
     for (int o = 16; o > 0; o >>= 1) t += __shfl_down_sync(0xffffffffu, t, o);
     if (tid == 0) tr_s = t;
   }
@@ -695,7 +682,7 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
 #pragma unroll
   for (int q = 0; q < NP * NP / 512; ++q) {
     const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
-    double v = (c <= r && r < n) ? wv[q] + (r == c ? add : 0.0) : 0.0;
+    double v = (c <= r && r < n) ? (double)wv[q] + (r == c ? add : 0.0) : 0.0;
     if (r >= n && r == c) v = 1.0;
     A[r * LD + c] = v;
   }
@@ -763,27 +750,10 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
     }
     __syncthreads();
   }
-  if (Rinv) {
-    double* o = Rinv + (int64_t)blockIdx.x * sR;
-    for (int e = tid; e < n * n; e += 512) {
-      const int r = e / n, c = e - r * n;
-      o[e] = (c >= r) ? A[r * LD + c] : 0.0;
-    }
-  }
-  if (rt0) {
-    // three bf16 parts of R^{-T} (entry (c, r) = R^{-1}[r][c]): v = h0 + h1 + h2 with each
-    // remainder formed in float64
-    const int64_t ob = (int64_t)blockIdx.x * n * n;
-    for (int e = tid; e < n * n; e += 512) {
-      const int c = e / n, r = e - c * n;
-      const double v = (c >= r) ? A[r * LD + c] : 0.0;
-      const __nv_bfloat16 h0 = __double2bfloat16(v);
-      const double r1 = v - (double)__bfloat162float(h0);
-      const __nv_bfloat16 h1 = __double2bfloat16(r1);
-      rt0[ob + e] = h0;
-      if (rt1) rt1[ob + e] = h1;
-      if (rt2) rt2[ob + e] = __double2bfloat16(r1 - (double)__bfloat162float(h1));
-    }
+  double* o = Rinv + (int64_t)blockIdx.x * sR;
+  for (int e = tid; e < n * n; e += 512) {
+    const int r = e / n, c = e - r * n;
+    o[e] = (c >= r) ? A[r * LD + c] : 0.0;
   }
   (void)lane;
 }
@@ -827,34 +797,28 @@ cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int
 }
 
 template <typename TW>
-static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, int nparts, double* Rinv, int64_t sR,
-                              __nv_bfloat16* const* rt, double shift, int32_t* status, cudaStream_t s) {
-  if (n <= 0 || n > kMaxN || nparts < 1) return cudaErrorInvalidValue;
+static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, double* Rinv, int64_t sR, double shift,
+                              int32_t* status, cudaStream_t s) {
+  if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
   if (batch <= 0) return cudaSuccess;
   // A (128 x 129), diagonal-block inverses (8 x 16 x 16), panel (16 x 128), diagonal factor
   // (16 x 17) and its reciprocal diagonal (16), float64
   const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 8 * 256 + 16 * kMaxN + 16 * 17 + 16) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_chol_inv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, nparts, Rinv, sR, rt ? rt[0] : nullptr, rt ? rt[1] : nullptr,
-                                          rt ? rt[2] : nullptr, shift, status);
+  k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv, int64_t sR,
                      double shift, int32_t* status, cudaStream_t s) {
-  return chol_inv_t<double>(batch, n, W, sW, 1, Rinv, sR, nullptr, shift, status, s);
+  return chol_inv_t<double>(batch, n, W, sW, Rinv, sR, shift, status, s);
 }
 
 cudaError_t chol_inv_f32(int batch, int n, const float* W, int64_t sW, double* Rinv, int64_t sR,
                          double shift, int32_t* status, cudaStream_t s) {
-  return chol_inv_t<float>(batch, n, W, sW, 1, Rinv, sR, nullptr, shift, status, s);
-}
-
-cudaError_t chol_inv_parts(int batch, int n, const float* Wparts, int nparts, __nv_bfloat16* const* RT,
-                           double shift, int32_t* status, cudaStream_t s) {
-  return chol_inv_t<float>(batch, n, Wparts, (int64_t)n * n, nparts, nullptr, 0, RT, shift, status, s);
+  return chol_inv_t<float>(batch, n, W, sW, Rinv, sR, shift, status, s);
 }
 
 }  // namespace jolt
