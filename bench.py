@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--encoder", choices=["sketch", "exact"], default="sketch")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true", help="skip the in-codec baselines (quantisation only, Tucker only)")
     ap.add_argument("--profile-out", default=None, help="write the per-phase trace JSON here")
     return ap.parse_args()
 
@@ -217,6 +218,58 @@ def run_reference(args):
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
+
+
+def in_codec_baselines(J, cfg, K, V, budget, encoder, steps=5, warmup=2):
+    """The codec restricted to its baselines on the same cache and budget: residual only
+    (factors = 0, b = 4: per-row 4-bit quantisation of the rotated rows) and Tucker only
+    (b = 0), plus JoLT itself at the 4-bit baseline's byte count, so that the errors compare at
+    equal bytes. Each is timed over `steps` device-timed steps (encode + decode + the two
+    errors, as the main step) after `warmup`; none of this is inside the main timed region."""
+    import torch
+    bf16_bytes = (K.numel() + V.numel()) * 2
+    Ko, Vo = torch.empty_like(K), torch.empty_like(V)
+    res = {}
+
+    def run(name, bits, factors, bud):
+        c = J.jolt_config_default()
+        c.encoder = encoder
+        c.split_kv_budget = int(cfg.split_kv)
+        c.bits_mask = sum(1 << b for b in bits)
+        c.factors = factors
+        plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, bud,
+                           cfg.groups, c)
+        errs = [None, None]
+
+        def step():
+            st = J.jolt_encode(plan, K, V, SEED)
+            J.jolt_decode(st, Ko, Vo)
+            errs[0] = J.jolt_rel_frob_error(K, Ko)
+            errs[1] = J.jolt_rel_frob_error(V, Vo)
+            return st
+
+        for _ in range(warmup):
+            st = step()
+        J.jolt_stream_status(st)
+        info = J.jolt_stream_info(st, cfg.groups)
+        nbytes = int(sum(info["bytes_by_part"].values()))
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            st = step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        res[name] = {"rel_frob_error": {"K": errs[0], "V": errs[1]}, "compressed_bytes": nbytes,
+                     "ratio": bf16_bytes / nbytes, "budget_bytes": int(bud),
+                     "tokens_per_s": cfg.tokens / (ms / 1e3), "ms_per_step": ms,
+                     "alloc": info["alloc"].tolist()}
+
+    run("residual_only_b4", (4,), 0, budget)
+    run("tucker_only", (0,), 1, budget)
+    run("jolt_at_residual_only_b4_bytes", cfg.bits, 1, res["residual_only_b4"]["compressed_bytes"])
+    return res
 
 
 def job_throughput(local_ms, tokens, steps, world, device):
@@ -427,6 +480,8 @@ def main():
            "roofline": roof,
            "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
                       "samples": clk["samples"]}}
+    if rank == 0 and not args.no_baselines:
+        out["in_codec_baselines"] = in_codec_baselines(J, cfg, K, V, budget, c.encoder)
     if args.profile_out and rank == 0:
         json.dump(prof, open(args.profile_out, "w"), indent=1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

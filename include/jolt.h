@@ -80,6 +80,11 @@ typedef struct {
   uint32_t bits_mask;        /* bit b set => residual bit-width b allowed (0x1FF = 0..8) */
   int32_t split_kv_budget;   /* 0: one budget pool for K and V; 1: half the budget each */
   int32_t max_jacobi_sweeps; /* eigensolver sweep limit (30) */
+  int32_t factors;           /* 1 (default): Tucker factors on the candidate grid; 0: residual
+                                only, r_t = r_d = 0 for every layer-tensor (with bits_mask = 1 << b
+                                this is per-row b-bit quantisation of the rotated cache, the
+                                quantisation-only in-codec baseline; the factor analysis is
+                                skipped). The Tucker-only baseline is bits_mask = 1 (b = 0). */
 } jolt_config;
 
 typedef struct jolt_plan_s* jolt_plan_t;

@@ -506,6 +506,7 @@ JOLT_API void jolt_config_default(jolt_config* c) {
   c->rank_step = 16;
   c->rt_max = 0;
   c->bits_mask = 0x1FFu;
+  c->factors = 1;
   c->split_kv_budget = 0;
   c->max_jacobi_sweeps = 30;
 }
@@ -536,6 +537,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   if ((cfg.bits_mask & 0x1FFu) == 0 || (cfg.bits_mask & ~0x1FFu))
     return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: bits_mask must select widths in 0..8");
   if (cfg.rt_max < 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: rt_max < 0");
+  if (cfg.factors != 0 && cfg.factors != 1) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: factors must be 0 or 1");
   if (byte_budget == 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: zero byte budget");
 
   jolt_plan_s* p = new (std::nothrow) jolt_plan_s();
@@ -553,6 +555,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   const int64_t per_lt = (int64_t)(byte_budget / (uint64_t)p->n_lt);
   int cap = 112;
   if (cfg.rt_max > 0) cap = std::min(cap, (int)cfg.rt_max);
+  if (cfg.factors == 0) cap = 0;   // residual only: the grid is the single point r_t = r_d = 0
   int64_t R = std::min<int64_t>({(int64_t)T, (int64_t)H * D, per_lt / (2 * (int64_t)T), (int64_t)cap});
   R -= R % p->step;
   p->R = (int)std::max<int64_t>(0, R);
@@ -759,6 +762,16 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       CK(sumsq_batched(L, HTD, X[k], xt, HTD, p->xx + (int64_t)k * L, p->xx_part + (int64_t)k * L * 64,
                        status, s));
     }
+  }
+  // residual only (factors = 0): the grid is the single point r_t = r_d = 0, whose energy is
+  // ||X||^2; no factor, core or sketch is needed
+  if (p->cfg.factors == 0) {
+    PROF("energy_table", s);
+    TableArgs ta;
+    ta.n_lt = n; ta.H = H; ta.R = 0; ta.D = D; ta.step = p->step; ta.lt_ids = p->d_lt_ids;
+    ta.Gmax = p->Gmax; ta.xx = p->xx; ta.E = p->E; ta.ngrid = p->ngrid;
+    CK(energy_table(ta, s));
+    return JOLT_OK;
   }
   CUtensorMap mx[2], mxt;
   if (p->use_tc) {

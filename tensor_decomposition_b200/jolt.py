@@ -47,7 +47,8 @@ class Config(ctypes.Structure):
     _fields_ = [("encoder", ctypes.c_int32), ("oversample", ctypes.c_int32),
                 ("power_iters", ctypes.c_int32), ("rank_step", ctypes.c_int32),
                 ("rt_max", ctypes.c_int32), ("bits_mask", ctypes.c_uint32),
-                ("split_kv_budget", ctypes.c_int32), ("max_jacobi_sweeps", ctypes.c_int32)]
+                ("split_kv_budget", ctypes.c_int32), ("max_jacobi_sweeps", ctypes.c_int32),
+                ("factors", ctypes.c_int32)]
 
 
 def _load():

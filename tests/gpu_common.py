@@ -2,6 +2,7 @@
 compare with the CPU oracle on the same seeded inputs."""
 from __future__ import annotations
 
+import copy
 import numpy as np
 
 import synth
@@ -159,3 +160,81 @@ def check_allocation(J, st, ost, op, cfg):
     alloc_o, _ = oj.allocate(op, units)
     assert np.array_equal(alloc_o, ost.alloc)
     return units
+
+
+def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits=None, factors=1):
+    """Encode and decode a whole workload on the GPU in the launch configuration bench.py
+    times and check it on sampled layer-tensors against the oracle: the allocation (whole
+    cache), principal angles of the factors (when the plan has them), residual codes, the decode
+    and the relative error at the GPU's allocation. `bits` restricts the residual widths and
+    `factors = 0` forces r_t = r_d = 0 (the in-codec baselines)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    K, V = synth.gen_cache_torch(cfg, dev, seq=seq)
+    budget = synth.kv.budget_bytes(cfg, ratio)
+    c = J.jolt_config_default()
+    c.encoder = J.JOLT_ENC_SKETCH if encoder == "sketch" else J.JOLT_ENC_EXACT
+    c.split_kv_budget = int(cfg.split_kv)
+    mask = 0
+    for b in (bits or cfg.bits):
+        mask |= 1 << b
+    c.bits_mask = mask
+    c.factors = factors
+    plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, budget,
+                       cfg.groups, c)
+    st = J.jolt_encode(plan, K, V, seed)
+    J.jolt_stream_status(st)
+    Ko, Vo = torch.empty_like(K), torch.empty_like(V)
+    J.jolt_decode(st, Ko, Vo)
+    torch.cuda.synchronize()
+    ost = ostream.parse(J.jolt_stream_to_host(st), lts=set(sample))
+    op = oracle_plan(cfg, budget, encoder, bits=bits, **({} if factors else {"rt_cap": 0}))
+    assert ost.rt_max == op.R()
+    check_allocation(J, st, ost, op, cfg)
+    Pi = J.jolt_export_debug(st, J.JOLT_DBG_PI).reshape(128, 128).astype(np.float64)
+    report = {"alloc": ost.alloc.tolist()}
+    for lt in sample:
+        l, k = lt // 2, lt % 2
+        X = host((K if k == 0 else V)[l])
+        worst, where = 0.0, None
+        a = oj.analyse_layer_tensor(op, X, seed, lt, spec=False) if factors else None
+        UD = J.jolt_export_debug(st, J.JOLT_DBG_UD_F32, lt).reshape(128, 128).astype(np.float64) if factors else None
+        kd = leading_count(a["wD"], 128) if factors else 0
+        if kd:
+            ang = oj.principal_angles(UD[:, :kd], a["U_D"][:, :kd]).max()
+            if ang > worst:
+                worst, where = ang, ("U_D", kd)
+        if op.R() and factors:
+            UT = J.jolt_export_debug(st, J.JOLT_DBG_UT_F32, lt).reshape(cfg.tokens, op.R()).astype(np.float64)
+            kt = leading_count(a["wT"], op.R())
+            if kt:
+                ang = oj.principal_angles(UT[:, :kt], a["U_T_unrounded"][:, :kt]).max()
+                if ang > worst:
+                    w = np.asarray(a["wT"], dtype=np.float64)
+                    worst, where = ang, ("U_T", kt, float((w[kt - 1] - w[kt]) / w[0]),
+                                         [float(np.arccos(np.clip(abs(UT[:, j] @ a["U_T_unrounded"][:, j]) /
+                                                                  np.linalg.norm(UT[:, j]), 0, 1))) for j in range(kt)])
+        assert worst < ANGLE_TOL, (lt, worst, where)
+        # codes of this layer-tensor
+        out_band, in_band, scale_bad, total = codes_parity(only_lt(ost, lt), {lt: X}, Pi)
+        assert scale_bad == 0 and out_band == 0, (lt, scale_bad, out_band, in_band, total)
+        # decode of this layer-tensor
+        ref = oj.round_output(oj.decode_lt(ost, lt, Pi=None), ost.out_f32)
+        got = host((Ko if k == 0 else Vo)[l])
+        assert (np.abs(got - ref) <= decode_tol(ref, ost.out_f32)).all(), (lt, np.abs(got - ref).max())
+        # error at the GPU's allocation
+        g = [gg for gg, lay in enumerate(oj.group_ranges(cfg.layers, op.num_groups)) if l in lay][0]
+        rt, rd, b = (int(v) for v in ost.alloc[g, k])
+        rec, _ = oracle_lt_reconstruction(op, X, seed, lt, rt, rd, b)
+        e_gpu, e_orc = oj.rel_frob(X, got), oj.rel_frob(X, rec)
+        assert abs(e_gpu / e_orc - 1.0) <= REL_ERR_TOL, (lt, e_gpu, e_orc)
+        report[lt] = dict(max_angle=worst, codes=total, boundary_mismatches=in_band, err=(e_gpu, e_orc))
+    J.jolt_stream_status(st)
+    return report
+
+
+def only_lt(ost, lt):
+    """A shallow copy of the parsed stream that holds one layer-tensor (codes_parity walks all)."""
+    one = copy.copy(ost)
+    one.lts = {lt: ost.lts[lt]}
+    return one

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(jolt):
 def test_config_defaults(jolt):
     c = jolt.jolt_config_default()
     assert (c.encoder, c.oversample, c.power_iters, c.rank_step, c.rt_max, c.bits_mask,
-            c.split_kv_budget, c.max_jacobi_sweeps) == (0, 16, 1, 16, 0, 0x1FF, 0, 30)
+            c.split_kv_budget, c.max_jacobi_sweeps, c.factors) == (0, 16, 1, 16, 0, 0x1FF, 0, 30, 1)
 
 
 @pytest.mark.parametrize("args", [
@@ -71,6 +71,10 @@ def test_plan_rejects_bad_options(jolt):
         jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 10 ** 6, 1, c)
     c = jolt.jolt_config_default()
     c.rank_step = 48
+    with pytest.raises(jolt.JoltError):
+        jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 10 ** 6, 1, c)
+    c = jolt.jolt_config_default()
+    c.factors = 2                    # 0 (residual only) or 1
     with pytest.raises(jolt.JoltError):
         jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 10 ** 6, 1, c)
 
