@@ -85,6 +85,11 @@ typedef struct {
                                 this is per-row b-bit quantisation of the rotated cache, the
                                 quantisation-only in-codec baseline; the factor analysis is
                                 skipped). The Tucker-only baseline is bits_mask = 1 (b = 0). */
+  int32_t measured_b;        /* 0 (default): the dual's errors use the phi(b) quantiser model.
+                                1: measured-b refinement: after the dual, one extra pass of the
+                                residual coder measures the exact squared error of every allowed
+                                b at each unit's chosen ranks, and a second dual re-chooses b per
+                                unit with those errors (ranks unchanged). */
 } jolt_config;
 
 typedef struct jolt_plan_s* jolt_plan_t;
@@ -101,7 +106,10 @@ enum { JOLT_DBG_PI = 0,        /* float32 [D][D] rotation Pi used by encode */
        JOLT_DBG_TABLE = 3,     /* float64 per-unit error table, unit = lt (group*2 + kind) */
        JOLT_DBG_XX = 4,        /* float64 [2*L] squared Frobenius norm of every layer-tensor */
        JOLT_DBG_LAMBDA = 5,    /* float64 [2] dual variable of each budget pool */
-       JOLT_DBG_OMEGA = 6 };   /* bf16 bits [HD][l] sketch matrix of layer-tensor lt */
+       JOLT_DBG_OMEGA = 6,     /* bf16 bits [HD][l] sketch matrix of layer-tensor lt */
+       JOLT_DBG_MEAS = 7 };    /* float64 [9] measured squared error of residual width b (index b,
+                                  zero for widths not allowed) at the chosen ranks, layer-tensor
+                                  lt; plans with measured_b = 1 only */
 
 JOLT_API void jolt_config_default(jolt_config* cfg);
 

@@ -350,6 +350,7 @@ class Plan:
     bits: tuple = tuple(range(9))
     split_kv: bool = False
     out_f32: bool = False
+    measured_b: bool = False   # re-choose b per unit with measured quantisation errors
 
     def kinds(self):
         return (0, 1) if self.has_v else (0,)
@@ -459,6 +460,49 @@ def allocate(plan: Plan, units):
     return alloc, lams
 
 
+def measure_b_errors(plan: Plan, tens: dict, A: dict, alloc, Pi, spec: bool = True):
+    """Exact squared error of every allowed b at each unit's chosen ranks (the refinement of the
+    phi(b) model, §8f-1 of the reading): with Y the rotated residual of the stored factors,
+    ||Y||^2 for b = 0 and ||Y - dequant(quant_b(Y))||^2 for b > 0, summed over the unit's
+    layers. Returns {(group, kind): {b: error}}."""
+    meas = {}
+    for g, lay in enumerate(group_ranges(plan.L, plan.num_groups)):
+        for k in plan.kinds():
+            rt, rd = int(alloc[g, k][0]), int(alloc[g, k][1])
+            acc = {int(b): 0.0 for b in plan.bits}
+            for l in lay:
+                lt = l * KINDS + k
+                a = A[lt]
+                G = a["Gmax"][:, :rt, :rd]
+                if spec:
+                    G = round_bf16(G)
+                Y = residual_rotated(tens[k][l], a["U_T"][:, :rt], G, a["U_D"][:, :rd], Pi)
+                for b in plan.bits:
+                    b = int(b)
+                    if b == 0:
+                        acc[b] += float(np.sum(Y * Y))
+                    else:
+                        s, c, _ = quantize_rows(Y, b, spec)
+                        d = Y - dequantize_rows(s, c, b)
+                        acc[b] += float(np.sum(d * d))
+            meas[(g, k)] = acc
+    return meas
+
+
+def refine_b(plan: Plan, units, alloc, meas):
+    """Second dual: every unit keeps the ranks of `alloc` and re-chooses b with the measured
+    errors (candidates at other ranks take an infinite error, so they are never chosen; the
+    bytes, tie-break and lambda search are those of the first dual). Returns (alloc, lambdas)."""
+    units2 = []
+    for u in units:
+        rt, rd = int(alloc[u.group, u.kind][0]), int(alloc[u.group, u.kind][1])
+        m = meas[(u.group, u.kind)]
+        err = np.array([m[int(b)] if (int(r1) == rt and int(r2) == rd) else np.inf
+                        for b, r1, r2 in zip(u.b, u.rt, u.rd)])
+        units2.append(Unit(u.group, u.kind, err, u.nbytes, u.b, u.rt, u.rd, u.energy))
+    return allocate(plan, units2)
+
+
 def encode(plan: Plan, K, V, seed: int, spec: bool = True, alloc=None, factors=None,
            Pi=None, keep=False):
     """Full encode. K, V: [L][H][T][D] arrays (V may be None). Returns (OracleStream, debug).
@@ -480,8 +524,12 @@ def encode(plan: Plan, K, V, seed: int, spec: bool = True, alloc=None, factors=N
             A[lt] = analyse_layer_tensor(plan, tens[k][l], seed, lt, spec, f)
     units = build_units(plan, {lt: a["E"] for lt, a in A.items()}, kap)
     lams = None
+    meas = None
     if alloc is None:
         alloc, lams = allocate(plan, units)
+        if plan.measured_b:
+            meas = measure_b_errors(plan, tens, A, alloc, Pi, spec)
+            alloc, lams = refine_b(plan, units, alloc, meas)
     st = OracleStream(plan.L, plan.H, plan.T, plan.D, plan.has_v, plan.num_groups, seed,
                       plan.encoder, plan.rank_step, plan.R(), plan.split_kv, plan.out_f32,
                       np.asarray(alloc, dtype=np.int64))
@@ -504,7 +552,7 @@ def encode(plan: Plan, K, V, seed: int, spec: bool = True, alloc=None, factors=N
                     s = np.zeros((plan.H, 0))
                     c = np.zeros((plan.H, plan.T, 0), dtype=np.int64)
                 st.lts[lt] = LTCode(rt, rd, b, U_T, U_D, G, s, c)
-    dbg = dict(analysis=A, units=units, lambdas=lams, kappa=kap, Pi=Pi)
+    dbg = dict(analysis=A, units=units, lambdas=lams, kappa=kap, Pi=Pi, measured=meas)
     return st, dbg
 
 

@@ -233,6 +233,7 @@ struct jolt_plan_s {
         *VT = nullptr, *lamT = nullptr;
   double *BB = nullptr, *CT = nullptr;   // sketch and token Grams, float64
   double *Wg = nullptr, *Rinv = nullptr, *E = nullptr, *unit_err = nullptr, *Nbuf = nullptr;
+  double *meas_part = nullptr, *meas_lt = nullptr;   // measured-b refinement
   float* Qfinal = nullptr;   // final sketch basis (one of Y / Y2)
   bool q_t = false;          // Qfinal stored as Q^T [l][T] (tensor-core path) instead of Q [T][l]
   bool use_tc = false;       // bf16 inputs with T % 8 == 0: contractions over X on tcgen05
@@ -507,6 +508,7 @@ JOLT_API void jolt_config_default(jolt_config* c) {
   c->rt_max = 0;
   c->bits_mask = 0x1FFu;
   c->factors = 1;
+  c->measured_b = 0;
   c->split_kv_budget = 0;
   c->max_jacobi_sweeps = 30;
 }
@@ -538,6 +540,8 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: bits_mask must select widths in 0..8");
   if (cfg.rt_max < 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: rt_max < 0");
   if (cfg.factors != 0 && cfg.factors != 1) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: factors must be 0 or 1");
+  if (cfg.measured_b != 0 && cfg.measured_b != 1)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: measured_b must be 0 or 1");
   if (byte_budget == 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: zero byte budget");
 
   jolt_plan_s* p = new (std::nothrow) jolt_plan_s();
@@ -652,6 +656,10 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     take(p->E, 2 * (int64_t)L * p->ngrid);
     take(p->unit_err, 2 * (int64_t)p->G * p->nbits * p->ngrid);
     take(p->Nbuf, n * H * Rm * D);
+    if (cfg.measured_b) {
+      take(p->meas_part, n * H * ((T + 255) / 256) * 9);
+      take(p->meas_lt, n * 9);
+    }
     take(p->Gpi, (int64_t)D * D);
     take(p->Pi32, (int64_t)D * D);
     take(p->Pib, (int64_t)D * D);
@@ -1268,6 +1276,33 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, ui
   ra.n_lt = p->n_lt; ra.H = sh.heads; ra.T = sh.tokens; ra.D = D; ra.lt_ids = p->d_lt_ids;
   ra.X[0] = K; ra.X[1] = V; ra.xt = sh.dtype == JOLT_BF16 ? EL_BF16 : EL_F32; ra.Pi = st->d_Pi;
   ra.meta = st->d_meta; ra.body = st->d_body;
+  if (p->cfg.measured_b) {
+    // measured-b refinement: exact errors of every allowed width at the chosen ranks (one pass of
+    // the residual coder that writes no codes), then a second dual over b with those errors; the
+    // layout and the packed factors follow the new widths
+    ResidualArgs rm = ra;
+    rm.measure = 1;
+    rm.bits_mask = p->cfg.bits_mask;
+    rm.meas_part = p->meas_part;
+    {
+      PROF("measure_b", s);
+      e = residual_encode(rm, p->Nbuf, std::max(p->R, 1), s);
+      if (e == cudaSuccess) e = measured_tables(da, p->meas_part, (sh.tokens + 255) / 256, p->meas_lt, s);
+    }
+    if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "measure_b: %s", cudaGetErrorString(e)));
+    DualArgs d2 = da;
+    d2.tables_ready = 1;
+    {
+      PROF("dual", s);
+      e = dual_allocate(d2, s);
+    }
+    if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "dual: %s", cudaGetErrorString(e)));
+    {
+      PROF("pack", s);
+      e = pack_factors(pa, s);
+    }
+    if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "pack: %s", cudaGetErrorString(e)));
+  }
   {
     PROF("residual", s);
     e = residual_encode(ra, p->Nbuf, std::max(p->R, 1), s);
@@ -1589,6 +1624,16 @@ JOLT_API jolt_status jolt_export_debug(jolt_stream_t st, int32_t what, int32_t l
         src = p->unit_err + (int64_t)lt * p->nbits * p->ngrid;
         n = sizeof(double) * p->nbits * p->ngrid;
         break;
+      case JOLT_DBG_MEAS: {
+        if (!p->meas_lt) return fail(JOLT_ERR_INVALID_ARG, "the plan has no measured-b refinement");
+        int i = -1;
+        for (size_t j = 0; j < p->lt_ids.size(); ++j)
+          if (p->lt_ids[j] == lt) i = (int)j;
+        if (i < 0) return fail(JOLT_ERR_INVALID_ARG, "bad layer-tensor");
+        src = p->meas_lt + (int64_t)i * 9;
+        n = sizeof(double) * 9;
+        break;
+      }
       case JOLT_DBG_XX:
         tmp.assign(2 * (size_t)st->L, 0.0);
         for (size_t j = 0; j < p->lt_ids.size(); ++j)

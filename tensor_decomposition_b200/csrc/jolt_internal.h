@@ -130,8 +130,15 @@ struct DualArgs {
   double* unit_err;   // [G*2][nbits*ngrid] debug copy of the tables
   const int32_t* cand_order;   // [nbits*ngrid] candidates (bi * ngrid + grid) by (bytes, b, r_t, r_d)
   StreamMeta* meta;
+  int tables_ready = 0;        // 1: unit_err is already filled (second dual of the measured-b refinement)
 };
 cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s);
+// Measured-b refinement: per-layer-tensor sums of the residual coder's partial errors
+// meas_part [n_lt][H][nchunk][9] (fixed order) into meas_lt [n_lt][9], and the units' tables
+// for the second dual: the measured error of each allowed b at the unit's chosen ranks (from
+// meta->alloc), +inf at every other rank.
+cudaError_t measured_tables(const DualArgs& a, const double* meas_part, int nchunk, double* meas_lt,
+                            cudaStream_t s);
 
 struct PackArgs {
   int n_lt, H, T, D, R;
@@ -152,6 +159,12 @@ struct ResidualArgs {
   const float* Pi;           // [D][D] float32
   const StreamMeta* meta;
   uint8_t* body;
+  // measured-b refinement: measure = 1 writes no codes; every layer-tensor (whatever its b) adds
+  // its exact squared quantisation error for each width in bits_mask (b = 0: ||y||^2) into
+  // meas_part [n_lt][H][ceil(T / 256)][9], one fixed-order sum per CTA
+  int measure = 0;
+  uint32_t bits_mask = 0;
+  double* meas_part = nullptr;
 };
 // Nbuf: float64 scratch [n_lt][H][R][D] for N_h = (G_h U_D^T) Pi.
 cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStream_t s);

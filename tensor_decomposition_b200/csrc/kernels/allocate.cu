@@ -128,6 +128,39 @@ __global__ void k_unit_tables(DualArgs a) {
   }
 }
 
+// Measured-b refinement. meas_lt[i][b] = sum over (head, chunk), in order, of the residual
+// coder's per-CTA sums; then one thread per (unit, allowed width): the unit's error for that
+// width is the sum over its layers (increasing layer order) of meas_lt, entered at the grid
+// point of the unit's chosen ranks (meta->alloc); every other grid point takes +inf, so the
+// second dual re-chooses b only.
+__global__ void k_meas_lt(int n_lt, int H, int nchunk, const double* meas_part, double* meas_lt) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n_lt * 9; e += gridDim.x * blockDim.x) {
+    const int i = e / 9, b = e % 9;
+    double s = 0.0;
+    for (int h = 0; h < H; ++h)
+      for (int c = 0; c < nchunk; ++c) s += meas_part[(((int64_t)i * H + h) * nchunk + c) * 9 + b];
+    meas_lt[e] = s;
+  }
+}
+
+__global__ void k_meas_units(DualArgs a, const double* meas_lt) {
+  const int ncand = a.nbits * a.ngrid;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < a.G * 2 * a.nbits; e += gridDim.x * blockDim.x) {
+    const int u = e / a.nbits, bi = e % a.nbits;
+    const int g = u / 2, k = u % 2;
+    if (k == 1 && !a.has_v) continue;
+    const int l0 = (int)(((int64_t)g * a.L) / a.G), l1 = (int)(((int64_t)(g + 1) * a.L) / a.G);
+    double s = 0.0;
+    for (int l = l0; l < l1; ++l) s += meas_lt[(int64_t)(k * a.L + l) * 9 + a.bits[bi]];   // position of lt = 2 l + k
+    const int rt = a.meta->alloc[g][k][0], rd = a.meta->alloc[g][k][1];
+    for (int gi = 0; gi < a.ngrid; ++gi) {
+      int r1, r2;
+      grid_rank(gi, a.step, a.D, r1, r2);
+      a.unit_err[(int64_t)u * ncand + bi * a.ngrid + gi] = (r1 == rt && r2 == rd) ? s : __longlong_as_double(0x7ff0000000000000LL);
+    }
+  }
+}
+
 constexpr size_t kDualSmem = 160 * 1024;
 
 // One CTA per budget pool. The candidates come ranked by the tie-break key (bytes, b, r_t,
@@ -412,8 +445,10 @@ cudaError_t energy_table(const TableArgs& a, cudaStream_t s) {
 cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s) {
   if (a.G > kMaxGroups || a.L > kMaxL) return cudaErrorInvalidValue;
   const int units = a.G * 2 * a.ngrid;
-  k_unit_tables<<<(units + 255) / 256, 256, 0, s>>>(a);
-  note_launch();
+  if (!a.tables_ready) {
+    k_unit_tables<<<(units + 255) / 256, 256, 0, s>>>(a);
+    note_launch();
+  }
   cudaError_t e = cudaFuncSetAttribute(k_dual_pool, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
   if (e != cudaSuccess) return e;
   const int npools = (a.has_v && a.split) ? 2 : 1;
@@ -423,6 +458,16 @@ cudaError_t dual_allocate(const DualArgs& a, cudaStream_t s) {
   k_dual_pool<<<npools, threads, kDualSmem, s>>>(a);
   note_launch();
   k_layout<<<1, kMaxLT, 0, s>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t measured_tables(const DualArgs& a, const double* meas_part, int nchunk, double* meas_lt,
+                            cudaStream_t s) {
+  const int n_lt = a.L * (a.has_v ? 2 : 1);
+  k_meas_lt<<<(n_lt * 9 + 255) / 256, 256, 0, s>>>(n_lt, a.H, nchunk, meas_part, meas_lt);
+  note_launch();
+  k_meas_units<<<1, 256, 0, s>>>(a, meas_lt);
   note_launch();
   return cudaGetLastError();
 }

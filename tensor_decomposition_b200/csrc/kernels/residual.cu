@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf
   const int lt = a.lt_ids[i];
   const StreamMeta* m = a.meta;
   const int rt = m->lt_rank[lt][0], rd = m->lt_rank[lt][1], b = m->lt_rank[lt][2];
-  if (b == 0 || rt == 0) return;
+  if ((b == 0 && !a.measure) || rt == 0) return;
   constexpr int D = kD, Q = kD / 4;
   const __nv_bfloat16* G = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_G]) +
                            (int64_t)h * rt * rd;
@@ -96,13 +96,14 @@ constexpr int kRows = 16;          // rows per tile
 constexpr int kPS = 132;           // row stride (floats) of Pi^T: conflict-free fragment loads
 constexpr int kGroups = 2;
 
+template <bool kMeasure>
 __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const double* Nbuf, int R) {
   extern __shared__ __align__(16) unsigned char smraw[];
   const int chunk = blockIdx.x, h = blockIdx.y, i = blockIdx.z;
   const int lt = a.lt_ids[i];
   const StreamMeta* m = a.meta;
   const int rt = m->lt_rank[lt][0], b = m->lt_rank[lt][2];
-  if (b == 0) return;
+  if (!kMeasure && b == 0) return;
   const int D = a.D;                       // 128
   const int K = D + rt;                    // GEMM depth
   const int SN = rt + 4;                   // row stride (doubles) of N^T
@@ -126,8 +127,9 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
   __half* scales = reinterpret_cast<__half*>(a.body + m->off[lt][JOLT_PART_SCALES]);
   unsigned char* codes = a.body + m->off[lt][JOLT_PART_CODES];
   const int rowbytes = D * b / 8;
-  const double half = (double)(1 << (b - 1));
+  const double half = b > 0 ? (double)(1 << (b - 1)) : 0.0;
   const int cmax = (1 << b) - 1;
+  double errs[9] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};   // measure mode: sum of (y - y_hat_b)^2
   const int t_begin = chunk * kChunk, t_end = min(a.T, t_begin + kChunk);
   // group g takes the tiles t_begin + (2 k + g) kRows
   const int g = tid >> 8, gt = tid & 255, warp = gt >> 5, lane = tid & 31;
@@ -225,6 +227,36 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
     mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     if ((lane & 3) == 0) pm[ar * 4 + cg] = mx;
     group_sync(g);
+    if constexpr (kMeasure) {
+      // exact squared error of every allowed width at this row's fp16 scale s: b = 0 stores no
+      // residual (error y^2); otherwise c = clamp(floor(y 2^(b-1) / s + 2^(b-1))) and
+      // y_hat = (2 c + 1 - 2^b) (s / 2^b), both products exact in float64 (s = 0: every code 0)
+      const double sd = (double)__half2float(row_scale(ar));
+#pragma unroll
+      for (int bb = 0; bb <= 8; ++bb) {
+        if (!((a.bits_mask >> bb) & 1u)) continue;
+        double e = 0.0;
+        if (bb == 0) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) e = fma(acc[j][1], acc[j][1], fma(acc[j][0], acc[j][0], e));
+        } else {
+          const double hb = (double)(1 << (bb - 1)), inv = sd > 0.0 ? hb / sd : 0.0;
+          const double cell = sd * (1.0 / (double)(1 << bb));
+          const double top = (double)((1 << bb) - 1);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int ee = 0; ee < 2; ++ee) {
+              double c = 0.0;
+              if (sd > 0.0) c = fmin(fmax(floor(fma(acc[j][ee], inv, hb)), 0.0), top);
+              const double d = acc[j][ee] - (2.0 * c + 1.0 - 2.0 * hb) * cell;
+              e = fma(d, d, e);
+            }
+        }
+        errs[bb] += e;
+      }
+      continue;
+    }
     // codes: c = floor(y * (2^(b-1) / s) + 2^(b-1)), clamped, with one reciprocal per row
     // (it can differ from a divide-per-entry only for values within ~1e-16 s of a cell boundary)
     {
@@ -267,6 +299,25 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
       }
     }
   }
+  if constexpr (kMeasure) {
+    // fixed-order reduction of the 512 threads' sums: warp butterflies, then warps in order
+#pragma unroll
+    for (int bb = 0; bb <= 8; ++bb)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) errs[bb] += __shfl_xor_sync(0xffffffffu, errs[bb], o);
+    __syncthreads();                                   // every group is past its last tile
+    double* red = reinterpret_cast<double*>(AT);       // [16][9]
+    if (lane == 0)
+#pragma unroll
+      for (int bb = 0; bb <= 8; ++bb) red[(tid >> 5) * 9 + bb] = errs[bb];
+    __syncthreads();
+    if (tid < 9) {
+      double sum = 0.0;
+      for (int w = 0; w < 16; ++w) sum += red[w * 9 + tid];
+      const int nchunk = (a.T + kChunk - 1) / kChunk;
+      a.meas_part[(((int64_t)i * a.H + h) * nchunk + chunk) * 9 + tid] = sum;
+    }
+  }
 }
 
 }  // namespace
@@ -284,10 +335,17 @@ cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStre
   const size_t sm = (size_t)kD * kPS * sizeof(float) + (size_t)kD * (R + 4) * sizeof(double) +
                     (size_t)kGroups * kRows * 4 * sizeof(double) +
                     (size_t)kGroups * kRows * (kD + R + 4) * sizeof(float) + (size_t)kGroups * kRows * kD;
-  e = cudaFuncSetAttribute(k_residual, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  e = cudaFuncSetAttribute(k_residual<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const dim3 g((a.T + kChunk - 1) / kChunk, a.H, a.n_lt);
-  k_residual<<<g, 512, sm, s>>>(a, Nbuf, R);
+  if (a.measure) {
+    if (!a.meas_part) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(k_residual<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    k_residual<true><<<g, 512, sm, s>>>(a, Nbuf, R);
+  } else {
+    k_residual<false><<<g, 512, sm, s>>>(a, Nbuf, R);
+  }
   note_launch();
   return cudaGetLastError();
 }

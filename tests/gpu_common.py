@@ -162,12 +162,14 @@ def check_allocation(J, st, ost, op, cfg):
     return units
 
 
-def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits=None, factors=1):
+def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits=None, factors=1, measured_b=0):
     """Encode and decode a whole workload on the GPU in the launch configuration bench.py
     times and check it on sampled layer-tensors against the oracle: the allocation (whole
     cache), principal angles of the factors (when the plan has them), residual codes, the decode
     and the relative error at the GPU's allocation. `bits` restricts the residual widths and
-    `factors = 0` forces r_t = r_d = 0 (the in-codec baselines)."""
+    `factors = 0` forces r_t = r_d = 0 (the in-codec baselines). With `measured_b = 1` the GPU's
+    measured error of every allowed width is also compared, per sampled layer-tensor, with the
+    oracle's measurement from the GPU's stored factors (float64, relative 1e-9)."""
     import torch
     dev = torch.device("cuda", 0)
     K, V = synth.gen_cache_torch(cfg, dev, seq=seq)
@@ -180,6 +182,7 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
         mask |= 1 << b
     c.bits_mask = mask
     c.factors = factors
+    c.measured_b = measured_b
     plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, budget,
                        cfg.groups, c)
     st = J.jolt_encode(plan, K, V, seed)
@@ -188,7 +191,8 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
     J.jolt_decode(st, Ko, Vo)
     torch.cuda.synchronize()
     ost = ostream.parse(J.jolt_stream_to_host(st), lts=set(sample))
-    op = oracle_plan(cfg, budget, encoder, bits=bits, **({} if factors else {"rt_cap": 0}))
+    op = oracle_plan(cfg, budget, encoder, bits=bits, measured_b=bool(measured_b),
+                     **({} if factors else {"rt_cap": 0}))
     assert ost.rt_max == op.R()
     check_allocation(J, st, ost, op, cfg)
     Pi = J.jolt_export_debug(st, J.JOLT_DBG_PI).reshape(128, 128).astype(np.float64)
@@ -215,6 +219,17 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
                                          [float(np.arccos(np.clip(abs(UT[:, j] @ a["U_T_unrounded"][:, j]) /
                                                                   np.linalg.norm(UT[:, j]), 0, 1))) for j in range(kt)])
         assert worst < ANGLE_TOL, (lt, worst, where)
+        if measured_b:
+            c_lt = ost.lts[lt]
+            Y = oj.residual_rotated(X, c_lt.U_T, c_lt.G, c_lt.U_D, Pi)
+            got_m = J.jolt_export_debug(st, J.JOLT_DBG_MEAS, lt)
+            for bb in op.bits:
+                if bb == 0:
+                    ref_m = float(np.sum(Y * Y))
+                else:
+                    s_, q_, _ = oj.quantize_rows(Y, bb)
+                    ref_m = float(np.sum((Y - oj.dequantize_rows(s_, q_, bb)) ** 2))
+                assert abs(got_m[bb] - ref_m) <= 1e-9 * max(ref_m, 1e-300), (lt, bb, got_m[bb], ref_m)
         # codes of this layer-tensor
         out_band, in_band, scale_bad, total = codes_parity(only_lt(ost, lt), {lt: X}, Pi)
         assert scale_bad == 0 and out_band == 0, (lt, scale_bad, out_band, in_band, total)

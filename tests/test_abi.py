@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(jolt):
 def test_config_defaults(jolt):
     c = jolt.jolt_config_default()
     assert (c.encoder, c.oversample, c.power_iters, c.rank_step, c.rt_max, c.bits_mask,
-            c.split_kv_budget, c.max_jacobi_sweeps, c.factors) == (0, 16, 1, 16, 0, 0x1FF, 0, 30, 1)
+            c.split_kv_budget, c.max_jacobi_sweeps, c.factors, c.measured_b) == (0, 16, 1, 16, 0, 0x1FF, 0, 30, 1, 0)
 
 
 @pytest.mark.parametrize("args", [
