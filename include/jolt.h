@@ -90,6 +90,10 @@ typedef struct {
                                 residual coder measures the exact squared error of every allowed
                                 b at each unit's chosen ranks, and a second dual re-chooses b per
                                 unit with those errors (ranks unchanged). */
+  int32_t rotation;          /* 0 (default): Haar rotation Pi (Q factor of a Gaussian matrix);
+                                1: randomized Hadamard Pi = diag(s) H / sqrt(D), s random signs of
+                                the seed's rotation stream, H the Sylvester Hadamard matrix (D a
+                                power of two); recorded in the stream header */
 } jolt_config;
 
 typedef struct jolt_plan_s* jolt_plan_t;
@@ -197,8 +201,9 @@ JOLT_API jolt_status jolt_stream_info(jolt_stream_t stream, uint64_t* bytes_by_p
                                       int32_t* alloc, double* lambdas);
 
 /*
- * jolt_stream_to_host - serialize: header (magic "JOLT", version 1, shape, seed, allocation
- *   table), body (per layer-tensor lt = 2*layer + kind: U_T [T][r_t] bf16, U_D [D][r_d] bf16,
+ * jolt_stream_to_host - serialize: header (magic "JOLT", version 1, flags (bit 0 has V, bit 1
+ *   float32 output, bit 2 separate K/V budgets, bit 3 randomized Hadamard rotation, bits 8..15
+ *   encoder), shape, seed, allocation table), body (per layer-tensor lt = 2*layer + kind: U_T [T][r_t] bf16, U_D [D][r_d] bf16,
  *   G [H][r_t][r_d] bf16, scales [H][T] fp16, codes [H][T][D*b/8] bytes with code i at bits
  *   [i*b, i*b+b) LSB first; each part starts at a multiple of 256 bytes), then CRC-32.
  * buf: host buffer of *len bytes, or NULL to query the size into *len.
@@ -206,7 +211,7 @@ JOLT_API jolt_status jolt_stream_info(jolt_stream_t stream, uint64_t* bytes_by_p
 JOLT_API jolt_status jolt_stream_to_host(jolt_stream_t stream, void* buf, uint64_t* len);
 
 /* jolt_stream_from_host - parse a serialized stream (checks magic, version, sizes, CRC)
- * into a new device stream; Pi is rebuilt from the stored seed on `cuda_stream`. */
+ * into a new device stream; Pi is rebuilt from the stored seed (and rotation kind) on `cuda_stream`. */
 JOLT_API jolt_status jolt_stream_from_host(const void* buf, uint64_t len, void* cuda_stream,
                                            jolt_stream_t* out);
 

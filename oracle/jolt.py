@@ -34,7 +34,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-from .numerics import (round_bf16, round_fp16_sat, round_f32, haar_rotation,
+from .numerics import (round_bf16, round_fp16_sat, round_f32, haar_rotation, rotation_matrix,
                        sketch_matrix)
 
 RANK_STEP = 16
@@ -328,6 +328,7 @@ class OracleStream:
     out_f32: bool
     alloc: np.ndarray                  # [G][2][3] (r_t, r_d, b)
     lts: dict = field(default_factory=dict)
+    rotation: str = "haar"             # "haar" or "hadamard"
 
     def kinds(self):
         return (0, 1) if self.has_v else (0,)
@@ -351,6 +352,7 @@ class Plan:
     split_kv: bool = False
     out_f32: bool = False
     measured_b: bool = False   # re-choose b per unit with measured quantisation errors
+    rotation: str = "haar"     # "haar" or "hadamard" (randomized Hadamard, §8f-3 of the reading)
 
     def kinds(self):
         return (0, 1) if self.has_v else (0,)
@@ -515,7 +517,7 @@ def encode(plan: Plan, K, V, seed: int, spec: bool = True, alloc=None, factors=N
         tens[1] = np.asarray(V, dtype=np.float64)
     kap = kappa(plan.D)
     if Pi is None:
-        Pi = haar_rotation(seed, plan.D)
+        Pi = rotation_matrix(seed, plan.D, plan.rotation)
     A = {}
     for l in range(plan.L):
         for k in plan.kinds():
@@ -532,7 +534,7 @@ def encode(plan: Plan, K, V, seed: int, spec: bool = True, alloc=None, factors=N
             alloc, lams = refine_b(plan, units, alloc, meas)
     st = OracleStream(plan.L, plan.H, plan.T, plan.D, plan.has_v, plan.num_groups, seed,
                       plan.encoder, plan.rank_step, plan.R(), plan.split_kv, plan.out_f32,
-                      np.asarray(alloc, dtype=np.int64))
+                      np.asarray(alloc, dtype=np.int64), rotation=plan.rotation)
     for g, lay in enumerate(group_ranges(plan.L, plan.num_groups)):
         for l in lay:
             for k in plan.kinds():
@@ -560,7 +562,7 @@ def decode_lt(st: OracleStream, lt: int, Pi=None):
     """float64 reconstruction of one layer-tensor: G x2 U_T x3 U_D + dequant(codes) Pi^T."""
     c = st.lts[lt]
     if Pi is None:
-        Pi = haar_rotation(st.seed, st.D)
+        Pi = rotation_matrix(st.seed, st.D, st.rotation)
     Xh = tucker_part(c.U_T, c.G, c.U_D, st.H, st.T, st.D)
     if c.b > 0:
         Yh = dequantize_rows(c.scales, c.codes, c.b)
@@ -575,7 +577,7 @@ def round_output(Xh, out_f32: bool):
 def decode(st: OracleStream, Pi=None, rounded=True):
     """Whole cache: returns (K_hat, V_hat) as float64 [L][H][T][D] on the output grid."""
     if Pi is None:
-        Pi = haar_rotation(st.seed, st.D)
+        Pi = rotation_matrix(st.seed, st.D, st.rotation)
     outs = []
     for k in st.kinds():
         arr = np.stack([decode_lt(st, l * KINDS + k, Pi) for l in range(st.L)])

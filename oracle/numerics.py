@@ -140,6 +140,35 @@ def haar_rotation(seed: int, D: int) -> np.ndarray:
     return Q * sgn[None, :]
 
 
+def hadamard_matrix(D: int) -> np.ndarray:
+    """Sylvester Hadamard matrix (D a power of two): H[i, j] = (-1)^popcount(i & j)."""
+    assert D > 0 and D & (D - 1) == 0
+    i = np.arange(D)
+    par = np.zeros((D, D), dtype=np.int64)
+    a = i[:, None] & i[None, :]
+    while a.any():
+        par ^= a & 1
+        a = a >> 1
+    return np.where(par == 1, -1.0, 1.0)
+
+
+def hadamard_signs(seed: int, D: int) -> np.ndarray:
+    """Random signs of the randomized Hadamard rotation: s_i = -1 when the top bit of word i of
+    the rotation stream is set, +1 otherwise."""
+    w = stream_words(seed, STREAM_ROTATION, 0, D)
+    return np.where((w >> np.uint64(63)) == 1, -1.0, 1.0)
+
+
+def hadamard_rotation(seed: int, D: int) -> np.ndarray:
+    """Randomized Hadamard rotation Pi = diag(s) H / sqrt(D) (float64)."""
+    return hadamard_signs(seed, D)[:, None] * hadamard_matrix(D) / np.sqrt(D)
+
+
+def rotation_matrix(seed: int, D: int, kind: str = "haar") -> np.ndarray:
+    """The codec's rotation: Haar (default) or randomized Hadamard."""
+    return hadamard_rotation(seed, D) if kind == "hadamard" else haar_rotation(seed, D)
+
+
 def sketch_matrix(seed: int, lt: int, HD: int, l: int) -> np.ndarray:
     """Gaussian sketch Omega (HD x l) of layer-tensor lt, entries rounded to bf16."""
     z = gaussians(seed, STREAM_SKETCH0 + lt, HD * l).reshape(HD, l)

@@ -9,7 +9,8 @@ Layout, all little-endian:
     4   4  u32 version (1)
     8   4  u32 header_bytes = 64 + 24 * num_groups rounded up to a multiple of 16
     12  4  u32 flags: bit0 has V, bit1 float32 output, bit2 separate K/V budgets,
-                      bits 8..15 encoder (1 exact, 2 sketch)
+                      bit3 randomized Hadamard rotation (else Haar), bits 8..15 encoder
+                      (1 exact, 2 sketch)
     16  4  i32 layers        20  4  i32 heads      24  4  i32 tokens
     28  4  i32 head_dim      32  4  i32 num_groups 36  4  i32 rank_step
     40  4  i32 rt_max        44  4  i32 reserved (0)
@@ -74,7 +75,8 @@ def body_layout(L, H, T, D, has_v, num_groups, alloc):
 
 def _flags(st: OracleStream) -> int:
     enc = 1 if st.encoder == "exact" else 2
-    return (int(st.has_v) | (int(st.out_f32) << 1) | (int(st.split_kv) << 2) | (enc << 8))
+    return (int(st.has_v) | (int(st.out_f32) << 1) | (int(st.split_kv) << 2) |
+            (int(st.rotation == "hadamard") << 3) | (enc << 8))
 
 
 def serialize(st: OracleStream) -> bytes:
@@ -125,7 +127,7 @@ def parse(buf: bytes, lts=None) -> OracleStream:
             alloc[g, k] = struct.unpack_from("<3i", buf, 64 + 24 * g + 12 * k)
     enc = "exact" if ((flags >> 8) & 0xFF) == 1 else "sketch"
     st = OracleStream(L, H, T, D, has_v, G, seed, enc, step, rtm, bool(flags & 4),
-                      bool(flags & 2), alloc)
+                      bool(flags & 2), alloc, rotation="hadamard" if flags & 8 else "haar")
     layout, n = body_layout(L, H, T, D, has_v, G, alloc)
     if n != body_n:
         raise CorruptStream("body size does not match the allocation table")

@@ -264,6 +264,7 @@ struct jolt_plan_s {
 
 struct jolt_stream_s {
   int L = 0, H = 0, T = 0, D = 0, has_v = 0, G = 1, encoder = 0, step = 16, R = 0, split = 0;
+  int rotation = 0;   // 0 Haar, 1 randomized Hadamard
   jolt_dtype dtype = JOLT_BF16;
   uint64_t seed = 0;
   StreamMeta* d_meta = nullptr;
@@ -509,6 +510,7 @@ JOLT_API void jolt_config_default(jolt_config* c) {
   c->bits_mask = 0x1FFu;
   c->factors = 1;
   c->measured_b = 0;
+  c->rotation = 0;
   c->split_kv_budget = 0;
   c->max_jacobi_sweeps = 30;
 }
@@ -542,6 +544,8 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   if (cfg.factors != 0 && cfg.factors != 1) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: factors must be 0 or 1");
   if (cfg.measured_b != 0 && cfg.measured_b != 1)
     return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: measured_b must be 0 or 1");
+  if (cfg.rotation != 0 && cfg.rotation != 1)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: rotation must be 0 (Haar) or 1 (randomized Hadamard)");
   if (byte_budget == 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: zero byte budget");
 
   jolt_plan_s* p = new (std::nothrow) jolt_plan_s();
@@ -737,6 +741,7 @@ static jolt_status make_stream(jolt_plan_s* p, uint64_t seed, cudaStream_t cs, j
   const jolt_shape& sh = p->shape;
   st->L = sh.layers; st->H = sh.heads; st->T = sh.tokens; st->D = sh.head_dim;
   st->has_v = sh.has_v ? 1 : 0; st->G = p->G; st->encoder = p->exact_by_iteration ? JOLT_ENC_EXACT : p->encoder; st->step = p->step;
+  st->rotation = p->cfg.rotation;
   st->R = p->R; st->split = (sh.has_v && p->cfg.split_kv_budget) ? 1 : 0; st->dtype = sh.dtype;
   st->seed = seed; st->cs = cs; st->plan = p; st->n_lt = p->n_lt;
   st->body_cap = align_up((size_t)p->budget + (size_t)JOLT_NUM_PARTS * kAlign * p->n_lt + kAlign, kAlign);
@@ -1240,8 +1245,13 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, ui
   // rotation Pi for this seed (cached in the plan), copied into the stream for decode
   if (!(p->pi_valid && p->pi_seed == seed)) {
     PROF("rotation", s);
-    cudaError_t e = gauss_f64(seed, 1, (int64_t)D * D, p->Gpi, s);
-    if (e == cudaSuccess) e = haar_from_gauss(p->Gpi, D, p->Pi32, p->Pib, s);
+    cudaError_t e;
+    if (p->cfg.rotation == 1) {
+      e = hadamard_pi(seed, D, p->Pi32, p->Pib, s);
+    } else {
+      e = gauss_f64(seed, 1, (int64_t)D * D, p->Gpi, s);
+      if (e == cudaSuccess) e = haar_from_gauss(p->Gpi, D, p->Pi32, p->Pib, s);
+    }
     if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "rotation: %s", cudaGetErrorString(e)));
     p->pi_valid = true;
     p->pi_seed = seed;
@@ -1461,7 +1471,8 @@ JOLT_API jolt_status jolt_stream_to_host(jolt_stream_t st, void* buf, uint64_t* 
   put32(head, 4, 1);
   put32(head, 8, (uint32_t)hb);
   const uint32_t flags = (uint32_t)st->has_v | ((st->dtype == JOLT_F32 ? 1u : 0u) << 1) |
-                         ((uint32_t)st->split << 2) | ((uint32_t)st->encoder << 8);
+                         ((uint32_t)st->split << 2) | ((uint32_t)(st->rotation & 1) << 3) |
+                         ((uint32_t)st->encoder << 8);
   put32(head, 12, flags);
   const int32_t ints[8] = {st->L, st->H, st->T, st->D, st->G, st->step, st->R, 0};
   memcpy(&head[16], ints, sizeof(ints));
@@ -1569,8 +1580,13 @@ JOLT_API jolt_status jolt_stream_from_host(const void* buf, uint64_t len, void* 
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->d_meta, &m, sizeof(m), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(st->d_lt_ids, ids.data(), sizeof(int32_t) * ids.size(), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = gauss_f64(seed, 1, (int64_t)D * D, st->d_Gpi, s);
-  if (e == cudaSuccess) e = haar_from_gauss(st->d_Gpi, D, st->d_Pi, nullptr, s);
+  st->rotation = (int)((flags >> 3) & 1u);
+  if (st->rotation == 1) {
+    if (e == cudaSuccess) e = hadamard_pi(seed, D, st->d_Pi, nullptr, s);
+  } else {
+    if (e == cudaSuccess) e = gauss_f64(seed, 1, (int64_t)D * D, st->d_Gpi, s);
+    if (e == cudaSuccess) e = haar_from_gauss(st->d_Gpi, D, st->d_Pi, nullptr, s);
+  }
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);   // host buffers above are stack / vector
   if (e != cudaSuccess) {
     jolt_stream_destroy(st);

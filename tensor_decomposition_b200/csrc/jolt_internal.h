@@ -68,6 +68,8 @@ cudaError_t gauss_f64(uint64_t seed, uint64_t stream_id, int64_t n, double* out,
 cudaError_t sketch_omega(uint64_t seed, const int32_t* lt_ids_host, int n_lt, int64_t HD, int l,
                          __nv_bfloat16* out, bool transposed, cudaStream_t s);
 // Haar rotation from a D x D float64 Gaussian (Householder QR, signs of diag(R) moved into Q).
+// Randomized Hadamard rotation diag(s) H / sqrt(D) of the seed's rotation stream (D a power of 2).
+cudaError_t hadamard_pi(uint64_t seed, int D, float* Pi_f32, __nv_bfloat16* Pi_bf16, cudaStream_t s);
 cudaError_t haar_from_gauss(const double* G, int D, float* Pi_f32, __nv_bfloat16* Pi_bf16,
                             cudaStream_t s);
 // Batched two-sided cyclic Jacobi, n even, n <= 128; V columns = eigenvectors, eigenvalues

@@ -1,5 +1,5 @@
 // Seeded randomness of the codec: the counter-based normal generator, the Gaussian sketch
-// matrices of the FlashJoLT token factor, and the Haar rotation Pi.
+// matrices of the FlashJoLT token factor, and the rotation Pi (Haar, or randomized Hadamard).
 //
 // "A JoLT for the KV Cache" (arXiv 2607.12550v2, Abstract) rotates the truncation residual
 // by "a random orthogonal rotation" before low-bit quantisation; the news summary of the
@@ -153,6 +153,22 @@ __global__ void k_haar_qr(const double* G, int n, float* Pi32, __nv_bfloat16* Pi
   }
 }
 
+// Randomized Hadamard rotation Pi = diag(s) H / sqrt(D) (the structured Johnson-Lindenstrauss
+// transform of Ailon & Chazelle 2006), D a power of two: H is the Sylvester Hadamard matrix,
+// H[i][j] = (-1)^popcount(i & j), and s_i = -1 when the top bit of word i of the rotation stream
+// is set, +1 otherwise. Entry (i, j) is formed in float64 and rounded like the Haar matrix.
+__global__ void k_hadamard_pi(uint64_t key, int D, float* Pi32, __nv_bfloat16* Pib) {
+  const double inv = 1.0 / sqrt((double)D);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < D * D; e += gridDim.x * blockDim.x) {
+    const int i = e / D, j = e - i * D;
+    const bool neg_s = (mix64(key + ((uint64_t)i + 1ull) * kGamma) >> 63) != 0;
+    const bool neg_h = (__popc(i & j) & 1) != 0;
+    const double v = (neg_s != neg_h) ? -inv : inv;
+    Pi32[e] = (float)v;
+    if (Pib) Pib[e] = __float2bfloat16_rn((float)v);
+  }
+}
+
 }  // namespace
 
 static uint64_t host_mix64(uint64_t z) {
@@ -179,6 +195,14 @@ cudaError_t sketch_omega(uint64_t seed, const int32_t* lt_ids, int n_lt, int64_t
   int bx = (int)((per + 255) / 256);
   if (bx > 64) bx = 64;
   k_sketch_omega<<<dim3(bx, n_lt), 256, 0, s>>>(keys, HD, l, transposed ? 1 : 0, out);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t hadamard_pi(uint64_t seed, int D, float* Pi_f32, __nv_bfloat16* Pi_bf16, cudaStream_t s) {
+  if (D <= 0 || (D & (D - 1))) return cudaErrorInvalidValue;
+  const uint64_t key = host_mix64(seed + host_mix64(1ull + 1ull));   // the rotation stream (1)
+  k_hadamard_pi<<<(D * D + 255) / 256, 256, 0, s>>>(key, D, Pi_f32, Pi_bf16);
   note_launch();
   return cudaGetLastError();
 }

@@ -21,6 +21,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "BUDGET_INFEASIBLE", 3: "OOM", 4: 
                 9: "UNSUPPORTED"}
 JOLT_BF16, JOLT_F32 = 0, 1
 JOLT_ENC_AUTO, JOLT_ENC_EXACT, JOLT_ENC_SKETCH = 0, 1, 2
+JOLT_ROT_HAAR, JOLT_ROT_HADAMARD = 0, 1
 JOLT_DBG_PI, JOLT_DBG_UT_F32, JOLT_DBG_UD_F32, JOLT_DBG_TABLE, JOLT_DBG_XX, JOLT_DBG_LAMBDA, \
     JOLT_DBG_OMEGA, JOLT_DBG_MEAS = range(8)
 PART_NAMES = ("U_T", "U_D", "G", "scales", "codes")
@@ -48,7 +49,7 @@ class Config(ctypes.Structure):
                 ("power_iters", ctypes.c_int32), ("rank_step", ctypes.c_int32),
                 ("rt_max", ctypes.c_int32), ("bits_mask", ctypes.c_uint32),
                 ("split_kv_budget", ctypes.c_int32), ("max_jacobi_sweeps", ctypes.c_int32),
-                ("factors", ctypes.c_int32), ("measured_b", ctypes.c_int32)]
+                ("factors", ctypes.c_int32), ("measured_b", ctypes.c_int32), ("rotation", ctypes.c_int32)]
 
 
 def _load():

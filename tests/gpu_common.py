@@ -110,7 +110,7 @@ def oracle_lt_reconstruction(plan, X, seed, lt, rt, rd, b, Pi=None):
     oracle's own factors (spec mode) and the same sketch stream as layer-tensor `lt`."""
     a = oj.analyse_layer_tensor(plan, X, seed, lt, spec=True)
     if Pi is None:
-        Pi = onum.haar_rotation(seed, plan.D)
+        Pi = onum.rotation_matrix(seed, plan.D, plan.rotation)
     U_T, U_D = a["U_T"][:, :rt], a["U_D"][:, :rd]
     G = onum.round_bf16(a["Gmax"][:, :rt, :rd])
     rec = oj.tucker_part(U_T, G, U_D, plan.H, plan.T, plan.D)
@@ -162,7 +162,8 @@ def check_allocation(J, st, ost, op, cfg):
     return units
 
 
-def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits=None, factors=1, measured_b=0):
+def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits=None, factors=1, measured_b=0,
+                   rotation=0, keep=False):
     """Encode and decode a whole workload on the GPU in the launch configuration bench.py
     times and check it on sampled layer-tensors against the oracle: the allocation (whole
     cache), principal angles of the factors (when the plan has them), residual codes, the decode
@@ -183,6 +184,7 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
     c.bits_mask = mask
     c.factors = factors
     c.measured_b = measured_b
+    c.rotation = rotation
     plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, budget,
                        cfg.groups, c)
     st = J.jolt_encode(plan, K, V, seed)
@@ -192,11 +194,14 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
     torch.cuda.synchronize()
     ost = ostream.parse(J.jolt_stream_to_host(st), lts=set(sample))
     op = oracle_plan(cfg, budget, encoder, bits=bits, measured_b=bool(measured_b),
-                     **({} if factors else {"rt_cap": 0}))
+                     rotation="hadamard" if rotation else "haar", **({} if factors else {"rt_cap": 0}))
     assert ost.rt_max == op.R()
     check_allocation(J, st, ost, op, cfg)
     Pi = J.jolt_export_debug(st, J.JOLT_DBG_PI).reshape(128, 128).astype(np.float64)
+    assert ost.rotation == ("hadamard" if rotation else "haar")
     report = {"alloc": ost.alloc.tolist()}
+    if keep:
+        report["_keep"] = (Ko, Vo, st)
     for lt in sample:
         l, k = lt // 2, lt % 2
         X = host((K if k == 0 else V)[l])
