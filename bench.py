@@ -224,20 +224,22 @@ def in_codec_baselines(J, cfg, K, V, budget, encoder, steps=5, warmup=2):
     """The codec restricted to its baselines on the same cache and budget: residual only
     (factors = 0, b = 4: per-row 4-bit quantisation of the rotated rows) and Tucker only
     (b = 0), plus JoLT itself at the 4-bit baseline's byte count, so that the errors compare at
-    equal bytes, and JoLT with the measured-b refinement at the metric's budget. Each is timed over `steps` device-timed steps (encode + decode + the two
+    equal bytes, and JoLT with the measured-b refinement and with the randomized Hadamard
+    rotation at the metric's budget. Each is timed over `steps` device-timed steps (encode + decode + the two
     errors, as the main step) after `warmup`; none of this is inside the main timed region."""
     import torch
     bf16_bytes = (K.numel() + V.numel()) * 2
     Ko, Vo = torch.empty_like(K), torch.empty_like(V)
     res = {}
 
-    def run(name, bits, factors, bud, measured_b=0):
+    def run(name, bits, factors, bud, measured_b=0, rotation=0):
         c = J.jolt_config_default()
         c.encoder = encoder
         c.split_kv_budget = int(cfg.split_kv)
         c.bits_mask = sum(1 << b for b in bits)
         c.factors = factors
         c.measured_b = measured_b
+        c.rotation = rotation
         plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, bud,
                            cfg.groups, c)
         errs = [None, None]
@@ -273,6 +275,8 @@ def in_codec_baselines(J, cfg, K, V, budget, encoder, steps=5, warmup=2):
     # the measured-b refinement of the JoLT allocation at the metric's budget (reported beside
     # the baselines; the metric itself uses the phi(b) model)
     run("jolt_measured_b", cfg.bits, 1, budget, measured_b=1)
+    # the randomized Hadamard rotation (fast Walsh-Hadamard transform in the residual coder)
+    run("jolt_hadamard", cfg.bits, 1, budget, rotation=1)
     return res
 
 

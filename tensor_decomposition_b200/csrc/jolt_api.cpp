@@ -1286,6 +1286,7 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, ui
   ra.n_lt = p->n_lt; ra.H = sh.heads; ra.T = sh.tokens; ra.D = D; ra.lt_ids = p->d_lt_ids;
   ra.X[0] = K; ra.X[1] = V; ra.xt = sh.dtype == JOLT_BF16 ? EL_BF16 : EL_F32; ra.Pi = st->d_Pi;
   ra.meta = st->d_meta; ra.body = st->d_body;
+  ra.hadamard = p->cfg.rotation == 1 ? 1 : 0;
   if (p->cfg.measured_b) {
     // measured-b refinement: exact errors of every allowed width at the chosen ranks (one pass of
     // the residual coder that writes no codes), then a second dual over b with those errors; the

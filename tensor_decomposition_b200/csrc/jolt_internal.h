@@ -167,6 +167,10 @@ struct ResidualArgs {
   int measure = 0;
   uint32_t bits_mask = 0;
   double* meas_part = nullptr;
+  // randomized Hadamard rotation (Pi = diag(s) H / sqrt(D), s = sign of Pi's first column):
+  // y = FWHT((x - u M_h) * s) / sqrt(D) with M_h = G_h U_D^T, the rotation as log2(D) butterfly
+  // stages instead of a D x D product
+  int hadamard = 0;
 };
 // Nbuf: float64 scratch [n_lt][H][R][D] for N_h = (G_h U_D^T) Pi.
 cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStream_t s);

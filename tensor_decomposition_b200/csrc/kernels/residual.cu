@@ -48,7 +48,12 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf
   for (int task = threadIdx.x; task < rd * Q; task += blockDim.x) {
     const int j = task / Q, e0 = 4 * (task - j * Q);
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int d = 0; d < D; ++d) {
+    if (a.hadamard) {
+      // M_h = G_h U_D^T: P = U_D^T (the rotation is applied by the residual coder)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = (double)__bfloat162float(UD[(e0 + q) * rd + j]);
+    }
+    for (int d = 0; d < (a.hadamard ? 0 : D); ++d) {
       const double u = (double)__bfloat162float(UD[d * rd + j]);
       const float4 pv = *reinterpret_cast<const float4*>(a.Pi + d * D + e0);
       acc[0] = fma(u, (double)pv.x, acc[0]);
@@ -96,7 +101,7 @@ constexpr int kRows = 16;          // rows per tile
 constexpr int kPS = 132;           // row stride (floats) of Pi^T: conflict-free fragment loads
 constexpr int kGroups = 2;
 
-template <bool kMeasure>
+template <bool kMeasure, bool kHad>
 __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const double* Nbuf, int R) {
   extern __shared__ __align__(16) unsigned char smraw[];
   const int chunk = blockIdx.x, h = blockIdx.y, i = blockIdx.z;
@@ -114,9 +119,11 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
   float* AT = reinterpret_cast<float*>(PM + kGroups * kRows * 4);                 // [2][kRows][SA]
   unsigned char* CS = reinterpret_cast<unsigned char*>(AT + (size_t)kGroups * kRows * SA);   // [2][kRows][D]
   const int tid = threadIdx.x;
-  for (int e = tid; e < D * D; e += 512) {
-    const int k = e / D, n = e % D;
-    PT[n * kPS + k] = a.Pi[e];
+  if (!kHad) {
+    for (int e = tid; e < D * D; e += 512) {
+      const int k = e / D, n = e % D;
+      PT[n * kPS + k] = a.Pi[e];
+    }
   }
   const double* Ng = Nbuf + (((int64_t)i * a.H + h) * R) * D;
   for (int e = tid; e < rt * D; e += 512) {
@@ -138,6 +145,17 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
   unsigned char* cs = CS + g * kRows * D;
   const int rg = warp >> 2, cg = warp & 3;
   const int ar = 8 * rg + (lane >> 2), ak = lane & 3;
+  // Hadamard mode: signs s_c of this thread's eight columns c = 32 cg + 8 j + 2 ak + e (bit
+  // 2 j + e set: negative; Pi[c][0] = s_c / sqrt(D)) and the group's exchange rows (padded)
+  constexpr int kXS = 132;
+  double* xg = reinterpret_cast<double*>(smraw) + (size_t)g * kRows * kXS;
+  uint32_t sneg = 0;
+  if (kHad)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (a.Pi[(32 * cg + 8 * j + 2 * ak + e) * D] < 0.0f) sneg |= 1u << (2 * j + e);
   const int wpr = rowbytes / 4;                         // 32-bit words per packed row (4 b)
   const int c_first = (32 * lane) / b;                  // codes overlapping word `lane`
   const int c_last = min(D - 1, (32 * lane + 31) / b);
@@ -197,17 +215,25 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
     group_sync(g);
     if (t0 + kGroups * kRows < t_end) fetch(t0 + kGroups * kRows);
     double acc[4][2];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = 0.0;
     const float* arow = At + ar * SA + ak;
-    const float* pb = PT + (32 * cg + (lane >> 2)) * kPS + ak;    // fragment j at + 8 j kPS
     const double* qb = NT + (32 * cg + (lane >> 2)) * SN + ak;
-    // K = D part (x Pi), fully unrolled so the fragment loads of later steps can be issued early
+    if constexpr (kHad) {
+      // accumulators start at x (this thread's entries of row ar); only -u M_h is multiplied
 #pragma unroll
-    for (int k0 = 0; k0 < kD; k0 += 4) {
-      const double av = (double)arow[k0];
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[j][0], acc[j][1], av, (double)pb[8 * j * kPS + k0]);
+        for (int e = 0; e < 2; ++e) acc[j][e] = (double)At[ar * SA + 32 * cg + 8 * j + 2 * ak + e];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = 0.0;
+      const float* pb = PT + (32 * cg + (lane >> 2)) * kPS + ak;    // fragment j at + 8 j kPS
+      // K = D part (x Pi), fully unrolled so the fragment loads of later steps can be issued early
+#pragma unroll
+      for (int k0 = 0; k0 < kD; k0 += 4) {
+        const double av = (double)arow[k0];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[j][0], acc[j][1], av, (double)pb[8 * j * kPS + k0]);
+      }
     }
     // K = r_t part (-u N), four steps per unrolled block (r_t is a multiple of 16)
     for (int k0 = 0; k0 < rt; k0 += 16) {
@@ -217,6 +243,60 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
 #pragma unroll
         for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[j][0], acc[j][1], av, qb[8 * j * SN + k0 + kk]);
       }
+    }
+    if constexpr (kHad) {
+      // y = FWHT(r * s) / sqrt(D) over the 128 columns of row ar: column bit 0 (e) and bits 3-4
+      // (j) inside the thread, bits 1-2 (ak) across lanes, bits 5-6 (cg) across the row's four
+      // warps through shared memory (a 4-point transform per entry)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if ((sneg >> (2 * j + e)) & 1u) acc[j][e] = -acc[j][e];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const double a0 = acc[j][0], a1 = acc[j][1];
+        acc[j][0] = a0 + a1;
+        acc[j][1] = a0 - a1;
+      }
+#pragma unroll
+      for (int jb = 1; jb <= 2; jb <<= 1)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (!(j & jb))
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const double lo = acc[j][e], hi = acc[j | jb][e];
+              acc[j][e] = lo + hi;
+              acc[j | jb][e] = lo - hi;
+            }
+#pragma unroll
+      for (int m = 1; m <= 2; m <<= 1)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const double p = __shfl_xor_sync(0xffffffffu, acc[j][e], m);
+            acc[j][e] = (ak & m) ? p - acc[j][e] : acc[j][e] + p;
+          }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) xg[ar * kXS + 32 * cg + 8 * j + 2 * ak + e] = acc[j][e];
+      group_sync(g);
+      const double inv = 1.0 / sqrt((double)kD);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          double o = 0.0;
+#pragma unroll
+          for (int c2 = 0; c2 < 4; ++c2) {
+            const double v = xg[ar * kXS + 32 * c2 + 8 * j + 2 * ak + e];
+            o = (__popc(cg & c2) & 1) ? o - v : o + v;
+          }
+          acc[j][e] = o * inv;
+        }
     }
     // row absmax: this thread's 8 entries of row ar, the 4 lanes of the row, then the 4 warps
     // of the row (columns 32 cg .. +31) through the table
@@ -335,17 +415,17 @@ cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStre
   const size_t sm = (size_t)kD * kPS * sizeof(float) + (size_t)kD * (R + 4) * sizeof(double) +
                     (size_t)kGroups * kRows * 4 * sizeof(double) +
                     (size_t)kGroups * kRows * (kD + R + 4) * sizeof(float) + (size_t)kGroups * kRows * kD;
-  e = cudaFuncSetAttribute(k_residual<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
   const dim3 g((a.T + kChunk - 1) / kChunk, a.H, a.n_lt);
-  if (a.measure) {
-    if (!a.meas_part) return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(k_residual<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    k_residual<true><<<g, 512, sm, s>>>(a, Nbuf, R);
-  } else {
-    k_residual<false><<<g, 512, sm, s>>>(a, Nbuf, R);
-  }
+  if (a.measure && !a.meas_part) return cudaErrorInvalidValue;
+  auto launch = [&](auto kern) {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e2 != cudaSuccess) return e2;
+    kern<<<g, 512, sm, s>>>(a, Nbuf, R);
+    return cudaSuccess;
+  };
+  if (a.measure) e = a.hadamard ? launch(k_residual<true, true>) : launch(k_residual<true, false>);
+  else e = a.hadamard ? launch(k_residual<false, true>) : launch(k_residual<false, false>);
+  if (e != cudaSuccess) return e;
   note_launch();
   return cudaGetLastError();
 }

@@ -198,6 +198,8 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
     assert ost.rt_max == op.R()
     check_allocation(J, st, ost, op, cfg)
     Pi = J.jolt_export_debug(st, J.JOLT_DBG_PI).reshape(128, 128).astype(np.float64)
+    if rotation:
+        Pi = onum.hadamard_rotation(seed, 128)   # the residual coder applies it exactly (float64 FWHT)
     assert ost.rotation == ("hadamard" if rotation else "haar")
     report = {"alloc": ost.alloc.tolist()}
     if keep:
