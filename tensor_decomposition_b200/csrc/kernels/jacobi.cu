@@ -167,9 +167,9 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
 // CUDA's float64 reciprocal square root) and inverts it; the panel below is L21 = A21 L11^{-T}
 // (1 x 4 strips per thread); the trailing lower triangle takes the rank-16 update in 4 x 4
 // register tiles. A pivot not above floor_v is raised to it and sets *floored (pivots of
-// the n x n problem only). Called by all 512 threads of the block.
+// the n x n problem only). Called by all NT threads of the block.
 constexpr int kCholLD = kMaxN + 1;
-template <bool kKeepL>
+template <bool kKeepL, int NT = 512>
 __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, double* Ls, double* Is, int n,
                                             double floor_v, int* floored) {
   constexpr int NP = kMaxN, LD = kCholLD, BS = 16, NBLK = NP / BS;
@@ -239,7 +239,7 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
     // panel L21 = A21 L11^{-T} into Pt only; thread = (group g of 4 columns, row), consecutive
     // lanes on consecutive rows. L11^{-1} is stored with zeros above its diagonal, so every
     // output is a full 16-term sum. A keeps A21 until the trailing phase copies L21 back.
-    for (int u = tid; u < 4 * rows; u += 512) {
+    for (int u = tid; u < 4 * rows; u += NT) {
       const int g = u / rows, i = k0 + BS + (u - g * rows);
       double v[BS];
 #pragma unroll
@@ -255,14 +255,14 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
     }
     __syncthreads();
     // L21 back into A (the trailing tiles below read Pt and write only columns >= k0 + BS)
-    for (int u = tid; u < BS * rows; u += 512) {
+    for (int u = tid; u < BS * rows; u += NT) {
       const int j = u / rows, i = k0 + BS + (u - j * rows);
       A[i * LD + k0 + j] = Pt[j * NP + i];
     }
     // trailing update of the lower triangle, 4 x 4 tiles (ti >= tj)
     const int t4 = rows / 4;
     const int cnt = t4 * (t4 + 1) / 2;
-    for (int p = tid; p < cnt; p += 512) {
+    for (int p = tid; p < cnt; p += NT) {
       int ti = (int)((sqrtf(8.0f * (float)p + 1.0f) - 1.0f) * 0.5f);
       while ((ti + 1) * (ti + 2) / 2 <= p) ++ti;
       while (ti * (ti + 1) / 2 > p) --ti;
@@ -321,9 +321,23 @@ struct EigBatch {
   int n, count;
 };
 
-// Two independent batches share one launch (blocks [0, b0.count) take the first).
-__global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int max_sweeps, int32_t* status) {
-  constexpr int NP = kMaxN;
+// f(integral_constant<int, K>) for K = K0 .. N - 1, unrolled at compile time
+constexpr int kEigWarps = 16;  // warps per eigenproblem (4 slots, 8 columns each; 8 warps of 8 slots ran 1.5x slower)
+
+template <int K0, int N, class F>
+__device__ __forceinline__ void unroll_phases(F& f) {
+  if constexpr (K0 < N) {
+    f(std::integral_constant<int, K0>{});
+    unroll_phases<K0 + 1, N>(f);
+  }
+}
+
+// Two independent batches share one launch (blocks [0, b0.count) take the first). W warps of
+// S = 64 / W tournament slots each (W = 8: 16 columns of 4 rows per lane in registers).
+template <int W>
+__global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, int max_sweeps, int32_t* status) {
+  constexpr int NP = kMaxN, NT = 32 * W, S = 64 / W, GL = 32 / S;   // GL lanes per slot group
+  static_assert(W * S == 64 && (S & (S - 1)) == 0 && S >= 2, "slots per warp");
   const bool first = (int)blockIdx.x < b0.count;
   const EigBatch& eb = first ? b0 : b1;
   const int bi = first ? (int)blockIdx.x : (int)blockIdx.x - b0.count;
@@ -348,10 +362,11 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
   double* Ls = Pt + 16 * NP;
   double* Is = Ls + 16 * 17;
   __shared__ int floored;
-  double cv[NP * NP / 512];
+  constexpr int PER = NP * NP / NT;
+  double cv[PER];
 #pragma unroll
-  for (int q = 0; q < NP * NP / 512; ++q) {
-    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+  for (int q = 0; q < PER; ++q) {
+    const int e = tid + NT * q, r = e >> 7, c = e & (NP - 1);
     cv[q] = (c <= r && r < n) ? c_in[(int64_t)r * n + c] : 0.0;
   }
   if (tid < 32) {
@@ -366,43 +381,42 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
   __syncthreads();
   const double sigma = sigma_s;
 #pragma unroll
-  for (int q = 0; q < NP * NP / 512; ++q) {
-    const int e = tid + 512 * q, r = e >> 7, c = e & (NP - 1);
+  for (int q = 0; q < PER; ++q) {
+    const int e = tid + NT * q, r = e >> 7, c = e & (NP - 1);
     double v = (c <= r && r < n) ? cv[q] + (r == c ? sigma : 0.0) : 0.0;
     if (r >= n && r == c) v = 1.0;
     A[r * kCholLD + c] = v;
   }
   __syncthreads();
-  chol_blocks<true>(A, Dv, Pt, Ls, Is, n, sigma * 1e-3, &floored);
+  chol_blocks<true, NT>(A, Dv, Pt, Ls, Is, n, sigma * 1e-3, &floored);
   // M = L column-major (column j of M is column j of L), padding columns zero
 #pragma unroll
-  for (int q = 0; q < NP * NP / 512; ++q) {
-    const int e = tid + 512 * q, c = e >> 7, r = e & (NP - 1);
+  for (int q = 0; q < PER; ++q) {
+    const int e = tid + NT * q, c = e >> 7, r = e & (NP - 1);
     cv[q] = (r >= c && r < n && c < n) ? A[r * kCholLD + c] : 0.0;
   }
   __syncthreads();
 #pragma unroll
-  for (int q = 0; q < NP * NP / 512; ++q) M[tid + 512 * q] = cv[q];
+  for (int q = 0; q < PER; ++q) M[tid + NT * q] = cv[q];
   __syncthreads();
-  // ---- sweeps with the columns in registers. Warp w holds the tournament slots 4w .. 4w + 3;
+  // ---- sweeps with the columns in registers. Warp w holds the tournament slots S w .. S w + S - 1;
   // slot k pairs position k (top) with position 127 - k (bottom), and position j starts with
-  // column j. Lane l holds rows l, l + 32, l + 64, l + 96 of its 8 columns.
+  // column j. Lane l holds rows l, l + 32, l + 64, l + 96 of its 2 S columns.
   constexpr int RPL = NP / 32;
-  double top[4][RPL], bot[4][RPL];
+  double top[S][RPL], bot[S][RPL];
 #pragma unroll
-  for (int s = 0; s < 4; ++s)
+  for (int s = 0; s < S; ++s)
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-      top[s][i] = M[(4 * warp + s) * NP + lane + 32 * i];
-      bot[s][i] = M[(NP - 1 - 4 * warp - s) * NP + lane + 32 * i];
+      top[s][i] = M[(S * warp + s) * NP + lane + 32 * i];
+      bot[s][i] = M[(NP - 1 - S * warp - s) * NP + lane + 32 * i];
     }
   __syncthreads();
   // column exchange at the warp boundaries, double-buffered by round parity (reuses M)
-  double* XT = M;                    // [2][16][NP]: top of slot 4w + 3 handed to warp w + 1
-  double* XB = M + 2 * 16 * NP;      // [2][16][NP]: bottom of slot 4w handed to warp w - 1
-  double* XN = M + 4 * 16 * NP;      // [2][16][2]: the squared norms of those two columns
-  const int grp = lane >> 3;
-  const int l4 = (lane >> 4) & 1, l3 = (lane >> 3) & 1;
+  double* XT = M;                    // [2][W][NP]: top of slot S w + S - 1 handed to warp w + 1
+  double* XB = M + 2 * W * NP;       // [2][W][NP]: bottom of slot S w handed to warp w - 1
+  double* XN = M + 4 * W * NP;       // [2][W][2]: the squared norms of those two columns
+  const int grp = lane / GL;         // the slot whose pair parameters this lane computes
   // rotated[sweep & 1] collects this sweep's flag; the other entry is reset for the next
   // sweep while nobody reads it
   if (tid == 0) rotated[0] = rotated[1] = 0;
@@ -412,83 +426,73 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
     int any = 0;
     // squared column norms of slot `grp` (top: na, bottom: nb), exact at the start of the
     // sweep: per-lane partial sums, then butterflies over the 32 lanes
-    double na, nb;
-    {
-      double v[8];
+    double na = 0.0, nb = 0.0;
 #pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        double a = 0.0, b = 0.0;
+    for (int s = 0; s < S; ++s) {
+      double a = 0.0, b = 0.0;
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-          a = fma(top[s][i], top[s][i], a);
-          b = fma(bot[s][i], bot[s][i], b);
-        }
-        v[2 * s] = a;
-        v[2 * s + 1] = b;
+      for (int i = 0; i < RPL; ++i) {
+        a = fma(top[s][i], top[s][i], a);
+        b = fma(bot[s][i], bot[s][i], b);
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v[j] += __shfl_xor_sync(0xffffffffu, v[j], o);
-      na = v[0];
-      nb = v[1];
-#pragma unroll
-      for (int s = 1; s < 4; ++s)
-        if (grp == s) {
-          na = v[2 * s];
-          nb = v[2 * s + 1];
-        }
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+      }
+      if (grp == s) {
+        na = a;
+        nb = b;
+      }
     }
-    // One round at tournament phase K (rounds done in this sweep, mod 4). The slots' columns
+    // One round at tournament phase K (rounds done in this sweep, mod S). The slots' columns
     // are not moved between registers from round to round: logical top slot s lives in
-    // top[(s - K) & 3] and logical bottom slot s in bot[(s + K) & 3], so the column leaving a
-    // warp and the one arriving share a register and nothing else is copied.
-    // partial sums (this lane's rows) of gamma for slots 1 and 2 at phase K
-    double vpre[2];
-    auto partials12 = [&](auto kc) {
+    // top[(s - K) mod S] and logical bottom slot s in bot[(s + K) mod S], so the column leaving
+    // a warp and the one arriving share a register and nothing else is copied.
+    // Partial sums (this lane's rows) of gamma for the local slots 1 .. S - 2 at phase K: their
+    // columns never wait for another warp.
+    double vpre[S - 2];
+    auto partials_local = [&](auto kc) {
       constexpr int K = decltype(kc)::value;
 #pragma unroll
-      for (int s = 1; s <= 2; ++s) {
+      for (int s = 1; s <= S - 2; ++s) {
         double g = 0.0;
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) g = fma(top[(s - K) & 3][i], bot[(s + K) & 3][i], g);
+        for (int i = 0; i < RPL; ++i) g = fma(top[(s - K + S) % S][i], bot[(s + K) % S][i], g);
         vpre[s - 1] = g;
       }
     };
-    partials12(std::integral_constant<int, 0>{});
+    partials_local(std::integral_constant<int, 0>{});
     auto round = [&](auto kc) {
       constexpr int K = decltype(kc)::value;
       // a power of two within a factor 2 of 1 / (a + b) for this group's pair
       const int ex = (__double2hiint(na + nb) >> 20) & 0x7ff;
       const double sc2 = __hiloint2double((2046 - ex) << 20, 0);
-      // gamma of the four slots: per-lane partial sums, then a transposed butterfly that leaves
-      // slot grp's sum in the 8 lanes of group grp (identical in all of them)
-      // (slots 1 and 2 never wait for another warp: their partial sums were formed before the
-      // previous round's barrier)
-      double v[4];
-      v[1] = vpre[0];
-      v[2] = vpre[1];
+      // gamma of the S slots: per-lane partial sums, then a transposed butterfly that leaves
+      // slot grp's sum in the GL lanes of group grp (identical in all of them): log2 S steps
+      // halve the values a lane carries, then plain steps finish the sum
+      double v[S];
 #pragma unroll
-      for (int s = 0; s < 4; s += 3) {
+      for (int s = 1; s <= S - 2; ++s) v[s] = vpre[s - 1];
+#pragma unroll
+      for (int s = 0; s < S; s += S - 1) {
         double g = 0.0;
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) g = fma(top[(s - K) & 3][i], bot[(s + K) & 3][i], g);
+        for (int i = 0; i < RPL; ++i) g = fma(top[(s - K + S) % S][i], bot[(s + K) % S][i], g);
         v[s] = g;
       }
-      double w2[2];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const double keep = l4 ? v[i + 2] : v[i], send = l4 ? v[i] : v[i + 2];
-        w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+      for (int half = S / 2, m = 16; half >= 1; half >>= 1, m >>= 1) {
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const double keep = up ? v[i + half] : v[i], send = up ? v[i] : v[i + half];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
       }
-      double g;
-      {
-        const double keep = l3 ? w2[1] : w2[0], send = l3 ? w2[0] : w2[1];
-        g = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-      }
-      g += __shfl_xor_sync(0xffffffffu, g, 4);
-      g += __shfl_xor_sync(0xffffffffu, g, 2);
-      g += __shfl_xor_sync(0xffffffffu, g, 1);
+      double g = v[0];
+#pragma unroll
+      for (int m = GL / 2; m >= 1; m >>= 1) g += __shfl_xor_sync(0xffffffffu, g, m);
       const double a = na, b = nb;
       // rotation angle in float on (b - a, 2 gamma) scaled by the power of two of a + b (both
       // are at most a + b, so the squares below stay in range): with d = b - a,
@@ -520,11 +524,11 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
       // warp none of whose pairs rotates skips the arithmetic
       if (__any_sync(0xffffffffu, rot)) {
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const double cs = __shfl_sync(0xffffffffu, c, 8 * s);
-          const double ss = __shfl_sync(0xffffffffu, sn, 8 * s);
-          double* tp = top[(s - K) & 3];
-          double* bp = bot[(s + K) & 3];
+        for (int s = 0; s < S; ++s) {
+          const double cs = __shfl_sync(0xffffffffu, c, GL * s);
+          const double ss = __shfl_sync(0xffffffffu, sn, GL * s);
+          double* tp = top[(s - K + S) % S];
+          double* bp = bot[(s + K) % S];
 #pragma unroll
           for (int i = 0; i < RPL; ++i) {
             // both s products first, so that each result overwrites its own input
@@ -537,22 +541,22 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
       // next round of the circle tournament: position 0 stays, positions 1 .. 127 advance by
       // one. Tops move to the next slot, bottoms to the previous; slot 0's bottom becomes
       // slot 1's top and slot 63's top becomes its own bottom. The squared norms move with
-      // their columns. Leaving: top slot 3 (to warp + 1) and bottom slot 0 (to warp - 1).
-      constexpr int kOutT = (3 - K) & 3, kOutB = K & 3, kFixed = (0 - K) & 3;
+      // their columns. Leaving: top slot S - 1 (to warp + 1) and bottom slot 0 (to warp - 1).
+      constexpr int kOutT = (S - 1 - K + S) % S, kOutB = K % S, kFixed = (S - K) % S;
       constexpr int par = K & 1;
-      double* xt = XT + (par * 16 + warp) * NP;
-      double* xb = XB + (par * 16 + warp) * NP;
+      double* xt = XT + (par * W + warp) * NP;
+      double* xb = XB + (par * W + warp) * NP;
 #pragma unroll
       for (int i = 0; i < RPL; ++i) {
-        if (warp < 15) xt[lane + 32 * i] = top[kOutT][i];
+        if (warp < W - 1) xt[lane + 32 * i] = top[kOutT][i];
         if (warp > 0) xb[lane + 32 * i] = bot[kOutB][i];
       }
-      if (warp < 15 && lane == 24) XN[(par * 16 + warp) * 2] = na;        // top of slot 4w + 3
-      if (warp > 0 && lane == 0) XN[(par * 16 + warp) * 2 + 1] = nb;      // bottom of slot 4w
-      const double up_a = __shfl_up_sync(0xffffffffu, (warp == 0 && grp == 0) ? nb : na, 8);
-      const double dn_b = __shfl_down_sync(0xffffffffu, nb, 8);
-      // moves that stay inside the edge warps, then the next round's partial sums of slots 1 and
-      // 2 (their columns are all here), then the barrier and the two arriving columns
+      if (warp < W - 1 && lane == GL * (S - 1)) XN[(par * W + warp) * 2] = na;   // top of slot S w + S - 1
+      if (warp > 0 && lane == 0) XN[(par * W + warp) * 2 + 1] = nb;              // bottom of slot S w
+      const double up_a = __shfl_up_sync(0xffffffffu, (warp == 0 && grp == 0) ? nb : na, GL);
+      const double dn_b = __shfl_down_sync(0xffffffffu, nb, GL);
+      // moves that stay inside the edge warps, then the next round's partial sums of the local
+      // slots (their columns are all here), then the barrier and the two arriving columns
       if (warp == 0) {
         // position 0 stays in slot 0's top; the leaving bottom becomes slot 1's top
 #pragma unroll
@@ -560,33 +564,28 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
           top[kOutT][i] = top[kFixed][i];
           top[kFixed][i] = bot[kOutB][i];
         }
-      } else if (warp == 15) {
+      } else if (warp == W - 1) {
         // slot 63's top turns into its own bottom
 #pragma unroll
         for (int i = 0; i < RPL; ++i) bot[kOutB][i] = top[kOutT][i];
       }
-      partials12(std::integral_constant<int, (K + 1) & 3>{});
+      partials_local(std::integral_constant<int, (K + 1) % S>{});
       __syncthreads();
-      const double* xin_t = XT + (par * 16 + (warp > 0 ? warp - 1 : 0)) * NP;
-      const double* xin_b = XB + (par * 16 + (warp < 15 ? warp + 1 : 15)) * NP;
+      const double* xin_t = XT + (par * W + (warp > 0 ? warp - 1 : 0)) * NP;
+      const double* xin_b = XB + (par * W + (warp < W - 1 ? warp + 1 : W - 1)) * NP;
 #pragma unroll
       for (int i = 0; i < RPL; ++i) {
         if (warp > 0) top[kOutT][i] = xin_t[lane + 32 * i];
-        if (warp < 15) bot[kOutB][i] = xin_b[lane + 32 * i];
+        if (warp < W - 1) bot[kOutB][i] = xin_b[lane + 32 * i];
       }
-      const double na_new = grp >= 1 ? up_a : (warp == 0 ? na : XN[(par * 16 + warp - 1) * 2]);
-      const double nb_new = grp <= 2 ? dn_b : (warp < 15 ? XN[(par * 16 + warp + 1) * 2 + 1] : na);
+      const double na_new = grp >= 1 ? up_a : (warp == 0 ? na : XN[(par * W + warp - 1) * 2]);
+      const double nb_new = grp <= S - 2 ? dn_b : (warp < W - 1 ? XN[(par * W + warp + 1) * 2 + 1] : na);
       na = na_new;
       nb = nb_new;
     };
     // 128 rounds: the 127 of the tournament and the first one again, so that every sweep starts
     // at phase 0 (the columns end one position further on per sweep; only their set matters)
-    for (int r = 0; r < NP; r += 4) {
-      round(std::integral_constant<int, 0>{});
-      round(std::integral_constant<int, 1>{});
-      round(std::integral_constant<int, 2>{});
-      round(std::integral_constant<int, 3>{});
-    }
+    for (int r = 0; r < NP; r += S) unroll_phases<0, S>(round);
     if (any) rotated[sweep & 1] = 1;
     if (tid == 0) rotated[(sweep + 1) & 1] = 0;
     __syncthreads();
@@ -596,15 +595,15 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
   // the columns, in the positions the last sweep left them in (their order does not matter:
   // they are ranked by norm below)
 #pragma unroll
-  for (int s = 0; s < 4; ++s)
+  for (int s = 0; s < S; ++s)
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-      M[(4 * warp + s) * NP + lane + 32 * i] = top[s][i];
-      M[(NP - 1 - 4 * warp - s) * NP + lane + 32 * i] = bot[s][i];
+      M[(S * warp + s) * NP + lane + 32 * i] = top[s][i];
+      M[(NP - 1 - S * warp - s) * NP + lane + 32 * i] = bot[s][i];
     }
   __syncthreads();
   // column norms, descending order (zero padding sorts last)
-  for (int j = warp; j < NP; j += 16) {
+  for (int j = warp; j < NP; j += W) {
     const double* mj = M + j * NP + 4 * lane;
     double a = mj[0] * mj[0] + mj[1] * mj[1] + mj[2] * mj[2] + mj[3] * mj[3];
 #pragma unroll
@@ -612,7 +611,7 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
     if (lane == 0) nrm[j] = a;
   }
   __syncthreads();
-  for (int i = tid; i < NP; i += 512) {
+  for (int i = tid; i < NP; i += NT) {
     const double li = nrm[i];
     int rk = 0;
     for (int j = 0; j < NP; ++j) {
@@ -623,14 +622,14 @@ __global__ void __launch_bounds__(512) k_eig_psd(EigBatch b0, EigBatch b1, int m
   }
   __syncthreads();
   float* vo = Vout + (int64_t)bi * sV;
-  for (int e = tid; e < n * NP; e += 512) {
+  for (int e = tid; e < n * NP; e += NT) {
     const int c = e >> 7, r = e & (NP - 1);   // column c of M, row r
     if (r >= n || rank[c] >= n) continue;
     const double inv = nrm[c] > 0.0 ? 1.0 / sqrt(nrm[c]) : 0.0;
     vo[(int64_t)r * n + rank[c]] = (float)(M[c * NP + r] * inv);
   }
   if (lam)
-    for (int c = tid; c < NP; c += 512)
+    for (int c = tid; c < NP; c += NT)
       if (rank[c] < n) lam[(int64_t)bi * sL + rank[c]] = (float)(nrm[c] - sigma);
 }
 
@@ -782,11 +781,11 @@ cudaError_t eig_psd2(int batch0, int n0, const double* C0, int64_t sC0, float* V
   // the blocked Cholesky's arrays (A, diagonal inverses, panel, diagonal factor) overlay M,
   // the column norms and the ranks
   const size_t smem = ((size_t)kMaxN * kCholLD + 8 * 256 + 16 * kMaxN + 16 * 17 + 16) * sizeof(double);
-  cudaError_t e = cudaFuncSetAttribute(k_eig_psd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(k_eig_psd<kEigWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   EigBatch b0{C0, sC0, V0, sV0, lam0, sL0, n0, batch0};
   EigBatch b1{C1, sC1, V1, sV1, lam1, sL1, batch1 > 0 ? n1 : n0, batch1 > 0 ? batch1 : 0};
-  k_eig_psd<<<batch0 + b1.count, 512, smem, s>>>(b0, b1, max_sweeps, status);
+  k_eig_psd<kEigWarps><<<batch0 + b1.count, 32 * kEigWarps, smem, s>>>(b0, b1, max_sweeps, status);
   note_launch();
   return cudaGetLastError();
 }
