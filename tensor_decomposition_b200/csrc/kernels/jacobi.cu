@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
     // a warp and the one arriving share a register and nothing else is copied.
     // Partial sums (this lane's rows) of gamma for the local slots 1 .. S - 2 at phase K: their
     // columns never wait for another warp.
-    double vpre[S - 2];
+    double vpre[S > 2 ? S - 2 : 1];
     auto partials_local = [&](auto kc) {
       constexpr int K = decltype(kc)::value;
 #pragma unroll
