@@ -332,6 +332,73 @@ __device__ __forceinline__ void unroll_phases(F& f) {
   }
 }
 
+// A sweep in which no pair was further than sqrt(kCheckCos2) from orthogonal (cosine of the
+// two columns) is followed by the Gram test below instead of a verifying sweep. Convergence is
+// quadratic at the end: after a sweep whose largest cosine is 1e-4 the next one rarely finds a
+// pair above the 1e-7 rotation threshold; a test that fails costs about a tenth of a sweep.
+constexpr double kCheckCos2 = 1e-8;
+// shared memory of k_eig_psd: the Cholesky's arrays (A, diagonal inverses, panel, diagonal
+// factor and its reciprocals), which the column array, the Gram test's padded copy and the
+// norms and ranks overlay
+constexpr size_t kEigSmemDoubles = (size_t)kMaxN * kCholLD + 8 * 256 + 16 * kMaxN + 16 * 17 + 16;
+static_assert((size_t)kMaxN * (kMaxN + 4) + kMaxN <= kEigSmemDoubles, "Gram test array (stride kMaxN + 4)");
+static_assert((size_t)kMaxN * kMaxN + kMaxN + kMaxN / 2 <= kEigSmemDoubles, "columns, norms, ranks");
+
+__device__ __forceinline__ void dmma_f64(double& d0, double& d1, double a, double b) {
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+      : "+d"(d0), "+d"(d1)
+      : "d"(a), "d"(b));
+}
+
+// The sweep's rotation criterion for a pair with dot product g and squared norms a, b: the
+// same power-of-two scale and float conversion as the angle computation.
+__device__ __forceinline__ bool pair_rotates(double g, double a, double b) {
+  const int ex = (__double2hiint(a + b) >> 20) & 0x7ff;
+  const double sc2 = __hiloint2double((2046 - ex) << 20, 0);
+  return g * g > 1e-14 * (a * b) && (float)(g * (2.0 * sc2)) != 0.0f;
+}
+
+// Whether every pair of the 128 columns, copied column-major at stride kGramLD with their
+// squared norms after them, passes the rotation criterion without rotating, i.e. whether a
+// sweep would leave them as they are. The upper triangle of M^T M is formed in 8 x 8 tiles on
+// the FP64 MMA (m8n8k4, fragments per the PTX ISA; warp w takes tiles w, w + W, ..., two
+// accumulator chains per tile; the stride makes the fragment loads conflict-free). Kept out of
+// line so that its registers do not add to those of the sweep. Ends with a barrier after its
+// last read of the copy (the next round's column exchange overwrites it) and returns the same
+// value in every thread.
+constexpr int kGramLD = kMaxN + 4;
+
+template <int W>
+__device__ __noinline__ bool gram_all_converged(const double* Mc, int* violated) {
+  constexpr int NP = kMaxN, NB = NP / 8;
+  const double* cn = Mc + NP * kGramLD;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = lane >> 2, kk = lane & 3;
+  bool bad = false;
+  for (int t = warp; t < NB * (NB + 1) / 2; t += W) {
+    int bi = 0, rem = t;          // t-th tile of the upper triangle, row by row
+    while (rem >= NB - bi) {
+      rem -= NB - bi;
+      ++bi;
+    }
+    const int bj = bi + rem;
+    const double* pa = Mc + (8 * bi + r) * kGramLD + kk;
+    const double* pb = Mc + (8 * bj + r) * kGramLD + kk;
+    double c0 = 0.0, c1 = 0.0, e0 = 0.0, e1 = 0.0;
+#pragma unroll 4
+    for (int k0 = 0; k0 < NP; k0 += 8) {
+      dmma_f64(c0, c1, pa[k0], pb[k0]);
+      dmma_f64(e0, e1, pa[k0 + 4], pb[k0 + 4]);
+    }
+    const int i = 8 * bi + r, j = 8 * bj + 2 * kk;
+    bad |= i < j && pair_rotates(c0 + e0, cn[i], cn[j]);
+    bad |= i < j + 1 && pair_rotates(c1 + e1, cn[i], cn[j + 1]);
+  }
+  if (bad) *violated = 1;
+  __syncthreads();
+  return *violated == 0;
+}
+
 // Two independent batches share one launch (blocks [0, b0.count) take the first). W warps of
 // S = 64 / W tournament slots each (W = 8: 16 columns of 4 rows per lane in registers).
 template <int W>
@@ -350,7 +417,7 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
   double* M = ms;                 // column-major: column j at M + j * NP (during Cholesky: row-major R)
   double* nrm = M + NP * NP;      // NP squared column norms
   int* rank = reinterpret_cast<int*>(nrm + NP);
-  __shared__ int rotated[2];
+  __shared__ int rotated[2], large[2], violated;
   __shared__ double sigma_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const double* c_in = Cin + (int64_t)bi * sC;
@@ -419,7 +486,7 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
   const int grp = lane / GL;         // the slot whose pair parameters this lane computes
   // rotated[sweep & 1] collects this sweep's flag; the other entry is reset for the next
   // sweep while nobody reads it
-  if (tid == 0) rotated[0] = rotated[1] = 0;
+  if (tid == 0) rotated[0] = rotated[1] = large[0] = large[1] = 0;
   __syncthreads();
   int sweep = 0;
   for (; sweep < max_sweeps; ++sweep) {
@@ -519,7 +586,8 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
         na = rot ? na_r : a;
         nb = rot ? nb_r : b;
       }
-      any |= (int)rot;
+      // bit 0: a pair rotated; bit 1: a pair was further from orthogonal than the Gram test's bound
+      any |= (int)rot | ((int)(g * g > kCheckCos2 * (a * b)) << 1);
       // rotate every slot with its group's (c, s); (1, 0) leaves a pair unchanged exactly, so a
       // warp none of whose pairs rotates skips the arithmetic
       if (__any_sync(0xffffffffu, rot)) {
@@ -586,10 +654,43 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
     // 128 rounds: the 127 of the tournament and the first one again, so that every sweep starts
     // at phase 0 (the columns end one position further on per sweep; only their set matters)
     for (int r = 0; r < NP; r += S) unroll_phases<0, S>(round);
-    if (any) rotated[sweep & 1] = 1;
-    if (tid == 0) rotated[(sweep + 1) & 1] = 0;
+    if (any & 1) rotated[sweep & 1] = 1;
+    if (any & 2) large[sweep & 1] = 1;
+    if (tid == 0) rotated[(sweep + 1) & 1] = large[(sweep + 1) & 1] = 0;
     __syncthreads();
     if (!rotated[sweep & 1]) break;
+    // A sweep whose pairs were all within kCheckCos2 of orthogonal is usually followed by one
+    // that rotates nothing. That sweep only tests every pair once against the rotation
+    // criterion with M unchanged, so the same test on the Gram matrix M^T M of the columns
+    // as they stand decides it at a tenth of the cost; the sweep runs only if a pair fails.
+    if (!large[sweep & 1]) {
+      double* Mc = ms;
+      double* cn = ms + NP * kGramLD;
+      if (tid == 0) violated = 0;
+#pragma unroll
+      for (int s = 0; s < S; ++s) {
+        const int pt = S * warp + s, pb = NP - 1 - S * warp - s;
+        double a = 0.0, b = 0.0;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+          Mc[pt * kGramLD + lane + 32 * i] = top[s][i];
+          Mc[pb * kGramLD + lane + 32 * i] = bot[s][i];
+          a = fma(top[s][i], top[s][i], a);
+          b = fma(bot[s][i], bot[s][i], b);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          a += __shfl_xor_sync(0xffffffffu, a, o);
+          b += __shfl_xor_sync(0xffffffffu, b, o);
+        }
+        if (lane == 0) {
+          cn[pt] = a;
+          cn[pb] = b;
+        }
+      }
+      __syncthreads();
+      if (gram_all_converged<W>(Mc, &violated)) break;
+    }
   }
   if (sweep == max_sweeps && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
   // the columns, in the positions the last sweep left them in (their order does not matter:
@@ -780,7 +881,7 @@ cudaError_t eig_psd2(int batch0, int n0, const double* C0, int64_t sC0, float* V
   if (batch0 + batch1 <= 0) return cudaSuccess;
   // the blocked Cholesky's arrays (A, diagonal inverses, panel, diagonal factor) overlay M,
   // the column norms and the ranks
-  const size_t smem = ((size_t)kMaxN * kCholLD + 8 * 256 + 16 * kMaxN + 16 * 17 + 16) * sizeof(double);
+  const size_t smem = kEigSmemDoubles * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_eig_psd<kEigWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   EigBatch b0{C0, sC0, V0, sV0, lam0, sL0, n0, batch0};
