@@ -11,8 +11,10 @@
 // TMA tile loads (128 rows x 64 bf16, 128-byte swizzle, no multicast) into a ring of stages
 // that runs on across tiles; warp 1 owns two Tensor Memory accumulators and issues
 // tcgen05.mma (M = 128, N = 128, K = 16) from one thread, alternating between them tile by
-// tile; warps 4-7 read a finished accumulator back with tcgen05.ld and store float32 (and/or
-// bf16 parts) while the next tile is being loaded and multiplied. Every wait is bounded and
+// tile; warps 4-11 read a finished accumulator back with tcgen05.ld and store float32 (and/or
+// bf16 parts) while the next tile is being loaded and multiplied (two warps per TMEM lane
+// quadrant, one per half of the columns, so that each SM sub-partition has two epilogue warps
+// to interleave). Every wait is bounded and
 // reports ST_TIMEOUT instead of hanging.
 #include "../jolt_internal.h"
 #include "sm100.cuh"
@@ -135,7 +137,8 @@ __device__ __forceinline__ void store_parts_chunk(__nv_bfloat16* const (&P)[3], 
   }
 }
 
-constexpr int kStgBytes = 4 * 32 * 33 * 4;   // epilogue staging: one 32 x 33 float chunk per warp
+constexpr int kEpiWarps = 8;                         // warps 4 .. 11
+constexpr int kStgBytes = kEpiWarps * 32 * 33 * 4;   // epilogue staging: one 32 x 33 float chunk per warp
 
 // Tile t of the launch: n tiles fastest (consecutive tiles of a CTA share A rows through L2),
 // then m tiles, then the batch.
@@ -149,11 +152,11 @@ __device__ __forceinline__ void tile_coords(int t, int ntn, int ntm, int& n0, in
 
 // Persistent: CTA c takes the tiles c, c + gridDim.x, ... Warp 0 streams the operand tiles of
 // all of them through the stage ring; warp 1 accumulates tile i in TMEM buffer i & 1 (two
-// 128-column buffers), so that warps 4-7 read tile i back and store it while tile i + 1 is
+// 128-column buffers), so that warps 4-11 read tile i back and store it while tile i + 1 is
 // loaded and multiplied. Barriers: full / empty per stage (TMA bytes / MMA completion),
-// acc_full per buffer (MMA completion), acc_empty per buffer (the four epilogue warps).
+// acc_full per buffer (MMA completion), acc_empty per buffer (the eight epilogue warps).
 template <int STAGES>
-__global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGemmParams p, int ntiles, int ntn,
+__global__ void __launch_bounds__(128 + 32 * kEpiWarps, 1) k_gemm_tc(const __grid_constant__ TcGemmParams p, int ntiles, int ntn,
                                                      int ntm) {
   extern __shared__ uint8_t smraw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -193,7 +196,7 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(&acc_full[j], 1);
-      mbar_init(&acc_empty[j], 4);
+      mbar_init(&acc_empty[j], kEpiWarps);
     }
     abort_s = 0;
     fence_barrier_init();
@@ -273,12 +276,15 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
       }
     }
   } else if (warp >= 4) {
-    const int e = warp - 4;                      // TMEM lanes 32e .. 32e + 31
+    // a warp reaches TMEM lanes 32 (warp % 4) .. + 31 only: warps 4 + e and 8 + e share lane
+    // quadrant e and take the first and the second half of the columns
+    const int e = warp & 3, half = (warp - 4) >> 2;
+    constexpr int kChunks = kTile / 32 / 2;       // 32-column chunks per warp and tile
     // Outputs contiguous along n (row-major C: c_sn = 1, or a part layout with unit n stride)
     // go through shared memory in 32 x 32 chunks, so that a store instruction covers
     // consecutive n of one row; outputs contiguous along m are stored from the registers
     // (consecutive lanes, consecutive m).
-    float* stg = reinterpret_cast<float*>(smem + STAGES * stage_bytes) + e * (32 * 33);
+    float* stg = reinterpret_cast<float*>(smem + STAGES * stage_bytes) + (warp - 4) * (32 * 33);
     const bool has_c = p.C != nullptr;
     const bool c_n = has_c && p.c_sn == 1;
     const bool parts = p.ps[0] || p.pt[0];
@@ -308,11 +314,11 @@ __global__ void __launch_bounds__(256, 1) k_gemm_tc(const __grid_constant__ TcGe
       const uint32_t tbase = tmem + (uint32_t)(ab * kTile) + ((uint32_t)(32 * e) << 16);
       const int mr0 = m0 + 32 * e;   // first row of this warp's chunks
 #pragma unroll 1
-      for (int c = 0; c < kTile / 32; ++c) {
+      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
         uint32_t r[32];
         tmem_ld32(tbase + (uint32_t)(c * 32), r);
         tmem_ld_wait();
-        if (c == kTile / 32 - 1) {
+        if (c == (half + 1) * kChunks - 1) {
           // the whole accumulator is in registers or staged: hand the buffer back to the MMA warp
           tc_fence_before();
           __syncwarp();
@@ -448,19 +454,19 @@ cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
   switch (stages) {
     case 2:
       e = cudaFuncSetAttribute(k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e == cudaSuccess) k_gemm_tc<2><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      if (e == cudaSuccess) k_gemm_tc<2><<<grid, 128 + 32 * kEpiWarps, smem, s>>>(p, ntiles, ntn, ntm);
       break;
     case 3:
       e = cudaFuncSetAttribute(k_gemm_tc<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e == cudaSuccess) k_gemm_tc<3><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      if (e == cudaSuccess) k_gemm_tc<3><<<grid, 128 + 32 * kEpiWarps, smem, s>>>(p, ntiles, ntn, ntm);
       break;
     case 4:
       e = cudaFuncSetAttribute(k_gemm_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e == cudaSuccess) k_gemm_tc<4><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      if (e == cudaSuccess) k_gemm_tc<4><<<grid, 128 + 32 * kEpiWarps, smem, s>>>(p, ntiles, ntn, ntm);
       break;
     default:
       e = cudaFuncSetAttribute(k_gemm_tc<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e == cudaSuccess) k_gemm_tc<6><<<grid, 256, smem, s>>>(p, ntiles, ntn, ntm);
+      if (e == cudaSuccess) k_gemm_tc<6><<<grid, 128 + 32 * kEpiWarps, smem, s>>>(p, ntiles, ntn, ntm);
       break;
   }
   if (e != cudaSuccess) return e;
