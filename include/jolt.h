@@ -238,6 +238,13 @@ JOLT_API uint64_t jolt_launch_count(void);
 JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const void* B,
                                              float* C, void* cuda_stream);
 
+/* jolt_selftest_gemm_bf16_layout - the same product with either operand stored transposed, as
+ * the analysis keeps its bf16 bases (the operand then enters the MMA MN-major): A is [M][K]
+ * (a_mn = 0) or [K][M] (a_mn = 1), B is [N][K] (b_mn = 0) or [K][N] (b_mn = 1); a transposed
+ * operand needs M (N) a multiple of 8. Otherwise as jolt_selftest_gemm_bf16. */
+JOLT_API jolt_status jolt_selftest_gemm_bf16_layout(int32_t M, int32_t N, int32_t K, const void* A, int32_t a_mn,
+                                                    const void* B, int32_t b_mn, float* C, void* cuda_stream);
+
 /* Release a stream. Its device memory is freed in order on the CUDA stream the stream was
  * created on (encode or jolt_stream_from_host); synchronise any other CUDA stream that still
  * reads it (e.g. a decode issued elsewhere) before destroying it. */

@@ -239,10 +239,8 @@ struct jolt_plan_s {
   bool use_tc = false;       // bf16 inputs with T % 8 == 0: contractions over X on tcgen05
   __nv_bfloat16* XT = nullptr;       // [n][H][D][T]
   float* Cpart = nullptr;            // [n][H][D][D] per-head Gram partials
-  __nv_bfloat16* QTp[3] = {nullptr, nullptr, nullptr};   // bf16 parts of a float32 basis
-  __nv_bfloat16* QNp[3] = {nullptr, nullptr, nullptr};   // the same parts, transposed layout
+  __nv_bfloat16* QTp[3] = {nullptr, nullptr, nullptr};   // bf16 parts of a float32 basis [n][l][rows]
   __nv_bfloat16* QTp2[3] = {nullptr, nullptr, nullptr};  // second part set (CholeskyQR ping-pong)
-  __nv_bfloat16* QNp2[3] = {nullptr, nullptr, nullptr};
   __nv_bfloat16* RTp[3] = {nullptr, nullptr, nullptr};   // parts of R^{-T} (CholeskyQR)
   float* Wpart = nullptr;                                // K-chunk partial Grams (CholeskyQR)
   int qset = 0;                                          // part set holding the final sketch basis
@@ -373,10 +371,10 @@ bool map_perhead(CUtensorMap* m, const void* P, int64_t K, int64_t D, int64_t H,
   const uint64_t str[3] = {(uint64_t)K * 2, (uint64_t)(D * K * 2), (uint64_t)(H * D * K * 2)};
   return tc_map_bf16(m, P, 4, dims, str);
 }
-// Three bf16 parts of a float32 basis [n][l][rows]: in that layout (s) and transposed (t).
+// Three bf16 parts of a float32 basis [n][l][rows] (rows contiguous). GEMMs that contract over
+// the rows read it K-major; those that contract over l read it MN-major (VIEW_MN).
 struct PartSet {
   __nv_bfloat16* s[3];
-  __nv_bfloat16* t[3];
 };
 
 // Products of two three-part operands kept for float32 accuracy: (0,0) (0,1) (1,0) (1,1) (0,2) (2,0).
@@ -408,11 +406,11 @@ int gram_chunks(int rows) {
 }
 
 // CholeskyQR on the tensor cores over bf16 parts. A basis Y^T [n][l][rows] is held as three
-// bf16 parts in its own layout (set.s) and transposed, [n][rows][l] (set.t). Each pass forms
-// the Gram W = Y^T Y from the six part products of order <= 2 as float32 partial sums over up to
-// 16 chunks of the rows (one CTA each), sums the chunks in float64, inverts its Cholesky
-// factor in float64, and forms Q^T = R^{-T} Y^T from the six part products of R^{-T} and Y,
-// whose epilogue writes Q's parts (both layouts) into the other set. Pass 1 adds 1e-6 trace(W)
+// bf16 parts (set.s). Each pass forms the Gram W = Y^T Y from the six part products of order
+// <= 2 as float32 partial sums over up to 16 chunks of the rows (one CTA each), sums the chunks
+// in float64, inverts its Cholesky factor in float64, and forms Q^T = R^{-T} Y^T from the six
+// part products of R^{-T} and Y (read MN-major from the same parts), whose epilogue writes Q's
+// parts into the other set. Pass 1 adds 1e-6 trace(W)
 // to the diagonal (a shifted CholeskyQR step; the accumulation error of the Gram is ~1e-7), so
 // the factorisation exists for any sketch; the column space is unchanged by the shift.
 // Returns the index of the set that holds the result.
@@ -448,20 +446,17 @@ int cholqr_tc(jolt_plan_s* p, int rows, PartSet* sets, int cur, int passes, int3
     TcGemmParams m;
     m.status = status;
     for (int i = 0; i < 3; ++i)
-      if (!map_rows(&m.amap[i], p->RTp[i], l, l, n) || !map_rows(&m.bmap[i], in.t[i], l, rows, n)) {
+      if (!map_rows(&m.amap[i], p->RTp[i], l, l, n) || !tc_map_bf16_mn(&m.bmap[i], in.s[i], rows, l, n)) {
         *st = fail(JOLT_ERR_CUDA, "tensor map rejected");
         return cur;
       }
+    m.bv.mode = VIEW_MN;             // Y from its [l][rows] parts, rows contiguous
     m.na = m.nb = 3;
     six_products(m);
     m.M = l; m.N = rows; m.KB = (l + 63) / 64;
     m.C = nullptr;
     m.c_sm = rows; m.c_sn = 1; m.c_sb = (int64_t)l * rows;       // Q^T parts [l][rows]
-    m.t_sm = 1; m.t_sn = l; m.t_sb = (int64_t)rows * l;          // Q parts [rows][l]
-    for (int i = 0; i < 3; ++i) {
-      m.ps[i] = out.s[i];
-      m.pt[i] = out.t[i];
-    }
+    for (int i = 0; i < 3; ++i) m.ps[i] = out.s[i];
     ck(gemm_tc(n, m, s));
     cur ^= 1;
   }
@@ -672,9 +667,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
       take(p->Cpart, n * H * D * D * k_chunks(T));   // per-head (and per K chunk) partials
       if (p->encoder == JOLT_ENC_SKETCH) {
         for (int i = 0; i < 3; ++i) take(p->QTp[i], n * l * std::max<int64_t>(T, HD));
-        for (int i = 0; i < 3; ++i) take(p->QNp[i], n * l * std::max<int64_t>(T, HD));
         for (int i = 0; i < 3; ++i) take(p->QTp2[i], n * l * std::max<int64_t>(T, HD));
-        for (int i = 0; i < 3; ++i) take(p->QNp2[i], n * l * std::max<int64_t>(T, HD));
         for (int i = 0; i < 3; ++i) take(p->RTp[i], n * l * l);
         take(p->Wf, n * l * l);
         take(p->Wpart, n * 16 * l * l);
@@ -856,8 +849,8 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       // two part sets: every basis lives as bf16 parts, written by the epilogue that makes it
       PartSet sets[2];
       for (int i = 0; i < 3; ++i) {
-        sets[0].s[i] = p->QTp[i]; sets[0].t[i] = p->QNp[i];
-        sets[1].s[i] = p->QTp2[i]; sets[1].t[i] = p->QNp2[i];
+        sets[0].s[i] = p->QTp[i];
+        sets[1].s[i] = p->QTp2[i];
       }
       auto tc_params = [&]() {
         TcGemmParams g;
@@ -878,11 +871,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
           g.M = T; g.N = l; g.KB = (int)(HD / 64);
           g.C = nullptr;
           g.c_sm = 1; g.c_sn = T; g.c_sb = (int64_t)l * T;
-          g.t_sm = l; g.t_sn = 1; g.t_sb = (int64_t)T * l;
-          for (int i = 0; i < 3; ++i) {
-            g.ps[i] = out.s[i] + (int64_t)k * L * l * T;
-            g.pt[i] = out.t[i] + (int64_t)k * L * l * T;
-          }
+          for (int i = 0; i < 3; ++i) g.ps[i] = out.s[i] + (int64_t)k * L * l * T;
           CK(gemm_tc(L, g, s));
         }
         return JOLT_OK;
@@ -916,11 +905,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
           const int kc = k_chunks(T);
           if (kc == 1) {
             g.C = nullptr;
-            g.t_sm = l; g.t_sn = 1; g.t_sb = (int64_t)HD * l;
-            for (int i = 0; i < 3; ++i) {
-              g.ps[i] = sets[cur ^ 1].s[i];
-              g.pt[i] = sets[cur ^ 1].t[i];
-            }
+            for (int i = 0; i < 3; ++i) g.ps[i] = sets[cur ^ 1].s[i];
             CK(gemm_tc(n, g, s));
           } else {
             // long K: float32 partials per chunk of tokens, float64 sum, then the parts
@@ -930,7 +915,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
             g.C = p->Cpart;
             CK(gemm_tc(n * kc, g, s));
             CK(sum_heads(n, kc, (int64_t)l * HD, p->Cpart, p->Z, nullptr, s));
-            CK(split_dual(n, l, (int)HD, p->Z, false, sets[cur ^ 1].s, sets[cur ^ 1].t, s));
+            CK(split_dual(n, l, (int)HD, p->Z, false, sets[cur ^ 1].s, nullptr, s));
           }
           cur ^= 1;
         }
@@ -964,17 +949,13 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         g.na = 3; g.nb = 1;
         g.M = l; g.N = (int)HD; g.KB = (T + 63) / 64;
         g.c_sm = HD; g.c_sn = 1; g.c_sb = (int64_t)l * HD;
-        // B's bf16 parts, [l][HD] for B B^T and [HD][l] for the per-head core, go to the part
+        // B's bf16 parts [l][HD] (for B B^T, and MN-major for the per-head core) go to the part
         // set that does not hold Q
         const PartSet& bs = sets[cur ^ 1];
         const int kc = k_chunks(T);
         if (kc == 1) {
           g.C = p->Bm;
-          g.t_sm = 1; g.t_sn = l; g.t_sb = (int64_t)HD * l;
-          for (int i = 0; i < 3; ++i) {
-            g.ps[i] = bs.s[i];
-            g.pt[i] = bs.t[i];
-          }
+          for (int i = 0; i < 3; ++i) g.ps[i] = bs.s[i];
           CK(gemm_tc(n, g, s));
         } else {
           // long K: float32 partials per chunk of tokens, summed in float64, then the parts
@@ -984,7 +965,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
           g.C = p->Cpart;
           CK(gemm_tc(n * kc, g, s));
           CK(sum_heads(n, kc, (int64_t)l * HD, p->Cpart, p->Bm, nullptr, s));
-          CK(split_dual(n, l, (int)HD, p->Bm, false, bs.s, bs.t, s));
+          CK(split_dual(n, l, (int)HD, p->Bm, false, bs.s, nullptr, s));
         }
       }
       p->Qfinal = nullptr;
@@ -1089,14 +1070,16 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       }
       {
         PROF("small_gemm", s);
-        // U_T = Q W[:, :R]: rows t, K = the sketch index; Q parts [T][l] from CholeskyQR, W^T parts
+        // U_T = Q W[:, :R]: rows t, K = the sketch index; Q from its parts [l][T] (MN-major),
+        // W^T parts
         CK(split_dual(n, l, l, p->Wv, false, nullptr, p->RTp, s));
-        __nv_bfloat16* const* qn = p->qset ? p->QNp2 : p->QNp;
+        __nv_bfloat16* const* qs = p->qset ? p->QTp2 : p->QTp;
         TcGemmParams g;
         g.status = status;
         for (int i = 0; i < 3; ++i)
-          if (!map_rows(&g.amap[i], qn[i], l, T, n) || !map_rows(&g.bmap[i], p->RTp[i], l, l, n))
+          if (!tc_map_bf16_mn(&g.amap[i], qs[i], T, l, n) || !map_rows(&g.bmap[i], p->RTp[i], l, l, n))
             return fail(JOLT_ERR_CUDA, "tensor map rejected");
+        g.av.mode = VIEW_MN;
         g.na = g.nb = 3;
         six_products(g);
         g.M = T; g.N = R; g.KB = (l + 63) / 64;
@@ -1110,16 +1093,17 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       }
       {
         PROF("core", s);
-        // P[h] = W_R^T B_h (R x D): W^T parts (signs fixed), B^T parts per head
+        // P[h] = W_R^T B_h (R x D): W^T parts (signs fixed), head h's columns of the B parts
+        // [l][HD] (set qset ^ 1), MN-major
         CK(split_dual(n, l, l, p->Wv, false, nullptr, p->RTp, s));
-        __nv_bfloat16* const* btr = p->qset ? p->QNp : p->QNp2;       // B parts [HD][l] (set qset ^ 1)
+        __nv_bfloat16* const* bsp = p->qset ? p->QTp : p->QTp2;
         TcGemmParams g;
         g.status = status;
         for (int i = 0; i < 3; ++i)
-          if (!map_rows(&g.amap[i], p->RTp[i], l, l, n) || !map_perhead(&g.bmap[i], btr[i], l, D, H, n))
+          if (!map_rows(&g.amap[i], p->RTp[i], l, l, n) || !tc_map_bf16_mn(&g.bmap[i], bsp[i], HD, l, n))
             return fail(JOLT_ERR_CUDA, "tensor map rejected");
         g.av.H = H;                       // W^T shared by the heads of a layer-tensor
-        g.bv.mode = VIEW_XT_PERHEAD;
+        g.bv.mode = VIEW_MN;
         g.bv.H = H;
         g.bv.D = D;
         g.na = g.nb = 3;
@@ -1685,17 +1669,21 @@ JOLT_API jolt_status jolt_export_debug(jolt_stream_t st, int32_t what, int32_t l
   return JOLT_OK;
 }
 
-JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const void* B,
-                                             float* C, void* cuda_stream) {
+namespace {
+jolt_status selftest_gemm(const char* who, int32_t M, int32_t N, int32_t K, const void* A, int32_t a_mn, const void* B,
+                          int32_t b_mn, float* C, void* cuda_stream) {
   g_err.clear();
-  if (M <= 0 || N <= 0 || K <= 0 || (K % 8) || !A || !B || !C)
-    return fail(JOLT_ERR_INVALID_ARG, "jolt_selftest_gemm_bf16: bad sizes or pointers");
+  if (M <= 0 || N <= 0 || K <= 0 || (K % 8) || !A || !B || !C || (a_mn && M % 8) || (b_mn && N % 8))
+    return fail(JOLT_ERR_INVALID_ARG, "%s: bad sizes or pointers", who);
   cudaStream_t s = (cudaStream_t)cuda_stream;
   TcGemmParams p;
   const uint64_t adims[3] = {(uint64_t)K, (uint64_t)M, 1}, astr[2] = {(uint64_t)K * 2, (uint64_t)K * M * 2};
   const uint64_t bdims[3] = {(uint64_t)K, (uint64_t)N, 1}, bstr[2] = {(uint64_t)K * 2, (uint64_t)K * N * 2};
-  if (!tc_map_bf16(&p.amap[0], A, 3, adims, astr) || !tc_map_bf16(&p.bmap[0], B, 3, bdims, bstr))
-    return fail(JOLT_ERR_INVALID_ARG, "jolt_selftest_gemm_bf16: tensor map rejected");
+  const bool aok = a_mn ? tc_map_bf16_mn(&p.amap[0], A, M, K, 1) : tc_map_bf16(&p.amap[0], A, 3, adims, astr);
+  const bool bok = b_mn ? tc_map_bf16_mn(&p.bmap[0], B, N, K, 1) : tc_map_bf16(&p.bmap[0], B, 3, bdims, bstr);
+  if (!aok || !bok) return fail(JOLT_ERR_INVALID_ARG, "%s: tensor map rejected", who);
+  if (a_mn) p.av.mode = VIEW_MN;
+  if (b_mn) p.bv.mode = VIEW_MN;
   p.na = p.nb = 1;
   p.M = M; p.N = N; p.KB = (K + 63) / 64;
   p.C = C; p.c_sm = N; p.c_sn = 1; p.c_sb = (int64_t)M * N;
@@ -1708,8 +1696,19 @@ JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, co
   if (e == cudaSuccess) e = cudaMemcpyAsync(&h, st, sizeof(h), cudaMemcpyDeviceToHost, s);
   cudaFreeAsync(st, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_selftest_gemm_bf16: %s", cudaGetErrorString(e));
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "%s: %s", who, cudaGetErrorString(e));
   return status_of(h);
+}
+}  // namespace
+
+JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const void* B,
+                                             float* C, void* cuda_stream) {
+  return selftest_gemm("jolt_selftest_gemm_bf16", M, N, K, A, 0, B, 0, C, cuda_stream);
+}
+
+JOLT_API jolt_status jolt_selftest_gemm_bf16_layout(int32_t M, int32_t N, int32_t K, const void* A, int32_t a_mn,
+                                                    const void* B, int32_t b_mn, float* C, void* cuda_stream) {
+  return selftest_gemm("jolt_selftest_gemm_bf16_layout", M, N, K, A, a_mn, B, b_mn, C, cuda_stream);
 }
 
 JOLT_API uint64_t jolt_launch_count(void) { return g_launches.load(); }

@@ -29,6 +29,7 @@ constexpr int kTile = 128;
 constexpr int kBK = 64;
 constexpr int kTileBytes = kTile * kBK * 2;   // 16 KB per operand part and stage
 constexpr uint32_t kMaxPoll = 1u << 22;
+constexpr uint32_t kMnHalf = 64 * kBK * 2;    // one 64-row half of an MN-major tile (8 KB)
 
 __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, int b, int& c0, int& c1, int& c2,
                                             int& c3) {
@@ -48,6 +49,9 @@ __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, i
     case VIEW_XT_PERHEAD:              // same map, batch b = i * H + h: rows d, K = t
       c0 = kb * kBK; c1 = row0; c2 = b % v.H; c3 = b / v.H;
       break;
+    case VIEW_MN:                      // map (rows, K, batch), rows contiguous
+      c0 = row0 + (b % v.H) * v.D; c1 = kb * kBK; c2 = b / v.H; c3 = 0;
+      break;
     default:                           // VIEW_ROWS_K: map (K, rows, batch), batch index b / H
       c0 = kb * kBK; c1 = row0; c2 = b / v.H; c3 = 0;
       break;
@@ -58,8 +62,15 @@ __device__ __forceinline__ void view_load(const TcView& v, const CUtensorMap* ma
                                           int row0, int kb, int b) {
   int c0, c1, c2, c3;
   view_coords(v, row0, kb, b, c0, c1, c2, c3);
-  if (v.mode == VIEW_ROWS_K) tma_load_3d(dst, map, bar, c0, c1, c2);
-  else tma_load_4d(dst, map, bar, c0, c1, c2, c3);
+  if (v.mode == VIEW_ROWS_K) {
+    tma_load_3d(dst, map, bar, c0, c1, c2);
+  } else if (v.mode == VIEW_MN) {
+    // two boxes of 64 rows x 64 k: the tile's MN-major halves, kMnHalf bytes apart
+    tma_load_3d(dst, map, bar, c0, c1, c2);
+    tma_load_3d(static_cast<uint8_t*>(dst) + kMnHalf, map, bar, c0 + 64, c1, c2);
+  } else {
+    tma_load_4d(dst, map, bar, c0, c1, c2, c3);
+  }
 }
 
 // bf16 parts of v at offset off: v = p0 + p1 + p2 (each remainder is exact in float32).
@@ -236,7 +247,8 @@ __global__ void __launch_bounds__(128 + 32 * kEpiWarps, 1) k_gemm_tc(const __gri
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc = idesc_bf16_f32(kTile, kTile);
+      const bool a_mn = p.av.mode == VIEW_MN, b_mn = p.bv.mode == VIEW_MN;
+      const uint32_t idesc = idesc_bf16_f32(kTile, kTile) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
       uint32_t g = 0;
       int i = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_v; t += gridDim.x, ++i) {
@@ -262,10 +274,14 @@ __global__ void __launch_bounds__(128 + 32 * kEpiWarps, 1) k_gemm_tc(const __gri
             const int ia = pa[q], ib = pb[q];
             const uint32_t abase = st + ia * kTileBytes;
             const uint32_t bbase = p.b_same ? st + ib * kTileBytes : st + (p.na + ib) * kTileBytes;
+            // K = 16 per MMA: 32 bytes along a K-major line, or 16 lines (two 8-line groups)
+            // of an MN-major tile
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
-              const uint64_t ad = desc_kmajor_sw128(abase + k * 32);
-              const uint64_t bd = desc_kmajor_sw128(bbase + k * 32);
+              const uint64_t ad = a_mn ? desc_mnmajor_sw128(abase + k * 2048, kMnHalf, 1024)
+                                       : desc_kmajor_sw128(abase + k * 32);
+              const uint64_t bd = b_mn ? desc_mnmajor_sw128(bbase + k * 2048, kMnHalf, 1024)
+                                       : desc_kmajor_sw128(bbase + k * 32);
               umma_bf16(d, ad, bd, idesc, (kb | q | k) != 0 ? 1u : 0u);
             }
           }
@@ -397,7 +413,8 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides) {
+static bool map_box(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                    uint32_t box1) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rank < 2 || rank > 5) return false;
   cuuint64_t gdim[5], gstr[4];
@@ -413,11 +430,22 @@ bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
   }
   if (reinterpret_cast<uintptr_t>(base) % 16) return false;
   box[0] = kBK;     // 64 bf16 = 128 bytes, the swizzle span
-  box[1] = kTile;   // 128 rows
+  box[1] = box1;
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gdim, gstr,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides) {
+  return map_box(map, base, rank, dims, strides, kTile);   // 64 K x 128 rows
+}
+
+bool tc_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t batch) {
+  if (rows <= 0 || K <= 0 || batch <= 0 || rows % 8) return false;
+  const uint64_t dims[3] = {(uint64_t)rows, (uint64_t)K, (uint64_t)batch};
+  const uint64_t str[2] = {(uint64_t)rows * 2, (uint64_t)(rows * K * 2)};
+  return map_box(map, base, 3, dims, str, kBK);   // 64 rows x 64 K
 }
 
 cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
@@ -426,7 +454,9 @@ cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
     return cudaErrorInvalidValue;
   for (int t = 0; t < p.npairs; ++t)
     if (p.pair_a[t] < 0 || p.pair_a[t] >= p.na || p.pair_b[t] < 0 || p.pair_b[t] >= p.nb) return cudaErrorInvalidValue;
-  if (p.b_same && (p.M > kTile || p.N > kTile || p.nb > p.na)) return cudaErrorInvalidValue;
+  if (p.b_same && (p.M > kTile || p.N > kTile || p.nb > p.na || p.av.mode == VIEW_MN)) return cudaErrorInvalidValue;
+  if ((p.av.mode == VIEW_MN && (p.av.D % 8 || p.av.H < 1)) || (p.bv.mode == VIEW_MN && (p.bv.D % 8 || p.bv.H < 1)))
+    return cudaErrorInvalidValue;
   if ((p.ps[0] || p.pt[0]) && p.c_batch_in > 0) return cudaErrorInvalidValue;
   const int stage_bytes = (p.na + (p.b_same ? 0 : p.nb)) * kTileBytes;
   const int ntn = (p.N + kTile - 1) / kTile, ntm = (p.M + kTile - 1) / kTile;

@@ -13,8 +13,11 @@ enum TcViewMode : int32_t {
   VIEW_ROWS_K = 0,        // 3-D map (K, rows, batch)
   VIEW_X_TOKENROWS = 1,   // 4-D map of X [L][H][T][D] as (D, T, H, L): rows = tokens, K = (head, feature)
   VIEW_XT_FEATROWS = 2,   // 4-D map of X^T [n][H][D][T] as (T, D, H, n): rows = (head, feature), K = tokens
-  VIEW_XT_PERHEAD = 3     // same map, batch index = layer-tensor * H + head: rows = features, K = tokens;
+  VIEW_XT_PERHEAD = 3,    // same map, batch index = layer-tensor * H + head: rows = features, K = tokens;
                           // any 4-D map (K, rows, H, n) is addressed this way
+  VIEW_MN = 4             // 3-D map (rows, K, batch) from tc_map_bf16_mn, rows contiguous: the operand
+                          // enters the MMA MN-major (two 64-row halves per tile); batch index b / H,
+                          // row offset (b % H) * D (D a multiple of 8). Not with b_same.
 };
 
 struct TcView {
@@ -55,6 +58,10 @@ struct TcGemmParams {
 // contiguous dimension; strides[i] is the byte stride of dims[i + 1]. False if the driver
 // entry point is missing or an alignment rule fails.
 bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides);
+
+// [batch][K][rows] bf16 (rows contiguous, rows a multiple of 8) as the 3-D map (rows, K, batch)
+// with a 64 x 64 box, for VIEW_MN operands.
+bool tc_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t batch);
 
 cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s);
 

@@ -122,7 +122,22 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B, f32 accumulator, both K-major.
+// Shared-memory matrix descriptor, MN-major operand with 128-byte swizzle (the image of TMA
+// boxes 64 rows wide in M or N): each 128-byte line holds 64 consecutive M (N) entries of one k,
+// lines of consecutive k follow each other, 8-line groups of k are `sbo` bytes apart and the
+// 64-entry blocks of M (N) `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;              // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;              // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, f32 accumulator, both K-major (bits 15 and
+// 16 select MN-major A and B).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                       // D format: f32
          | (1u << 7)                     // A format: bf16

@@ -30,7 +30,7 @@ EXPORTED = ["jolt_config_default", "jolt_plan", "jolt_plan_info", "jolt_encode",
             "jolt_rel_frob_error", "jolt_rel_frob_error_noalloc", "jolt_stream_status",
             "jolt_stream_info", "jolt_stream_to_host", "jolt_stream_from_host", "jolt_export_debug", "jolt_stream_destroy",
             "jolt_plan_destroy", "jolt_last_error", "jolt_profile_enable", "jolt_profile_report",
-            "jolt_launch_count", "jolt_selftest_gemm_bf16"]
+            "jolt_launch_count", "jolt_selftest_gemm_bf16", "jolt_selftest_gemm_bf16_layout"]
 
 
 class JoltError(RuntimeError):
@@ -78,6 +78,7 @@ def _load():
         "jolt_profile_report": (st, [ctypes.c_char_p, ctypes.POINTER(u64)]),
         "jolt_launch_count": (u64, []),
         "jolt_selftest_gemm_bf16": (st, [i32, i32, i32, vp, vp, vp, vp]),
+        "jolt_selftest_gemm_bf16_layout": (st, [i32, i32, i32, vp, i32, vp, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -253,3 +254,12 @@ def jolt_selftest_gemm_bf16(A, B, C, cuda_stream=None):
     M, K = A.shape
     N = B.shape[0]
     _check(_lib.jolt_selftest_gemm_bf16(M, N, K, _dptr(A), _dptr(B), _dptr(C), _stream_ptr(cuda_stream)))
+
+
+def jolt_selftest_gemm_bf16_layout(A, a_mn, B, b_mn, C, cuda_stream=None):
+    """C = A B^T on the tensor cores with either operand stored transposed: A is [M][K] (a_mn
+    false) or [K][M] (a_mn true), B is [N][K] or [K][N]; C [M][N] float32 (CUDA tensors)."""
+    M, K = (A.shape[1], A.shape[0]) if a_mn else A.shape
+    N = B.shape[1] if b_mn else B.shape[0]
+    _check(_lib.jolt_selftest_gemm_bf16_layout(M, N, K, _dptr(A), int(bool(a_mn)), _dptr(B), int(bool(b_mn)),
+                                               _dptr(C), _stream_ptr(cuda_stream)))

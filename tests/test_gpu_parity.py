@@ -251,6 +251,24 @@ def test_corrupt_stream_rejected(J):
 
 
 # ------------------------------------------------------------------ tensor-core GEMM building block
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (200, 136, 200), (256, 384, 128), (1024, 128, 128)])
+def test_tcgen05_gemm_transposed_operands(J, M, N, K, a_mn, b_mn):
+    """Operands stored [K][M] / [K][N] (MN-major in the MMA, as the analysis feeds its bases)
+    against float64, including ragged M, N and K."""
+    import torch
+    g = torch.Generator(device="cuda").manual_seed(M * 11 + N * 5 + K + 3 * a_mn + b_mn)
+    A = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    B = torch.randn((N, K), generator=g, device="cuda").to(torch.bfloat16)
+    C = torch.full((M, N), float("nan"), device="cuda", dtype=torch.float32)
+    J.jolt_selftest_gemm_bf16_layout(A.T.contiguous() if a_mn else A, a_mn, B.T.contiguous() if b_mn else B, b_mn, C)
+    ref = A.double() @ B.double().T
+    err = (C.double() - ref).abs().max().item()
+    scale = (A.double().abs() @ B.double().abs().T).max().item()
+    assert torch.isfinite(C).all()
+    assert err <= 1e-5 * scale, (err, scale)
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (200, 136, 200), (256, 128, 1024), (384, 256, 72)])
 def test_tcgen05_gemm_matches_float64(J, M, N, K):
     import torch
