@@ -161,17 +161,23 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
 // Right-looking Cholesky by 16-column blocks of the 128 x 128 array A (row stride LD): on
 // entry the lower triangle holds the matrix (identity on the padding, upper triangle zero),
 // on exit the blocks below the diagonal hold L (A = L L^T) and Dv the inverses of the
-// diagonal blocks of L (zero above their diagonal). The diagonal blocks then hold
-// T = L_kk^{-T} in their upper half (kKeepL = false) or L_kk in their lower half
-// (kKeepL = true). Warp 0 factors each diagonal block in registers (shuffle broadcasts,
-// CUDA's float64 reciprocal square root) and inverts it; the panel below is L21 = A21 L11^{-T}
-// (1 x 4 strips per thread); the trailing lower triangle takes the rank-16 update in 4 x 4
-// register tiles. A pivot not above floor_v is raised to it and sets *floored (pivots of
-// the n x n problem only). Called by all NT threads of the block.
+// diagonal blocks of L (zero above their diagonal). kKeepL = true: the diagonal blocks hold
+// L_kk in their lower half. kKeepL = false: the upper triangle holds X^T with X = L^{-1},
+// formed alongside the factorisation (right-looking block forward substitution of L X = I with
+// B = I kept transposed in the upper triangle: at step k, X_k = L_kk^{-1} B_k, then
+// B_i -= L_ik X_k below), through the scratch Xs [16][128].
+//  * Diagonal block: warp 0, lane i holding row i in registers. The next pivot is broadcast
+//    as soon as its lane has it, so that its reciprocal square root (CUDA's float64 rsqrt)
+//    overlaps the broadcast of column k (through Ls) and the row updates; then L_kk^{-1}.
+//  * Panel phase: L21 = A21 L_kk^{-T} (into Pt) and X_k (into Xs), one pass of 512 items.
+//  * Trailing phase: L21 back into A, the rank-16 update of the trailing lower triangle and
+//    the update of B below block k, in 4 x 4 register tiles; X_k back into the upper triangle.
+// A pivot not above floor_v is raised to it and sets *floored (pivots of the n x n problem
+// only). Called by all NT threads of the block.
 constexpr int kCholLD = kMaxN + 1;
 template <bool kKeepL, int NT = 512>
-__device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, double* Ls, double* Is, int n,
-                                            double floor_v, int* floored) {
+__device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, double* Ls, double* Is, double* Xs,
+                                            int n, double floor_v, int* floored) {
   constexpr int NP = kMaxN, LD = kCholLD, BS = 16, NBLK = NP / BS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int kb = 0; kb < NBLK; ++kb) {
@@ -184,31 +190,42 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
 #pragma unroll
       for (int j = 0; j < BS; ++j) a[j] = A[(k0 + i) * LD + k0 + j];
       bool fl = false;
-      // next pivot: lane k + 1 forms its updated diagonal from its own l_{k+1,k}, so the
-      // broadcast of the pivot does not wait for the column shuffles of step k
-      double dn = a[0];
+      double isv = 0.0;   // lane i: 1 / l_ii
+      double d = __shfl_sync(0xffffffffu, a[0], 0);
+      {
+        const bool low = !(d > floor_v);
+        fl = fl | (low & (k0 < n));
+        d = low ? floor_v : d;
+      }
+      double inv = rsqrt(d);
 #pragma unroll
       for (int k = 0; k < BS; ++k) {
-        double d = __shfl_sync(0xffffffffu, dn, k);
-        if (!(d > floor_v)) {
-          d = floor_v;
-          fl = fl || (k0 + k < n);
-        }
-        const double inv = rsqrt(d);
         const double lk = (i == k) ? d * inv : (i > k ? a[k] * inv : 0.0);
         a[k] = lk;
-        if (k + 1 < BS) dn = fma(-lk, lk, a[k + 1]);
-        if (i == k && lane < BS) Is[k] = inv;
-        // all broadcasts of column k first, then the updates: the shuffles overlap
+        isv = (i == k) ? inv : isv;
+        // lane k + 1's updated diagonal goes out first: the next pivot's square root does
+        // not wait for column k's broadcast
+        double dnext = 0.0;
+        if (k + 1 < BS) dnext = __shfl_sync(0xffffffffu, fma(-lk, lk, a[k + 1]), k + 1);
         double lj[BS];
+        if (lane < BS) Ls[k * BS + i] = lk;
+        __syncwarp();
 #pragma unroll
         for (int j = 1; j < BS; ++j)
-          if (j > k) lj[j] = __shfl_sync(0xffffffffu, lk, j);
+          if (j > k) lj[j] = Ls[k * BS + j];
 #pragma unroll
         for (int j = 1; j < BS; ++j)
           if (j > k && i >= j) a[j] = fma(-lk, lj[j], a[j]);
+        if (k + 1 < BS) {
+          const bool low = !(dnext > floor_v);
+          fl = fl | (low & (k0 + k + 1 < n));
+          d = low ? floor_v : dnext;
+          inv = rsqrt(d);
+        }
       }
+      __syncwarp();   // the column broadcasts are read; Ls takes the factor
       if (lane < BS) {
+        Is[i] = isv;
 #pragma unroll
         for (int j = 0; j < BS; ++j) Ls[i * (BS + 1) + j] = a[j];
       }
@@ -239,57 +256,117 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
     // panel L21 = A21 L11^{-T} into Pt only; thread = (group g of 4 columns, row), consecutive
     // lanes on consecutive rows. L11^{-1} is stored with zeros above its diagonal, so every
     // output is a full 16-term sum. A keeps A21 until the trailing phase copies L21 back.
-    for (int u = tid; u < 4 * rows; u += NT) {
-      const int g = u / rows, i = k0 + BS + (u - g * rows);
-      double v[BS];
+    // With the inverse: X_k[:, c] = L_kk^{-1} B_k[:, c] for c < k0 (thread = (group g of 4
+    // rows, column c)) and X_kk = L_kk^{-1} into Xs [m][c]; 4 rows + 4 k0 + 64 = 512 items.
+    const int nx = kKeepL ? 0 : 4 * k0 + 64;
+    for (int u = tid; u < 4 * rows + nx; u += NT) {
+      if (u < 4 * rows) {
+        const int g = u / rows, i = k0 + BS + (u - g * rows);
+        double v[BS];
 #pragma unroll
-      for (int m = 0; m < BS; ++m) v[m] = A[i * LD + k0 + m];
+        for (int m = 0; m < BS; ++m) v[m] = A[i * LD + k0 + m];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = 4 * g + jj;
-        double o = 0.0;
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = 4 * g + jj;
+          double o = 0.0;
 #pragma unroll
-        for (int m = 0; m < BS; ++m) o = fma(v[m], D[j * BS + m], o);
-        Pt[j * NP + i] = o;
+          for (int m = 0; m < BS; ++m) o = fma(v[m], D[j * BS + m], o);
+          Pt[j * NP + i] = o;
+        }
+      } else if (u < 4 * rows + 4 * k0) {
+        const int w = u - 4 * rows, g = w / k0, c = w - g * k0;
+        double bv[BS];
+#pragma unroll
+        for (int m = 0; m < BS; ++m) bv[m] = A[c * LD + k0 + m];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          double o = 0.0;
+#pragma unroll
+          for (int m = 0; m < BS; ++m) o = fma(D[(4 * g + rr) * BS + m], bv[m], o);
+          Xs[(4 * g + rr) * NP + c] = o;
+        }
+      } else {
+        const int w = u - 4 * rows - 4 * k0;   // 64 items: row w / 4, columns 4 (w % 4) ..
+        const int r = w >> 2, c4 = 4 * (w & 3);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) Xs[r * NP + k0 + c4 + cc] = D[r * BS + c4 + cc];
       }
     }
     __syncthreads();
-    // L21 back into A (the trailing tiles below read Pt and write only columns >= k0 + BS)
+    // L21 back into A (the trailing tiles below read Pt and write only columns >= k0 + BS);
+    // X_k back into the upper triangle (block row k of X^T's columns c < k0)
     for (int u = tid; u < BS * rows; u += NT) {
       const int j = u / rows, i = k0 + BS + (u - j * rows);
       A[i * LD + k0 + j] = Pt[j * NP + i];
     }
-    // trailing update of the lower triangle, 4 x 4 tiles (ti >= tj)
+    if (!kKeepL)
+      for (int u = tid; u < BS * k0; u += NT) {
+        const int m = u / k0, c = u - m * k0;
+        A[c * LD + k0 + m] = Xs[m * NP + c];
+      }
+    // trailing update of the lower triangle, 4 x 4 tiles (ti >= tj), then (inverse) the update
+    // B_i[:, c] -= L_ik X_k[:, c] of the rows below block k, c < k0 + 16, 4 x 4 tiles: a thread
+    // takes rows q, q + rows / 4, ... (consecutive lanes on consecutive rows) and 4 columns
     const int t4 = rows / 4;
     const int cnt = t4 * (t4 + 1) / 2;
-    for (int p = tid; p < cnt; p += NT) {
-      int ti = (int)((sqrtf(8.0f * (float)p + 1.0f) - 1.0f) * 0.5f);
-      while ((ti + 1) * (ti + 2) / 2 <= p) ++ti;
-      while (ti * (ti + 1) / 2 > p) --ti;
-      const int tj = p - ti * (ti + 1) / 2;
-      const int i0 = k0 + BS + 4 * ti, j0 = k0 + BS + 4 * tj;
-      double c[4][4];
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) c[ii][jj] = A[(i0 + ii) * LD + j0 + jj];
-#pragma unroll
-      for (int m = 0; m < BS; ++m) {
-        const double2 a01 = *reinterpret_cast<const double2*>(Pt + m * NP + i0);
-        const double2 a23 = *reinterpret_cast<const double2*>(Pt + m * NP + i0 + 2);
-        const double2 b01 = *reinterpret_cast<const double2*>(Pt + m * NP + j0);
-        const double2 b23 = *reinterpret_cast<const double2*>(Pt + m * NP + j0 + 2);
-        const double av[4] = {a01.x, a01.y, a23.x, a23.y};
-        const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+    const int q4 = rows / 4, cntb = kKeepL ? 0 : q4 * ((k0 + BS) / 4);
+    for (int p = tid; p < cnt + cntb; p += NT) {
+      if (p < cnt) {
+        int ti = (int)((sqrtf(8.0f * (float)p + 1.0f) - 1.0f) * 0.5f);
+        while ((ti + 1) * (ti + 2) / 2 <= p) ++ti;
+        while (ti * (ti + 1) / 2 > p) --ti;
+        const int tj = p - ti * (ti + 1) / 2;
+        const int i0 = k0 + BS + 4 * ti, j0 = k0 + BS + 4 * tj;
+        double c[4][4];
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) c[ii][jj] = fma(-av[ii], bv[jj], c[ii][jj]);
+          for (int jj = 0; jj < 4; ++jj) c[ii][jj] = A[(i0 + ii) * LD + j0 + jj];
+#pragma unroll
+        for (int m = 0; m < BS; ++m) {
+          const double2 a01 = *reinterpret_cast<const double2*>(Pt + m * NP + i0);
+          const double2 a23 = *reinterpret_cast<const double2*>(Pt + m * NP + i0 + 2);
+          const double2 b01 = *reinterpret_cast<const double2*>(Pt + m * NP + j0);
+          const double2 b23 = *reinterpret_cast<const double2*>(Pt + m * NP + j0 + 2);
+          const double av[4] = {a01.x, a01.y, a23.x, a23.y};
+          const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) c[ii][jj] = fma(-av[ii], bv[jj], c[ii][jj]);
+        }
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) A[(i0 + ii) * LD + j0 + jj] = c[ii][jj];
+      } else {
+        const int pb = p - cnt, q = pb % q4, c0 = 4 * (pb / q4);
+        int ri[4];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) ri[ii] = k0 + BS + q + ii * q4;
+        double acc[4][4];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = A[(c0 + cc) * LD + ri[ii]];
+#pragma unroll
+        for (int m = 0; m < BS; ++m) {
+          const double2 x01 = *reinterpret_cast<const double2*>(Xs + m * NP + c0);
+          const double2 x23 = *reinterpret_cast<const double2*>(Xs + m * NP + c0 + 2);
+          const double xv[4] = {x01.x, x01.y, x23.x, x23.y};
+          double lv[4];
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii) lv[ii] = Pt[m * NP + ri[ii]];
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = fma(-lv[ii], xv[cc], acc[ii][cc]);
+        }
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) A[(c0 + cc) * LD + ri[ii]] = acc[ii][cc];
       }
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) A[(i0 + ii) * LD + j0 + jj] = c[ii][jj];
     }
     __syncthreads();
   }
@@ -455,7 +532,7 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
     A[r * kCholLD + c] = v;
   }
   __syncthreads();
-  chol_blocks<true, NT>(A, Dv, Pt, Ls, Is, n, sigma * 1e-3, &floored);
+  chol_blocks<true, NT>(A, Dv, Pt, Ls, Is, nullptr, n, sigma * 1e-3, &floored);
   // M = L column-major (column j of M is column j of L), padding columns zero
 #pragma unroll
   for (int q = 0; q < PER; ++q) {
@@ -739,13 +816,11 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
 // With L = R^T (W = L L^T) and X = L^{-1}, R^{-1} = X^T. One shared 128 x 129 array holds L
 // in its lower triangle and T = X^T in its upper triangle; the diagonal blocks of L are not
 // needed once their inverses are formed, so T takes over their upper half.
-//  * Cholesky, right-looking by 16-column blocks: warp 0 factors the diagonal block in
-//    registers (shuffle broadcasts, CUDA's float64 reciprocal square root) and inverts it;
-//    the panel below is L21 = A21 L11^{-T} (1 x 4 strips per thread); the trailing lower
-//    triangle takes the rank-16 update in 4 x 4 register tiles. A pivot below a tiny floor
-//    is raised to it and flags ST_NOT_CONVERGED.
-//  * Inverse, right-looking block forward substitution of L X = I: X_k = L_kk^{-1} B_k, then
-//    B_i -= L_ik X_k for the block rows below (B = I initially, kept transposed in T).
+// The blocked Cholesky (chol_blocks) forms X alongside L: at block step k, X_k = L_kk^{-1} B_k
+// in the panel phase and B_i -= L_ik X_k for the block rows below in the trailing phase
+// (right-looking block forward substitution of L X = I, B = I initially, kept transposed in
+// T), so the inverse takes no barriers of its own. A pivot below a tiny floor is raised to it
+// and flags ST_NOT_CONVERGED.
 template <typename TW>
 __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW, double* Rinv,
                                                   int64_t sR, double shift, int32_t* status) {
@@ -756,6 +831,7 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   double* Pt = Dv + NBLK * BS * BS;        // BS x NP: the current panel, transposed
   double* Ls = Pt + BS * NP;               // BS x (BS + 1): the current diagonal factor
   double* Is = Ls + BS * (BS + 1);         // BS: 1 / L_kk diagonal
+  double* Xs = Is + BS;                    // BS x NP: the current block row of X
   __shared__ double tr_s;
   __shared__ int floored;
   const int tid = threadIdx.x, lane = tid & 31;
@@ -787,69 +863,8 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
     A[r * LD + c] = v;
   }
   __syncthreads();
-  chol_blocks<false>(A, Dv, Pt, Ls, Is, n, floor_v, &floored);
+  chol_blocks<false>(A, Dv, Pt, Ls, Is, Xs, n, floor_v, &floored);
   if (floored && tid == 0 && status) atomicOr(status, ST_NOT_CONVERGED);
-  // Inverse. B (transposed in the upper triangle, zero off the diagonal blocks) -> X^T.
-  for (int kb = 0; kb < NBLK; ++kb) {
-    const int k0 = kb * BS;
-    const double* D = Dv + kb * BS * BS;
-    // X_k[:, c] = L_kk^{-1} B_k[:, c] for the columns c < k0 (the diagonal block is already T);
-    // thread = (group g of 4 rows, column c): all reads, a barrier, then the in-place writes
-    {
-      const bool act = tid < 4 * k0;
-      const int g = act ? tid / k0 : 0, c = act ? tid - g * k0 : 0;
-      double o[4] = {0.0, 0.0, 0.0, 0.0};
-      if (act) {
-        double bv[BS];
-#pragma unroll
-        for (int m = 0; m < BS; ++m) bv[m] = A[c * LD + k0 + m];
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-          for (int m = 0; m < BS; ++m) o[rr] = fma(D[(4 * g + rr) * BS + m], bv[m], o[rr]);
-      }
-      __syncthreads();
-      if (act) {
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) A[c * LD + k0 + 4 * g + rr] = o[rr];
-      }
-    }
-    __syncthreads();
-    if (kb == NBLK - 1) break;
-    // B_i[:, c] -= L_ik X_k[:, c] for rows i below the block and columns c < k0 + BS; a thread
-    // takes rows q, q + rows/4, ... (consecutive lanes on consecutive rows) and 4 columns
-    const int rows = NP - k0 - BS, q4 = rows / 4, tc = (k0 + BS) / 4;
-    for (int p = tid; p < q4 * tc; p += 512) {
-      const int q = p % q4, c0 = 4 * (p / q4);
-      int ri[4];
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii) ri[ii] = k0 + BS + q + ii * q4;
-      double acc[4][4];
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = A[(c0 + cc) * LD + ri[ii]];
-      const bool diag = c0 >= k0;
-#pragma unroll
-      for (int m = 0; m < BS; ++m) {
-        double xv[4], lv[4];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          xv[cc] = diag ? D[m * BS + (c0 - k0) + cc] : A[(c0 + cc) * LD + k0 + m];
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) lv[ii] = A[ri[ii] * LD + k0 + m];
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = fma(-lv[ii], xv[cc], acc[ii][cc]);
-      }
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) A[(c0 + cc) * LD + ri[ii]] = acc[ii][cc];
-    }
-    __syncthreads();
-  }
   double* o = Rinv + (int64_t)blockIdx.x * sR;
   for (int e = tid; e < n * n; e += 512) {
     const int r = e / n, c = e - r * n;
@@ -902,8 +917,8 @@ static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, double*
   if (n <= 0 || n > kMaxN) return cudaErrorInvalidValue;
   if (batch <= 0) return cudaSuccess;
   // A (128 x 129), diagonal-block inverses (8 x 16 x 16), panel (16 x 128), diagonal factor
-  // (16 x 17) and its reciprocal diagonal (16), float64
-  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 8 * 256 + 16 * kMaxN + 16 * 17 + 16) * sizeof(double);
+  // (16 x 17), its reciprocal diagonal (16) and the current block row of X (16 x 128), float64
+  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 8 * 256 + 16 * kMaxN + 16 * 17 + 16 + 16 * kMaxN) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_chol_inv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
