@@ -175,6 +175,16 @@ __global__ void __launch_bounds__(512) k_jacobi(int n, const float* Ain, int64_t
 // A pivot not above floor_v is raised to it and sets *floored (pivots of the n x n problem
 // only). Called by all NT threads of the block.
 constexpr int kCholLD = kMaxN + 1;
+constexpr int kPanelLD = kMaxN + 8;   // row stride of the panel and X scratch: conflict-free MMA fragments
+
+// D += A B on the FP64 tensor-core MMA (m8n8k4, row.col): lane l holds A[l / 4][l % 4],
+// B[l % 4][l / 4] and D[l / 4][2 (l % 4) .. + 1] (fragments per the PTX ISA).
+__device__ __forceinline__ void dmma_f64(double& d0, double& d1, double a, double b) {
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+      : "+d"(d0), "+d"(d1)
+      : "d"(a), "d"(b));
+}
+
 template <bool kKeepL, int NT = 512>
 __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, double* Ls, double* Is, double* Xs,
                                             int n, double floor_v, int* floored) {
@@ -271,7 +281,7 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
           double o = 0.0;
 #pragma unroll
           for (int m = 0; m < BS; ++m) o = fma(v[m], D[j * BS + m], o);
-          Pt[j * NP + i] = o;
+          Pt[j * kPanelLD + i] = o;
         }
       } else if (u < 4 * rows + 4 * k0) {
         const int w = u - 4 * rows, g = w / k0, c = w - g * k0;
@@ -283,13 +293,13 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
           double o = 0.0;
 #pragma unroll
           for (int m = 0; m < BS; ++m) o = fma(D[(4 * g + rr) * BS + m], bv[m], o);
-          Xs[(4 * g + rr) * NP + c] = o;
+          Xs[(4 * g + rr) * kPanelLD + c] = o;
         }
       } else {
         const int w = u - 4 * rows - 4 * k0;   // 64 items: row w / 4, columns 4 (w % 4) ..
         const int r = w >> 2, c4 = 4 * (w & 3);
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) Xs[r * NP + k0 + c4 + cc] = D[r * BS + c4 + cc];
+        for (int cc = 0; cc < 4; ++cc) Xs[r * kPanelLD + k0 + c4 + cc] = D[r * BS + c4 + cc];
       }
     }
     __syncthreads();
@@ -297,76 +307,47 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
     // X_k back into the upper triangle (block row k of X^T's columns c < k0)
     for (int u = tid; u < BS * rows; u += NT) {
       const int j = u / rows, i = k0 + BS + (u - j * rows);
-      A[i * LD + k0 + j] = Pt[j * NP + i];
+      A[i * LD + k0 + j] = Pt[j * kPanelLD + i];
     }
     if (!kKeepL)
       for (int u = tid; u < BS * k0; u += NT) {
         const int m = u / k0, c = u - m * k0;
-        A[c * LD + k0 + m] = Xs[m * NP + c];
+        A[c * LD + k0 + m] = Xs[m * kPanelLD + c];
       }
-    // trailing update of the lower triangle, 4 x 4 tiles (ti >= tj), then (inverse) the update
-    // B_i[:, c] -= L_ik X_k[:, c] of the rows below block k, c < k0 + 16, 4 x 4 tiles: a thread
-    // takes rows q, q + rows / 4, ... (consecutive lanes on consecutive rows) and 4 columns
-    const int t4 = rows / 4;
-    const int cnt = t4 * (t4 + 1) / 2;
-    const int q4 = rows / 4, cntb = kKeepL ? 0 : q4 * ((k0 + BS) / 4);
-    for (int p = tid; p < cnt + cntb; p += NT) {
-      if (p < cnt) {
-        int ti = (int)((sqrtf(8.0f * (float)p + 1.0f) - 1.0f) * 0.5f);
-        while ((ti + 1) * (ti + 2) / 2 <= p) ++ti;
-        while (ti * (ti + 1) / 2 > p) --ti;
-        const int tj = p - ti * (ti + 1) / 2;
-        const int i0 = k0 + BS + 4 * ti, j0 = k0 + BS + 4 * tj;
-        double c[4][4];
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) c[ii][jj] = A[(i0 + ii) * LD + j0 + jj];
-#pragma unroll
-        for (int m = 0; m < BS; ++m) {
-          const double2 a01 = *reinterpret_cast<const double2*>(Pt + m * NP + i0);
-          const double2 a23 = *reinterpret_cast<const double2*>(Pt + m * NP + i0 + 2);
-          const double2 b01 = *reinterpret_cast<const double2*>(Pt + m * NP + j0);
-          const double2 b23 = *reinterpret_cast<const double2*>(Pt + m * NP + j0 + 2);
-          const double av[4] = {a01.x, a01.y, a23.x, a23.y};
-          const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
-#pragma unroll
-          for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) c[ii][jj] = fma(-av[ii], bv[jj], c[ii][jj]);
-        }
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) A[(i0 + ii) * LD + j0 + jj] = c[ii][jj];
+    // trailing update of the lower triangle, A22 -= L21 L21^T, and (inverse) of B below block
+    // k, B_i[:, c] -= L_ik X_k[:, c] for c < k0 + 16 (kept transposed: T[c][i] -= sum_m
+    // X_k[m][c] L21[i][m]), in 8 x 8 tiles on the FP64 MMA (four k = 4 steps over the panel
+    // width; warp w takes tiles w, w + NT / 32, ...). Diagonal tiles of A22 store their lower
+    // half only: the upper triangle belongs to T.
+    const int t8 = rows / 8, cnt = t8 * (t8 + 1) / 2, cntb = kKeepL ? 0 : t8 * ((k0 + BS) / 8);
+    const int fr = lane >> 2, fq = lane & 3;
+    for (int t = warp; t < cnt + cntb; t += NT / 32) {
+      const double* pa;
+      const double* pb;
+      double* cp;
+      bool diag = false;
+      if (t < cnt) {
+        int bi = (int)((sqrtf(8.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
+        while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
+        while (bi * (bi + 1) / 2 > t) --bi;
+        const int bj = t - bi * (bi + 1) / 2;
+        const int i0 = k0 + BS + 8 * bi, j0 = k0 + BS + 8 * bj;
+        pa = Pt + fq * kPanelLD + i0 + fr;         // A[r][q] = L21[i0 + r][q]
+        pb = Pt + fq * kPanelLD + j0 + fr;         // B[q][c] = L21[j0 + c][q]
+        cp = A + (i0 + fr) * LD + j0 + 2 * fq;
+        diag = bi == bj;
       } else {
-        const int pb = p - cnt, q = pb % q4, c0 = 4 * (pb / q4);
-        int ri[4];
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) ri[ii] = k0 + BS + q + ii * q4;
-        double acc[4][4];
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = A[(c0 + cc) * LD + ri[ii]];
-#pragma unroll
-        for (int m = 0; m < BS; ++m) {
-          const double2 x01 = *reinterpret_cast<const double2*>(Xs + m * NP + c0);
-          const double2 x23 = *reinterpret_cast<const double2*>(Xs + m * NP + c0 + 2);
-          const double xv[4] = {x01.x, x01.y, x23.x, x23.y};
-          double lv[4];
-#pragma unroll
-          for (int ii = 0; ii < 4; ++ii) lv[ii] = Pt[m * NP + ri[ii]];
-#pragma unroll
-          for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) acc[ii][cc] = fma(-lv[ii], xv[cc], acc[ii][cc]);
-        }
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) A[(c0 + cc) * LD + ri[ii]] = acc[ii][cc];
+        const int tb = t - cnt, cb = tb / t8, bi = tb - cb * t8;
+        const int c0 = 8 * cb, r0 = k0 + BS + 8 * bi;
+        pa = Xs + fq * kPanelLD + c0 + fr;         // A[c][q] = X_k[q][c0 + c]
+        pb = Pt + fq * kPanelLD + r0 + fr;         // B[q][i] = L21[r0 + i][q]
+        cp = A + (c0 + fr) * LD + r0 + 2 * fq;
       }
+      double d0 = cp[0], d1 = cp[1];
+#pragma unroll
+      for (int m0 = 0; m0 < BS; m0 += 4) dmma_f64(d0, d1, -pa[m0 * kPanelLD], pb[m0 * kPanelLD]);
+      if (!diag || 2 * fq <= fr) cp[0] = d0;
+      if (!diag || 2 * fq + 1 <= fr) cp[1] = d1;
     }
     __syncthreads();
   }
@@ -417,15 +398,9 @@ constexpr double kCheckCos2 = 1e-8;
 // shared memory of k_eig_psd: the Cholesky's arrays (A, diagonal inverses, panel, diagonal
 // factor and its reciprocals), which the column array, the Gram test's padded copy and the
 // norms and ranks overlay
-constexpr size_t kEigSmemDoubles = (size_t)kMaxN * kCholLD + 8 * 256 + 16 * kMaxN + 16 * 17 + 16;
+constexpr size_t kEigSmemDoubles = (size_t)kMaxN * kCholLD + 8 * 256 + 16 * kPanelLD + 16 * 17 + 16;
 static_assert((size_t)kMaxN * (kMaxN + 4) + kMaxN <= kEigSmemDoubles, "Gram test array (stride kMaxN + 4)");
 static_assert((size_t)kMaxN * kMaxN + kMaxN + kMaxN / 2 <= kEigSmemDoubles, "columns, norms, ranks");
-
-__device__ __forceinline__ void dmma_f64(double& d0, double& d1, double a, double b) {
-  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-      : "+d"(d0), "+d"(d1)
-      : "d"(a), "d"(b));
-}
 
 // The sweep's rotation criterion for a pair with dot product g and squared norms a, b: the
 // same power-of-two scale and float conversion as the angle computation.
@@ -503,7 +478,7 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
   double* A = ms;                                  // NP x kCholLD
   double* Dv = A + NP * kCholLD;
   double* Pt = Dv + NP * 16;
-  double* Ls = Pt + 16 * NP;
+  double* Ls = Pt + 16 * kPanelLD;
   double* Is = Ls + 16 * 17;
   __shared__ int floored;
   constexpr int PER = NP * NP / NT;
@@ -828,10 +803,10 @@ __global__ void __launch_bounds__(512) k_chol_inv(int n, const TW* W, int64_t sW
   extern __shared__ double dm[];
   double* A = dm;                          // NP x LD
   double* Dv = A + NP * LD;                // NBLK x BS x BS: L_kk^{-1} (lower, zero above)
-  double* Pt = Dv + NBLK * BS * BS;        // BS x NP: the current panel, transposed
-  double* Ls = Pt + BS * NP;               // BS x (BS + 1): the current diagonal factor
+  double* Pt = Dv + NBLK * BS * BS;        // BS x kPanelLD: the current panel, transposed
+  double* Ls = Pt + BS * kPanelLD;         // BS x (BS + 1): the current diagonal factor
   double* Is = Ls + BS * (BS + 1);         // BS: 1 / L_kk diagonal
-  double* Xs = Is + BS;                    // BS x NP: the current block row of X
+  double* Xs = Is + BS;                    // BS x kPanelLD: the current block row of X
   __shared__ double tr_s;
   __shared__ int floored;
   const int tid = threadIdx.x, lane = tid & 31;
@@ -918,7 +893,7 @@ static cudaError_t chol_inv_t(int batch, int n, const TW* W, int64_t sW, double*
   if (batch <= 0) return cudaSuccess;
   // A (128 x 129), diagonal-block inverses (8 x 16 x 16), panel (16 x 128), diagonal factor
   // (16 x 17), its reciprocal diagonal (16) and the current block row of X (16 x 128), float64
-  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 8 * 256 + 16 * kMaxN + 16 * 17 + 16 + 16 * kMaxN) * sizeof(double);
+  const size_t smem = ((size_t)kMaxN * (kMaxN + 1) + 8 * 256 + 16 * kPanelLD + 16 * 17 + 16 + 16 * kPanelLD) * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_chol_inv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_chol_inv<TW><<<batch, 512, smem, s>>>(n, W, sW, Rinv, sR, shift, status);
