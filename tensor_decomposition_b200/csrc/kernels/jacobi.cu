@@ -316,10 +316,11 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
       }
     // trailing update of the lower triangle, A22 -= L21 L21^T, and (inverse) of B below block
     // k, B_i[:, c] -= L_ik X_k[:, c] for c < k0 + 16 (kept transposed: T[c][i] -= sum_m
-    // X_k[m][c] L21[i][m]), in 8 x 8 tiles on the FP64 MMA (four k = 4 steps over the panel
-    // width; warp w takes tiles w, w + NT / 32, ...). Diagonal tiles of A22 store their lower
-    // half only: the upper triangle belongs to T.
-    const int t8 = rows / 8, cnt = t8 * (t8 + 1) / 2, cntb = kKeepL ? 0 : t8 * ((k0 + BS) / 8);
+    // X_k[m][c] L21[i][m]), on the FP64 MMA: warp w takes the 16 x 16 blocks w, w + NT / 32, ...
+    // as 2 x 2 tiles of 8 x 8 (four k = 4 steps over the panel width, two A and two B fragments
+    // per step). Diagonal blocks of A22 skip their upper tile and store the lower half of their
+    // diagonal tiles only: the upper triangle belongs to T.
+    const int t16 = rows / 16, cnt = t16 * (t16 + 1) / 2, cntb = kKeepL ? 0 : t16 * (kb + 1);
     const int fr = lane >> 2, fq = lane & 3;
     for (int t = warp; t < cnt + cntb; t += NT / 32) {
       const double* pa;
@@ -331,23 +332,46 @@ __device__ __forceinline__ void chol_blocks(double* A, double* Dv, double* Pt, d
         while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
         while (bi * (bi + 1) / 2 > t) --bi;
         const int bj = t - bi * (bi + 1) / 2;
-        const int i0 = k0 + BS + 8 * bi, j0 = k0 + BS + 8 * bj;
+        const int i0 = k0 + BS + 16 * bi, j0 = k0 + BS + 16 * bj;
         pa = Pt + fq * kPanelLD + i0 + fr;         // A[r][q] = L21[i0 + r][q]
         pb = Pt + fq * kPanelLD + j0 + fr;         // B[q][c] = L21[j0 + c][q]
         cp = A + (i0 + fr) * LD + j0 + 2 * fq;
         diag = bi == bj;
       } else {
-        const int tb = t - cnt, cb = tb / t8, bi = tb - cb * t8;
-        const int c0 = 8 * cb, r0 = k0 + BS + 8 * bi;
+        const int tb = t - cnt, cb = tb / t16, bi = tb - cb * t16;
+        const int c0 = 16 * cb, r0 = k0 + BS + 16 * bi;
         pa = Xs + fq * kPanelLD + c0 + fr;         // A[c][q] = X_k[q][c0 + c]
         pb = Pt + fq * kPanelLD + r0 + fr;         // B[q][i] = L21[r0 + i][q]
         cp = A + (c0 + fr) * LD + r0 + 2 * fq;
       }
-      double d0 = cp[0], d1 = cp[1];
+      // tile (u, v): rows 8 u .., columns 8 v ..; d[u][v][0..1]
+      double d[2][2][2];
 #pragma unroll
-      for (int m0 = 0; m0 < BS; m0 += 4) dmma_f64(d0, d1, -pa[m0 * kPanelLD], pb[m0 * kPanelLD]);
-      if (!diag || 2 * fq <= fr) cp[0] = d0;
-      if (!diag || 2 * fq + 1 <= fr) cp[1] = d1;
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const bool skip = diag && u < v;
+          d[u][v][0] = skip ? 0.0 : cp[8 * u * LD + 8 * v];
+          d[u][v][1] = skip ? 0.0 : cp[8 * u * LD + 8 * v + 1];
+        }
+#pragma unroll
+      for (int m0 = 0; m0 < BS; m0 += 4) {
+        const double a0 = -pa[m0 * kPanelLD], a1 = -pa[m0 * kPanelLD + 8];
+        const double b0 = pb[m0 * kPanelLD], b1 = pb[m0 * kPanelLD + 8];
+        dmma_f64(d[0][0][0], d[0][0][1], a0, b0);
+        dmma_f64(d[1][0][0], d[1][0][1], a1, b0);
+        dmma_f64(d[1][1][0], d[1][1][1], a1, b1);
+        if (!diag) dmma_f64(d[0][1][0], d[0][1][1], a0, b1);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          if (diag && u < v) continue;
+          const bool dt = diag && u == v;
+          if (!dt || 2 * fq <= fr) cp[8 * u * LD + 8 * v] = d[u][v][0];
+          if (!dt || 2 * fq + 1 <= fr) cp[8 * u * LD + 8 * v + 1] = d[u][v][1];
+        }
     }
     __syncthreads();
   }
