@@ -237,7 +237,6 @@ struct jolt_plan_s {
   float* Qfinal = nullptr;   // final sketch basis (one of Y / Y2)
   bool q_t = false;          // Qfinal stored as Q^T [l][T] (tensor-core path) instead of Q [T][l]
   bool use_tc = false;       // bf16 inputs with T % 8 == 0: contractions over X on tcgen05
-  __nv_bfloat16* XT = nullptr;       // [n][H][D][T]
   float* Cpart = nullptr;            // [n][H][D][D] per-head Gram partials
   __nv_bfloat16* QTp[3] = {nullptr, nullptr, nullptr};   // bf16 parts of a float32 basis [n][l][rows]
   __nv_bfloat16* QTp2[3] = {nullptr, nullptr, nullptr};  // second part set (CholeskyQR ping-pong)
@@ -346,11 +345,6 @@ bool map_x(CUtensorMap* m, const void* X, int L, int H, int T, int D) {
   const uint64_t dims[4] = {(uint64_t)D, (uint64_t)T, (uint64_t)H, (uint64_t)L};
   const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)T * D * 2, (uint64_t)H * T * D * 2};
   return tc_map_bf16(m, X, 4, dims, str);
-}
-bool map_xt(CUtensorMap* m, const void* XT, int n, int H, int T, int D) {
-  const uint64_t dims[4] = {(uint64_t)T, (uint64_t)D, (uint64_t)H, (uint64_t)n};
-  const uint64_t str[3] = {(uint64_t)T * 2, (uint64_t)D * T * 2, (uint64_t)H * D * T * 2};
-  return tc_map_bf16(m, XT, 4, dims, str);
 }
 bool map_rows(CUtensorMap* m, const void* P, int64_t K, int64_t rows, int64_t batch) {
   const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)batch};
@@ -663,7 +657,6 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     take(p->Pi32, (int64_t)D * D);
     take(p->Pib, (int64_t)D * D);
     if (p->use_tc) {
-      take(p->XT, n * HD * T);
       take(p->Cpart, n * H * D * D * k_chunks(T));   // per-head (and per K chunk) partials
       if (p->encoder == JOLT_ENC_SKETCH) {
         for (int i = 0; i < 3; ++i) take(p->QTp[i], n * l * std::max<int64_t>(T, HD));
@@ -779,27 +772,28 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
     CK(energy_table(ta, s));
     return JOLT_OK;
   }
-  CUtensorMap mx[2], mxt;
+  // Tensor maps of X [L][H][T][D] per kind: K-major tiles (rows = tokens, K = features) for
+  // the contractions over the features, MN-major tiles (rows = features, K = tokens) for those
+  // over the tokens, so X is read in place by both.
+  CUtensorMap mx[2], mxm[2];
   if (p->use_tc) {
-    {
-      PROF("transpose", s);
-      for (int k = 0; k < kinds; ++k)
-        CK(transpose_x((const __nv_bfloat16*)X[k], p->XT, L, H, T, D, k * L, s));
-    }
     for (int k = 0; k < kinds; ++k)
-      if (!map_x(&mx[k], X[k], L, H, T, D)) return fail(JOLT_ERR_CUDA, "tensor map of X rejected");
-    if (!map_xt(&mxt, p->XT, n, H, T, D)) return fail(JOLT_ERR_CUDA, "tensor map of X^T rejected");
+      if (!map_x(&mx[k], X[k], L, H, T, D) || !tc_map_bf16_x_mn(&mxm[k], X[k], L, H, T, D))
+        return fail(JOLT_ERR_CUDA, "tensor map of X rejected");
     PROF("feature_gram", s);
-    // per-head partials C_D[lt][h] = X_h^T X_h on the tensor cores, then a float64 sum over heads
-    TcGemmParams g;
-    g.amap[0] = mxt;
-    g.bmap[0] = mxt;
-    g.av.mode = g.bv.mode = VIEW_XT_PERHEAD;
-    g.av.H = g.bv.H = H;
-    g.av.D = g.bv.D = D;
+    // per-head partials C_D[lt][h] = X_h^T X_h on the tensor cores (one operand tile serves A
+    // and B), then a float64 sum over heads
     const int kc = k_chunks(T);
-    g.av.nch = g.bv.nch = kc;
-    g.av.ckb = g.bv.ckb = T / kc / 64;
+    TcGemmParams g;
+    g.amap[0] = mxm[0];
+    g.amap[1] = mxm[kinds - 1];
+    g.av.mode = VIEW_MN_XHEAD;
+    g.av.H = H;
+    g.av.D = D;
+    g.av.ksplit = kinds > 1 ? L * H : 0;   // (layer, head) batches of V after those of K
+    g.b_same = 1;
+    g.av.nch = kc;
+    g.av.ckb = T / kc / 64;
     g.M = D; g.N = D; g.KB = kc > 1 ? T / kc / 64 : (T + 63) / 64;
     g.C = p->Cpart; g.c_sm = D; g.c_sn = 1; g.c_sb = (int64_t)D * D;
     g.status = status;
@@ -892,17 +886,19 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       for (int it = 0; it < q; ++it) {
         {
           PROF("sketch_gemm", s);
-          // Z^T = (A^T Q)^T: rows (h, d), K = t; parts of Z^T [l][HD] and Z [HD][l]
+          // Z^T = (A^T Q)^T: rows (h, d), K = t (X read MN-major); parts of Z^T [l][HD]
+          const int kc = k_chunks(T);
           TcGemmParams g = tc_params();
-          g.amap[0] = mxt;
-          g.av.mode = VIEW_XT_FEATROWS;
+          g.amap[0] = mxm[0];
+          g.amap[1] = mxm[kinds - 1];
+          g.av.mode = VIEW_MN_XFEAT;
           g.av.D = D;
+          g.av.ksplit = kinds > 1 ? L : 0;
           for (int i = 0; i < 2; ++i)
             if (!map_rows(&g.bmap[i], sets[cur].s[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
           g.na = 1; g.nb = 2;
           g.M = (int)HD; g.N = l; g.KB = (T + 63) / 64;
           g.c_sm = 1; g.c_sn = HD; g.c_sb = (int64_t)l * HD;
-          const int kc = k_chunks(T);
           if (kc == 1) {
             g.C = nullptr;
             for (int i = 0; i < 3; ++i) g.ps[i] = sets[cur ^ 1].s[i];
@@ -939,20 +935,22 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
       }
       {
         PROF("sketch_gemm", s);
-        // B = Q^T A (l x HD): rows j, K = t; Q^T in three bf16 parts for float32 accuracy
+        // B = Q^T A (l x HD): rows j, K = t; Q^T in three bf16 parts for float32 accuracy, X
+        // read MN-major. B's bf16 parts [l][HD] (for B B^T, and MN-major for the per-head core)
+        // go to the part set that does not hold Q.
+        const PartSet& bs = sets[cur ^ 1];
+        const int kc = k_chunks(T);
         TcGemmParams g = tc_params();
         for (int i = 0; i < 3; ++i)
           if (!map_rows(&g.amap[i], sets[cur].s[i], T, l, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
-        g.bmap[0] = mxt;
-        g.bv.mode = VIEW_XT_FEATROWS;
+        g.bmap[0] = mxm[0];
+        g.bmap[1] = mxm[kinds - 1];
+        g.bv.mode = VIEW_MN_XFEAT;
         g.bv.D = D;
+        g.bv.ksplit = kinds > 1 ? L : 0;
         g.na = 3; g.nb = 1;
         g.M = l; g.N = (int)HD; g.KB = (T + 63) / 64;
         g.c_sm = HD; g.c_sn = 1; g.c_sb = (int64_t)l * HD;
-        // B's bf16 parts [l][HD] (for B B^T, and MN-major for the per-head core) go to the part
-        // set that does not hold Q
-        const PartSet& bs = sets[cur ^ 1];
-        const int kc = k_chunks(T);
         if (kc == 1) {
           g.C = p->Bm;
           for (int i = 0; i < 3; ++i) g.ps[i] = bs.s[i];

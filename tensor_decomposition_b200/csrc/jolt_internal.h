@@ -187,8 +187,6 @@ struct DecodeArgs {
 cudaError_t decode(const DecodeArgs& a, cudaStream_t s);
 
 // Layout helpers of the tensor-core path (layout.cu).
-cudaError_t transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int L, int H, int T, int D, int lt_base,
-                        cudaStream_t s);
 cudaError_t split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2,
                        cudaStream_t s);
 cudaError_t sum_heads(int n, int H, int64_t per, const float* part, float* out32, double* out64, cudaStream_t s);

@@ -31,12 +31,17 @@ constexpr int kTileBytes = kTile * kBK * 2;   // 16 KB per operand part and stag
 constexpr uint32_t kMaxPoll = 1u << 22;
 constexpr uint32_t kMnHalf = 64 * kBK * 2;    // one 64-row half of an MN-major tile (8 KB)
 
+__host__ __device__ __forceinline__ bool is_mn(int mode) {
+  return mode == VIEW_MN || mode == VIEW_MN_XFEAT || mode == VIEW_MN_XHEAD;
+}
+
 __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, int b, int& c0, int& c1, int& c2,
                                             int& c3) {
   if (v.nch > 1) {
     kb += (b % v.nch) * v.ckb;
     b /= v.nch;
   }
+  if (v.ksplit > 0 && b >= v.ksplit) b -= v.ksplit;
   switch (v.mode) {
     case VIEW_X_TOKENROWS: {           // map (D, T, H, L): rows t, K = (h, d)
       const int kpd = v.D / kBK;
@@ -52,6 +57,12 @@ __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, i
     case VIEW_MN:                      // map (rows, K, batch), rows contiguous
       c0 = row0 + (b % v.H) * v.D; c1 = kb * kBK; c2 = b / v.H; c3 = 0;
       break;
+    case VIEW_MN_XFEAT:                // map (D, T, H, L): rows (h, d), K = t
+      c0 = row0 % v.D; c1 = kb * kBK; c2 = row0 / v.D; c3 = b;
+      break;
+    case VIEW_MN_XHEAD:                // same map, batch b = layer * H + h: rows d, K = t
+      c0 = row0; c1 = kb * kBK; c2 = b % v.H; c3 = b / v.H;
+      break;
     default:                           // VIEW_ROWS_K: map (K, rows, batch), batch index b / H
       c0 = kb * kBK; c1 = row0; c2 = b / v.H; c3 = 0;
       break;
@@ -60,6 +71,7 @@ __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, i
 
 __device__ __forceinline__ void view_load(const TcView& v, const CUtensorMap* map, void* dst, uint64_t* bar,
                                           int row0, int kb, int b) {
+  if (v.ksplit > 0 && (v.nch > 1 ? b / v.nch : b) >= v.ksplit) ++map;   // the second source
   int c0, c1, c2, c3;
   view_coords(v, row0, kb, b, c0, c1, c2, c3);
   if (v.mode == VIEW_ROWS_K) {
@@ -68,6 +80,9 @@ __device__ __forceinline__ void view_load(const TcView& v, const CUtensorMap* ma
     // two boxes of 64 rows x 64 k: the tile's MN-major halves, kMnHalf bytes apart
     tma_load_3d(dst, map, bar, c0, c1, c2);
     tma_load_3d(static_cast<uint8_t*>(dst) + kMnHalf, map, bar, c0 + 64, c1, c2);
+  } else if (v.mode == VIEW_MN_XFEAT || v.mode == VIEW_MN_XHEAD) {
+    tma_load_4d(dst, map, bar, c0, c1, c2, c3);
+    tma_load_4d(static_cast<uint8_t*>(dst) + kMnHalf, map, bar, c0 + 64, c1, c2, c3);
   } else {
     tma_load_4d(dst, map, bar, c0, c1, c2, c3);
   }
@@ -247,7 +262,7 @@ __global__ void __launch_bounds__(128 + 32 * kEpiWarps, 1) k_gemm_tc(const __gri
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const bool a_mn = p.av.mode == VIEW_MN, b_mn = p.bv.mode == VIEW_MN;
+      const bool a_mn = is_mn(p.av.mode), b_mn = p.b_same ? a_mn : is_mn(p.bv.mode);
       const uint32_t idesc = idesc_bf16_f32(kTile, kTile) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
       uint32_t g = 0;
       int i = 0;
@@ -441,6 +456,13 @@ bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
   return map_box(map, base, rank, dims, strides, kTile);   // 64 K x 128 rows
 }
 
+bool tc_map_bf16_x_mn(CUtensorMap* map, const void* X, int64_t L, int64_t H, int64_t T, int64_t D) {
+  if (L <= 0 || H <= 0 || T <= 0 || D <= 0 || D % 8) return false;
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)T, (uint64_t)H, (uint64_t)L};
+  const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)(T * D * 2), (uint64_t)(H * T * D * 2)};
+  return map_box(map, X, 4, dims, str, kBK);   // 64 features x 64 tokens
+}
+
 bool tc_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t batch) {
   if (rows <= 0 || K <= 0 || batch <= 0 || rows % 8) return false;
   const uint64_t dims[3] = {(uint64_t)rows, (uint64_t)K, (uint64_t)batch};
@@ -454,8 +476,14 @@ cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s) {
     return cudaErrorInvalidValue;
   for (int t = 0; t < p.npairs; ++t)
     if (p.pair_a[t] < 0 || p.pair_a[t] >= p.na || p.pair_b[t] < 0 || p.pair_b[t] >= p.nb) return cudaErrorInvalidValue;
-  if (p.b_same && (p.M > kTile || p.N > kTile || p.nb > p.na || p.av.mode == VIEW_MN)) return cudaErrorInvalidValue;
+  if (p.b_same && (p.M > kTile || p.N > kTile || p.nb > p.na)) return cudaErrorInvalidValue;
+  if ((p.av.ksplit > 0 && p.na != 1) || (p.bv.ksplit > 0 && p.nb != 1) || p.av.ksplit < 0 || p.bv.ksplit < 0)
+    return cudaErrorInvalidValue;
   if ((p.av.mode == VIEW_MN && (p.av.D % 8 || p.av.H < 1)) || (p.bv.mode == VIEW_MN && (p.bv.D % 8 || p.bv.H < 1)))
+    return cudaErrorInvalidValue;
+  // X views: a tile's 128 rows lie within one head
+  if (((p.av.mode == VIEW_MN_XFEAT || p.av.mode == VIEW_MN_XHEAD) && (p.av.D % kTile || p.av.H < 1)) ||
+      ((p.bv.mode == VIEW_MN_XFEAT || p.bv.mode == VIEW_MN_XHEAD) && (p.bv.D % kTile || p.bv.H < 1)))
     return cudaErrorInvalidValue;
   if ((p.ps[0] || p.pt[0]) && p.c_batch_in > 0) return cudaErrorInvalidValue;
   const int stage_bytes = (p.na + (p.b_same ? 0 : p.nb)) * kTileBytes;

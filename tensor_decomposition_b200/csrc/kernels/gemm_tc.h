@@ -15,9 +15,13 @@ enum TcViewMode : int32_t {
   VIEW_XT_FEATROWS = 2,   // 4-D map of X^T [n][H][D][T] as (T, D, H, n): rows = (head, feature), K = tokens
   VIEW_XT_PERHEAD = 3,    // same map, batch index = layer-tensor * H + head: rows = features, K = tokens;
                           // any 4-D map (K, rows, H, n) is addressed this way
-  VIEW_MN = 4             // 3-D map (rows, K, batch) from tc_map_bf16_mn, rows contiguous: the operand
+  VIEW_MN = 4,            // 3-D map (rows, K, batch) from tc_map_bf16_mn, rows contiguous: the operand
                           // enters the MMA MN-major (two 64-row halves per tile); batch index b / H,
-                          // row offset (b % H) * D (D a multiple of 8). Not with b_same.
+                          // row offset (b % H) * D (D a multiple of 8)
+  VIEW_MN_XFEAT = 5,      // 4-D map of X [L][H][T][D] as (D, T, H, L) from tc_map_bf16_x_mn, MN-major:
+                          // rows = (head, feature) (a tile within one head: D a multiple of 128),
+                          // K = tokens, batch = layer
+  VIEW_MN_XHEAD = 6       // same map, batch index = layer * H + head: rows = features, K = tokens
 };
 
 struct TcView {
@@ -28,6 +32,9 @@ struct TcView {
   // 64-entry K blocks [chunk * ckb, chunk * ckb + ckb) of the view
   int32_t nch = 1;
   int32_t ckb = 0;
+  // Two sources: batch indices (after the K split) >= ksplit read the operand's next map
+  // (maps[i + 1]; single-part operands only) at index b - ksplit. 0: one source.
+  int32_t ksplit = 0;
 };
 
 struct TcGemmParams {
@@ -62,6 +69,10 @@ bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
 // [batch][K][rows] bf16 (rows contiguous, rows a multiple of 8) as the 3-D map (rows, K, batch)
 // with a 64 x 64 box, for VIEW_MN operands.
 bool tc_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t batch);
+
+// X [L][H][T][D] bf16 as the 4-D map (D, T, H, L) with a 64 x 64 box, for VIEW_MN_XFEAT and
+// VIEW_MN_XHEAD operands.
+bool tc_map_bf16_x_mn(CUtensorMap* map, const void* X, int64_t L, int64_t H, int64_t T, int64_t D);
 
 cudaError_t gemm_tc(int batch, const TcGemmParams& p, cudaStream_t s);
 

@@ -1,46 +1,10 @@
 // Layout helpers for the tensor-core path of the factor analysis:
-//  * the token-contiguous copy X^T[lt][h][d][t] of every layer-tensor, so that contractions
-//    over tokens read K-major tiles (the JoLT token unfolding, "A JoLT for the KV Cache",
-//    arXiv 2607.12550v2, Abstract, is contracted over tokens for the sketch passes A^T Q and
-//    Q^T A and for the feature Gram);
 //  * splitting a float32 array into up to three bf16 parts (x = p0 + p1 + p2 to ~2^-24);
 //  * summing per-head float32 Gram partials in float64.
 #include "../jolt_internal.h"
 
 namespace jolt {
 namespace {
-
-// One 64 x 64 tile of X[l][h] (T x D) -> X^T[base + l][h] (D x T): 16-byte loads of 8
-// features, a shared tile, 16-byte stores of 8 tokens. T and D are multiples of 8.
-constexpr int kTT = 64, kTS = kTT + 8;   // tile edge, shared row stride (bf16)
-__global__ void __launch_bounds__(256) k_transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int H, int T, int D,
-                                                     int lt_base) {
-  __shared__ __align__(16) __nv_bfloat16 tile[kTT * kTS];
-  const int lh = blockIdx.z;                   // l * H + h within this kind
-  const int t0 = blockIdx.x * kTT, d0 = blockIdx.y * kTT;
-  const __nv_bfloat16* src = X + (int64_t)lh * T * D;
-  const int l = lh / H, h = lh % H;
-  __nv_bfloat16* dst = XT + ((int64_t)(lt_base + l) * H + h) * D * T;
-#pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const int q = threadIdx.x + 256 * v, r = q >> 3, c = q & 7;   // token row r, 8-feature chunk c
-    const int t = t0 + r, d = d0 + 8 * c;
-    uint4 w = make_uint4(0, 0, 0, 0);
-    if (t < T && d < D) w = *reinterpret_cast<const uint4*>(src + (int64_t)t * D + d);
-    *reinterpret_cast<uint4*>(tile + r * kTS + 8 * c) = w;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int v = 0; v < 2; ++v) {
-    const int q = threadIdx.x + 256 * v, r = q >> 3, c = q & 7;   // feature row r, 8-token chunk c
-    const int d = d0 + r, t = t0 + 8 * c;
-    if (d >= D || t >= T) continue;
-    __align__(16) __nv_bfloat16 o[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) o[j] = tile[(8 * c + j) * kTS + r];
-    *reinterpret_cast<uint4*>(dst + (int64_t)d * T + t) = *reinterpret_cast<const uint4*>(o);
-  }
-}
 
 __global__ void k_split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1,
                              __nv_bfloat16* p2) {
@@ -115,15 +79,6 @@ int grid_for(int64_t n) {
 }
 
 }  // namespace
-
-cudaError_t transpose_x(const __nv_bfloat16* X, __nv_bfloat16* XT, int L, int H, int T, int D, int lt_base,
-                        cudaStream_t s) {
-  if (T % 8 || D % 8) return cudaErrorInvalidValue;
-  const dim3 g((T + kTT - 1) / kTT, (D + kTT - 1) / kTT, L * H);
-  k_transpose_x<<<g, 256, 0, s>>>(X, XT, H, T, D, lt_base);
-  note_launch();
-  return cudaGetLastError();
-}
 
 cudaError_t split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2,
                        cudaStream_t s) {
