@@ -33,13 +33,14 @@ constexpr int kThreads = 288;                 // 9 warps
 constexpr int kOpBytes = 128 * 128 * 2;       // one 128 x 128 bf16 operand (two swizzle atoms)
 constexpr int kCodesBytes = 128 * 128;        // codes of one tile, b <= 8
 constexpr uint32_t kMaxPoll = 1u << 22;
-// dynamic shared memory: B1 parts, B2 parts, A1, A2, codes
+// dynamic shared memory: B1 parts, B2 parts, A1, A2, two codes buffers
 constexpr int kOffB1 = 0;
 constexpr int kOffB2 = 2 * kOpBytes;
 constexpr int kOffA1 = 4 * kOpBytes;
 constexpr int kOffA2 = 5 * kOpBytes;
 constexpr int kOffCodes = 6 * kOpBytes;
-constexpr int kSmemBytes = kOffCodes + kCodesBytes + 1024;
+constexpr int kSmemBytes = kOffCodes + 2 * kCodesBytes + 1024;
+constexpr int kUtVec = 16;   // 16-byte U_T vectors per producer thread and tile (128 rows x r_t <= 128)
 
 // Byte offset of the 16-byte chunk `c16` (8 bf16, k = 8 c16 ..) of row `row` in a K-major
 // 128-row operand with 128-byte swizzling: 64-element atoms of 16 KB, rows of 128 bytes, the
@@ -85,7 +86,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
 
 __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
   extern __shared__ uint8_t smraw[];
-  __shared__ __align__(8) uint64_t bar_pro, bar_afull, bar_aempty, bar_codes;
+  __shared__ __align__(8) uint64_t bar_pro, bar_afull, bar_aempty, bar_codes[2];
   __shared__ __align__(8) uint64_t bar_accfull[2], bar_accempty[2];
   __shared__ uint32_t tmem_base;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -112,7 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
     mbar_init(&bar_pro, 1);
     mbar_init(&bar_afull, 128);
     mbar_init(&bar_aempty, 1);
-    mbar_init(&bar_codes, 1);
+    mbar_init(&bar_codes[0], 1);
+    mbar_init(&bar_codes[1], 1);
     for (int j = 0; j < 2; ++j) {
       mbar_init(&bar_accfull[j], 1);
       mbar_init(&bar_accempty[j], 128);
@@ -197,31 +199,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
 
   // ---------------------------------------------------------------- tiles of 128 rows
   if (warp >= 4 && warp < 8) {
-    // producers: U_T rows -> A1, unpacked cell centres -> A2
+    // producers: U_T rows -> A1, unpacked cell centres -> A2. The codes of tile it + 1 are
+    // copied (one bulk copy, two buffers) and its U_T rows loaded into registers while tile it
+    // is unpacked and multiplied.
     const int pt = tid - 128;
     const float inv2b = resid ? 1.0f / (float)(1 << b) : 0.0f;
     const float off2b = resid ? 1.0f - (float)(1 << b) : 0.0f;
     const uint32_t mask = resid ? (1u << b) - 1u : 0u;
-    const uint32_t* cw = reinterpret_cast<const uint32_t*>(sm + kOffCodes);
+    const int cpr = tucker ? rt / 8 : 0;   // 16-byte vectors per U_T row
+    auto issue_codes = [&](int it2) {
+      if (resid && pt == 0 && it2 < ntiles) {
+        const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
+        const uint32_t bytes = (uint32_t)(rows2 * rowbytes);
+        mbar_arrive_expect_tx(&bar_codes[it2 & 1], bytes);
+        bulk_load(sm + kOffCodes + (it2 & 1) * kCodesBytes, codes + ((int64_t)h * T + t2) * rowbytes, bytes,
+                  &bar_codes[it2 & 1]);
+      }
+    };
+    uint4 ut[kUtVec];
+    auto load_ut = [&](int it2) {
+      const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
+      const __nv_bfloat16* src = UT + (int64_t)t2 * rt;
+#pragma unroll
+      for (int q = 0; q < kUtVec; ++q) {
+        const int u = pt + 128 * q;
+        ut[q] = u < rows2 * cpr ? *reinterpret_cast<const uint4*>(src + (int64_t)(u / cpr) * rt + 8 * (u % cpr))
+                                : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    if (tucker) load_ut(0);
+    issue_codes(0);
     for (int it = 0; it < ntiles; ++it) {
       const int t0 = it * kTileRows, rows = min(kTileRows, T - t0);
-      if (resid && pt == 0) {
-        const uint32_t bytes = (uint32_t)(rows * rowbytes);
-        mbar_arrive_expect_tx(&bar_codes, bytes);
-        bulk_load(sm + kOffCodes, codes + ((int64_t)h * T + t0) * rowbytes, bytes, &bar_codes);
-      }
+      // the other codes buffer was last read by tile it - 1, whose unpack ended at the barrier
+      issue_codes(it + 1);
       wait_or_flag(&bar_aempty, (uint32_t)((it & 1) ^ 1), status);
       if (tucker) {
-        const int cpr = rt / 8;
-        const __nv_bfloat16* src = UT + (int64_t)t0 * rt;
-        for (int u = pt; u < rows * cpr; u += 128) {
-          const int r = u / cpr, c = u - r * cpr;
-          *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(r, c)) =
-              *reinterpret_cast<const uint4*>(src + (int64_t)r * rt + 8 * c);
+#pragma unroll
+        for (int q = 0; q < kUtVec; ++q) {
+          const int u = pt + 128 * q;
+          if (u < rows * cpr) *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(u / cpr, u % cpr)) = ut[q];
         }
+        if (it + 1 < ntiles) load_ut(it + 1);
       }
       if (resid) {
-        wait_or_flag(&bar_codes, (uint32_t)(it & 1), status);
+        wait_or_flag(&bar_codes[it & 1], (uint32_t)((it >> 1) & 1), status);
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(sm + kOffCodes + (it & 1) * kCodesBytes);
         for (int u = pt; u < rows * 16; u += 128) {
           const int r = u >> 4, c = u & 15;
           const int byte0 = r * rowbytes + c * b;   // eight codes = b bytes
@@ -241,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
       }
       fence_async_shared();
       mbar_arrive(&bar_afull);
-      // every producer is done with the codes buffer before the next tile's copy lands in it
+      // every producer is done with this tile's codes buffer before tile it + 2's copy lands in it
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
   } else if (warp == 8) {
@@ -272,13 +295,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
     // epilogue: TMEM lanes 32 warp .. 32 warp + 31 = rows of the tile
     const int layer = lt >> 1, kind = lt & 1;
     const int64_t obase = ((int64_t)layer * H + h) * T * 128;
+    // the row's scale for tile it + 1 is loaded while tile it is waited for and stored
+    auto load_scale = [&](int it2) {
+      const int t2 = it2 * kTileRows + 32 * warp + lane;
+      return (resid && t2 < T) ? __half2float(scales[(int64_t)h * T + t2]) : 0.0f;
+    };
+    float s_next = load_scale(0);
     for (int it = 0; it < ntiles; ++it) {
       const int buf = it & 1, use = it >> 1;
+      const float s = s_next;
+      if (it + 1 < ntiles) s_next = load_scale(it + 1);
       wait_or_flag(&bar_accfull[buf], (uint32_t)(use & 1), status);
       tc_fence_after();
       const int t = it * kTileRows + 32 * warp + lane;
       const bool valid = t < T;
-      const float s = (resid && valid) ? __half2float(scales[(int64_t)h * T + t]) : 0.0f;
       const uint32_t tb = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(buf * 256);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
