@@ -151,11 +151,14 @@ __global__ void k_relfrob_final(int nb, const double* part, double* out2) {
 }
 
 // Sign rule per column: the entry of largest magnitude (first on ties) becomes positive.
-// Block = 32 columns x 8 row lanes; the same block then flips U's and W's columns.
-__global__ void k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU, float* W,
-                           int w_rows, int64_t ldw, int64_t sW) {
-  __shared__ float bv[8][32];
-  __shared__ int bi[8][32];
+// Block = 32 columns x kSignLanes row lanes (a warp reads 128 contiguous bytes of a row); the
+// same block then flips U's and W's columns.
+constexpr int kSignLanes = 32;
+__global__ void __launch_bounds__(32 * kSignLanes) k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU,
+                                                             float* W, int w_rows, int64_t ldw, int64_t sW) {
+  constexpr int RL = kSignLanes;
+  __shared__ float bv[RL][32];
+  __shared__ int bi[RL][32];
   __shared__ float sgn[32];
   const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + cx;
@@ -163,17 +166,17 @@ __global__ void k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU
   float best = -1.0f;
   int bidx = 0x7fffffff;
   if (c < cols) {
-    // rows visited in increasing order (first wins ties), eight loads in flight per thread
+    // rows visited in increasing order (first wins ties), four loads in flight per thread
     int r = ry;
-    for (; r + 56 < rows; r += 64) {
-      float a[8];
+    for (; r + 3 * RL < rows; r += 4 * RL) {
+      float a[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) a[k] = fabsf(u[(int64_t)(r + 8 * k) * ldu + c]);
+      for (int k = 0; k < 4; ++k) a[k] = fabsf(u[(int64_t)(r + RL * k) * ldu + c]);
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (a[k] > best) { best = a[k]; bidx = r + 8 * k; }
+      for (int k = 0; k < 4; ++k)
+        if (a[k] > best) { best = a[k]; bidx = r + RL * k; }
     }
-    for (; r < rows; r += 8) {
+    for (; r < rows; r += RL) {
       const float a = fabsf(u[(int64_t)r * ldu + c]);
       if (a > best) { best = a; bidx = r; }
     }
@@ -182,7 +185,7 @@ __global__ void k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU
   bi[ry][cx] = bidx;
   __syncthreads();
   if (ry == 0) {
-    for (int k = 1; k < 8; ++k) {
+    for (int k = 1; k < RL; ++k) {
       const float v = bv[k][cx];
       const int i = bi[k][cx];
       if (v > best || (v == best && i < bidx)) { best = v; bidx = i; }
@@ -195,12 +198,12 @@ __global__ void k_sign_fix(int rows, int cols, float* U, int64_t ldu, int64_t sU
   if (c >= cols) return;
   const float sg = sgn[cx];
   if (sg > 0.0f) return;
-#pragma unroll 8
-  for (int r = ry; r < rows; r += 8) u[(int64_t)r * ldu + c] = -u[(int64_t)r * ldu + c];
+#pragma unroll 4
+  for (int r = ry; r < rows; r += RL) u[(int64_t)r * ldu + c] = -u[(int64_t)r * ldu + c];
   if (W) {
     float* w = W + (int64_t)blockIdx.y * sW;
-#pragma unroll 8
-    for (int r = ry; r < w_rows; r += 8) w[(int64_t)r * ldw + c] = -w[(int64_t)r * ldw + c];
+#pragma unroll 4
+    for (int r = ry; r < w_rows; r += RL) w[(int64_t)r * ldw + c] = -w[(int64_t)r * ldw + c];
   }
 }
 
@@ -278,7 +281,7 @@ cudaError_t relfrob_partial(const void* ref, const void* approx, uint64_t n, Ele
 cudaError_t sign_fix(int batch, int rows, int cols, float* U, int64_t ldu, int64_t sU, float* W,
                      int w_rows, int64_t ldw, int64_t sW, cudaStream_t s) {
   dim3 g((cols + 31) / 32, batch);
-  k_sign_fix<<<g, 256, 0, s>>>(rows, cols, U, ldu, sU, W, w_rows, ldw, sW);
+  k_sign_fix<<<g, 32 * kSignLanes, 0, s>>>(rows, cols, U, ldu, sU, W, w_rows, ldw, sW);
   note_launch();
   return cudaGetLastError();
 }
