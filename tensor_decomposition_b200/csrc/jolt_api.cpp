@@ -232,7 +232,7 @@ struct jolt_plan_s {
         *Wv = nullptr, *lamB = nullptr, *UT32 = nullptr, *UTf = nullptr, *P = nullptr, *Gmax = nullptr,
         *VT = nullptr, *lamT = nullptr;
   double *BB = nullptr, *CT = nullptr;   // sketch and token Grams, float64
-  double *Wg = nullptr, *Rinv = nullptr, *E = nullptr, *unit_err = nullptr, *Nbuf = nullptr;
+  double *Wg = nullptr, *Rinv = nullptr, *E = nullptr, *unit_err = nullptr, *Nbuf = nullptr, *Pbuf = nullptr;
   double *meas_part = nullptr, *meas_lt = nullptr;   // measured-b refinement
   float* Qfinal = nullptr;   // final sketch basis (one of Y / Y2)
   bool q_t = false;          // Qfinal stored as Q^T [l][T] (tensor-core path) instead of Q [T][l]
@@ -649,6 +649,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     take(p->E, 2 * (int64_t)L * p->ngrid);
     take(p->unit_err, 2 * (int64_t)p->G * p->nbits * p->ngrid);
     take(p->Nbuf, n * H * Rm * D);
+    take(p->Pbuf, n * D * D);
     if (cfg.measured_b) {
       take(p->meas_part, n * H * ((T + 255) / 256) * 9);
       take(p->meas_lt, n * 9);
@@ -1279,7 +1280,7 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, ui
     rm.meas_part = p->meas_part;
     {
       PROF("measure_b", s);
-      e = residual_encode(rm, p->Nbuf, std::max(p->R, 1), s);
+      e = residual_encode(rm, p->Pbuf, p->Nbuf, std::max(p->R, 1), s);
       if (e == cudaSuccess) e = measured_tables(da, p->meas_part, (sh.tokens + 255) / 256, p->meas_lt, s);
     }
     if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "measure_b: %s", cudaGetErrorString(e)));
@@ -1298,7 +1299,7 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, ui
   }
   {
     PROF("residual", s);
-    e = residual_encode(ra, p->Nbuf, std::max(p->R, 1), s);
+    e = residual_encode(ra, p->Pbuf, p->Nbuf, std::max(p->R, 1), s);
   }
   if (e != cudaSuccess) return bail(fail(JOLT_ERR_CUDA, "residual: %s", cudaGetErrorString(e)));
   p->last = st;

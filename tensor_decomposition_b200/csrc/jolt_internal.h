@@ -172,8 +172,9 @@ struct ResidualArgs {
   // stages instead of a D x D product
   int hadamard = 0;
 };
-// Nbuf: float64 scratch [n_lt][H][R][D] for N_h = (G_h U_D^T) Pi.
-cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStream_t s);
+// Pbuf: float64 scratch [n_lt][D][D] for P = U_D^T Pi; Nbuf: float64 scratch [n_lt][H][R][D]
+// for N_h = G_h P.
+cudaError_t residual_encode(const ResidualArgs& a, double* Pbuf, double* Nbuf, int R, cudaStream_t s);
 
 struct DecodeArgs {
   int n_lt, H, T, D;

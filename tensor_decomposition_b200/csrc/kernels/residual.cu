@@ -30,11 +30,45 @@ __device__ __forceinline__ const void* x_row_ptr(const ResidualArgs& a, int lt, 
              : (const void*)(reinterpret_cast<const float*>(a.X[kind]) + off);
 }
 
-// N_h = G_h (U_D^T Pi) in float64 for one (layer-tensor, head): P = U_D[:, :r_d]^T Pi (r_d x D)
-// in shared memory, then N_h = G_h P. Every product of stored values (bf16 x fp32) is exact in
-// float64; only the sums round.
-__global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf, int R) {
-  extern __shared__ double P_s[];                 // [r_d][D]
+// P = U_D[:, :r_d]^T Pi (r_d x D, float64) once per layer-tensor (with the Hadamard rotation,
+// which the residual coder applies itself, P = U_D^T). Thread = (row j, four columns e0 ..):
+// a chain of D fused multiply-adds in d order. Every product of stored values (bf16 x fp32) is
+// exact in float64; only the sums round.
+__global__ void __launch_bounds__(256) k_resid_p(ResidualArgs a, double* Pbuf) {
+  const int i = blockIdx.y;
+  const int lt = a.lt_ids[i];
+  const StreamMeta* m = a.meta;
+  const int rt = m->lt_rank[lt][0], rd = m->lt_rank[lt][1], b = m->lt_rank[lt][2];
+  if ((b == 0 && !a.measure) || rt == 0) return;
+  constexpr int D = kD, Q = kD / 4;
+  const __nv_bfloat16* UD = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UD]);
+  double* P = Pbuf + (int64_t)i * D * D;
+  for (int task = blockIdx.x * blockDim.x + threadIdx.x; task < rd * Q; task += gridDim.x * blockDim.x) {
+    const int j = task / Q, e0 = 4 * (task - j * Q);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    if (a.hadamard) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = (double)__bfloat162float(UD[(e0 + q) * rd + j]);
+    } else {
+      for (int d = 0; d < D; ++d) {
+        const double u = (double)__bfloat162float(UD[d * rd + j]);
+        const float4 pv = *reinterpret_cast<const float4*>(a.Pi + d * D + e0);
+        acc[0] = fma(u, (double)pv.x, acc[0]);
+        acc[1] = fma(u, (double)pv.y, acc[1]);
+        acc[2] = fma(u, (double)pv.z, acc[2]);
+        acc[3] = fma(u, (double)pv.w, acc[3]);
+      }
+    }
+    *reinterpret_cast<double2*>(P + j * D + e0) = make_double2(acc[0], acc[1]);
+    *reinterpret_cast<double2*>(P + j * D + e0 + 2) = make_double2(acc[2], acc[3]);
+  }
+}
+
+// N_h = G_h P in float64 for one (layer-tensor, head): P and G_h in shared memory, thread =
+// 4 x 4 block of N_h (rows k0 .., columns e0 ..), each entry a chain of r_d fused multiply-adds
+// in j order.
+__global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, const double* Pbuf, double* Nbuf, int R) {
+  extern __shared__ double P_s[];                 // [r_d][D], then G_h [r_t][r_d] as float
   const int h = blockIdx.x, i = blockIdx.y;
   const int lt = a.lt_ids[i];
   const StreamMeta* m = a.meta;
@@ -43,40 +77,35 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, double* Nbuf
   constexpr int D = kD, Q = kD / 4;
   const __nv_bfloat16* G = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_G]) +
                            (int64_t)h * rt * rd;
-  const __nv_bfloat16* UD = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UD]);
-  // P[j][e0 .. e0 + 3] = sum_d U_D[d][j] Pi[d][e0 ..]
-  for (int task = threadIdx.x; task < rd * Q; task += blockDim.x) {
-    const int j = task / Q, e0 = 4 * (task - j * Q);
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    if (a.hadamard) {
-      // M_h = G_h U_D^T: P = U_D^T (the rotation is applied by the residual coder)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[q] = (double)__bfloat162float(UD[(e0 + q) * rd + j]);
-    }
-    for (int d = 0; d < (a.hadamard ? 0 : D); ++d) {
-      const double u = (double)__bfloat162float(UD[d * rd + j]);
-      const float4 pv = *reinterpret_cast<const float4*>(a.Pi + d * D + e0);
-      acc[0] = fma(u, (double)pv.x, acc[0]);
-      acc[1] = fma(u, (double)pv.y, acc[1]);
-      acc[2] = fma(u, (double)pv.z, acc[2]);
-      acc[3] = fma(u, (double)pv.w, acc[3]);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) P_s[j * D + e0 + q] = acc[q];
-  }
+  float* G_s = reinterpret_cast<float*>(P_s + rd * D);
+  const double2* P = reinterpret_cast<const double2*>(Pbuf + (int64_t)i * D * D);
+  for (int u = threadIdx.x; u < rd * D / 2; u += blockDim.x) reinterpret_cast<double2*>(P_s)[u] = P[u];
+  for (int u = threadIdx.x; u < rt * rd; u += blockDim.x) G_s[u] = __bfloat162float(G[u]);
   __syncthreads();
-  // N_h[k][e0 ..] = sum_j G_h[k][j] P[j][e0 ..]
   double* N = Nbuf + (((int64_t)i * a.H + h) * R) * D;
-  for (int task = threadIdx.x; task < rt * Q; task += blockDim.x) {
-    const int k = task / Q, e0 = 4 * (task - k * Q);
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int j = 0; j < rd; ++j) {
-      const double g = (double)__bfloat162float(G[k * rd + j]);
+  for (int task = threadIdx.x; task < (rt / 4) * Q; task += blockDim.x) {
+    const int k0 = 4 * (task / Q), e0 = 4 * (task % Q);
+    double acc[4][4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[q] = fma(g, P_s[j * D + e0 + q], acc[q]);
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[r][q] = 0.0;
+    for (int j = 0; j < rd; ++j) {
+      const double2 p01 = *reinterpret_cast<const double2*>(P_s + j * D + e0);
+      const double2 p23 = *reinterpret_cast<const double2*>(P_s + j * D + e0 + 2);
+      const double pv[4] = {p01.x, p01.y, p23.x, p23.y};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const double g = (double)G_s[(k0 + r) * rd + j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[r][q] = fma(g, pv[q], acc[r][q]);
+      }
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) N[(int64_t)k * D + e0 + q] = acc[q];
+    for (int r = 0; r < 4; ++r) {
+      *reinterpret_cast<double2*>(N + (int64_t)(k0 + r) * D + e0) = make_double2(acc[r][0], acc[r][1]);
+      *reinterpret_cast<double2*>(N + (int64_t)(k0 + r) * D + e0 + 2) = make_double2(acc[r][2], acc[r][3]);
+    }
   }
 }
 
@@ -402,14 +431,17 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
 
 }  // namespace
 
-static size_t residual_prep_smem() { return (size_t)kD * kD * sizeof(double); }
+// P [r_d][D] float64 and G_h [r_t][r_d] float32 at the largest ranks
+static size_t residual_prep_smem() { return (size_t)kD * kD * sizeof(double) + (size_t)kD * kD * sizeof(float); }
 
-cudaError_t residual_encode(const ResidualArgs& a, double* Nbuf, int R, cudaStream_t s) {
+cudaError_t residual_encode(const ResidualArgs& a, double* Pbuf, double* Nbuf, int R, cudaStream_t s) {
   if (a.D != kD) return cudaErrorInvalidValue;
+  k_resid_p<<<dim3(kD * (kD / 4) / 256, a.n_lt), 256, 0, s>>>(a, Pbuf);
+  note_launch();
   const size_t sp = residual_prep_smem();
   cudaError_t e = cudaFuncSetAttribute(k_resid_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp);
   if (e != cudaSuccess) return e;
-  k_resid_prep<<<dim3(a.H, a.n_lt), 256, sp, s>>>(a, Nbuf, R);
+  k_resid_prep<<<dim3(a.H, a.n_lt), 256, sp, s>>>(a, Pbuf, Nbuf, R);
   note_launch();
   // Pi^T (float), -N^T (float64), the row-max tables, the two groups' A tiles (float) and codes
   const size_t sm = (size_t)kD * kPS * sizeof(float) + (size_t)kD * (R + 4) * sizeof(double) +
