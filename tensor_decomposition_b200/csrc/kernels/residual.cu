@@ -31,36 +31,51 @@ __device__ __forceinline__ const void* x_row_ptr(const ResidualArgs& a, int lt, 
 }
 
 // P = U_D[:, :r_d]^T Pi (r_d x D, float64) once per layer-tensor (with the Hadamard rotation,
-// which the residual coder applies itself, P = U_D^T). Thread = (row j, four columns e0 ..):
-// a chain of D fused multiply-adds in d order. Every product of stored values (bf16 x fp32) is
-// exact in float64; only the sums round.
-__global__ void __launch_bounds__(256) k_resid_p(ResidualArgs a, double* Pbuf) {
+// which the residual coder applies itself, P = U_D^T). Thread = 8 rows j0 .. x 4 columns e0 ..
+// (a warp spans the 128 columns of its 8 rows): per d one 16-byte load of Pi's row, one of
+// U_D's, 32 fused multiply-adds, each entry a chain in d order. Every product of stored values
+// (bf16 x fp32) is exact in float64; only the sums round.
+constexpr int kPRows = 8;
+__global__ void __launch_bounds__(128) k_resid_p(ResidualArgs a, double* Pbuf) {
   const int i = blockIdx.y;
   const int lt = a.lt_ids[i];
   const StreamMeta* m = a.meta;
   const int rt = m->lt_rank[lt][0], rd = m->lt_rank[lt][1], b = m->lt_rank[lt][2];
   if ((b == 0 && !a.measure) || rt == 0) return;
-  constexpr int D = kD, Q = kD / 4;
+  constexpr int D = kD;
+  const int j0 = kPRows * (4 * blockIdx.x + (threadIdx.x >> 5)), e0 = 4 * (threadIdx.x & 31);
+  if (j0 >= rd) return;   // rd is a multiple of 16
   const __nv_bfloat16* UD = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UD]);
   double* P = Pbuf + (int64_t)i * D * D;
-  for (int task = blockIdx.x * blockDim.x + threadIdx.x; task < rd * Q; task += gridDim.x * blockDim.x) {
-    const int j = task / Q, e0 = 4 * (task - j * Q);
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    if (a.hadamard) {
+  double acc[kPRows][4];
+  if (a.hadamard) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[q] = (double)__bfloat162float(UD[(e0 + q) * rd + j]);
-    } else {
-      for (int d = 0; d < D; ++d) {
-        const double u = (double)__bfloat162float(UD[d * rd + j]);
-        const float4 pv = *reinterpret_cast<const float4*>(a.Pi + d * D + e0);
-        acc[0] = fma(u, (double)pv.x, acc[0]);
-        acc[1] = fma(u, (double)pv.y, acc[1]);
-        acc[2] = fma(u, (double)pv.z, acc[2]);
-        acc[3] = fma(u, (double)pv.w, acc[3]);
+    for (int r = 0; r < kPRows; ++r)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[r][q] = (double)__bfloat162float(UD[(e0 + q) * rd + j0 + r]);
+  } else {
+#pragma unroll
+    for (int r = 0; r < kPRows; ++r)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[r][q] = 0.0;
+#pragma unroll 4
+    for (int d = 0; d < D; ++d) {
+      const float4 pv = *reinterpret_cast<const float4*>(a.Pi + d * D + e0);
+      const uint4 uw = *reinterpret_cast<const uint4*>(UD + d * rd + j0);   // U_D[d][j0 .. j0 + 7]
+      const uint32_t w[4] = {uw.x, uw.y, uw.z, uw.w};
+      const double p4[4] = {(double)pv.x, (double)pv.y, (double)pv.z, (double)pv.w};
+#pragma unroll
+      for (int r = 0; r < kPRows; ++r) {
+        const double u = (double)__uint_as_float((r & 1) ? (w[r >> 1] & 0xffff0000u) : (w[r >> 1] << 16));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[r][q] = fma(u, p4[q], acc[r][q]);
       }
     }
-    *reinterpret_cast<double2*>(P + j * D + e0) = make_double2(acc[0], acc[1]);
-    *reinterpret_cast<double2*>(P + j * D + e0 + 2) = make_double2(acc[2], acc[3]);
+  }
+#pragma unroll
+  for (int r = 0; r < kPRows; ++r) {
+    *reinterpret_cast<double2*>(P + (j0 + r) * D + e0) = make_double2(acc[r][0], acc[r][1]);
+    *reinterpret_cast<double2*>(P + (j0 + r) * D + e0 + 2) = make_double2(acc[r][2], acc[r][3]);
   }
 }
 
@@ -436,7 +451,7 @@ static size_t residual_prep_smem() { return (size_t)kD * kD * sizeof(double) + (
 
 cudaError_t residual_encode(const ResidualArgs& a, double* Pbuf, double* Nbuf, int R, cudaStream_t s) {
   if (a.D != kD) return cudaErrorInvalidValue;
-  k_resid_p<<<dim3(kD * (kD / 4) / 256, a.n_lt), 256, 0, s>>>(a, Pbuf);
+  k_resid_p<<<dim3(kD / (4 * kPRows), a.n_lt), 128, 0, s>>>(a, Pbuf);
   note_launch();
   const size_t sp = residual_prep_smem();
   cudaError_t e = cudaFuncSetAttribute(k_resid_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp);
