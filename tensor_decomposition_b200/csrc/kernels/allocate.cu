@@ -56,19 +56,23 @@ __global__ void k_energy_table(int H, int R, int D, int step, const float* Gmax,
   }
 }
 
-// The same table for the default grid (step 16, D = 128): warp w sums row block I = w, w + 8,
-// .. over every head and its 16 rows with coalesced float4 loads (lane l holds columns
-// 4l .. 4l + 3, so the 4 lanes 4J .. 4J + 3 cover column block J), in float64 and a fixed order.
-__global__ void __launch_bounds__(256) k_energy_table16(int H, int R, const float* Gmax, const double* xx,
-                                                        double* E, int ngrid, const int32_t* lt_ids) {
+// The same table for the default grid (step 16, D = 128): warp w sums row block I = w % 8 over
+// the heads h = w / 8, w / 8 + 4, .. (four head groups, 32 warps: four times the loads in
+// flight) and its 16 rows with coalesced float4 loads (lane l holds columns 4l .. 4l + 3, so the
+// 4 lanes 4J .. 4J + 3 cover column block J), in float64; the four head groups are then added in
+// a fixed order.
+constexpr int kEtGroups = 4;
+__global__ void __launch_bounds__(256 * kEtGroups) k_energy_table16(int H, int R, const float* Gmax, const double* xx,
+                                                                    double* E, int ngrid, const int32_t* lt_ids) {
   constexpr int D = kD, step = 16, nJ = D / step;
+  __shared__ double sp[kEtGroups][(kMaxN / step) * nJ];
   __shared__ double sb[(kMaxN / step) * nJ];
   const int lt = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nI = R / step;
+  const int nI = R / step, I = warp & 7, hg = warp >> 3;
   const float* g = Gmax + (int64_t)lt * H * R * D;
-  for (int I = warp; I < nI; I += 8) {
+  if (I < nI) {
     double acc = 0.0;
-    for (int h = 0; h < H; ++h) {
+    for (int h = hg; h < H; h += kEtGroups) {
       const float4* row = reinterpret_cast<const float4*>(g + ((int64_t)h * R + I * step) * D) + lane;
 #pragma unroll 4
       for (int i = 0; i < step; ++i) {
@@ -78,7 +82,14 @@ __global__ void __launch_bounds__(256) k_energy_table16(int H, int R, const floa
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if ((lane & 3) == 0) sb[I * nJ + (lane >> 2)] = acc;
+    if ((lane & 3) == 0) sp[hg][I * nJ + (lane >> 2)] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x < nI * nJ) {
+    double t = 0.0;
+#pragma unroll
+    for (int q = 0; q < kEtGroups; ++q) t += sp[q][threadIdx.x];
+    sb[threadIdx.x] = t;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -431,7 +442,7 @@ __global__ void k_pack_factors(PackArgs a) {
 
 cudaError_t energy_table(const TableArgs& a, cudaStream_t s) {
   if (a.step == 16 && a.D == kD && a.R <= kMaxN) {
-    k_energy_table16<<<a.n_lt, 256, 0, s>>>(a.H, a.R, a.Gmax, a.xx, a.E, a.ngrid, a.lt_ids);
+    k_energy_table16<<<a.n_lt, 256 * kEtGroups, 0, s>>>(a.H, a.R, a.Gmax, a.xx, a.E, a.ngrid, a.lt_ids);
     note_launch();
     return cudaGetLastError();
   }
