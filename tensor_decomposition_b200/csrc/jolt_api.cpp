@@ -426,7 +426,7 @@ int cholqr_tc(jolt_plan_s* p, int rows, PartSet* sets, int cur, int passes, int3
         *st = fail(JOLT_ERR_CUDA, "tensor map rejected");
         return cur;
       }
-    g.av.mode = VIEW_XT_PERHEAD;      // (K chunk, rows, chunk, i)
+    g.av.mode = VIEW_ROWS_K_HEAD;      // (K chunk, rows, chunk, i)
     g.av.H = nch;
     g.na = g.nb = 3;
     g.b_same = 1;
@@ -1051,7 +1051,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         g.status = status;
         for (int i = 0; i < 3; ++i)
           if (!map_kchunk(&g.amap[i], bsame[i], l, HD, 128, n)) return fail(JOLT_ERR_CUDA, "tensor map rejected");
-        g.av.mode = VIEW_XT_PERHEAD;      // (K, rows, chunk, i)
+        g.av.mode = VIEW_ROWS_K_HEAD;      // (K, rows, chunk, i)
         g.av.H = nch;
         g.na = g.nb = 3;
         g.b_same = 1;

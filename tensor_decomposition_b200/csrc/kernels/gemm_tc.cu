@@ -48,10 +48,7 @@ __device__ __forceinline__ void view_coords(const TcView& v, int row0, int kb, i
       c0 = (kb % kpd) * kBK; c1 = row0; c2 = kb / kpd; c3 = b;
       break;
     }
-    case VIEW_XT_FEATROWS:             // map (T, D, H, n): rows (h, d), K = t
-      c0 = kb * kBK; c1 = row0 % v.D; c2 = row0 / v.D; c3 = b;
-      break;
-    case VIEW_XT_PERHEAD:              // same map, batch b = i * H + h: rows d, K = t
+    case VIEW_ROWS_K_HEAD:             // map (K, rows, H, n), batch b = i * H + h
       c0 = kb * kBK; c1 = row0; c2 = b % v.H; c3 = b / v.H;
       break;
     case VIEW_MN:                      // map (rows, K, batch), rows contiguous

@@ -12,9 +12,8 @@ namespace jolt {
 enum TcViewMode : int32_t {
   VIEW_ROWS_K = 0,        // 3-D map (K, rows, batch)
   VIEW_X_TOKENROWS = 1,   // 4-D map of X [L][H][T][D] as (D, T, H, L): rows = tokens, K = (head, feature)
-  VIEW_XT_FEATROWS = 2,   // 4-D map of X^T [n][H][D][T] as (T, D, H, n): rows = (head, feature), K = tokens
-  VIEW_XT_PERHEAD = 3,    // same map, batch index = layer-tensor * H + head: rows = features, K = tokens;
-                          // any 4-D map (K, rows, H, n) is addressed this way
+  VIEW_ROWS_K_HEAD = 3,   // 4-D map (K, rows, H, n), batch index = i * H + h (e.g. K-chunked Grams:
+                          // (chunk entries, rows, chunk, i))
   VIEW_MN = 4,            // 3-D map (rows, K, batch) from tc_map_bf16_mn, rows contiguous: the operand
                           // enters the MMA MN-major (two 64-row halves per tile); batch index b / H,
                           // row offset (b % H) * D (D a multiple of 8)
