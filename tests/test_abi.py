@@ -103,3 +103,21 @@ def test_stream_from_host_rejects_corrupt_buffers(jolt):
     with pytest.raises(jolt.JoltError) as e:
         jolt.jolt_stream_from_host(bytes(v2), cuda_stream=0)
     assert e.value.status == 8
+
+
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn", [
+    (0, 128, 64, 0, 0),      # empty
+    (128, 128, 60, 0, 0),    # K not a multiple of 8
+    (100, 128, 64, 1, 0),    # transposed A needs M a multiple of 8
+    (128, 100, 64, 0, 1),    # transposed B needs N a multiple of 8
+])
+def test_gemm_selftest_rejects_bad_sizes(jolt, M, N, K, a_mn, b_mn):
+    """The layout self-test checks its sizes before any device call (no GPU needed)."""
+    lib = ctypes.CDLL(jolt.LIB_PATH)
+    f = lib.jolt_selftest_gemm_bf16_layout
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+                  ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert f(M, N, K, p, a_mn, p, b_mn, p, None) == 1
