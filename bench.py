@@ -62,9 +62,10 @@ def measured_peaks():
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled during the timed region.
 
-    In-process NVML queries every 100 ms from a background thread (a separate nvidia-smi
-    process polling the driver perturbed the timed kernels); nvidia-smi is the fallback when
-    the NVML binding is missing. Reads only, no GPU setting is changed."""
+    In-process NVML queries every 10 ms from a background thread (the timed region of the
+    default run lasts well under a second; a separate nvidia-smi process polling the driver
+    perturbed the timed kernels); nvidia-smi is the fallback when the NVML binding is missing.
+    Reads only, no GPU setting is changed."""
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
                ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
@@ -125,7 +126,7 @@ class ClockSampler:
                 self.samples.append((float(sm), float(smax), reasons))
             except Exception:
                 pass
-            if self.stop_ev.wait(0.1):
+            if self.stop_ev.wait(0.01):
                 break
 
     def _read_smi(self):
