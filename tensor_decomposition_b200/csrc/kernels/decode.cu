@@ -13,11 +13,12 @@
 //    (float32) are kept in shared memory as two bf16 parts each (hi + lo, ~2^-17 relative);
 //  * producers (warps 4-7) copy the tile's U_T rows and unpack its codes into bf16 cell
 //    centres (exact: odd integers below 2^8 over 2^b), both in the 128-byte-swizzled K-major
-//    layout; the codes arrive by one bulk copy per tile;
+//    layout; the codes arrive by one bulk copy per tile into two alternating buffers, and the
+//    next tile's copy and U_T rows (held in registers) are in flight while a tile is unpacked;
 //  * warp 8 issues tcgen05.mma: acc1 = U_T (M_h^T)_p^T and acc2 = Y_hat Pi_p^T over the
 //    parts p, double-buffered in Tensor Memory (4 x 128 columns);
 //  * the epilogue (warps 0-3, one row per thread) forms acc1 + s acc2 and stores bf16
-//    (round to nearest even) or float32.
+//    (round to nearest even) or float32; the row's next scale is loaded a tile ahead.
 // Every wait is bounded: a timeout sets ST_TIMEOUT in the stream status and the CTA runs on
 // to its end without hanging.
 #include "../jolt_internal.h"
