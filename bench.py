@@ -311,8 +311,8 @@ def config_dict(cfg, args):
 # while that file is unchanged (profiles/launch_list_c1_mistral7b_2x_sketch.md).
 NCU_TRAFFIC = {
     "jacobi": ("tensor_decomposition_b200/csrc/kernels/jacobi.cu", "0d23bba0b65e8d05", 9_553_024),
-    "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "9de1f842bf37c902", 179_766_784),
-    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "74e9f46a9cfaa1d6", 147_118_720),
+    "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "4a0da90ab5592dd5", 180_089_344),
+    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "35bee190c9fdc25f", 147_005_824),
 }
 
 
