@@ -330,7 +330,8 @@ def ncu_traffic(phase):
 
 
 def phase_models(cfg, plan_info, alloc, ratio, peaks):
-    """Algorithmic work of each traced phase per step (measurement section)."""
+    """Algorithmic work of each traced phase per step: flops or bytes the method needs, the
+    numerator of the roofline fraction."""
     H, T, D, L = cfg.heads, cfg.tokens, cfg.head_dim, cfg.layers
     n_lt = L * 2
     N = H * T * D                      # entries per layer-tensor

@@ -8,7 +8,7 @@ Notation: one layer-tensor X in R^{H x T x D} (heads x tokens x features). The t
 unfolding A = X_(2) in R^{T x HD} has A[t, h*D + d] = X[h, t, d]. U_T (T x r_t) and
 U_D (D x r_d) are shared by all heads; the core is G[h] = U_T^T X_h U_D (H x r_t x r_d).
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 * truncated HOSVD: each factor comes from the Gram of the original tensor, no HOOI sweeps;
   factors are computed once at the largest candidate rank and truncated to leading
   columns, so every candidate core is a leading block of one core G_max;

@@ -1,6 +1,6 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 CPU oracle.
 
-Tolerances (each stated where it is asserted, derived in the design doc):
+Tolerances (each stated where it is asserted, with the arithmetic behind it):
 * factors: principal angles < 1e-3 rad on the leading columns whose relative eigengap is
   at least 1e-3 (float32 eigensolvers on float64-accumulated Grams);
 * relative Frobenius error within 1% (relative) of the oracle's at the GPU's allocation;
