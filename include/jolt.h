@@ -28,7 +28,7 @@
  *  - A plan holds one workspace: encodes that share a plan must be issued on one CUDA
  *    stream (or otherwise serialised).
  *
- * This build supports head_dim == 128, batch of one sequence per stream, and token
+ * The library supports head_dim == 128, batch of one sequence per stream, and token
  * ranks r_t <= 112 (the sketch width r_t + oversample must stay <= 128).
  */
 #ifndef JOLT_H
@@ -56,7 +56,7 @@ typedef enum {
   JOLT_ERR_NONFINITE = 6,         /* NaN or Inf met in the input */
   JOLT_ERR_TIMEOUT = 7,           /* a bounded device wait gave up */
   JOLT_ERR_CORRUPT_STREAM = 8,    /* bad magic, version, size or CRC in a serialized stream */
-  JOLT_ERR_UNSUPPORTED = 9        /* valid request outside what this build implements */
+  JOLT_ERR_UNSUPPORTED = 9        /* valid request outside what the library implements */
 } jolt_status;
 
 typedef enum { JOLT_BF16 = 0, JOLT_F32 = 1 } jolt_dtype;

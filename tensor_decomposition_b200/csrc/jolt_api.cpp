@@ -518,7 +518,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   if (sh.layers <= 0 || sh.heads <= 0 || sh.tokens <= 0 || sh.head_dim <= 0)
     return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: non-positive dimension");
   if (sh.head_dim != kD)
-    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: head_dim %d unsupported (this build: 128)", sh.head_dim);
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: head_dim %d unsupported (supported: 128)", sh.head_dim);
   if (sh.layers > kMaxL) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: at most %d layers", kMaxL);
   if (sh.dtype != JOLT_BF16 && sh.dtype != JOLT_F32) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: dtype");
   if (num_groups <= 0 || num_groups > sh.layers || num_groups > kMaxGroups)

@@ -11,7 +11,7 @@
 
 namespace jolt {
 
-constexpr int kD = 128;            // head_dim supported by this build
+constexpr int kD = 128;            // the supported head_dim
 constexpr int kMaxL = 128;         // layers per stream
 constexpr int kMaxLT = 2 * kMaxL;  // layer-tensors per stream
 constexpr int kMaxGroups = 64;

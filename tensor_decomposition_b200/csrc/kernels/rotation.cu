@@ -4,7 +4,7 @@
 // "A JoLT for the KV Cache" (arXiv 2607.12550v2, Abstract) rotates the truncation residual
 // by "a random orthogonal rotation" before low-bit quantisation; the news summary of the
 // paper (aimodeling.com, English summary) calls it a Johnson-Lindenstrauss rotation that
-// whitens the residual. This build draws it as a Haar matrix: the Q factor of a D x D
+// whitens the residual. The library draws it as a Haar matrix: the Q factor of a D x D
 // standard-normal matrix with the signs of R's diagonal moved into Q (Mezzadri 2007).
 //
 // Generator (stated here because the CPU oracle implements it independently):
