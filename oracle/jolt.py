@@ -24,7 +24,8 @@ Readings taken where the pages are silent:
 * error model for the dual: exact truncation energy E(r_t, r_d) = ||X||^2 - ||G_lead||^2
   times phi(b), with phi(0) = 1 and phi(b) = kappa_D / (3 * 4^b), kappa_D = E[max_i z_i^2]
   for z ~ N(0, I_D): the whitened residual's quantisation error is treated as uniform
-  over a cell (the news summary's "close to an independent uniform distribution");
+  over a cell (the news summary describes the rotated residual as nearly independent and
+  uniformly distributed within a cell);
 * bytes per layer-tensor = 2 (T r_t + D r_d + H r_t r_d) + [b > 0] H T (D b / 8 + 2).
 """
 from __future__ import annotations

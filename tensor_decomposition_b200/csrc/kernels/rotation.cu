@@ -2,7 +2,7 @@
 // matrices of the FlashJoLT token factor, and the rotation Pi (Haar, or randomized Hadamard).
 //
 // "A JoLT for the KV Cache" (arXiv 2607.12550v2, Abstract) rotates the truncation residual
-// by "a random orthogonal rotation" before low-bit quantisation; the news summary of the
+// by a random orthogonal matrix before the low-bit quantisation; the news summary of the
 // paper (aimodeling.com, English summary) calls it a Johnson-Lindenstrauss rotation that
 // whitens the residual. The library draws it as a Haar matrix: the Q factor of a D x D
 // standard-normal matrix with the signs of R's diagonal moved into Q (Mezzadri 2007).
