@@ -30,6 +30,9 @@ sys.path.insert(0, ROOT)
 METRIC = "KV tokens/s encode+decode (Mistral-7B-shape, 2x); rel. Frobenius error"
 UNIT = "tokens/s"
 SEED = 42
+# Token-rank cap of the benchmarked plans (jolt_config.rt_max, the oracle's rt_cap): the method's
+# default grid reaches rank 256 on this workload, the kernels implement ranks up to 112.
+RT_MAX = 112
 
 
 def parse():
@@ -179,7 +182,7 @@ def oracle_sample_tokens_per_s(cfg, ratio, encoder, budget_s=12.0, max_s=30.0):
         kinds = 2 if cfg.has_v else 1
         plan = oj.Plan(L=1, H=cfg.heads, T=cfg.tokens, D=cfg.head_dim, has_v=cfg.has_v,
                        budget=budget_full * kinds // n_lt_full, num_groups=1, encoder=encoder,
-                       split_kv=cfg.split_kv, bits=tuple(cfg.bits))
+                       split_kv=cfg.split_kv, bits=tuple(cfg.bits), rt_cap=RT_MAX)
         t0 = time.perf_counter()
         st, _ = oj.encode(plan, K, V, SEED)
         oj.decode(st)
@@ -236,6 +239,7 @@ def in_codec_baselines(J, cfg, K, V, budget, encoder, steps=5, warmup=2):
     def run(name, bits, factors, bud, measured_b=0, rotation=0):
         c = J.jolt_config_default()
         c.encoder = encoder
+        c.rt_max = RT_MAX
         c.split_kv_budget = int(cfg.split_kv)
         c.bits_mask = sum(1 << b for b in bits)
         c.factors = factors
@@ -299,7 +303,7 @@ def config_dict(cfg, args):
                         f"{cfg.groups} layer groups, separate K/V budgets, {args.encoder} token factor",
             "layers": cfg.layers, "kv_heads": cfg.heads, "tokens": cfg.tokens, "head_dim": cfg.head_dim,
             "kinds": "K+V" if cfg.has_v else "K", "ratio": args.ratio, "encoder": args.encoder,
-            "groups": cfg.groups, "seq_per_gpu": 1,
+            "groups": cfg.groups, "seq_per_gpu": 1, "rt_max": RT_MAX,
             "l2": "inputs larger than L2 (K+V bf16 = 134 MB > 126 MB L2), no flush",
             "codec_seed": "fixed across steps: the seed-derived rotation and sketch matrices are built once per plan"}
 
@@ -394,6 +398,7 @@ def main():
     budget = synth.kv.budget_bytes(cfg, args.ratio)
     c = J.jolt_config_default()
     c.encoder = J.JOLT_ENC_SKETCH if args.encoder == "sketch" else J.JOLT_ENC_EXACT
+    c.rt_max = RT_MAX
     c.split_kv_budget = int(cfg.split_kv)
     plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, budget,
                        cfg.groups, c)

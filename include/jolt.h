@@ -28,8 +28,11 @@
  *  - A plan holds one workspace: encodes that share a plan must be issued on one CUDA
  *    stream (or otherwise serialised).
  *
- * The library supports head_dim == 128, batch of one sequence per stream, and token
- * ranks r_t <= 112 (the sketch width r_t + oversample must stay <= 128).
+ * The library supports head_dim == 128 and a batch of one sequence per stream. The candidate
+ * token ranks run to R = min(T, H*D, byte_budget / (layer-tensors * 2T)), at most 256 for the
+ * randomized-SVD encoder and at most jolt_config.rt_max when that is set; the kernels implement
+ * R <= 112 (sketch width R + oversample <= 128), and jolt_plan refuses a larger R with
+ * JOLT_ERR_UNSUPPORTED (set rt_max <= 112).
  */
 #ifndef JOLT_H
 #define JOLT_H
@@ -76,7 +79,8 @@ typedef struct {
   int32_t oversample;        /* sketch oversampling p (16) */
   int32_t power_iters;       /* sketch power iterations q (1) */
   int32_t rank_step;         /* candidate ranks are multiples of this (16) */
-  int32_t rt_max;            /* cap on the token rank; 0 = 112 */
+  int32_t rt_max;            /* cap on the candidate token ranks; 0 = none beyond the grid's own
+                                (see the preamble); plans need R <= 112 */
   uint32_t bits_mask;        /* bit b set => residual bit-width b allowed (0x1FF = 0..8) */
   int32_t split_kv_budget;   /* 0: one budget pool for K and V; 1: half the budget each */
   int32_t max_jacobi_sweeps; /* eigensolver sweep limit (30) */
@@ -128,6 +132,7 @@ JOLT_API void jolt_config_default(jolt_config* cfg);
  * cfg: NULL for defaults.
  * Errors: INVALID_ARG (non-positive sizes, head_dim != 128, groups > layers, bad options),
  *   BUDGET_INFEASIBLE (the cheapest allowed choice of every group exceeds the budget),
+ *   UNSUPPORTED (the candidate grid's largest token rank exceeds 112, see the preamble),
  *   OOM, CUDA. On success *out owns device workspace until jolt_plan_destroy.
  */
 JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, int32_t num_groups,
@@ -182,7 +187,9 @@ JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, ui
  *   Set-up: the first call on each device looks up the array's device address (with that
  *   device current) and keeps it; make that first call before any stream capture. The call
  *   synchronises `cuda_stream`. The array is shared by every caller on a device: overlapping
- *   calls (other threads, or other streams) race on it and may return wrong values.
+ *   calls (other threads, or other streams) race on it and may return wrong values. The kept
+ *   address belongs to the device context in which it was looked up: after cudaDeviceReset (or
+ *   any teardown of the primary context) later calls of this entry point are invalid.
  */
 #define JOLT_REL_FROB_NOALLOC_MAX_N (1ULL << 62)
 JOLT_API jolt_status jolt_rel_frob_error_noalloc(const void* ref, const void* approx, uint64_t n,
@@ -225,10 +232,13 @@ JOLT_API jolt_status jolt_export_debug(jolt_stream_t stream, int32_t what, int32
  * jolt_profile_report synchronises the device, writes a JSON object
  * {"phase": {"calls": n, "launches": k, "total_ms": t}, ...} (NUL-terminated; buf NULL queries
  * *len) and clears the records. jolt_launch_count returns the number of kernels this library
- * has launched since it was loaded. */
+ * has launched since it was loaded; jolt_alloc_count the number of device allocations it has
+ * requested (plan workspaces, stream bodies, scratch), whether served by the driver or by the
+ * library's memory pool. */
 JOLT_API jolt_status jolt_profile_enable(int32_t on);
 JOLT_API jolt_status jolt_profile_report(char* buf, uint64_t* len);
 JOLT_API uint64_t jolt_launch_count(void);
+JOLT_API uint64_t jolt_alloc_count(void);
 
 /* jolt_selftest_gemm_bf16 - C = A B^T on the tensor cores (tcgen05.mma with TMA tile loads),
  * the building block of the factor analysis, exposed so its numerics can be tested alone.

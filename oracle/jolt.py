@@ -39,7 +39,11 @@ from .numerics import (round_bf16, round_fp16_sat, round_f32, haar_rotation, rot
                        sketch_matrix)
 
 RANK_STEP = 16
-RT_CAP = 112
+# Largest token rank on the grid of the randomized-SVD encoder. The pages fix no grid; the reading
+# taken: ranks run to min(T, HD, budget per layer-tensor / (2T)) (a larger token factor alone
+# would exceed the layer-tensor's share of the budget), and the FlashJoLT sketch, which exists for
+# long contexts, stops at 256 columns before oversampling. The exact encoder has no extra cap.
+SKETCH_RT_CAP = 256
 OVERSAMPLE = 16
 POWER_ITERS = 1
 KINDS = 2          # layer-tensor index lt = layer * 2 + kind (kind 0 = K, 1 = V)
@@ -58,9 +62,12 @@ def layer_bytes(H: int, T: int, D: int, rt: int, rd: int, b: int) -> int:
     return tucker + resid
 
 
-def rt_max(H: int, T: int, D: int, budget_per_lt: int, step: int, cap: int) -> int:
-    """Largest token rank on the grid: min(T, HD, budget / (2T), cap), rounded down to `step`."""
-    r = min(T, H * D, budget_per_lt // (2 * T), cap)
+def rt_max(H: int, T: int, D: int, budget_per_lt: int, step: int, cap: int | None) -> int:
+    """Largest token rank on the grid: min(T, HD, budget / (2T), cap), rounded down to `step`
+    (`cap` None: no cap beyond the first three)."""
+    r = min(T, H * D, budget_per_lt // (2 * T))
+    if cap is not None:
+        r = min(r, cap)
     return max(0, r - r % step)
 
 
@@ -346,7 +353,7 @@ class Plan:
     num_groups: int
     encoder: str = "exact"
     rank_step: int = RANK_STEP
-    rt_cap: int = RT_CAP
+    rt_cap: int | None = None  # None: the reading (SKETCH_RT_CAP for the sketch, none for exact)
     oversample: int = OVERSAMPLE
     power_iters: int = POWER_ITERS
     bits: tuple = tuple(range(9))
@@ -368,8 +375,14 @@ class Plan:
             return [((0,), bk), ((1,), self.budget - bk)]
         return [(self.kinds(), self.budget)]
 
+    def cap(self):
+        """Token-rank cap: an explicit `rt_cap`, else the reading's (256 for the sketch)."""
+        if self.rt_cap is not None:
+            return self.rt_cap
+        return SKETCH_RT_CAP if self.encoder == "sketch" else None
+
     def R(self):
-        return rt_max(self.H, self.T, self.D, self.budget // self.n_lt(), self.rank_step, self.rt_cap)
+        return rt_max(self.H, self.T, self.D, self.budget // self.n_lt(), self.rank_step, self.cap())
 
     def grid(self):
         return rank_grid(self.R(), self.D, self.rank_step)

@@ -173,7 +173,20 @@ constexpr int kPoolDevices = 64;
 std::mutex g_pool_mu;
 cudaMemPool_t g_pools[kPoolDevices] = {};
 
+// Device allocations requested by the library (read through jolt_alloc_count).
+std::atomic<uint64_t> g_allocs{0};
+
+cudaError_t dev_malloc(void** ptr, size_t bytes) {
+  g_allocs.fetch_add(1, std::memory_order_relaxed);
+  return cudaMalloc(ptr, bytes);
+}
+template <typename T>
+cudaError_t dev_malloc(T** ptr, size_t bytes) {
+  return dev_malloc(reinterpret_cast<void**>(ptr), bytes);
+}
+
 cudaError_t pool_malloc(void** ptr, size_t bytes, cudaStream_t s) {
+  g_allocs.fetch_add(1, std::memory_order_relaxed);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -550,14 +563,25 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   for (int k = 0; k < kinds; ++k)
     for (int l = 0; l < L; ++l) p->lt_ids.push_back(2 * l + k);
   const int64_t per_lt = (int64_t)(byte_budget / (uint64_t)p->n_lt);
-  int cap = 112;
-  if (cfg.rt_max > 0) cap = std::min(cap, (int)cfg.rt_max);
-  if (cfg.factors == 0) cap = 0;   // residual only: the grid is the single point r_t = r_d = 0
-  int64_t R = std::min<int64_t>({(int64_t)T, (int64_t)H * D, per_lt / (2 * (int64_t)T), (int64_t)cap});
-  R -= R % p->step;
-  p->R = (int)std::max<int64_t>(0, R);
   int enc = cfg.encoder;
   if (enc == JOLT_ENC_AUTO) enc = T <= 1024 ? JOLT_ENC_EXACT : JOLT_ENC_SKETCH;
+  // Largest token rank of the candidate grid: min(T, HD, budget per layer-tensor / (2T)) (a
+  // larger token factor alone would exceed the layer-tensor's share of the budget), at most
+  // kSketchRankCap for the randomized-SVD encoder, and at most rt_max when the caller sets it.
+  int64_t cap = enc == JOLT_ENC_SKETCH ? kSketchRankCap : INT32_MAX;
+  if (cfg.rt_max > 0) cap = std::min<int64_t>(cap, cfg.rt_max);
+  if (cfg.factors == 0) cap = 0;   // residual only: the grid is the single point r_t = r_d = 0
+  int64_t R = std::min<int64_t>({(int64_t)T, (int64_t)H * D, per_lt / (2 * (int64_t)T), cap});
+  R -= R % p->step;
+  p->R = (int)std::max<int64_t>(0, R);
+  if (p->R > kMaxRank) {
+    const int R0 = p->R;
+    delete p;
+    return fail(JOLT_ERR_UNSUPPORTED,
+                "jolt_plan: the candidate grid reaches token rank %d; this library implements token ranks up to "
+                "%d (set jolt_config.rt_max <= %d)",
+                R0, kMaxRank, kMaxRank);
+  }
   p->q_iters = cfg.power_iters;
   if (enc == JOLT_ENC_EXACT && T > kMaxN) {
     // The token Gram is too large for one CTA's eigensolver: its leading eigenvectors come from
@@ -623,8 +647,11 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
                   (long long)(minb_lt * per_pool_lts));
     }
   }
-  // tensor-core path: bf16 inputs whose token stride is a multiple of 16 bytes (TMA rule)
-  p->use_tc = sh.dtype == JOLT_BF16 && (T % 8) == 0;
+  // tensor-core path: bf16 inputs whose token stride is a multiple of 16 bytes (TMA rule), and
+  // whose contractions over the tokens split into float32 chunks of at most 2048 tokens (whole
+  // 64-token blocks); other token counts take the SIMT kernels, which accumulate in float64
+  p->use_tc = sh.dtype == JOLT_BF16 && (T % 8) == 0 && (T <= 2048 || k_chunks(T) > 1) &&
+              T / gram_chunks(T) <= 2048;
   // workspace
   const int64_t n = p->n_lt, HD = (int64_t)H * D, Rm = std::max(p->R, 1), l = std::max(p->l, 2);
   auto layout = [&](char* base, bool assign) -> size_t {
@@ -690,9 +717,9 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   };
   p->ws_bytes = layout(nullptr, false);
   cudaError_t e = cudaGetDevice(&p->device);
-  if (e == cudaSuccess) e = cudaMalloc(&p->ws, p->ws_bytes);
-  if (e == cudaSuccess) e = cudaMalloc(&p->d_lt_ids, sizeof(int32_t) * p->lt_ids.size());
-  if (e == cudaSuccess) e = cudaMalloc(&p->d_cand_order, sizeof(int32_t) * p->cand_order.size());
+  if (e == cudaSuccess) e = dev_malloc(&p->ws, p->ws_bytes);
+  if (e == cudaSuccess) e = dev_malloc(&p->d_lt_ids, sizeof(int32_t) * p->lt_ids.size());
+  if (e == cudaSuccess) e = dev_malloc(&p->d_cand_order, sizeof(int32_t) * p->cand_order.size());
   if (e == cudaSuccess)
     e = cudaMemcpy(p->d_cand_order, p->cand_order.data(), sizeof(int32_t) * p->cand_order.size(),
                    cudaMemcpyHostToDevice);
@@ -1711,6 +1738,8 @@ JOLT_API jolt_status jolt_selftest_gemm_bf16_layout(int32_t M, int32_t N, int32_
 }
 
 JOLT_API uint64_t jolt_launch_count(void) { return g_launches.load(); }
+
+JOLT_API uint64_t jolt_alloc_count(void) { return g_allocs.load(); }
 
 JOLT_API jolt_status jolt_profile_enable(int32_t on) {
   std::lock_guard<std::mutex> g(g_prof_mu);

@@ -16,6 +16,8 @@ constexpr int kMaxL = 128;         // layers per stream
 constexpr int kMaxLT = 2 * kMaxL;  // layer-tensors per stream
 constexpr int kMaxGroups = 64;
 constexpr int kMaxN = 128;         // largest in-shared-memory eigenproblem / sketch width
+constexpr int kSketchRankCap = 256;   // token-rank cap of the randomized-SVD encoder's grid
+constexpr int kMaxRank = 112;      // largest token rank implemented (sketch width rank + 16 <= kMaxN)
 constexpr int kAlign = 256;        // byte alignment of every stream part
 
 // Device status word bits (OR-ed by kernels, read by the host after a sync).

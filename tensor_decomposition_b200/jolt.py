@@ -30,7 +30,7 @@ EXPORTED = ["jolt_config_default", "jolt_plan", "jolt_plan_info", "jolt_encode",
             "jolt_rel_frob_error", "jolt_rel_frob_error_noalloc", "jolt_stream_status",
             "jolt_stream_info", "jolt_stream_to_host", "jolt_stream_from_host", "jolt_export_debug", "jolt_stream_destroy",
             "jolt_plan_destroy", "jolt_last_error", "jolt_profile_enable", "jolt_profile_report",
-            "jolt_launch_count", "jolt_selftest_gemm_bf16", "jolt_selftest_gemm_bf16_layout"]
+            "jolt_launch_count", "jolt_alloc_count", "jolt_selftest_gemm_bf16", "jolt_selftest_gemm_bf16_layout"]
 
 
 class JoltError(RuntimeError):
@@ -77,6 +77,7 @@ def _load():
         "jolt_profile_enable": (st, [i32]),
         "jolt_profile_report": (st, [ctypes.c_char_p, ctypes.POINTER(u64)]),
         "jolt_launch_count": (u64, []),
+        "jolt_alloc_count": (u64, []),
         "jolt_selftest_gemm_bf16": (st, [i32, i32, i32, vp, vp, vp, vp]),
         "jolt_selftest_gemm_bf16_layout": (st, [i32, i32, i32, vp, i32, vp, i32, vp, vp]),
     }
@@ -247,6 +248,10 @@ def jolt_profile_report() -> dict:
 
 def jolt_launch_count() -> int:
     return int(_lib.jolt_launch_count())
+
+
+def jolt_alloc_count() -> int:
+    return int(_lib.jolt_alloc_count())
 
 
 def jolt_selftest_gemm_bf16(A, B, C, cuda_stream=None):

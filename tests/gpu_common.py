@@ -11,7 +11,11 @@ from oracle import numerics as onum
 from oracle import stream as ostream
 
 ANGLE_TOL = 1e-3           # rad, leading subspace of the exact HOSVD factors
-GAP_REL = 1e-3             # eigengap (relative to the top eigenvalue) that makes a column "leading"
+GAP_REL = 1e-4             # eigengap (relative to the top eigenvalue) that makes a column "leading"
+# Token-rank cap given to both sides of every test plan: the library implements ranks up to 112,
+# while the method's default grid reaches 256 (sketch) or the budget bound (exact) on these
+# workloads; both the GPU plan (jolt_config.rt_max) and the oracle plan (rt_cap) get it explicitly.
+RT_MAX = 112
 REL_ERR_TOL = 0.01         # GPU relative Frobenius error within 1% (relative) of the oracle's
 BOUNDARY_BAND = 1e-6       # codes may differ only within this distance (units of the row scale)
 
@@ -35,6 +39,7 @@ def decode_tol(ref: np.ndarray, out_f32: bool) -> np.ndarray:
 
 
 def oracle_plan(cfg, budget, encoder, groups=None, split=None, bits=None, **kw):
+    kw.setdefault("rt_cap", RT_MAX)
     return oj.Plan(L=cfg.layers, H=cfg.heads, T=cfg.tokens, D=cfg.head_dim, has_v=cfg.has_v,
                    budget=budget, num_groups=groups or cfg.groups, encoder=encoder,
                    split_kv=cfg.split_kv if split is None else split,
@@ -46,6 +51,7 @@ def gpu_encode(cfg, K, V, budget, encoder, seed=42, groups=None, split=None, bit
     from tensor_decomposition_b200 import jolt as J
     c = J.jolt_config_default()
     c.encoder = J.JOLT_ENC_EXACT if encoder == "exact" else J.JOLT_ENC_SKETCH
+    c.rt_max = RT_MAX
     c.split_kv_budget = int(cfg.split_kv if split is None else split)
     mask = 0
     for b in (bits or cfg.bits):
@@ -177,6 +183,7 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
     budget = synth.kv.budget_bytes(cfg, ratio)
     c = J.jolt_config_default()
     c.encoder = J.JOLT_ENC_SKETCH if encoder == "sketch" else J.JOLT_ENC_EXACT
+    c.rt_max = RT_MAX
     c.split_kv_budget = int(cfg.split_kv)
     mask = 0
     for b in (bits or cfg.bits):
@@ -194,7 +201,7 @@ def fullsize_check(J, cfg, ratio, sample, seq=0, encoder="sketch", seed=42, bits
     torch.cuda.synchronize()
     ost = ostream.parse(J.jolt_stream_to_host(st), lts=set(sample))
     op = oracle_plan(cfg, budget, encoder, bits=bits, measured_b=bool(measured_b),
-                     rotation="hadamard" if rotation else "haar", **({} if factors else {"rt_cap": 0}))
+                     rotation="hadamard" if rotation else "haar", rt_cap=RT_MAX if factors else 0)
     assert ost.rt_max == op.R()
     check_allocation(J, st, ost, op, cfg)
     Pi = J.jolt_export_debug(st, J.JOLT_DBG_PI).reshape(128, 128).astype(np.float64)

@@ -121,3 +121,20 @@ def test_gemm_selftest_rejects_bad_sizes(jolt, M, N, K, a_mn, b_mn):
     buf = ctypes.create_string_buffer(64)
     p = ctypes.cast(buf, ctypes.c_void_p)
     assert f(M, N, K, p, a_mn, p, b_mn, p, None) == 1
+
+
+@pytest.mark.parametrize("tokens,heads,encoder,rank", [
+    (1024, 8, 2, 256),     # Mistral-7B shape, sketch at 2x: the grid's own cap, 256
+    (1024, 8, 1, 512),     # the same with the exact encoder: budget / (2T) = 512
+    (256, 8, 0, 256),      # single layer, automatic (exact) encoder: T = 256
+])
+def test_plan_refuses_token_ranks_beyond_the_kernels(jolt, tokens, heads, encoder, rank):
+    """The default grid follows the method's reading; a grid above the implemented rank 112 is
+    refused before any device call, with the rank in the message."""
+    c = jolt.jolt_config_default()
+    c.encoder = encoder
+    budget = 2 * heads * tokens * 128 * 2 // 2          # 2 layer-tensors at 2x
+    with pytest.raises(jolt.JoltError) as e:
+        jolt.jolt_plan(1, heads, tokens, 128, True, jolt.JOLT_BF16, budget, 1, c)
+    assert e.value.status == 9
+    assert f"token rank {rank}" in str(e.value) and "rt_max" in str(e.value)

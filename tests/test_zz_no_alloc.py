@@ -30,9 +30,11 @@ def test_noalloc_matches_allocating_entry_point(J, dtype, n):
     b = (a + 0.01 * rng.standard_normal(n)).astype(np.float32)
     ta, tb = to_torch(a, dtype), to_torch(b, dtype)
     want = J.jolt_rel_frob_error(ta, tb)
+    before = J.jolt_alloc_count()
     first = J.jolt_rel_frob_error_noalloc(ta, tb)
     second = J.jolt_rel_frob_error_noalloc(ta, tb)          # twice in a row: scratch reused
     assert first == want and second == want
+    assert J.jolt_alloc_count() == before                   # no device allocation by the library
     z = to_torch(np.zeros(16, np.float32), dtype)
     assert J.jolt_rel_frob_error_noalloc(z, z) == 0.0       # zero reference -> 0 (same rule)
 
