@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true", help="skip the in-codec baselines (quantisation only, Tucker only)")
     ap.add_argument("--profile-out", default=None, help="write the per-phase trace JSON here")
+    ap.add_argument("--no-suite", action="store_true",
+                    help="skip the other workloads (encode / decode per config, decode sweep, new-seed step)")
     return ap.parse_args()
 
 
@@ -206,19 +208,26 @@ def run_reference(args):
     if rank != 0:
         return
     cfg = synth.config(args.config)
-    times = []
+    spent = []
     threads = 1
     sample = ""
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         tps, threads, sample = oracle_sample_tokens_per_s(cfg, args.ratio, args.encoder, budget_s=0.0, max_s=30.0)
         if i >= args.warmup:
-            times.append(cfg.tokens / tps)
-    ms = 1e3 * sum(times) / len(times)
-    value = cfg.tokens / (ms / 1e3)
+            spent.append(time.perf_counter() - t0)
+    # each step is one sampled layer (K and V) of the cache; ms_per_step is the time it took, and
+    # the throughput counts the fraction of every token that step processed (1 / layers of it)
+    ms = 1e3 * sum(spent) / len(spent)
+    value = cfg.tokens / cfg.layers / (ms / 1e3)
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
            "config": config_dict(cfg, args),
+           "step": f"oracle encode + decode of one layer (K and V) of the {cfg.layers}-layer cache; "
+                   f"value = {cfg.tokens} tokens x 1/{cfg.layers} of their layers per step time",
+           "extrapolated": {"ms_per_full_cache_step": ms * cfg.layers,
+                            "note": "the same per-layer time times the layer count (not measured)"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
@@ -285,6 +294,122 @@ def in_codec_baselines(J, cfg, K, V, budget, encoder, steps=5, warmup=2):
     return res
 
 
+def codec_record(J, cfg, ratio, encoder, dev, peaks, steps=5, warmup=2, seq=0):
+    """Encode and decode throughput of one workload, timed apart: `steps` encodes (CUDA events on
+    the launch stream, inputs resident in HBM), then `steps` decodes of the last stream. Reports
+    tokens/s of each, the per-phase trace of the encodes, the roofline of the encode's dominant
+    phase and of the decode, and the relative errors."""
+    import torch
+    import synth
+    K, V = synth.gen_cache_torch(cfg, dev, seq=seq)
+    budget = synth.kv.budget_bytes(cfg, ratio)
+    c = J.jolt_config_default()
+    c.encoder = J.JOLT_ENC_SKETCH if encoder == "sketch" else J.JOLT_ENC_EXACT
+    c.rt_max = RT_MAX
+    c.split_kv_budget = int(cfg.split_kv)
+    c.bits_mask = sum(1 << b for b in cfg.bits)
+    plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, budget,
+                       cfg.groups, c)
+    info = J.jolt_plan_info(plan)
+    Ko, Vo = torch.empty_like(K), torch.empty_like(V)
+    for _ in range(warmup):
+        st = J.jolt_encode(plan, K, V, SEED)
+        J.jolt_decode(st, Ko, Vo)
+    J.jolt_stream_status(st)
+    alloc = J.jolt_stream_info(st, cfg.groups)["alloc"]
+    del st
+    torch.cuda.synchronize()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    J.jolt_profile_enable(True)
+    e[0].record()
+    for _ in range(steps):
+        st = J.jolt_encode(plan, K, V, SEED)
+    e[1].record()
+    torch.cuda.synchronize()
+    prof = J.jolt_profile_report()
+    J.jolt_profile_enable(False)
+    J.jolt_stream_status(st)
+    e[2].record()
+    for _ in range(steps):
+        J.jolt_decode(st, Ko, Vo)
+    e[3].record()
+    torch.cuda.synchronize()
+    enc_ms, dec_ms = e[0].elapsed_time(e[1]) / steps, e[2].elapsed_time(e[3]) / steps
+    errs = {"K": J.jolt_rel_frob_error(K, Ko), "V": J.jolt_rel_frob_error(V, Vo)}
+    models, stream_bytes = phase_models(cfg, info, alloc, ratio, peaks, q=power_iterations(cfg, encoder))
+    phases = {k: round(v["total_ms"] / steps, 4) for k, v in prof.items()}
+    top = max(phases, key=phases.get)
+    roof = {}
+    for name, ms in ((top, phases[top]), ("decode", dec_ms)):
+        m = models.get(name)
+        if m:
+            a = m["work"] / (ms / 1e3)
+            roof[name] = {"bound": m["bound"], "achieved": a, "peak": m["peak"], "unit": m["unit"],
+                          "frac": a / m["peak"], "ms": ms, "note": m["note"]}
+    del st, K, V, Ko, Vo, plan
+    torch.cuda.empty_cache()
+    return {"workload": cfg.name, "ratio": ratio, "encoder": encoder, "rt_max": RT_MAX,
+            "encode_ms": enc_ms, "decode_ms": dec_ms,
+            "encode_tokens_per_s": cfg.tokens / (enc_ms / 1e3), "decode_tokens_per_s": cfg.tokens / (dec_ms / 1e3),
+            "compressed_bytes": stream_bytes, "bf16_bytes": synth.bf16_bytes(cfg),
+            "rel_frob_error": errs, "alloc": alloc.tolist(), "encode_phase_ms": phases,
+            "encode_dominant_phase": top, "roofline": roof}
+
+
+def decode_sweep(J, dev, peaks, reps=5, warmup=2):
+    """The decode-throughput sweep: 16 sequences of the Mistral-7B layout at T = 8192, each encoded
+    once per budget (2x, 2.5x, 3x); then all 16 streams are decoded to bf16, `reps` times over
+    (CUDA events), into one output pair (1.07 GB, larger than L2). Per budget: tokens/s and the
+    algorithmic bytes (bf16 cache written + stream read) per second against the HBM peak."""
+    import torch
+    import synth
+    cfg = synth.config(4)
+    out = {}
+    Ko = torch.empty((cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim), dtype=torch.bfloat16, device=dev)
+    Vo = torch.empty_like(Ko)
+    for ratio in cfg.ratios:
+        budget = synth.kv.budget_bytes(cfg, ratio)
+        c = J.jolt_config_default()
+        c.encoder = J.JOLT_ENC_SKETCH
+        c.rt_max = RT_MAX
+        c.split_kv_budget = int(cfg.split_kv)
+        plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16, budget,
+                           cfg.groups, c)
+        streams, sbytes = [], 0
+        for seq in range(cfg.batch):
+            K, V = synth.gen_cache_torch(cfg, dev, seq=seq)
+            st = J.jolt_encode(plan, K, V, SEED)
+            J.jolt_stream_status(st)
+            sbytes += int(sum(J.jolt_stream_info(st, cfg.groups)["bytes_by_part"].values()))
+            streams.append(st)
+            del K, V
+        for _ in range(warmup):
+            for st in streams:
+                J.jolt_decode(st, Ko, Vo)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            for st in streams:
+                J.jolt_decode(st, Ko, Vo)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        nbytes = cfg.batch * 2 * Ko.numel() * 2 + sbytes
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[f"{ratio:g}x"] = {"ms_per_pass": ms, "sequences": cfg.batch, "tokens_per_s": cfg.batch * cfg.tokens / (ms / 1e3),
+                              "algorithmic_bytes": nbytes, "stream_bytes": sbytes, "GB_per_s": gbs,
+                              "hbm_peak_GB_per_s": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"]}
+        for st in streams:
+            J.jolt_stream_status(st)
+        del streams, plan
+        torch.cuda.synchronize()
+    del Ko, Vo
+    torch.cuda.empty_cache()
+    return {"workload": cfg.name, "note": "decode of every layer of 16 sequences per pass; bytes = bf16 output "
+                                          "(2 B per entry) + compressed stream read", "by_ratio": out}
+
+
 def job_throughput(local_ms, tokens, steps, world, device):
     """Whole-job throughput of a weak-scaling run. Every rank processed `tokens` tokens per step
     for `steps` steps; the job takes as long as its slowest rank (a MAX all-reduce over the
@@ -333,9 +458,18 @@ def ncu_traffic(phase):
     return rec[2] if sha == rec[1] else None
 
 
-def phase_models(cfg, plan_info, alloc, ratio, peaks):
+def power_iterations(cfg, encoder):
+    """Power iterations of the subspace iteration the plan runs: 1 for the sketch (the workloads'
+    q), 24 for the exact token factor above 128 tokens (realised as converged subspace iteration),
+    0 for the exact factor of a token Gram small enough for one eigensolver."""
+    if encoder == "sketch":
+        return 1
+    return 24 if cfg.tokens > 128 else 0
+
+
+def phase_models(cfg, plan_info, alloc, ratio, peaks, q=1):
     """Algorithmic work of each traced phase per step: flops or bytes the method needs, the
-    numerator of the roofline fraction."""
+    numerator of the roofline fraction. `q` is the number of power iterations."""
     H, T, D, L = cfg.heads, cfg.tokens, cfg.head_dim, cfg.layers
     n_lt = L * 2
     N = H * T * D                      # entries per layer-tensor
@@ -350,13 +484,15 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks):
                        for rt, rd, b in ranks)
     clock = peaks["sm_max_mhz"] * 1e6
     fp64_peak = 148 * 64 * 2 * clock / 1e12       # TFLOP/s, 64 FP64 FMA / clk / SM
-    # CholeskyQR passes: 1 for Omega's and the transposed sketch's bases, 3 for the final one
-    cholqr_flops = n_lt * 4.0 * l * l * (1 * T + 1 * H * D + 3 * T)
+    # CholeskyQR passes: 1 for every intermediate basis (A Omega, each A^T Q and all but the last
+    # A Q'), 3 for the final one
+    cholqr_flops = n_lt * 4.0 * l * l * ((q + 3) * T + q * H * D) if q else n_lt * 4.0 * l * l * 3 * T
+    passes = 2 + 2 * q
     resid_flops = sum(2.0 * N * (D + rt) for rt, rd, b in ranks if b > 0)
     dec_flops = sum(2.0 * N * (rt + (D if b else 0)) for rt, rd, b in ranks)
     return {
-        "sketch_gemm": dict(bound="tensor", work=8.0 * T * H * D * l * n_lt / 1e12, unit="TFLOP/s",
-                            peak=peaks["bf16_tflops"], note="4 passes over X, 2 T HD l flops each"),
+        "sketch_gemm": dict(bound="tensor", work=passes * 2.0 * T * H * D * l * n_lt / 1e12, unit="TFLOP/s",
+                            peak=peaks["bf16_tflops"], note=f"{passes} passes over X, 2 T HD l flops each"),
         "feature_gram": dict(bound="tensor", work=2.0 * N * D * n_lt / 1e12, unit="TFLOP/s",
                              peak=peaks["bf16_tflops"], note="C_D = sum_h X_h^T X_h"),
         "residual": dict(bound="alu", work=resid_flops / 1e12, unit="TFLOP/s", peak=fp64_peak,
@@ -507,7 +643,10 @@ def main():
            "compressed_bytes": stream_bytes, "budget_bytes": budget,
            "alloc": alloc.tolist(),
            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(K.numel() * 2 + V.numel() * 2),
-                   "d2h_bytes_per_step": 16},
+                   "d2h_bytes_per_step": 16,
+                   "note": "each step copies its K and V in from pinned host memory (overlapped with the previous "
+                           "step) and reads the two errors back; the compressed stream and the decoded cache stay "
+                           "in device memory, as a device-resident KV cache would"},
            "gpu_launches": int(launches),
            "phase_ms_per_step": phases,
            "roofline": roof,
@@ -515,11 +654,45 @@ def main():
                       "samples": clk["samples"]}}
     if rank == 0 and not args.no_baselines:
         out["in_codec_baselines"] = in_codec_baselines(J, cfg, K, V, budget, c.encoder)
+    if rank == 0 and world == 1 and not args.no_suite:
+        # a step whose codec seed is new every time: the rotation and the sketch matrices (functions
+        # of the seed alone, kept by the plan between encodes) are rebuilt inside the timed region
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for i in range(args.steps):
+            st = J.jolt_encode(plan, K, V, SEED + 1 + i)
+            J.jolt_decode(st, Ko, Vo)
+            errs_ns = (J.jolt_rel_frob_error(K, Ko), J.jolt_rel_frob_error(V, Vo))
+        g1.record()
+        torch.cuda.synchronize()
+        del st
+        ms_ns = g0.elapsed_time(g1) / args.steps
+        out["new_seed_step"] = {"ms_per_step": ms_ns, "tokens_per_s": cfg.tokens / (ms_ns / 1e3),
+                                "rel_frob_error": {"K": errs_ns[0], "V": errs_ns[1]},
+                                "note": "codec seed changes every step: rotation Pi and sketch matrices rebuilt"}
+        suite = []
+        for ci, ratio, enc in ((1, 2.0, "sketch"), (1, 3.0, "sketch"), (1, 2.0, "exact"), (1, 3.0, "exact"),
+                               (2, 2.0, "sketch"), (3, 3.0, "sketch")):
+            suite.append(codec_record(J, synth.config(ci), ratio, enc, dev, peaks))
+        out["per_workload"] = suite
+        rec = {(r["workload"], r["ratio"], r["encoder"]): r for r in suite}
+        ex, sk = rec[(cfg.name, 2.0, "exact")], rec[(cfg.name, 2.0, "sketch")]
+        out["exact_over_sketch_encode_time"] = {
+            "ratio": ex["encode_ms"] / sk["encode_ms"], "exact_ms": ex["encode_ms"], "sketch_ms": sk["encode_ms"],
+            "workload": f"{cfg.name}, 2x",
+            "note": "the exact token factor above 128 tokens is realised as subspace iteration with 24 power "
+                    "iterations (one for the sketch); the pages' FlashJoLT speedup at 1024 tokens is 5-13x"}
+        out["decode_sweep"] = decode_sweep(J, dev, peaks)
     if args.profile_out and rank == 0:
         json.dump(prof, open(args.profile_out, "w"), indent=1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_limits
         tps, threads, sample = oracle_sample_tokens_per_s(cfg, args.ratio, args.encoder)
-        out["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+        with threadpool_limits(limits=1):
+            tps1, _, sample1 = oracle_sample_tokens_per_s(cfg, args.ratio, args.encoder, budget_s=8.0, max_s=20.0)
+        out["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+                               "single_thread": {"value": tps1, "unit": UNIT, "cores": 1, "sample": sample1}}
     if rank == 0:
         print(json.dumps(out))
     if world > 1:
