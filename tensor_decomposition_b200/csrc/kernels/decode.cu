@@ -11,12 +11,14 @@
 //  * prologue: M_h^T = U_D G_h^T on the tensor core (both operands are the stored bf16
 //    factors, so the products are exact and only the float32 sum rounds); M_h^T and Pi
 //    (float32) are kept in shared memory as two bf16 parts each (hi + lo, ~2^-17 relative);
-//  * producers (warps 4-7) copy the tile's U_T rows and unpack its codes into bf16 cell
+//  * producers (warps 4-11) copy the tile's U_T rows and unpack its codes into bf16 cell
 //    centres (exact: odd integers below 2^8 over 2^b), both in the 128-byte-swizzled K-major
-//    layout; the codes arrive by one bulk copy per tile into two alternating buffers, and the
-//    next tile's copy and U_T rows (held in registers) are in flight while a tile is unpacked;
-//  * warp 8 issues tcgen05.mma: acc1 = U_T (M_h^T)_p^T and acc2 = Y_hat Pi_p^T over the
-//    parts p, double-buffered in Tensor Memory (4 x 128 columns);
+//    layout. The codes of the next tile and its U_T rows are loaded into registers while the
+//    current tile is unpacked; the cell centres go to two alternating buffers, so a tile is
+//    unpacked while the previous one is multiplied;
+//  * warp 12 issues tcgen05.mma: acc1 = U_T (M_h^T)_p^T, then acc2 = Y_hat Pi_p^T over the parts
+//    p, double-buffered in Tensor Memory (4 x 128 columns). The U_T buffer is single: it is
+//    released as soon as the Tucker products of a tile complete, ahead of the residual ones;
 //  * the epilogue (warps 0-3, one row per thread) forms acc1 + s acc2 and stores bf16
 //    (round to nearest even) or float32; the row's next scale is loaded a tile ahead.
 // Every wait is bounded: a timeout sets ST_TIMEOUT in the stream status and the CTA runs on
@@ -30,18 +32,19 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileRows = 128;
-constexpr int kThreads = 288;                 // 9 warps
+constexpr int kProducers = 256;               // warps 4-11
+constexpr int kMmaWarp = 12;
+constexpr int kThreads = 32 * (kMmaWarp + 1);  // 13 warps
 constexpr int kOpBytes = 128 * 128 * 2;       // one 128 x 128 bf16 operand (two swizzle atoms)
-constexpr int kCodesBytes = 128 * 128;        // codes of one tile, b <= 8
 constexpr uint32_t kMaxPoll = 1u << 22;
-// dynamic shared memory: B1 parts, B2 parts, A1, A2, two codes buffers
+// dynamic shared memory: B1 parts (M_h^T), B2 parts (Pi), A1 (U_T tile), two A2 (cell centres)
 constexpr int kOffB1 = 0;
 constexpr int kOffB2 = 2 * kOpBytes;
 constexpr int kOffA1 = 4 * kOpBytes;
 constexpr int kOffA2 = 5 * kOpBytes;
-constexpr int kOffCodes = 6 * kOpBytes;
-constexpr int kSmemBytes = kOffCodes + 2 * kCodesBytes + 1024;
-constexpr int kUtVec = 16;   // 16-byte U_T vectors per producer thread and tile (128 rows x r_t <= 128)
+constexpr int kSmemBytes = 7 * kOpBytes + 1024;
+constexpr int kUtVec = 8;      // 16-byte U_T vectors per producer thread and tile (128 rows x r_t <= 128)
+constexpr int kChunks = 8;     // 8-code chunks per producer thread and tile (128 rows x 16 chunks)
 
 // Byte offset of the 16-byte chunk `c16` (8 bf16, k = 8 c16 ..) of row `row` in a K-major
 // 128-row operand with 128-byte swizzling: 64-element atoms of 16 KB, rows of 128 bytes, the
@@ -53,13 +56,6 @@ __device__ __forceinline__ uint32_t sw128(int row, int c16) {
 // Descriptor of the 16-wide K slice `kk` of a 128-row operand at shared address `base`.
 __device__ __forceinline__ uint64_t slice_desc(uint32_t base, int kk) {
   return desc_kmajor_sw128(base + (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32));
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -87,7 +83,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
 
 __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
   extern __shared__ uint8_t smraw[];
-  __shared__ __align__(8) uint64_t bar_pro, bar_afull, bar_aempty, bar_codes[2];
+  __shared__ __align__(8) uint64_t bar_pro, bar_afull[2], bar_a1free, bar_a2free[2];
   __shared__ __align__(8) uint64_t bar_accfull[2], bar_accempty[2];
   __shared__ uint32_t tmem_base;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -112,17 +108,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
 
   if (tid == 0) {
     mbar_init(&bar_pro, 1);
-    mbar_init(&bar_afull, 128);
-    mbar_init(&bar_aempty, 1);
-    mbar_init(&bar_codes[0], 1);
-    mbar_init(&bar_codes[1], 1);
+    mbar_init(&bar_a1free, 1);
     for (int j = 0; j < 2; ++j) {
+      mbar_init(&bar_afull[j], kProducers);
+      mbar_init(&bar_a2free[j], 1);
       mbar_init(&bar_accfull[j], 1);
       mbar_init(&bar_accempty[j], 128);
     }
     fence_barrier_init();
   }
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&tmem_base, 512);
     tmem_relinquish();
   }
@@ -160,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
   fence_async_shared();
   __syncthreads();
   if (tucker) {
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
       if (elect_one()) {
         tc_fence_after();
         const uint32_t id = idesc_bf16_f32(128, rt);
@@ -199,22 +194,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
   tc_fence_after();
 
   // ---------------------------------------------------------------- tiles of 128 rows
-  if (warp >= 4 && warp < 8) {
-    // producers: U_T rows -> A1, unpacked cell centres -> A2. The codes of tile it + 1 are
-    // copied (one bulk copy, two buffers) and its U_T rows loaded into registers while tile it
-    // is unpacked and multiplied.
+  if (warp >= 4 && warp < kMmaWarp) {
+    // producers: U_T rows -> A1, unpacked cell centres -> A2[tile parity]. Each thread takes 8
+    // chunks of 8 codes (b bytes each, at byte u b of the tile's code block for chunk u); the
+    // next tile's chunks (two aligned 8-byte words around each) and U_T rows are loaded into
+    // registers before the current tile is unpacked.
     const int pt = tid - 128;
     const float inv2b = resid ? 1.0f / (float)(1 << b) : 0.0f;
     const float off2b = resid ? 1.0f - (float)(1 << b) : 0.0f;
-    const uint32_t mask = resid ? (1u << b) - 1u : 0u;
+    const uint64_t mask = resid ? (1ull << b) - 1ull : 0ull;
     const int cpr = tucker ? rt / 8 : 0;   // 16-byte vectors per U_T row
-    auto issue_codes = [&](int it2) {
-      if (resid && pt == 0 && it2 < ntiles) {
-        const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
-        const uint32_t bytes = (uint32_t)(rows2 * rowbytes);
-        mbar_arrive_expect_tx(&bar_codes[it2 & 1], bytes);
-        bulk_load(sm + kOffCodes + (it2 & 1) * kCodesBytes, codes + ((int64_t)h * T + t2) * rowbytes, bytes,
-                  &bar_codes[it2 & 1]);
+    uint64_t cw[kChunks][2];
+    auto load_codes = [&](int it2) {
+      const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
+      const uint8_t* blk = codes + ((int64_t)h * T + t2) * rowbytes;
+#pragma unroll
+      for (int q = 0; q < kChunks; ++q) {
+        const int u = pt + kProducers * q;
+        const int byte0 = u * b;
+        const uint64_t* w = reinterpret_cast<const uint64_t*>(blk + (byte0 & ~7));
+        const bool ok = resid && it2 < ntiles && (u >> 4) < rows2;
+        cw[q][0] = ok ? __ldg(w) : 0ull;
+        cw[q][1] = ok ? __ldg(w + 1) : 0ull;
       }
     };
     uint4 ut[kUtVec];
@@ -223,57 +224,59 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
       const __nv_bfloat16* src = UT + (int64_t)t2 * rt;
 #pragma unroll
       for (int q = 0; q < kUtVec; ++q) {
-        const int u = pt + 128 * q;
-        ut[q] = u < rows2 * cpr ? *reinterpret_cast<const uint4*>(src + (int64_t)(u / cpr) * rt + 8 * (u % cpr))
-                                : make_uint4(0u, 0u, 0u, 0u);
+        const int u = pt + kProducers * q;
+        ut[q] = (it2 < ntiles && u < rows2 * cpr)
+                    ? *reinterpret_cast<const uint4*>(src + (int64_t)(u / cpr) * rt + 8 * (u % cpr))
+                    : make_uint4(0u, 0u, 0u, 0u);
       }
     };
+    if (resid) load_codes(0);
     if (tucker) load_ut(0);
-    issue_codes(0);
     for (int it = 0; it < ntiles; ++it) {
-      const int t0 = it * kTileRows, rows = min(kTileRows, T - t0);
-      // the other codes buffer was last read by tile it - 1, whose unpack ended at the barrier
-      issue_codes(it + 1);
-      wait_or_flag(&bar_aempty, (uint32_t)((it & 1) ^ 1), status);
-      if (tucker) {
-#pragma unroll
-        for (int q = 0; q < kUtVec; ++q) {
-          const int u = pt + 128 * q;
-          if (u < rows * cpr) *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(u / cpr, u % cpr)) = ut[q];
-        }
-        if (it + 1 < ntiles) load_ut(it + 1);
-      }
+      const int buf = it & 1, use = it >> 1;
+      const int rows = min(kTileRows, T - it * kTileRows);
       if (resid) {
-        wait_or_flag(&bar_codes[it & 1], (uint32_t)((it >> 1) & 1), status);
-        const uint32_t* cw = reinterpret_cast<const uint32_t*>(sm + kOffCodes + (it & 1) * kCodesBytes);
-        for (int u = pt; u < rows * 16; u += 128) {
+        // A2[buf] was last read by the residual products of tile it - 2
+        wait_or_flag(&bar_a2free[buf], (uint32_t)((use & 1) ^ 1), status);
+        uint8_t* a2 = sm + kOffA2 + buf * kOpBytes;
+#pragma unroll
+        for (int q = 0; q < kChunks; ++q) {
+          const int u = pt + kProducers * q;
           const int r = u >> 4, c = u & 15;
-          const int byte0 = r * rowbytes + c * b;   // eight codes = b bytes
-          const int w0 = byte0 >> 2, sh = (byte0 & 3) * 8;
-          uint64_t v = ((uint64_t)cw[w0] | ((uint64_t)cw[w0 + 1] << 32)) >> sh;
-          if (sh) v |= (uint64_t)cw[w0 + 2] << (64 - sh);
+          const int sh = ((u * b) & 7) * 8;
+          const uint64_t v = sh ? (cw[q][0] >> sh) | (cw[q][1] << (64 - sh)) : cw[q][0];
           float y[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const uint32_t q = (uint32_t)(v >> (e * b)) & mask;
-            y[e] = ((float)(2 * q) + off2b) * inv2b;
+            const uint32_t cq = (uint32_t)((v >> (e * b)) & mask);
+            y[e] = ((float)(2 * cq) + off2b) * inv2b;
           }
-          *reinterpret_cast<uint4*>(sm + kOffA2 + sw128(r, c)) =
-              make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                         pack_bf16x2(y[6], y[7]));
+          if (r < rows)
+            *reinterpret_cast<uint4*>(a2 + sw128(r, c)) =
+                make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                           pack_bf16x2(y[6], y[7]));
         }
+        load_codes(it + 1);
+      }
+      if (tucker) {
+        // A1 was last read by the Tucker products of tile it - 1
+        wait_or_flag(&bar_a1free, (uint32_t)((it & 1) ^ 1), status);
+#pragma unroll
+        for (int q = 0; q < kUtVec; ++q) {
+          const int u = pt + kProducers * q;
+          if (u < rows * cpr) *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(u / cpr, u % cpr)) = ut[q];
+        }
+        load_ut(it + 1);
       }
       fence_async_shared();
-      mbar_arrive(&bar_afull);
-      // every producer is done with this tile's codes buffer before tile it + 2's copy lands in it
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      mbar_arrive(&bar_afull[buf]);
     }
-  } else if (warp == 8) {
+  } else if (warp == kMmaWarp) {
     if (elect_one()) {
       const uint32_t id = idesc_bf16_f32(128, 128);
       for (int it = 0; it < ntiles; ++it) {
         const int buf = it & 1, use = it >> 1;
-        wait_or_flag(&bar_afull, (uint32_t)(it & 1), status);
+        wait_or_flag(&bar_afull[buf], (uint32_t)(use & 1), status);
         wait_or_flag(&bar_accempty[buf], (uint32_t)((use & 1) ^ 1), status);
         tc_fence_after();
         const uint32_t d1 = tmem + (uint32_t)(buf * 256), d2 = d1 + 128;
@@ -282,12 +285,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
 #pragma unroll
             for (int p = 0; p < 2; ++p)
               umma_bf16(d1, slice_desc(sA1, kk), slice_desc(sB1 + p * kOpBytes, kk), id, (kk | p) ? 1u : 0u);
-        if (resid)
+        umma_commit(&bar_a1free);         // the U_T tile may be overwritten once these complete
+        if (resid) {
+          const uint32_t a2 = sA2 + (uint32_t)(buf * kOpBytes);
           for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
             for (int p = 0; p < 2; ++p)
-              umma_bf16(d2, slice_desc(sA2, kk), slice_desc(sB2 + p * kOpBytes, kk), id, (kk | p) ? 1u : 0u);
-        umma_commit(&bar_aempty);
+              umma_bf16(d2, slice_desc(a2, kk), slice_desc(sB2 + p * kOpBytes, kk), id, (kk | p) ? 1u : 0u);
+        }
+        umma_commit(&bar_a2free[buf]);
         umma_commit(&bar_accfull[buf]);
       }
     }
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
