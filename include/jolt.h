@@ -166,6 +166,24 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t plan, const void* K, const void* V,
 JOLT_API jolt_status jolt_decode(jolt_stream_t stream, void* K_out, void* V_out, void* cuda_stream);
 
 /*
+ * jolt_attention - attention of a few queries per head over the compressed cache of a stream,
+ *   for every layer, without rebuilding the cache:
+ *       out[l][j][i] = sum_t softmax_t(scale * Q[l][j][i] . K_hat[l][h][t]) V_hat[l][h][t],
+ *   h = j / (q_heads / heads) (grouped-query attention; q_heads = heads is multi-head). K_hat and
+ *   V_hat are the stream's reconstructions G x2 U_T x3 U_D + dequant(codes) Pi^T, used in factored
+ *   form: scores from U_T, G_h U_D^T q, the codes, the scales and Pi^T q; the value sum from the
+ *   softmax-weighted sums of U_T rows and of scaled cell centres, mapped back through G_h, U_D, Pi.
+ *   The method's pages compress the cache that attention reads (Abstract); this consumer of the
+ *   stream is this library's own, with the same linear algebra as the decode.
+ * Q: device bf16 [layers][q_heads][n_queries][head_dim]; out: device float32, same shape. The
+ *   stream must hold K and V (bf16). Enqueued on `cuda_stream`; takes scratch from the library's
+ *   memory pool. Errors: INVALID_ARG (null pointers, q_heads not a multiple of the KV heads, no V),
+ *   UNSUPPORTED (float32 streams).
+ */
+JOLT_API jolt_status jolt_attention(jolt_stream_t stream, const void* Q, int32_t q_heads, int32_t n_queries,
+                                    float scale, float* out, void* cuda_stream);
+
+/*
  * jolt_rel_frob_error - ||ref - approx||_F / ||ref||_F over n elements (the error measure the
  *   Abstract reports), accumulated in float64. ref, approx: device arrays of `dtype`.
  *   Synchronises `cuda_stream`; *out is host memory. Returns 0 when ||ref|| = 0.
@@ -254,6 +272,17 @@ JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, co
  * operand needs M (N) a multiple of 8. Otherwise as jolt_selftest_gemm_bf16. */
 JOLT_API jolt_status jolt_selftest_gemm_bf16_layout(int32_t M, int32_t N, int32_t K, const void* A, int32_t a_mn,
                                                     const void* B, int32_t b_mn, float* C, void* cuda_stream);
+
+/* jolt_selftest_eig_dense - the R largest eigenvalues (descending) and their eigenvectors of
+ * `batch` dense symmetric n x n float64 matrices, by the solver of the exact token factor above 128
+ * tokens (Householder tridiagonalisation, bisection, inverse iteration, back-transformation, then
+ * two CholeskyQR passes), exposed so its numerics can be tested alone.
+ * A: device float64 [batch][n][n] (only read), V: device float64 [batch][n][R] (eigenvector r in
+ * column r), lam: device float64 [batch][R]. 2 <= n <= 4096, 1 <= R <= min(n, 128). Allocates its
+ * own scratch; synchronises `cuda_stream`; NOT_CONVERGED when the vectors were too close to
+ * dependent for the re-orthonormalisation. */
+JOLT_API jolt_status jolt_selftest_eig_dense(int32_t batch, int32_t n, int32_t R, const double* A, double* V,
+                                             double* lam, void* cuda_stream);
 
 /* Release a stream. Its device memory is freed in order on the CUDA stream the stream was
  * created on (encode or jolt_stream_from_host); synchronise any other CUDA stream that still

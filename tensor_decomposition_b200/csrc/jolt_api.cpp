@@ -27,11 +27,9 @@ using namespace jolt;
 
 namespace {
 
-// Power iterations that realise the exact token factor for T > 128 (subspace iteration on the
-// token Gram with a subspace of R + 16 columns). The slowest asserted eigenvectors sit at the
-// top of the noise bulk, where lambda_{l+1} / lambda_j ~ 0.57 per step: 16 steps left 5e-4 rad
-// against a dense eigensolver at T = 1024, 24 steps take it below 1e-5 rad.
-constexpr int kExactPowerIters = 24;
+// Largest token count of the exact encoder: its token Gram is a dense T x T float64 matrix per
+// layer-tensor, reduced to tridiagonal form on one SM each.
+constexpr int kExactMaxTokens = 4096;
 
 thread_local std::string g_err;
 
@@ -257,7 +255,9 @@ struct jolt_plan_s {
   float* Wpart = nullptr;                                // K-chunk partial Grams (CholeskyQR)
   int qset = 0;                                          // part set holding the final sketch basis
   int q_iters = 1;                                       // power iterations of the subspace iteration
-  bool exact_by_iteration = false;                       // exact encoder realised by converged iteration
+  bool exact_dense = false;                              // exact token factor by the dense eigensolver (T > 128)
+  double* tri = nullptr;                                 // its scratch (tridiag_scratch_doubles)
+  double *Qx = nullptr, *Gx = nullptr, *Rx = nullptr;    // its CholeskyQR: [n][T][R], [n][R][R] x 2
   float* Wf = nullptr;                                   // float32 CholeskyQR Grams
   __nv_bfloat16* UDt = nullptr;                          // U_D^T (rounded factor, exact in bf16)
   __nv_bfloat16* Pp[3] = {nullptr, nullptr, nullptr};    // bf16 parts of the core intermediate P
@@ -497,6 +497,38 @@ float* cholqr_t(jolt_plan_s* p, int rows, float* bufA, float* bufB, int passes, 
   return src;
 }
 
+// Leading R eigenvectors of `batch` symmetric T x T float64 matrices A (overwritten) by the dense
+// eigensolver, then two CholeskyQR passes in float64 (Q = Z R^-1 with R^T R = Z^T Z) so that the R
+// columns are orthonormal to rounding. `out` receives [batch][T][R] (float32 or float64), `lam`
+// (optional, float64 [batch][R]) the eigenvalues, descending. tri: tridiag_scratch_doubles(batch,
+// T, R); Qx: batch T R, Gx and Rx: batch R^2 float64.
+cudaError_t dense_top_eig(int batch, int T, int R, double* A, int64_t sA, double* tri, double* Qx, double* Gx,
+                          double* Rx, void* out, ElemType out_t, double* lam, int32_t* status, cudaStream_t s) {
+  double *Z = nullptr, *lz = nullptr;
+  cudaError_t e = eig_top_dense(batch, T, R, A, sA, tri, &Z, &lz, s);
+  if (e != cudaSuccess) return e;
+  const int Rp = tridiag_rpad(R);
+  const double* src = Z;
+  int64_t ld = Rp;
+  for (int pass = 0; pass < 2 && e == cudaSuccess; ++pass) {
+    e = gemm_simt(batch, R, R, T, opnd(src, EL_F64, I1((int64_t)T * ld), I1(1), I1(ld)),
+                  opnd(src, EL_F64, I1((int64_t)T * ld), I1(1), I1(ld)),
+                  outd(Gx, EL_F64, I1((int64_t)R * R), I1(R), I1(1)), 1.0, 0.0, s);
+    if (e == cudaSuccess) e = chol_inv(batch, R, Gx, (int64_t)R * R, Rx, (int64_t)R * R, 0.0, status, s);
+    if (e == cudaSuccess)
+      e = gemm_simt(batch, T, R, R, opnd(src, EL_F64, I1((int64_t)T * ld), I1(ld), I1(1)),
+                    opnd(Rx, EL_F64, I1((int64_t)R * R), I1(1), I1(R)),
+                    outd(pass == 0 ? (void*)Qx : out, pass == 0 ? EL_F64 : out_t, I1((int64_t)T * R), I1(R), I1(1)),
+                    1.0, 0.0, s);
+    src = Qx;
+    ld = R;
+  }
+  if (e == cudaSuccess && lam)
+    e = cudaMemcpy2DAsync(lam, sizeof(double) * R, lz, sizeof(double) * Rp, sizeof(double) * R, (size_t)batch,
+                          cudaMemcpyDeviceToDevice, s);
+  return e;
+}
+
 }  // namespace
 
 // ============================================================================ API
@@ -584,12 +616,15 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   }
   p->q_iters = cfg.power_iters;
   if (enc == JOLT_ENC_EXACT && T > kMaxN) {
-    // The token Gram is too large for one CTA's eigensolver: its leading eigenvectors come from
-    // block subspace iteration on C_T = A A^T, orthonormalised at every step, followed by the
-    // Rayleigh-Ritz step of the sketch path, run long enough to converge (kExactPowerIters).
-    p->exact_by_iteration = true;
-    p->q_iters = kExactPowerIters;
-    enc = JOLT_ENC_SKETCH;
+    // The token Gram is too large for one CTA's Jacobi eigensolver: its leading eigenvectors
+    // come from the dense float64 eigensolver (tridiagonalisation, bisection, inverse iteration)
+    if (T > kExactMaxTokens) {
+      delete p;
+      return fail(JOLT_ERR_UNSUPPORTED,
+                  "jolt_plan: the exact encoder forms the %d x %d token Gram; above %d tokens use the sketch encoder",
+                  T, T, kExactMaxTokens);
+    }
+    p->exact_dense = p->R > 0;
   }
   p->encoder = enc;
   if (enc == JOLT_ENC_SKETCH) {
@@ -710,8 +745,15 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
       take(p->lamB, n * l);
     } else {
       take(p->CT, n * T * T);
-      take(p->VT, n * T * T);
-      take(p->lamT, n * T);
+      if (p->exact_dense) {
+        take(p->tri, tridiag_scratch_doubles((int)n, T, (int)Rm));
+        take(p->Qx, n * T * Rm);
+        take(p->Gx, n * Rm * Rm);
+        take(p->Rx, n * Rm * Rm);
+      } else {
+        take(p->VT, n * T * T);
+        take(p->lamT, n * T);
+      }
     }
     return (size_t)(cur - base) + 256;
   };
@@ -744,7 +786,7 @@ JOLT_API jolt_status jolt_plan_info(jolt_plan_t p, int32_t* rt_max, int32_t* ske
   if (!p) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan_info: null plan");
   if (rt_max) *rt_max = p->R;
   if (sketch_l) *sketch_l = p->encoder == JOLT_ENC_SKETCH ? p->l : 0;
-  if (encoder) *encoder = p->exact_by_iteration ? JOLT_ENC_EXACT : p->encoder;
+  if (encoder) *encoder = p->encoder;
   if (workspace_bytes) *workspace_bytes = p->ws_bytes;
   return JOLT_OK;
 }
@@ -754,7 +796,7 @@ static jolt_status make_stream(jolt_plan_s* p, uint64_t seed, cudaStream_t cs, j
   if (!st) return fail(JOLT_ERR_OOM, "stream: host allocation");
   const jolt_shape& sh = p->shape;
   st->L = sh.layers; st->H = sh.heads; st->T = sh.tokens; st->D = sh.head_dim;
-  st->has_v = sh.has_v ? 1 : 0; st->G = p->G; st->encoder = p->exact_by_iteration ? JOLT_ENC_EXACT : p->encoder; st->step = p->step;
+  st->has_v = sh.has_v ? 1 : 0; st->G = p->G; st->encoder = p->encoder; st->step = p->step;
   st->rotation = p->cfg.rotation;
   st->R = p->R; st->split = (sh.has_v && p->cfg.split_kv_budget) ? 1 : 0; st->dtype = sh.dtype;
   st->seed = seed; st->cs = cs; st->plan = p; st->n_lt = p->n_lt;
@@ -1182,16 +1224,25 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
                        opnd(X[k], xt, I1(HTD), I1(D), I2(D, 1, (int64_t)T * D)),
                        outd(p->CT + (int64_t)k * L * T * T, EL_F64, I1((int64_t)T * T), I1(T), I1(1)), 1.0, 0.0, s));
       }
-      {
+      if (!p->exact_dense) {
         jolt_status r = eig_feature_and(T, p->CT, p->VT, p->lamT);
         if (r != JOLT_OK) return r;
         r = feature_sign_round();
         if (r != JOLT_OK) return r;
-      }
-      {
         PROF("sign_round", s);
         CK(cudaMemcpy2DAsync(p->UT32, sizeof(float) * R, p->VT, sizeof(float) * T, sizeof(float) * R,
                              (size_t)n * T, cudaMemcpyDeviceToDevice, s));
+      } else {
+        jolt_status r = eig_feature_and(0, nullptr, nullptr, nullptr);
+        if (r != JOLT_OK) return r;
+        r = feature_sign_round();
+        if (r != JOLT_OK) return r;
+        PROF("token_eig", s);
+        CK(dense_top_eig(n, T, R, p->CT, (int64_t)T * T, p->tri, p->Qx, p->Gx, p->Rx, p->UT32, EL_F32, nullptr,
+                         status, s));
+      }
+      {
+        PROF("sign_round", s);
         CK(sign_fix(n, T, R, p->UT32, R, (int64_t)T * R, nullptr, 0, 0, 0, s));
         CK(round_bf16((int64_t)n * T * R, p->UT32, p->UTb, p->UTf, s));
       }
@@ -1339,11 +1390,40 @@ JOLT_API jolt_status jolt_decode(jolt_stream_t st, void* K_out, void* V_out, voi
   if (!st || !K_out) return fail(JOLT_ERR_INVALID_ARG, "jolt_decode: null stream or K_out");
   if (st->has_v && !V_out) return fail(JOLT_ERR_INVALID_ARG, "jolt_decode: stream has V but V_out is null");
   DecodeArgs a;
-  a.n_lt = st->n_lt; a.H = st->H; a.T = st->T; a.D = st->D; a.lt_ids = st->d_lt_ids;
+  a.n_lt = st->n_lt; a.L = st->L; a.H = st->H; a.T = st->T; a.D = st->D; a.lt_ids = st->d_lt_ids;
   a.out[0] = K_out; a.out[1] = V_out; a.ot = st->dtype == JOLT_BF16 ? EL_BF16 : EL_F32;
   a.Pi = st->d_Pi; a.meta = st->d_meta; a.body = st->d_body;
   PROF("decode", (cudaStream_t)cuda_stream);
   CK(decode(a, (cudaStream_t)cuda_stream));
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_attention(jolt_stream_t st, const void* Q, int32_t q_heads, int32_t n_queries,
+                                    float scale, float* out, void* cuda_stream) {
+  g_err.clear();
+  if (!st || !Q || !out) return fail(JOLT_ERR_INVALID_ARG, "jolt_attention: null stream, Q or out");
+  if (!st->has_v) return fail(JOLT_ERR_INVALID_ARG, "jolt_attention: the stream holds keys only");
+  if (st->dtype != JOLT_BF16) return fail(JOLT_ERR_UNSUPPORTED, "jolt_attention: bf16 streams only");
+  if (q_heads <= 0 || n_queries <= 0 || q_heads % st->H != 0)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_attention: q_heads must be a positive multiple of the %d KV heads", st->H);
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  AttnArgs a;
+  a.L = st->L; a.H = st->H; a.T = st->T; a.D = st->D; a.Hq = q_heads; a.n = n_queries; a.R = std::max(st->R, 1);
+  a.scale = scale; a.meta = st->d_meta; a.body = st->d_body; a.Pi = st->d_Pi;
+  a.Q = reinterpret_cast<const __nv_bfloat16*>(Q); a.out = out;
+  a.nchunk = attn_chunks(st->T); a.ngroups = attn_groups(q_heads, st->H, n_queries);
+  const size_t nqv = (size_t)a.L * q_heads * n_queries;
+  const size_t floats = nqv * (kD + a.R) + (size_t)a.L * a.H * a.nchunk * a.ngroups * attn_part_floats(a.R);
+  float* scratch = nullptr;
+  PROF("attention", s);
+  CK(pool_malloc(&scratch, floats * sizeof(float), s));
+  a.qpi = scratch;
+  a.qhat = scratch + nqv * kD;
+  a.part = a.qhat + nqv * a.R;
+  cudaError_t e = attention(a, s);
+  cudaError_t e2 = cudaFreeAsync(scratch, s);
+  if (e == cudaSuccess) e = e2;
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_attention: %s", cudaGetErrorString(e));
   return JOLT_OK;
 }
 
@@ -1735,6 +1815,35 @@ JOLT_API jolt_status jolt_selftest_gemm_bf16(int32_t M, int32_t N, int32_t K, co
 JOLT_API jolt_status jolt_selftest_gemm_bf16_layout(int32_t M, int32_t N, int32_t K, const void* A, int32_t a_mn,
                                                     const void* B, int32_t b_mn, float* C, void* cuda_stream) {
   return selftest_gemm("jolt_selftest_gemm_bf16_layout", M, N, K, A, a_mn, B, b_mn, C, cuda_stream);
+}
+
+JOLT_API jolt_status jolt_selftest_eig_dense(int32_t batch, int32_t n, int32_t R, const double* A, double* V,
+                                             double* lam, void* cuda_stream) {
+  g_err.clear();
+  if (batch <= 0 || n < 2 || n > kExactMaxTokens || R < 1 || R > n || R > kMaxN || !A || !V || !lam)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_selftest_eig_dense: need batch >= 1, 2 <= n <= %d, 1 <= R <= min(n, %d)",
+                kExactMaxTokens, kMaxN);
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  double *a = nullptr, *tri = nullptr, *qx = nullptr, *gx = nullptr, *rx = nullptr;
+  int32_t* st = nullptr;
+  const size_t nn = (size_t)batch * n * n;
+  cudaError_t e = dev_malloc(&a, nn * sizeof(double));
+  if (e == cudaSuccess) e = dev_malloc(&tri, tridiag_scratch_doubles(batch, n, R) * sizeof(double));
+  if (e == cudaSuccess) e = dev_malloc(&qx, (size_t)batch * n * R * sizeof(double));
+  if (e == cudaSuccess) e = dev_malloc(&gx, (size_t)batch * R * R * sizeof(double));
+  if (e == cudaSuccess) e = dev_malloc(&rx, (size_t)batch * R * R * sizeof(double));
+  if (e == cudaSuccess) e = dev_malloc(&st, sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMemsetAsync(st, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(a, A, nn * sizeof(double), cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = dense_top_eig(batch, n, R, a, (int64_t)n * n, tri, qx, gx, rx, V, EL_F64, lam, st, s);
+  int32_t hs = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&hs, st, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  for (void* q : {(void*)a, (void*)tri, (void*)qx, (void*)gx, (void*)rx, (void*)st})
+    if (q) cudaFree(q);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_selftest_eig_dense: %s", cudaGetErrorString(e));
+  if (hs & ST_NOT_CONVERGED) return fail(JOLT_ERR_NOT_CONVERGED, "jolt_selftest_eig_dense: a Cholesky pivot was floored");
+  return JOLT_OK;
 }
 
 JOLT_API uint64_t jolt_launch_count(void) { return g_launches.load(); }

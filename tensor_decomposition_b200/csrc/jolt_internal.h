@@ -86,6 +86,15 @@ cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int
 cudaError_t eig_psd2(int batch0, int n0, const double* C0, int64_t sC0, float* V0, int64_t sV0, float* lam0,
                      int64_t sL0, int batch1, int n1, const double* C1, int64_t sC1, float* V1, int64_t sV1,
                      float* lam1, int64_t sL1, int max_sweeps, int32_t* status, cudaStream_t s);
+// Leading eigenpairs of batch dense symmetric n x n float64 matrices (A, batch stride sA; A is
+// overwritten) by Householder tridiagonalisation, bisection and inverse iteration (tridiag.cu):
+// on return *Z points at the R eigenvectors, [batch][n][tridiag_rpad(R)] float64 (column r,
+// eigenvalues descending; orthonormal to about eps ||A|| / gap), *lam at the R eigenvalues,
+// [batch][tridiag_rpad(R)]. Both live in `scratch` (tridiag_scratch_doubles doubles).
+int tridiag_rpad(int R);
+size_t tridiag_scratch_doubles(int batch, int n, int R);
+cudaError_t eig_top_dense(int batch, int n, int R, double* A, int64_t sA, double* scratch, double** Z,
+                         double** lam, cudaStream_t s);
 // Shifted-CholeskyQR helper: Rinv = inverse of chol(W + shift * trace(W)/n * I), W n x n.
 cudaError_t chol_inv(int batch, int n, const double* W, int64_t sW, double* Rinv, int64_t sR,
                      double shift, int32_t* status, cudaStream_t s);
@@ -179,7 +188,7 @@ struct ResidualArgs {
 cudaError_t residual_encode(const ResidualArgs& a, double* Pbuf, double* Nbuf, int R, cudaStream_t s);
 
 struct DecodeArgs {
-  int n_lt, H, T, D;
+  int n_lt, L, H, T, D;
   const int32_t* lt_ids;     // device [n_lt]
   void* out[2];              // K_out, V_out
   ElemType ot;
@@ -188,6 +197,26 @@ struct DecodeArgs {
   const uint8_t* body;
 };
 cudaError_t decode(const DecodeArgs& a, cudaStream_t s);
+
+// Attention over the compressed cache (attention.cu): out = softmax(scale Q K_hat^T) V_hat per
+// query, K_hat / V_hat never formed. Q, out: [L][Hq][n][D]; query head j reads KV head j / (Hq/H).
+struct AttnArgs {
+  int L, H, T, D, Hq, n, R;      // R: the stream's largest token rank (>= 1)
+  float scale;
+  const StreamMeta* meta;
+  const uint8_t* body;
+  const float* Pi;               // [D][D]
+  const __nv_bfloat16* Q;
+  float* out;
+  float* qpi;                    // scratch [L][Hq][n][D]
+  float* qhat;                   // scratch [L][Hq][n][R]
+  float* part;                   // scratch [L][H][nchunk][ngroups][attn_part_floats(R)]
+  int nchunk, ngroups;
+};
+int attn_groups(int Hq, int H, int n);
+int attn_chunks(int T);
+int attn_part_floats(int R);
+cudaError_t attention(const AttnArgs& a, cudaStream_t s);
 
 // Layout helpers of the tensor-core path (layout.cu).
 cudaError_t split_bf16(int64_t n, const float* x, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2,

@@ -24,6 +24,7 @@
 // Every wait is bounded: a timeout sets ST_TIMEOUT in the stream status and the CTA runs on
 // to its end without hanging.
 #include "../jolt_internal.h"
+#include "gemm_tc.h"
 #include "sm100.cuh"
 
 namespace jolt {
@@ -32,8 +33,10 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileRows = 128;
-constexpr int kProducers = 256;               // warps 4-11
-constexpr int kMmaWarp = 12;
+constexpr int kEpiWarps = 4;                  // warps 0-3: TMEM lane quadrant = warp
+constexpr int kProducers = 256;               // warps 8-15
+constexpr int kProdWarp0 = kEpiWarps;
+constexpr int kMmaWarp = kProdWarp0 + kProducers / 32;
 constexpr int kThreads = 32 * (kMmaWarp + 1);  // 13 warps
 constexpr int kOpBytes = 128 * 128 * 2;       // one 128 x 128 bf16 operand (two swizzle atoms)
 constexpr uint32_t kMaxPoll = 1u << 22;
@@ -58,6 +61,18 @@ __device__ __forceinline__ uint64_t slice_desc(uint32_t base, int kk) {
   return desc_kmajor_sw128(base + (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32));
 }
 
+// Tile store: the box at (c0, c1, c2) of `map` from shared memory (128-byte swizzled image), then
+// a commit of the bulk group; wait_group_read(0) before the shared memory is written again.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -81,7 +96,13 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
   return false;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
+// Output tensor maps: [L][H][T][128] bf16 as (128, T, L * H) with a 64 x 32 box (one epilogue
+// warp's rows, half of the features), 128-byte swizzle; used when the output is bf16.
+struct OutMaps {
+  CUtensorMap m[2];
+};
+
+__global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const __grid_constant__ OutMaps om) {
   extern __shared__ uint8_t smraw[];
   __shared__ __align__(8) uint64_t bar_pro, bar_afull[2], bar_a1free, bar_a2free[2];
   __shared__ __align__(8) uint64_t bar_accfull[2], bar_accempty[2];
@@ -113,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
       mbar_init(&bar_afull[j], kProducers);
       mbar_init(&bar_a2free[j], 1);
       mbar_init(&bar_accfull[j], 1);
-      mbar_init(&bar_accempty[j], 128);
+      mbar_init(&bar_accempty[j], 32 * kEpiWarps);
     }
     fence_barrier_init();
   }
@@ -194,12 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
   tc_fence_after();
 
   // ---------------------------------------------------------------- tiles of 128 rows
-  if (warp >= 4 && warp < kMmaWarp) {
+  if (warp >= kProdWarp0 && warp < kMmaWarp) {
     // producers: U_T rows -> A1, unpacked cell centres -> A2[tile parity]. Each thread takes 8
     // chunks of 8 codes (b bytes each, at byte u b of the tile's code block for chunk u); the
     // next tile's chunks (two aligned 8-byte words around each) and U_T rows are loaded into
     // registers before the current tile is unpacked.
-    const int pt = tid - 128;
+    const int pt = tid - 32 * kProdWarp0;
     const float inv2b = resid ? 1.0f / (float)(1 << b) : 0.0f;
     const float off2b = resid ? 1.0f - (float)(1 << b) : 0.0f;
     const uint64_t mask = resid ? (1ull << b) - 1ull : 0ull;
@@ -298,13 +319,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
       }
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // epilogue: TMEM lanes 32 warp .. 32 warp + 31 = rows of the tile
+  } else if (warp < kEpiWarps) {
+    // epilogue: TMEM lanes 32 warp .. 32 warp + 31 are rows of the tile
+    const int q4 = warp;
     const int layer = lt >> 1, kind = lt & 1;
     const int64_t obase = ((int64_t)layer * H + h) * T * 128;
+    // With r_t <= 64 the second halves of the two M_h^T parts are unused: each warp stages its
+    // 32 rows there as two boxes of 64 features (4 KB each, the 128-byte swizzled image of a box;
+    // features 0-63 in part 0's half, 64-127 in part 1's) and stores them with two tensor copies;
+    // otherwise every thread stores its row directly.
+    const bool staged = a.ot == EL_BF16 && rt <= 64;
+    uint8_t* stage0 = sm + kOffB1 + kOpBytes / 2 + warp * 4096;
     // the row's scale for tile it + 1 is loaded while tile it is waited for and stored
     auto load_scale = [&](int it2) {
-      const int t2 = it2 * kTileRows + 32 * warp + lane;
+      const int t2 = it2 * kTileRows + 32 * q4 + lane;
       return (resid && t2 < T) ? __half2float(scales[(int64_t)h * T + t2]) : 0.0f;
     };
     float s_next = load_scale(0);
@@ -314,9 +342,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
       if (it + 1 < ntiles) s_next = load_scale(it + 1);
       wait_or_flag(&bar_accfull[buf], (uint32_t)(use & 1), status);
       tc_fence_after();
-      const int t = it * kTileRows + 32 * warp + lane;
+      const int t = it * kTileRows + 32 * q4 + lane;
       const bool valid = t < T;
-      const uint32_t tb = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(buf * 256);
+      const uint32_t tb = tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(buf * 256);
+      if (staged) {
+        // the previous tile's tensor copy has read the staging buffer
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+      }
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t r1[32], r2[32];
@@ -330,7 +363,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
           if (resid) v = fmaf(s, __uint_as_float(r2[j]), v);
           o[j] = v;
         }
-        if (valid) {
+        if (staged) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int g = 4 * (c & 1) + q;     // 16-byte granule of the 128-byte box row
+            *reinterpret_cast<uint4*>(stage0 + (c >> 1) * kOpBytes + lane * 128 + ((g ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                           pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+          }
+        } else if (valid) {
           if (a.ot == EL_BF16) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out[kind]) + obase +
                                                   (int64_t)t * 128 + 32 * c);
@@ -348,7 +389,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a) {
       }
       tc_fence_before();
       mbar_arrive(&bar_accempty[buf]);
+      if (staged) {
+        fence_async_shared();
+        __syncwarp();
+        // rows beyond T fall outside the map and are not written
+        if (lane == 0) {
+          tma_store_3d(&om.m[kind], stage0, 0, it * kTileRows + 32 * q4, layer * H + h);
+          tma_store_3d(&om.m[kind], stage0 + kOpBytes, 64, it * kTileRows + 32 * q4, layer * H + h);
+        }
+      }
     }
+    if (staged && lane == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -365,8 +416,16 @@ cudaError_t decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.n_lt <= 0 || a.T <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(k_decode_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
+  OutMaps om;
+  memset(&om, 0, sizeof(om));
+  if (a.ot == EL_BF16) {
+    const uint64_t dims[3] = {128, (uint64_t)a.T, (uint64_t)a.L * a.H};
+    const uint64_t str[2] = {256, (uint64_t)a.T * 256};
+    for (int k = 0; k < 2; ++k)
+      if (a.out[k] && !tc_map_bf16_rows32(&om.m[k], a.out[k], 3, dims, str)) return cudaErrorInvalidValue;
+  }
   const dim3 g(a.H, a.n_lt);
-  k_decode_tc<<<g, kThreads, kSmemBytes, s>>>(a);
+  k_decode_tc<<<g, kThreads, kSmemBytes, s>>>(a, om);
   note_launch();
   return cudaGetLastError();
 }

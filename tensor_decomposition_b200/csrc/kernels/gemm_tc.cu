@@ -453,6 +453,10 @@ bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
   return map_box(map, base, rank, dims, strides, kTile);   // 64 K x 128 rows
 }
 
+bool tc_map_bf16_rows32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides) {
+  return map_box(map, base, rank, dims, strides, 32);      // 64 entries x 32 rows
+}
+
 bool tc_map_bf16_x_mn(CUtensorMap* map, const void* X, int64_t L, int64_t H, int64_t T, int64_t D) {
   if (L <= 0 || H <= 0 || T <= 0 || D <= 0 || D % 8) return false;
   const uint64_t dims[4] = {(uint64_t)D, (uint64_t)T, (uint64_t)H, (uint64_t)L};

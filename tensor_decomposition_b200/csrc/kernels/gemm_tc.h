@@ -65,6 +65,9 @@ struct TcGemmParams {
 // entry point is missing or an alignment rule fails.
 bool tc_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides);
 
+// The same with a 64 x 32 box (tiles of 32 rows, e.g. one warp's rows of a stored tile).
+bool tc_map_bf16_rows32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides);
+
 // [batch][K][rows] bf16 (rows contiguous, rows a multiple of 8) as the 3-D map (rows, K, batch)
 // with a 64 x 64 box, for VIEW_MN operands.
 bool tc_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t batch);

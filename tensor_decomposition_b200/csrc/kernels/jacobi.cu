@@ -671,6 +671,9 @@ __global__ void __launch_bounds__(32 * W) k_eig_psd(EigBatch b0, EigBatch b1, in
         for (int s = 0; s < S; ++s) {
           const double cs = __shfl_sync(0xffffffffu, c, GL * s);
           const double ss = __shfl_sync(0xffffffffu, sn, GL * s);
+          // a slot whose pair does not rotate has (c, s) = (1, 0) exactly: skipping it leaves the
+          // same bits (the branch is uniform over the warp)
+          if (ss == 0.0) continue;
           double* tp = top[(s - K + S) % S];
           double* bp = bot[(s + K) % S];
 #pragma unroll

@@ -30,7 +30,8 @@ EXPORTED = ["jolt_config_default", "jolt_plan", "jolt_plan_info", "jolt_encode",
             "jolt_rel_frob_error", "jolt_rel_frob_error_noalloc", "jolt_stream_status",
             "jolt_stream_info", "jolt_stream_to_host", "jolt_stream_from_host", "jolt_export_debug", "jolt_stream_destroy",
             "jolt_plan_destroy", "jolt_last_error", "jolt_profile_enable", "jolt_profile_report",
-            "jolt_launch_count", "jolt_alloc_count", "jolt_selftest_gemm_bf16", "jolt_selftest_gemm_bf16_layout"]
+            "jolt_launch_count", "jolt_alloc_count", "jolt_selftest_gemm_bf16", "jolt_selftest_gemm_bf16_layout",
+            "jolt_selftest_eig_dense", "jolt_attention"]
 
 
 class JoltError(RuntimeError):
@@ -80,6 +81,8 @@ def _load():
         "jolt_alloc_count": (u64, []),
         "jolt_selftest_gemm_bf16": (st, [i32, i32, i32, vp, vp, vp, vp]),
         "jolt_selftest_gemm_bf16_layout": (st, [i32, i32, i32, vp, i32, vp, i32, vp, vp]),
+        "jolt_selftest_eig_dense": (st, [i32, i32, i32, vp, vp, vp, vp]),
+        "jolt_attention": (st, [vp, vp, i32, i32, ctypes.c_float, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -268,3 +271,17 @@ def jolt_selftest_gemm_bf16_layout(A, a_mn, B, b_mn, C, cuda_stream=None):
     N = B.shape[1] if b_mn else B.shape[0]
     _check(_lib.jolt_selftest_gemm_bf16_layout(M, N, K, _dptr(A), int(bool(a_mn)), _dptr(B), int(bool(b_mn)),
                                                _dptr(C), _stream_ptr(cuda_stream)))
+
+
+def jolt_selftest_eig_dense(A, R, V, lam, cuda_stream=None):
+    """A: [batch][n][n] float64 CUDA tensor; V: [batch][n][R] and lam: [batch][R] float64 outputs."""
+    _check(_lib.jolt_selftest_eig_dense(int(A.shape[0]), int(A.shape[1]), int(R), _dptr(A), _dptr(V), _dptr(lam),
+                                        _stream_ptr(cuda_stream)))
+
+
+def jolt_attention(stream: Stream, Q, out, scale: float, cuda_stream=None):
+    """Q: bf16 CUDA tensor [layers][q_heads][n][head_dim]; out: float32 CUDA tensor of the same shape."""
+    if Q.dim() != 4 or tuple(out.shape) != tuple(Q.shape):
+        raise ValueError("Q and out must be [layers][q_heads][n][head_dim] of the same shape")
+    _check(_lib.jolt_attention(stream.handle, _dptr(Q), int(Q.shape[1]), int(Q.shape[2]), float(scale), _dptr(out),
+                               _stream_ptr(cuda_stream)))
