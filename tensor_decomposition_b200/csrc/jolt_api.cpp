@@ -257,6 +257,7 @@ struct jolt_plan_s {
   int q_iters = 1;                                       // power iterations of the subspace iteration
   bool exact_dense = false;                              // exact token factor by the dense eigensolver (T > 128)
   double* tri = nullptr;                                 // its scratch (tridiag_scratch_doubles)
+  float* CTpart = nullptr;                               // per-head token Gram partials [n][H][T][T] (tensor cores)
   double *Qx = nullptr, *Gx = nullptr, *Rx = nullptr;    // its CholeskyQR: [n][T][R], [n][R][R] x 2
   float* Wf = nullptr;                                   // float32 CholeskyQR Grams
   __nv_bfloat16* UDt = nullptr;                          // U_D^T (rounded factor, exact in bf16)
@@ -745,6 +746,7 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
       take(p->lamB, n * l);
     } else {
       take(p->CT, n * T * T);
+      if (p->exact_dense && p->use_tc) take(p->CTpart, n * H * T * T);
       if (p->exact_dense) {
         take(p->tri, tridiag_scratch_doubles((int)n, T, (int)Rm));
         take(p->Qx, n * T * Rm);
@@ -1216,7 +1218,27 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
                      outd(p->P, EL_F32, I1((int64_t)R * D), I1(D), I1(1)), 1.0, 0.0, s));
       }
     } else {
-      {
+      if (p->use_tc && p->CTpart) {
+        PROF("token_gram", s);
+        // exact: C_T = sum_h X_h X_h^T. Per-head partials on the tensor cores (rows t, K = the
+        // head's 128 features, one K chunk per head: the bf16 products are exact, the float32 sum
+        // runs over 128 terms), summed over the heads in float64.
+        for (int k = 0; k < kinds; ++k) {
+          TcGemmParams g;
+          g.status = status;
+          g.amap[0] = mx[k];
+          g.bmap[0] = mx[k];
+          g.av.mode = g.bv.mode = VIEW_X_TOKENROWS;
+          g.av.D = g.bv.D = D;
+          g.av.nch = g.bv.nch = H;
+          g.av.ckb = g.bv.ckb = D / 64;
+          g.M = T; g.N = T; g.KB = D / 64;
+          g.C = p->CTpart + (int64_t)k * L * H * T * T;
+          g.c_sm = T; g.c_sn = 1; g.c_sb = (int64_t)T * T;
+          CK(gemm_tc(L * H, g, s));
+        }
+        CK(sum_heads(n, H, (int64_t)T * T, p->CTpart, nullptr, p->CT, s));
+      } else {
         PROF("token_gram", s);
         // exact: C_T = A A^T (T x T), all eigenvectors, keep the leading R
         for (int k = 0; k < kinds; ++k)
@@ -1246,7 +1268,28 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
         CK(sign_fix(n, T, R, p->UT32, R, (int64_t)T * R, nullptr, 0, 0, 0, s));
         CK(round_bf16((int64_t)n * T * R, p->UT32, p->UTb, p->UTf, s));
       }
-      {
+      if (p->use_tc && p->CTpart && T <= 2048) {
+        PROF("core", s);
+        // P[h] = U_T(rounded)^T X_h (R x D) on the tensor cores: U_T is exact in bf16 (one part,
+        // MN-major from its [T][R] layout, shared by the heads), X_h MN-major in place
+        for (int k = 0; k < kinds; ++k) {
+          TcGemmParams g;
+          g.status = status;
+          if (!tc_map_bf16_mn(&g.amap[0], p->UTb + (int64_t)k * L * T * R, R, T, L))
+            return fail(JOLT_ERR_CUDA, "tensor map rejected");
+          g.bmap[0] = mxm[k];
+          g.av.mode = VIEW_MN;
+          g.av.H = H;
+          g.av.D = 0;
+          g.bv.mode = VIEW_MN_XHEAD;
+          g.bv.H = H;
+          g.bv.D = D;
+          g.M = R; g.N = D; g.KB = (T + 63) / 64;
+          g.C = p->P + (int64_t)k * L * H * R * D;
+          g.c_sm = D; g.c_sn = 1; g.c_sb = (int64_t)R * D;
+          CK(gemm_tc(L * H, g, s));
+        }
+      } else {
         PROF("core", s);
         // P[h] = U_T(rounded)^T X_h  (R x D)
         for (int k = 0; k < kinds; ++k)

@@ -118,19 +118,53 @@ __global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int6
       }
       __syncthreads();
       // 3. y = (A - V W^T - W V^T) v over rows and columns k + 1 .. n - 1; A is the matrix as at
-      // the start of the panel. One thread per column (rows read in order: coalesced).
-      for (int col = k + 1 + tid; col < n; col += kSyThreads) {
-        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-        const double* Ac = A + col;
-        int i = k + 1;
-        for (; i + 3 < n; i += 4) {
-          a0 = fma(Ac[(int64_t)i * n], cs[i], a0);
-          a1 = fma(Ac[(int64_t)(i + 1) * n], cs[i + 1], a1);
-          a2 = fma(Ac[(int64_t)(i + 2) * n], cs[i + 2], a2);
-          a3 = fma(Ac[(int64_t)(i + 3) * n], cs[i + 3], a3);
+      // the start of the panel. A thread takes two adjacent columns (one 16-byte load per row;
+      // the pair starts at an even column, the one below k + 1 is computed and dropped) and
+      // keeps sixteen rows' loads in flight; the rows are read in order, so a row of the block's
+      // loads is one contiguous stretch.
+      if (n & 1) {
+        // odd order: rows are not 16-byte aligned pairs; one column per thread
+        for (int col = k + 1 + tid; col < n; col += kSyThreads) {
+          double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+          const double* Ac = A + col;
+          int i = k + 1;
+          for (; i + 3 < n; i += 4) {
+            a0 = fma(Ac[(int64_t)i * n], cs[i], a0);
+            a1 = fma(Ac[(int64_t)(i + 1) * n], cs[i + 1], a1);
+            a2 = fma(Ac[(int64_t)(i + 2) * n], cs[i + 2], a2);
+            a3 = fma(Ac[(int64_t)(i + 3) * n], cs[i + 3], a3);
+          }
+          for (; i < n; ++i) a0 = fma(Ac[(int64_t)i * n], cs[i], a0);
+          ys[col] = (a0 + a1) + (a2 + a3);
         }
-        for (; i < n; ++i) a0 = fma(Ac[(int64_t)i * n], cs[i], a0);
-        ys[col] = (a0 + a1) + (a2 + a3);
+      } else {
+        const int c0 = (k + 1) & ~1;
+        for (int col = c0 + 2 * tid; col < n; col += 2 * kSyThreads) {
+          double ax[8], ay[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ax[u] = ay[u] = 0.0;
+          const double* Ac = A + col;
+          int i = k + 1;
+          for (; i + 15 < n; i += 16) {
+            double2 t[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) t[u] = *reinterpret_cast<const double2*>(Ac + (int64_t)(i + u) * n);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              ax[u & 7] = fma(t[u].x, cs[i + u], ax[u & 7]);
+              ay[u & 7] = fma(t[u].y, cs[i + u], ay[u & 7]);
+            }
+          }
+          for (; i < n; ++i) {
+            const double2 t = *reinterpret_cast<const double2*>(Ac + (int64_t)i * n);
+            ax[0] = fma(t.x, cs[i], ax[0]);
+            ay[0] = fma(t.y, cs[i], ay[0]);
+          }
+          const double sx = ((ax[0] + ax[1]) + (ax[2] + ax[3])) + ((ax[4] + ax[5]) + (ax[6] + ax[7]));
+          const double sy = ((ay[0] + ay[1]) + (ay[2] + ay[3])) + ((ay[4] + ay[5]) + (ay[6] + ay[7]));
+          if (col >= k + 1) ys[col] = sx;
+          ys[col + 1] = sy;
+        }
       }
       // W^T v and V^T v for the panel's earlier columns (warp l takes column l)
       for (int l = warp; l < j; l += kSyThreads / 32) {
