@@ -410,6 +410,51 @@ def decode_sweep(J, dev, peaks, reps=5, warmup=2):
                                           "(2 B per entry) + compressed stream read", "by_ratio": out}
 
 
+def attention_record(J, cfg, ratio, dev, peaks, q_heads=32, n_queries=1, reps=10, warmup=2):
+    """Attention over the compressed cache (one decoding step's attention for every layer): one
+    stream encoded at `ratio`, then `reps` calls of jolt_attention with q_heads x n_queries bf16
+    queries per layer (CUDA events). Reports the cached tokens attended per second and the stream
+    bytes read per second against the HBM peak (the kernel reads each layer's codes, scales and
+    factors once), beside the bf16 bytes a dense attention over the decoded cache would read."""
+    import torch
+    import synth
+    K, V = synth.gen_cache_torch(cfg, dev)
+    c = J.jolt_config_default()
+    c.encoder = J.JOLT_ENC_SKETCH
+    c.rt_max = RT_MAX
+    c.split_kv_budget = int(cfg.split_kv)
+    plan = J.jolt_plan(cfg.layers, cfg.heads, cfg.tokens, cfg.head_dim, cfg.has_v, J.JOLT_BF16,
+                       synth.kv.budget_bytes(cfg, ratio), cfg.groups, c)
+    st = J.jolt_encode(plan, K, V, SEED)
+    J.jolt_stream_status(st)
+    sbytes = int(sum(J.jolt_stream_info(st, cfg.groups)["bytes_by_part"].values()))
+    del K, V
+    g = torch.Generator(device=dev).manual_seed(5)
+    Q = torch.randn((cfg.layers, q_heads, n_queries, cfg.head_dim), generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    for _ in range(warmup):
+        J.jolt_attention(st, Q, out, scale)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        J.jolt_attention(st, Q, out, scale)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    gbs = sbytes / (ms / 1e3) / 1e9
+    dense = 2 * cfg.layers * cfg.heads * cfg.tokens * cfg.head_dim * 2
+    del st, plan, Q, out
+    torch.cuda.empty_cache()
+    return {"workload": cfg.name, "ratio": ratio, "q_heads": q_heads, "n_queries": n_queries, "ms": ms,
+            "cached_tokens_per_s": cfg.tokens / (ms / 1e3), "stream_bytes": sbytes, "GB_per_s": gbs,
+            "hbm_peak_GB_per_s": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+            "dense_bf16_bytes": dense,
+            "note": "bytes = the compressed stream (codes, scales, factors) read once; a dense attention over "
+                    "the decoded bf16 cache would read dense_bf16_bytes"}
+
+
 def job_throughput(local_ms, tokens, steps, world, device):
     """Whole-job throughput of a weak-scaling run. Every rank processed `tokens` tokens per step
     for `steps` steps; the job takes as long as its slowest rank (a MAX all-reduce over the
@@ -505,6 +550,12 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks, q=1):
                             "each (Golub & Van Loan count), float64 one-sided Jacobi: FP64 peak"),
         "cholqr": dict(bound="tensor", work=cholqr_flops / 1e12, unit="TFLOP/s", peak=peaks["bf16_tflops"] * 0.5,
                        note="per pass 4 rows l^2 flops (Gram + triangular update) on float32 data: tf32 peak = bf16 x 1/2"),
+        "token_gram": dict(bound="tensor", work=2.0 * T * T * H * D * n_lt / 1e12, unit="TFLOP/s",
+                           peak=peaks["bf16_tflops"], note="C_T = sum_h X_h X_h^T: 2 T^2 HD flops per layer-tensor"),
+        "token_eig": dict(bound="alu", work=(4.0 / 3.0 * T ** 3 + 2.0 * T * T * plan_info["rt_max"]) * n_lt / 1e12,
+                          unit="TFLOP/s", peak=fp64_peak,
+                          note="dense symmetric eigensolver for the R leading eigenpairs of C_T: 4 T^3 / 3 flops "
+                               "(Householder tridiagonalisation) + 2 T^2 R (back-transformation), float64: FP64 peak"),
     }, stream_bytes
 
 
@@ -684,6 +735,8 @@ def main():
             "note": "the exact token factor above 128 tokens is realised as subspace iteration with 24 power "
                     "iterations (one for the sketch); the pages' FlashJoLT speedup at 1024 tokens is 5-13x"}
         out["decode_sweep"] = decode_sweep(J, dev, peaks)
+        out["attention"] = [attention_record(J, synth.config(1), 2.0, dev, peaks),
+                            attention_record(J, synth.config(4), 2.0, dev, peaks)]
     if args.profile_out and rank == 0:
         json.dump(prof, open(args.profile_out, "w"), indent=1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

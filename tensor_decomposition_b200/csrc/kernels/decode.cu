@@ -34,7 +34,7 @@ using namespace sm100;
 
 constexpr int kTileRows = 128;
 constexpr int kEpiWarps = 4;                  // warps 0-3: TMEM lane quadrant = warp
-constexpr int kProducers = 256;               // warps 8-15
+constexpr int kProducers = 256;               // warps 4-11
 constexpr int kProdWarp0 = kEpiWarps;
 constexpr int kMmaWarp = kProdWarp0 + kProducers / 32;
 constexpr int kThreads = 32 * (kMmaWarp + 1);  // 13 warps
