@@ -66,6 +66,8 @@ typedef enum { JOLT_BF16 = 0, JOLT_F32 = 1 } jolt_dtype;
 
 typedef enum { JOLT_ENC_AUTO = 0, JOLT_ENC_EXACT = 1, JOLT_ENC_SKETCH = 2 } jolt_encoder;
 
+typedef enum { JOLT_EIG_TRIDIAG = 0, JOLT_EIG_JACOBI = 1 } jolt_eig_solver;
+
 /* Shape of one sequence's cache. `dtype` is both the input and the decoded output type. */
 typedef struct {
   int32_t layers, heads, tokens, head_dim;
@@ -83,7 +85,7 @@ typedef struct {
                                 (see the preamble); plans need R <= 112 */
   uint32_t bits_mask;        /* bit b set => residual bit-width b allowed (0x1FF = 0..8) */
   int32_t split_kv_budget;   /* 0: one budget pool for K and V; 1: half the budget each */
-  int32_t max_jacobi_sweeps; /* eigensolver sweep limit (30) */
+  int32_t max_jacobi_sweeps; /* sweep limit of the Jacobi eigensolver (30; eig_solver = JACOBI) */
   int32_t factors;           /* 1 (default): Tucker factors on the candidate grid; 0: residual
                                 only, r_t = r_d = 0 for every layer-tensor (with bits_mask = 1 << b
                                 this is per-row b-bit quantisation of the rotated cache, the
@@ -98,6 +100,10 @@ typedef struct {
                                 1: randomized Hadamard Pi = diag(s) H / sqrt(D), s random signs of
                                 the seed's rotation stream, H the Sylvester Hadamard matrix (D a
                                 power of two); recorded in the stream header */
+  jolt_eig_solver eig_solver; /* solver of the feature and sketch eigenproblems (n <= 128):
+                                TRIDIAG (default): Householder tridiagonalisation, bisection,
+                                twisted-factorisation vectors, back-transformation; JACOBI:
+                                one-sided Jacobi on a Cholesky factor, to convergence */
 } jolt_config;
 
 typedef struct jolt_plan_s* jolt_plan_t;
@@ -283,6 +289,17 @@ JOLT_API jolt_status jolt_selftest_gemm_bf16_layout(int32_t M, int32_t N, int32_
  * dependent for the re-orthonormalisation. */
 JOLT_API jolt_status jolt_selftest_eig_dense(int32_t batch, int32_t n, int32_t R, const double* A, double* V,
                                              double* lam, void* cuda_stream);
+
+/* jolt_selftest_eig_small - all n eigenpairs of `batch` dense symmetric n x n float64 matrices by
+ * the solver of the feature and sketch eigenproblems (`solver`: JOLT_EIG_TRIDIAG or
+ * JOLT_EIG_JACOBI), exposed so its numerics can be tested alone.
+ * A: device float64 [batch][n][n] (the lower triangle is read), V: device float32 [batch][n][n]
+ * (eigenvector r in column r), lam: device float32 [batch][n], eigenvalues descending.
+ * 1 <= n <= 128. Synchronises
+ * `cuda_stream`; NOT_CONVERGED when Jacobi reached its sweep limit, NONFINITE for a non-finite
+ * input or result. */
+JOLT_API jolt_status jolt_selftest_eig_small(int32_t batch, int32_t n, const double* A, float* V, float* lam,
+                                             int32_t solver, void* cuda_stream);
 
 /* Release a stream. Its device memory is freed in order on the CUDA stream the stream was
  * created on (encode or jolt_stream_from_host); synchronise any other CUDA stream that still

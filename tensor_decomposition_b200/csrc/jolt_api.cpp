@@ -548,6 +548,7 @@ JOLT_API void jolt_config_default(jolt_config* c) {
   c->rotation = 0;
   c->split_kv_budget = 0;
   c->max_jacobi_sweeps = 30;
+  c->eig_solver = JOLT_EIG_TRIDIAG;
 }
 
 JOLT_API const char* jolt_last_error(void) { return g_err.c_str(); }
@@ -576,6 +577,8 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
   if ((cfg.bits_mask & 0x1FFu) == 0 || (cfg.bits_mask & ~0x1FFu))
     return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: bits_mask must select widths in 0..8");
   if (cfg.rt_max < 0) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: rt_max < 0");
+  if (cfg.eig_solver != JOLT_EIG_TRIDIAG && cfg.eig_solver != JOLT_EIG_JACOBI)
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: eig_solver must be TRIDIAG (0) or JACOBI (1)");
   if (cfg.factors != 0 && cfg.factors != 1) return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: factors must be 0 or 1");
   if (cfg.measured_b != 0 && cfg.measured_b != 1)
     return fail(JOLT_ERR_INVALID_ARG, "jolt_plan: measured_b must be 0 or 1");
@@ -888,8 +891,12 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
   };
   auto eig_feature_and = [&](int n1, const double* C1, float* V1, float* lam1) -> jolt_status {
     PROF("jacobi", s);
-    CK(eig_psd2(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, n1 > 0 ? n : 0, n1, C1,
-                (int64_t)n1 * n1, V1, (int64_t)n1 * n1, lam1, n1, p->cfg.max_jacobi_sweeps, status, s));
+    if (p->cfg.eig_solver == JOLT_EIG_JACOBI)
+      CK(eig_psd2(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, n1 > 0 ? n : 0, n1, C1,
+                  (int64_t)n1 * n1, V1, (int64_t)n1 * n1, lam1, n1, p->cfg.max_jacobi_sweeps, status, s));
+    else
+      CK(eig_small2(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, n1 > 0 ? n : 0, n1, C1,
+                    (int64_t)n1 * n1, V1, (int64_t)n1 * n1, lam1, n1, status, s));
     return JOLT_OK;
   };
   if (R == 0) {
@@ -1886,6 +1893,31 @@ JOLT_API jolt_status jolt_selftest_eig_dense(int32_t batch, int32_t n, int32_t R
     if (q) cudaFree(q);
   if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_selftest_eig_dense: %s", cudaGetErrorString(e));
   if (hs & ST_NOT_CONVERGED) return fail(JOLT_ERR_NOT_CONVERGED, "jolt_selftest_eig_dense: a Cholesky pivot was floored");
+  return JOLT_OK;
+}
+
+JOLT_API jolt_status jolt_selftest_eig_small(int32_t batch, int32_t n, const double* A, float* V, float* lam,
+                                             int32_t solver, void* cuda_stream) {
+  g_err.clear();
+  if (batch <= 0 || n < 1 || n > kMaxN || !A || !V || !lam ||
+      (solver != JOLT_EIG_TRIDIAG && solver != JOLT_EIG_JACOBI))
+    return fail(JOLT_ERR_INVALID_ARG, "jolt_selftest_eig_small: need batch >= 1, 1 <= n <= %d, solver 0 or 1", kMaxN);
+  cudaStream_t s = (cudaStream_t)cuda_stream;
+  int32_t* st = nullptr;
+  cudaError_t e = dev_malloc(&st, sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMemsetAsync(st, 0, sizeof(int32_t), s);
+  const int64_t nn = (int64_t)n * n;
+  if (e == cudaSuccess)
+    e = solver == JOLT_EIG_JACOBI
+            ? eig_psd2(batch, n, A, nn, V, nn, lam, n, 0, 0, nullptr, 0, nullptr, 0, nullptr, 0, 30, st, s)
+            : eig_small2(batch, n, A, nn, V, nn, lam, n, 0, 0, nullptr, 0, nullptr, 0, nullptr, 0, st, s);
+  int32_t hs = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&hs, st, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (st) cudaFree(st);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "jolt_selftest_eig_small: %s", cudaGetErrorString(e));
+  if (hs & ST_NONFINITE) return fail(JOLT_ERR_NONFINITE, "jolt_selftest_eig_small: non-finite input or result");
+  if (hs & ST_NOT_CONVERGED) return fail(JOLT_ERR_NOT_CONVERGED, "jolt_selftest_eig_small: Jacobi sweep limit");
   return JOLT_OK;
 }
 

@@ -86,6 +86,12 @@ cudaError_t eig_psd(int batch, int n, const double* C, int64_t sC, float* V, int
 cudaError_t eig_psd2(int batch0, int n0, const double* C0, int64_t sC0, float* V0, int64_t sV0, float* lam0,
                      int64_t sL0, int batch1, int n1, const double* C1, int64_t sC1, float* V1, int64_t sV1,
                      float* lam1, int64_t sL1, int max_sweeps, int32_t* status, cudaStream_t s);
+// The same two-batch eigenproblems by Householder tridiagonalisation, bisection, twisted
+// factorisations and back-transformation (eig_small.cu); any n <= 128, status flags
+// ST_NONFINITE for a non-finite input or result.
+cudaError_t eig_small2(int batch0, int n0, const double* C0, int64_t sC0, float* V0, int64_t sV0, float* lam0,
+                       int64_t sL0, int batch1, int n1, const double* C1, int64_t sC1, float* V1, int64_t sV1,
+                       float* lam1, int64_t sL1, int32_t* status, cudaStream_t s);
 // Leading eigenpairs of batch dense symmetric n x n float64 matrices (A, batch stride sA; A is
 // overwritten) by Householder tridiagonalisation, bisection and inverse iteration (tridiag.cu):
 // on return *Z points at the R eigenvectors, [batch][n][tridiag_rpad(R)] float64 (column r,

@@ -21,6 +21,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "BUDGET_INFEASIBLE", 3: "OOM", 4: 
                 9: "UNSUPPORTED"}
 JOLT_BF16, JOLT_F32 = 0, 1
 JOLT_ENC_AUTO, JOLT_ENC_EXACT, JOLT_ENC_SKETCH = 0, 1, 2
+JOLT_EIG_TRIDIAG, JOLT_EIG_JACOBI = 0, 1
 JOLT_ROT_HAAR, JOLT_ROT_HADAMARD = 0, 1
 JOLT_DBG_PI, JOLT_DBG_UT_F32, JOLT_DBG_UD_F32, JOLT_DBG_TABLE, JOLT_DBG_XX, JOLT_DBG_LAMBDA, \
     JOLT_DBG_OMEGA, JOLT_DBG_MEAS = range(8)
@@ -31,7 +32,7 @@ EXPORTED = ["jolt_config_default", "jolt_plan", "jolt_plan_info", "jolt_encode",
             "jolt_stream_info", "jolt_stream_to_host", "jolt_stream_from_host", "jolt_export_debug", "jolt_stream_destroy",
             "jolt_plan_destroy", "jolt_last_error", "jolt_profile_enable", "jolt_profile_report",
             "jolt_launch_count", "jolt_alloc_count", "jolt_selftest_gemm_bf16", "jolt_selftest_gemm_bf16_layout",
-            "jolt_selftest_eig_dense", "jolt_attention"]
+            "jolt_selftest_eig_dense", "jolt_selftest_eig_small", "jolt_attention"]
 
 
 class JoltError(RuntimeError):
@@ -50,7 +51,8 @@ class Config(ctypes.Structure):
                 ("power_iters", ctypes.c_int32), ("rank_step", ctypes.c_int32),
                 ("rt_max", ctypes.c_int32), ("bits_mask", ctypes.c_uint32),
                 ("split_kv_budget", ctypes.c_int32), ("max_jacobi_sweeps", ctypes.c_int32),
-                ("factors", ctypes.c_int32), ("measured_b", ctypes.c_int32), ("rotation", ctypes.c_int32)]
+                ("factors", ctypes.c_int32), ("measured_b", ctypes.c_int32), ("rotation", ctypes.c_int32),
+                ("eig_solver", ctypes.c_int32)]
 
 
 def _load():
@@ -82,6 +84,7 @@ def _load():
         "jolt_selftest_gemm_bf16": (st, [i32, i32, i32, vp, vp, vp, vp]),
         "jolt_selftest_gemm_bf16_layout": (st, [i32, i32, i32, vp, i32, vp, i32, vp, vp]),
         "jolt_selftest_eig_dense": (st, [i32, i32, i32, vp, vp, vp, vp]),
+        "jolt_selftest_eig_small": (st, [i32, i32, vp, vp, vp, i32, vp]),
         "jolt_attention": (st, [vp, vp, i32, i32, ctypes.c_float, vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -271,6 +274,12 @@ def jolt_selftest_gemm_bf16_layout(A, a_mn, B, b_mn, C, cuda_stream=None):
     N = B.shape[1] if b_mn else B.shape[0]
     _check(_lib.jolt_selftest_gemm_bf16_layout(M, N, K, _dptr(A), int(bool(a_mn)), _dptr(B), int(bool(b_mn)),
                                                _dptr(C), _stream_ptr(cuda_stream)))
+
+
+def jolt_selftest_eig_small(A, V, lam, solver=0, cuda_stream=None):
+    """A: [batch][n][n] float64 CUDA tensor; V: [batch][n][n] and lam: [batch][n] float32 outputs."""
+    _check(_lib.jolt_selftest_eig_small(int(A.shape[0]), int(A.shape[1]), _dptr(A), _dptr(V), _dptr(lam),
+                                        int(solver), _stream_ptr(cuda_stream)))
 
 
 def jolt_selftest_eig_dense(A, R, V, lam, cuda_stream=None):

@@ -40,6 +40,7 @@ def test_config_defaults(jolt):
     c = jolt.jolt_config_default()
     assert (c.encoder, c.oversample, c.power_iters, c.rank_step, c.rt_max, c.bits_mask,
             c.split_kv_budget, c.max_jacobi_sweeps, c.factors, c.measured_b) == (0, 16, 1, 16, 0, 0x1FF, 0, 30, 1, 0)
+    assert c.eig_solver == jolt.JOLT_EIG_TRIDIAG
 
 
 @pytest.mark.parametrize("args", [
@@ -77,6 +78,23 @@ def test_plan_rejects_bad_options(jolt):
     c.factors = 2                    # 0 (residual only) or 1
     with pytest.raises(jolt.JoltError):
         jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 10 ** 6, 1, c)
+    c = jolt.jolt_config_default()
+    c.eig_solver = 2                 # TRIDIAG (0) or JACOBI (1)
+    with pytest.raises(jolt.JoltError):
+        jolt.jolt_plan(2, 8, 64, 128, True, jolt.JOLT_BF16, 10 ** 6, 1, c)
+
+
+@pytest.mark.parametrize("batch,n,solver", [(0, 16, 0), (1, 0, 0), (1, 129, 0), (1, 16, 2)])
+def test_eig_small_selftest_rejects_bad_sizes(jolt, batch, n, solver):
+    """The small eigensolver self-test checks its arguments before any device call."""
+    lib = ctypes.CDLL(jolt.LIB_PATH)
+    f = lib.jolt_selftest_eig_small
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_int32, ctypes.c_void_p]
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert f(batch, n, p, p, p, solver, None) == 1
 
 
 def test_stream_from_host_rejects_corrupt_buffers(jolt):
