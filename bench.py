@@ -484,7 +484,6 @@ def config_dict(cfg, args):
 # hex digits of the sha256 of the kernel's source file when it was captured: reported only
 # while that file is unchanged (profiles/launch_list_c1_mistral7b_2x_sketch.md).
 NCU_TRAFFIC = {
-    "jacobi": ("tensor_decomposition_b200/csrc/kernels/jacobi.cu", "0d23bba0b65e8d05", 9_553_024),
     "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "4a0da90ab5592dd5", 180_089_344),
     "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "35bee190c9fdc25f", 147_005_824),
 }
@@ -542,9 +541,10 @@ def phase_models(cfg, plan_info, alloc, ratio, peaks, q=1):
                               "FP64 peak 148 SMs x 64 FMA x 2 x max clock (the DMMA pipe reaches the same rate)"),
         "decode": dict(bound="hbm", work=(2.0 * N * n_lt + stream_bytes) / 1e9, unit="GB/s", peak=peaks["hbm_gbs"],
                        note="reads the stream, writes the bf16 cache: 2 N bytes per layer-tensor + stream bytes"),
-        "jacobi": dict(bound="alu", work=9.0 * (D ** 3 + l ** 3) * n_lt / 1e12, unit="TFLOP/s", peak=fp64_peak,
-                       note="feature (n = D) and sketch (n = l) symmetric eigenproblems with vectors, 9 n^3 flops "
-                            "each (Golub & Van Loan count), float64 one-sided Jacobi: FP64 peak"),
+        "small_eig": dict(bound="alu", work=9.0 * (D ** 3 + l ** 3) * n_lt / 1e12, unit="TFLOP/s", peak=fp64_peak,
+                          note="feature (n = D) and sketch (n = l) symmetric eigenproblems with vectors, 9 n^3 flops "
+                               "each (Golub & Van Loan count); float64 Householder tridiagonalisation, bisection, "
+                               "twisted-factorisation vectors and back-transformation, one CTA per matrix: FP64 peak"),
         "cholqr": dict(bound="tensor", work=cholqr_flops / 1e12, unit="TFLOP/s", peak=peaks["bf16_tflops"] * 0.5,
                        note="per pass 4 rows l^2 flops (Gram + triangular update) on float32 data: tf32 peak = bf16 x 1/2"),
         "token_gram": dict(bound="tensor", work=2.0 * T * T * H * D * n_lt / 1e12, unit="TFLOP/s",

@@ -890,7 +890,7 @@ static jolt_status analyse(jolt_plan_s* p, jolt_stream_s* st, const void* X[2], 
     return JOLT_OK;
   };
   auto eig_feature_and = [&](int n1, const double* C1, float* V1, float* lam1) -> jolt_status {
-    PROF("jacobi", s);
+    PROF("small_eig", s);
     if (p->cfg.eig_solver == JOLT_EIG_JACOBI)
       CK(eig_psd2(n, D, p->CD, (int64_t)D * D, p->UD32, (int64_t)D * D, p->lamD, D, n1 > 0 ? n : 0, n1, C1,
                   (int64_t)n1 * n1, V1, (int64_t)n1 * n1, lam1, n1, p->cfg.max_jacobi_sweeps, status, s));

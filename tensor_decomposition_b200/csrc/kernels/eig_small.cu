@@ -42,21 +42,23 @@ constexpr int kN = kMaxN;                  // padded order
 constexpr int kT = 512;                    // threads per matrix
 constexpr int kStage = kN + 1;             // row stride of the staged input
 constexpr double kEps = 2.220446049250313e-16;
-constexpr double kSturmFloor = 0x1p-60;    // |d_i - x| below this is raised to it (||T|| < 1)
+constexpr double kSturmFloor = 0x1p-60;    // added to |d_i - x| in the Sturm count (||T|| < 1)
 constexpr double kTwistPiv = 0x1p-400;     // smallest magnitude of a twisted-factorisation pivot
 constexpr double kClusterTol = 1e-8;       // relative to ||T||: orthogonality ~eps / 1e-8 outside clusters
 
-// Reflector k (rows k + 1 .. n - 1) is kept at Up[rbase(k) + row]: the bases are even (16-byte
-// aligned pairs of rows) and each reflector starts after the previous one ends.
-constexpr int kUp = 8448;
+// Reflector k is kept from the first row of the 32-row group holding row k + 1 to row kN - 1,
+// zeros up to row k and beyond row n - 1, at Up[ub[k] + row]: a thread reading its group's 32
+// rows of a reflector needs no mask. Every reflector takes a multiple of 32 entries, so the
+// pairs of rows are 16-byte aligned.
+constexpr int kUp = 10080;   // sum over k < kN - 2 of kN - 32 floor((k + 1) / 32)
 
 // shared memory, in doubles
 constexpr int kOffUp = 0;
 constexpr int kOffZ = kOffUp + kUp;             // Z: [kN][kN], vector c in column c
 constexpr int kOffD = kOffZ + kN * kN;          // d, e, e2, tau, lam, znrm
 constexpr int kOffX = kOffD + 6 * kN;           // the current column x, two buffers
-constexpr int kOffW = kOffX + 2 * kN;           // w
-constexpr int kOffP = kOffW + kN;               // partial sums [2][4][kN]; LU scratch of a cluster
+constexpr int kOffW = kOffX + 2 * kN;           // row k + 1 of A, two buffers
+constexpr int kOffP = kOffW + 2 * kN;           // partial sums [2][4][kN]; LU scratch of a cluster
 constexpr int kOffMisc = kOffP + 8 * kN;        // 64 scalars, then the reflector bases (kN ints)
 constexpr int kSmemDoubles = kOffMisc + 64 + kN / 2;
 static_assert(kOffZ + kN * kStage <= kOffX, "the staged input overlays Z and the vectors after it");
@@ -97,31 +99,61 @@ __device__ __forceinline__ double wmin(double v) {
   return v;
 }
 
-// Number of eigenvalues of T (diagonal d, squared subdiagonal e2) below x: sign changes along
-// p_0 = 1, p_1, ..., p_n (p_i the leading i x i minor of T - x I). A zero minor inside the
-// sequence adds exactly one change either way. |d_i - x| is floored at kSturmFloor (a change of
-// T far below eps ||T||, an exact zero counting as positive): across a split (e_i = 0) the
-// minors are products of the d_i - x, and repeated diagonal values hit exactly by x would
-// otherwise underflow them to zero between two rescalings, after which no sign change counts.
-__device__ __forceinline__ double sturm_term(double v) {
-  return fabs(v) >= kSturmFloor ? v : (v < 0.0 ? -kSturmFloor : kSturmFloor);
+// Rescale the pair (p, pp) by the power of two that brings the larger into [1, 2) (exact).
+__device__ __forceinline__ void rescale_pair(double& p, double& pp) {
+  const double m = fmax(fabs(p), fabs(pp));
+  const int ex = ((__double2hiint(m) >> 20) & 0x7ff) - 1023;
+  const double sc = __hiloint2double((1023 - ex) << 20, 0);   // 2^-ex
+  p *= sc;
+  pp *= sc;
 }
 
-__device__ __forceinline__ int sturm_below(int n, const double* d, const double* e2, double x) {
-  double pp = 1.0, p = sturm_term(d[0] - x);
-  int c = p < 0.0;
-  for (int i = 1; i < n; ++i) {
-    const double ti = sturm_term(d[i] - x);
-    const double pn = fma(ti, p, -(e2[i - 1] * pp));
-    c += (pn < 0.0) != (p < 0.0);
-    pp = p;
-    p = pn;
-    if ((i & 7) == 0) {
-      const double m = fmax(fabs(p), fabs(pp));
-      const int ex = ((__double2hiint(m) >> 20) & 0x7ff) - 1023;
-      const double sc = __hiloint2double((1023 - ex) << 20, 0);   // 2^-ex
-      p *= sc;
-      pp *= sc;
+// Number of eigenvalues of T below x: sign changes along p_{-1} = 1, p_0, ..., p_{n-1}, p_i the
+// leading (i + 1) x (i + 1) minor of T - x I, p_i = (d_i - x) p_{i-1} - f_i p_{i-2} with f_i =
+// e_{i-1}^2 (f_0 = 0). A zero minor inside the sequence adds exactly one change whichever sign it
+// is given. |d_i - x| is raised by kSturmFloor, keeping the sign bit (a change of T far below
+// eps ||T||): across a split (e_i = 0) the minors are products of the d_i - x, and a
+// repeated diagonal value hit exactly by x would otherwise underflow them to zero between two
+// rescalings, after which no sign change counts. d and f are padded to n8 (a multiple of 8) with
+// d_i = 4 > x and f_i = 0, which change no sign; eight terms per chunk, the next chunk's
+// coefficients loaded while the current one runs.
+__device__ __forceinline__ double sturm_term(double v) {
+  return v + copysign(kSturmFloor, v);   // (|v| + 2^-60) with the sign bit of v
+}
+
+__device__ __forceinline__ int sturm_below(int n8, const double* d, const double* f, double x) {
+  const double2* d2 = reinterpret_cast<const double2*>(d);
+  const double2* f2 = reinterpret_cast<const double2*>(f);
+  double p = 1.0, pp = 0.0;
+  int c = 0;
+  double2 dv[4], fv[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    dv[u] = d2[u];
+    fv[u] = f2[u];
+  }
+  for (int i0 = 0; i0 < n8; i0 += 8) {
+    const int nx = (i0 + 8 < n8 ? i0 + 8 : i0) >> 1;
+    double2 dn[4], fn[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      dn[u] = d2[nx + u];
+      fn[u] = f2[nx + u];
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const double dd = (u & 1) ? dv[u >> 1].y : dv[u >> 1].x;
+      const double ff = (u & 1) ? fv[u >> 1].y : fv[u >> 1].x;
+      const double pn = fma(sturm_term(dd - x), p, -(ff * pp));
+      c += (int)((unsigned)(__double2hiint(pn) ^ __double2hiint(p)) >> 31);
+      pp = p;
+      p = pn;
+    }
+    rescale_pair(p, pp);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      dv[u] = dn[u];
+      fv[u] = fn[u];
     }
   }
   return c;
@@ -132,30 +164,47 @@ __device__ __forceinline__ double twist_pivot(double v) {
 }
 
 // Eigenvector of T for the eigenvalue lmb by the twisted factorisation; z is column j of Z
-// (stride kN), used for the pivots on the way. Returns 1 / ||z||.
-__device__ double twisted_vector(int n, const double* d, const double* e, const double* e2, double lmb,
+// (stride kN), used for the pivots on the way. Returns 1 / ||z||. The forward pivots are
+// D+_i = p_i / p_{i-1} with p the leading minors of T - lmb I, the backward ones D-_i =
+// s_i / s_{i+1} with s the trailing minors (s_i = (d_i - lmb) s_{i+1} - f_{i+1} s_{i+2}): the
+// recurrences run on the minors (rescaled by powers of two every eight terms), so the divisions
+// stay off their dependency chains. A minor that comes out exactly zero is replaced by kTwistPiv
+// times the previous one (pivot +-kTwistPiv, as for the quotient form).
+__device__ double twisted_vector(int n, const double* d, const double* e, const double* f, double lmb,
                                  double* z) {
-  double Dp = twist_pivot(d[0] - lmb);
-  z[0] = Dp;
-  for (int i = 1; i < n; ++i) {
-    Dp = twist_pivot((d[i] - lmb) - e2[i - 1] / Dp);
-    z[i * kN] = Dp;
+  double p = 1.0, pp = 0.0;
+  for (int i = 0; i < n; ++i) {
+    double pn = fma(d[i] - lmb, p, -(f[i] * pp));
+    if (pn == 0.0) pn = kTwistPiv * p;
+    z[i * kN] = twist_pivot(pn / p);
+    pp = p;
+    p = pn;
+    if ((i & 7) == 7) rescale_pair(p, pp);
   }
-  double Dm = twist_pivot(d[n - 1] - lmb), best = fabs(z[(n - 1) * kN]);
+  double s = 1.0, ss = 0.0, best = 0.0;
   int r = n - 1;
-  for (int i = n - 2; i >= 0; --i) {
+  for (int i = n - 1; i >= 0; --i) {
     const double ti = d[i] - lmb;
-    Dm = twist_pivot(ti - e2[i] / Dm);
-    const double g = fabs(z[i * kN] + Dm - ti);
-    if (g < best) {
+    double sn = fma(ti, s, -((i + 1 < n ? f[i + 1] : 0.0) * ss));
+    if (sn == 0.0) sn = kTwistPiv * s;
+    const double g = fabs(z[i * kN] + twist_pivot(sn / s) - ti);
+    if (i == n - 1 || g < best) {
       best = g;
       r = i;
     }
+    ss = s;
+    s = sn;
+    if ((i & 7) == 0) rescale_pair(s, ss);
   }
-  Dm = twist_pivot(d[n - 1] - lmb);
+  s = 1.0;
+  ss = 0.0;
   for (int i = n - 1; i > r; --i) {
-    if (i < n - 1) Dm = twist_pivot((d[i] - lmb) - e2[i] / Dm);
-    z[i * kN] = Dm;
+    double sn = fma(d[i] - lmb, s, -((i + 1 < n ? f[i + 1] : 0.0) * ss));
+    if (sn == 0.0) sn = kTwistPiv * s;
+    z[i * kN] = twist_pivot(sn / s);
+    ss = s;
+    s = sn;
+    if ((i & 7) == 0) rescale_pair(s, ss);
   }
   double v = 1.0, nn = 1.0;
   z[r * kN] = 1.0;
@@ -306,8 +355,6 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
   int* ub = reinterpret_cast<int*>(misc + 64);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int i = t & (kN - 1), q = t >> 7, rb = warp & 3;
-  float* vo = sb.V + (int64_t)bi * sb.sV;
-  float* lo_out = sb.lam ? sb.lam + (int64_t)bi * sb.sL : nullptr;
 
   // ---- 1. the lower triangle staged in shared memory (coalesced), mirrored into registers
   const double* Cb = sb.C + (int64_t)bi * sb.sC;
@@ -316,10 +363,10 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
   for (int x = t; x < kUp; x += kT) Up[x] = 0.0;
   if (t == 0) {
     int base = 0;
-    ub[0] = 0;
-    for (int k = 1; k <= kN - 3; ++k) {
-      base = (base + kN - k - 1 + 1) & ~1;     // even, and base + k + 1 >= end of reflector k - 1
-      ub[k] = base;
+    for (int k = 0; k <= kN - 3; ++k) {
+      const int g0 = 32 * ((k + 1) >> 5);
+      ub[k] = base - g0;
+      base += kN - g0;
     }
   }
   __syncthreads();
@@ -341,6 +388,8 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
   __syncthreads();
   const double anorm = fmax(fmax(misc[0], misc[1]), fmax(misc[2], misc[3]));
   if (bad || anorm == 0.0) {
+    float* vo = sb.V + (int64_t)bi * sb.sV;
+    float* lo_out = sb.lam ? sb.lam + (int64_t)bi * sb.sL : nullptr;
     // a non-finite input gives NaN output and the status flag; the zero matrix has the unit
     // vectors and zero eigenvalues
     const float fill = bad ? __int_as_float(0x7fc00000) : 0.0f;
@@ -350,15 +399,22 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
     if (bad && t == 0 && status) atomicOr(status, ST_NONFINITE);
     return;
   }
-  int ex;
+  int ex;   // the scale 2^-ex (kept in shared memory until the output)
   frexp(anorm, &ex);
+  int* ex_s = reinterpret_cast<int*>(misc + 12);
+  if (t == 0) *ex_s = ex;
   {
     const double sc = ldexp(1.0, -ex);
 #pragma unroll
     for (int j = 0; j < 32; ++j) a[j] *= sc;
   }
 
-  // ---- 2. Householder tridiagonalisation
+  // ---- 2. Householder tridiagonalisation. Two barriers per step: after the column x is
+  // published, and after the partial products A u (p4, one per row and column quarter) and the
+  // per-warp partial sums of u^T A u (red) are; each warp then forms the w entries it needs
+  // (its rows' and its 32 columns') itself. The steps of each column quarter are unrolled, so
+  // that column k + 1 (the one u = x - beta e_{k+1} changes) is a fixed register.
+  double* red = misc + 16;
   auto step = [&](auto JJ, int Q) {
     constexpr int jj = decltype(JJ)::value;
     const int k = 32 * Q + jj;
@@ -368,6 +424,21 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
       if (i == k) d[k] = a[jj];
     }
     __syncthreads();
+    const int qmin = (k + 1) >> 5;
+    const bool active = (32 * rb + 31 > k) && q >= qmin;
+    // sum_j A_ij x_j over this thread's columns (corrected for u below)
+    double s = 0.0;
+    if (active) {
+      const double2* xq = reinterpret_cast<const double2*>(x + 32 * q);
+      double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const double2 v = xq[j];
+        s0 = fma(a[2 * j], v.x, s0);
+        s1 = fma(a[2 * j + 1], v.y, s1);
+      }
+      s = s0 + s1;
+    }
     double sg = 0.0;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -385,25 +456,19 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
     }
     const double beta = -copysign(sqrt(fma(alpha, alpha, sg)), alpha);
     const double tk = 1.0 / (beta * (beta - alpha));
-    const int qmin = (k + 1) >> 5;
-    const bool active = (32 * rb + 31 > k) && q >= qmin;
+    double su = 0.0;
     if (active) {
-      // (A u)_i over this thread's columns, u = x - beta e_{k+1}
-      const double2* xq = reinterpret_cast<const double2*>(x + 32 * q);
-      double s0 = 0.0, s1 = 0.0;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const double2 v = xq[j];
-        s0 = fma(a[2 * j], v.x, s0);
-        s1 = fma(a[2 * j + 1], v.y, s1);
-      }
       if constexpr (jj < 31) {
-        if (q == Q) s0 = fma(-beta, a[jj + 1], s0);
+        if (q == Q) s = fma(-beta, a[jj + 1], s);
       } else {
-        if (q == Q + 1) s0 = fma(-beta, a[0], s0);
+        if (q == Q + 1) s = fma(-beta, a[0], s);
       }
-      p4[q * kN + i] = s0 + s1;
+      p4[q * kN + i] = s;
+      su = s * (i == k + 1 ? alpha - beta : x[i]);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) su += __shfl_down_sync(0xffffffffu, su, o);
+    if (lane == 0) red[warp] = su;
     if (warp == 0) {   // the reflector, for the back-transformation
       double* ur = Up + ub[k];
 #pragma unroll
@@ -417,42 +482,48 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
       }
     }
     __syncthreads();
-    if (warp < 4) {   // w = p - (tau / 2)(p^T u) u; warp w writes rows 32 w .. 32 w + 31
-      double pu = 0.0, pmine = 0.0, umine = 0.0;
+    if (active) {
+      // p = tau A u, K = (tau / 2) p^T u, w = p - K u: this thread's row i and column c of
+      // the warp's quarter (each warp keeps its own copy of its 32 columns' w)
+      const double2* r2 = reinterpret_cast<const double2*>(red);
+      double rv[8];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int row = lane + 32 * m;
-        double pr = 0.0;
-        for (int qq = qmin; qq < 4; ++qq) pr += p4[qq * kN + row];
-        pr = row > k ? pr * tk : 0.0;
-        const double ur = row == k + 1 ? alpha - beta : x[row];
-        pu = fma(pr, ur, pu);
-        if (m == warp) {
-          pmine = pr;
-          umine = ur;
+      for (int w8 = 0; w8 < 8; ++w8) {
+        const double2 v = r2[w8];
+        rv[w8] = v.x + v.y;
+      }
+      const double uau = ((rv[0] + rv[1]) + (rv[2] + rv[3])) + ((rv[4] + rv[5]) + (rv[6] + rv[7]));
+      const double K = 0.5 * tk * tk * uau;
+      const int c = 32 * q + lane;
+      double pi = 0.0, pc = 0.0;
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        if (qq >= qmin) {
+          pi += p4[qq * kN + i];
+          pc += p4[qq * kN + c];
         }
       }
-      pu = wsum(pu);
-      ws[32 * warp + lane] = fma(-0.5 * tk * pu, umine, pmine);
-    }
-    __syncthreads();
-    if (active) {   // A <- A - u w^T - w u^T on this thread's entries
-      const double ui = i == k + 1 ? x[i] - beta : x[i];
-      const double wi = ws[i];
+      const double ui = i == k + 1 ? alpha - beta : x[i];
+      const double uc = c == k + 1 ? alpha - beta : x[c];
+      const double wi = i > k ? fma(-K, ui, tk * pi) : 0.0;
+      double* wq = p4 + 4 * kN + 32 * warp;
+      wq[lane] = c > k ? fma(-K, uc, tk * pc) : 0.0;
+      __syncwarp();
+      // A <- A - u w^T - w u^T on this thread's entries (u_j = x_j but at column k + 1)
       const double2* xq = reinterpret_cast<const double2*>(x + 32 * q);
-      const double2* wq = reinterpret_cast<const double2*>(ws + 32 * q);
+      const double2* wq2 = reinterpret_cast<const double2*>(wq);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const double2 xv = xq[j], wv = wq[j];
+        const double2 xv = xq[j], wv = wq2[j];
         a[2 * j] = fma(-ui, wv.x, fma(-wi, xv.x, a[2 * j]));
         a[2 * j + 1] = fma(-ui, wv.y, fma(-wi, xv.y, a[2 * j + 1]));
       }
-      // column k + 1 of u is x - beta
       if constexpr (jj < 31) {
         if (q == Q) a[jj + 1] = fma(wi, beta, a[jj + 1]);
       } else {
         if (q == Q + 1) a[0] = fma(wi, beta, a[0]);
       }
+      __syncwarp();
     }
   };
   for (int Q = 0; Q < 4 && 32 * Q <= n - 3; ++Q) {
@@ -471,14 +542,20 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
   }
   __syncthreads();
 
-  // ---- 3. eigenvalues by bisection
+  // ---- 3. eigenvalues: one round of multisection over the Gershgorin interval at 511 points
+  // (one per thread), then bisection from the bracket each eigenvalue falls in
+  const int n8 = (n + 7) & ~7;
   if (warp == 0) {
     double glo = 1e300, ghi = -1e300;
-    for (int r = lane; r < n; r += 32) {
-      const double rad = (r > 0 ? fabs(e[r - 1]) : 0.0) + (r < n - 1 ? fabs(e[r]) : 0.0);
-      glo = fmin(glo, d[r] - rad);
-      ghi = fmax(ghi, d[r] + rad);
-      e2[r] = r < n - 1 ? e[r] * e[r] : 0.0;
+    for (int r = lane; r < kN; r += 32) {
+      if (r < n) {
+        const double rad = (r > 0 ? fabs(e[r - 1]) : 0.0) + (r < n - 1 ? fabs(e[r]) : 0.0);
+        glo = fmin(glo, d[r] - rad);
+        ghi = fmax(ghi, d[r] + rad);
+      } else {
+        d[r] = 4.0;   // Sturm-count padding (no sign change)
+      }
+      e2[r] = (r >= 1 && r < n) ? e[r - 1] * e[r - 1] : 0.0;
     }
     glo = wmin(glo);
     ghi = wmax(ghi);
@@ -491,32 +568,65 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
     }
   }
   __syncthreads();
-  const double tn = misc[10];
+  const double tn = misc[10], g0 = misc[8], g1 = misc[9];
+  auto grid_pt = [&](int m) { return m <= 0 ? g0 : (m >= kT ? g1 : fma((double)m, (g1 - g0) * (1.0 / kT), g0)); };
+  int* cnt = reinterpret_cast<int*>(p4);   // counts at the kT + 1 grid points
+  if (t < kT - 1) cnt[t + 1] = sturm_below(n8, d, e2, grid_pt(t + 1));
+  if (t == 0) {
+    cnt[0] = 0;
+    cnt[kT] = n;
+  }
+  __syncthreads();
   if (t < n) {
-    double lo = misc[8], hi = misc[9];
+    int mlo = 0, mhi = kT;
+    while (mhi - mlo > 1) {
+      const int mid = (mlo + mhi) >> 1;
+      if (cnt[mid] <= t) mlo = mid;
+      else mhi = mid;
+    }
+    double lo = grid_pt(mlo), hi = grid_pt(mhi);
     const double atol = 4.0 * kEps * tn;
     for (int it = 0; it < 128; ++it) {
       if (hi - lo <= fmax(2.0 * kEps * fmax(fabs(lo), fabs(hi)), atol)) break;
       const double mid = 0.5 * (lo + hi);
       if (!(mid > lo && mid < hi)) break;
-      if (sturm_below(n, d, e2, mid) <= t) lo = mid;
+      if (sturm_below(n8, d, e2, mid) <= t) lo = mid;
       else hi = mid;
     }
     lam[t] = 0.5 * (lo + hi);
   }
   __syncthreads();
 
-  // ---- 4. eigenvectors of T
+  // ---- 4. eigenvectors of T, one thread per eigenvalue (warps 0-3); meanwhile warps 4-15 form
+  // the products cc[delta - 1][k] = u_k^T u_{k+delta}, delta = 1..3, of the blocked
+  // back-transformation (in the x and y buffers, free after step 2)
+  double* cc = xs;
   const double ctol = kClusterTol * tn;
   if (t < n) {
     const bool clustered = (t > 0 && lam[t] - lam[t - 1] <= ctol) || (t < n - 1 && lam[t + 1] - lam[t] <= ctol);
     if (!clustered) znrm[t] = twisted_vector(n, d, e, e2, lam[t], Zs + t);
+  } else if (warp >= 4) {
+    for (int idx = warp - 4; idx < 3 * kN; idx += kT / 32 - 4) {
+      const int k = idx / 3, dl = idx - 3 * k + 1;
+      double v = 0.0;
+      if (k + dl <= n - 3) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int row = lane + 32 * m;
+          if (row > k + dl && row < n) v = fma(Up[ub[k] + row], Up[ub[k + dl] + row], v);
+        }
+        v = wsum(v);
+      }
+      if (lane == 0) cc[(dl - 1) * kN + k] = v;
+    }
   }
   __syncthreads();
   if (warp == 0) cluster_vectors(n, d, e, lam, ctol, fmax(tn * kEps, 1e-280), Zs, znrm, p4);
   __syncthreads();
 
-  // ---- 5. back-transformation, thread (c, g) = (i, q)
+  // ---- 5. back-transformation, thread (c, g) = (i, q), four reflectors per barrier: for
+  // H_{k-3} H_{k-2} H_{k-1} H_k z, with a_m = u_{k-m}^T z from the z on entry,
+  // w_m = tau_{k-m} (a_m - sum_{m' < m} (u_{k-m}^T u_{k-m'}) w_{m'}) and z <- z - sum_m u_{k-m} w_m
   double z[32];
   {
     const double zn = i < n ? znrm[i] : 0.0;
@@ -526,41 +636,62 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
       z[j] = (row < n && i < n) ? Zs[row * kN + i] * zn : 0.0;
     }
   }
-  int par = 0;   // partial-sum buffer; alternates over the reflectors applied (tau = 0 is skipped)
-  for (int k = n - 3; k >= 0; --k) {
-    const double tk = tau[k];
-    if (tk == 0.0) continue;
-    const int gmin = (k + 1) >> 5;
-    double* pb = p4 + par * 4 * kN;
-    par ^= 1;
-    const double2* u2 = reinterpret_cast<const double2*>(Up + ub[k] + 32 * q);
+  __syncthreads();   // Z becomes the partial-sum buffer [2][4 reflectors][4 row groups][kN]
+  int par = 0;
+  const int row0 = 32 * q;
+  for (int kb = n - 3; kb >= 0; kb -= 4) {
+    const int gmin = (max(kb - 3, 0) + 1) >> 5;
     const bool act = q >= gmin;
-    const int row0 = 32 * q;
+    double* pb = Zs + par * 16 * kN;
+    par ^= 1;
     if (act) {
-      double s0 = 0.0, s1 = 0.0;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const double2 uv = u2[j];
-        s0 = fma(row0 + 2 * j > k ? uv.x : 0.0, z[2 * j], s0);
-        s1 = fma(row0 + 2 * j + 1 > k ? uv.y : 0.0, z[2 * j + 1], s1);
+      for (int m = 0; m < 4; ++m) {
+        const int k = kb - m;
+        double s0 = 0.0, s1 = 0.0;
+        if (k >= 0 && q >= ((k + 1) >> 5)) {   // reflector k is stored from group (k + 1) / 32 on
+          const double2* u2 = reinterpret_cast<const double2*>(Up + ub[k] + row0);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const double2 uv = u2[j];
+            s0 = fma(uv.x, z[2 * j], s0);
+            s1 = fma(uv.y, z[2 * j + 1], s1);
+          }
+        }
+        pb[(4 * m + q) * kN + i] = s0 + s1;
       }
-      pb[q * kN + i] = s0 + s1;
     }
     __syncthreads();
     if (act) {
-      double w = 0.0;
-      for (int gg = gmin; gg < 4; ++gg) w += pb[gg * kN + i];
-      w *= tk;
+      double w[4];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const double2 uv = u2[j];
-        z[2 * j] = fma(-(row0 + 2 * j > k ? uv.x : 0.0), w, z[2 * j]);
-        z[2 * j + 1] = fma(-(row0 + 2 * j + 1 > k ? uv.y : 0.0), w, z[2 * j + 1]);
+      for (int m = 0; m < 4; ++m) {
+        const int k = kb - m;
+        double v = 0.0;
+        for (int gg = gmin; gg < 4; ++gg) v += pb[(4 * m + gg) * kN + i];
+#pragma unroll
+        for (int mp = 0; mp < m; ++mp) v = fma(-cc[(m - mp - 1) * kN + (k >= 0 ? k : 0)], w[mp], v);
+        w[m] = k >= 0 ? tau[k] * v : 0.0;
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int k = kb - m;
+        if (k >= 0 && q >= ((k + 1) >> 5)) {
+          const double2* u2 = reinterpret_cast<const double2*>(Up + ub[k] + row0);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const double2 uv = u2[j];
+            z[2 * j] = fma(-uv.x, w[m], z[2 * j]);
+            z[2 * j + 1] = fma(-uv.y, w[m], z[2 * j + 1]);
+          }
+        }
       }
     }
   }
 
   // ---- 6. output: eigenvalues descending, vector of ascending index c in column n - 1 - c
+  float* vo = sb.V + (int64_t)bi * sb.sV;
+  float* lo_out = sb.lam ? sb.lam + (int64_t)bi * sb.sL : nullptr;
   bool nonfinite = false;
   if (i < n) {
 #pragma unroll
@@ -573,7 +704,7 @@ __global__ void __launch_bounds__(kT, 1) k_eig_small(SmallBatch b0, SmallBatch b
     }
   }
   if (t < n) {
-    const double l = ldexp(lam[t], ex);
+    const double l = ldexp(lam[t], *ex_s);
     nonfinite |= !isfinite(l);
     if (lo_out) lo_out[n - 1 - t] = (float)l;
   }
