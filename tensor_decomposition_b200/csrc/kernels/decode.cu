@@ -9,18 +9,22 @@
 //
 // One CTA per (layer-tensor, head) walks the T rows in tiles of 128:
 //  * prologue: M_h^T = U_D G_h^T on the tensor core (both operands are the stored bf16
-//    factors, so the products are exact and only the float32 sum rounds); M_h^T and Pi
-//    (float32) are kept in shared memory as two bf16 parts each (hi + lo, ~2^-17 relative);
-//  * producers (warps 4-11) copy the tile's U_T rows and unpack its codes into bf16 cell
-//    centres (exact: odd integers below 2^8 over 2^b), both in the 128-byte-swizzled K-major
-//    layout. The codes of the next tile and its U_T rows are loaded into registers while the
-//    current tile is unpacked; the cell centres go to two alternating buffers, so a tile is
-//    unpacked while the previous one is multiplied;
-//  * warp 12 issues tcgen05.mma: acc1 = U_T (M_h^T)_p^T, then acc2 = Y_hat Pi_p^T over the parts
-//    p, double-buffered in Tensor Memory (4 x 128 columns). The U_T buffer is single: it is
-//    released as soon as the Tucker products of a tile complete, ahead of the residual ones;
-//  * the epilogue (warps 0-3, one row per thread) forms acc1 + s acc2 and stores bf16
-//    (round to nearest even) or float32; the row's next scale is loaded a tile ahead.
+//    factors, so the products are exact and only the float32 sum rounds); M_h^T is kept in
+//    shared memory as two bf16 parts (hi + lo, ~2^-17 relative), Pi (float32) scaled by 2^10 as
+//    two fp16 parts (~2^-22 relative; the scale keeps the low parts out of the subnormals);
+//  * producers (warps 4-11) copy the tile's U_T rows and unpack its codes into the fp16
+//    integers m = 2 c + 1 - 2^b (exact: |m| < 2^8), both in the 128-byte-swizzled K-major
+//    layout. Two codes become one 32-bit word by an integer multiply-add onto the bit pattern of
+//    fp16 1024 and one packed fp16 subtraction (no integer-to-float conversion). The codes of the
+//    next tile and its U_T rows are loaded into registers while the current tile is unpacked;
+//    the code tiles go to two alternating buffers, so a tile is unpacked while the previous one
+//    is multiplied;
+//  * warp 12 issues tcgen05.mma: acc1 = U_T (M_h^T)_p^T (bf16), then acc2 = m (2^10 Pi)_p^T over
+//    the parts p (fp16), double-buffered in Tensor Memory (4 x 128 columns). The U_T buffer is
+//    single: it is released as soon as the Tucker products of a tile complete, ahead of the
+//    residual ones;
+//  * the epilogue (warps 0-3, one row per thread) forms acc1 + (s 2^-(b+10)) acc2 and stores
+//    bf16 (round to nearest even) or float32; the row's next scale is loaded a tile ahead.
 // Every wait is bounded: a timeout sets ST_TIMEOUT in the stream status and the CTA runs on
 // to its end without hanging.
 #include "../jolt_internal.h"
@@ -90,6 +94,33 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo
   lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
 }
 
+// Split 8 floats, scaled by 2^10, into fp16 hi and lo parts (16 bytes each).
+constexpr float kPiScale = 1024.0f;
+__device__ __forceinline__ void split8_f16(const float (&v)[8], uint4& hi, uint4& lo) {
+  uint32_t h2[4], l2[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a0 = v[2 * i] * kPiScale, a1 = v[2 * i + 1] * kPiScale;
+    const __half x0 = __float2half_rn(a0), x1 = __float2half_rn(a1);
+    const __half y0 = __float2half_rn(a0 - __half2float(x0)), y1 = __float2half_rn(a1 - __half2float(x1));
+    const __half2 hx = __halves2half2(x0, x1), hy = __halves2half2(y0, y1);
+    h2[i] = *reinterpret_cast<const uint32_t*>(&hx);
+    l2[i] = *reinterpret_cast<const uint32_t*>(&hy);
+  }
+  hi = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+  lo = make_uint4(l2[0], l2[1], l2[2], l2[3]);
+}
+
+// Two b-bit codes c0 (low half) and c1 (high half), packed as 16-bit fields in `cc`, to the fp16
+// pair (2 c0 + 1 - 2^b, 2 c1 + 1 - 2^b): 2 cc + (0x6400 + 513 - 2^b) per half is the bit pattern
+// of fp16 1536 + m (0x6400 is 1024.0; 257 <= 512 + m <= 767 stays in its binade, no carry between
+// the halves), and subtracting 1536 leaves m exactly.
+__device__ __forceinline__ uint32_t codes_to_f16x2(uint32_t cc, uint32_t bias2) {
+  const uint32_t biased = cc * 2u + bias2;
+  const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&biased), __floats2half2_rn(1536.0f, 1536.0f));
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int32_t* status) {
   if (mbar_wait(bar, parity, kMaxPoll)) return true;
   atomicOr(status, ST_TIMEOUT);
@@ -148,14 +179,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
   const uint32_t tmem = tmem_base;
 
   // ---------------------------------------------------------------- prologue
-  // Pi (float32, row n = output feature, k = rotated coordinate) -> two bf16 parts (B2)
+  // Pi (float32, row n = output feature, k = rotated coordinate) -> 2^10 Pi as two fp16 parts (B2)
   for (int u = tid; u < 128 * 16; u += kThreads) {
     const int n = u >> 4, c = u & 15;
     const float4 p0 = *reinterpret_cast<const float4*>(a.Pi + n * 128 + 8 * c);
     const float4 p1 = *reinterpret_cast<const float4*>(a.Pi + n * 128 + 8 * c + 4);
     const float v[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
     uint4 hi, lo;
-    split8(v, hi, lo);
+    split8_f16(v, hi, lo);
     *reinterpret_cast<uint4*>(sm + kOffB2 + sw128(n, c)) = hi;
     *reinterpret_cast<uint4*>(sm + kOffB2 + kOpBytes + sw128(n, c)) = lo;
   }
@@ -221,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
     // next tile's chunks (two aligned 8-byte words around each) and U_T rows are loaded into
     // registers before the current tile is unpacked.
     const int pt = tid - 32 * kProdWarp0;
-    const float inv2b = resid ? 1.0f / (float)(1 << b) : 0.0f;
-    const float off2b = resid ? 1.0f - (float)(1 << b) : 0.0f;
+    const uint32_t bias = resid ? 0x6400u + 513u - (1u << b) : 0u;
+    const uint32_t bias2 = bias | (bias << 16);
     const uint64_t mask = resid ? (1ull << b) - 1ull : 0ull;
     const int cpr = tucker ? rt / 8 : 0;   // 16-byte vectors per U_T row
     uint64_t cw[kChunks][2];
@@ -266,16 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
           const int r = u >> 4, c = u & 15;
           const int sh = ((u * b) & 7) * 8;
           const uint64_t v = sh ? (cw[q][0] >> sh) | (cw[q][1] << (64 - sh)) : cw[q][0];
-          float y[8];
+          uint32_t y[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t cq = (uint32_t)((v >> (e * b)) & mask);
-            y[e] = ((float)(2 * cq) + off2b) * inv2b;
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t c0 = (uint32_t)((v >> (2 * e * b)) & mask);
+            const uint32_t c1 = (uint32_t)((v >> ((2 * e + 1) * b)) & mask);
+            y[e] = codes_to_f16x2(c0 | (c1 << 16), bias2);
           }
-          if (r < rows)
-            *reinterpret_cast<uint4*>(a2 + sw128(r, c)) =
-                make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                           pack_bf16x2(y[6], y[7]));
+          if (r < rows) *reinterpret_cast<uint4*>(a2 + sw128(r, c)) = make_uint4(y[0], y[1], y[2], y[3]);
         }
         load_codes(it + 1);
       }
@@ -295,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
   } else if (warp == kMmaWarp) {
     if (elect_one()) {
       const uint32_t id = idesc_bf16_f32(128, 128);
+      const uint32_t id16 = idesc_f16_f32(128, 128);
       for (int it = 0; it < ntiles; ++it) {
         const int buf = it & 1, use = it >> 1;
         wait_or_flag(&bar_afull[buf], (uint32_t)(use & 1), status);
@@ -312,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
           for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
             for (int p = 0; p < 2; ++p)
-              umma_bf16(d2, slice_desc(a2, kk), slice_desc(sB2 + p * kOpBytes, kk), id, (kk | p) ? 1u : 0u);
+              umma_bf16(d2, slice_desc(a2, kk), slice_desc(sB2 + p * kOpBytes, kk), id16, (kk | p) ? 1u : 0u);
         }
         umma_commit(&bar_a2free[buf]);
         umma_commit(&bar_accfull[buf]);
@@ -331,9 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
     const bool staged = a.ot == EL_BF16 && rt <= 64;
     uint8_t* stage0 = sm + kOffB1 + kOpBytes / 2 + warp * 4096;
     // the row's scale for tile it + 1 is loaded while tile it is waited for and stored
+    // s 2^-(b+10): the cell centre is m / 2^b and Pi entered scaled by 2^10 (exact powers of two)
+    const float unscale = resid ? 1.0f / ((float)(1 << b) * kPiScale) : 0.0f;
     auto load_scale = [&](int it2) {
       const int t2 = it2 * kTileRows + 32 * q4 + lane;
-      return (resid && t2 < T) ? __half2float(scales[(int64_t)h * T + t2]) : 0.0f;
+      return (resid && t2 < T) ? __half2float(scales[(int64_t)h * T + t2]) * unscale : 0.0f;
     };
     float s_next = load_scale(0);
     for (int it = 0; it < ntiles; ++it) {
