@@ -244,6 +244,7 @@ struct jolt_plan_s {
         *VT = nullptr, *lamT = nullptr;
   double *BB = nullptr, *CT = nullptr;   // sketch and token Grams, float64
   double *Wg = nullptr, *Rinv = nullptr, *E = nullptr, *unit_err = nullptr, *Nbuf = nullptr, *Pbuf = nullptr;
+  float* PiT = nullptr;   // Pi^T in the residual coder's shared-memory layout
   double *meas_part = nullptr, *meas_lt = nullptr;   // measured-b refinement
   float* Qfinal = nullptr;   // final sketch basis (one of Y / Y2)
   bool q_t = false;          // Qfinal stored as Q^T [l][T] (tensor-core path) instead of Q [T][l]
@@ -714,7 +715,8 @@ JOLT_API jolt_status jolt_plan(const jolt_shape* shape, uint64_t byte_budget, in
     take(p->Gmax, n * H * Rm * D);
     take(p->E, 2 * (int64_t)L * p->ngrid);
     take(p->unit_err, 2 * (int64_t)p->G * p->nbits * p->ngrid);
-    take(p->Nbuf, n * H * Rm * D);
+    take(p->Nbuf, n * H * D * (Rm + 4));
+    take(p->PiT, (int64_t)D * 132);
     take(p->Pbuf, n * D * D);
     if (cfg.measured_b) {
       take(p->meas_part, n * H * ((T + 255) / 256) * 9);
@@ -1396,7 +1398,7 @@ JOLT_API jolt_status jolt_encode(jolt_plan_t p, const void* K, const void* V, ui
   ResidualArgs ra;
   ra.n_lt = p->n_lt; ra.H = sh.heads; ra.T = sh.tokens; ra.D = D; ra.lt_ids = p->d_lt_ids;
   ra.X[0] = K; ra.X[1] = V; ra.xt = sh.dtype == JOLT_BF16 ? EL_BF16 : EL_F32; ra.Pi = st->d_Pi;
-  ra.meta = st->d_meta; ra.body = st->d_body;
+  ra.meta = st->d_meta; ra.body = st->d_body; ra.PiT = p->PiT;
   ra.hadamard = p->cfg.rotation == 1 ? 1 : 0;
   if (p->cfg.measured_b) {
     // measured-b refinement: exact errors of every allowed width at the chosen ranks (one pass of

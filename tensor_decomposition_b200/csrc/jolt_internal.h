@@ -188,9 +188,12 @@ struct ResidualArgs {
   // y = FWHT((x - u M_h) * s) / sqrt(D) with M_h = G_h U_D^T, the rotation as log2(D) butterfly
   // stages instead of a D x D product
   int hadamard = 0;
+  // scratch [D][132] float32 for Pi^T in the coder's shared-memory layout (written by
+  // residual_encode)
+  float* PiT = nullptr;
 };
-// Pbuf: float64 scratch [n_lt][D][D] for P = U_D^T Pi; Nbuf: float64 scratch [n_lt][H][R][D]
-// for N_h = G_h P.
+// Pbuf: float64 scratch [n_lt][D][D] for P = U_D^T Pi; Nbuf: float64 scratch [n_lt][H][D][R + 4]
+// for -N_h^T (N_h = G_h P) in the coder's shared-memory layout (row stride r_t + 4).
 cudaError_t residual_encode(const ResidualArgs& a, double* Pbuf, double* Nbuf, int R, cudaStream_t s);
 
 struct DecodeArgs {

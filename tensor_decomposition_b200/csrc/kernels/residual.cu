@@ -79,6 +79,13 @@ __global__ void __launch_bounds__(128) k_resid_p(ResidualArgs a, double* Pbuf) {
   }
 }
 
+// Pi^T (float32) in the coder's shared-memory layout: row n at stride kPSRow, PiT[n][k] = Pi[k][n].
+constexpr int kPSRow = 132;
+__global__ void __launch_bounds__(256) k_pi_t(const float* Pi, float* PiT) {
+  const int n = blockIdx.x;
+  for (int k = threadIdx.x; k < kPSRow; k += blockDim.x) PiT[n * kPSRow + k] = k < kD ? Pi[k * kD + n] : 0.0f;
+}
+
 // N_h = G_h P in float64 for one (layer-tensor, head): P and G_h in shared memory, thread =
 // 4 x 4 block of N_h (rows k0 .., columns e0 ..), each entry a chain of r_d fused multiply-adds
 // in j order.
@@ -97,7 +104,9 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, const double
   for (int u = threadIdx.x; u < rd * D / 2; u += blockDim.x) reinterpret_cast<double2*>(P_s)[u] = P[u];
   for (int u = threadIdx.x; u < rt * rd; u += blockDim.x) G_s[u] = __bfloat162float(G[u]);
   __syncthreads();
-  double* N = Nbuf + (((int64_t)i * a.H + h) * R) * D;
+  // -N_h^T in the coder's layout: row n (feature) of r_t entries at stride r_t + 4
+  double* NT = Nbuf + ((int64_t)i * a.H + h) * D * (R + 4);
+  const int SN = rt + 4;
   for (int task = threadIdx.x; task < (rt / 4) * Q; task += blockDim.x) {
     const int k0 = 4 * (task / Q), e0 = 4 * (task % Q);
     double acc[4][4];
@@ -117,9 +126,9 @@ __global__ void __launch_bounds__(256) k_resid_prep(ResidualArgs a, const double
       }
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      *reinterpret_cast<double2*>(N + (int64_t)(k0 + r) * D + e0) = make_double2(acc[r][0], acc[r][1]);
-      *reinterpret_cast<double2*>(N + (int64_t)(k0 + r) * D + e0 + 2) = make_double2(acc[r][2], acc[r][3]);
+    for (int q = 0; q < 4; ++q) {
+      *reinterpret_cast<double2*>(NT + (int64_t)(e0 + q) * SN + k0) = make_double2(-acc[0][q], -acc[1][q]);
+      *reinterpret_cast<double2*>(NT + (int64_t)(e0 + q) * SN + k0 + 2) = make_double2(-acc[2][q], -acc[3][q]);
     }
   }
 }
@@ -142,7 +151,7 @@ __device__ __forceinline__ void group_sync(int g) {
 }
 
 constexpr int kRows = 16;          // rows per tile
-constexpr int kPS = 132;           // row stride (floats) of Pi^T: conflict-free fragment loads
+constexpr int kPS = kPSRow;        // row stride (floats) of Pi^T: conflict-free fragment loads
 constexpr int kGroups = 2;
 
 template <bool kMeasure, bool kHad>
@@ -163,16 +172,13 @@ __global__ void __launch_bounds__(512, 1) k_residual(ResidualArgs a, const doubl
   float* AT = reinterpret_cast<float*>(PM + kGroups * kRows * 4);                 // [2][kRows][SA]
   unsigned char* CS = reinterpret_cast<unsigned char*>(AT + (size_t)kGroups * kRows * SA);   // [2][kRows][D]
   const int tid = threadIdx.x;
-  if (!kHad) {
-    for (int e = tid; e < D * D; e += 512) {
-      const int k = e / D, n = e % D;
-      PT[n * kPS + k] = a.Pi[e];
-    }
-  }
-  const double* Ng = Nbuf + (((int64_t)i * a.H + h) * R) * D;
-  for (int e = tid; e < rt * D; e += 512) {
-    const int kk = e / D, n = e % D;
-    NT[n * SN + kk] = -Ng[e];
+  // Pi^T and -N^T arrive in their shared-memory images: straight 16-byte copies
+  if (!kHad)
+    for (int e = tid; e < D * kPS / 4; e += 512)
+      reinterpret_cast<float4*>(PT)[e] = reinterpret_cast<const float4*>(a.PiT)[e];
+  {
+    const double2* Ng = reinterpret_cast<const double2*>(Nbuf + ((int64_t)i * a.H + h) * D * (R + 4));
+    for (int e = tid; e < D * SN / 2; e += 512) reinterpret_cast<double2*>(NT)[e] = Ng[e];
   }
   const __nv_bfloat16* UT = reinterpret_cast<const __nv_bfloat16*>(a.body + m->off[lt][JOLT_PART_UT]);
   __half* scales = reinterpret_cast<__half*>(a.body + m->off[lt][JOLT_PART_SCALES]);
@@ -451,6 +457,11 @@ static size_t residual_prep_smem() { return (size_t)kD * kD * sizeof(double) + (
 
 cudaError_t residual_encode(const ResidualArgs& a, double* Pbuf, double* Nbuf, int R, cudaStream_t s) {
   if (a.D != kD) return cudaErrorInvalidValue;
+  if (!a.hadamard) {
+    if (!a.PiT) return cudaErrorInvalidValue;
+    k_pi_t<<<kD, 128, 0, s>>>(a.Pi, a.PiT);
+    note_launch();
+  }
   k_resid_p<<<dim3(kD / (4 * kPRows), a.n_lt), 128, 0, s>>>(a, Pbuf);
   note_launch();
   const size_t sp = residual_prep_smem();
