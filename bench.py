@@ -479,13 +479,14 @@ def config_dict(cfg, args):
 
 
 # ------------------------------------------------------------------ work models for the roofline
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, median of the six launches)
-# of the kernel behind a phase, from the ncu launch list of this workload, with the first 16
-# hex digits of the sha256 of the kernel's source file when it was captured: reported only
-# while that file is unchanged (profiles/launch_list_c1_mistral7b_2x_sketch.md).
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, median of three launches)
+# of the kernel behind a phase, from an ncu capture of this workload, with the first 16 hex
+# digits of the sha256 of the kernel's source file when it was captured: reported only while
+# that file is unchanged (profiles/dram_traffic_c1_mistral7b_2x_sketch.md).
 NCU_TRAFFIC = {
-    "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "4a0da90ab5592dd5", 180_089_344),
-    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "35bee190c9fdc25f", 147_005_824),
+    "small_eig": ("tensor_decomposition_b200/csrc/kernels/eig_small.cu", "192536f1cfb8b54f", 9_763_328),
+    "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "e6dbc62f94742acd", 182_135_040),
+    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "1972320fb2d3c989", 146_271_744),
 }
 
 
