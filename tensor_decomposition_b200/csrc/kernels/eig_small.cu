@@ -11,12 +11,14 @@
 //     beta = -sign(x_0) ||x||, u = x - beta e_1 (rows k + 1 .. n - 1), tau = 2 / u^T u =
 //     1 / (beta (beta - x_0)), p = tau A u, w = p - (tau / 2)(p^T u) u and A <- A - u w^T - w u^T;
 //     T's diagonal entry is A[k][k], its subdiagonal entry beta. A warp whose rows or columns
-//     all lie in the reduced part skips the step's products.
+//     all lie in the reduced part skips the step's products. The reflectors are kept for step 5
+//     from the 32-row group of row k + 1 on, zeros below, so that step needs no masks.
 //  3. All n eigenvalues of T by bisection (sec. 8.4.1) on the Sturm count, the number of sign
 //     changes along the leading principal minors p_i(x) of T - x I, which follow
 //     p_i = (d_i - x) p_{i-1} - e_{i-1}^2 p_{i-2}: no division, the pair rescaled by a power of
-//     two every eight terms. One thread per eigenvalue, down to an interval of
-//     2 eps max(|lo|, |hi|) + 4 eps ||T||.
+//     two every eight terms. A first round counts at 511 points of the Gershgorin interval (one
+//     per thread) and gives each eigenvalue its bracket; then one thread per eigenvalue bisects
+//     down to an interval of 2 eps max(|lo|, |hi|) + 4 eps ||T||.
 //  4. The eigenvector of T for each eigenvalue from the twisted factorisation of T - lambda I
 //     (Parlett & Dhillon, "Fernando's solution to Wilkinson's problem: an application of double
 //     factorization", Linear Algebra Appl. 267 (1997)): forward pivots D+_i, backward pivots
@@ -28,7 +30,9 @@
 //     elimination with partial pivoting), each solve followed by Gram-Schmidt against the
 //     members already done (one warp).
 //  5. Back-transformation Z <- H_0 H_1 ... H_{n-3} Z (sec. 5.1.6) with Z in registers: thread
-//     (c, g) holds rows 32 g .. 32 g + 31 of vector c.
+//     (c, g) holds rows 32 g .. 32 g + 31 of vector c. Four reflectors per barrier, in the
+//     compact form of their product: the four dot products u^T z from the same z, corrected by
+//     the u^T u of the pairs (formed by the idle warps during step 4).
 // Output as the one-sided Jacobi solver's: eigenvalues descending, the vectors as columns of a
 // row-major n x n array, float32. Vectors are orthonormal to ~eps ||A|| / gap, eigenvalues
 // accurate to a few eps ||A||.
