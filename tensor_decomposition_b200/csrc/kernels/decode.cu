@@ -15,8 +15,9 @@
 //  * producers (warps 4-11) copy the tile's U_T rows and unpack its codes into the fp16
 //    integers m = 2 c + 1 - 2^b (exact: |m| < 2^8), both in the 128-byte-swizzled K-major
 //    layout. Two codes become one 32-bit word by an integer multiply-add onto the bit pattern of
-//    fp16 1024 and one packed fp16 subtraction (no integer-to-float conversion). The codes of the
-//    next tile and its U_T rows are loaded into registers while the current tile is unpacked;
+//    fp16 1024 and one packed fp16 subtraction (no integer-to-float conversion). The codes and
+//    U_T rows of the tile three ahead are prefetched into L2, those of the next tile loaded into
+//    registers while the current tile is unpacked;
 //    the code tiles go to two alternating buffers, so a tile is unpacked while the previous one
 //    is multiplied;
 //  * warp 12 issues tcgen05.mma: acc1 = U_T (M_h^T)_p^T (bf16), then acc2 = m (2^10 Pi)_p^T over
@@ -282,9 +283,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
                     : make_uint4(0u, 0u, 0u, 0u);
       }
     };
+    // the codes and U_T rows of tile it2 into L2 (one thread): the register loads of a tile,
+    // issued one tile ahead, then find them there instead of waiting on DRAM
+    auto prefetch_tile = [&](int it2) {
+      if (pt != 0 || it2 >= ntiles) return;
+      const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
+      if (resid) prefetch_l2(codes + ((int64_t)h * T + t2) * rowbytes, (uint32_t)(rows2 * rowbytes));
+      if (tucker) prefetch_l2(UT + (int64_t)t2 * rt, (uint32_t)(rows2 * rt * 2));
+    };
+    prefetch_tile(1);
+    prefetch_tile(2);
     if (resid) load_codes(0);
     if (tucker) load_ut(0);
     for (int it = 0; it < ntiles; ++it) {
+      prefetch_tile(it + 3);
       const int buf = it & 1, use = it >> 1;
       const int rows = min(kTileRows, T - it * kTileRows);
       if (resid) {
