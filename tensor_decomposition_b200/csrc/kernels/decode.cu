@@ -257,6 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
     const uint32_t bias2 = bias | (bias << 16);
     const uint64_t mask = resid ? (1ull << b) - 1ull : 0ull;
     const int cpr = tucker ? rt / 8 : 0;   // 16-byte vectors per U_T row
+    // u / cpr for u < 2048 as (u * cmul) >> 20, cmul = ceil(2^20 / cpr): exact, since the
+    // fraction u / cpr is at most 1 - 1 / cpr and the error u (cmul - 2^20 / cpr) / 2^20 is below
+    // 2^-9 for cpr <= 16
+    const uint32_t cmul = tucker ? ((1u << 20) + (uint32_t)cpr - 1u) / (uint32_t)cpr : 0u;
+    auto udiv = [&](int u) { return (int)(((uint32_t)u * cmul) >> 20); };
     uint64_t cw[kChunks][2];
     auto load_codes = [&](int it2) {
       const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
       for (int q = 0; q < kUtVec; ++q) {
         const int u = pt + kProducers * q;
         ut[q] = (it2 < ntiles && u < rows2 * cpr)
-                    ? *reinterpret_cast<const uint4*>(src + (int64_t)(u / cpr) * rt + 8 * (u % cpr))
+                    ? *reinterpret_cast<const uint4*>(src + (int64_t)udiv(u) * rt + 8 * (u - udiv(u) * cpr))
                     : make_uint4(0u, 0u, 0u, 0u);
       }
     };
@@ -326,7 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
 #pragma unroll
         for (int q = 0; q < kUtVec; ++q) {
           const int u = pt + kProducers * q;
-          if (u < rows * cpr) *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(u / cpr, u % cpr)) = ut[q];
+          if (u < rows * cpr) {
+            const int ur = udiv(u);
+            *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(ur, u - ur * cpr)) = ut[q];
+          }
         }
         load_ut(it + 1);
       }
