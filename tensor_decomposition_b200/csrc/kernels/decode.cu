@@ -31,6 +31,7 @@
 #include "../jolt_internal.h"
 #include "gemm_tc.h"
 #include "sm100.cuh"
+#include <type_traits>
 
 namespace jolt {
 namespace {
@@ -52,7 +53,6 @@ constexpr int kOffA1 = 4 * kOpBytes;
 constexpr int kOffA2 = 5 * kOpBytes;
 constexpr int kSmemBytes = 7 * kOpBytes + 1024;
 constexpr int kUtVec = 8;      // 16-byte U_T vectors per producer thread and tile (128 rows x r_t <= 128)
-constexpr int kChunks = 8;     // 8-code chunks per producer thread and tile (128 rows x 16 chunks)
 
 // Byte offset of the 16-byte chunk `c16` (8 bf16, k = 8 c16 ..) of row `row` in a K-major
 // 128-row operand with 128-byte swizzling: 64-element atoms of 16 KB, rows of 128 bytes, the
@@ -248,34 +248,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
 
   // ---------------------------------------------------------------- tiles of 128 rows
   if (warp >= kProdWarp0 && warp < kMmaWarp) {
-    // producers: U_T rows -> A1, unpacked cell centres -> A2[tile parity]. Each thread takes 8
-    // chunks of 8 codes (b bytes each, at byte u b of the tile's code block for chunk u); the
-    // next tile's chunks (two aligned 8-byte words around each) and U_T rows are loaded into
-    // registers before the current tile is unpacked.
+    // producers: U_T rows -> A1, unpacked codes -> A2[tile parity]. Thread pt takes half a row of
+    // codes (row pt / 2, codes 64 (pt % 2) ..): 64 codes of b bits are 8 b contiguous bytes at byte
+    // 8 b pt of the tile's code block, loaded as b aligned 8-byte words one tile ahead. The loop
+    // is instantiated per code width, so every bit position is a constant: a pair of codes is one
+    // shift of 2b bits and one spread of the second code to bit 16. U_T rows go through registers
+    // one tile ahead as well; the tile three ahead is prefetched into L2.
     const int pt = tid - 32 * kProdWarp0;
-    const uint32_t bias = resid ? 0x6400u + 513u - (1u << b) : 0u;
-    const uint32_t bias2 = bias | (bias << 16);
-    const uint64_t mask = resid ? (1ull << b) - 1ull : 0ull;
     const int cpr = tucker ? rt / 8 : 0;   // 16-byte vectors per U_T row
     // u / cpr for u < 2048 as (u * cmul) >> 20, cmul = ceil(2^20 / cpr): exact, since the
     // fraction u / cpr is at most 1 - 1 / cpr and the error u (cmul - 2^20 / cpr) / 2^20 is below
     // 2^-9 for cpr <= 16
     const uint32_t cmul = tucker ? ((1u << 20) + (uint32_t)cpr - 1u) / (uint32_t)cpr : 0u;
     auto udiv = [&](int u) { return (int)(((uint32_t)u * cmul) >> 20); };
-    uint64_t cw[kChunks][2];
-    auto load_codes = [&](int it2) {
-      const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
-      const uint8_t* blk = codes + ((int64_t)h * T + t2) * rowbytes;
-#pragma unroll
-      for (int q = 0; q < kChunks; ++q) {
-        const int u = pt + kProducers * q;
-        const int byte0 = u * b;
-        const uint64_t* w = reinterpret_cast<const uint64_t*>(blk + (byte0 & ~7));
-        const bool ok = resid && it2 < ntiles && (u >> 4) < rows2;
-        cw[q][0] = ok ? __ldg(w) : 0ull;
-        cw[q][1] = ok ? __ldg(w + 1) : 0ull;
-      }
-    };
     uint4 ut[kUtVec];
     auto load_ut = [&](int it2) {
       const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
@@ -296,50 +281,79 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
       if (resid) prefetch_l2(codes + ((int64_t)h * T + t2) * rowbytes, (uint32_t)(rows2 * rowbytes));
       if (tucker) prefetch_l2(UT + (int64_t)t2 * rt, (uint32_t)(rows2 * rt * 2));
     };
-    prefetch_tile(1);
-    prefetch_tile(2);
-    if (resid) load_codes(0);
-    if (tucker) load_ut(0);
-    for (int it = 0; it < ntiles; ++it) {
-      prefetch_tile(it + 3);
-      const int buf = it & 1, use = it >> 1;
-      const int rows = min(kTileRows, T - it * kTileRows);
-      if (resid) {
-        // A2[buf] was last read by the residual products of tile it - 2
-        wait_or_flag(&bar_a2free[buf], (uint32_t)((use & 1) ^ 1), status);
-        uint8_t* a2 = sm + kOffA2 + buf * kOpBytes;
+    const int r_own = pt >> 1, hf = pt & 1;
+    auto run = [&](auto Bc) {
+      constexpr int B = decltype(Bc)::value;    // code width; 0: no residual
+      constexpr int NW = B > 0 ? B : 1;         // 8-byte words per half row
+      uint64_t cw[NW];
+      auto load_codes = [&](int it2) {
+        if constexpr (B > 0) {
+          const int t2 = it2 * kTileRows, rows2 = min(kTileRows, T - t2);
+          const uint64_t* w = reinterpret_cast<const uint64_t*>(codes + ((int64_t)h * T + t2) * rowbytes) + NW * pt;
+          const bool ok = it2 < ntiles && r_own < rows2;
 #pragma unroll
-        for (int q = 0; q < kChunks; ++q) {
-          const int u = pt + kProducers * q;
-          const int r = u >> 4, c = u & 15;
-          const int sh = ((u * b) & 7) * 8;
-          const uint64_t v = sh ? (cw[q][0] >> sh) | (cw[q][1] << (64 - sh)) : cw[q][0];
-          uint32_t y[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t c0 = (uint32_t)((v >> (2 * e * b)) & mask);
-            const uint32_t c1 = (uint32_t)((v >> ((2 * e + 1) * b)) & mask);
-            y[e] = codes_to_f16x2(c0 | (c1 << 16), bias2);
-          }
-          if (r < rows) *reinterpret_cast<uint4*>(a2 + sw128(r, c)) = make_uint4(y[0], y[1], y[2], y[3]);
+          for (int q = 0; q < NW; ++q) cw[q] = ok ? __ldg(w + q) : 0ull;
         }
-        load_codes(it + 1);
-      }
-      if (tucker) {
-        // A1 was last read by the Tucker products of tile it - 1
-        wait_or_flag(&bar_a1free, (uint32_t)((it & 1) ^ 1), status);
+      };
+      const uint32_t bias = B > 0 ? 0x6400u + 513u - (1u << B) : 0u;
+      const uint32_t bias2 = bias | (bias << 16);
+      prefetch_tile(1);
+      prefetch_tile(2);
+      load_codes(0);
+      if (tucker) load_ut(0);
+      for (int it = 0; it < ntiles; ++it) {
+        prefetch_tile(it + 3);
+        const int buf = it & 1, use = it >> 1;
+        const int rows = min(kTileRows, T - it * kTileRows);
+        if constexpr (B > 0) {
+          // A2[buf] was last read by the residual products of tile it - 2
+          wait_or_flag(&bar_a2free[buf], (uint32_t)((use & 1) ^ 1), status);
+          uint8_t* a2 = sm + kOffA2 + buf * kOpBytes;
+          constexpr uint32_t m1 = (1u << B) - 1u;
 #pragma unroll
-        for (int q = 0; q < kUtVec; ++q) {
-          const int u = pt + kProducers * q;
-          if (u < rows * cpr) {
-            const int ur = udiv(u);
-            *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(ur, u - ur * cpr)) = ut[q];
+          for (int j = 0; j < 8; ++j) {          // 16-byte chunk j: codes 8 j .. 8 j + 7 of the half row
+            uint32_t y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              constexpr int kPair = 2 * B;
+              const int bit = (8 * j + 2 * e) * B, wi = bit >> 6, sh = bit & 63;
+              uint64_t v = cw[wi] >> sh;
+              if (sh + kPair > 64) v |= cw[wi + 1] << (64 - sh);
+              const uint32_t x = (uint32_t)v;
+              y[e] = codes_to_f16x2((x & m1) | ((x << (16 - B)) & (m1 << 16)), bias2);
+            }
+            if (r_own < rows)
+              *reinterpret_cast<uint4*>(a2 + sw128(r_own, 8 * hf + j)) = make_uint4(y[0], y[1], y[2], y[3]);
           }
+          load_codes(it + 1);
         }
-        load_ut(it + 1);
+        if (tucker) {
+          // A1 was last read by the Tucker products of tile it - 1
+          wait_or_flag(&bar_a1free, (uint32_t)((it & 1) ^ 1), status);
+#pragma unroll
+          for (int q = 0; q < kUtVec; ++q) {
+            const int u = pt + kProducers * q;
+            if (u < rows * cpr) {
+              const int ur = udiv(u);
+              *reinterpret_cast<uint4*>(sm + kOffA1 + sw128(ur, u - ur * cpr)) = ut[q];
+            }
+          }
+          load_ut(it + 1);
+        }
+        fence_async_shared();
+        mbar_arrive(&bar_afull[buf]);
       }
-      fence_async_shared();
-      mbar_arrive(&bar_afull[buf]);
+    };
+    switch (resid ? b : 0) {
+      case 1: run(std::integral_constant<int, 1>{}); break;
+      case 2: run(std::integral_constant<int, 2>{}); break;
+      case 3: run(std::integral_constant<int, 3>{}); break;
+      case 4: run(std::integral_constant<int, 4>{}); break;
+      case 5: run(std::integral_constant<int, 5>{}); break;
+      case 6: run(std::integral_constant<int, 6>{}); break;
+      case 7: run(std::integral_constant<int, 7>{}); break;
+      case 8: run(std::integral_constant<int, 8>{}); break;
+      default: run(std::integral_constant<int, 0>{}); break;
     }
   } else if (warp == kMmaWarp) {
     if (elect_one()) {
