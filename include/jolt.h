@@ -208,12 +208,11 @@ JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, ui
  *   Arguments, layout and the result are those of jolt_rel_frob_error; ref and approx must be
  *   on the current device. n above JOLT_REL_FROB_NOALLOC_MAX_N returns JOLT_ERR_INVALID_ARG
  *   (any smaller n fits the fixed scratch: the grid is capped at 1184 blocks).
- *   Set-up: the first call on each device looks up the array's device address (with that
- *   device current) and keeps it; make that first call before any stream capture. The call
- *   synchronises `cuda_stream`. The array is shared by every caller on a device: overlapping
- *   calls (other threads, or other streams) race on it and may return wrong values. The kept
- *   address belongs to the device context in which it was looked up: after cudaDeviceReset (or
- *   any teardown of the primary context) later calls of this entry point are invalid.
+ *   Every call looks up the array's device address in the current context (a symbol lookup,
+ *   no allocation), so calls after cudaDeviceReset or a new primary context stay valid. The
+ *   call synchronises `cuda_stream` (it cannot be captured in a CUDA graph). The array is shared
+ *   by every caller on a device: overlapping calls (other threads, or other streams) race on it
+ *   and may return wrong values.
  */
 #define JOLT_REL_FROB_NOALLOC_MAX_N (1ULL << 62)
 JOLT_API jolt_status jolt_rel_frob_error_noalloc(const void* ref, const void* approx, uint64_t n,

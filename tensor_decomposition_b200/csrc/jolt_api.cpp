@@ -1500,14 +1500,6 @@ JOLT_API jolt_status jolt_rel_frob_error(const void* ref, const void* approx, ui
   return JOLT_OK;
 }
 
-// Device address of the fixed scratch of jolt_rel_frob_error_noalloc, looked up once per
-// device (with that device current) on the first call made on it.
-namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_rf_mu;
-double* g_rf_scratch[kMaxDevices] = {};
-}  // namespace
-
 JOLT_API jolt_status jolt_rel_frob_error_noalloc(const void* ref, const void* approx, uint64_t n,
                                                  jolt_dtype dtype, void* cuda_stream, double* out) {
   g_err.clear();
@@ -1521,22 +1513,13 @@ JOLT_API jolt_status jolt_rel_frob_error_noalloc(const void* ref, const void* ap
   if (nb > kRelfrobStaticBlocks)
     return fail(JOLT_ERR_INVALID_ARG, "jolt_rel_frob_error_noalloc: %d partial sums exceed the fixed scratch of %d",
                 nb, kRelfrobStaticBlocks);
-  int dev = -1;
-  CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices)
-    return fail(JOLT_ERR_UNSUPPORTED, "jolt_rel_frob_error_noalloc: device ordinal %d", dev);
+  // The fixed scratch's device address in the current context, looked up on every call (a
+  // symbol lookup allocates nothing), so a context torn down and created again is followed.
   double* scratch = nullptr;
   {
-    std::lock_guard<std::mutex> lk(g_rf_mu);
-    if (!g_rf_scratch[dev]) {
-      double* p = nullptr;
-      const cudaError_t e = relfrob_static_scratch(&p);
-      if (e != cudaSuccess || !p)
-        return fail(JOLT_ERR_CUDA, "jolt_rel_frob_error_noalloc: scratch set-up on device %d: %s", dev,
-                    cudaGetErrorString(e));
-      g_rf_scratch[dev] = p;
-    }
-    scratch = g_rf_scratch[dev];
+    const cudaError_t e = relfrob_static_scratch(&scratch);
+    if (e != cudaSuccess || !scratch)
+      return fail(JOLT_ERR_CUDA, "jolt_rel_frob_error_noalloc: scratch address: %s", cudaGetErrorString(e));
   }
   cudaStream_t s = (cudaStream_t)cuda_stream;
   Prof prof_rf("rel_frob", s);
