@@ -20,8 +20,12 @@
 //  4. k_ormtr: back-transformation Z <- H_0 ... H_{n-3} Z of the R vectors.
 // The caller re-orthonormalises the R vectors (CholeskyQR in float64): inverse iteration gives
 // vectors orthogonal to ~eps ||T|| / gap only, and coincident eigenvalues need it.
-// One CTA per matrix for steps 1 and 2, one thread per eigenvector (one warp per tight cluster) in
-// step 3, one warp per vector in step 4. No step waits on another CTA.
+// Step 1 runs on a cluster of two CTAs per matrix: each CTA forms the matrix-vector product of a
+// column step for one half of the columns (its threads also split the rows when the trailing
+// block has fewer column pairs than threads) and reads the other half from its peer's shared
+// memory; the rest of a column step is computed by both CTAs alike, and the panel's trailing
+// update is split by columns. One CTA per matrix in step 2, one thread per eigenvector (one warp
+// per tight cluster) in step 3, one warp per vector in step 4.
 #include "../jolt_internal.h"
 
 namespace jolt {
@@ -30,6 +34,27 @@ namespace {
 constexpr int kNB = 32;           // panel width of the tridiagonalisation
 constexpr int kSyThreads = 512;   // threads of k_sytrd
 constexpr int kRowChunk = 32;     // rows per register block of the trailing update
+constexpr int kSyCluster = 2;     // CTAs per matrix in k_sytrd
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Barrier over both CTAs of the cluster; memory written before it (shared memory of either CTA,
+// and global memory after a __threadfence) is visible to both after it.
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The double at the same shared-memory offset as `p`, in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ double peer_f64(const double* p, uint32_t rank) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  double v;
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(ra) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -52,27 +77,34 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
 }
 
 // Householder tridiagonalisation of one n x n symmetric matrix (full storage, row-major) per
-// CTA. On exit d, e hold the diagonal and subdiagonal of T, tau and row k of A (entries
-// k + 1 .. n - 1) the reflector H_k. Vp / Wp: [kNB][n] scratch per matrix (the panel's v and w).
-__global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int64_t sA, double* d_all,
-                                                      double* e_all, double* tau_all, double* Vp_all,
-                                                      double* Wp_all) {
+// cluster of kSyCluster CTAs. On exit d, e hold the diagonal and subdiagonal of T, tau and row k of
+// A (entries k + 1 .. n - 1) the reflector H_k (written by the cluster's first CTA). Vp / Wp:
+// [kNB][n] scratch per CTA (the panel's v and w; both CTAs of a matrix hold the same values).
+// Every barrier of the loop is reached by both CTAs the same number of times: the trip counts
+// depend on n alone. A is read at L2 (ld.global.cg), since the peer's SM writes parts of it.
+__global__ void __cluster_dims__(kSyCluster, 1, 1) __launch_bounds__(kSyThreads)
+    k_sytrd(int n, double* A_all, int64_t sA, double* d_all, double* e_all, double* tau_all, double* Vp_all,
+            double* Wp_all) {
   extern __shared__ double sm[];
   double* cs = sm;                  // [n] current column k, then the Householder vector v
   double* ys = cs + n;              // [n] y = A v, then w
-  double* red = ys + n;             // [kSyThreads / 32] block reduction
+  double* xb = ys + n;              // [2][n] this CTA's half of y = A v, by column-step parity (read by the peer)
+  double* red = xb + 2 * n;         // [kSyThreads / 32] block reduction
   double* t1 = red + kSyThreads / 32;   // [kNB] W^T v
   double* t2 = t1 + kNB;                // [kNB] V^T v
   double* bc = t2 + kNB;                // [4] broadcast: tau, scale, beta, flag
   double* stg = bc + 4;                 // [2][kNB][kRowChunk] trailing-update row factors
+  double* part = stg + 2 * kNB * kRowChunk;   // [2 kSyThreads] partial sums of the row slices
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.x;
+  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+  const bool lead = rank == 0;
+  const int b = blockIdx.x / kSyCluster;
   double* A = A_all + (int64_t)b * sA;
   double* d = d_all + (int64_t)b * n;
   double* e = e_all + (int64_t)b * n;
   double* tau = tau_all + (int64_t)b * n;
-  double* Vp = Vp_all + (int64_t)b * kNB * n;
-  double* Wp = Wp_all + (int64_t)b * kNB * n;
+  double* Vp = Vp_all + (int64_t)blockIdx.x * kNB * n;
+  double* Wp = Wp_all + (int64_t)blockIdx.x * kNB * n;
   for (int k0 = 0; k0 < n - 2; k0 += kNB) {
     const int kb = min(kNB, n - 2 - k0);
     for (int j = 0; j < kb; ++j) {
@@ -81,7 +113,7 @@ __global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int6
       // corrections, rows k .. n - 1
       double ss = 0.0;
       for (int i = k + tid; i < n; i += kSyThreads) {
-        double c = A[(int64_t)k * n + i];
+        double c = __ldcg(A + (int64_t)k * n + i);
         for (int l = 0; l < j; ++l)
           c -= Vp[(int64_t)l * n + i] * Wp[(int64_t)l * n + k] + Wp[(int64_t)l * n + i] * Vp[(int64_t)l * n + k];
         cs[i] = c;
@@ -100,9 +132,11 @@ __global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int6
         }
         bc[0] = t;
         bc[1] = scal;
-        d[k] = cs[k];
-        e[k] = beta;
-        tau[k] = t;
+        if (lead) {
+          d[k] = cs[k];
+          e[k] = beta;
+          tau[k] = t;
+        }
       }
       __syncthreads();
       const double tk = bc[0], scal = bc[1];
@@ -110,62 +144,106 @@ __global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int6
         double v = 0.0;
         if (i == k + 1) v = 1.0;
         else if (i > k + 1) v = cs[i] * scal;
-        if (i >= k + 1) {
-          A[(int64_t)k * n + i] = v;        // reflector storage in row k (dead from here on)
-          cs[i] = v;
-        }
+        if (i >= k + 1) cs[i] = v;
         Vp[(int64_t)j * n + i] = v;
       }
       __syncthreads();
       // 3. y = (A - V W^T - W V^T) v over rows and columns k + 1 .. n - 1; A is the matrix as at
-      // the start of the panel. A thread takes two adjacent columns (one 16-byte load per row;
-      // the pair starts at an even column, the one below k + 1 is computed and dropped) and
-      // keeps sixteen rows' loads in flight; the rows are read in order, so a row of the block's
-      // loads is one contiguous stretch.
+      // the start of the panel. This CTA takes one half of the columns, the peer the other. A
+      // thread takes two adjacent columns (one 16-byte load per row; the pairs start at an even
+      // column, the one below k + 1 is computed and dropped) over a slice of the rows, keeping
+      // sixteen rows' loads in flight; when the CTA has fewer column pairs than threads the rows
+      // are cut into S slices whose sums are added in slice order. The CTA's results go to ys
+      // and to xb[k % 2], from which the peer copies them after the cluster barrier.
+      double* xk = xb + (k & 1) * n;
+      int pa, pb;   // the peer's columns [pa, pb)
       if (n & 1) {
-        // odd order: rows are not 16-byte aligned pairs; one column per thread
-        for (int col = k + 1 + tid; col < n; col += kSyThreads) {
+        // odd order: rows are not 16-byte aligned pairs; one column per thread over all rows
+        const int nc = n - k - 1, h = (nc + 1) >> 1;
+        const int ca = lead ? k + 1 : k + 1 + h, cb = lead ? k + 1 + h : n;
+        pa = lead ? k + 1 + h : k + 1;
+        pb = lead ? n : k + 1 + h;
+        for (int col = ca + tid; col < cb; col += kSyThreads) {
           double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
           const double* Ac = A + col;
           int i = k + 1;
           for (; i + 3 < n; i += 4) {
-            a0 = fma(Ac[(int64_t)i * n], cs[i], a0);
-            a1 = fma(Ac[(int64_t)(i + 1) * n], cs[i + 1], a1);
-            a2 = fma(Ac[(int64_t)(i + 2) * n], cs[i + 2], a2);
-            a3 = fma(Ac[(int64_t)(i + 3) * n], cs[i + 3], a3);
+            a0 = fma(__ldcg(Ac + (int64_t)i * n), cs[i], a0);
+            a1 = fma(__ldcg(Ac + (int64_t)(i + 1) * n), cs[i + 1], a1);
+            a2 = fma(__ldcg(Ac + (int64_t)(i + 2) * n), cs[i + 2], a2);
+            a3 = fma(__ldcg(Ac + (int64_t)(i + 3) * n), cs[i + 3], a3);
           }
-          for (; i < n; ++i) a0 = fma(Ac[(int64_t)i * n], cs[i], a0);
-          ys[col] = (a0 + a1) + (a2 + a3);
+          for (; i < n; ++i) a0 = fma(__ldcg(Ac + (int64_t)i * n), cs[i], a0);
+          const double y = (a0 + a1) + (a2 + a3);
+          ys[col] = y;
+          xk[col] = y;
         }
       } else {
         const int c0 = (k + 1) & ~1;
-        for (int col = c0 + 2 * tid; col < n; col += 2 * kSyThreads) {
+        const int np = (n - c0) >> 1, h = (np + 1) >> 1;
+        const int qa = lead ? 0 : h, nq = lead ? h : np - h;   // this CTA's pairs [qa, qa + nq)
+        pa = c0 + 2 * (lead ? h : 0);
+        pb = lead ? n : c0 + 2 * h;
+        const int m = n - (k + 1);
+        int S = 1;
+        while (2 * S * nq <= kSyThreads && 2 * S * 16 <= m) S *= 2;
+        const int rs = (m + S - 1) / S;   // rows per slice
+        for (int u = tid; u < S * nq; u += kSyThreads) {
+          const int sl = u / nq, q = u - sl * nq;
+          const int col = c0 + 2 * (qa + q);
           double ax[8], ay[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) ax[u] = ay[u] = 0.0;
+          for (int v = 0; v < 8; ++v) ax[v] = ay[v] = 0.0;
           const double* Ac = A + col;
-          int i = k + 1;
-          for (; i + 15 < n; i += 16) {
+          int i = k + 1 + sl * rs;
+          const int iend = min(n, i + rs);
+          for (; i + 15 < iend; i += 16) {
             double2 t[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) t[u] = *reinterpret_cast<const double2*>(Ac + (int64_t)(i + u) * n);
+            for (int v = 0; v < 16; ++v) t[v] = __ldcg(reinterpret_cast<const double2*>(Ac + (int64_t)(i + v) * n));
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              ax[u & 7] = fma(t[u].x, cs[i + u], ax[u & 7]);
-              ay[u & 7] = fma(t[u].y, cs[i + u], ay[u & 7]);
+            for (int v = 0; v < 16; ++v) {
+              ax[v & 7] = fma(t[v].x, cs[i + v], ax[v & 7]);
+              ay[v & 7] = fma(t[v].y, cs[i + v], ay[v & 7]);
             }
           }
-          for (; i < n; ++i) {
-            const double2 t = *reinterpret_cast<const double2*>(Ac + (int64_t)i * n);
+          for (; i < iend; ++i) {
+            const double2 t = __ldcg(reinterpret_cast<const double2*>(Ac + (int64_t)i * n));
             ax[0] = fma(t.x, cs[i], ax[0]);
             ay[0] = fma(t.y, cs[i], ay[0]);
           }
           const double sx = ((ax[0] + ax[1]) + (ax[2] + ax[3])) + ((ax[4] + ax[5]) + (ax[6] + ax[7]));
           const double sy = ((ay[0] + ay[1]) + (ay[2] + ay[3])) + ((ay[4] + ay[5]) + (ay[6] + ay[7]));
-          if (col >= k + 1) ys[col] = sx;
-          ys[col + 1] = sy;
+          if (S == 1) {
+            if (col >= k + 1) ys[col] = xk[col] = sx;
+            ys[col + 1] = xk[col + 1] = sy;
+          } else {
+            part[2 * u] = sx;
+            part[2 * u + 1] = sy;
+          }
+        }
+        if (S > 1) {
+          __syncthreads();
+          for (int q = tid; q < nq; q += kSyThreads) {
+            const int col = c0 + 2 * (qa + q);
+            double sx = part[2 * q], sy = part[2 * q + 1];
+            for (int sl = 1; sl < S; ++sl) {
+              sx += part[2 * (sl * nq + q)];
+              sy += part[2 * (sl * nq + q) + 1];
+            }
+            if (col >= k + 1) ys[col] = xk[col] = sx;
+            ys[col + 1] = xk[col + 1] = sy;
+          }
         }
       }
+      // the peer's half of y (it is not overwritten before the next column step's barrier: xb
+      // alternates with the step's parity)
+      cluster_barrier();
+      for (int col = max(pa, k + 1) + tid; col < pb; col += kSyThreads) ys[col] = peer_f64(xk + col, peer);
+      // reflector storage in row k (dead from here on), written once both CTAs have read the
+      // column from that row (step 1 of this column step precedes the barrier in each)
+      if (lead)
+        for (int i = k + 1 + tid; i < n; i += kSyThreads) A[(int64_t)k * n + i] = cs[i];
       // W^T v and V^T v for the panel's earlier columns (warp l takes column l)
       for (int l = warp; l < j; l += kSyThreads / 32) {
         double s1 = 0.0, s2 = 0.0;
@@ -199,6 +277,8 @@ __global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int6
     // takes a column and a block of kRowChunk rows (accumulators in registers); the rows' factors
     // are staged in shared memory.
     const int k1 = k0 + kb;
+    const int hc = (n - k1 + 1) >> 1;
+    const int ca = lead ? k1 : k1 + hc, cb = lead ? k1 + hc : n;   // this CTA's columns
     double* sV = stg;
     double* sW = stg + kNB * kRowChunk;
     for (int i0 = k1; i0 < n; i0 += kRowChunk) {
@@ -211,7 +291,7 @@ __global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int6
         sW[u] = ok ? Wp[(int64_t)l * n + i0 + rr] : 0.0;
       }
       __syncthreads();
-      for (int c = k1 + tid; c < n; c += kSyThreads) {
+      for (int c = ca + tid; c < cb; c += kSyThreads) {
         double acc[kRowChunk];
 #pragma unroll
         for (int rr = 0; rr < kRowChunk; ++rr) acc[rr] = 0.0;
@@ -223,18 +303,20 @@ __global__ void __launch_bounds__(kSyThreads) k_sytrd(int n, double* A_all, int6
         }
 #pragma unroll
         for (int rr = 0; rr < kRowChunk; ++rr)
-          if (rr < nr) A[(int64_t)(i0 + rr) * n + c] -= acc[rr];
+          if (rr < nr) A[(int64_t)(i0 + rr) * n + c] = __ldcg(A + (int64_t)(i0 + rr) * n + c) - acc[rr];
       }
     }
-    __syncthreads();
+    // the next panel reads rows of the columns the peer updated
+    __threadfence();
+    cluster_barrier();
   }
-  if (tid == 0) {
+  if (lead && tid == 0) {
     if (n >= 2) {
-      d[n - 2] = A[(int64_t)(n - 2) * n + n - 2];
-      e[n - 2] = A[(int64_t)(n - 1) * n + n - 2];
+      d[n - 2] = __ldcg(A + (int64_t)(n - 2) * n + n - 2);
+      e[n - 2] = __ldcg(A + (int64_t)(n - 1) * n + n - 2);
       tau[n - 2] = 0.0;
     }
-    d[n - 1] = A[(int64_t)(n - 1) * n + n - 1];
+    d[n - 1] = __ldcg(A + (int64_t)(n - 1) * n + n - 1);
     e[n - 1] = 0.0;
     tau[n - 1] = 0.0;
   }
@@ -505,7 +587,7 @@ int tridiag_rpad(int R) { return (R + 31) / 32 * 32; }
 size_t tridiag_scratch_doubles(int batch, int n, int R) {
   const size_t Rp = (size_t)tridiag_rpad(R);
   return (size_t)batch * (3 * (size_t)n          // d, e, tau
-                          + 2 * (size_t)kNB * n  // panel v, w
+                          + 2 * (size_t)kSyCluster * kNB * n   // panel v, w of each CTA
                           + Rp                   // eigenvalues
                           + 5 * (size_t)n * Rp   // LU of T - lambda I per vector
                           + (size_t)n * Rp);     // eigenvectors [n][Rp]
@@ -520,15 +602,16 @@ cudaError_t eig_top_dense(int batch, int n, int R, double* A, int64_t sA, double
   double* e = d + (size_t)batch * n;
   double* tau = e + (size_t)batch * n;
   double* Vp = tau + (size_t)batch * n;
-  double* Wp = Vp + (size_t)batch * kNB * n;
-  double* lam = Wp + (size_t)batch * kNB * n;
+  double* Wp = Vp + (size_t)batch * kSyCluster * kNB * n;
+  double* lam = Wp + (size_t)batch * kSyCluster * kNB * n;
   double* work = lam + (size_t)batch * Rp;
   double* Z = work + (size_t)batch * 5 * n * Rp;
-  const size_t sm1 = (2 * (size_t)n + kSyThreads / 32 + 2 * kNB + 4 + 2 * kNB * kRowChunk) * sizeof(double);
+  const size_t sm1 =
+      (4 * (size_t)n + kSyThreads / 32 + 2 * kNB + 4 + 2 * kNB * kRowChunk + 2 * kSyThreads) * sizeof(double);
   if (sm1 > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e1 = cudaFuncSetAttribute(k_sytrd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
   if (e1 != cudaSuccess) return e1;
-  k_sytrd<<<batch, kSyThreads, sm1, s>>>(n, A, sA, d, e, tau, Vp, Wp);
+  k_sytrd<<<batch * kSyCluster, kSyThreads, sm1, s>>>(n, A, sA, d, e, tau, Vp, Wp);
   note_launch();
   const size_t sm2 = 2 * (size_t)n * sizeof(double);
   e1 = cudaFuncSetAttribute(k_stebz, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
