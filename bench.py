@@ -486,7 +486,7 @@ def config_dict(cfg, args):
 NCU_TRAFFIC = {
     "small_eig": ("tensor_decomposition_b200/csrc/kernels/eig_small.cu", "6fbe5289334b77df", 9_763_328),
     "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "e6dbc62f94742acd", 182_135_040),
-    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "1972320fb2d3c989", 146_271_744),
+    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "3b853cb6561efc69", 146_554_965),
 }
 
 
