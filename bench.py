@@ -485,8 +485,8 @@ def config_dict(cfg, args):
 # that file is unchanged (profiles/dram_traffic_c1_mistral7b_2x_sketch.md).
 NCU_TRAFFIC = {
     "small_eig": ("tensor_decomposition_b200/csrc/kernels/eig_small.cu", "6fbe5289334b77df", 9_763_328),
-    "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "e6dbc62f94742acd", 182_135_040),
-    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "3b853cb6561efc69", 146_554_965),
+    "residual": ("tensor_decomposition_b200/csrc/kernels/residual.cu", "a158d4f1be1fbf0d", 179_262_037),
+    "decode": ("tensor_decomposition_b200/csrc/kernels/decode.cu", "584d9544bb2c8a47", 140_734_379),
 }
 
 

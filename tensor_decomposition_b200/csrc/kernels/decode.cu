@@ -388,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
     const int q4 = warp;
     const int layer = lt >> 1, kind = lt & 1;
     const int64_t obase = ((int64_t)layer * H + h) * T * 128;
+    void* const outk = kind ? a.out[1] : a.out[0];   // constant indices: the argument stays in parameter space
     // With r_t <= 64 the second halves of the two M_h^T parts are unused: each warp stages its
     // 32 rows there as two boxes of 64 features (4 KB each, the 128-byte swizzled image of a box;
     // features 0-63 in part 0's half, 64-127 in part 1's) and stores them with two tensor copies;
@@ -439,14 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_tc(DecodeArgs a, const _
           }
         } else if (valid) {
           if (a.ot == EL_BF16) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out[kind]) + obase +
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(outk) + obase +
                                                   (int64_t)t * 128 + 32 * c);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               dst[q] = make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
                                   pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
           } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out[kind]) + obase +
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(outk) + obase +
                                                     (int64_t)t * 128 + 32 * c);
 #pragma unroll
             for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);

@@ -25,9 +25,9 @@ constexpr int kChunk = 256;          // tokens per CTA
 __device__ __forceinline__ const void* x_row_ptr(const ResidualArgs& a, int lt, int h, int t) {
   const int layer = lt >> 1, kind = lt & 1;
   const int64_t off = (((int64_t)layer * a.H + h) * a.T + t) * a.D;
-  return a.xt == EL_BF16
-             ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.X[kind]) + off)
-             : (const void*)(reinterpret_cast<const float*>(a.X[kind]) + off);
+  const void* x = kind ? a.X[1] : a.X[0];   // constant indices: the argument stays in parameter space
+  return a.xt == EL_BF16 ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(x) + off)
+                         : (const void*)(reinterpret_cast<const float*>(x) + off);
 }
 
 // P = U_D[:, :r_d]^T Pi (r_d x D, float64) once per layer-tensor (with the Hadamard rotation,
