@@ -767,7 +767,12 @@ def main():
         json.dump(prof, open(args.profile_out, "w"), indent=1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from threadpoolctl import threadpool_limits
-        tps, threads, sample = oracle_full_step_tokens_per_s(cfg, args.ratio, args.encoder)
+        try:
+            tps, threads, sample = oracle_full_step_tokens_per_s(cfg, args.ratio, args.encoder)
+        except MemoryError as exc:
+            # a host without room for the whole float64 cache: the bounded per-layer sample
+            tps, threads, sample = oracle_sample_tokens_per_s(cfg, args.ratio, args.encoder)
+            sample += f" (the whole-workload run needed more host memory: {exc!r})"
         # one thread: a bounded sample (whole layers, each its own single-group plan at the same
         # per-layer budget) instead of the whole workload
         with threadpool_limits(limits=1):
