@@ -156,3 +156,78 @@ def test_plan_refuses_token_ranks_beyond_the_kernels(jolt, tokens, heads, encode
         jolt.jolt_plan(1, heads, tokens, 128, True, jolt.JOLT_BF16, budget, 1, c)
     assert e.value.status == 9
     assert f"token rank {rank}" in str(e.value) and "rt_max" in str(e.value)
+
+
+def test_entry_points_reject_null_handles_without_device_work(jolt):
+    """Every entry point that takes a plan, a stream or device buffers rejects null ones with
+    JOLT_ERR_INVALID_ARG and a message, before any launch or device allocation; the destroy
+    calls accept null."""
+    L = jolt._lib
+    launches, allocs = L.jolt_launch_count(), L.jolt_alloc_count()
+    i32, u64, dbl = ctypes.c_int32(), ctypes.c_uint64(), ctypes.c_double()
+    out = ctypes.c_void_p()
+    calls = {
+        "jolt_plan_info": lambda: L.jolt_plan_info(None, ctypes.byref(i32), ctypes.byref(i32), ctypes.byref(i32),
+                                                   ctypes.byref(u64)),
+        "jolt_encode": lambda: L.jolt_encode(None, None, None, 42, None, ctypes.byref(out)),
+        "jolt_decode": lambda: L.jolt_decode(None, None, None, None),
+        "jolt_attention": lambda: L.jolt_attention(None, None, 32, 1, 1.0, None, None),
+        "jolt_rel_frob_error": lambda: L.jolt_rel_frob_error(None, None, 16, jolt.JOLT_BF16, None, ctypes.byref(dbl)),
+        "jolt_rel_frob_error_noalloc": lambda: L.jolt_rel_frob_error_noalloc(None, None, 16, jolt.JOLT_BF16, None,
+                                                                             ctypes.byref(dbl)),
+        "jolt_stream_status": lambda: L.jolt_stream_status(None),
+        "jolt_stream_info": lambda: L.jolt_stream_info(None, ctypes.byref(u64), ctypes.byref(i32), ctypes.byref(dbl)),
+        "jolt_stream_to_host": lambda: L.jolt_stream_to_host(None, None, ctypes.byref(u64)),
+        "jolt_export_debug": lambda: L.jolt_export_debug(None, 0, 0, None, ctypes.byref(u64)),
+        "jolt_profile_report": lambda: L.jolt_profile_report(None, None),
+    }
+    for name, call in calls.items():
+        assert call() == 1, name
+        msg = L.jolt_last_error().decode()
+        assert msg.startswith(name) and "null" in msg, (name, msg)
+    L.jolt_stream_destroy(None)
+    L.jolt_plan_destroy(None)
+    assert L.jolt_launch_count() == launches
+    assert L.jolt_alloc_count() == allocs
+
+
+def test_error_calls_reject_bad_dtype_and_size(jolt):
+    """The relative-error entry points check the element type, and the allocation-free one its
+    size limit, on the host (the buffers below are never dereferenced)."""
+    L = jolt._lib
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    d = ctypes.c_double()
+    for f in (L.jolt_rel_frob_error, L.jolt_rel_frob_error_noalloc):
+        assert f(p, p, 16, 7, None, ctypes.byref(d)) == 1
+        assert "dtype" in L.jolt_last_error().decode()
+    too_big = (1 << 62) + 1
+    assert L.jolt_rel_frob_error_noalloc(p, p, too_big, jolt.JOLT_BF16, None, ctypes.byref(d)) == 1
+    assert "exceeds the limit" in L.jolt_last_error().decode()
+
+
+@pytest.mark.parametrize("batch,n,R", [
+    (0, 256, 16),       # empty batch
+    (1, 1, 1),          # order below 2
+    (1, 4097, 16),      # above the exact encoder's 4096 tokens
+    (1, 256, 0),        # no eigenpair asked for
+    (1, 100, 101),      # more eigenpairs than the order
+    (1, 1024, 129),     # more than the 128 leading eigenpairs the solver returns
+])
+def test_dense_eig_selftest_rejects_bad_sizes(jolt, batch, n, R):
+    L = jolt._lib
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert L.jolt_selftest_eig_dense(batch, n, R, p, p, p, None) == 1
+    assert "jolt_selftest_eig_dense" in L.jolt_last_error().decode()
+
+
+def test_dense_eig_selftest_rejects_null_buffers(jolt):
+    L = jolt._lib
+    assert L.jolt_selftest_eig_dense(1, 256, 16, None, None, None, None) == 1
+
+
+def test_profile_switch_needs_no_device(jolt):
+    L = jolt._lib
+    assert L.jolt_profile_enable(1) == 0
+    assert L.jolt_profile_enable(0) == 0
